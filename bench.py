@@ -1,0 +1,464 @@
+#!/usr/bin/env python
+"""Benchmark of libm3ssd on one node: scan Mtokens/s (forward, L = 4096) and
+decode steps/s, each against the B200 HBM roofline, plus an end-to-end figure
+through host buffers and the fp64 CPU oracle as a reported baseline.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one m3ssd_fwd over the full Mamba-3 SISO workload (b8 L4096 H32 P64
+N128, bf16 X/B/C, fp32 logdecay/beta/gamma/theta/h0, every optional input
+present), i.e. one pass of every forward stage: decay and angle cumsums,
+rotation, the fused trapezoid intra-chunk products, the chunk-state update,
+the inter-chunk state walk and the state-to-output product.  Inputs are
+synthetic and seeded; they are resident in HBM when the timed region starts and
+larger than L2 (583 MB of algorithmic traffic per step), so no flush is needed.
+With N > 1 (torchrun, one process per GPU) every rank runs its own batch
+(weak scaling, no collective on the data path); time is the max over ranks.
+
+The decode figure (b256 H32 P64 N128 fp32 cache after a 512-token prefill)
+replays one CUDA graph of 1000 m3ssd_step calls.
+
+Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from selective_state_space_m3ssd_b200.synth import (  # noqa: E402
+    DECODE_PREFILL, DECODE_STEPS, WORKLOADS, make_inputs, rank_workload, slice_inputs)
+
+METRIC = "scan Mtokens/s (fwd, L=4096)"
+UNIT = "Mtokens/s"
+FWD_KEY = "siso"
+PROFILES = os.path.join(ROOT, "profiles")
+CHUNK_SRC = os.path.join(ROOT, "selective_state_space_m3ssd_b200", "csrc", "fwd_chunk.cu")
+STEP_SRC = os.path.join(ROOT, "selective_state_space_m3ssd_b200", "csrc", "step.cu")
+
+
+# ----------------------------------------------------------------------------
+# helpers
+# ----------------------------------------------------------------------------
+
+def nbytes(*ts) -> int:
+    return sum(t.numel() * t.element_size() for t in ts if t is not None)
+
+
+def load_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "source": "fallback"}
+
+
+def src_sha(path: str) -> str:
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def recorded_traffic(name: str, src: str):
+    """DRAM bytes per launch from a committed ncu summary, only while the
+    kernel source is the one the counters were taken on."""
+    p = os.path.join(PROFILES, f"traffic_{name}.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    if d.get("source_sha256_16") != src_sha(src):
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle sampling in the background during a region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines: list[str] = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._t = threading.Thread(target=self._read, daemon=True)
+            self._t.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self._t.join(timeout=2)
+        return False
+
+    def summary(self) -> dict:
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        busy = [s for s in sm if mx and s >= 0.5 * mx] or sm
+        return {"sm_mhz": statistics.median(busy), "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------
+# CPU oracle baseline (reported, not the target)
+# ----------------------------------------------------------------------------
+
+def oracle_sample(inp_cpu: dict, npairs: int):
+    """Run the fp64 oracle on the first ``npairs`` (b, h) sequences of the
+    workload (full length each) and return (token-heads, seconds, threads)."""
+    import oracle
+    b, L, H, P = inp_cpu["X"].shape
+    threads = oracle.default_threads()
+    pairs = [(k // H, k % H) for k in range(npairs)]
+    by_b: dict[int, list[int]] = {}
+    for bi, hi in pairs:
+        by_b.setdefault(bi, []).append(hi)
+    t0 = time.perf_counter()
+    for bi, heads in by_b.items():
+        sub = slice_inputs(inp_cpu, b=bi, heads=heads)
+        oracle.oracle_fwd(**sub, nthreads=threads)
+    dt = time.perf_counter() - t0
+    return npairs * L, dt, threads
+
+
+def cpu_baseline(inp_cpu: dict, target_s: float = 10.0) -> dict:
+    b, L, H, P = inp_cpu["X"].shape
+    import oracle
+    threads = oracle.default_threads()
+    n0 = min(b * H, max(1, threads))
+    th, dt, _ = oracle_sample(inp_cpu, n0)
+    n1 = int(min(b * H, max(n0, n0 * target_s / max(dt, 1e-3))))
+    if n1 > n0:
+        th, dt, _ = oracle_sample(inp_cpu, n1)
+    else:
+        n1 = n0
+    tokens = th / H
+    return {"value": tokens / dt / 1e6, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{n1} of {b * H} (b,h) sequences of the workload, full length L={L} "
+                      f"({th} token-heads, {dt:.1f} s, fp64 C loop, {threads} threads)"}
+
+
+# ----------------------------------------------------------------------------
+# our arm
+# ----------------------------------------------------------------------------
+
+def fwd_config(w) -> dict:
+    return {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen, "nheads": w.nheads,
+            "headdim": w.headdim, "dstate": w.dstate, "ngroups": w.ngroups, "chunk": 64,
+            "x_dtype": w.dtype, "state_dtype": "f32", "global_batch": None,
+            "l2": "inputs larger than L2 (no flush needed)"}
+
+
+def bench_forward(w, dev, steps, warmup, world, rank):
+    import selective_state_space_m3ssd_b200 as m3
+    inp = make_inputs(w)
+    d = {k: (None if v is None else v.to(dev)) for k, v in inp.items()}
+    hT = torch.empty(w.batch, w.nheads, w.dstate, w.headdim, dtype=torch.float32, device=dev)
+    call = m3.PreparedFwd(d["X"], d["logdecay"], d["beta"], d["gamma"], d["B"], d["C"],
+                          d["theta"], d["D"], d["h0"], hT=hT)
+    algo_bytes = nbytes(*(d[k] for k in ("X", "logdecay", "beta", "gamma", "B", "C", "theta",
+                                        "D", "h0")), call.Y, hT)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(warmup):
+        call()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        call()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        torch.distributed.barrier()
+        ms = float(t.item())
+    torch.cuda.synchronize(dev)
+    return {"ms_total": ms, "ms_per_step": ms / steps, "algo_bytes": algo_bytes, "inp": inp,
+            "dev_inputs": d, "call": call, "launches": steps}
+
+
+def bench_e2e(w, dev, steps, warmup, inp_cpu, world):
+    """Same metric through host buffers: pinned H2D of every input, the C-ABI
+    forward, D2H of Y and hT, all inside the timed region."""
+    import selective_state_space_m3ssd_b200 as m3
+    keys = ("X", "logdecay", "beta", "gamma", "B", "C", "theta", "D", "h0")
+    host = {k: (None if inp_cpu[k] is None else inp_cpu[k].pin_memory()) for k in keys}
+    d = {k: (None if host[k] is None else torch.empty_like(host[k], device=dev)) for k in keys}
+    hT = torch.empty(w.batch, w.nheads, w.dstate, w.headdim, dtype=torch.float32, device=dev)
+    call = m3.PreparedFwd(d["X"], d["logdecay"], d["beta"], d["gamma"], d["B"], d["C"],
+                          d["theta"], d["D"], d["h0"], hT=hT)
+    Yh = torch.empty(call.Y.shape, dtype=call.Y.dtype).pin_memory()
+    hTh = torch.empty(hT.shape, dtype=hT.dtype).pin_memory()
+    h2d = nbytes(*(host[k] for k in keys))
+    d2h = nbytes(Yh, hTh)
+
+    def one():
+        for k in keys:
+            if d[k] is not None:
+                d[k].copy_(host[k], non_blocking=True)
+        call()
+        Yh.copy_(call.Y, non_blocking=True)
+        hTh.copy_(hT, non_blocking=True)
+
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(warmup):
+        one()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        one()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    tokens = w.batch * w.seqlen * steps * world
+    return {"value": tokens / (ms / 1e3) / 1e6, "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": ms / steps}
+
+
+def bench_decode(dev, rank, steps_graph_replays: int, peaks: dict):
+    """Prefill 512 tokens with m3ssd_fwd (fp32 path), then replay one CUDA graph
+    of 1000 m3ssd_step calls on pre-staged per-step inputs."""
+    import selective_state_space_m3ssd_b200 as m3
+    w = rank_workload(WORKLOADS["decode"], rank)
+    inp = make_inputs(w, device=dev)
+    Lp = DECODE_PREFILL
+    pre = {k: (None if inp[k] is None else inp[k][:, :Lp].contiguous())
+           for k in ("X", "logdecay", "beta", "gamma", "B", "C", "theta")}
+    Y, hT, cache = m3.fwd(pre["X"], pre["logdecay"], pre["beta"], pre["gamma"], pre["B"],
+                          pre["C"], pre["theta"], inp["D"], None, want_cache=True)
+    cache["ssm"] = hT
+    del Y, pre
+    steps = {k: (None if inp[k] is None else inp[k][:, Lp:].transpose(0, 1).contiguous())
+             for k in ("X", "logdecay", "beta", "gamma", "B", "C", "theta")}
+    D = inp["D"]
+    del inp
+    ys = torch.empty_like(steps["X"])
+    torch.cuda.synchronize(dev)
+
+    def run_steps():
+        for t in range(DECODE_STEPS):
+            m3.step(cache, steps["X"][t], steps["logdecay"][t], steps["beta"][t],
+                    steps["gamma"][t], steps["B"][t], steps["C"][t], steps["theta"][t], D,
+                    y_t=ys[t])
+
+    s = torch.cuda.Stream(dev)
+    s.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(s):
+        run_steps()  # warm-up outside the graph
+    torch.cuda.current_stream(dev).wait_stream(s)
+    torch.cuda.synchronize(dev)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        run_steps()
+    torch.cuda.synchronize(dev)
+    for _ in range(2):
+        g.replay()
+    torch.cuda.synchronize(dev)
+    stream = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps_graph_replays):
+        g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1)
+    nsteps = DECODE_STEPS * steps_graph_replays
+    ms_step = ms / nsteps
+    b, H, P, N, G = w.batch, w.nheads, w.headdim, w.dstate, w.ngroups
+    f = 4
+    step_bytes = (2 * b * H * N * P * f          # ssm read + write
+                  + 2 * b * H * (N // 2) * f     # angle read + write
+                  + 2 * b * H * P * f            # x_prev read + write
+                  + 2 * b * G * N * f            # b_prev read + write
+                  + b * H * P * f                # x_t
+                  + b * H * (N // 2) * f         # theta_t
+                  + 2 * b * G * N * f            # B_t, C_t
+                  + 3 * b * H * f + H * f        # logdecay_t, beta_t, gamma_t, D
+                  + b * H * P * f)               # y_t
+    achieved = step_bytes / (ms_step / 1e3) / 1e9
+    del g
+    return {"metric": "decode steps/s", "value": 1e3 / ms_step, "unit": "steps/s",
+            "ms_per_step": ms_step, "graph_steps": nsteps,
+            "config": {"workload": w.name, "batch": b, "nheads": H, "headdim": P, "dstate": N,
+                       "prefill": Lp, "steps_per_graph": DECODE_STEPS, "dtype": "f32"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                         "peak_source": peaks["source"],
+                         "traffic": recorded_traffic("step_decode", STEP_SRC),
+                         "algo_bytes_per_step": step_bytes,
+                         "note": "per step = step kernel + b_prev update kernel (2 launches)"},
+            "gpu_launches": 2 * nsteps}
+
+
+def run_ours(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.gpus != world:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=dev)
+    from selective_state_space_m3ssd_b200 import build as m3build
+    if rank == 0 or world == 1:
+        m3build.build()
+    if world > 1:
+        torch.distributed.barrier()
+    peaks = load_peaks()
+    w = rank_workload(WORKLOADS[FWD_KEY], rank)
+
+    with ClockSampler(torch.cuda.get_device_properties(dev).index
+                      if hasattr(torch.cuda.get_device_properties(dev), "index") else local) as clk:
+        fw = bench_forward(w, dev, args.steps, args.warmup, world, rank)
+        dec = bench_decode(dev, rank, max(1, args.decode_replays), peaks)
+    e2e = bench_e2e(w, dev, max(1, min(args.steps, 5)), 1, fw["inp"], world)
+
+    tokens = w.batch * w.seqlen * args.steps * world
+    value = tokens / (fw["ms_total"] / 1e3) / 1e6
+    achieved = fw["algo_bytes"] / (fw["ms_per_step"] / 1e3) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": fw["ms_per_step"], "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(fwd_config(w), global_batch=w.batch * world,
+                       parallelism=f"dp{world}" if world > 1 else "single"),
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                     "traffic": recorded_traffic("fwd_chunk_siso", CHUNK_SRC),
+                     "peak_source": peaks["source"], "algo_bytes_per_launch": fw["algo_bytes"],
+                     "kernel": "fwd_chunk_kernel<theta, beta>"},
+        "e2e": e2e,
+        "gpu_launches": fw["launches"],
+        "decode": dec,
+        "clocks": clk.summary(),
+    }
+    if world > 1:
+        torch.distributed.barrier()
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(fw["inp"])
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+# ----------------------------------------------------------------------------
+# reference arm: the fp64 oracle on the host cores
+# ----------------------------------------------------------------------------
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    oracle.build()
+    w = WORKLOADS[FWD_KEY]
+    inp = make_inputs(w)
+    threads = oracle.default_threads()
+    npairs = max(1, min(w.batch * w.nheads, threads))
+    for _ in range(args.warmup):
+        oracle_sample(inp, min(npairs, 2))
+    total_th, total_s = 0, 0.0
+    for _ in range(args.steps):
+        th, dt, _ = oracle_sample(inp, npairs)
+        total_th += th
+        total_s += dt
+    value = total_th / w.nheads / total_s / 1e6
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * total_s / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "impl": "reference",
+        "config": dict(fwd_config(w), global_batch=w.batch, parallelism="host threads"),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": f"each step: {npairs} of {w.batch * w.nheads} (b,h) sequences, "
+                                   f"full length L={w.seqlen}"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--decode-replays", type=int, default=3,
+                    help="replays of the 1000-step decode graph in the timed region")
+    ap.add_argument("--no-cpu-baseline", action="store_true",
+                    help="omit the oracle timing (it never runs inside a GPU timed region)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,172 @@
+/*
+ * m3ssd.h -- C ABI of libm3ssd, a B200-native (sm_100a) Mamba-3 SISO selective scan.
+ *
+ * The operation (sources, by page title and section):
+ *   "TorchMamba" README, table "Models" (Mamba-3 SISO row) and "Math notes",
+ *   paragraph "M3 SISO": the exponential-trapezoidal three-term recurrence
+ *
+ *       h_t = alpha_t h_{t-1} + beta_t Bbar_{t-1} x_{t-1}^T + gamma_t Bbar_t x_t^T
+ *       y_t = Cbar_t^T h_t + D_h x_t
+ *
+ *   with alpha_t = exp(logdecay_t) and Bbar_t, Cbar_t equal to B_t, C_t rotated
+ *   pairwise by the running data-dependent angle phi_t = angle0 + sum_{s<=t} theta_s
+ *   (the "RoPE trick" for a complex state).  "VikramLex/mamba3-minimal",
+ *   section "Two-SSD Decomposition": the beta term carries the previous step's
+ *   B and x.  "TorchMamba" README, "Behavioral notes": lambda = 1 is the exact
+ *   two-term path and theta absent is the real-only path; the Mamba-2 SSD scan
+ *   is the lambda = 1, theta = 0 special case ("Reductions").
+ *
+ * Conventions fixed by this library where the pages are silent:
+ *   - pair i is components (2i, 2i+1) and is rotated by theta index i;
+ *   - R(phi) = [[cos phi, -sin phi], [sin phi, cos phi]] (counter-clockwise),
+ *     applied to both B and C;
+ *   - the running angle is inclusive: token t is rotated by phi_t, which
+ *     already contains theta_t;
+ *   - theta is taken as given (already multiplied by the step size);
+ *   - head h reads B/C group g = h / (H / G);
+ *   - h0 and hT are in the same absolute frame as Bbar (the cache frame);
+ *   - angles written by the library (angleT, cache angle) are reduced to
+ *     [-pi, pi] (the same rotation; it keeps fp32 angles precise over long runs).
+ *
+ * Layouts (row-major, contiguous, element strides implied by the shapes):
+ *   X, Y        (b, L, H, P)    dtype x_dtype (fp32 or bf16)
+ *   logdecay    (b, L, H)       fp32  (alpha = exp(logdecay))
+ *   beta, gamma (b, L, H)       fp32
+ *   B, C        (b, L, G, N)    dtype x_dtype
+ *   theta       (b, L, H, N/2)  fp32
+ *   D           (H)             fp32
+ *   h0, hT      (b, H, N, P)    fp32
+ *   cache:  angle (b, H, N/2), ssm (b, H, N, P), x_prev (b, H, P),
+ *           b_prev (b, G, N) -- all fp32; b_prev holds B_{t-1} UNROTATED and
+ *           is rotated at use by the stored angle phi_{t-1}.
+ * Decode-step tensors drop the L axis.
+ *
+ * Ownership and execution: every pointer is a DEVICE pointer owned by the
+ * caller.  The library allocates no memory, performs no host synchronisation
+ * and enqueues all work on the given stream (a cudaStream_t passed as void*;
+ * NULL is the legacy default stream).  Results are complete when the stream
+ * reaches the enqueued work.  m3ssd_step is safe to capture in a CUDA graph.
+ *
+ * Errors: arguments are validated on the host before anything is enqueued;
+ * a bad argument returns a status and enqueues nothing.  A launch failure
+ * returns M3SSD_ERR_CUDA (the CUDA error is cleared).  Nothing aborts or traps.
+ */
+#ifndef M3SSD_H_
+#define M3SSD_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define M3SSD_ABI_VERSION 1
+
+typedef enum {
+  M3SSD_OK = 0,
+  M3SSD_ERR_INVALID_ARG = 1,  /* NULL required pointer, odd N, H % G != 0, negative size, aliasing */
+  M3SSD_ERR_UNSUPPORTED = 2,  /* valid request outside what this build implements (sizes, chunk, flags) */
+  M3SSD_ERR_WORKSPACE = 3,    /* workspace smaller than m3ssd_fwd_workspace_size() or misaligned */
+  M3SSD_ERR_CUDA = 4,         /* a CUDA launch failed */
+  M3SSD_ERR_NONFINITE = 5,    /* reserved: non-finite input found by the optional check */
+  M3SSD_ERR_TIMEOUT = 6       /* reserved: a bounded device-side wait ran out */
+} m3ssd_status;
+
+typedef enum { M3SSD_F32 = 0, M3SSD_BF16 = 1 } m3ssd_dtype;
+
+/* flags (m3ssd_dims.flags); no flag is defined yet -- pass 0. */
+
+typedef struct {
+  int64_t batch;    /* b >= 0 */
+  int64_t seqlen;   /* L >= 0 (ignored by m3ssd_step) */
+  int64_t nheads;   /* H >= 1 */
+  int64_t headdim;  /* P >= 1 */
+  int64_t dstate;   /* N >= 2, even */
+  int64_t ngroups;  /* G >= 1, H % G == 0 */
+  int32_t chunk;    /* chunk length of the chunked forward: 0 = library choice, else 64 */
+  int32_t x_dtype;  /* m3ssd_dtype of X, B, C, Y (and x_t, B_t, C_t, y_t) */
+  uint32_t flags;   /* must be 0 */
+  uint32_t reserved;/* must be 0 */
+} m3ssd_dims;
+
+/* Optional cache-shaped inputs and outputs of the forward, so that a forward
+ * can start from a decode cache and hand one back (prefill -> decode).
+ * Inputs may be NULL (read as zero); outputs may be NULL (not written).
+ * angleT/xprevT may alias angle0/xprev0; bprevT must NOT alias bprev0
+ * (several heads read a group's b_prev).  Note h0/hT live in m3ssd_fwd's own
+ * arguments and may alias each other. */
+typedef struct {
+  const float* angle0;  /* (b, H, N/2): phi_{-1} */
+  const float* xprev0;  /* (b, H, P):   x_{-1}   */
+  const float* bprev0;  /* (b, G, N):   B_{-1}, unrotated */
+  float* angleT;        /* (b, H, N/2): phi_{L-1} */
+  float* xprevT;        /* (b, H, P):   x_{L-1} as fp32 */
+  float* bprevT;        /* (b, G, N):   B_{L-1} as fp32, unrotated */
+} m3ssd_fwd_extra;
+
+typedef struct {
+  float* angle;   /* (b, H, N/2) */
+  float* ssm;     /* (b, H, N, P) */
+  float* x_prev;  /* (b, H, P) */
+  float* b_prev;  /* (b, G, N), unrotated */
+} m3ssd_cache;
+
+/* Bytes of device workspace m3ssd_fwd needs for these dims (0 today).
+ * Returns 0 as well for invalid dims (m3ssd_fwd then reports the error). */
+size_t m3ssd_fwd_workspace_size(const m3ssd_dims* dims);
+
+/*
+ * Forward scan over a whole sequence ("TorchMamba" README, "Functional cores":
+ * trap_rope_loop(X, logdecay, B, C, theta_dt, lam) -> (y, h)).
+ *
+ *   X, logdecay, gamma, B, C, Y : required when b*L > 0.
+ *   beta   : NULL selects the exact two-term path (lambda = 1).
+ *   theta  : NULL selects the real-only path (no rotation).
+ *   D      : NULL means D = 0.
+ *   h0     : NULL means a zero initial state.
+ *   hT     : NULL means the final state is not written.
+ *   extra  : NULL means no cache inputs/outputs (see m3ssd_fwd_extra).
+ *   workspace, workspace_bytes : device scratch of at least
+ *            m3ssd_fwd_workspace_size(dims) bytes, 256-byte aligned (may be
+ *            NULL when that size is 0).
+ *
+ * Paths: x_dtype = BF16 with N = 128, P = 64 and 16-byte aligned tensors runs
+ * the chunked tensor-core forward (fp32 accumulation and state, bf16 operands);
+ * every other valid request runs the sequential fp32 forward (N <= 256,
+ * P <= 256, N*P <= 16384, else M3SSD_ERR_UNSUPPORTED).  Y is rounded once to
+ * x_dtype (round-to-nearest-even); hT and the extra outputs are fp32.
+ */
+m3ssd_status m3ssd_fwd(const m3ssd_dims* dims, const void* X, const float* logdecay,
+                       const float* beta, const float* gamma, const void* B, const void* C,
+                       const float* theta, const float* D, const float* h0, void* Y, float* hT,
+                       const m3ssd_fwd_extra* extra, void* workspace, size_t workspace_bytes,
+                       void* stream);
+
+/*
+ * One decode step on a cache ("TorchMamba" README, "API reference": step(u_t,
+ * cache) with Mamba3SisoCache(angle, ssm, x_prev, b_prev)):
+ *   phi' = angle + theta_t;  Bbar_prev = R(angle) b_prev;  Bbar = R(phi') B_t;
+ *   Cbar = R(phi') C_t;  ssm = alpha ssm + beta Bbar_prev x_prev^T + gamma Bbar x_t^T;
+ *   y_t = Cbar^T ssm + D x_t;  then angle = phi', x_prev = x_t, b_prev = B_t.
+ * x_t, y_t (b, H, P) and B_t, C_t (b, G, N) have dtype dims->x_dtype;
+ * logdecay_t, beta_t, gamma_t (b, H) and theta_t (b, H, N/2) are fp32.
+ * beta_t, theta_t, D may be NULL (zero).  dims->seqlen is ignored.
+ * Limits: N <= 256, P <= 256, N*P <= 16384.  Capture-safe (no allocation, no sync).
+ */
+m3ssd_status m3ssd_step(const m3ssd_dims* dims, const void* x_t, const float* logdecay_t,
+                        const float* beta_t, const float* gamma_t, const void* B_t,
+                        const void* C_t, const float* theta_t, const float* D,
+                        const m3ssd_cache* cache, void* y_t, void* stream);
+
+/* Static, human-readable name of a status. */
+const char* m3ssd_status_string(m3ssd_status status);
+
+/* M3SSD_ABI_VERSION of the loaded library. */
+int m3ssd_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* M3SSD_H_ */

@@ -1,7 +1,266 @@
 """B200-native Mamba-3 SISO selective scan: Python binding of ``libm3ssd``.
 
 The binding only marshals arguments (device pointers, sizes, the current CUDA
-stream) into the C-ABI of ``libm3ssd.so``; every step of the scan runs in the
-library's CUDA kernels.  Importing this package does not load the library; the
-first call does, and it raises if the library is missing.
+stream) into the C ABI declared in ``include/m3ssd.h``; every step of the scan
+runs in the library's CUDA kernels.  Importing this package does not load the
+library; the first call does, and raises ``LibraryMissing`` if it has not been
+built (``python -m selective_state_space_m3ssd_b200.build``).  There is no
+other implementation behind these functions.
 """
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libm3ssd.so")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_NONFINITE, ERR_TIMEOUT = range(7)
+F32, BF16 = 0, 1
+
+_lib = None
+_lock = threading.Lock()
+
+
+class LibraryMissing(RuntimeError):
+    pass
+
+
+class M3SSDError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {status_string(status)} (status {status})")
+        self.status = status
+
+
+class M3SSDInvalidArgument(M3SSDError, ValueError):
+    pass
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int64), ("seqlen", ctypes.c_int64),
+                ("nheads", ctypes.c_int64), ("headdim", ctypes.c_int64),
+                ("dstate", ctypes.c_int64), ("ngroups", ctypes.c_int64),
+                ("chunk", ctypes.c_int32), ("x_dtype", ctypes.c_int32),
+                ("flags", ctypes.c_uint32), ("reserved", ctypes.c_uint32)]
+
+
+class FwdExtra(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("angle0", "xprev0", "bprev0", "angleT", "xprevT", "bprevT")]
+
+
+class Cache(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("angle", "ssm", "x_prev", "b_prev")]
+
+
+def load(path: str | None = None):
+    """Load ``libm3ssd.so`` (once) and declare the C signatures."""
+    global _lib
+    with _lock:
+        if _lib is not None and path is None:
+            return _lib
+        p = path or LIB_PATH
+        if not os.path.exists(p):
+            raise LibraryMissing(
+                f"{p} is not built; run `python -m selective_state_space_m3ssd_b200.build`")
+        lib = ctypes.CDLL(p)
+        vp, sz = ctypes.c_void_p, ctypes.c_size_t
+        lib.m3ssd_fwd_workspace_size.argtypes = [ctypes.POINTER(Dims)]
+        lib.m3ssd_fwd_workspace_size.restype = sz
+        lib.m3ssd_fwd.argtypes = [ctypes.POINTER(Dims)] + [vp] * 11 + \
+            [ctypes.POINTER(FwdExtra), vp, sz, vp]
+        lib.m3ssd_fwd.restype = ctypes.c_int
+        lib.m3ssd_step.argtypes = [ctypes.POINTER(Dims)] + [vp] * 8 + \
+            [ctypes.POINTER(Cache), vp, vp]
+        lib.m3ssd_step.restype = ctypes.c_int
+        lib.m3ssd_status_string.argtypes = [ctypes.c_int]
+        lib.m3ssd_status_string.restype = ctypes.c_char_p
+        lib.m3ssd_abi_version.argtypes = []
+        lib.m3ssd_abi_version.restype = ctypes.c_int
+        if path is None:
+            _lib = lib
+        return lib
+
+
+def status_string(status: int) -> str:
+    return load().m3ssd_status_string(int(status)).decode()
+
+
+def _check(status: int, what: str):
+    if status == OK:
+        return
+    if status == ERR_INVALID_ARG:
+        raise M3SSDInvalidArgument(status, what)
+    raise M3SSDError(status, what)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(device):
+    import torch
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _xdtype(t) -> int:
+    import torch
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype == torch.float32:
+        return F32
+    raise ValueError(f"X/B/C must be bf16 or fp32, got {t.dtype}")
+
+
+def _need(t, name, dtype=None, shape=None, device=None):
+    if t is None:
+        return
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+
+
+def make_dims(batch, seqlen, nheads, headdim, dstate, ngroups, x_dtype, chunk=0, flags=0) -> Dims:
+    return Dims(batch, seqlen, nheads, headdim, dstate, ngroups, chunk, x_dtype, flags, 0)
+
+
+def fwd_workspace_size(dims: Dims) -> int:
+    return int(load().m3ssd_fwd_workspace_size(ctypes.byref(dims)))
+
+
+def fwd(X, logdecay, beta, gamma, B, C, theta=None, D=None, h0=None, *, Y=None,
+        want_hT: bool = True, hT=None, angle0=None, xprev0=None, bprev0=None,
+        want_cache: bool = False, chunk: int = 0, workspace=None):
+    """Forward scan through ``m3ssd_fwd`` on the current CUDA stream.
+
+    Shapes as in ``include/m3ssd.h``.  Returns ``(Y, hT, cache_out)`` where
+    ``cache_out`` is a dict with angleT/xprevT/bprevT when ``want_cache``.
+    Output tensors are allocated by torch unless passed in.
+    """
+    import torch
+    b, L, H, P = X.shape
+    G, N = B.shape[2], B.shape[3]
+    dev = X.device
+    f32 = torch.float32
+    _need(X, "X", device=dev)
+    xd = X.dtype
+    _need(logdecay, "logdecay", f32, (b, L, H), dev)
+    _need(beta, "beta", f32, (b, L, H), dev)
+    _need(gamma, "gamma", f32, (b, L, H), dev)
+    _need(B, "B", xd, (b, L, G, N), dev)
+    _need(C, "C", xd, (b, L, G, N), dev)
+    _need(theta, "theta", f32, (b, L, H, N // 2), dev)
+    _need(D, "D", f32, (H,), dev)
+    _need(h0, "h0", f32, (b, H, N, P), dev)
+    _need(angle0, "angle0", f32, (b, H, N // 2), dev)
+    _need(xprev0, "xprev0", f32, (b, H, P), dev)
+    _need(bprev0, "bprev0", f32, (b, G, N), dev)
+    if Y is None:
+        Y = torch.empty_like(X)
+    _need(Y, "Y", xd, (b, L, H, P), dev)
+    if hT is None and want_hT:
+        hT = torch.empty(b, H, N, P, dtype=f32, device=dev)
+    _need(hT, "hT", f32, (b, H, N, P), dev)
+    cache_out = None
+    extra = None
+    if want_cache or angle0 is not None or xprev0 is not None or bprev0 is not None:
+        if want_cache:
+            cache_out = {"angle": torch.empty(b, H, N // 2, dtype=f32, device=dev),
+                         "x_prev": torch.empty(b, H, P, dtype=f32, device=dev),
+                         "b_prev": torch.empty(b, G, N, dtype=f32, device=dev)}
+        extra = FwdExtra(
+            *(None if t is None else t.data_ptr() for t in (angle0, xprev0, bprev0)),
+            *(None if cache_out is None else cache_out[k].data_ptr()
+              for k in ("angle", "x_prev", "b_prev")))
+    dims = make_dims(b, L, H, P, N, G, _xdtype(X), chunk)
+    ws_bytes = fwd_workspace_size(dims)
+    if ws_bytes and workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    st = load().m3ssd_fwd(ctypes.byref(dims), _ptr(X), _ptr(logdecay), _ptr(beta), _ptr(gamma),
+                          _ptr(B), _ptr(C), _ptr(theta), _ptr(D), _ptr(h0), _ptr(Y), _ptr(hT),
+                          None if extra is None else ctypes.byref(extra), _ptr(workspace),
+                          0 if workspace is None else workspace.numel() * workspace.element_size(),
+                          _stream_handle(dev))
+    _check(st, "m3ssd_fwd")
+    return Y, hT, cache_out
+
+
+def new_cache(batch, nheads, headdim, dstate, ngroups, device):
+    """A zeroed fp32 decode cache (angle, ssm, x_prev, b_prev) allocated by torch."""
+    import torch
+    z = dict(dtype=torch.float32, device=device)
+    return {"angle": torch.zeros(batch, nheads, dstate // 2, **z),
+            "ssm": torch.zeros(batch, nheads, dstate, headdim, **z),
+            "x_prev": torch.zeros(batch, nheads, headdim, **z),
+            "b_prev": torch.zeros(batch, ngroups, dstate, **z)}
+
+
+def step(cache: dict, x_t, logdecay_t, beta_t, gamma_t, B_t, C_t, theta_t=None, D=None, *,
+         y_t=None):
+    """One decode step through ``m3ssd_step``; updates ``cache`` in place and
+    returns y_t (b, H, P) in the dtype of x_t."""
+    import torch
+    b, H, P = x_t.shape
+    G, N = B_t.shape[1], B_t.shape[2]
+    dev = x_t.device
+    f32 = torch.float32
+    xd = x_t.dtype
+    _need(x_t, "x_t", device=dev)
+    _need(logdecay_t, "logdecay_t", f32, (b, H), dev)
+    _need(beta_t, "beta_t", f32, (b, H), dev)
+    _need(gamma_t, "gamma_t", f32, (b, H), dev)
+    _need(B_t, "B_t", xd, (b, G, N), dev)
+    _need(C_t, "C_t", xd, (b, G, N), dev)
+    _need(theta_t, "theta_t", f32, (b, H, N // 2), dev)
+    _need(D, "D", f32, (H,), dev)
+    _need(cache["angle"], "cache.angle", f32, (b, H, N // 2), dev)
+    _need(cache["ssm"], "cache.ssm", f32, (b, H, N, P), dev)
+    _need(cache["x_prev"], "cache.x_prev", f32, (b, H, P), dev)
+    _need(cache["b_prev"], "cache.b_prev", f32, (b, G, N), dev)
+    if y_t is None:
+        y_t = torch.empty_like(x_t)
+    _need(y_t, "y_t", xd, (b, H, P), dev)
+    c = Cache(cache["angle"].data_ptr(), cache["ssm"].data_ptr(), cache["x_prev"].data_ptr(),
+              cache["b_prev"].data_ptr())
+    dims = make_dims(b, 1, H, P, N, G, _xdtype(x_t))
+    st = load().m3ssd_step(ctypes.byref(dims), _ptr(x_t), _ptr(logdecay_t), _ptr(beta_t),
+                           _ptr(gamma_t), _ptr(B_t), _ptr(C_t), _ptr(theta_t), _ptr(D),
+                           ctypes.byref(c), _ptr(y_t), _stream_handle(dev))
+    _check(st, "m3ssd_step")
+    return y_t
+
+
+class PreparedFwd:
+    """A forward call with its C arguments marshalled once, for loops that
+    launch the same problem many times (benchmarks, graph capture).  Calling
+    it enqueues ``m3ssd_fwd`` on the current stream of the tensors' device."""
+
+    def __init__(self, X, logdecay, beta, gamma, B, C, theta=None, D=None, h0=None, *,
+                 Y=None, hT=None, chunk: int = 0):
+        import torch
+        b, L, H, P = X.shape
+        G, N = B.shape[2], B.shape[3]
+        self.Y = torch.empty_like(X) if Y is None else Y
+        self.hT = hT
+        self._keep = (X, logdecay, beta, gamma, B, C, theta, D, h0, self.Y, hT)
+        self._dims = make_dims(b, L, H, P, N, G, _xdtype(X), chunk)
+        self._args = [_ptr(t) for t in self._keep]
+        self.device = X.device
+        ws = fwd_workspace_size(self._dims)
+        self._ws = torch.empty(ws, dtype=torch.uint8, device=X.device) if ws else None
+        self._lib = load()
+
+    def __call__(self):
+        st = self._lib.m3ssd_fwd(ctypes.byref(self._dims), *self._args, None, _ptr(self._ws),
+                                 0 if self._ws is None else self._ws.numel(),
+                                 _stream_handle(self.device))
+        _check(st, "m3ssd_fwd")
+        return self.Y

@@ -1,0 +1,59 @@
+// Internal launch interface shared by the C-ABI layer and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace m3ssd {
+
+// Everything one forward launch needs; validated by the C-ABI layer.
+struct FwdArgs {
+  int64_t b, L, H, P, N, G;
+  int chunk;
+  bool bf16;  // X, B, C, Y are bf16 (else fp32)
+  const void* X;
+  const float* logdecay;
+  const float* beta;   // nullable
+  const float* gamma;
+  const void* B;
+  const void* C;
+  const float* theta;  // nullable
+  const float* D;      // nullable
+  const float* h0;     // nullable
+  void* Y;
+  float* hT;           // nullable
+  const float* angle0; // nullable
+  const float* xprev0; // nullable
+  const float* bprev0; // nullable
+  float* angleT;       // nullable
+  float* xprevT;       // nullable
+  float* bprevT;       // nullable
+};
+
+struct StepArgs {
+  int64_t b, H, P, N, G;
+  bool bf16;
+  const void* x_t;
+  const float* logdecay_t;
+  const float* beta_t;   // nullable
+  const float* gamma_t;
+  const void* B_t;
+  const void* C_t;
+  const float* theta_t;  // nullable
+  const float* D;        // nullable
+  float* angle;
+  float* ssm;
+  float* x_prev;
+  float* b_prev;
+  void* y_t;
+};
+
+// Sequential fp32 forward: one CTA per (b, h), token by token.
+cudaError_t launch_fwd_seq(const FwdArgs& a, cudaStream_t s);
+// Chunked bf16 tensor-core forward (N = 128, P = 64).
+cudaError_t launch_fwd_chunk(const FwdArgs& a, cudaStream_t s);
+bool fwd_chunk_supported(const FwdArgs& a);
+// Decode step (two launches: the state/outputs, then b_prev <- B_t).
+cudaError_t launch_step(const StepArgs& a, cudaStream_t s);
+
+}  // namespace m3ssd

@@ -1,0 +1,146 @@
+// C-ABI entry points of libm3ssd: host-side validation and dispatch.
+//
+// Nothing here computes a step of the scan; it checks arguments, picks the
+// kernel path and enqueues the launches on the caller's stream.  No memory is
+// allocated and no host synchronisation is performed.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "../../include/m3ssd.h"
+#include "internal.h"
+
+namespace {
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Validation shared by the forward and the step.
+m3ssd_status check_dims(const m3ssd_dims* d) {
+  if (!d) return M3SSD_ERR_INVALID_ARG;
+  if (d->batch < 0 || d->seqlen < 0) return M3SSD_ERR_INVALID_ARG;
+  if (d->nheads < 1 || d->headdim < 1 || d->ngroups < 1) return M3SSD_ERR_INVALID_ARG;
+  if (d->dstate < 2 || d->dstate % 2 != 0) return M3SSD_ERR_INVALID_ARG;
+  if (d->nheads % d->ngroups != 0) return M3SSD_ERR_INVALID_ARG;
+  if (d->x_dtype != M3SSD_F32 && d->x_dtype != M3SSD_BF16) return M3SSD_ERR_INVALID_ARG;
+  if (d->reserved != 0) return M3SSD_ERR_INVALID_ARG;
+  if (d->flags != 0) return M3SSD_ERR_UNSUPPORTED;
+  if (d->batch * d->nheads > INT32_MAX) return M3SSD_ERR_UNSUPPORTED;
+  return M3SSD_OK;
+}
+
+// Shapes every kernel of this build can take (the sequential and step paths
+// keep an (N, P) fp32 state in one CTA's shared memory).
+bool general_shape_ok(const m3ssd_dims* d) {
+  return d->dstate <= 256 && d->headdim <= 256 && d->dstate * d->headdim <= 16384;
+}
+
+m3ssd_status from_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return M3SSD_OK;
+  (void)cudaGetLastError();
+  return M3SSD_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int m3ssd_abi_version(void) { return M3SSD_ABI_VERSION; }
+
+const char* m3ssd_status_string(m3ssd_status s) {
+  switch (s) {
+    case M3SSD_OK: return "ok";
+    case M3SSD_ERR_INVALID_ARG: return "invalid argument";
+    case M3SSD_ERR_UNSUPPORTED: return "unsupported request";
+    case M3SSD_ERR_WORKSPACE: return "workspace too small or misaligned";
+    case M3SSD_ERR_CUDA: return "CUDA launch failed";
+    case M3SSD_ERR_NONFINITE: return "non-finite input";
+    case M3SSD_ERR_TIMEOUT: return "device-side wait timed out";
+  }
+  return "unknown status";
+}
+
+size_t m3ssd_fwd_workspace_size(const m3ssd_dims* dims) {
+  (void)dims;
+  return 0;
+}
+
+m3ssd_status m3ssd_fwd(const m3ssd_dims* dims, const void* X, const float* logdecay,
+                       const float* beta, const float* gamma, const void* B, const void* C,
+                       const float* theta, const float* D, const float* h0, void* Y, float* hT,
+                       const m3ssd_fwd_extra* extra, void* workspace, size_t workspace_bytes,
+                       void* stream) {
+  m3ssd_status st = check_dims(dims);
+  if (st != M3SSD_OK) return st;
+  if (dims->chunk != 0 && dims->chunk != 64) return M3SSD_ERR_UNSUPPORTED;
+
+  const bool bf16 = dims->x_dtype == M3SSD_BF16;
+  const uintptr_t esz = bf16 ? 2 : 4;
+  const bool has_tokens = dims->batch * dims->seqlen > 0;
+  if (has_tokens && (!X || !logdecay || !gamma || !B || !C || !Y)) return M3SSD_ERR_INVALID_ARG;
+  if (!aligned(X, esz) || !aligned(B, esz) || !aligned(C, esz) || !aligned(Y, esz))
+    return M3SSD_ERR_INVALID_ARG;
+  const void* f32ptrs[] = {logdecay, beta, gamma, theta, D, h0, hT};
+  for (const void* p : f32ptrs)
+    if (!aligned(p, 4)) return M3SSD_ERR_INVALID_ARG;
+
+  m3ssd::FwdArgs a{};
+  a.b = dims->batch; a.L = dims->seqlen; a.H = dims->nheads; a.P = dims->headdim;
+  a.N = dims->dstate; a.G = dims->ngroups; a.chunk = dims->chunk; a.bf16 = bf16;
+  a.X = X; a.logdecay = logdecay; a.beta = beta; a.gamma = gamma; a.B = B; a.C = C;
+  a.theta = theta; a.D = D; a.h0 = h0; a.Y = Y; a.hT = hT;
+  if (extra) {
+    if (extra->bprevT && extra->bprevT == extra->bprev0) return M3SSD_ERR_INVALID_ARG;
+    const void* eptrs[] = {extra->angle0, extra->xprev0, extra->bprev0,
+                           extra->angleT, extra->xprevT, extra->bprevT};
+    for (const void* p : eptrs)
+      if (!aligned(p, 4)) return M3SSD_ERR_INVALID_ARG;
+    a.angle0 = extra->angle0; a.xprev0 = extra->xprev0; a.bprev0 = extra->bprev0;
+    a.angleT = extra->angleT; a.xprevT = extra->xprevT; a.bprevT = extra->bprevT;
+  }
+
+  const size_t need = m3ssd_fwd_workspace_size(dims);
+  if (workspace_bytes < need || (need > 0 && (!workspace || !aligned(workspace, 256))))
+    return M3SSD_ERR_WORKSPACE;
+
+  const bool chunked = m3ssd::fwd_chunk_supported(a);
+  if (!chunked && !general_shape_ok(dims)) return M3SSD_ERR_UNSUPPORTED;
+  if (dims->batch == 0) return M3SSD_OK;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return from_cuda(chunked ? m3ssd::launch_fwd_chunk(a, s) : m3ssd::launch_fwd_seq(a, s));
+}
+
+m3ssd_status m3ssd_step(const m3ssd_dims* dims, const void* x_t, const float* logdecay_t,
+                        const float* beta_t, const float* gamma_t, const void* B_t,
+                        const void* C_t, const float* theta_t, const float* D,
+                        const m3ssd_cache* cache, void* y_t, void* stream) {
+  m3ssd_status st = check_dims(dims);
+  if (st != M3SSD_OK) return st;
+  if (!general_shape_ok(dims)) return M3SSD_ERR_UNSUPPORTED;
+  if (!cache) return M3SSD_ERR_INVALID_ARG;
+  const bool bf16 = dims->x_dtype == M3SSD_BF16;
+  const uintptr_t esz = bf16 ? 2 : 4;
+  if (dims->batch > 0) {
+    if (!x_t || !logdecay_t || !gamma_t || !B_t || !C_t || !y_t) return M3SSD_ERR_INVALID_ARG;
+    if (!cache->angle || !cache->ssm || !cache->x_prev || !cache->b_prev)
+      return M3SSD_ERR_INVALID_ARG;
+  }
+  if (!aligned(x_t, esz) || !aligned(B_t, esz) || !aligned(C_t, esz) || !aligned(y_t, esz))
+    return M3SSD_ERR_INVALID_ARG;
+  const void* f32ptrs[] = {logdecay_t, beta_t, gamma_t, theta_t, D,
+                           cache->angle, cache->ssm, cache->x_prev, cache->b_prev};
+  for (const void* p : f32ptrs)
+    if (!aligned(p, 4)) return M3SSD_ERR_INVALID_ARG;
+  if (dims->batch == 0) return M3SSD_OK;
+
+  m3ssd::StepArgs a{};
+  a.b = dims->batch; a.H = dims->nheads; a.P = dims->headdim; a.N = dims->dstate;
+  a.G = dims->ngroups; a.bf16 = bf16;
+  a.x_t = x_t; a.logdecay_t = logdecay_t; a.beta_t = beta_t; a.gamma_t = gamma_t;
+  a.B_t = B_t; a.C_t = C_t; a.theta_t = theta_t; a.D = D;
+  a.angle = cache->angle; a.ssm = cache->ssm; a.x_prev = cache->x_prev; a.b_prev = cache->b_prev;
+  a.y_t = y_t;
+  return from_cuda(m3ssd::launch_step(a, static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -63,6 +63,12 @@ DECODE_PREFILL = 512
 DECODE_STEPS = 1000
 
 
+def rank_workload(w: Workload, rank: int) -> Workload:
+    """The workload rank ``rank`` of a weak-scaling run processes: the same
+    shapes with its own seed (independent batches, no exchange between ranks)."""
+    return w.with_(seed=w.seed + 7919 * rank)
+
+
 def torch_dtype(name: str) -> torch.dtype:
     return {"f32": torch.float32, "bf16": torch.bfloat16}[name]
 

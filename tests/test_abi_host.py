@@ -1,0 +1,135 @@
+"""The C-ABI library loads, exports every declared symbol and validates its
+arguments on the host (no GPU needed: nothing here reaches a kernel)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import selective_state_space_m3ssd_b200 as m3
+from selective_state_space_m3ssd_b200 import build as m3build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "m3ssd.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    m3build.build()
+    return m3.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(m3ssd_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for n in ("m3ssd_fwd", "m3ssd_step", "m3ssd_fwd_workspace_size", "m3ssd_status_string",
+              "m3ssd_abi_version"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", m3.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (m3ssd_\w+)", out))
+    missing = [n for n in declared_functions() if n not in exported]
+    assert not missing, f"declared but not exported: {missing}"
+    for n in declared_functions():
+        assert hasattr(lib, n)
+
+
+def test_header_compiles_as_c_and_cxx(tmp_path):
+    src = tmp_path / "t.c"
+    src.write_text('#include "m3ssd.h"\nint main(void){m3ssd_dims d={0};(void)d;'
+                   'return m3ssd_abi_version()==M3SSD_ABI_VERSION?0:1;}\n')
+    for cc, std in (("gcc", "-std=c99"), ("g++", "-std=c++17")):
+        subprocess.run([cc, std, "-fsyntax-only", "-x", "c" if cc == "gcc" else "c++",
+                        "-I", os.path.join(ROOT, "include"), str(src)], check=True)
+
+
+def test_version_and_status_strings(lib):
+    assert lib.m3ssd_abi_version() == 1
+    assert m3.status_string(m3.OK) == "ok"
+    assert "invalid" in m3.status_string(m3.ERR_INVALID_ARG)
+    assert m3.status_string(99) == "unknown status"
+
+
+def _dims(**kw):
+    d = dict(batch=1, seqlen=8, nheads=2, headdim=8, dstate=8, ngroups=1, x_dtype=m3.F32,
+             chunk=0, flags=0)
+    d.update(kw)
+    return m3.make_dims(d["batch"], d["seqlen"], d["nheads"], d["headdim"], d["dstate"],
+                        d["ngroups"], d["x_dtype"], d["chunk"], d["flags"])
+
+
+FAKE = ctypes.c_void_p(0x10000)  # never dereferenced: every call below fails validation
+
+
+def _fwd(lib, dims, X=FAKE, ld=FAKE, beta=None, gamma=FAKE, B=FAKE, C=FAKE, theta=None,
+         D=None, h0=None, Y=FAKE, hT=None, extra=None, ws=None, ws_bytes=0):
+    return lib.m3ssd_fwd(ctypes.byref(dims), X, ld, beta, gamma, B, C, theta, D, h0, Y, hT,
+                         None if extra is None else ctypes.byref(extra), ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(dstate=7), m3.ERR_INVALID_ARG),
+    (dict(dstate=0), m3.ERR_INVALID_ARG),
+    (dict(nheads=3, ngroups=2), m3.ERR_INVALID_ARG),
+    (dict(nheads=0), m3.ERR_INVALID_ARG),
+    (dict(headdim=0), m3.ERR_INVALID_ARG),
+    (dict(batch=-1), m3.ERR_INVALID_ARG),
+    (dict(seqlen=-5), m3.ERR_INVALID_ARG),
+    (dict(x_dtype=7), m3.ERR_INVALID_ARG),
+    (dict(flags=1), m3.ERR_UNSUPPORTED),
+    (dict(chunk=48), m3.ERR_UNSUPPORTED),
+    (dict(dstate=512), m3.ERR_UNSUPPORTED),
+    (dict(headdim=300), m3.ERR_UNSUPPORTED),
+])
+def test_fwd_rejects_bad_dims(lib, kw, status):
+    assert _fwd(lib, _dims(**kw)) == status
+
+
+def test_fwd_rejects_null_and_misaligned_pointers(lib):
+    d = _dims()
+    for name in ("X", "ld", "gamma", "B", "C", "Y"):
+        assert _fwd(lib, d, **{name: None}) == m3.ERR_INVALID_ARG, name
+    assert _fwd(lib, d, X=ctypes.c_void_p(0x10002)) == m3.ERR_INVALID_ARG
+    assert _fwd(lib, d, theta=ctypes.c_void_p(0x10001)) == m3.ERR_INVALID_ARG
+    assert _fwd(lib, _dims(x_dtype=m3.BF16), X=ctypes.c_void_p(0x10001)) == m3.ERR_INVALID_ARG
+    e = m3.FwdExtra(None, None, 0x20000, None, None, 0x20000)
+    assert _fwd(lib, d, extra=e) == m3.ERR_INVALID_ARG  # bprevT aliases bprev0
+
+
+def test_fwd_with_no_batch_is_a_no_op(lib):
+    assert _fwd(lib, _dims(batch=0), X=None, ld=None, gamma=None, B=None, C=None, Y=None) == m3.OK
+    assert lib.m3ssd_fwd_workspace_size(ctypes.byref(_dims())) == 0
+    assert lib.m3ssd_fwd_workspace_size(None) == 0
+
+
+def _step(lib, dims, cache=None, x=FAKE, y=FAKE):
+    c = cache or m3.Cache(0x10000, 0x10000, 0x10000, 0x10000)
+    return lib.m3ssd_step(ctypes.byref(dims), x, FAKE, None, FAKE, FAKE, FAKE, None, None,
+                          ctypes.byref(c), y, None)
+
+
+def test_step_validation(lib):
+    assert _step(lib, _dims(dstate=5)) == m3.ERR_INVALID_ARG
+    assert _step(lib, _dims(), x=None) == m3.ERR_INVALID_ARG
+    assert _step(lib, _dims(), y=None) == m3.ERR_INVALID_ARG
+    assert _step(lib, _dims(), cache=m3.Cache(0x10000, None, 0x10000, 0x10000)) == m3.ERR_INVALID_ARG
+    assert _step(lib, _dims(), cache=m3.Cache(0x10000, 0x10002, 0x10000, 0x10000)) == m3.ERR_INVALID_ARG
+    assert lib.m3ssd_step(ctypes.byref(_dims()), FAKE, FAKE, None, FAKE, FAKE, FAKE, None, None,
+                          None, FAKE, None) == m3.ERR_INVALID_ARG
+    assert _step(lib, _dims(batch=0), x=None, y=None) == m3.OK
+
+
+def test_python_binding_raises_value_error_on_invalid_args(lib):
+    with pytest.raises(ValueError):
+        m3._check(m3.ERR_INVALID_ARG, "m3ssd_fwd")
+    with pytest.raises(m3.M3SSDError):
+        m3._check(m3.ERR_UNSUPPORTED, "m3ssd_fwd")

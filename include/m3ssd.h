@@ -159,6 +159,13 @@ m3ssd_status m3ssd_step(const m3ssd_dims* dims, const void* x_t, const float* lo
                         const void* C_t, const float* theta_t, const float* D,
                         const m3ssd_cache* cache, void* y_t, void* stream);
 
+/* Number of bounded device-side waits of the chunked forward that ran out
+ * (each makes its CTA stop and leave its outputs unwritten) since the last
+ * call; the count is then reset.  This call synchronises the current device
+ * and must not be captured in a CUDA graph.  Returns M3SSD_ERR_INVALID_ARG for
+ * a NULL pointer and M3SSD_ERR_CUDA if the device cannot be read. */
+m3ssd_status m3ssd_device_wait_timeouts(uint32_t* count);
+
 /* Static, human-readable name of a status. */
 const char* m3ssd_status_string(m3ssd_status status);
 

@@ -78,6 +78,8 @@ def load(path: str | None = None):
         lib.m3ssd_status_string.restype = ctypes.c_char_p
         lib.m3ssd_abi_version.argtypes = []
         lib.m3ssd_abi_version.restype = ctypes.c_int
+        lib.m3ssd_device_wait_timeouts.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
+        lib.m3ssd_device_wait_timeouts.restype = ctypes.c_int
         if path is None:
             _lib = lib
         return lib
@@ -126,6 +128,13 @@ def _need(t, name, dtype=None, shape=None, device=None):
         raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
     if device is not None and t.device != device:
         raise ValueError(f"{name} is on {t.device}, expected {device}")
+
+
+def device_wait_timeouts() -> int:
+    """Bounded device-side waits that ran out since the last call (synchronises)."""
+    n = ctypes.c_uint32(0)
+    _check(load().m3ssd_device_wait_timeouts(ctypes.byref(n)), "m3ssd_device_wait_timeouts")
+    return int(n.value)
 
 
 def make_dims(batch, seqlen, nheads, headdim, dstate, ngroups, x_dtype, chunk=0, flags=0) -> Dims:

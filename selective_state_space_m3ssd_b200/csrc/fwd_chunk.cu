@@ -1,41 +1,50 @@
-// Chunked bf16 forward of the Mamba-3 SISO scan (N = 128, P = 64).
+// Chunked bf16 forward of the Mamba-3 SISO scan on the sm_100a tensor cores
+// (tcgen05 MMA, TMEM accumulators), for N = 128, P = 64.
 //
 // One CTA owns one (b, h) sequence and walks its chunks in order, keeping the
 // fp32 state h on chip for the whole sequence (no chunk state goes to HBM).
 //
 // Chunk layout.  Chunk c has Q = 64 source rows: row 0 is the token just
 // before the chunk (t0 - 1, the carry-in of the trapezoid's beta term) and rows
-// 1..63 are the chunk's own tokens t0 .. t0+62 (t0 = 63 c).  With the running
-// angle phi and the chunk-local sums (row 0 has cs_0 = 0, psi_0 = 0)
+// 1..63 are the chunk's own tokens t0 .. t0+62 (t0 = 63 c).  With the chunk-local
+// sums (row 0 has cs_0 = 0, psi_0 = 0)
 //     cs_r = sum_{k=1..r} logdecay_k,   psi_r = sum_{k=1..r} theta_k,
-// the rotated vectors are Bbar_r = R(Phi_c + psi_r) B_r, Cbar_r likewise, where
-// Phi_c = phi_{t0-1} is carried from chunk to chunk, and the recurrence
-// ("TorchMamba" README, "Math notes", M3 SISO: exponential-trapezoidal update
-// h_t = alpha_t h_{t-1} + beta_t Bbar_{t-1} x_{t-1}^T + gamma_t Bbar_t x_t^T)
-// unrolled over the chunk reads, for output rows r = 1..63,
+// the rotated vectors are Bbar_r = R(Phi_c + psi_r) B_r and Cbar_r likewise, with
+// Phi_c = phi_{t0-1} carried from chunk to chunk.  The recurrence ("TorchMamba"
+// README, "Math notes", M3 SISO: h_t = alpha_t h_{t-1} + beta_t Bbar_{t-1} x_{t-1}^T
+// + gamma_t Bbar_t x_t^T) unrolled over the chunk reads, for output rows r = 1..63,
 //     y_r   = exp(cs_r) Cbar_r^T h + sum_{u<=r} W(r,u) (Cbar_r^T Bbar_u) x_u + D x_r
 //     h_end = exp(cs_63) h + sum_u W(63,u) Bbar_u x_u^T
 //     W(r,r) = gamma_r,   W(r,u<r) = exp(cs_r - cs_{u+1}) (gamma_u alpha_{u+1} + beta_{u+1}),
 // with gamma_0 := 0 (row 0's own gamma term belongs to the previous chunk), so
-// the column u = 0 carries exactly the beta boundary term.  The gamma and beta
-// terms form one mask ("TorchMamba" README: "the parallel mask is L = 1SS @
-// band") applied to the Gram matrix in a single pass.
+// column u = 0 carries exactly the beta boundary term: the gamma and beta terms
+// form one mask ("TorchMamba" README: "the parallel mask is L = 1SS @ band").
 //
-// Tensor-core work per chunk (mma.sync m16n8k16, bf16 in, fp32 accumulate):
-//   G   = Cbar Bbar^T                 lower-triangular 16x8 tiles only
-//   Y   = diag(exp cs) Cbar h  +  (W o G) X
-//   h   = exp(cs_63) h + (W_end o Bbar)^T X, with W_end o Bbar split into a
-//         bf16 high part and a bf16 residual so the state update carries one
-//         rounding of ~2^-17 instead of two of 2^-9 (X itself is exact bf16).
-// Decay/angle cumsums, sincos, rotations, masks and epilogues run on the SIMT
-// pipes.  Shared tiles use a 16-byte XOR swizzle so ldmatrix is conflict-free
-// without padding, which keeps two CTAs resident per SM.
+// Tensor-core work per chunk (tcgen05.mma kind::f16, bf16 in, fp32 in TMEM),
+// issued by one thread:
+//   G  = Cbar Bbar^T                 M=64  N=64 K=128   (TMEM cols   0..63)
+//   Y1 = Cbar h_bf16                 M=64  N=64 K=128   (TMEM cols  64..127)
+//   S  = (W_end o Bbar)^T X          M=128 N=64 K=64 x2 (TMEM cols 192..255), the
+//        operand split into a bf16 high part and a bf16 residual, so the state
+//        update carries one rounding of ~2^-17 (X itself is exact bf16)
+//   Y2 = (W o G) X                   M=64  N=64 K=64    (TMEM cols 128..191)
+// and y = exp(cs) Y1 + Y2 + D x, h = exp(cs_63) h + S on the SIMT pipes, where the
+// decay/angle cumsums, sincos, rotations and the mask also run.  Operand tiles
+// live in shared memory in the 128-byte-swizzled canonical layouts: K-major rows
+// of 128 B for Cbar, Bbar and the mask; MN-major 64-element atoms for X, h and
+// W_end o Bbar.  Loads use cp.async with zero-fill for the ragged last chunk.
+// Two CTAs share an SM (about 100 KB of shared memory and 256 TMEM columns each).
 #include <cuda_bf16.h>
 
 #include "common.cuh"
 #include "internal.h"
+#include "tc5.cuh"
 
 namespace m3ssd {
+
+// Number of bounded device-side waits that ran out (read by the host query).
+__device__ unsigned int g_chunk_wait_timeouts;
+
 namespace {
 
 constexpr int Q = 64;       // source rows per chunk (1 carry-in + 63 tokens)
@@ -45,62 +54,54 @@ constexpr int PD = 64;      // head dim P
 constexpr int NH = NS / 2;  // rotation pairs
 constexpr int kThreads = 256;
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kColG = 0, kColY1 = 64, kColY2 = 128, kColS = 192;
+constexpr uint32_t kAtom = Q * 128;       // bytes of one 64-element atom of a Q-row tile
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // an mbarrier wait gives up after 2 s
+constexpr uint32_t kIdescG = tc5::idesc_bf16(64, 64, false, false);   // G
+constexpr uint32_t kIdescY = tc5::idesc_bf16(64, 64, false, true);    // Y1, Y2
+constexpr uint32_t kIdescS = tc5::idesc_bf16(128, 64, true, true);    // S
 
 typedef __nv_bfloat16 bf16;
 
-// 16-byte-chunk XOR swizzle of a row-major bf16 tile with RL elements a row.
-template <int RL>
-__device__ __forceinline__ int swz(int r, int c) {
-  return r * RL + ((((c >> 3) ^ (r & 7))) << 3) + (c & 7);
+// Byte offset of element (r, n) in a Q-row tile of 128 elements a row, stored
+// as two 64-element atoms of 128-byte rows with the 16-byte XOR swizzle.
+__device__ __forceinline__ uint32_t off2(int r, int n) {
+  return (uint32_t)((n >> 6) * kAtom + r * 128 + ((((n & 63) >> 3) ^ (r & 7)) << 4) +
+                    ((n & 7) << 1));
+}
+// Byte offset of element (r, c) in a tile of 64 elements (128 B) a row.
+__device__ __forceinline__ uint32_t off1(int r, int c) {
+  return (uint32_t)(r * 128 + ((((c >> 3) ^ (r & 7))) << 4) + ((c & 7) << 1));
 }
 
 struct Smem {
   union {
-    float theta[Q][NH];  // raw theta of the chunk (phase R1 only)
-    bf16 bw_hi[Q * NS];  // high part of W_end o Bbar (phase R2 .. S)
+    float theta[Q][NH];        // raw theta of the chunk (phase R1 only)
+    uint8_t bw_hi[2 * kAtom];  // high part of W_end o Bbar (phase R2 .. S MMA)
   } u;
-  bf16 bw_lo[Q * NS];    // residual of W_end o Bbar
-  bf16 B[Q * NS];        // raw B, then Bbar
-  bf16 C[Q * NS];        // raw C, then Cbar
-  bf16 X[Q * PD];        // X rows of the chunk (row 0 = carry-in token)
-  bf16 M[Q * Q];         // masked Gram W o G
-  bf16 Hs[NS * PD];      // bf16 copy of h for the state-to-output product
+  uint8_t bw_lo[2 * kAtom];    // residual of W_end o Bbar
+  uint8_t B[2 * kAtom];        // raw B, then Bbar
+  uint8_t C[2 * kAtom];        // raw C, then Cbar
+  uint8_t X[Q * 128];          // X rows of the chunk (row 0 = carry-in token)
+  uint8_t M[Q * 128];          // masked Gram W o G
+  uint8_t Hs[NS * 128];        // bf16 copy of h for the state-to-output product
   float segtot[4][NH];
   float cs2[Q], ecs[Q], cvec[Q], wend[Q], gam[Q];
-  float ecos[NH], esin[NH], Phi[NH];  // exp(i Phi_c) per pair and Phi_c itself
+  float ecos[NH], esin[NH], Phi[NH];     // exp(i Phi_c) per pair and Phi_c itself
   float necos[NH], nesin[NH], nPhi[NH];  // the same for the next chunk
   float scal[4];
+  uint64_t mbar[2];
+  uint32_t tmem;
+  uint32_t err;
 };
 
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(smem_u32(dst)), "l"(src),
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src),
                "r"(valid ? 16 : 0));
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;\n" ::); }
-
-__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void* p) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(smem_u32(p)));
-}
-__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], const void* p) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(smem_u32(p)));
-}
-// D += A * B, m16n8k16, bf16 inputs, fp32 accumulators.
-__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
-                                         uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-      "{%8,%9}, {%0,%1,%2,%3};\n"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -110,16 +111,12 @@ __device__ __forceinline__ float2 unpack_bf16(uint32_t u) {
   return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
 }
 
-// Lower-triangular 16x8 tile u (0..19) of the 64x64 Gram: block row bi, column tile nj.
-__device__ __forceinline__ void gram_unit(int u, int& bi, int& nj) {
-  bi = (u < 2) ? 0 : (u < 6) ? 1 : (u < 12) ? 2 : 3;
-  nj = u - bi * (bi + 1);
-}
-
 template <bool ROT>
 __global__ void __launch_bounds__(kThreads, 2) fwd_chunk_kernel(FwdArgs a) {
-  extern __shared__ __align__(128) unsigned char smem_raw[];
-  Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  // operand tiles need a 1024-byte aligned shared-space address
+  const uint32_t raw_addr = tc5::saddr(smem_raw);
+  Smem& sm = *reinterpret_cast<Smem*>(smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr));
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t H = a.H, L = a.L, G = a.G;
   const int64_t bh = blockIdx.x;
@@ -130,6 +127,10 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_chunk_kernel(FwdArgs a) {
   const bf16* Cg = static_cast<const bf16*>(a.C);
   bf16* Yg = static_cast<bf16*>(a.Y);
   const float Dh = a.D ? a.D[h] : 0.f;
+  const uint32_t aB = tc5::saddr(sm.B), aC = tc5::saddr(sm.C), aX = tc5::saddr(sm.X);
+  const uint32_t aM = tc5::saddr(sm.M), aH = tc5::saddr(sm.Hs);
+  const uint32_t aWh = tc5::saddr(sm.u.bw_hi), aWl = tc5::saddr(sm.bw_lo);
+  const uint32_t aT = tc5::saddr(&sm.u.theta[0][0]);
 
   // Row r of chunk c holds token c*QT - 1 + r; rows outside [0, L) are zero-filled.
   auto row_token = [&](int c, int r) -> int64_t { return (int64_t)c * QT - 1 + r; };
@@ -141,29 +142,29 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_chunk_kernel(FwdArgs a) {
       const int64_t t = row_token(c, row);
       const bool ok = a.theta && t >= 0 && t < L;
       const float* src = ok ? a.theta + ((b * L + t) * H + h) * NH + col : a.logdecay;
-      cp_async16(&sm.u.theta[row][col], src, ok);
+      cp_async16(aT + (uint32_t)(row * NH + col) * 4u, src, ok);
     }
   };
-  auto load_b = [&](int c, const bf16* base, bf16* dst) {
+  auto load_bc = [&](int c, const bf16* base, uint32_t dst) {
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       const int idx = tid + k * kThreads;
-      const int row = idx >> 4, col = (idx & 15) * 8;
+      const int row = idx >> 4, c8 = idx & 15;
       const int64_t t = row_token(c, row);
       const bool ok = t >= 0 && t < L;
-      const bf16* src = ok ? base + ((b * L + t) * G + g) * NS + col : base;
-      if (t >= 0) cp_async16(&dst[swz<NS>(row, col)], src, ok);
+      const bf16* src = ok ? base + ((b * L + t) * G + g) * NS + c8 * 8 : base;
+      if (t >= 0) cp_async16(dst + off2(row, c8 * 8), src, ok);
     }
   };
   auto load_x = [&](int c) {
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
       const int idx = tid + k * kThreads;
-      const int row = idx >> 3, col = (idx & 7) * 8;
+      const int row = idx >> 3, c8 = idx & 7;
       const int64_t t = row_token(c, row);
       const bool ok = t >= 0 && t < L;
-      const bf16* src = ok ? Xg + ((b * L + t) * H + h) * PD + col : Xg;
-      if (t >= 0) cp_async16(&sm.X[swz<PD>(row, col)], src, ok);
+      const bf16* src = ok ? Xg + ((b * L + t) * H + h) * PD + c8 * 8 : Xg;
+      if (t >= 0) cp_async16(aX + off1(row, c8 * 8), src, ok);
     }
   };
   // warp 0 keeps logdecay / beta / gamma of rows lane and lane + 32 in registers
@@ -182,18 +183,29 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_chunk_kernel(FwdArgs a) {
   };
 
   // ---- prologue -------------------------------------------------------------
+  if (warp == 0) tc5::tmem_alloc(&sm.tmem, kTmemCols);
+  if (tid == 0) {
+    tc5::mbar_init(&sm.mbar[0], 1);
+    tc5::mbar_init(&sm.mbar[1], 1);
+    tc5::fence_mbar_init();
+    sm.err = 0;
+  }
   if (ROT) load_theta(0);
-  load_b(0, Bg, sm.B);
-  load_b(0, Cg, sm.C);
+  load_bc(0, Bg, aB);
+  load_bc(0, Cg, aC);
   load_x(0);
   cp_async_commit();
   if (warp == 0) load_params(0);
   // row 0 of chunk 0 is the cache's previous token (zero when absent)
   if (tid < NS) {
-    sm.B[swz<NS>(0, tid)] = __float2bfloat16_rn(a.bprev0 ? a.bprev0[(b * G + g) * NS + tid] : 0.f);
-    sm.C[swz<NS>(0, tid)] = __float2bfloat16_rn(0.f);
+    const float bp = a.bprev0 ? a.bprev0[(b * G + g) * NS + tid] : 0.f;
+    *reinterpret_cast<bf16*>(sm.B + off2(0, tid)) = __float2bfloat16_rn(bp);
+    *reinterpret_cast<bf16*>(sm.C + off2(0, tid)) = __float2bfloat16_rn(0.f);
   }
-  if (tid < PD) sm.X[swz<PD>(0, tid)] = __float2bfloat16_rn(a.xprev0 ? a.xprev0[bh * PD + tid] : 0.f);
+  if (tid < PD) {
+    const float xp = a.xprev0 ? a.xprev0[bh * PD + tid] : 0.f;
+    *reinterpret_cast<bf16*>(sm.X + off1(0, tid)) = __float2bfloat16_rn(xp);
+  }
   if (ROT && tid < NH) {
     const float ph0 = a.angle0 ? a.angle0[bh * NH + tid] : 0.f;
     sm.Phi[tid] = ph0;
@@ -203,40 +215,41 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_chunk_kernel(FwdArgs a) {
     sm.esin[tid] = s;
   }
 
-  // state fragment: rows rb + mi*16 + lane/4 (+8), cols ph*32 + j*8 + 2*(lane%4) (+1)
-  const int rb = 32 * (warp & 3), ph = warp >> 2;
-  float hs[2][4][4];
+  // state fragment: row n = 32 (warp % 4) + lane, columns cb .. cb + 31
+  const int n_row = 32 * (warp & 3) + lane, cb = 32 * (warp >> 2);
+  float hs[32];
+  {
+    const float4* src = reinterpret_cast<const float4*>(a.h0 + (bh * NS + n_row) * PD + cb);
 #pragma unroll
-  for (int mi = 0; mi < 2; ++mi)
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-#pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        const int n = rb + mi * 16 + (lane >> 2) + 8 * hf;
-        const int p = ph * 32 + j * 8 + 2 * (lane & 3);
-        float2 v = make_float2(0.f, 0.f);
-        if (a.h0) v = *reinterpret_cast<const float2*>(&a.h0[(bh * NS + n) * PD + p]);
-        hs[mi][j][2 * hf] = v.x;
-        hs[mi][j][2 * hf + 1] = v.y;
-      }
+    for (int j = 0; j < 8; ++j) {
+      const float4 v = a.h0 ? src[j] : make_float4(0.f, 0.f, 0.f, 0.f);
+      hs[4 * j] = v.x; hs[4 * j + 1] = v.y; hs[4 * j + 2] = v.z; hs[4 * j + 3] = v.w;
+    }
+  }
   auto store_state_bf16 = [&]() {
 #pragma unroll
-    for (int mi = 0; mi < 2; ++mi)
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          const int n = rb + mi * 16 + (lane >> 2) + 8 * hf;
-          const int p = ph * 32 + j * 8 + 2 * (lane & 3);
-          *reinterpret_cast<uint32_t*>(&sm.Hs[swz<PD>(n, p)]) =
-              pack_bf16(hs[mi][j][2 * hf], hs[mi][j][2 * hf + 1]);
-        }
+    for (int q = 0; q < 4; ++q) {
+      uint4 v;
+      v.x = pack_bf16(hs[8 * q + 0], hs[8 * q + 1]);
+      v.y = pack_bf16(hs[8 * q + 2], hs[8 * q + 3]);
+      v.z = pack_bf16(hs[8 * q + 4], hs[8 * q + 5]);
+      v.w = pack_bf16(hs[8 * q + 6], hs[8 * q + 7]);
+      *reinterpret_cast<uint4*>(sm.Hs + off1(n_row, cb + 8 * q)) = v;
+    }
   };
   store_state_bf16();
+  tc5::fence_proxy_async();
+  tc5::fence_before_sync();
+  __syncthreads();
+  tc5::fence_after_sync();
+  const uint32_t tmem = sm.tmem;
+  // this warp's TMEM lane quarter (rows of the M=64 and M=128 accumulators)
+  const uint32_t tlane = (uint32_t)(32 * (warp & 3)) << 16;
 
   // ---- chunk walk -------------------------------------------------------------
   for (int c = 0; c < nC; ++c) {
     const int64_t tbase = (int64_t)c * QT - 1;  // token of row 0
+    const uint32_t par = (uint32_t)(c & 1);
     cp_async_wait_all();
     __syncthreads();  // S1: theta, B, C, X of this chunk are in shared memory
 
@@ -306,11 +319,12 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_chunk_kernel(FwdArgs a) {
 #pragma unroll 4
       for (int k = 0; k < 16; ++k) {
         const int r = seg * 16 + k;
-        uint32_t* pb = reinterpret_cast<uint32_t*>(&sm.B[swz<NS>(r, 2 * pi)]);
-        uint32_t* pc = reinterpret_cast<uint32_t*>(&sm.C[swz<NS>(r, 2 * pi)]);
+        const uint32_t o = off2(r, 2 * pi);
+        uint32_t* pb = reinterpret_cast<uint32_t*>(sm.B + o);
+        uint32_t* pc = reinterpret_cast<uint32_t*>(sm.C + o);
         float2 bv = unpack_bf16(*pb);
-        float2 cv = unpack_bf16(*pc);
         if (ROT) {
+          float2 cv = unpack_bf16(*pc);
           float s, co;
           fast_sincos(psi[k] + off, &s, &co);
           // exp(i (Phi_c + psi)) = exp(i Phi_c) exp(i psi)
@@ -324,8 +338,8 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_chunk_kernel(FwdArgs a) {
         const float w0 = we * bv.x, w1 = we * bv.y;
         const uint32_t hi = pack_bf16(w0, w1);
         const float2 hv = unpack_bf16(hi);
-        *reinterpret_cast<uint32_t*>(&sm.u.bw_hi[swz<NS>(r, 2 * pi)]) = hi;
-        *reinterpret_cast<uint32_t*>(&sm.bw_lo[swz<NS>(r, 2 * pi)]) = pack_bf16(w0 - hv.x, w1 - hv.y);
+        *reinterpret_cast<uint32_t*>(sm.u.bw_hi + o) = hi;
+        *reinterpret_cast<uint32_t*>(sm.bw_lo + o) = pack_bf16(w0 - hv.x, w1 - hv.y);
       }
       if (ROT && seg == 3) {
         const float pnext = wrap_angle(sm.Phi[pi] + psi[15] + off);
@@ -336,152 +350,121 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_chunk_kernel(FwdArgs a) {
         sm.nesin[pi] = s;
       }
     }
-    __syncthreads();  // S3: Bbar, Cbar, W_end o Bbar ready
+    tc5::fence_proxy_async();
+    __syncthreads();  // S3: Cbar, Bbar, W_end o Bbar ready
+    if (tid == 0) {
+      tc5::fence_after_sync();
+      // G = Cbar Bbar^T (both K-major), K = 128 in 8 steps of 16
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const uint32_t ko = (uint32_t)((j >> 2) * kAtom + (j & 3) * 32);
+        tc5::mma_bf16(tmem + kColG, tc5::desc_sw128(aC + ko, 16, 1024),
+                      tc5::desc_sw128(aB + ko, 16, 1024), kIdescG, j > 0);
+      }
+      tc5::commit(&sm.mbar[0]);
+      // Y1 = Cbar h (h MN-major: K = n, rows of 128 B)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const uint32_t ko = (uint32_t)((j >> 2) * kAtom + (j & 3) * 32);
+        tc5::mma_bf16(tmem + kColY1, tc5::desc_sw128(aC + ko, 16, 1024),
+                      tc5::desc_sw128(aH + (uint32_t)j * 2048u, kAtom, 1024), kIdescY, j > 0);
+      }
+      // S = (W_end o Bbar)^T X with the operand in two parts (A and B MN-major), K = 64
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const uint32_t aw = (j < 4 ? aWh : aWl) + (uint32_t)(j & 3) * 2048u;
+        tc5::mma_bf16(tmem + kColS, tc5::desc_sw128(aw, kAtom, 1024),
+                      tc5::desc_sw128(aX + (uint32_t)(j & 3) * 2048u, kAtom, 1024), kIdescS,
+                      j > 0);
+      }
+    }
     if (ROT && tid < NH) {
       sm.Phi[tid] = sm.nPhi[tid];
       sm.ecos[tid] = sm.necos[tid];
       sm.esin[tid] = sm.nesin[tid];
     }
 
-    // -- phase G: masked Gram -> M ---------------------------------------------
-    for (int u = warp; u < 20; u += 8) {
-      int bi, nj;
-      gram_unit(u, bi, nj);
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int kk = 0; kk < 8; kk += 2) {
-        uint32_t bfr[4];
-        ldsm_x4(bfr, &sm.B[swz<NS>(nj * 8 + (lane & 7), kk * 16 + 8 * (lane >> 3))]);
-#pragma unroll
-        for (int k2 = 0; k2 < 2; ++k2) {
-          uint32_t afr[4];
-          ldsm_x4(afr, &sm.C[swz<NS>(bi * 16 + (lane & 7) + 8 * ((lane >> 3) & 1),
-                                     (kk + k2) * 16 + 8 * (lane >> 4))]);
-          mma16816(acc, afr, bfr[2 * k2], bfr[2 * k2 + 1]);
-        }
-      }
+    // -- phase G: masked Gram -> M (rows 16 (warp % 4) + .., columns cb + ..) -------
+    {
+      if (!tc5::mbar_wait(&sm.mbar[0], par, kWaitLimitNs)) sm.err = 1;
+      tc5::fence_after_sync();
+      uint32_t gr[16];
+      tc5::ld_16x256b_x4(tmem + tlane + kColG + (uint32_t)cb, gr);
+      tc5::wait_ld();
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf) {
-        const int t = bi * 16 + (lane >> 2) + 8 * hf;
-        const int s0 = nj * 8 + 2 * (lane & 3);
-        float w[2];
+        const int t = 16 * (warp & 3) + (lane >> 2) + 8 * hf;
+        const float cst = sm.cs2[t], gt = sm.gam[t];
 #pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          const int s = s0 + j;
-          w[j] = (s > t) ? 0.f
-                 : (s == t) ? sm.gam[t]
-                            : exp2f(sm.cs2[t] - sm.cs2[s + 1]) * sm.cvec[s];
+        for (int q = 0; q < 4; ++q) {
+          const int s0 = cb + 8 * q + 2 * (lane & 3);
+          float wv[2];
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const int s = s0 + j;
+            wv[j] = (s > t) ? 0.f : (s == t) ? gt : exp2f(cst - sm.cs2[s + 1]) * sm.cvec[s];
+          }
+          *reinterpret_cast<uint32_t*>(sm.M + off1(t, s0)) =
+              pack_bf16(__uint_as_float(gr[4 * q + 2 * hf]) * wv[0],
+                        __uint_as_float(gr[4 * q + 2 * hf + 1]) * wv[1]);
         }
-        *reinterpret_cast<uint32_t*>(&sm.M[swz<Q>(t, s0)]) =
-            pack_bf16(acc[2 * hf] * w[0], acc[2 * hf + 1] * w[1]);
       }
     }
-    __syncthreads();  // S4: M ready; Bbar (sm.B) is free
-    if (c + 1 < nC) {
-      load_b(c + 1, Bg, sm.B);
-      cp_async_commit();
-    }
-
-    // -- phase Y: outputs, 16 rows x 32 columns per warp ------------------------
-    {
-      const int mt = warp & 3;
-      float acc[4][4];
+    tc5::fence_proxy_async();
+    tc5::fence_before_sync();
+    __syncthreads();  // S4: M ready; the Gram has consumed Bbar
+    if (tid == 0) {
+      tc5::fence_after_sync();
 #pragma unroll
       for (int j = 0; j < 4; ++j)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) acc[j][e] = 0.f;
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        uint32_t afr[4];
-        ldsm_x4(afr, &sm.C[swz<NS>(mt * 16 + (lane & 7) + 8 * ((lane >> 3) & 1),
-                                   kk * 16 + 8 * (lane >> 4))]);
-#pragma unroll
-        for (int np = 0; np < 2; ++np) {
-          uint32_t bfr[4];
-          ldsm_x4_t(bfr, &sm.Hs[swz<PD>(kk * 16 + (lane & 7) + 8 * ((lane >> 3) & 1),
-                                        ph * 32 + np * 16 + 8 * (lane >> 4))]);
-          mma16816(acc[2 * np], afr, bfr[0], bfr[1]);
-          mma16816(acc[2 * np + 1], afr, bfr[2], bfr[3]);
-        }
-      }
-      const float e_lo = sm.ecs[mt * 16 + (lane >> 2)];
-      const float e_hi = sm.ecs[mt * 16 + (lane >> 2) + 8];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        acc[j][0] *= e_lo; acc[j][1] *= e_lo;
-        acc[j][2] *= e_hi; acc[j][3] *= e_hi;
-      }
-      for (int kk = 0; kk <= mt; ++kk) {
-        uint32_t afr[4];
-        ldsm_x4(afr, &sm.M[swz<Q>(mt * 16 + (lane & 7) + 8 * ((lane >> 3) & 1),
-                                  kk * 16 + 8 * (lane >> 4))]);
-#pragma unroll
-        for (int np = 0; np < 2; ++np) {
-          uint32_t bfr[4];
-          ldsm_x4_t(bfr, &sm.X[swz<PD>(kk * 16 + (lane & 7) + 8 * ((lane >> 3) & 1),
-                                       ph * 32 + np * 16 + 8 * (lane >> 4))]);
-          mma16816(acc[2 * np], afr, bfr[0], bfr[1]);
-          mma16816(acc[2 * np + 1], afr, bfr[2], bfr[3]);
-        }
-      }
-#pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        const int r = mt * 16 + (lane >> 2) + 8 * hf;
-        const int64_t t = tbase + r;
-        if (r > 0 && t < L) {
-          bf16* yrow = Yg + ((b * L + t) * H + h) * PD;
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int p = ph * 32 + j * 8 + 2 * (lane & 3);
-            const float2 xv = unpack_bf16(*reinterpret_cast<const uint32_t*>(&sm.X[swz<PD>(r, p)]));
-            *reinterpret_cast<uint32_t*>(yrow + p) =
-                pack_bf16(acc[j][2 * hf] + Dh * xv.x, acc[j][2 * hf + 1] + Dh * xv.y);
-          }
-        }
-      }
+        tc5::mma_bf16(tmem + kColY2, tc5::desc_sw128(aM + (uint32_t)j * 32u, 16, 1024),
+                      tc5::desc_sw128(aX + (uint32_t)j * 2048u, kAtom, 1024), kIdescY, j > 0);
+      tc5::commit(&sm.mbar[1]);
     }
-    __syncthreads();  // S5: readers of Hs and Cbar are done
     if (c + 1 < nC) {
-      load_b(c + 1, Cg, sm.C);
+      load_bc(c + 1, Bg, aB);
       cp_async_commit();
     }
 
-    // -- phase S: h = exp(cs_end) h + (W_end o Bbar)^T X ---------------------------
+    // -- phase Y + S: outputs and the state update ---------------------------------
     {
-      const float eE = sm.scal[0];
+      if (!tc5::mbar_wait(&sm.mbar[1], par, kWaitLimitNs)) sm.err = 1;
+      tc5::fence_after_sync();
+      uint32_t y1[16], y2[16], sv[32];
+      tc5::ld_16x256b_x4(tmem + tlane + kColY1 + (uint32_t)cb, y1);
+      tc5::ld_16x256b_x4(tmem + tlane + kColY2 + (uint32_t)cb, y2);
+      tc5::ld_32x32b_x32(tmem + tlane + kColS + (uint32_t)cb, sv);
+      tc5::wait_ld();
 #pragma unroll
-      for (int mi = 0; mi < 2; ++mi)
+      for (int hf = 0; hf < 2; ++hf) {
+        const int r = 16 * (warp & 3) + (lane >> 2) + 8 * hf;
+        const int64_t t = tbase + r;
+        if (r > 0 && t < L) {
+          const float er = sm.ecs[r];
+          bf16* yrow = Yg + ((b * L + t) * H + h) * PD;
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) hs[mi][j][e] *= eE;
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        uint32_t bx[2][4];
-#pragma unroll
-        for (int np = 0; np < 2; ++np)
-          ldsm_x4_t(bx[np], &sm.X[swz<PD>(kk * 16 + (lane & 7) + 8 * ((lane >> 3) & 1),
-                                          ph * 32 + np * 16 + 8 * (lane >> 4))]);
-#pragma unroll
-        for (int mi = 0; mi < 2; ++mi) {
-          const int arow = kk * 16 + (lane & 7) + 8 * (lane >> 4);
-          const int acol = rb + mi * 16 + 8 * ((lane >> 3) & 1);
-          uint32_t ahi[4], alo[4];
-          ldsm_x4_t(ahi, &sm.u.bw_hi[swz<NS>(arow, acol)]);
-          ldsm_x4_t(alo, &sm.bw_lo[swz<NS>(arow, acol)]);
-#pragma unroll
-          for (int np = 0; np < 2; ++np) {
-            mma16816(hs[mi][2 * np], ahi, bx[np][0], bx[np][1]);
-            mma16816(hs[mi][2 * np + 1], ahi, bx[np][2], bx[np][3]);
-            mma16816(hs[mi][2 * np], alo, bx[np][0], bx[np][1]);
-            mma16816(hs[mi][2 * np + 1], alo, bx[np][2], bx[np][3]);
+          for (int q = 0; q < 4; ++q) {
+            const int p = cb + 8 * q + 2 * (lane & 3);
+            const float2 xv = unpack_bf16(*reinterpret_cast<const uint32_t*>(sm.X + off1(r, p)));
+            const float v0 = er * __uint_as_float(y1[4 * q + 2 * hf]) +
+                             __uint_as_float(y2[4 * q + 2 * hf]) + Dh * xv.x;
+            const float v1 = er * __uint_as_float(y1[4 * q + 2 * hf + 1]) +
+                             __uint_as_float(y2[4 * q + 2 * hf + 1]) + Dh * xv.y;
+            *reinterpret_cast<uint32_t*>(yrow + p) = pack_bf16(v0, v1);
           }
         }
       }
+      const float eE = sm.scal[0];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) hs[j] = fmaf(eE, hs[j], __uint_as_float(sv[j]));
       store_state_bf16();
     }
-    __syncthreads();  // S6: theta / W_end o Bbar / X buffers are free
+    tc5::fence_proxy_async();
+    tc5::fence_before_sync();
+    __syncthreads();  // S5: every tensor-core operand of this chunk is consumed
+    if (sm.err) break;
     if (c + 1 < nC) {
+      load_bc(c + 1, Cg, aC);
       if (ROT) load_theta(c + 1);
       load_x(c + 1);
       cp_async_commit();
@@ -489,30 +472,32 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_chunk_kernel(FwdArgs a) {
   }
   cp_async_wait_all();
 
-  // ---- outputs of the last token ----------------------------------------------
-  if (a.hT) {
+  // ---- outputs of the last token, TMEM release ---------------------------------
+  if (sm.err) {
+    if (tid == 0) atomicAdd(&g_chunk_wait_timeouts, 1u);
+  } else {
+    if (a.hT) {
+      float4* dst = reinterpret_cast<float4*>(a.hT + (bh * NS + n_row) * PD + cb);
 #pragma unroll
-    for (int mi = 0; mi < 2; ++mi)
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          const int n = rb + mi * 16 + (lane >> 2) + 8 * hf;
-          const int p = ph * 32 + j * 8 + 2 * (lane & 3);
-          *reinterpret_cast<float2*>(&a.hT[(bh * NS + n) * PD + p]) =
-              make_float2(hs[mi][j][2 * hf], hs[mi][j][2 * hf + 1]);
-        }
+      for (int j = 0; j < 8; ++j)
+        dst[j] = make_float4(hs[4 * j], hs[4 * j + 1], hs[4 * j + 2], hs[4 * j + 3]);
+    }
+    if (a.angleT && tid < NH)
+      a.angleT[bh * NH + tid] = ROT ? sm.Phi[tid] : (a.angle0 ? a.angle0[bh * NH + tid] : 0.f);
+    if (a.xprevT && tid < PD)
+      a.xprevT[bh * PD + tid] = __bfloat162float(Xg[((b * L + L - 1) * H + h) * PD + tid]);
+    if (a.bprevT && h % (H / G) == 0 && tid < NS)
+      a.bprevT[(b * G + g) * NS + tid] =
+          __bfloat162float(Bg[((b * L + L - 1) * G + g) * NS + tid]);
   }
-  if (a.angleT && tid < NH)
-    a.angleT[bh * NH + tid] = ROT ? sm.Phi[tid] : (a.angle0 ? a.angle0[bh * NH + tid] : 0.f);
-  if (a.xprevT && tid < PD) a.xprevT[bh * PD + tid] = __bfloat162float(Xg[((b * L + L - 1) * H + h) * PD + tid]);
-  if (a.bprevT && h % (H / G) == 0 && tid < NS)
-    a.bprevT[(b * G + g) * NS + tid] = __bfloat162float(Bg[((b * L + L - 1) * G + g) * NS + tid]);
+  tc5::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) tc5::tmem_dealloc(tmem, kTmemCols);
 }
 
 template <bool ROT>
 cudaError_t launch_variant(const FwdArgs& a, cudaStream_t s) {
-  const size_t smem = sizeof(Smem);
+  const size_t smem = sizeof(Smem) + 1024;
   cudaError_t e = cudaFuncSetAttribute(fwd_chunk_kernel<ROT>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -534,6 +519,13 @@ cudaError_t launch_fwd_chunk(const FwdArgs& a, cudaStream_t s) {
   if (a.b * a.H == 0) return cudaSuccess;
   if (a.theta != nullptr || a.angle0 != nullptr) return launch_variant<true>(a, s);
   return launch_variant<false>(a, s);
+}
+
+cudaError_t read_and_clear_wait_timeouts(unsigned int* count) {
+  const unsigned int zero = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(count, g_chunk_wait_timeouts, sizeof(unsigned int));
+  if (e != cudaSuccess) return e;
+  return cudaMemcpyToSymbol(g_chunk_wait_timeouts, &zero, sizeof(unsigned int));
 }
 
 }  // namespace m3ssd

@@ -53,6 +53,9 @@ cudaError_t launch_fwd_seq(const FwdArgs& a, cudaStream_t s);
 // Chunked bf16 tensor-core forward (N = 128, P = 64).
 cudaError_t launch_fwd_chunk(const FwdArgs& a, cudaStream_t s);
 bool fwd_chunk_supported(const FwdArgs& a);
+// Count of bounded device-side waits in the chunked forward that ran out since
+// the last call; reading it synchronises the device and clears the count.
+cudaError_t read_and_clear_wait_timeouts(unsigned int* count);
 // Decode step (two launches: the state/outputs, then b_prev <- B_t).
 cudaError_t launch_step(const StepArgs& a, cudaStream_t s);
 

@@ -59,6 +59,14 @@ const char* m3ssd_status_string(m3ssd_status s) {
   return "unknown status";
 }
 
+m3ssd_status m3ssd_device_wait_timeouts(uint32_t* count) {
+  if (!count) return M3SSD_ERR_INVALID_ARG;
+  unsigned int n = 0;
+  const m3ssd_status st = from_cuda(m3ssd::read_and_clear_wait_timeouts(&n));
+  *count = n;
+  return st;
+}
+
 size_t m3ssd_fwd_workspace_size(const m3ssd_dims* dims) {
   (void)dims;
   return 0;

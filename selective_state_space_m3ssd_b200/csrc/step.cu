@@ -137,6 +137,86 @@ __global__ void __launch_bounds__(kThreads) step_kernel(StepArgs a) {
   }
 }
 
+// Specialised step for N = 128, P = 64 (the decode workload): 128 threads, each
+// owning one 4-wide column slice of 16 state rows.  The 16 float4 loads of the
+// state are issued before the rotation prologue, so the state stream (32 KB per
+// CTA) is in flight while the angles, sincos and rotations are computed.
+constexpr int kN = 128, kP = 64, kThreads128 = 128, kRows = kN / (kThreads128 / (kP / 4));
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads128) step_kernel_n128p64(StepArgs a) {
+  __shared__ float Bb[kN], Cb[kN], Bpb[kN], xs[kP], xps[kP];
+  __shared__ float4 red[kThreads128 / 32][kP / 4];
+  const int64_t H = a.H, G = a.G;
+  const int64_t bh = blockIdx.x;
+  const int64_t b = bh / H, h = bh % H, g = h / (H / G);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int q = tid & 15, r0 = tid >> 4;  // column slice q, rows r0 + 8k
+  float4* S = reinterpret_cast<float4*>(a.ssm + bh * kN * kP);
+  float4 hv[kRows];
+#pragma unroll
+  for (int k = 0; k < kRows; ++k) hv[k] = S[(r0 + 8 * k) * (kP / 4) + q];
+
+  const T* Bt = static_cast<const T*>(a.B_t) + (b * G + g) * kN;
+  const T* Ct = static_cast<const T*>(a.C_t) + (b * G + g) * kN;
+  const float* bprev = a.b_prev + (b * G + g) * kN;
+  if (tid < kN / 2) {
+    const int i = tid;
+    const float ang = a.angle[bh * (kN / 2) + i];
+    const float ph = wrap_angle(ang + (a.theta_t ? a.theta_t[bh * (kN / 2) + i] : 0.f));
+    float s, c, s0, c0;
+    sincosf(ph, &s, &c);
+    sincosf(ang, &s0, &c0);
+    const float2 rb = rot2(c, s, to_f32(Bt[2 * i]), to_f32(Bt[2 * i + 1]));
+    const float2 rc = rot2(c, s, to_f32(Ct[2 * i]), to_f32(Ct[2 * i + 1]));
+    const float2 rp = rot2(c0, s0, bprev[2 * i], bprev[2 * i + 1]);
+    Bb[2 * i] = rb.x; Bb[2 * i + 1] = rb.y;
+    Cb[2 * i] = rc.x; Cb[2 * i + 1] = rc.y;
+    Bpb[2 * i] = rp.x; Bpb[2 * i + 1] = rp.y;
+    a.angle[bh * (kN / 2) + i] = ph;
+  } else {
+    const int p = tid - kN / 2;
+    const float x = to_f32(static_cast<const T*>(a.x_t)[bh * kP + p]);
+    xs[p] = x;
+    xps[p] = a.x_prev[bh * kP + p];
+    a.x_prev[bh * kP + p] = x;
+  }
+  const float alpha = expf(a.logdecay_t[bh]);
+  const float be = a.beta_t ? a.beta_t[bh] : 0.f;
+  const float ga = a.gamma_t[bh];
+  __syncthreads();
+
+  const float4 xv = reinterpret_cast<const float4*>(xs)[q];
+  const float4 xpv = reinterpret_cast<const float4*>(xps)[q];
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+  for (int k = 0; k < kRows; ++k) {
+    const int n = r0 + 8 * k;
+    const float bp = be * Bpb[n], bc = ga * Bb[n], cc = Cb[n];
+    float4 v;
+    v.x = alpha * hv[k].x + bp * xpv.x + bc * xv.x;
+    v.y = alpha * hv[k].y + bp * xpv.y + bc * xv.y;
+    v.z = alpha * hv[k].z + bp * xpv.z + bc * xv.z;
+    v.w = alpha * hv[k].w + bp * xpv.w + bc * xv.w;
+    S[n * (kP / 4) + q] = v;
+    acc.x += cc * v.x; acc.y += cc * v.y; acc.z += cc * v.z; acc.w += cc * v.w;
+  }
+  // lanes l and l + 16 hold the same column slice
+  acc.x += __shfl_xor_sync(0xffffffffu, acc.x, 16);
+  acc.y += __shfl_xor_sync(0xffffffffu, acc.y, 16);
+  acc.z += __shfl_xor_sync(0xffffffffu, acc.z, 16);
+  acc.w += __shfl_xor_sync(0xffffffffu, acc.w, 16);
+  if (lane < 16) red[warp][q] = acc;
+  __syncthreads();
+  if (tid < kP) {
+    const float* rf = reinterpret_cast<const float*>(red);
+    float y = a.D ? a.D[h] * xs[tid] : 0.f;
+#pragma unroll
+    for (int w = 0; w < kThreads128 / 32; ++w) y += rf[w * kP + tid];
+    static_cast<T*>(a.y_t)[bh * kP + tid] = from_f32<T>(y);
+  }
+}
+
 template <typename T>
 __global__ void bprev_update_kernel(const T* __restrict__ B_t, float* __restrict__ b_prev,
                                     int64_t n) {
@@ -163,8 +243,21 @@ cudaError_t launch_typed(const StepArgs& a, cudaStream_t s) {
 
 }  // namespace
 
+template <typename T>
+cudaError_t launch_n128p64(const StepArgs& a, cudaStream_t s) {
+  step_kernel_n128p64<T><<<(unsigned)(a.b * a.H), kThreads128, 0, s>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int64_t nb = a.b * a.G * a.N;
+  bprev_update_kernel<T><<<(unsigned)((nb + 255) / 256), 256, 0, s>>>(
+      static_cast<const T*>(a.B_t), a.b_prev, nb);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_step(const StepArgs& a, cudaStream_t s) {
   if (a.b * a.H == 0) return cudaSuccess;
+  if (a.N == kN && a.P == kP && (reinterpret_cast<uintptr_t>(a.ssm) % 16 == 0))
+    return a.bf16 ? launch_n128p64<__nv_bfloat16>(a, s) : launch_n128p64<float>(a, s);
   const bool vec4 = (a.P % 4 == 0) && (reinterpret_cast<uintptr_t>(a.ssm) % 16 == 0) &&
                     (a.P / 4 <= kThreads);
   if (a.bf16)

@@ -29,7 +29,7 @@ def declared_functions():
 def test_header_declares_the_boundary():
     names = declared_functions()
     for n in ("m3ssd_fwd", "m3ssd_step", "m3ssd_fwd_workspace_size", "m3ssd_status_string",
-              "m3ssd_abi_version"):
+              "m3ssd_abi_version", "m3ssd_device_wait_timeouts"):
         assert n in names
 
 
@@ -126,6 +126,10 @@ def test_step_validation(lib):
     assert lib.m3ssd_step(ctypes.byref(_dims()), FAKE, FAKE, None, FAKE, FAKE, FAKE, None, None,
                           None, FAKE, None) == m3.ERR_INVALID_ARG
     assert _step(lib, _dims(batch=0), x=None, y=None) == m3.OK
+
+
+def test_wait_timeout_query_rejects_null(lib):
+    assert lib.m3ssd_device_wait_timeouts(None) == m3.ERR_INVALID_ARG
 
 
 def test_python_binding_raises_value_error_on_invalid_args(lib):

@@ -61,6 +61,12 @@ def test_chunked_paths(has_beta, has_theta, with_D):
     assert rel_max_err(got["hT"], ref["hT"]) <= TOL
 
 
+def test_no_device_wait_timed_out():
+    """Every bounded tensor-core wait of the runs above completed."""
+    gpu_fwd(make_inputs(BASE.with_(seqlen=130, seed=12)))
+    assert m3.device_wait_timeouts() == 0
+
+
 def test_theta_is_not_dropped():
     """Differ-guard: with theta the output must differ from the theta-free run."""
     inp = make_inputs(BASE.with_(seqlen=128, seed=6))

@@ -75,6 +75,16 @@ __device__ __forceinline__ uint32_t off1(int r, int c) {
   return (uint32_t)(r * 128 + ((((c >> 3) ^ (r & 7))) << 4) + ((c & 7) << 1));
 }
 
+// Per-chunk scalars: decay cumsum (scaled by log2 e), exp(cs), the mask
+// coefficients gamma_u alpha_{u+1} + beta_{u+1}, the state weights W(63, u),
+// gamma, and exp(cs_63).  Double-buffered: chunk c+1's set is computed while
+// chunk c is finishing.
+struct ChunkParams {
+  float cs2[Q], ecs[Q], cvec[Q], wend[Q], gam[Q];
+  float eE;
+  float pad[3];
+};
+
 struct Smem {
   union {
     float theta[Q][NH];        // raw theta of the chunk (phase R1 only)
@@ -83,14 +93,13 @@ struct Smem {
   uint8_t bw_lo[2 * kAtom];    // residual of W_end o Bbar
   uint8_t B[2 * kAtom];        // raw B, then Bbar
   uint8_t C[2 * kAtom];        // raw C, then Cbar
-  uint8_t X[Q * 128];          // X rows of the chunk (row 0 = carry-in token)
+  uint8_t X[2][Q * 128];       // X rows of chunks c, c+1 (row 0 = carry-in token)
   uint8_t M[Q * 128];          // masked Gram W o G
   uint8_t Hs[NS * 128];        // bf16 copy of h for the state-to-output product
+  ChunkParams prm[2];
   float segtot[4][NH];
-  float cs2[Q], ecs[Q], cvec[Q], wend[Q], gam[Q];
   float ecos[NH], esin[NH], Phi[NH];     // exp(i Phi_c) per pair and Phi_c itself
   float necos[NH], nesin[NH], nPhi[NH];  // the same for the next chunk
-  float scal[4];
   uint64_t mbar[2];
   uint32_t tmem;
   uint32_t err;
@@ -111,6 +120,51 @@ __device__ __forceinline__ float2 unpack_bf16(uint32_t u) {
   return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
 }
 
+// Warp 0: the scalars of one chunk from its per-row logdecay / beta / gamma
+// (rows lane and lane + 32; row 0 holds zeros).
+__device__ __forceinline__ void chunk_params(ChunkParams& P, const float (&pld)[2],
+                                             const float (&pbe)[2], const float (&pga)[2],
+                                             int lane) {
+  float s0 = pld[0], s1 = pld[1];
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const float u0 = __shfl_up_sync(0xffffffffu, s0, o);
+    const float u1 = __shfl_up_sync(0xffffffffu, s1, o);
+    if (lane >= o) { s0 += u0; s1 += u1; }
+  }
+  s1 += __shfl_sync(0xffffffffu, s0, 31);
+  const float cs[2] = {s0, s1};
+  const float cs_end = __shfl_sync(0xffffffffu, s1, 31);
+  const float ld_dn0 = __shfl_down_sync(0xffffffffu, pld[0], 1);
+  const float ld_dn1 = __shfl_down_sync(0xffffffffu, pld[1], 1);
+  const float be_dn0 = __shfl_down_sync(0xffffffffu, pbe[0], 1);
+  const float be_dn1 = __shfl_down_sync(0xffffffffu, pbe[1], 1);
+  const float cs_dn0 = __shfl_down_sync(0xffffffffu, s0, 1);
+  const float cs_dn1 = __shfl_down_sync(0xffffffffu, s1, 1);
+  const float ld_32 = __shfl_sync(0xffffffffu, pld[1], 0);
+  const float be_32 = __shfl_sync(0xffffffffu, pbe[1], 0);
+  const float cs_32 = __shfl_sync(0xffffffffu, s1, 0);
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int r = lane + 32 * k;
+    const float ld_next = k == 0 ? (lane < 31 ? ld_dn0 : ld_32) : ld_dn1;
+    const float be_next = k == 0 ? (lane < 31 ? be_dn0 : be_32) : be_dn1;
+    const float cs_next = k == 0 ? (lane < 31 ? cs_dn0 : cs_32) : cs_dn1;
+    P.cs2[r] = cs[k] * kLog2e;
+    P.ecs[r] = expf(cs[k]);
+    P.gam[r] = pga[k];
+    if (r < Q - 1) {
+      const float cv = pga[k] * expf(ld_next) + be_next;
+      P.cvec[r] = cv;
+      P.wend[r] = expf(cs_end - cs_next) * cv;
+    } else {
+      P.cvec[r] = pga[k];
+      P.wend[r] = pga[k];
+    }
+  }
+  if (lane == 0) P.eE = expf(cs_end);
+}
+
 template <bool ROT>
 __global__ void __launch_bounds__(kThreads, 2) fwd_chunk_kernel(FwdArgs a) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -127,44 +181,57 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_chunk_kernel(FwdArgs a) {
   const bf16* Cg = static_cast<const bf16*>(a.C);
   bf16* Yg = static_cast<bf16*>(a.Y);
   const float Dh = a.D ? a.D[h] : 0.f;
-  const uint32_t aB = tc5::saddr(sm.B), aC = tc5::saddr(sm.C), aX = tc5::saddr(sm.X);
+  const uint32_t aB = tc5::saddr(sm.B), aC = tc5::saddr(sm.C);
+  const uint32_t aX0 = tc5::saddr(sm.X[0]);
   const uint32_t aM = tc5::saddr(sm.M), aH = tc5::saddr(sm.Hs);
   const uint32_t aWh = tc5::saddr(sm.u.bw_hi), aWl = tc5::saddr(sm.bw_lo);
   const uint32_t aT = tc5::saddr(&sm.u.theta[0][0]);
 
-  // Row r of chunk c holds token c*QT - 1 + r; rows outside [0, L) are zero-filled.
-  auto row_token = [&](int c, int r) -> int64_t { return (int64_t)c * QT - 1 + r; };
+  // Each thread's cp.async slots: rows lr + 16 k (k = 0..3) of theta / B / C at a
+  // fixed 16-byte column, and rows xr + 32 k (k = 0..1) of X.  Row r of chunk c
+  // holds token c*QT - 1 + r; rows outside [0, L) are zero-filled (row 0 of
+  // chunk 0 is the cache's previous token, written directly).
+  const int lr = tid >> 4, lc = tid & 15;
+  const int xr = tid >> 3, xc = tid & 7;
+  const int64_t hstride_t = H * NH;                       // theta elements per token
+  const int64_t gstride_t = G * NS;                       // B/C elements per token
+  const int64_t xstride_t = H * PD;                       // X elements per token
+  const float* theta_seq = a.theta ? a.theta + (b * L * H + h) * NH + lc * 4 : nullptr;
+  const bf16* B_seq = Bg + (b * L * G + g) * NS + lc * 8;
+  const bf16* C_seq = Cg + (b * L * G + g) * NS + lc * 8;
+  const bf16* X_seq = Xg + (b * L * H + h) * PD + xc * 8;
+  uint32_t dT[4], dBC[4], dX[2];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    dT[k] = aT + (uint32_t)((lr + 16 * k) * NH + lc * 4) * 4u;
+    dBC[k] = off2(lr + 16 * k, lc * 8);
+  }
+#pragma unroll
+  for (int k = 0; k < 2; ++k) dX[k] = off1(xr + 32 * k, xc * 8);
+
   auto load_theta = [&](int c) {
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-      const int idx = tid + k * kThreads;
-      const int row = idx >> 4, col = (idx & 15) * 4;
-      const int64_t t = row_token(c, row);
-      const bool ok = a.theta && t >= 0 && t < L;
-      const float* src = ok ? a.theta + ((b * L + t) * H + h) * NH + col : a.logdecay;
-      cp_async16(aT + (uint32_t)(row * NH + col) * 4u, src, ok);
+      const int64_t t = (int64_t)c * QT - 1 + lr + 16 * k;
+      const bool ok = theta_seq && t >= 0 && t < L;
+      cp_async16(dT[k], ok ? theta_seq + t * hstride_t : a.logdecay, ok);
     }
   };
-  auto load_bc = [&](int c, const bf16* base, uint32_t dst) {
+  auto load_bc = [&](int c, const bf16* seq, uint32_t base) {
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-      const int idx = tid + k * kThreads;
-      const int row = idx >> 4, c8 = idx & 15;
-      const int64_t t = row_token(c, row);
+      const int64_t t = (int64_t)c * QT - 1 + lr + 16 * k;
       const bool ok = t >= 0 && t < L;
-      const bf16* src = ok ? base + ((b * L + t) * G + g) * NS + c8 * 8 : base;
-      if (t >= 0) cp_async16(dst + off2(row, c8 * 8), src, ok);
+      if (t >= 0) cp_async16(base + dBC[k], ok ? seq + t * gstride_t : seq, ok);
     }
   };
   auto load_x = [&](int c) {
+    const uint32_t base = aX0 + (uint32_t)(c & 1) * (Q * 128);
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
-      const int idx = tid + k * kThreads;
-      const int row = idx >> 3, c8 = idx & 7;
-      const int64_t t = row_token(c, row);
+      const int64_t t = (int64_t)c * QT - 1 + xr + 32 * k;
       const bool ok = t >= 0 && t < L;
-      const bf16* src = ok ? Xg + ((b * L + t) * H + h) * PD + c8 * 8 : Xg;
-      if (t >= 0) cp_async16(aX + off1(row, c8 * 8), src, ok);
+      if (t >= 0) cp_async16(base + dX[k], ok ? X_seq + t * xstride_t : X_seq, ok);
     }
   };
   // warp 0 keeps logdecay / beta / gamma of rows lane and lane + 32 in registers
@@ -173,7 +240,7 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_chunk_kernel(FwdArgs a) {
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
       const int r = lane + 32 * k;
-      const int64_t t = row_token(c, r);
+      const int64_t t = (int64_t)c * QT - 1 + r;
       const bool ok = r > 0 && t < L;  // row 0 (carry-in) has a = gamma = beta = 0 here
       const int64_t idx = (b * L + (ok ? t : 0)) * H + h;
       pld[k] = ok ? a.logdecay[idx] : 0.f;
@@ -191,11 +258,15 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_chunk_kernel(FwdArgs a) {
     sm.err = 0;
   }
   if (ROT) load_theta(0);
-  load_bc(0, Bg, aB);
-  load_bc(0, Cg, aC);
+  load_bc(0, B_seq, aB);
+  load_bc(0, C_seq, aC);
   load_x(0);
   cp_async_commit();
-  if (warp == 0) load_params(0);
+  if (warp == 0) {
+    load_params(0);
+    chunk_params(sm.prm[0], pld, pbe, pga, lane);
+    if (nC > 1) load_params(1);
+  }
   // row 0 of chunk 0 is the cache's previous token (zero when absent)
   if (tid < NS) {
     const float bp = a.bprev0 ? a.bprev0[(b * G + g) * NS + tid] : 0.f;
@@ -204,7 +275,7 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_chunk_kernel(FwdArgs a) {
   }
   if (tid < PD) {
     const float xp = a.xprev0 ? a.xprev0[bh * PD + tid] : 0.f;
-    *reinterpret_cast<bf16*>(sm.X + off1(0, tid)) = __float2bfloat16_rn(xp);
+    *reinterpret_cast<bf16*>(sm.X[0] + off1(0, tid)) = __float2bfloat16_rn(xp);
   }
   if (ROT && tid < NH) {
     const float ph0 = a.angle0 ? a.angle0[bh * NH + tid] : 0.f;
@@ -245,57 +316,23 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_chunk_kernel(FwdArgs a) {
   const uint32_t tmem = sm.tmem;
   // this warp's TMEM lane quarter (rows of the M=64 and M=128 accumulators)
   const uint32_t tlane = (uint32_t)(32 * (warp & 3)) << 16;
+  const int pi = tid & 63, seg = tid >> 6;  // rotation: pair pi, rows 16 seg .. 16 seg + 15
 
   // ---- chunk walk -------------------------------------------------------------
   for (int c = 0; c < nC; ++c) {
     const int64_t tbase = (int64_t)c * QT - 1;  // token of row 0
     const uint32_t par = (uint32_t)(c & 1);
+    const ChunkParams& P = sm.prm[c & 1];
+    const uint8_t* Xs = sm.X[c & 1];
+    const uint32_t aX = aX0 + (uint32_t)(c & 1) * (Q * 128);
     cp_async_wait_all();
     __syncthreads();  // S1: theta, B, C, X of this chunk are in shared memory
-
-    // -- phase R1: decay cumsum and chunk parameters (warp 0), angle cumsum -------
-    if (warp == 0) {
-      float s0 = pld[0], s1 = pld[1];
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const float u0 = __shfl_up_sync(0xffffffffu, s0, o);
-        const float u1 = __shfl_up_sync(0xffffffffu, s1, o);
-        if (lane >= o) { s0 += u0; s1 += u1; }
-      }
-      s1 += __shfl_sync(0xffffffffu, s0, 31);
-      const float cs[2] = {s0, s1};
-      const float cs_end = __shfl_sync(0xffffffffu, s1, 31);
-      const float ld_dn0 = __shfl_down_sync(0xffffffffu, pld[0], 1);
-      const float ld_dn1 = __shfl_down_sync(0xffffffffu, pld[1], 1);
-      const float be_dn0 = __shfl_down_sync(0xffffffffu, pbe[0], 1);
-      const float be_dn1 = __shfl_down_sync(0xffffffffu, pbe[1], 1);
-      const float cs_dn0 = __shfl_down_sync(0xffffffffu, s0, 1);
-      const float cs_dn1 = __shfl_down_sync(0xffffffffu, s1, 1);
-      const float ld_32 = __shfl_sync(0xffffffffu, pld[1], 0);
-      const float be_32 = __shfl_sync(0xffffffffu, pbe[1], 0);
-      const float cs_32 = __shfl_sync(0xffffffffu, s1, 0);
-#pragma unroll
-      for (int k = 0; k < 2; ++k) {
-        const int r = lane + 32 * k;
-        const float ld_next = k == 0 ? (lane < 31 ? ld_dn0 : ld_32) : ld_dn1;
-        const float be_next = k == 0 ? (lane < 31 ? be_dn0 : be_32) : be_dn1;
-        const float cs_next = k == 0 ? (lane < 31 ? cs_dn0 : cs_32) : cs_dn1;
-        sm.cs2[r] = cs[k] * kLog2e;
-        sm.ecs[r] = expf(cs[k]);
-        sm.gam[r] = pga[k];
-        if (r < Q - 1) {
-          const float cv = pga[k] * expf(ld_next) + be_next;
-          sm.cvec[r] = cv;
-          sm.wend[r] = expf(cs_end - cs_next) * cv;
-        } else {
-          sm.cvec[r] = pga[k];
-          sm.wend[r] = pga[k];
-        }
-      }
-      if (lane == 0) sm.scal[0] = expf(cs_end);
-      if (c + 1 < nC) load_params(c + 1);
+    if (c + 1 < nC) {
+      load_x(c + 1);
+      cp_async_commit();
     }
-    const int pi = tid & 63, seg = tid >> 6;
+
+    // -- phase R1: chunk-local angle cumsum ------------------------------------
     float psi[16];
     if (ROT) {
       float run = 0.f;
@@ -306,40 +343,61 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_chunk_kernel(FwdArgs a) {
       }
       sm.segtot[seg][pi] = run;
     }
-    __syncthreads();  // S2: parameters ready; theta no longer read
+    __syncthreads();  // S2: segment totals ready; theta no longer read
 
     // -- phase R2: rotation into the absolute frame, W_end o Bbar hi/lo ----------
+    // Two rows at a time in packed fp32 pairs (row k, row k+1).
     {
-      float off = 0.f, ec = 1.f, es = 0.f;
+      float off = 0.f;
+      float2 ec2 = make_float2(1.f, 1.f), es2 = make_float2(0.f, 0.f);
       if (ROT) {
         for (int s2 = 0; s2 < seg; ++s2) off += sm.segtot[s2][pi];
-        ec = sm.ecos[pi];
-        es = sm.esin[pi];
+        ec2 = make_float2(sm.ecos[pi], sm.ecos[pi]);
+        es2 = make_float2(sm.esin[pi], sm.esin[pi]);
       }
-#pragma unroll 4
-      for (int k = 0; k < 16; ++k) {
+      const float2 nes2 = make_float2(-es2.x, -es2.y);
+#pragma unroll
+      for (int k = 0; k < 16; k += 2) {
         const int r = seg * 16 + k;
-        const uint32_t o = off2(r, 2 * pi);
-        uint32_t* pb = reinterpret_cast<uint32_t*>(sm.B + o);
-        uint32_t* pc = reinterpret_cast<uint32_t*>(sm.C + o);
-        float2 bv = unpack_bf16(*pb);
+        const uint32_t oa = off2(r, 2 * pi), ob = off2(r + 1, 2 * pi);
+        uint32_t* pba = reinterpret_cast<uint32_t*>(sm.B + oa);
+        uint32_t* pbb = reinterpret_cast<uint32_t*>(sm.B + ob);
+        const float2 ba = unpack_bf16(*pba), bb = unpack_bf16(*pbb);
+        float2 bre = make_float2(ba.x, bb.x), bim = make_float2(ba.y, bb.y);
         if (ROT) {
-          float2 cv = unpack_bf16(*pc);
-          float s, co;
-          fast_sincos(psi[k] + off, &s, &co);
+          uint32_t* pca = reinterpret_cast<uint32_t*>(sm.C + oa);
+          uint32_t* pcb = reinterpret_cast<uint32_t*>(sm.C + ob);
+          const float2 ca = unpack_bf16(*pca), cbv = unpack_bf16(*pcb);
+          const float2 cre = make_float2(ca.x, cbv.x), cim = make_float2(ca.y, cbv.y);
+          float s0, c0, s1, c1;
+          fast_sincos(psi[k] + off, &s0, &c0);
+          fast_sincos(psi[k + 1] + off, &s1, &c1);
+          const float2 co2 = make_float2(c0, c1), si2 = make_float2(s0, s1);
           // exp(i (Phi_c + psi)) = exp(i Phi_c) exp(i psi)
-          const float cr = ec * co - es * s, sr = es * co + ec * s;
-          bv = rot2(cr, sr, bv.x, bv.y);
-          cv = rot2(cr, sr, cv.x, cv.y);
-          *pb = pack_bf16(bv.x, bv.y);
-          *pc = pack_bf16(cv.x, cv.y);
+          const float2 cr = __ffma2_rn(nes2, si2, __fmul2_rn(ec2, co2));
+          const float2 sr = __ffma2_rn(ec2, si2, __fmul2_rn(es2, co2));
+          const float2 nsr = make_float2(-sr.x, -sr.y);
+          const float2 bre2 = __ffma2_rn(nsr, bim, __fmul2_rn(cr, bre));
+          const float2 bim2 = __ffma2_rn(cr, bim, __fmul2_rn(sr, bre));
+          const float2 cre2 = __ffma2_rn(nsr, cim, __fmul2_rn(cr, cre));
+          const float2 cim2 = __ffma2_rn(cr, cim, __fmul2_rn(sr, cre));
+          bre = bre2;
+          bim = bim2;
+          *pba = pack_bf16(bre.x, bim.x);
+          *pbb = pack_bf16(bre.y, bim.y);
+          *pca = pack_bf16(cre2.x, cim2.x);
+          *pcb = pack_bf16(cre2.y, cim2.y);
         }
-        const float we = sm.wend[r];
-        const float w0 = we * bv.x, w1 = we * bv.y;
-        const uint32_t hi = pack_bf16(w0, w1);
-        const float2 hv = unpack_bf16(hi);
-        *reinterpret_cast<uint32_t*>(sm.u.bw_hi + o) = hi;
-        *reinterpret_cast<uint32_t*>(sm.bw_lo + o) = pack_bf16(w0 - hv.x, w1 - hv.y);
+        const float2 we = *reinterpret_cast<const float2*>(&P.wend[r]);
+        const float2 wre = __fmul2_rn(we, bre), wim = __fmul2_rn(we, bim);
+        const uint32_t hia = pack_bf16(wre.x, wim.x), hib = pack_bf16(wre.y, wim.y);
+        const float2 ha = unpack_bf16(hia), hb = unpack_bf16(hib);
+        const float2 lre = __fadd2_rn(wre, make_float2(-ha.x, -hb.x));
+        const float2 lim = __fadd2_rn(wim, make_float2(-ha.y, -hb.y));
+        *reinterpret_cast<uint32_t*>(sm.u.bw_hi + oa) = hia;
+        *reinterpret_cast<uint32_t*>(sm.u.bw_hi + ob) = hib;
+        *reinterpret_cast<uint32_t*>(sm.bw_lo + oa) = pack_bf16(lre.x, lim.x);
+        *reinterpret_cast<uint32_t*>(sm.bw_lo + ob) = pack_bf16(lre.y, lim.y);
       }
       if (ROT && seg == 3) {
         const float pnext = wrap_angle(sm.Phi[pi] + psi[15] + off);
@@ -388,31 +446,36 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_chunk_kernel(FwdArgs a) {
     {
       if (!tc5::mbar_wait(&sm.mbar[0], par, kWaitLimitNs)) sm.err = 1;
       tc5::fence_after_sync();
+      // the Gram has consumed Bbar: the next chunk's raw B can stream in now
+      if (c + 1 < nC) {
+        load_bc(c + 1, B_seq, aB);
+        cp_async_commit();
+      }
       uint32_t gr[16];
       tc5::ld_16x256b_x4(tmem + tlane + kColG + (uint32_t)cb, gr);
       tc5::wait_ld();
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf) {
         const int t = 16 * (warp & 3) + (lane >> 2) + 8 * hf;
-        const float cst = sm.cs2[t], gt = sm.gam[t];
+        const float cst = P.cs2[t], gt = P.gam[t];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const int s0 = cb + 8 * q + 2 * (lane & 3);
-          float wv[2];
-#pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            const int s = s0 + j;
-            wv[j] = (s > t) ? 0.f : (s == t) ? gt : exp2f(cst - sm.cs2[s + 1]) * sm.cvec[s];
+          float w0 = 0.f, w1 = 0.f;
+          if (cb + 8 * q <= t) {  // this 8-column group reaches the diagonal or below
+            const float2 cv = *reinterpret_cast<const float2*>(&P.cvec[s0]);
+            w0 = (s0 == t) ? gt : (s0 < t) ? exp2f(cst - P.cs2[s0 + 1]) * cv.x : 0.f;
+            w1 = (s0 + 1 == t) ? gt : (s0 + 1 < t) ? exp2f(cst - P.cs2[s0 + 2]) * cv.y : 0.f;
           }
           *reinterpret_cast<uint32_t*>(sm.M + off1(t, s0)) =
-              pack_bf16(__uint_as_float(gr[4 * q + 2 * hf]) * wv[0],
-                        __uint_as_float(gr[4 * q + 2 * hf + 1]) * wv[1]);
+              pack_bf16(__uint_as_float(gr[4 * q + 2 * hf]) * w0,
+                        __uint_as_float(gr[4 * q + 2 * hf + 1]) * w1);
         }
       }
     }
     tc5::fence_proxy_async();
     tc5::fence_before_sync();
-    __syncthreads();  // S4: M ready; the Gram has consumed Bbar
+    __syncthreads();  // S4: M ready
     if (tid == 0) {
       tc5::fence_after_sync();
 #pragma unroll
@@ -421,54 +484,62 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_chunk_kernel(FwdArgs a) {
                       tc5::desc_sw128(aX + (uint32_t)j * 2048u, kAtom, 1024), kIdescY, j > 0);
       tc5::commit(&sm.mbar[1]);
     }
-    if (c + 1 < nC) {
-      load_bc(c + 1, Bg, aB);
-      cp_async_commit();
-    }
 
     // -- phase Y + S: outputs and the state update ---------------------------------
     {
+      // warp 0 prepares the next chunk's scalars while the products finish
+      if (warp == 0 && c + 1 < nC) {
+        chunk_params(sm.prm[(c + 1) & 1], pld, pbe, pga, lane);
+        if (c + 2 < nC) load_params(c + 2);
+      }
       if (!tc5::mbar_wait(&sm.mbar[1], par, kWaitLimitNs)) sm.err = 1;
       tc5::fence_after_sync();
+      // every product of this chunk is done: Cbar, theta / W_end o Bbar can be refilled
+      if (c + 1 < nC) {
+        load_bc(c + 1, C_seq, aC);
+        if (ROT) load_theta(c + 1);
+        cp_async_commit();
+      }
       uint32_t y1[16], y2[16], sv[32];
       tc5::ld_16x256b_x4(tmem + tlane + kColY1 + (uint32_t)cb, y1);
       tc5::ld_16x256b_x4(tmem + tlane + kColY2 + (uint32_t)cb, y2);
       tc5::ld_32x32b_x32(tmem + tlane + kColS + (uint32_t)cb, sv);
       tc5::wait_ld();
+      const float2 D2 = make_float2(Dh, Dh);
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf) {
         const int r = 16 * (warp & 3) + (lane >> 2) + 8 * hf;
         const int64_t t = tbase + r;
         if (r > 0 && t < L) {
-          const float er = sm.ecs[r];
+          const float2 er2 = make_float2(P.ecs[r], P.ecs[r]);
           bf16* yrow = Yg + ((b * L + t) * H + h) * PD;
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             const int p = cb + 8 * q + 2 * (lane & 3);
-            const float2 xv = unpack_bf16(*reinterpret_cast<const uint32_t*>(sm.X + off1(r, p)));
-            const float v0 = er * __uint_as_float(y1[4 * q + 2 * hf]) +
-                             __uint_as_float(y2[4 * q + 2 * hf]) + Dh * xv.x;
-            const float v1 = er * __uint_as_float(y1[4 * q + 2 * hf + 1]) +
-                             __uint_as_float(y2[4 * q + 2 * hf + 1]) + Dh * xv.y;
-            *reinterpret_cast<uint32_t*>(yrow + p) = pack_bf16(v0, v1);
+            const float2 xv = unpack_bf16(*reinterpret_cast<const uint32_t*>(Xs + off1(r, p)));
+            const float2 a1 = make_float2(__uint_as_float(y1[4 * q + 2 * hf]),
+                                          __uint_as_float(y1[4 * q + 2 * hf + 1]));
+            const float2 a2 = make_float2(__uint_as_float(y2[4 * q + 2 * hf]),
+                                          __uint_as_float(y2[4 * q + 2 * hf + 1]));
+            const float2 v = __ffma2_rn(D2, xv, __ffma2_rn(er2, a1, a2));
+            *reinterpret_cast<uint32_t*>(yrow + p) = pack_bf16(v.x, v.y);
           }
         }
       }
-      const float eE = sm.scal[0];
+      const float2 eE2 = make_float2(P.eE, P.eE);
 #pragma unroll
-      for (int j = 0; j < 32; ++j) hs[j] = fmaf(eE, hs[j], __uint_as_float(sv[j]));
+      for (int j = 0; j < 32; j += 2) {
+        const float2 hv = __ffma2_rn(eE2, make_float2(hs[j], hs[j + 1]),
+                                     make_float2(__uint_as_float(sv[j]), __uint_as_float(sv[j + 1])));
+        hs[j] = hv.x;
+        hs[j + 1] = hv.y;
+      }
       store_state_bf16();
     }
     tc5::fence_proxy_async();
     tc5::fence_before_sync();
-    __syncthreads();  // S5: every tensor-core operand of this chunk is consumed
+    __syncthreads();  // S5: this chunk's operands and accumulators are consumed
     if (sm.err) break;
-    if (c + 1 < nC) {
-      load_bc(c + 1, Cg, aC);
-      if (ROT) load_theta(c + 1);
-      load_x(c + 1);
-      cp_async_commit();
-    }
   }
   cp_async_wait_all();
 

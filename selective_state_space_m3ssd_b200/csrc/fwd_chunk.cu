@@ -21,7 +21,8 @@
 // form one mask ("TorchMamba" README: "the parallel mask is L = 1SS @ band").
 //
 // Tensor-core work per chunk (tcgen05.mma kind::f16, bf16 in, fp32 in TMEM),
-// issued by one thread:
+// issued by one thread and tracked by three mbarriers (G done; Y1 and S done;
+// Y2 done) so each input buffer is refilled as soon as its last reader finishes:
 //   G  = Cbar Bbar^T                 M=64  N=64 K=128   (TMEM cols   0..63)
 //   Y1 = Cbar h_bf16                 M=64  N=64 K=128   (TMEM cols  64..127)
 //   S  = (W_end o Bbar)^T X          M=128 N=64 K=64 x2 (TMEM cols 192..255), the
@@ -32,9 +33,17 @@
 // decay/angle cumsums, sincos, rotations and the mask also run.  Operand tiles
 // live in shared memory in the 128-byte-swizzled canonical layouts: K-major rows
 // of 128 B for Cbar, Bbar and the mask; MN-major 64-element atoms for X, h and
-// W_end o Bbar.  Loads use cp.async with zero-fill for the ragged last chunk.
+// W_end o Bbar.  The inputs of a chunk (theta, B, C, X) arrive by TMA (4-D tensor
+// maps over (inner, head or group, token, batch), so the carry-in row of the
+// first chunk and the rows past the end are zero-filled by the hardware, and
+// the 128-byte swizzle of the operand layouts is written by the copy itself).
 // Two CTAs share an SM (about 100 KB of shared memory and 256 TMEM columns each).
+#include <cuda.h>
 #include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+
+#include <cstring>
+#include <mutex>
 
 #include "common.cuh"
 #include "internal.h"
@@ -97,20 +106,14 @@ struct Smem {
   uint8_t M[Q * 128];          // masked Gram W o G
   uint8_t Hs[NS * 128];        // bf16 copy of h for the state-to-output product
   ChunkParams prm[2];
-  float segtot[4][NH];
+  float segtot[8][NH];
   float ecos[NH], esin[NH], Phi[NH];     // exp(i Phi_c) per pair and Phi_c itself
   float necos[NH], nesin[NH], nPhi[NH];  // the same for the next chunk
-  uint64_t mbar[2];
+  uint64_t mbar[3];
+  uint64_t lmbar;              // TMA loads of the next chunk
   uint32_t tmem;
   uint32_t err;
 };
-
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src),
-               "r"(valid ? 16 : 0));
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;\n" ::); }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -165,8 +168,17 @@ __device__ __forceinline__ void chunk_params(ChunkParams& P, const float (&pld)[
   if (lane == 0) P.eE = expf(cs_end);
 }
 
+// Tensor maps of the chunk inputs, built on the host for each launch.
+struct TmaMaps {
+  CUtensorMap theta;  // fp32 (pair, head, token, batch), box 64 x 1 x 64 x 1, no swizzle
+  CUtensorMap B;      // bf16 (n, group, token, batch), box 64 x 1 x 64 x 1, 128-byte swizzle
+  CUtensorMap C;      // same as B
+  CUtensorMap X;      // bf16 (p, head, token, batch), box 64 x 1 x 64 x 1, 128-byte swizzle
+};
+
 template <bool ROT>
-__global__ void __launch_bounds__(kThreads, 2) fwd_chunk_kernel(FwdArgs a) {
+__global__ void __launch_bounds__(kThreads, 2)
+    fwd_chunk_kernel(FwdArgs a, const __grid_constant__ TmaMaps tm) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   // operand tiles need a 1024-byte aligned shared-space address
   const uint32_t raw_addr = tc5::saddr(smem_raw);
@@ -187,53 +199,24 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_chunk_kernel(FwdArgs a) {
   const uint32_t aWh = tc5::saddr(sm.u.bw_hi), aWl = tc5::saddr(sm.bw_lo);
   const uint32_t aT = tc5::saddr(&sm.u.theta[0][0]);
 
-  // Each thread's cp.async slots: rows lr + 16 k (k = 0..3) of theta / B / C at a
-  // fixed 16-byte column, and rows xr + 32 k (k = 0..1) of X.  Row r of chunk c
-  // holds token c*QT - 1 + r; rows outside [0, L) are zero-filled (row 0 of
-  // chunk 0 is the cache's previous token, written directly).
-  const int lr = tid >> 4, lc = tid & 15;
-  const int xr = tid >> 3, xc = tid & 7;
-  const int64_t hstride_t = H * NH;                       // theta elements per token
-  const int64_t gstride_t = G * NS;                       // B/C elements per token
-  const int64_t xstride_t = H * PD;                       // X elements per token
-  const float* theta_seq = a.theta ? a.theta + (b * L * H + h) * NH + lc * 4 : nullptr;
-  const bf16* B_seq = Bg + (b * L * G + g) * NS + lc * 8;
-  const bf16* C_seq = Cg + (b * L * G + g) * NS + lc * 8;
-  const bf16* X_seq = Xg + (b * L * H + h) * PD + xc * 8;
-  uint32_t dT[4], dBC[4], dX[2];
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    dT[k] = aT + (uint32_t)((lr + 16 * k) * NH + lc * 4) * 4u;
-    dBC[k] = off2(lr + 16 * k, lc * 8);
-  }
-#pragma unroll
-  for (int k = 0; k < 2; ++k) dX[k] = off1(xr + 32 * k, xc * 8);
+  bf16* const Y_seq = Yg + (b * L * H + h) * PD;
+  const int64_t xstride_t = H * PD;  // X / Y elements per token
+  // TMA issue (one thread): chunk c's rows start at token c*QT - 1
+  const bool has_theta = a.theta != nullptr;  // ROT without theta: rotation by angle0 only
+  const uint32_t chunk_bytes = (ROT && has_theta ? 16384u : 0u) + 2u * 16384u + 8192u;
+  auto tma_theta = [&](int c) {
+    tc5::tma_load_4d(aT, &tm.theta, &sm.lmbar, 0, (int)h, c * QT - 1, (int)b);
+  };
+  auto tma_bc = [&](int c, const CUtensorMap* map, uint32_t base) {
+    tc5::tma_load_4d(base, map, &sm.lmbar, 0, (int)g, c * QT - 1, (int)b);
+    tc5::tma_load_4d(base + kAtom, map, &sm.lmbar, 64, (int)g, c * QT - 1, (int)b);
+  };
+  auto tma_x = [&](int c) {
+    tc5::tma_load_4d(aX0 + (uint32_t)(c & 1) * (Q * 128), &tm.X, &sm.lmbar, 0, (int)h, c * QT - 1,
+                     (int)b);
+  };
+  const bool loader = tid == 32;
 
-  auto load_theta = [&](int c) {
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int64_t t = (int64_t)c * QT - 1 + lr + 16 * k;
-      const bool ok = theta_seq && t >= 0 && t < L;
-      cp_async16(dT[k], ok ? theta_seq + t * hstride_t : a.logdecay, ok);
-    }
-  };
-  auto load_bc = [&](int c, const bf16* seq, uint32_t base) {
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int64_t t = (int64_t)c * QT - 1 + lr + 16 * k;
-      const bool ok = t >= 0 && t < L;
-      if (t >= 0) cp_async16(base + dBC[k], ok ? seq + t * gstride_t : seq, ok);
-    }
-  };
-  auto load_x = [&](int c) {
-    const uint32_t base = aX0 + (uint32_t)(c & 1) * (Q * 128);
-#pragma unroll
-    for (int k = 0; k < 2; ++k) {
-      const int64_t t = (int64_t)c * QT - 1 + xr + 32 * k;
-      const bool ok = t >= 0 && t < L;
-      if (t >= 0) cp_async16(base + dX[k], ok ? X_seq + t * xstride_t : X_seq, ok);
-    }
-  };
   // warp 0 keeps logdecay / beta / gamma of rows lane and lane + 32 in registers
   float pld[2], pbe[2], pga[2];
   auto load_params = [&](int c) {
@@ -254,29 +237,29 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_chunk_kernel(FwdArgs a) {
   if (tid == 0) {
     tc5::mbar_init(&sm.mbar[0], 1);
     tc5::mbar_init(&sm.mbar[1], 1);
+    tc5::mbar_init(&sm.mbar[2], 1);
+    tc5::mbar_init(&sm.lmbar, 1);
     tc5::fence_mbar_init();
     sm.err = 0;
   }
-  if (ROT) load_theta(0);
-  load_bc(0, B_seq, aB);
-  load_bc(0, C_seq, aC);
-  load_x(0);
-  cp_async_commit();
+  __syncthreads();  // mbarriers initialised
+  if (loader) {
+    tc5::mbar_arrive_expect_tx(&sm.lmbar, chunk_bytes);
+    if (ROT && has_theta) tma_theta(0);
+    tma_bc(0, &tm.B, aB);
+    tma_bc(0, &tm.C, aC);
+    tma_x(0);
+  }
   if (warp == 0) {
     load_params(0);
     chunk_params(sm.prm[0], pld, pbe, pga, lane);
     if (nC > 1) load_params(1);
   }
-  // row 0 of chunk 0 is the cache's previous token (zero when absent)
-  if (tid < NS) {
-    const float bp = a.bprev0 ? a.bprev0[(b * G + g) * NS + tid] : 0.f;
-    *reinterpret_cast<bf16*>(sm.B + off2(0, tid)) = __float2bfloat16_rn(bp);
-    *reinterpret_cast<bf16*>(sm.C + off2(0, tid)) = __float2bfloat16_rn(0.f);
-  }
-  if (tid < PD) {
-    const float xp = a.xprev0 ? a.xprev0[bh * PD + tid] : 0.f;
-    *reinterpret_cast<bf16*>(sm.X[0] + off1(0, tid)) = __float2bfloat16_rn(xp);
-  }
+  // row 0 of chunk 0 is the cache's previous token (the TMA zero-fills it; it is
+  // patched once that copy has landed)
+  const float bp0 = (tid < NS && a.bprev0) ? a.bprev0[(b * G + g) * NS + tid] : 0.f;
+  const float xp0 = (tid < PD && a.xprev0) ? a.xprev0[bh * PD + tid] : 0.f;
+  const bool patch_row0 = a.bprev0 != nullptr || a.xprev0 != nullptr;
   if (ROT && tid < NH) {
     const float ph0 = a.angle0 ? a.angle0[bh * NH + tid] : 0.f;
     sm.Phi[tid] = ph0;
@@ -316,7 +299,6 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_chunk_kernel(FwdArgs a) {
   const uint32_t tmem = sm.tmem;
   // this warp's TMEM lane quarter (rows of the M=64 and M=128 accumulators)
   const uint32_t tlane = (uint32_t)(32 * (warp & 3)) << 16;
-  const int pi = tid & 63, seg = tid >> 6;  // rotation: pair pi, rows 16 seg .. 16 seg + 15
 
   // ---- chunk walk -------------------------------------------------------------
   for (int c = 0; c < nC; ++c) {
@@ -325,55 +307,73 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_chunk_kernel(FwdArgs a) {
     const ChunkParams& P = sm.prm[c & 1];
     const uint8_t* Xs = sm.X[c & 1];
     const uint32_t aX = aX0 + (uint32_t)(c & 1) * (Q * 128);
-    cp_async_wait_all();
+    if (!tc5::mbar_wait(&sm.lmbar, par, kWaitLimitNs)) sm.err = 1;
     __syncthreads();  // S1: theta, B, C, X of this chunk are in shared memory
-    if (c + 1 < nC) {
-      load_x(c + 1);
-      cp_async_commit();
+    if (loader && c + 1 < nC) {
+      tc5::mbar_arrive_expect_tx(&sm.lmbar, chunk_bytes);
+      tma_x(c + 1);
+    }
+    if (c == 0 && patch_row0) {
+      if (tid < NS) *reinterpret_cast<bf16*>(sm.B + off2(0, tid)) = __float2bfloat16_rn(bp0);
+      if (tid < PD) *reinterpret_cast<bf16*>(sm.X[0] + off1(0, tid)) = __float2bfloat16_rn(xp0);
     }
 
     // -- phase R1: chunk-local angle cumsum ------------------------------------
-    float psi[16];
+    // Thread (lane, warp) owns the adjacent pairs 2 lane, 2 lane + 1 (elements
+    // 4 lane .. 4 lane + 3) in rows 8 warp .. 8 warp + 7; the two pairs travel
+    // together in packed fp32 pairs.
+    float2 psi[8];
     if (ROT) {
-      float run = 0.f;
+      float2 run = make_float2(0.f, 0.f);
+      if (has_theta) {
 #pragma unroll
-      for (int k = 0; k < 16; ++k) {
-        if (seg > 0 || k > 0) run += sm.u.theta[seg * 16 + k][pi];  // psi_0 = 0
+      for (int k = 0; k < 8; ++k) {
+        if (warp > 0 || k > 0) {  // psi_0 = 0
+          const float2 th = *reinterpret_cast<const float2*>(&sm.u.theta[8 * warp + k][2 * lane]);
+          run = __fadd2_rn(run, th);
+        }
         psi[k] = run;
       }
-      sm.segtot[seg][pi] = run;
+      } else {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) psi[k] = run;
+      }
+      *reinterpret_cast<float2*>(&sm.segtot[warp][2 * lane]) = run;
     }
     __syncthreads();  // S2: segment totals ready; theta no longer read
 
     // -- phase R2: rotation into the absolute frame, W_end o Bbar hi/lo ----------
-    // Two rows at a time in packed fp32 pairs (row k, row k+1).
     {
-      float off = 0.f;
+      float2 off = make_float2(0.f, 0.f);
       float2 ec2 = make_float2(1.f, 1.f), es2 = make_float2(0.f, 0.f);
       if (ROT) {
-        for (int s2 = 0; s2 < seg; ++s2) off += sm.segtot[s2][pi];
-        ec2 = make_float2(sm.ecos[pi], sm.ecos[pi]);
-        es2 = make_float2(sm.esin[pi], sm.esin[pi]);
+        for (int s2 = 0; s2 < warp; ++s2)
+          off = __fadd2_rn(off, *reinterpret_cast<const float2*>(&sm.segtot[s2][2 * lane]));
+        ec2 = *reinterpret_cast<const float2*>(&sm.ecos[2 * lane]);
+        es2 = *reinterpret_cast<const float2*>(&sm.esin[2 * lane]);
       }
       const float2 nes2 = make_float2(-es2.x, -es2.y);
 #pragma unroll
-      for (int k = 0; k < 16; k += 2) {
-        const int r = seg * 16 + k;
-        const uint32_t oa = off2(r, 2 * pi), ob = off2(r + 1, 2 * pi);
-        uint32_t* pba = reinterpret_cast<uint32_t*>(sm.B + oa);
-        uint32_t* pbb = reinterpret_cast<uint32_t*>(sm.B + ob);
-        const float2 ba = unpack_bf16(*pba), bb = unpack_bf16(*pbb);
-        float2 bre = make_float2(ba.x, bb.x), bim = make_float2(ba.y, bb.y);
+      for (int k = 0; k < 8; ++k) {
+        const int r = 8 * warp + k;
+        const uint32_t o = off2(r, 4 * lane);
+        uint2* pb = reinterpret_cast<uint2*>(sm.B + o);
+        const uint2 bw2 = *pb;
+        float2 bre = make_float2(__uint_as_float(bw2.x << 16), __uint_as_float(bw2.y << 16));
+        float2 bim = make_float2(__uint_as_float(bw2.x & 0xffff0000u),
+                                 __uint_as_float(bw2.y & 0xffff0000u));
         if (ROT) {
-          uint32_t* pca = reinterpret_cast<uint32_t*>(sm.C + oa);
-          uint32_t* pcb = reinterpret_cast<uint32_t*>(sm.C + ob);
-          const float2 ca = unpack_bf16(*pca), cbv = unpack_bf16(*pcb);
-          const float2 cre = make_float2(ca.x, cbv.x), cim = make_float2(ca.y, cbv.y);
+          uint2* pc = reinterpret_cast<uint2*>(sm.C + o);
+          const uint2 cw2 = *pc;
+          const float2 cre = make_float2(__uint_as_float(cw2.x << 16), __uint_as_float(cw2.y << 16));
+          const float2 cim = make_float2(__uint_as_float(cw2.x & 0xffff0000u),
+                                         __uint_as_float(cw2.y & 0xffff0000u));
+          const float2 ang = __fadd2_rn(psi[k], off);
           float s0, c0, s1, c1;
-          fast_sincos(psi[k] + off, &s0, &c0);
-          fast_sincos(psi[k + 1] + off, &s1, &c1);
+          fast_sincos(ang.x, &s0, &c0);
+          fast_sincos(ang.y, &s1, &c1);
           const float2 co2 = make_float2(c0, c1), si2 = make_float2(s0, s1);
-          // exp(i (Phi_c + psi)) = exp(i Phi_c) exp(i psi)
+          // exp(i (Phi_c + psi)) = exp(i Phi_c) exp(i psi), per pair
           const float2 cr = __ffma2_rn(nes2, si2, __fmul2_rn(ec2, co2));
           const float2 sr = __ffma2_rn(ec2, si2, __fmul2_rn(es2, co2));
           const float2 nsr = make_float2(-sr.x, -sr.y);
@@ -383,29 +383,34 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_chunk_kernel(FwdArgs a) {
           const float2 cim2 = __ffma2_rn(cr, cim, __fmul2_rn(sr, cre));
           bre = bre2;
           bim = bim2;
-          *pba = pack_bf16(bre.x, bim.x);
-          *pbb = pack_bf16(bre.y, bim.y);
-          *pca = pack_bf16(cre2.x, cim2.x);
-          *pcb = pack_bf16(cre2.y, cim2.y);
+          *pb = make_uint2(pack_bf16(bre.x, bim.x), pack_bf16(bre.y, bim.y));
+          *pc = make_uint2(pack_bf16(cre2.x, cim2.x), pack_bf16(cre2.y, cim2.y));
         }
-        const float2 we = *reinterpret_cast<const float2*>(&P.wend[r]);
-        const float2 wre = __fmul2_rn(we, bre), wim = __fmul2_rn(we, bim);
+        const float we = P.wend[r];
+        const float2 we2 = make_float2(we, we);
+        const float2 wre = __fmul2_rn(we2, bre), wim = __fmul2_rn(we2, bim);
         const uint32_t hia = pack_bf16(wre.x, wim.x), hib = pack_bf16(wre.y, wim.y);
-        const float2 ha = unpack_bf16(hia), hb = unpack_bf16(hib);
-        const float2 lre = __fadd2_rn(wre, make_float2(-ha.x, -hb.x));
-        const float2 lim = __fadd2_rn(wim, make_float2(-ha.y, -hb.y));
-        *reinterpret_cast<uint32_t*>(sm.u.bw_hi + oa) = hia;
-        *reinterpret_cast<uint32_t*>(sm.u.bw_hi + ob) = hib;
-        *reinterpret_cast<uint32_t*>(sm.bw_lo + oa) = pack_bf16(lre.x, lim.x);
-        *reinterpret_cast<uint32_t*>(sm.bw_lo + ob) = pack_bf16(lre.y, lim.y);
+        const float2 hre = make_float2(__uint_as_float(hia << 16), __uint_as_float(hib << 16));
+        const float2 him = make_float2(__uint_as_float(hia & 0xffff0000u),
+                                       __uint_as_float(hib & 0xffff0000u));
+        const float2 lre = __fadd2_rn(wre, make_float2(-hre.x, -hre.y));
+        const float2 lim = __fadd2_rn(wim, make_float2(-him.x, -him.y));
+        *reinterpret_cast<uint2*>(sm.u.bw_hi + o) = make_uint2(hia, hib);
+        *reinterpret_cast<uint2*>(sm.bw_lo + o) =
+            make_uint2(pack_bf16(lre.x, lim.x), pack_bf16(lre.y, lim.y));
       }
-      if (ROT && seg == 3) {
-        const float pnext = wrap_angle(sm.Phi[pi] + psi[15] + off);
-        float s, co;
-        sincosf(pnext, &s, &co);
-        sm.nPhi[pi] = pnext;
-        sm.necos[pi] = co;
-        sm.nesin[pi] = s;
+      if (ROT && warp == 7) {
+        const float2 pend = __fadd2_rn(psi[7], off);
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const int pi = 2 * lane + j;
+          const float pnext = wrap_angle(sm.Phi[pi] + (j == 0 ? pend.x : pend.y));
+          float s, co;
+          sincosf(pnext, &s, &co);
+          sm.nPhi[pi] = pnext;
+          sm.necos[pi] = co;
+          sm.nesin[pi] = s;
+        }
       }
     }
     tc5::fence_proxy_async();
@@ -435,6 +440,7 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_chunk_kernel(FwdArgs a) {
                       tc5::desc_sw128(aX + (uint32_t)(j & 3) * 2048u, kAtom, 1024), kIdescS,
                       j > 0);
       }
+      tc5::commit(&sm.mbar[1]);
     }
     if (ROT && tid < NH) {
       sm.Phi[tid] = sm.nPhi[tid];
@@ -447,10 +453,7 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_chunk_kernel(FwdArgs a) {
       if (!tc5::mbar_wait(&sm.mbar[0], par, kWaitLimitNs)) sm.err = 1;
       tc5::fence_after_sync();
       // the Gram has consumed Bbar: the next chunk's raw B can stream in now
-      if (c + 1 < nC) {
-        load_bc(c + 1, B_seq, aB);
-        cp_async_commit();
-      }
+      if (loader && c + 1 < nC) tma_bc(c + 1, &tm.B, aB);
       uint32_t gr[16];
       tc5::ld_16x256b_x4(tmem + tlane + kColG + (uint32_t)cb, gr);
       tc5::wait_ld();
@@ -472,6 +475,12 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_chunk_kernel(FwdArgs a) {
                         __uint_as_float(gr[4 * q + 2 * hf + 1]) * w1);
         }
       }
+      // Y1 and S are done with Cbar and W_end o Bbar (which shares theta's space)
+      if (loader && c + 1 < nC) {
+        if (!tc5::mbar_wait(&sm.mbar[1], par, kWaitLimitNs)) sm.err = 1;
+        tma_bc(c + 1, &tm.C, aC);
+        if (ROT && has_theta) tma_theta(c + 1);
+      }
     }
     tc5::fence_proxy_async();
     tc5::fence_before_sync();
@@ -482,7 +491,7 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_chunk_kernel(FwdArgs a) {
       for (int j = 0; j < 4; ++j)
         tc5::mma_bf16(tmem + kColY2, tc5::desc_sw128(aM + (uint32_t)j * 32u, 16, 1024),
                       tc5::desc_sw128(aX + (uint32_t)j * 2048u, kAtom, 1024), kIdescY, j > 0);
-      tc5::commit(&sm.mbar[1]);
+      tc5::commit(&sm.mbar[2]);
     }
 
     // -- phase Y + S: outputs and the state update ---------------------------------
@@ -492,14 +501,8 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_chunk_kernel(FwdArgs a) {
         chunk_params(sm.prm[(c + 1) & 1], pld, pbe, pga, lane);
         if (c + 2 < nC) load_params(c + 2);
       }
-      if (!tc5::mbar_wait(&sm.mbar[1], par, kWaitLimitNs)) sm.err = 1;
+      if (!tc5::mbar_wait(&sm.mbar[2], par, kWaitLimitNs)) sm.err = 1;
       tc5::fence_after_sync();
-      // every product of this chunk is done: Cbar, theta / W_end o Bbar can be refilled
-      if (c + 1 < nC) {
-        load_bc(c + 1, C_seq, aC);
-        if (ROT) load_theta(c + 1);
-        cp_async_commit();
-      }
       uint32_t y1[16], y2[16], sv[32];
       tc5::ld_16x256b_x4(tmem + tlane + kColY1 + (uint32_t)cb, y1);
       tc5::ld_16x256b_x4(tmem + tlane + kColY2 + (uint32_t)cb, y2);
@@ -512,7 +515,7 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_chunk_kernel(FwdArgs a) {
         const int64_t t = tbase + r;
         if (r > 0 && t < L) {
           const float2 er2 = make_float2(P.ecs[r], P.ecs[r]);
-          bf16* yrow = Yg + ((b * L + t) * H + h) * PD;
+          bf16* yrow = Y_seq + t * xstride_t;
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             const int p = cb + 8 * q + 2 * (lane & 3);
@@ -539,9 +542,12 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_chunk_kernel(FwdArgs a) {
     tc5::fence_proxy_async();
     tc5::fence_before_sync();
     __syncthreads();  // S5: this chunk's operands and accumulators are consumed
-    if (sm.err) break;
+    if (sm.err) {
+      // let the next chunk's copies land before the CTA exits
+      if (c + 1 < nC) (void)tc5::mbar_wait(&sm.lmbar, par ^ 1u, kWaitLimitNs);
+      break;
+    }
   }
-  cp_async_wait_all();
 
   // ---- outputs of the last token, TMEM release ---------------------------------
   if (sm.err) {
@@ -566,13 +572,54 @@ __global__ void __launch_bounds__(kThreads, 2) fwd_chunk_kernel(FwdArgs a) {
   if (warp == 0) tc5::tmem_dealloc(tmem, kTmemCols);
 }
 
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// A 4-D map (d0 innermost, dense) with a box of d0-extent `box0` by 64 tokens.
+bool encode_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t d0, uint64_t d1,
+                uint64_t d2, uint64_t d3, uint64_t esz, uint32_t box0, CUtensorMapSwizzle sw) {
+  PFN_cuTensorMapEncodeTiled_v12000 fn = tensor_map_encoder();
+  if (!fn) return false;
+  const cuuint64_t dims[4] = {d0, d1, d2, d3};
+  const cuuint64_t strides[3] = {d0 * esz, d0 * d1 * esz, d0 * d1 * d2 * esz};
+  const cuuint32_t box[4] = {box0, 1, (cuuint32_t)Q, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(m, dt, 4, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <bool ROT>
 cudaError_t launch_variant(const FwdArgs& a, cudaStream_t s) {
+  TmaMaps tm;
+  memset(&tm, 0, sizeof(tm));
+  const uint64_t L = (uint64_t)a.L, b = (uint64_t)a.b, H = (uint64_t)a.H, G = (uint64_t)a.G;
+  bool ok = encode_map(&tm.B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.B, NS, G, L, b, 2, 64,
+                       CU_TENSOR_MAP_SWIZZLE_128B) &&
+            encode_map(&tm.C, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.C, NS, G, L, b, 2, 64,
+                       CU_TENSOR_MAP_SWIZZLE_128B) &&
+            encode_map(&tm.X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.X, PD, H, L, b, 2, 64,
+                       CU_TENSOR_MAP_SWIZZLE_128B);
+  if (ok && a.theta)
+    ok = encode_map(&tm.theta, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.theta, NH, H, L, b, 4, NH,
+                    CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (!ok) return cudaErrorInvalidValue;
   const size_t smem = sizeof(Smem) + 1024;
   cudaError_t e = cudaFuncSetAttribute(fwd_chunk_kernel<ROT>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  fwd_chunk_kernel<ROT><<<(unsigned)(a.b * a.H), kThreads, smem, s>>>(a);
+  fwd_chunk_kernel<ROT><<<(unsigned)(a.b * a.H), kThreads, smem, s>>>(a, tm);
   return cudaGetLastError();
 }
 

@@ -108,6 +108,26 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* mbar, uint32_t parity, uint6
   }
 }
 
+// Adds `bytes` to the transaction count the current phase waits for and
+// arrives once (the issuing thread's arrival).
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* mbar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(saddr(mbar)),
+               "r"(bytes)
+               : "memory");
+}
+
+// TMA: one box of a 4-D tensor map (coordinates innermost first) into shared
+// memory; completion is counted in bytes on the mbarrier.  Out-of-range box
+// elements (negative or past the end) are filled with zeros.
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const void* tmap, uint64_t* mbar, int c0,
+                                            int c1, int c2, int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(saddr(mbar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
+
 // TMEM -> registers.  16x256b.x4: thread t gets lanes base + t/4 and base + t/4 + 8,
 // 32-bit columns c + 8 g + 2 (t % 4) + {0, 1} for g = 0..3 (r[4g .. 4g+3]).
 __device__ __forceinline__ void ld_16x256b_x4(uint32_t taddr, uint32_t (&r)[16]) {

@@ -10,7 +10,7 @@
 // sums (row 0 has cs_0 = 0, psi_0 = 0)
 //     cs_r = sum_{k=1..r} logdecay_k,   psi_r = sum_{k=1..r} theta_k,
 // the rotated vectors are Bbar_r = R(Phi_c + psi_r) B_r and Cbar_r likewise, with
-// Phi_c = phi_{t0-1} carried from chunk to chunk.  The recurrence ("TorchMamba"
+// Phi_c = phi_{t0-1} (reduced to [-pi, pi]) carried from chunk to chunk.  The recurrence ("TorchMamba"
 // README, "Math notes", M3 SISO: h_t = alpha_t h_{t-1} + beta_t Bbar_{t-1} x_{t-1}^T
 // + gamma_t Bbar_t x_t^T) unrolled over the chunk reads, for output rows r = 1..63,
 //     y_r   = exp(cs_r) Cbar_r^T h + sum_{u<=r} W(r,u) (Cbar_r^T Bbar_u) x_u + D x_r
@@ -61,7 +61,8 @@ constexpr int QT = Q - 1;   // tokens per chunk
 constexpr int NS = 128;     // state size N
 constexpr int PD = 64;      // head dim P
 constexpr int NH = NS / 2;  // rotation pairs
-constexpr int kThreads = 256;
+constexpr int kCtrlWarp = 8;                 // the control warp
+constexpr int kThreads = 32 * (kCtrlWarp + 1);  // 8 compute warps + 1 control warp
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kColG = 0, kColY1 = 64, kColY2 = 128, kColS = 192;
@@ -107,8 +108,8 @@ struct Smem {
   uint8_t Hs[NS * 128];        // bf16 copy of h for the state-to-output product
   ChunkParams prm[2];
   float segtot[8][NH];
-  float ecos[NH], esin[NH], Phi[NH];     // exp(i Phi_c) per pair and Phi_c itself
-  float necos[NH], nesin[NH], nPhi[NH];  // the same for the next chunk
+  float Phi[NH];               // absolute angle at the chunk start, in [-pi, pi]
+  float nPhi[NH];              // the same for the next chunk
   uint64_t mbar[3];
   uint64_t lmbar;              // TMA loads of the next chunk
   uint32_t tmem;
@@ -184,13 +185,16 @@ __global__ void __launch_bounds__(kThreads, 2)
   const uint32_t raw_addr = tc5::saddr(smem_raw);
   Smem& sm = *reinterpret_cast<Smem*>(smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr));
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // warps 0..7 compute; warp 8 (kCtrlWarp) issues the TMA copies and the tensor-core
+  // products and prepares the next chunk's scalars
+  const bool ctrl = warp == kCtrlWarp;
+  const bool ctrl_lead = tid == kCtrlWarp * 32;
   const int64_t H = a.H, L = a.L, G = a.G;
   const int64_t bh = blockIdx.x;
   const int64_t b = bh / H, h = bh % H, g = h / (H / G);
   const int nC = (int)((L + QT - 1) / QT);
   const bf16* Xg = static_cast<const bf16*>(a.X);
   const bf16* Bg = static_cast<const bf16*>(a.B);
-  const bf16* Cg = static_cast<const bf16*>(a.C);
   bf16* Yg = static_cast<bf16*>(a.Y);
   const float Dh = a.D ? a.D[h] : 0.f;
   const uint32_t aB = tc5::saddr(sm.B), aC = tc5::saddr(sm.C);
@@ -201,7 +205,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 
   bf16* const Y_seq = Yg + (b * L * H + h) * PD;
   const int64_t xstride_t = H * PD;  // X / Y elements per token
-  // TMA issue (one thread): chunk c's rows start at token c*QT - 1
+  // TMA issue (control thread): chunk c's rows start at token c*QT - 1
   const bool has_theta = a.theta != nullptr;  // ROT without theta: rotation by angle0 only
   const uint32_t chunk_bytes = (ROT && has_theta ? 16384u : 0u) + 2u * 16384u + 8192u;
   auto tma_theta = [&](int c) {
@@ -215,9 +219,9 @@ __global__ void __launch_bounds__(kThreads, 2)
     tc5::tma_load_4d(aX0 + (uint32_t)(c & 1) * (Q * 128), &tm.X, &sm.lmbar, 0, (int)h, c * QT - 1,
                      (int)b);
   };
-  const bool loader = tid == 32;
 
-  // warp 0 keeps logdecay / beta / gamma of rows lane and lane + 32 in registers
+  // the control warp keeps logdecay / beta / gamma of rows lane and lane + 32 of
+  // the next chunk in registers
   float pld[2], pbe[2], pga[2];
   auto load_params = [&](int c) {
 #pragma unroll
@@ -234,7 +238,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 
   // ---- prologue -------------------------------------------------------------
   if (warp == 0) tc5::tmem_alloc(&sm.tmem, kTmemCols);
-  if (tid == 0) {
+  if (ctrl_lead) {
     tc5::mbar_init(&sm.mbar[0], 1);
     tc5::mbar_init(&sm.mbar[1], 1);
     tc5::mbar_init(&sm.mbar[2], 1);
@@ -243,14 +247,14 @@ __global__ void __launch_bounds__(kThreads, 2)
     sm.err = 0;
   }
   __syncthreads();  // mbarriers initialised
-  if (loader) {
+  if (ctrl_lead) {
     tc5::mbar_arrive_expect_tx(&sm.lmbar, chunk_bytes);
     if (ROT && has_theta) tma_theta(0);
     tma_bc(0, &tm.B, aB);
     tma_bc(0, &tm.C, aC);
     tma_x(0);
   }
-  if (warp == 0) {
+  if (ctrl) {
     load_params(0);
     chunk_params(sm.prm[0], pld, pbe, pga, lane);
     if (nC > 1) load_params(1);
@@ -260,23 +264,18 @@ __global__ void __launch_bounds__(kThreads, 2)
   const float bp0 = (tid < NS && a.bprev0) ? a.bprev0[(b * G + g) * NS + tid] : 0.f;
   const float xp0 = (tid < PD && a.xprev0) ? a.xprev0[bh * PD + tid] : 0.f;
   const bool patch_row0 = a.bprev0 != nullptr || a.xprev0 != nullptr;
-  if (ROT && tid < NH) {
-    const float ph0 = a.angle0 ? a.angle0[bh * NH + tid] : 0.f;
-    sm.Phi[tid] = ph0;
-    float s, c;
-    sincosf(ph0, &s, &c);
-    sm.ecos[tid] = c;
-    sm.esin[tid] = s;
-  }
+  if (ROT && tid < NH) sm.Phi[tid] = wrap_angle(a.angle0 ? a.angle0[bh * NH + tid] : 0.f);
 
-  // state fragment: row n = 32 (warp % 4) + lane, columns cb .. cb + 31
-  const int n_row = 32 * (warp & 3) + lane, cb = 32 * (warp >> 2);
+  // state fragment (compute warps): row n = 32 (warp % 4) + lane, columns cb .. cb + 31
+  const int n_row = 32 * (warp & 3) + lane, cb = 32 * ((warp >> 2) & 1);
   float hs[32];
-  {
+#pragma unroll
+  for (int j = 0; j < 32; ++j) hs[j] = 0.f;
+  if (!ctrl && a.h0) {
     const float4* src = reinterpret_cast<const float4*>(a.h0 + (bh * NS + n_row) * PD + cb);
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      const float4 v = a.h0 ? src[j] : make_float4(0.f, 0.f, 0.f, 0.f);
+      const float4 v = src[j];
       hs[4 * j] = v.x; hs[4 * j + 1] = v.y; hs[4 * j + 2] = v.z; hs[4 * j + 3] = v.w;
     }
   }
@@ -291,7 +290,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       *reinterpret_cast<uint4*>(sm.Hs + off1(n_row, cb + 8 * q)) = v;
     }
   };
-  store_state_bf16();
+  if (!ctrl) store_state_bf16();
   tc5::fence_proxy_async();
   tc5::fence_before_sync();
   __syncthreads();
@@ -308,11 +307,76 @@ __global__ void __launch_bounds__(kThreads, 2)
     const uint8_t* Xs = sm.X[c & 1];
     const uint32_t aX = aX0 + (uint32_t)(c & 1) * (Q * 128);
     if (!tc5::mbar_wait(&sm.lmbar, par, kWaitLimitNs)) sm.err = 1;
-    __syncthreads();  // S1: theta, B, C, X of this chunk are in shared memory
-    if (loader && c + 1 < nC) {
-      tc5::mbar_arrive_expect_tx(&sm.lmbar, chunk_bytes);
-      tma_x(c + 1);
+    tc5::fence_before_sync();
+    __syncthreads();  // S1: theta, B, C, X of this chunk are in shared memory; the
+                      // previous chunk's accumulators and operands are consumed
+    tc5::fence_after_sync();
+    if (sm.err) {
+      // let the copies in flight land before the CTA exits
+      (void)tc5::mbar_wait(&sm.lmbar, par, kWaitLimitNs);
+      break;
     }
+
+    if (ctrl) {
+      // ===================== control warp ======================================
+      if (ctrl_lead && c + 1 < nC) {
+        tc5::mbar_arrive_expect_tx(&sm.lmbar, chunk_bytes);
+        tma_x(c + 1);
+      }
+      if (c + 1 < nC) {
+        chunk_params(sm.prm[(c + 1) & 1], pld, pbe, pga, lane);
+        if (c + 2 < nC) load_params(c + 2);
+      }
+      __syncthreads();  // S2
+      __syncthreads();  // S3: Cbar, Bbar, W_end o Bbar ready
+      if (ctrl_lead) {
+        tc5::fence_after_sync();
+        // G = Cbar Bbar^T (both K-major), K = 128 in 8 steps of 16
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const uint32_t ko = (uint32_t)((j >> 2) * kAtom + (j & 3) * 32);
+          tc5::mma_bf16(tmem + kColG, tc5::desc_sw128(aC + ko, 16, 1024),
+                        tc5::desc_sw128(aB + ko, 16, 1024), kIdescG, j > 0);
+        }
+        tc5::commit(&sm.mbar[0]);
+        // Y1 = Cbar h (h MN-major: K = n, rows of 128 B)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const uint32_t ko = (uint32_t)((j >> 2) * kAtom + (j & 3) * 32);
+          tc5::mma_bf16(tmem + kColY1, tc5::desc_sw128(aC + ko, 16, 1024),
+                        tc5::desc_sw128(aH + (uint32_t)j * 2048u, kAtom, 1024), kIdescY, j > 0);
+        }
+        // S = (W_end o Bbar)^T X with the operand in two parts (A and B MN-major), K = 64
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const uint32_t aw = (j < 4 ? aWh : aWl) + (uint32_t)(j & 3) * 2048u;
+          tc5::mma_bf16(tmem + kColS, tc5::desc_sw128(aw, kAtom, 1024),
+                        tc5::desc_sw128(aX + (uint32_t)(j & 3) * 2048u, kAtom, 1024), kIdescS,
+                        j > 0);
+        }
+        tc5::commit(&sm.mbar[1]);
+        if (c + 1 < nC) {
+          // the Gram consumes Bbar; Y1 and S consume Cbar and W_end o Bbar (theta's space)
+          if (!tc5::mbar_wait(&sm.mbar[0], par, kWaitLimitNs)) sm.err = 1;
+          tma_bc(c + 1, &tm.B, aB);
+          if (!tc5::mbar_wait(&sm.mbar[1], par, kWaitLimitNs)) sm.err = 1;
+          tma_bc(c + 1, &tm.C, aC);
+          if (ROT && has_theta) tma_theta(c + 1);
+        }
+      }
+      __syncthreads();  // S4: M ready
+      if (ctrl_lead) {
+        tc5::fence_after_sync();
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          tc5::mma_bf16(tmem + kColY2, tc5::desc_sw128(aM + (uint32_t)j * 32u, 16, 1024),
+                        tc5::desc_sw128(aX + (uint32_t)j * 2048u, kAtom, 1024), kIdescY, j > 0);
+        tc5::commit(&sm.mbar[2]);
+      }
+      continue;
+    }
+
+    // ===================== compute warps (0..7) ===================================
     if (c == 0 && patch_row0) {
       if (tid < NS) *reinterpret_cast<bf16*>(sm.B + off2(0, tid)) = __float2bfloat16_rn(bp0);
       if (tid < PD) *reinterpret_cast<bf16*>(sm.X[0] + off1(0, tid)) = __float2bfloat16_rn(xp0);
@@ -327,13 +391,13 @@ __global__ void __launch_bounds__(kThreads, 2)
       float2 run = make_float2(0.f, 0.f);
       if (has_theta) {
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        if (warp > 0 || k > 0) {  // psi_0 = 0
-          const float2 th = *reinterpret_cast<const float2*>(&sm.u.theta[8 * warp + k][2 * lane]);
-          run = __fadd2_rn(run, th);
+        for (int k = 0; k < 8; ++k) {
+          if (warp > 0 || k > 0) {  // psi_0 = 0
+            const float2 th = *reinterpret_cast<const float2*>(&sm.u.theta[8 * warp + k][2 * lane]);
+            run = __fadd2_rn(run, th);
+          }
+          psi[k] = run;
         }
-        psi[k] = run;
-      }
       } else {
 #pragma unroll
         for (int k = 0; k < 8; ++k) psi[k] = run;
@@ -343,16 +407,16 @@ __global__ void __launch_bounds__(kThreads, 2)
     __syncthreads();  // S2: segment totals ready; theta no longer read
 
     // -- phase R2: rotation into the absolute frame, W_end o Bbar hi/lo ----------
+    // The absolute angle of row r is Phi_c + psi_r with Phi_c kept in [-pi, pi];
+    // its magnitude is bounded by pi plus one chunk's sum of theta, where the
+    // hardware sincos keeps an absolute error of about 2^-21 + |angle| 2^-24.
     {
-      float2 off = make_float2(0.f, 0.f);
-      float2 ec2 = make_float2(1.f, 1.f), es2 = make_float2(0.f, 0.f);
+      float2 base = make_float2(0.f, 0.f);
       if (ROT) {
+        base = *reinterpret_cast<const float2*>(&sm.Phi[2 * lane]);
         for (int s2 = 0; s2 < warp; ++s2)
-          off = __fadd2_rn(off, *reinterpret_cast<const float2*>(&sm.segtot[s2][2 * lane]));
-        ec2 = *reinterpret_cast<const float2*>(&sm.ecos[2 * lane]);
-        es2 = *reinterpret_cast<const float2*>(&sm.esin[2 * lane]);
+          base = __fadd2_rn(base, *reinterpret_cast<const float2*>(&sm.segtot[s2][2 * lane]));
       }
-      const float2 nes2 = make_float2(-es2.x, -es2.y);
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
         const int r = 8 * warp + k;
@@ -368,15 +432,12 @@ __global__ void __launch_bounds__(kThreads, 2)
           const float2 cre = make_float2(__uint_as_float(cw2.x << 16), __uint_as_float(cw2.y << 16));
           const float2 cim = make_float2(__uint_as_float(cw2.x & 0xffff0000u),
                                          __uint_as_float(cw2.y & 0xffff0000u));
-          const float2 ang = __fadd2_rn(psi[k], off);
+          const float2 ang = __fadd2_rn(psi[k], base);
           float s0, c0, s1, c1;
-          fast_sincos(ang.x, &s0, &c0);
-          fast_sincos(ang.y, &s1, &c1);
-          const float2 co2 = make_float2(c0, c1), si2 = make_float2(s0, s1);
-          // exp(i (Phi_c + psi)) = exp(i Phi_c) exp(i psi), per pair
-          const float2 cr = __ffma2_rn(nes2, si2, __fmul2_rn(ec2, co2));
-          const float2 sr = __ffma2_rn(ec2, si2, __fmul2_rn(es2, co2));
-          const float2 nsr = make_float2(-sr.x, -sr.y);
+          __sincosf(ang.x, &s0, &c0);
+          __sincosf(ang.y, &s1, &c1);
+          const float2 cr = make_float2(c0, c1), sr = make_float2(s0, s1);
+          const float2 nsr = make_float2(-s0, -s1);
           const float2 bre2 = __ffma2_rn(nsr, bim, __fmul2_rn(cr, bre));
           const float2 bim2 = __ffma2_rn(cr, bim, __fmul2_rn(sr, bre));
           const float2 cre2 = __ffma2_rn(nsr, cim, __fmul2_rn(cr, cre));
@@ -400,63 +461,19 @@ __global__ void __launch_bounds__(kThreads, 2)
             make_uint2(pack_bf16(lre.x, lim.x), pack_bf16(lre.y, lim.y));
       }
       if (ROT && warp == 7) {
-        const float2 pend = __fadd2_rn(psi[7], off);
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          const int pi = 2 * lane + j;
-          const float pnext = wrap_angle(sm.Phi[pi] + (j == 0 ? pend.x : pend.y));
-          float s, co;
-          sincosf(pnext, &s, &co);
-          sm.nPhi[pi] = pnext;
-          sm.necos[pi] = co;
-          sm.nesin[pi] = s;
-        }
+        const float2 pend = __fadd2_rn(psi[7], base);  // Phi_c + psi_63
+        sm.nPhi[2 * lane] = wrap_angle(pend.x);
+        sm.nPhi[2 * lane + 1] = wrap_angle(pend.y);
       }
     }
     tc5::fence_proxy_async();
     __syncthreads();  // S3: Cbar, Bbar, W_end o Bbar ready
-    if (tid == 0) {
-      tc5::fence_after_sync();
-      // G = Cbar Bbar^T (both K-major), K = 128 in 8 steps of 16
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const uint32_t ko = (uint32_t)((j >> 2) * kAtom + (j & 3) * 32);
-        tc5::mma_bf16(tmem + kColG, tc5::desc_sw128(aC + ko, 16, 1024),
-                      tc5::desc_sw128(aB + ko, 16, 1024), kIdescG, j > 0);
-      }
-      tc5::commit(&sm.mbar[0]);
-      // Y1 = Cbar h (h MN-major: K = n, rows of 128 B)
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const uint32_t ko = (uint32_t)((j >> 2) * kAtom + (j & 3) * 32);
-        tc5::mma_bf16(tmem + kColY1, tc5::desc_sw128(aC + ko, 16, 1024),
-                      tc5::desc_sw128(aH + (uint32_t)j * 2048u, kAtom, 1024), kIdescY, j > 0);
-      }
-      // S = (W_end o Bbar)^T X with the operand in two parts (A and B MN-major), K = 64
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const uint32_t aw = (j < 4 ? aWh : aWl) + (uint32_t)(j & 3) * 2048u;
-        tc5::mma_bf16(tmem + kColS, tc5::desc_sw128(aw, kAtom, 1024),
-                      tc5::desc_sw128(aX + (uint32_t)(j & 3) * 2048u, kAtom, 1024), kIdescS,
-                      j > 0);
-      }
-      tc5::commit(&sm.mbar[1]);
-    }
-    if (ROT && tid < NH) {
-      sm.Phi[tid] = sm.nPhi[tid];
-      sm.ecos[tid] = sm.necos[tid];
-      sm.esin[tid] = sm.nesin[tid];
-    }
+    if (ROT && tid < NH) sm.Phi[tid] = sm.nPhi[tid];
 
     // -- phase G: masked Gram -> M (rows 16 (warp % 4) + .., columns cb + ..) -------
     {
-      if (!tc5::mbar_wait(&sm.mbar[0], par, kWaitLimitNs)) sm.err = 1;
-      tc5::fence_after_sync();
-      // the Gram has consumed Bbar: the next chunk's raw B can stream in now
-      if (loader && c + 1 < nC) tma_bc(c + 1, &tm.B, aB);
-      uint32_t gr[16];
-      tc5::ld_16x256b_x4(tmem + tlane + kColG + (uint32_t)cb, gr);
-      tc5::wait_ld();
+      // the mask depends only on the chunk scalars: compute it while the Gram runs
+      float wv[2][4][2];
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf) {
         const int t = 16 * (warp & 3) + (lane >> 2) + 8 * hf;
@@ -470,43 +487,38 @@ __global__ void __launch_bounds__(kThreads, 2)
             w0 = (s0 == t) ? gt : (s0 < t) ? exp2f(cst - P.cs2[s0 + 1]) * cv.x : 0.f;
             w1 = (s0 + 1 == t) ? gt : (s0 + 1 < t) ? exp2f(cst - P.cs2[s0 + 2]) * cv.y : 0.f;
           }
-          *reinterpret_cast<uint32_t*>(sm.M + off1(t, s0)) =
-              pack_bf16(__uint_as_float(gr[4 * q + 2 * hf]) * w0,
-                        __uint_as_float(gr[4 * q + 2 * hf + 1]) * w1);
+          wv[hf][q][0] = w0;
+          wv[hf][q][1] = w1;
         }
       }
-      // Y1 and S are done with Cbar and W_end o Bbar (which shares theta's space)
-      if (loader && c + 1 < nC) {
-        if (!tc5::mbar_wait(&sm.mbar[1], par, kWaitLimitNs)) sm.err = 1;
-        tma_bc(c + 1, &tm.C, aC);
-        if (ROT && has_theta) tma_theta(c + 1);
+      if (!tc5::mbar_wait(&sm.mbar[0], par, kWaitLimitNs)) sm.err = 1;
+      tc5::fence_after_sync();
+      uint32_t gr[16];
+      tc5::ld_16x256b_x4(tmem + tlane + kColG + (uint32_t)cb, gr);
+      tc5::wait_ld();
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        const int t = 16 * (warp & 3) + (lane >> 2) + 8 * hf;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int s0 = cb + 8 * q + 2 * (lane & 3);
+          *reinterpret_cast<uint32_t*>(sm.M + off1(t, s0)) =
+              pack_bf16(__uint_as_float(gr[4 * q + 2 * hf]) * wv[hf][q][0],
+                        __uint_as_float(gr[4 * q + 2 * hf + 1]) * wv[hf][q][1]);
+        }
       }
     }
     tc5::fence_proxy_async();
     tc5::fence_before_sync();
     __syncthreads();  // S4: M ready
-    if (tid == 0) {
-      tc5::fence_after_sync();
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-        tc5::mma_bf16(tmem + kColY2, tc5::desc_sw128(aM + (uint32_t)j * 32u, 16, 1024),
-                      tc5::desc_sw128(aX + (uint32_t)j * 2048u, kAtom, 1024), kIdescY, j > 0);
-      tc5::commit(&sm.mbar[2]);
-    }
 
     // -- phase Y + S: outputs and the state update ---------------------------------
     {
-      // warp 0 prepares the next chunk's scalars while the products finish
-      if (warp == 0 && c + 1 < nC) {
-        chunk_params(sm.prm[(c + 1) & 1], pld, pbe, pga, lane);
-        if (c + 2 < nC) load_params(c + 2);
-      }
       if (!tc5::mbar_wait(&sm.mbar[2], par, kWaitLimitNs)) sm.err = 1;
       tc5::fence_after_sync();
-      uint32_t y1[16], y2[16], sv[32];
+      uint32_t y1[16], y2[16];
       tc5::ld_16x256b_x4(tmem + tlane + kColY1 + (uint32_t)cb, y1);
       tc5::ld_16x256b_x4(tmem + tlane + kColY2 + (uint32_t)cb, y2);
-      tc5::ld_32x32b_x32(tmem + tlane + kColS + (uint32_t)cb, sv);
       tc5::wait_ld();
       const float2 D2 = make_float2(Dh, Dh);
 #pragma unroll
@@ -529,6 +541,9 @@ __global__ void __launch_bounds__(kThreads, 2)
           }
         }
       }
+      uint32_t sv[32];
+      tc5::ld_32x32b_x32(tmem + tlane + kColS + (uint32_t)cb, sv);
+      tc5::wait_ld();
       const float2 eE2 = make_float2(P.eE, P.eE);
 #pragma unroll
       for (int j = 0; j < 32; j += 2) {
@@ -540,19 +555,12 @@ __global__ void __launch_bounds__(kThreads, 2)
       store_state_bf16();
     }
     tc5::fence_proxy_async();
-    tc5::fence_before_sync();
-    __syncthreads();  // S5: this chunk's operands and accumulators are consumed
-    if (sm.err) {
-      // let the next chunk's copies land before the CTA exits
-      if (c + 1 < nC) (void)tc5::mbar_wait(&sm.lmbar, par ^ 1u, kWaitLimitNs);
-      break;
-    }
   }
 
   // ---- outputs of the last token, TMEM release ---------------------------------
   if (sm.err) {
     if (tid == 0) atomicAdd(&g_chunk_wait_timeouts, 1u);
-  } else {
+  } else if (!ctrl) {
     if (a.hT) {
       float4* dst = reinterpret_cast<float4*>(a.hT + (bh * NS + n_row) * PD + cb);
 #pragma unroll

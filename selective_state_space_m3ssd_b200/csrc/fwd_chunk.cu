@@ -90,10 +90,20 @@ __device__ __forceinline__ uint32_t off1(int r, int c) {
 // gamma, and exp(cs_63).  Double-buffered: chunk c+1's set is computed while
 // chunk c is finishing.
 struct ChunkParams {
-  float cs2[Q], ecs[Q], cvec[Q], wend[Q], gam[Q];
-  float eE;
+  float cs2[Q];    // cs_r log2(e)
+  float ecs[Q];    // exp(cs_r)
+  float cvec[Q];   // gamma_r alpha_{r+1} + beta_{r+1}  (gamma_63 for r = 63)
+  float wend[Q];   // W(63, r)
+  float gam[Q];    // gamma_r
+  float et[Q];     // exp(cs_t - cs_{8 floor(t/8)})
+  float fs[224];   // exp(cs_{8k} - cs_{s+1}) cvec_s for s < 8k, at fs_index(k, s)
+  float eE;        // exp(cs_63)
   float pad[3];
 };
+
+// The factor table keeps only the entries below the diagonal blocks: block
+// row k = 1..7 holds the 8k columns s < 8k, starting at 4 k (k - 1).
+__host__ __device__ constexpr int fs_index(int k, int s) { return 4 * k * (k - 1) + s; }
 
 struct Smem {
   union {
@@ -115,6 +125,9 @@ struct Smem {
   uint32_t tmem;
   uint32_t err;
 };
+// two CTAs per SM: 228 KB of shared memory, 1 KB of it reserved per CTA, plus the
+// 1 KB alignment slack of each CTA's dynamic block
+static_assert(2 * (sizeof(Smem) + 1024 + 1024) <= 233472, "two CTAs per SM");
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -124,12 +137,22 @@ __device__ __forceinline__ float2 unpack_bf16(uint32_t u) {
   return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
 }
 
-// Warp 0: the scalars of one chunk from its per-row logdecay / beta / gamma
-// (rows lane and lane + 32; row 0 holds zeros).
+// 2^x by the hardware approximation (relative error about 2^-22; flushes
+// results below 2^-126 to zero).  The arguments are differences of fp32 decay
+// sums, whose own rounding (about |cs| 2^-24) dominates that error.
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// One warp: the scalars of one chunk from its per-row logdecay / beta / gamma
+// (rows lane and lane + 32; row 0 and rows past the end hold zeros).
 __device__ __forceinline__ void chunk_params(ChunkParams& P, const float (&pld)[2],
                                              const float (&pbe)[2], const float (&pga)[2],
                                              int lane) {
-  float s0 = pld[0], s1 = pld[1];
+  // decay sums in log2 units
+  float s0 = pld[0] * kLog2e, s1 = pld[1] * kLog2e;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
     const float u0 = __shfl_up_sync(0xffffffffu, s0, o);
@@ -148,25 +171,38 @@ __device__ __forceinline__ void chunk_params(ChunkParams& P, const float (&pld)[
   const float ld_32 = __shfl_sync(0xffffffffu, pld[1], 0);
   const float be_32 = __shfl_sync(0xffffffffu, pbe[1], 0);
   const float cs_32 = __shfl_sync(0xffffffffu, s1, 0);
+  // the sum at the first row of each 8-row block, and at this lane's own block
+  float mk[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k)
+    mk[k] = __shfl_sync(0xffffffffu, k < 4 ? s0 : s1, (8 * k) & 31);
+  const float mown0 = __shfl_sync(0xffffffffu, s0, lane & ~7);
+  const float mown1 = __shfl_sync(0xffffffffu, s1, lane & ~7);
 #pragma unroll
   for (int k = 0; k < 2; ++k) {
     const int r = lane + 32 * k;
     const float ld_next = k == 0 ? (lane < 31 ? ld_dn0 : ld_32) : ld_dn1;
     const float be_next = k == 0 ? (lane < 31 ? be_dn0 : be_32) : be_dn1;
     const float cs_next = k == 0 ? (lane < 31 ? cs_dn0 : cs_32) : cs_dn1;
-    P.cs2[r] = cs[k] * kLog2e;
-    P.ecs[r] = expf(cs[k]);
+    P.cs2[r] = cs[k];
+    P.ecs[r] = ex2(cs[k]);
     P.gam[r] = pga[k];
+    P.et[r] = ex2(cs[k] - (k == 0 ? mown0 : mown1));
+    float cv;
     if (r < Q - 1) {
-      const float cv = pga[k] * expf(ld_next) + be_next;
-      P.cvec[r] = cv;
-      P.wend[r] = expf(cs_end - cs_next) * cv;
+      cv = pga[k] * ex2(ld_next * kLog2e) + be_next;
+      P.wend[r] = ex2(cs_end - cs_next) * cv;
     } else {
-      P.cvec[r] = pga[k];
-      P.wend[r] = pga[k];
+      cv = pga[k];
+      P.wend[r] = cv;
     }
+    P.cvec[r] = cv;
+    // the factor table, for the blocks k2 strictly below this column's block
+#pragma unroll
+    for (int k2 = 0; k2 < 8; ++k2)
+      if (8 * k2 > r) P.fs[fs_index(k2, r)] = ex2(mk[k2] - cs_next) * cv;
   }
-  if (lane == 0) P.eE = expf(cs_end);
+  if (lane == 0) P.eE = ex2(cs_end);
 }
 
 // Tensor maps of the chunk inputs, built on the host for each launch.
@@ -306,7 +342,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     const ChunkParams& P = sm.prm[c & 1];
     const uint8_t* Xs = sm.X[c & 1];
     const uint32_t aX = aX0 + (uint32_t)(c & 1) * (Q * 128);
-    if (!tc5::mbar_wait(&sm.lmbar, par, kWaitLimitNs)) sm.err = 1;
+    if (tid == 0 && !tc5::mbar_wait(&sm.lmbar, par, kWaitLimitNs)) sm.err = 1;
     tc5::fence_before_sync();
     __syncthreads();  // S1: theta, B, C, X of this chunk are in shared memory; the
                       // previous chunk's accumulators and operands are consumed
@@ -331,28 +367,29 @@ __global__ void __launch_bounds__(kThreads, 2)
       __syncthreads();  // S3: Cbar, Bbar, W_end o Bbar ready
       if (ctrl_lead) {
         tc5::fence_after_sync();
+        // descriptors of the operand tiles: an offset inside a tile only adds
+        // (offset >> 4) to the start-address field (shared addresses stay below 256 KB)
+        const uint64_t dC = tc5::desc_sw128(aC, 16, 1024), dB = tc5::desc_sw128(aB, 16, 1024);
+        const uint64_t dH = tc5::desc_sw128(aH, kAtom, 1024), dX = tc5::desc_sw128(aX, kAtom, 1024);
+        const uint64_t dWh = tc5::desc_sw128(aWh, kAtom, 1024), dWl = tc5::desc_sw128(aWl, kAtom, 1024);
         // G = Cbar Bbar^T (both K-major), K = 128 in 8 steps of 16
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          const uint32_t ko = (uint32_t)((j >> 2) * kAtom + (j & 3) * 32);
-          tc5::mma_bf16(tmem + kColG, tc5::desc_sw128(aC + ko, 16, 1024),
-                        tc5::desc_sw128(aB + ko, 16, 1024), kIdescG, j > 0);
+          const uint64_t ko = (uint64_t)(((j >> 2) * kAtom + (j & 3) * 32) >> 4);
+          tc5::mma_bf16(tmem + kColG, dC + ko, dB + ko, kIdescG, j > 0);
         }
         tc5::commit(&sm.mbar[0]);
         // Y1 = Cbar h (h MN-major: K = n, rows of 128 B)
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          const uint32_t ko = (uint32_t)((j >> 2) * kAtom + (j & 3) * 32);
-          tc5::mma_bf16(tmem + kColY1, tc5::desc_sw128(aC + ko, 16, 1024),
-                        tc5::desc_sw128(aH + (uint32_t)j * 2048u, kAtom, 1024), kIdescY, j > 0);
+          const uint64_t ko = (uint64_t)(((j >> 2) * kAtom + (j & 3) * 32) >> 4);
+          tc5::mma_bf16(tmem + kColY1, dC + ko, dH + (uint64_t)(j * (2048 >> 4)), kIdescY, j > 0);
         }
         // S = (W_end o Bbar)^T X with the operand in two parts (A and B MN-major), K = 64
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          const uint32_t aw = (j < 4 ? aWh : aWl) + (uint32_t)(j & 3) * 2048u;
-          tc5::mma_bf16(tmem + kColS, tc5::desc_sw128(aw, kAtom, 1024),
-                        tc5::desc_sw128(aX + (uint32_t)(j & 3) * 2048u, kAtom, 1024), kIdescS,
-                        j > 0);
+          const uint64_t kofs = (uint64_t)((j & 3) * (2048 >> 4));
+          tc5::mma_bf16(tmem + kColS, (j < 4 ? dWh : dWl) + kofs, dX + kofs, kIdescS, j > 0);
         }
         tc5::commit(&sm.mbar[1]);
         if (c + 1 < nC) {
@@ -367,10 +404,11 @@ __global__ void __launch_bounds__(kThreads, 2)
       __syncthreads();  // S4: M ready
       if (ctrl_lead) {
         tc5::fence_after_sync();
+        const uint64_t dM = tc5::desc_sw128(aM, 16, 1024), dX = tc5::desc_sw128(aX, kAtom, 1024);
 #pragma unroll
         for (int j = 0; j < 4; ++j)
-          tc5::mma_bf16(tmem + kColY2, tc5::desc_sw128(aM + (uint32_t)j * 32u, 16, 1024),
-                        tc5::desc_sw128(aX + (uint32_t)j * 2048u, kAtom, 1024), kIdescY, j > 0);
+          tc5::mma_bf16(tmem + kColY2, dM + (uint64_t)(j * (32 >> 4)), dX + (uint64_t)(j * (2048 >> 4)),
+                        kIdescY, j > 0);
         tc5::commit(&sm.mbar[2]);
       }
       continue;
@@ -472,20 +510,32 @@ __global__ void __launch_bounds__(kThreads, 2)
 
     // -- phase G: masked Gram -> M (rows 16 (warp % 4) + .., columns cb + ..) -------
     {
-      // the mask depends only on the chunk scalars: compute it while the Gram runs
+      // the mask depends only on the chunk scalars: compute it while the Gram runs.
+      // Row t = 16 (warp % 4) + lane/4 + 8 hf lies in 8-row block kr = t / 8; column
+      // block kc = cb/8 + q.  Below the diagonal blocks the weight factorises through
+      // the decay at the block's first row (both factors at most 1); the diagonal
+      // block takes the direct exponential; blocks with kc > kr are zero.
       float wv[2][4][2];
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf) {
         const int t = 16 * (warp & 3) + (lane >> 2) + 8 * hf;
-        const float cst = P.cs2[t], gt = P.gam[t];
+        const int kr = 2 * (warp & 3) + hf;
+        const float et = P.et[t];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
+          const int kc = (cb >> 3) + q;
           const int s0 = cb + 8 * q + 2 * (lane & 3);
           float w0 = 0.f, w1 = 0.f;
-          if (cb + 8 * q <= t) {  // this 8-column group reaches the diagonal or below
-            const float2 cv = *reinterpret_cast<const float2*>(&P.cvec[s0]);
-            w0 = (s0 == t) ? gt : (s0 < t) ? exp2f(cst - P.cs2[s0 + 1]) * cv.x : 0.f;
-            w1 = (s0 + 1 == t) ? gt : (s0 + 1 < t) ? exp2f(cst - P.cs2[s0 + 2]) * cv.y : 0.f;
+          if (kc < kr) {
+            const float2 f = *reinterpret_cast<const float2*>(&P.fs[fs_index(kr, s0)]);
+            w0 = et * f.x;
+            w1 = et * f.y;
+          } else if (kc == kr) {
+            const float cst = P.cs2[t];
+            if (s0 < t) w0 = ex2(cst - P.cs2[s0 + 1]) * P.cvec[s0];
+            else if (s0 == t) w0 = P.gam[t];
+            if (s0 + 1 < t) w1 = ex2(cst - P.cs2[s0 + 2]) * P.cvec[s0 + 1];
+            else if (s0 + 1 == t) w1 = P.gam[t];
           }
           wv[hf][q][0] = w0;
           wv[hf][q][1] = w1;

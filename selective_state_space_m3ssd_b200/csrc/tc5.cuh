@@ -90,12 +90,19 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
-// Waits for the phase of the given parity to complete; gives up after
-// `limit_ns` nanoseconds of wall time and returns false.
-__device__ __forceinline__ bool mbar_wait(uint64_t* mbar, uint32_t parity, uint64_t limit_ns) {
+// Waits for the phase of the given parity to complete (each probe may block
+// for a short, hardware-chosen time).  Gives up and returns false after
+// `limit_ns` nanoseconds of wall time, or as soon as `*err` (if given) is
+// non-zero.  A suspend-time hint on the probe made every hand-off slower on
+// B200 (suspended threads resumed late), so none is given; a waiter off the
+// critical path passes `backoff_ns` to sleep between probes instead of taking
+// issue slots from the warps that do the work.
+__device__ __forceinline__ bool mbar_wait(uint64_t* mbar, uint32_t parity, uint64_t limit_ns,
+                                          const volatile uint32_t* err = nullptr,
+                                          uint32_t backoff_ns = 0) {
   const uint32_t a = saddr(mbar);
-  const uint64_t t0 = globaltimer_ns();
-  for (uint32_t i = 0;; ++i) {
+  uint64_t t0 = 0;
+  for (uint32_t i = 1;; ++i) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred P1;\n\tmbarrier.try_wait.parity.shared::cta.b64 P1, [%1], %2;\n\t"
@@ -104,8 +111,46 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* mbar, uint32_t parity, uint6
         : "r"(a), "r"(parity)
         : "memory");
     if (ok) return true;
-    if ((i & 63u) == 63u && globaltimer_ns() - t0 > limit_ns) return false;
+    if (backoff_ns) __nanosleep(backoff_ns);
+    if ((i & 15u) == 0) {  // the clock and the error flag every 16 probes
+      const uint64_t now = globaltimer_ns();
+      if (t0 == 0) {
+        t0 = now;
+      } else if (now - t0 > limit_ns) {
+        return false;
+      }
+      if (err && *err) return false;
+    }
   }
+}
+
+// Non-blocking probe: has the phase of the given parity completed?
+__device__ __forceinline__ bool mbar_test(uint64_t* mbar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred P1;\n\tmbarrier.test_wait.parity.shared::cta.b64 P1, [%1], %2;\n\t"
+      "selp.b32 %0, 1, 0, P1;\n\t}\n"
+      : "=r"(ok)
+      : "r"(saddr(mbar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// One arrival (release semantics at CTA scope).
+__device__ __forceinline__ void mbar_arrive(uint64_t* mbar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(saddr(mbar)) : "memory");
+}
+
+// Named barrier `id` over `nthreads` threads that also ORs a flag across them.
+__device__ __forceinline__ bool bar_or(uint32_t id, uint32_t nthreads, bool flag) {
+  uint32_t out;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\tsetp.ne.u32 pi, %1, 0;\n\t"
+      "bar.red.or.pred po, %2, %3, pi;\n\tselp.u32 %0, 1, 0, po;\n\t}\n"
+      : "=r"(out)
+      : "r"(flag ? 1u : 0u), "r"(id), "r"(nthreads)
+      : "memory");
+  return out != 0;
 }
 
 // Adds `bytes` to the transaction count the current phase waits for and
@@ -149,6 +194,23 @@ __device__ __forceinline__ void ld_32x32b_x32(uint32_t taddr, uint32_t (&r)[32])
         "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
         "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
         "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+// 16x256b.x2: as x4 with g = 0..1 (r[4g .. 4g+3]).
+__device__ __forceinline__ void ld_16x256b_x2(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.16x256b.x2.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                 "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+}
+// 32x32b.x16: thread t gets lane base + t, 32-bit columns c .. c + 15.
+__device__ __forceinline__ void ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15},"
+      " [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
       : "r"(taddr));
 }
 __device__ __forceinline__ void wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }

@@ -56,6 +56,8 @@ def _bind(path: str):
     lib.oracle_fwd.restype = ctypes.c_int
     lib.oracle_step.argtypes = [ctypes.POINTER(_Dims)] + [dp] * 13
     lib.oracle_step.restype = ctypes.c_int
+    lib.oracle_bwd.argtypes = [ctypes.POINTER(_Dims)] + [dp] * 26 + [ctypes.c_int]
+    lib.oracle_bwd.restype = ctypes.c_int
     return lib
 
 
@@ -169,6 +171,52 @@ def oracle_fwd(X, logdecay, beta, gamma, B, C, theta=None, D=None, h0=None,
         if h0 is not None:
             hT[:] = h0
     return {"Y": Y, "hT": hT, "angleT": angleT, "xprevT": xprevT, "bprevT": bprevT}
+
+
+def oracle_bwd(X, logdecay, beta, gamma, B, C, theta=None, D=None, h0=None,
+               angle0=None, xprev0=None, bprev0=None, *, dY, dhT=None,
+               nthreads: int | None = None):
+    """Reverse-mode derivatives of :func:`oracle_fwd` (fp64, sequential in t).
+
+    ``dY`` (b,L,H,P) and ``dhT`` (b,H,N,P, None = 0) are the upstream
+    gradients of Y and hT.  Returns a dict with dX, dlogdecay, dbeta, dgamma,
+    dB, dC, dtheta, dD, dh0, dangle0, dxprev0, dbprev0 (float64, each shaped
+    like its input; an input passed as None is read as zero and its gradient is
+    the derivative there).
+    """
+    X, logdecay, beta, gamma = _f64(X), _f64(logdecay), _f64(beta), _f64(gamma)
+    B, C, theta, D, h0 = _f64(B), _f64(C), _f64(theta), _f64(D), _f64(h0)
+    angle0, xprev0, bprev0 = _f64(angle0), _f64(xprev0), _f64(bprev0)
+    dY, dhT = _f64(dY), _f64(dhT)
+    b, L, H, P = X.shape
+    G, N = B.shape[2], B.shape[3]
+    if N % 2 or H % G:
+        raise ValueError("oracle_bwd: N must be even and H divisible by G")
+    if dY.shape != X.shape:
+        raise ValueError("oracle_bwd: dY shape")
+    if dhT is not None and dhT.shape != (b, H, N, P):
+        raise ValueError("oracle_bwd: dhT shape")
+    d = _Dims(b, L, H, P, N, G)
+    out = {"dX": np.zeros((b, L, H, P)), "dlogdecay": np.zeros((b, L, H)),
+           "dbeta": np.zeros((b, L, H)), "dgamma": np.zeros((b, L, H)),
+           "dB": np.zeros((b, L, G, N)), "dC": np.zeros((b, L, G, N)),
+           "dtheta": np.zeros((b, L, H, N // 2)), "dD": np.zeros((H,)),
+           "dh0": np.zeros((b, H, N, P)), "dangle0": np.zeros((b, H, N // 2)),
+           "dxprev0": np.zeros((b, H, P)), "dbprev0": np.zeros((b, G, N))}
+    o = out
+    rc = _load().oracle_bwd(ctypes.byref(d), _ptr(X), _ptr(logdecay), _ptr(beta), _ptr(gamma),
+                            _ptr(B), _ptr(C), _ptr(theta), _ptr(D), _ptr(h0), _ptr(angle0),
+                            _ptr(xprev0), _ptr(bprev0), _ptr(dY), _ptr(dhT),
+                            _ptr(o["dX"]), _ptr(o["dlogdecay"]), _ptr(o["dbeta"]),
+                            _ptr(o["dgamma"]), _ptr(o["dB"]), _ptr(o["dC"]), _ptr(o["dtheta"]),
+                            _ptr(o["dD"]), _ptr(o["dh0"]), _ptr(o["dangle0"]),
+                            _ptr(o["dxprev0"]), _ptr(o["dbprev0"]),
+                            int(nthreads or default_threads()))
+    if rc != 0:
+        raise RuntimeError(f"oracle_bwd failed with code {rc}")
+    if L == 0 and dhT is not None:
+        out["dh0"][:] = dhT
+    return out
 
 
 def oracle_step(cache, x_t, logdecay_t, beta_t, gamma_t, B_t, C_t, theta_t=None, D=None):

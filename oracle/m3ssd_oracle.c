@@ -265,3 +265,279 @@ int oracle_step(const oracle_dims* d, const double* x_t, const double* logdecay_
   free(phi_new); free(Bbar); free(Cbar); free(Bpbar);
   return 0;
 }
+
+/* ---------------------------------------------------------------------------
+ * Backward (reverse-mode derivatives of the forward above).
+ *
+ * For one (b, h) the forward is recomputed with every state S_t kept, then the
+ * adjoint of each step is taken in reverse time order.  With g = dL/dS_t (it
+ * starts as dhT and collects every later step's contribution):
+ *   y_t = Cbar_t^T S_t + D x_t      -> dCbar_t = S_t dy_t,  g += Cbar_t dy_t^T,
+ *                                      dD += dy_t . x_t,    dx_t += D dy_t
+ *   S_t = a_t S_{t-1} + beta_t Bpbar xp^T + gamma_t Bbar_t x_t^T, a_t = exp(logdecay_t)
+ *                                   -> dlogdecay_t = a_t <g, S_{t-1}>,
+ *                                      dbeta_t = Bpbar^T g xp,  dgamma_t = Bbar_t^T g x_t,
+ *                                      dBbar_t = gamma_t g x_t, dx_t += gamma_t g^T Bbar_t,
+ *                                      dBpbar = beta_t g xp,    dxp += beta_t g^T Bpbar,
+ *                                      and g <- a_t g becomes dL/dS_{t-1}
+ *   vbar = R(phi) v (each pair)     -> dv = R(phi)^T dvbar,
+ *                                      dphi_i += dvbar_{2i} (-vbar_{2i+1}) + dvbar_{2i+1} vbar_{2i}
+ *   phi_t = angle0 + sum_{s<=t} theta_s -> dtheta_s = sum_{t>=s} dphi_t,
+ *                                      dangle0 = sum_{t>=-1} dphi_t
+ * The previous-step inputs of token 0 are the cache entries xprev0 and bprev0
+ * (rotated by angle0 = phi_{-1}); h0 = S_{-1} gets g after the last step.
+ * --------------------------------------------------------------------------- */
+typedef struct {
+  const oracle_dims* d;
+  const double *X, *logdecay, *beta, *gamma, *B, *C, *theta, *D, *h0;
+  const double *angle0, *xprev0, *bprev0, *dY, *dhT;
+  double *dX, *dlogdecay, *dbeta, *dgamma, *dtheta, *dh0, *dangle0, *dxprev0;
+  double *dB_head;      /* (b,L,H,N): each head's share of dB, summed over the group later */
+  double *dC_head;      /* (b,L,H,N) likewise for dC */
+  double *dbprev_head;  /* (b,H,N) likewise for dbprev0 */
+  double *dD_bh;        /* (b,H) partial sums of dD */
+  int64_t next_pair;
+  pthread_mutex_t mu;
+  int status;
+} bwd_job;
+
+/* d(R(phi) v)/dphi_i . dvbar for each pair, and dv = R(phi)^T dvbar (accumulated). */
+static void rotate_pairs_adjoint(const double* vbar, const double* dvbar, const double* phi,
+                                 int64_t n, double* dv_acc, double* dphi_acc) {
+  for (int64_t i = 0; i < n / 2; ++i) {
+    const double c = cos(phi[i]);
+    const double s = sin(phi[i]);
+    const double d0 = dvbar[2 * i], d1 = dvbar[2 * i + 1];
+    dv_acc[2 * i] += c * d0 + s * d1;
+    dv_acc[2 * i + 1] += -s * d0 + c * d1;
+    dphi_acc[i] += -d0 * vbar[2 * i + 1] + d1 * vbar[2 * i];
+  }
+}
+
+static int bwd_one(bwd_job* j, int64_t b, int64_t h) {
+  const oracle_dims* d = j->d;
+  const int64_t L = d->seqlen, H = d->nheads, P = d->headdim, N = d->dstate, G = d->ngroups;
+  const int64_t g = h / (H / G), NH = N / 2, NP = N * P, bh = b * H + h;
+  /* phi_t and S_t for t = -1 .. L-1 live at index t + 1 */
+  double* phi = calloc((size_t)((L + 1) * NH), sizeof(double));
+  double* S = calloc((size_t)((L + 1) * NP), sizeof(double));
+  double* dphi = calloc((size_t)((L + 1) * NH), sizeof(double));
+  double* gS = calloc((size_t)NP, sizeof(double));
+  double* zero = calloc((size_t)(N > P ? N : P), sizeof(double));
+  double* vb = malloc((size_t)(6 * N) * sizeof(double));
+  if (!phi || !S || !dphi || !gS || !zero || !vb) {
+    free(phi); free(S); free(dphi); free(gS); free(zero); free(vb);
+    return 1;
+  }
+  double *Bbar = vb, *Cbar = vb + N, *Bpbar = vb + 2 * N;
+  double *dBbar = vb + 3 * N, *dCbar = vb + 4 * N, *dBpbar = vb + 5 * N;
+  const double Dh = j->D ? j->D[h] : 0.0;
+  const double* xprev0 = j->xprev0 ? j->xprev0 + bh * P : zero;
+  const double* bprev0 = j->bprev0 ? j->bprev0 + (b * G + g) * N : zero;
+
+  /* forward recompute, keeping every angle and state */
+  for (int64_t i = 0; i < NH; ++i) phi[i] = j->angle0 ? j->angle0[bh * NH + i] : 0.0;
+  if (j->h0)
+    for (int64_t e = 0; e < NP; ++e) S[e] = j->h0[bh * NP + e];
+  for (int64_t t = 0; t < L; ++t) {
+    const int64_t th = (b * L + t) * H + h, tg = (b * L + t) * G + g;
+    const double* x = j->X + th * P;
+    const double* xp = t > 0 ? j->X + (th - H) * P : xprev0;
+    const double* Bprev = t > 0 ? j->B + (tg - G) * N : bprev0;
+    double* ph = phi + (t + 1) * NH;
+    for (int64_t i = 0; i < NH; ++i) ph[i] = ph[i - NH] + (j->theta ? j->theta[th * NH + i] : 0.0);
+    rotate_pairs(j->B + tg * N, ph, N, Bbar);
+    rotate_pairs(Bprev, ph - NH, N, Bpbar);
+    const double a = exp(j->logdecay[th]);
+    const double be = j->beta ? j->beta[th] : 0.0, ga = j->gamma[th];
+    const double* Sp = S + t * NP;
+    double* St = S + (t + 1) * NP;
+    for (int64_t n = 0; n < N; ++n)
+      for (int64_t p = 0; p < P; ++p)
+        St[n * P + p] = a * Sp[n * P + p] + be * Bpbar[n] * xp[p] + ga * Bbar[n] * x[p];
+  }
+
+  /* reverse sweep */
+  for (int64_t t = 0; t < L; ++t)
+    for (int64_t p = 0; p < P; ++p) j->dX[((b * L + t) * H + h) * P + p] = 0.0;
+  if (j->dhT)
+    for (int64_t e = 0; e < NP; ++e) gS[e] = j->dhT[bh * NP + e];
+  double dD = 0.0;
+  for (int64_t t = L - 1; t >= 0; --t) {
+    const int64_t th = (b * L + t) * H + h, tg = (b * L + t) * G + g;
+    const double* x = j->X + th * P;
+    const double* xp = t > 0 ? j->X + (th - H) * P : xprev0;
+    const double* Bprev = t > 0 ? j->B + (tg - G) * N : bprev0;
+    const double* ph = phi + (t + 1) * NH;
+    const double* St = S + (t + 1) * NP;
+    const double* Sp = S + t * NP;
+    const double* dy = j->dY + th * P;
+    double* dx = j->dX + th * P;
+    rotate_pairs(j->B + tg * N, ph, N, Bbar);
+    rotate_pairs(j->C + tg * N, ph, N, Cbar);
+    rotate_pairs(Bprev, ph - NH, N, Bpbar);
+
+    /* y_t = Cbar_t^T S_t + D x_t */
+    for (int64_t n = 0; n < N; ++n) {
+      double acc = 0.0;
+      for (int64_t p = 0; p < P; ++p) acc += St[n * P + p] * dy[p];
+      dCbar[n] = acc;
+    }
+    for (int64_t n = 0; n < N; ++n)
+      for (int64_t p = 0; p < P; ++p) gS[n * P + p] += Cbar[n] * dy[p];
+    for (int64_t p = 0; p < P; ++p) {
+      dD += dy[p] * x[p];
+      dx[p] += Dh * dy[p];
+    }
+
+    /* S_t = a S_{t-1} + beta Bpbar xp^T + gamma Bbar x^T */
+    const double a = exp(j->logdecay[th]);
+    const double be = j->beta ? j->beta[th] : 0.0, ga = j->gamma[th];
+    double da = 0.0, dbe = 0.0, dga = 0.0;
+    for (int64_t n = 0; n < N; ++n) {
+      double gx = 0.0, gxp = 0.0;
+      for (int64_t p = 0; p < P; ++p) {
+        const double gv = gS[n * P + p];
+        da += gv * Sp[n * P + p];
+        gx += gv * x[p];
+        gxp += gv * xp[p];
+      }
+      dga += Bbar[n] * gx;
+      dbe += Bpbar[n] * gxp;
+      dBbar[n] = ga * gx;
+      dBpbar[n] = be * gxp;
+    }
+    for (int64_t p = 0; p < P; ++p) {
+      double gb = 0.0, gbp = 0.0;
+      for (int64_t n = 0; n < N; ++n) {
+        gb += gS[n * P + p] * Bbar[n];
+        gbp += gS[n * P + p] * Bpbar[n];
+      }
+      dx[p] += ga * gb;
+      if (t > 0)
+        j->dX[(th - H) * P + p] += be * gbp;
+      else if (j->dxprev0)
+        j->dxprev0[bh * P + p] = be * gbp;
+    }
+    j->dlogdecay[th] = a * da;
+    j->dgamma[th] = dga;
+    if (j->dbeta) j->dbeta[th] = dbe;
+    for (int64_t e = 0; e < NP; ++e) gS[e] *= a;
+
+    /* rotations: Bbar_t and Cbar_t by phi_t, the previous step's B by phi_{t-1} */
+    double* dph = dphi + (t + 1) * NH;
+    rotate_pairs_adjoint(Bbar, dBbar, ph, N, j->dB_head + th * N, dph);
+    rotate_pairs_adjoint(Cbar, dCbar, ph, N, j->dC_head + th * N, dph);
+    rotate_pairs_adjoint(Bpbar, dBpbar, ph - NH, N,
+                         t > 0 ? j->dB_head + (th - H) * N : j->dbprev_head + bh * N, dph - NH);
+  }
+  if (j->dh0)
+    for (int64_t e = 0; e < NP; ++e) j->dh0[bh * NP + e] = gS[e];
+  /* phi_t = angle0 + sum_{s<=t} theta_s: suffix sums of dphi */
+  for (int64_t i = 0; i < NH; ++i) {
+    double run = 0.0;
+    for (int64_t t = L - 1; t >= 0; --t) {
+      run += dphi[(t + 1) * NH + i];
+      if (j->dtheta) j->dtheta[((b * L + t) * H + h) * NH + i] = run;
+    }
+    if (j->dangle0) j->dangle0[bh * NH + i] = run + dphi[i];
+  }
+  j->dD_bh[bh] = dD;
+  free(phi); free(S); free(dphi); free(gS); free(zero); free(vb);
+  return 0;
+}
+
+static void* bwd_worker(void* arg) {
+  bwd_job* j = (bwd_job*)arg;
+  const int64_t npairs = j->d->batch * j->d->nheads;
+  for (;;) {
+    pthread_mutex_lock(&j->mu);
+    const int64_t k = j->next_pair++;
+    pthread_mutex_unlock(&j->mu);
+    if (k >= npairs) break;
+    if (bwd_one(j, k / j->d->nheads, k % j->d->nheads) != 0) {
+      pthread_mutex_lock(&j->mu);
+      j->status = 1;
+      pthread_mutex_unlock(&j->mu);
+    }
+  }
+  return NULL;
+}
+
+/*
+ * Backward of oracle_fwd for upstream gradients dY (b,L,H,P) and dhT
+ * (b,H,N,P, NULL = 0).  Outputs use the layouts of the matching inputs:
+ * dX, dlogdecay, dgamma, dB, dC are required; dbeta, dtheta, dD, dh0,
+ * dangle0, dxprev0, dbprev0 may be NULL (not written).  The cache outputs
+ * angleT, xprevT and bprevT get no upstream gradient.  An input passed as
+ * NULL is read as zero and its gradient is the derivative there.  Group-shared
+ * gradients (dB, dbprev0) and dD are summed in a fixed order after the
+ * per-sequence work, so the result does not depend on the thread count.
+ * Returns 0 on success, 1 on bad dimensions or pointers, 2 on allocation failure.
+ */
+int oracle_bwd(const oracle_dims* d, const double* X, const double* logdecay, const double* beta,
+               const double* gamma, const double* B, const double* C, const double* theta,
+               const double* D, const double* h0, const double* angle0, const double* xprev0,
+               const double* bprev0, const double* dY, const double* dhT, double* dX,
+               double* dlogdecay, double* dbeta, double* dgamma, double* dB, double* dC,
+               double* dtheta, double* dD, double* dh0, double* dangle0, double* dxprev0,
+               double* dbprev0, int nthreads) {
+  if (!dims_ok(d)) return 1;
+  const int64_t Bt = d->batch, L = d->seqlen, H = d->nheads, N = d->dstate, G = d->ngroups;
+  if (Bt * L > 0 && (!X || !logdecay || !gamma || !B || !C || !dY || !dX || !dlogdecay ||
+                     !dgamma || !dB || !dC))
+    return 1;
+  double* dB_head = calloc((size_t)(Bt * L * H * N + 1), sizeof(double));
+  double* dC_head = calloc((size_t)(Bt * L * H * N + 1), sizeof(double));
+  double* dbprev_head = calloc((size_t)(Bt * H * N + 1), sizeof(double));
+  double* dD_bh = calloc((size_t)(Bt * H + 1), sizeof(double));
+  if (!dB_head || !dC_head || !dbprev_head || !dD_bh) {
+    free(dB_head); free(dC_head); free(dbprev_head); free(dD_bh);
+    return 2;
+  }
+  bwd_job j = {d, X, logdecay, beta, gamma, B, C, theta, D, h0, angle0, xprev0, bprev0, dY, dhT,
+               dX, dlogdecay, dbeta, dgamma, dtheta, dh0, dangle0, dxprev0,
+               dB_head, dC_head, dbprev_head, dD_bh, 0, PTHREAD_MUTEX_INITIALIZER, 0};
+  if (nthreads < 1) nthreads = 1;
+  const int64_t npairs = Bt * H;
+  if (nthreads > npairs) nthreads = (int)(npairs > 0 ? npairs : 1);
+  pthread_t* th = malloc((size_t)nthreads * sizeof(pthread_t));
+  int started = 0;
+  if (th)
+    for (int k = 0; k < nthreads; ++k) {
+      if (pthread_create(&th[k], NULL, bwd_worker, &j) != 0) break;
+      ++started;
+    }
+  if (started == 0) bwd_worker(&j);
+  for (int k = 0; k < started; ++k) pthread_join(th[k], NULL);
+  free(th);
+  /* group sums over the heads h = g (H/G) .. (g+1) (H/G) - 1, in head order */
+  const int64_t hpg = H / G;
+  for (int64_t bt = 0; bt < Bt * L; ++bt)
+    for (int64_t gg = 0; gg < G; ++gg)
+      for (int64_t n = 0; n < N; ++n) {
+        double sb = 0.0, sc = 0.0;
+        for (int64_t k = 0; k < hpg; ++k) {
+          sb += dB_head[(bt * H + gg * hpg + k) * N + n];
+          sc += dC_head[(bt * H + gg * hpg + k) * N + n];
+        }
+        dB[(bt * G + gg) * N + n] = sb;
+        dC[(bt * G + gg) * N + n] = sc;
+      }
+  if (dbprev0)
+    for (int64_t b = 0; b < Bt; ++b)
+      for (int64_t gg = 0; gg < G; ++gg)
+        for (int64_t n = 0; n < N; ++n) {
+          double sb = 0.0;
+          for (int64_t k = 0; k < hpg; ++k) sb += dbprev_head[(b * H + gg * hpg + k) * N + n];
+          dbprev0[(b * G + gg) * N + n] = sb;
+        }
+  if (dD)
+    for (int64_t hh = 0; hh < H; ++hh) {
+      double s = 0.0;
+      for (int64_t b = 0; b < Bt; ++b) s += dD_bh[b * H + hh];
+      dD[hh] = s;
+    }
+  free(dB_head); free(dC_head); free(dbprev_head); free(dD_bh);
+  return j.status ? 2 : 0;
+}

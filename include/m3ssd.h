@@ -159,6 +159,59 @@ m3ssd_status m3ssd_step(const m3ssd_dims* dims, const void* x_t, const float* lo
                         const void* C_t, const float* theta_t, const float* D,
                         const m3ssd_cache* cache, void* y_t, void* stream);
 
+/* fp32 gradient outputs of m3ssd_bwd, each shaped like the matching input of
+ * m3ssd_fwd (dB, dC, dbprev0 per group; dD per head).  dX, dlogdecay, dgamma,
+ * dB, dC are required when b*L > 0; the others may be NULL (not written).  An
+ * input passed to the forward as NULL is read as zero, and its gradient is the
+ * derivative there. */
+typedef struct {
+  float* dX;         /* (b, L, H, P) */
+  float* dlogdecay;  /* (b, L, H) */
+  float* dbeta;      /* (b, L, H) */
+  float* dgamma;     /* (b, L, H) */
+  float* dB;         /* (b, L, G, N) */
+  float* dC;         /* (b, L, G, N) */
+  float* dtheta;     /* (b, L, H, N/2) */
+  float* dD;         /* (H) */
+  float* dh0;        /* (b, H, N, P) */
+  float* dangle0;    /* (b, H, N/2) */
+  float* dxprev0;    /* (b, H, P) */
+  float* dbprev0;    /* (b, G, N) */
+} m3ssd_bwd_grads;
+
+/* Bytes of device workspace m3ssd_bwd needs for these dims (0 for invalid
+ * dims).  It holds a state checkpoint every 64 tokens of every sequence, the
+ * states of one 64-token block per sequence, and per-head shares of the
+ * group-summed gradients: about 4 (b H ceil(L/64) (N P + N/2) + b H 65 N P +
+ * 2 b L H N) bytes. */
+size_t m3ssd_bwd_workspace_size(const m3ssd_dims* dims);
+
+/*
+ * Backward of m3ssd_fwd: reverse-mode derivatives of the recurrence of the
+ * "TorchMamba" README, "Math notes", M3 SISO.  Training through the scan is on
+ * the pages: "mamba-rs" crate page, feature list (CUDA forward and backward
+ * kernels); "TorchMamba" README, "Verification" (fp64 gradchecks per core).
+ *
+ * Takes the forward's inputs (same pointers, dtypes and NULL conventions;
+ * extra supplies angle0, xprev0, bprev0 and its outputs are ignored), the
+ * upstream gradients dY (b, L, H, P, dtype x_dtype) and dhT (b, H, N, P,
+ * fp32, NULL = 0), and writes the fp32 gradients in *grads.  The cache outputs
+ * angleT, xprevT and bprevT take no upstream gradient.
+ *
+ * The sequential backward recomputes the forward in fp32 from state
+ * checkpoints; group-shared gradients are summed over heads in a fixed
+ * order, so results are deterministic.  Limits as the sequential forward:
+ * N <= 256, P <= 256, N*P <= 16384 (else M3SSD_ERR_UNSUPPORTED).  workspace
+ * must hold m3ssd_bwd_workspace_size(dims) bytes, 256-byte aligned (else
+ * M3SSD_ERR_WORKSPACE).  No allocation, no synchronisation.
+ */
+m3ssd_status m3ssd_bwd(const m3ssd_dims* dims, const void* X, const float* logdecay,
+                       const float* beta, const float* gamma, const void* B, const void* C,
+                       const float* theta, const float* D, const float* h0,
+                       const m3ssd_fwd_extra* extra, const void* dY, const float* dhT,
+                       const m3ssd_bwd_grads* grads, void* workspace, size_t workspace_bytes,
+                       void* stream);
+
 /* Number of bounded device-side waits of the chunked forward that ran out
  * (each makes its CTA stop and leave its outputs unwritten) since the last
  * call; the count is then reset.  This call synchronises the current device

@@ -50,6 +50,14 @@ class FwdExtra(ctypes.Structure):
                 ("angle0", "xprev0", "bprev0", "angleT", "xprevT", "bprevT")]
 
 
+GRAD_NAMES = ("dX", "dlogdecay", "dbeta", "dgamma", "dB", "dC", "dtheta", "dD", "dh0",
+              "dangle0", "dxprev0", "dbprev0")
+
+
+class BwdGrads(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in GRAD_NAMES]
+
+
 class Cache(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in ("angle", "ssm", "x_prev", "b_prev")]
 
@@ -74,6 +82,11 @@ def load(path: str | None = None):
         lib.m3ssd_step.argtypes = [ctypes.POINTER(Dims)] + [vp] * 8 + \
             [ctypes.POINTER(Cache), vp, vp]
         lib.m3ssd_step.restype = ctypes.c_int
+        lib.m3ssd_bwd_workspace_size.argtypes = [ctypes.POINTER(Dims)]
+        lib.m3ssd_bwd_workspace_size.restype = sz
+        lib.m3ssd_bwd.argtypes = [ctypes.POINTER(Dims)] + [vp] * 9 + \
+            [ctypes.POINTER(FwdExtra), vp, vp, ctypes.POINTER(BwdGrads), vp, sz, vp]
+        lib.m3ssd_bwd.restype = ctypes.c_int
         lib.m3ssd_status_string.argtypes = [ctypes.c_int]
         lib.m3ssd_status_string.restype = ctypes.c_char_p
         lib.m3ssd_abi_version.argtypes = []
@@ -200,6 +213,66 @@ def fwd(X, logdecay, beta, gamma, B, C, theta=None, D=None, h0=None, *, Y=None,
                           _stream_handle(dev))
     _check(st, "m3ssd_fwd")
     return Y, hT, cache_out
+
+
+def bwd_workspace_size(dims: Dims) -> int:
+    return int(load().m3ssd_bwd_workspace_size(ctypes.byref(dims)))
+
+
+def bwd(X, logdecay, beta, gamma, B, C, theta=None, D=None, h0=None, *, dY, dhT=None,
+        angle0=None, xprev0=None, bprev0=None, grads=None, workspace=None):
+    """Backward of :func:`fwd` through ``m3ssd_bwd`` on the current CUDA stream.
+
+    Takes the forward's inputs and the upstream gradients ``dY`` (dtype of X)
+    and ``dhT`` (fp32 or None).  Returns a dict of fp32 gradients named as in
+    ``GRAD_NAMES``, each shaped like its input (allocated by torch unless
+    ``grads`` supplies them).
+    """
+    import torch
+    b, L, H, P = X.shape
+    G, N = B.shape[2], B.shape[3]
+    dev = X.device
+    f32 = torch.float32
+    xd = X.dtype
+    _need(X, "X", device=dev)
+    _need(logdecay, "logdecay", f32, (b, L, H), dev)
+    _need(beta, "beta", f32, (b, L, H), dev)
+    _need(gamma, "gamma", f32, (b, L, H), dev)
+    _need(B, "B", xd, (b, L, G, N), dev)
+    _need(C, "C", xd, (b, L, G, N), dev)
+    _need(theta, "theta", f32, (b, L, H, N // 2), dev)
+    _need(D, "D", f32, (H,), dev)
+    _need(h0, "h0", f32, (b, H, N, P), dev)
+    _need(angle0, "angle0", f32, (b, H, N // 2), dev)
+    _need(xprev0, "xprev0", f32, (b, H, P), dev)
+    _need(bprev0, "bprev0", f32, (b, G, N), dev)
+    _need(dY, "dY", xd, (b, L, H, P), dev)
+    _need(dhT, "dhT", f32, (b, H, N, P), dev)
+    shapes = {"dX": (b, L, H, P), "dlogdecay": (b, L, H), "dbeta": (b, L, H),
+              "dgamma": (b, L, H), "dB": (b, L, G, N), "dC": (b, L, G, N),
+              "dtheta": (b, L, H, N // 2), "dD": (H,), "dh0": (b, H, N, P),
+              "dangle0": (b, H, N // 2), "dxprev0": (b, H, P), "dbprev0": (b, G, N)}
+    if grads is None:
+        grads = {k: torch.empty(v, dtype=f32, device=dev) for k, v in shapes.items()}
+    for k in GRAD_NAMES:
+        _need(grads.get(k), k, f32, shapes[k], dev)
+    gs = BwdGrads(*(None if grads.get(k) is None else grads[k].data_ptr() for k in GRAD_NAMES))
+    extra = None
+    if angle0 is not None or xprev0 is not None or bprev0 is not None:
+        extra = FwdExtra(*(None if t is None else t.data_ptr() for t in (angle0, xprev0, bprev0)),
+                         None, None, None)
+    dims = make_dims(b, L, H, P, N, G, _xdtype(X), 0)
+    ws_bytes = bwd_workspace_size(dims)
+    if ws_bytes and workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    st = load().m3ssd_bwd(ctypes.byref(dims), _ptr(X), _ptr(logdecay), _ptr(beta), _ptr(gamma),
+                          _ptr(B), _ptr(C), _ptr(theta), _ptr(D), _ptr(h0),
+                          None if extra is None else ctypes.byref(extra), _ptr(dY), _ptr(dhT),
+                          ctypes.byref(gs), _ptr(workspace),
+                          0 if workspace is None else workspace.numel() * workspace.element_size(),
+                          _stream_handle(dev))
+    _check(st, "m3ssd_bwd")
+    return grads
 
 
 def new_cache(batch, nheads, headdim, dstate, ngroups, device):

@@ -48,6 +48,35 @@ struct StepArgs {
   void* y_t;
 };
 
+// Everything one backward launch needs (gradients are fp32; the nullable
+// outputs are not written when absent).
+struct BwdArgs {
+  int64_t b, L, H, P, N, G;
+  bool bf16;  // X, B, C, dY are bf16 (else fp32)
+  const void* X;
+  const float* logdecay;
+  const float* beta;    // nullable
+  const float* gamma;
+  const void* B;
+  const void* C;
+  const float* theta;   // nullable
+  const float* D;       // nullable
+  const float* h0;      // nullable
+  const float* angle0;  // nullable
+  const float* xprev0;  // nullable
+  const float* bprev0;  // nullable
+  const void* dY;
+  const float* dhT;     // nullable
+  float *dX, *dlogdecay, *dbeta, *dgamma, *dB, *dC, *dtheta, *dD, *dh0, *dangle0, *dxprev0,
+      *dbprev0;
+  void* workspace;      // bwd_workspace_bytes(...) bytes, 256-byte aligned
+};
+
+// Workspace of the sequential backward: state checkpoints, the states of one
+// block per sequence, and per-head shares of the group-summed gradients.
+size_t bwd_workspace_bytes(int64_t b, int64_t L, int64_t H, int64_t P, int64_t N);
+cudaError_t launch_bwd_seq(const BwdArgs& a, cudaStream_t s);
+
 // Sequential fp32 forward: one CTA per (b, h), token by token.
 cudaError_t launch_fwd_seq(const FwdArgs& a, cudaStream_t s);
 // Chunked bf16 tensor-core forward (N = 128, P = 64).

@@ -118,6 +118,57 @@ m3ssd_status m3ssd_fwd(const m3ssd_dims* dims, const void* X, const float* logde
   return from_cuda(chunked ? m3ssd::launch_fwd_chunk(a, s) : m3ssd::launch_fwd_seq(a, s));
 }
 
+size_t m3ssd_bwd_workspace_size(const m3ssd_dims* dims) {
+  if (check_dims(dims) != M3SSD_OK || !general_shape_ok(dims)) return 0;
+  return m3ssd::bwd_workspace_bytes(dims->batch, dims->seqlen, dims->nheads, dims->headdim,
+                                    dims->dstate);
+}
+
+m3ssd_status m3ssd_bwd(const m3ssd_dims* dims, const void* X, const float* logdecay,
+                       const float* beta, const float* gamma, const void* B, const void* C,
+                       const float* theta, const float* D, const float* h0,
+                       const m3ssd_fwd_extra* extra, const void* dY, const float* dhT,
+                       const m3ssd_bwd_grads* grads, void* workspace, size_t workspace_bytes,
+                       void* stream) {
+  m3ssd_status st = check_dims(dims);
+  if (st != M3SSD_OK) return st;
+  if (!general_shape_ok(dims)) return M3SSD_ERR_UNSUPPORTED;
+  if (!grads) return M3SSD_ERR_INVALID_ARG;
+  const bool bf16 = dims->x_dtype == M3SSD_BF16;
+  const uintptr_t esz = bf16 ? 2 : 4;
+  if (dims->batch * dims->seqlen > 0 &&
+      (!X || !logdecay || !gamma || !B || !C || !dY || !grads->dX || !grads->dlogdecay ||
+       !grads->dgamma || !grads->dB || !grads->dC))
+    return M3SSD_ERR_INVALID_ARG;
+  if (!aligned(X, esz) || !aligned(B, esz) || !aligned(C, esz) || !aligned(dY, esz))
+    return M3SSD_ERR_INVALID_ARG;
+  const void* f32ptrs[] = {logdecay, beta, gamma, theta, D, h0, dhT, grads->dX, grads->dlogdecay,
+                           grads->dbeta, grads->dgamma, grads->dB, grads->dC, grads->dtheta,
+                           grads->dD, grads->dh0, grads->dangle0, grads->dxprev0, grads->dbprev0};
+  for (const void* p : f32ptrs)
+    if (!aligned(p, 4)) return M3SSD_ERR_INVALID_ARG;
+  m3ssd::BwdArgs a{};
+  if (extra) {
+    const void* eptrs[] = {extra->angle0, extra->xprev0, extra->bprev0};
+    for (const void* p : eptrs)
+      if (!aligned(p, 4)) return M3SSD_ERR_INVALID_ARG;
+    a.angle0 = extra->angle0; a.xprev0 = extra->xprev0; a.bprev0 = extra->bprev0;
+  }
+  const size_t need = m3ssd_bwd_workspace_size(dims);
+  if (workspace_bytes < need || (need > 0 && (!workspace || !aligned(workspace, 256))))
+    return M3SSD_ERR_WORKSPACE;
+  if (dims->batch == 0) return M3SSD_OK;
+  a.b = dims->batch; a.L = dims->seqlen; a.H = dims->nheads; a.P = dims->headdim;
+  a.N = dims->dstate; a.G = dims->ngroups; a.bf16 = bf16;
+  a.X = X; a.logdecay = logdecay; a.beta = beta; a.gamma = gamma; a.B = B; a.C = C;
+  a.theta = theta; a.D = D; a.h0 = h0; a.dY = dY; a.dhT = dhT;
+  a.dX = grads->dX; a.dlogdecay = grads->dlogdecay; a.dbeta = grads->dbeta;
+  a.dgamma = grads->dgamma; a.dB = grads->dB; a.dC = grads->dC; a.dtheta = grads->dtheta;
+  a.dD = grads->dD; a.dh0 = grads->dh0; a.dangle0 = grads->dangle0; a.dxprev0 = grads->dxprev0;
+  a.dbprev0 = grads->dbprev0; a.workspace = workspace;
+  return from_cuda(m3ssd::launch_bwd_seq(a, static_cast<cudaStream_t>(stream)));
+}
+
 m3ssd_status m3ssd_step(const m3ssd_dims* dims, const void* x_t, const float* logdecay_t,
                         const float* beta_t, const float* gamma_t, const void* B_t,
                         const void* C_t, const float* theta_t, const float* D,

@@ -128,6 +128,33 @@ def test_step_validation(lib):
     assert _step(lib, _dims(batch=0), x=None, y=None) == m3.OK
 
 
+def _bwd(lib, dims, grads=None, X=FAKE, dY=FAKE, ws=None, ws_bytes=0):
+    g = grads if grads is not None else m3.BwdGrads(*([0x10000] * 6 + [None] * 6))
+    return lib.m3ssd_bwd(ctypes.byref(dims), X, FAKE, None, FAKE, FAKE, FAKE, None, None, None,
+                         None, dY, None, ctypes.byref(g), ws, ws_bytes, None)
+
+
+def test_bwd_validation(lib):
+    d = _dims()
+    need = lib.m3ssd_bwd_workspace_size(ctypes.byref(d))
+    assert need > 0 and lib.m3ssd_bwd_workspace_size(None) == 0
+    assert need == lib.m3ssd_bwd_workspace_size(ctypes.byref(_dims()))
+    assert lib.m3ssd_bwd_workspace_size(ctypes.byref(_dims(seqlen=200))) > need
+    assert _bwd(lib, d) == m3.ERR_WORKSPACE                              # no workspace
+    assert _bwd(lib, d, ws=FAKE, ws_bytes=need - 1) == m3.ERR_WORKSPACE  # too small
+    assert _bwd(lib, d, ws=ctypes.c_void_p(0x10010), ws_bytes=need) == m3.ERR_WORKSPACE
+    assert _bwd(lib, d, dY=None) == m3.ERR_INVALID_ARG
+    assert _bwd(lib, d, X=ctypes.c_void_p(0x10002)) == m3.ERR_INVALID_ARG
+    for k in ("dX", "dlogdecay", "dgamma", "dB", "dC"):
+        g = m3.BwdGrads(*([0x10000] * 6 + [None] * 6))
+        setattr(g, k, None)
+        assert _bwd(lib, d, grads=g) == m3.ERR_INVALID_ARG, k
+    assert lib.m3ssd_bwd(ctypes.byref(d), FAKE, FAKE, None, FAKE, FAKE, FAKE, None, None, None,
+                         None, FAKE, None, None, None, 0, None) == m3.ERR_INVALID_ARG
+    assert _bwd(lib, _dims(dstate=512)) == m3.ERR_UNSUPPORTED
+    assert _bwd(lib, _dims(batch=0), X=None, dY=None, ws=FAKE, ws_bytes=1 << 20) == m3.OK
+
+
 def test_wait_timeout_query_rejects_null(lib):
     assert lib.m3ssd_device_wait_timeouts(None) == m3.ERR_INVALID_ARG
 

@@ -1,0 +1,108 @@
+"""GPU backward through the C ABI (m3ssd_bwd) against the fp64 oracle's backward.
+
+Every gradient output is compared element by element with oracle.oracle_bwd on
+the same inputs (bf16 inputs are rounded before either side sees them).  The
+bar is max |err| / RMS(reference) <= 2e-4: the backward recomputes the forward
+and sweeps it back in fp32.  Recurrence, rotations and per-column reductions
+each carry an error of order 1e-6 of a gradient's scale.  Over a few hundred
+tokens that stays within a few 1e-5, so the bar is about ten times the
+observed error.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import selective_state_space_m3ssd_b200 as m3
+from selective_state_space_m3ssd_b200.synth import WORKLOADS, make_inputs
+from tests.gpu_util import np64, rel_max_err, to_dev
+from tests.test_gpu_seq_step import with_cache_inputs
+
+pytestmark = pytest.mark.gpu
+
+TOL = 2e-4
+SMALL = WORKLOADS["tiny"].with_(batch=2, nheads=4, ngroups=2, headdim=16, dstate=16, seed=77)
+ARGS = ("X", "logdecay", "beta", "gamma", "B", "C", "theta", "D", "h0")
+
+
+def upstream(inp, seed, with_dhT=True):
+    g = torch.Generator().manual_seed(seed)
+    b, L, H, P = inp["X"].shape
+    N = inp["B"].shape[3]
+    dY = torch.randn(b, L, H, P, generator=g).to(inp["X"].dtype)
+    dhT = torch.randn(b, H, N, P, generator=g) if with_dhT else None
+    return dY, dhT
+
+
+def run_both(inp, dY, dhT):
+    ref = oracle.oracle_bwd(**inp, dY=dY, dhT=dhT)
+    d = to_dev(inp)
+    got = m3.bwd(*(d.get(k) for k in ARGS), dY=dY.cuda(), dhT=None if dhT is None else dhT.cuda(),
+                 angle0=d.get("angle0"), xprev0=d.get("xprev0"), bprev0=d.get("bprev0"))
+    torch.cuda.synchronize()
+    return {k: np64(v) for k, v in got.items()}, ref
+
+
+def check_all(got, ref, tol=TOL, skip=()):
+    for k, r in ref.items():
+        if k in skip:
+            continue
+        if not np.any(r):
+            assert np.max(np.abs(got[k])) == 0.0, k
+            continue
+        assert rel_max_err(got[k], r) <= tol, (k, rel_max_err(got[k], r))
+
+
+@pytest.mark.parametrize("L", [1, 17, 64, 65, 130])
+def test_bwd_fp32_lengths(L):
+    inp = with_cache_inputs(make_inputs(SMALL.with_(seqlen=L)), seed=L)
+    dY, dhT = upstream(inp, 10 + L)
+    got, ref = run_both(inp, dY, dhT)
+    check_all(got, ref)
+
+
+@pytest.mark.parametrize("variant", ["no_beta", "no_theta", "no_cache", "no_dhT", "one_group"])
+def test_bwd_fp32_paths(variant):
+    w = SMALL.with_(seqlen=70)
+    if variant == "no_beta":
+        w = w.with_(has_beta=False)
+    if variant == "no_theta":
+        w = w.with_(has_theta=False)
+    if variant == "one_group":
+        w = w.with_(ngroups=1)
+    inp = make_inputs(w)
+    if variant != "no_cache":
+        inp = with_cache_inputs(inp, seed=3)
+    dY, dhT = upstream(inp, 5, with_dhT=variant != "no_dhT")
+    got, ref = run_both(inp, dY, dhT)
+    check_all(got, ref)
+
+
+def test_bwd_bf16_siso_shape():
+    # the shape of the chunked forward (N = 128, P = 64) with bf16 X, B, C, dY
+    w = WORKLOADS["siso"].with_(batch=1, nheads=2, seqlen=100, seed=88)
+    inp = with_cache_inputs(make_inputs(w), seed=9)
+    dY, dhT = upstream(inp, 11)
+    got, ref = run_both(inp, dY, dhT)
+    check_all(got, ref)
+
+
+def test_bwd_is_deterministic():
+    inp = make_inputs(SMALL.with_(seqlen=90))
+    dY, dhT = upstream(inp, 21)
+    d = to_dev(inp)
+    args = [d.get(k) for k in ARGS]
+    g1 = m3.bwd(*args, dY=dY.cuda(), dhT=dhT.cuda())
+    g2 = m3.bwd(*args, dY=dY.cuda(), dhT=dhT.cuda())
+    torch.cuda.synchronize()
+    for k in g1:
+        assert torch.equal(g1[k], g2[k]), k
+
+
+def test_bwd_rejects_small_workspace():
+    inp = make_inputs(SMALL.with_(seqlen=20))
+    dY, _ = upstream(inp, 1)
+    d = to_dev(inp)
+    with pytest.raises(m3.M3SSDError):
+        m3.bwd(*(d.get(k) for k in ARGS), dY=dY.cuda(),
+               workspace=torch.empty(256, dtype=torch.uint8, device="cuda"))

@@ -212,6 +212,21 @@ m3ssd_status m3ssd_bwd(const m3ssd_dims* dims, const void* X, const float* logde
                        const m3ssd_bwd_grads* grads, void* workspace, size_t workspace_bytes,
                        void* stream);
 
+/*
+ * m3ssd_bwd without a caller workspace: the scratch is a fixed 64 MiB device
+ * array inside the library, reserved when its device code is loaded.  The
+ * pages have no counterpart for this entry point; it is a convenience of this
+ * library.  Arguments and results are those of m3ssd_bwd.  Requests whose
+ * m3ssd_bwd_workspace_size exceeds 64 MiB return M3SSD_ERR_UNSUPPORTED before
+ * any device call.  Every call uses the same array, so calls must not overlap
+ * (issue them on one stream, or synchronise between streams).
+ */
+m3ssd_status m3ssd_bwd_noalloc(const m3ssd_dims* dims, const void* X, const float* logdecay,
+                               const float* beta, const float* gamma, const void* B,
+                               const void* C, const float* theta, const float* D,
+                               const float* h0, const m3ssd_fwd_extra* extra, const void* dY,
+                               const float* dhT, const m3ssd_bwd_grads* grads, void* stream);
+
 /* Number of bounded device-side waits of the chunked forward that ran out
  * (each makes its CTA stop and leave its outputs unwritten) since the last
  * call; the count is then reset.  This call synchronises the current device

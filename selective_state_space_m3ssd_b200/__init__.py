@@ -87,6 +87,9 @@ def load(path: str | None = None):
         lib.m3ssd_bwd.argtypes = [ctypes.POINTER(Dims)] + [vp] * 9 + \
             [ctypes.POINTER(FwdExtra), vp, vp, ctypes.POINTER(BwdGrads), vp, sz, vp]
         lib.m3ssd_bwd.restype = ctypes.c_int
+        lib.m3ssd_bwd_noalloc.argtypes = [ctypes.POINTER(Dims)] + [vp] * 9 + \
+            [ctypes.POINTER(FwdExtra), vp, vp, ctypes.POINTER(BwdGrads), vp]
+        lib.m3ssd_bwd_noalloc.restype = ctypes.c_int
         lib.m3ssd_status_string.argtypes = [ctypes.c_int]
         lib.m3ssd_status_string.restype = ctypes.c_char_p
         lib.m3ssd_abi_version.argtypes = []
@@ -272,6 +275,40 @@ def bwd(X, logdecay, beta, gamma, B, C, theta=None, D=None, h0=None, *, dY, dhT=
                           0 if workspace is None else workspace.numel() * workspace.element_size(),
                           _stream_handle(dev))
     _check(st, "m3ssd_bwd")
+    return grads
+
+
+def bwd_noalloc(X, logdecay, beta, gamma, B, C, theta=None, D=None, h0=None, *, dY,
+                dhT=None, angle0=None, xprev0=None, bprev0=None, grads=None):
+    """:func:`bwd` through ``m3ssd_bwd_noalloc`` (scratch inside the library;
+    calls must not overlap).  Returns the same dict of fp32 gradients."""
+    import torch
+    b, L, H, P = X.shape
+    G, N = B.shape[2], B.shape[3]
+    dev = X.device
+    f32 = torch.float32
+    shapes = {"dX": (b, L, H, P), "dlogdecay": (b, L, H), "dbeta": (b, L, H),
+              "dgamma": (b, L, H), "dB": (b, L, G, N), "dC": (b, L, G, N),
+              "dtheta": (b, L, H, N // 2), "dD": (H,), "dh0": (b, H, N, P),
+              "dangle0": (b, H, N // 2), "dxprev0": (b, H, P), "dbprev0": (b, G, N)}
+    for name, t, dt in (("X", X, None), ("dY", dY, X.dtype), ("B", B, X.dtype),
+                        ("C", C, X.dtype), ("dhT", dhT, f32)):
+        _need(t, name, dt, device=dev)
+    if grads is None:
+        grads = {k: torch.empty(v, dtype=f32, device=dev) for k, v in shapes.items()}
+    for k in GRAD_NAMES:
+        _need(grads.get(k), k, f32, shapes[k], dev)
+    gs = BwdGrads(*(None if grads.get(k) is None else grads[k].data_ptr() for k in GRAD_NAMES))
+    extra = None
+    if angle0 is not None or xprev0 is not None or bprev0 is not None:
+        extra = FwdExtra(*(None if t is None else t.data_ptr() for t in (angle0, xprev0, bprev0)),
+                         None, None, None)
+    dims = make_dims(b, L, H, P, N, G, _xdtype(X), 0)
+    st = load().m3ssd_bwd_noalloc(ctypes.byref(dims), _ptr(X), _ptr(logdecay), _ptr(beta),
+                                  _ptr(gamma), _ptr(B), _ptr(C), _ptr(theta), _ptr(D), _ptr(h0),
+                                  None if extra is None else ctypes.byref(extra), _ptr(dY),
+                                  _ptr(dhT), ctypes.byref(gs), _stream_handle(dev))
+    _check(st, "m3ssd_bwd_noalloc")
     return grads
 
 

@@ -347,6 +347,42 @@ def bench_decode(dev, rank, steps_graph_replays: int, peaks: dict):
             "gpu_launches": 2 * nsteps}
 
 
+def bench_backward(w, dev, steps, world, d, peaks):
+    """The backward (m3ssd_bwd) on the forward's workload: dY, dhT synthetic,
+    every gradient output written; inputs resident in HBM."""
+    import selective_state_space_m3ssd_b200 as m3
+    gen = torch.Generator().manual_seed(7)
+    dY = torch.randn(tuple(d["X"].shape), generator=gen).to(d["X"].dtype).to(dev)
+    dhT = torch.randn(w.batch, w.nheads, w.dstate, w.headdim, generator=gen).to(dev)
+    args = [d[k] for k in ("X", "logdecay", "beta", "gamma", "B", "C", "theta", "D", "h0")]
+    dims = m3.make_dims(w.batch, w.seqlen, w.nheads, w.headdim, w.dstate, w.ngroups,
+                        m3.BF16 if d["X"].dtype == torch.bfloat16 else m3.F32, 0)
+    ws = torch.empty(m3.bwd_workspace_size(dims), dtype=torch.uint8, device=dev)
+    grads = m3.bwd(*args, dY=dY, dhT=dhT, workspace=ws)  # warm-up, allocates the outputs
+    torch.cuda.synchronize(dev)
+    stream = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        m3.bwd(*args, dY=dY, dhT=dhT, grads=grads, workspace=ws)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / steps
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    algo = nbytes(*args, dY, dhT, *grads.values())
+    achieved = algo / (ms / 1e3) / 1e9
+    return {"metric": "bwd Mtokens/s", "value": w.batch * w.seqlen * world / (ms / 1e3) / 1e6,
+            "unit": "Mtokens/s", "ms_per_step": ms, "steps": steps,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                         "algo_bytes_per_step": algo, "traffic": None,
+                         "peak_source": peaks["source"]},
+            "kernel": "bwd_seq_kernel + bwd_reduce_kernel (sequential fp32, 2 launches)"}
+
+
 def run_ours(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -373,6 +409,8 @@ def run_ours(args):
                       if hasattr(torch.cuda.get_device_properties(dev), "index") else local) as clk:
         fw = bench_forward(w, dev, args.steps, args.warmup, world, rank)
         dec = bench_decode(dev, rank, max(1, args.decode_replays), peaks)
+        bwd = None if args.no_backward else bench_backward(
+            w, dev, max(1, min(args.steps, 3)), world, fw["dev_inputs"], peaks)
     e2e = bench_e2e(w, dev, max(1, min(args.steps, 5)), 1, fw["inp"], world)
 
     tokens = w.batch * w.seqlen * args.steps * world
@@ -392,6 +430,7 @@ def run_ours(args):
         "e2e": e2e,
         "gpu_launches": fw["launches"],
         "decode": dec,
+        "backward": bwd,
         "clocks": clk.summary(),
     }
     if world > 1:
@@ -449,6 +488,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--decode-replays", type=int, default=3,
                     help="replays of the 1000-step decode graph in the timed region")
+    ap.add_argument("--no-backward", action="store_true",
+                    help="skip the backward measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="omit the oracle timing (it never runs inside a GPU timed region)")
     args = ap.parse_args()

@@ -363,7 +363,6 @@ __global__ void __launch_bounds__(kThreads, 2)
         chunk_params(sm.prm[(c + 1) & 1], pld, pbe, pga, lane);
         if (c + 2 < nC) load_params(c + 2);
       }
-      __syncthreads();  // S2
       __syncthreads();  // S3: Cbar, Bbar, W_end o Bbar ready
       if (ctrl_lead) {
         tc5::fence_after_sync();
@@ -442,7 +441,9 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
       *reinterpret_cast<float2*>(&sm.segtot[warp][2 * lane]) = run;
     }
-    __syncthreads();  // S2: segment totals ready; theta no longer read
+    // S2 (compute warps only, so that the control warp's scalars for the next chunk
+    // overlap phases R1 and R2): segment totals ready; theta no longer read
+    asm volatile("bar.sync 1, %0;" ::"n"(32 * kCtrlWarp) : "memory");
 
     // -- phase R2: rotation into the absolute frame, W_end o Bbar hi/lo ----------
     // The absolute angle of row r is Phi_c + psi_r with Phi_c kept in [-pi, pi];

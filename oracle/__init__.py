@@ -36,6 +36,11 @@ class _Dims(ctypes.Structure):
                 ("batch", "seqlen", "nheads", "headdim", "dstate", "ngroups")]
 
 
+class _MimoDims(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int64) for n in
+                ("batch", "seqlen", "nheads", "headdim", "dstate", "ngroups", "rank")]
+
+
 def build(force: bool = False) -> str:
     """Compile ``liboracle.so`` with gcc (plain -O2, IEEE semantics, no fast-math)."""
     stale = (not os.path.exists(_LIB_PATH)
@@ -58,6 +63,10 @@ def _bind(path: str):
     lib.oracle_step.restype = ctypes.c_int
     lib.oracle_bwd.argtypes = [ctypes.POINTER(_Dims)] + [dp] * 26 + [ctypes.c_int]
     lib.oracle_bwd.restype = ctypes.c_int
+    lib.oracle_mimo_fwd.argtypes = [ctypes.POINTER(_MimoDims)] + [dp] * 17 + [ctypes.c_int]
+    lib.oracle_mimo_fwd.restype = ctypes.c_int
+    lib.oracle_mimo_step.argtypes = [ctypes.POINTER(_MimoDims)] + [dp] * 13
+    lib.oracle_mimo_step.restype = ctypes.c_int
     return lib
 
 
@@ -238,6 +247,60 @@ def oracle_step(cache, x_t, logdecay_t, beta_t, gamma_t, B_t, C_t, theta_t=None,
                              _ptr(cache["b_prev"]), _ptr(y))
     if rc != 0:
         raise RuntimeError(f"oracle_step failed with code {rc}")
+    return y
+
+
+def oracle_mimo_fwd(X, logdecay, beta, gamma, B, C, theta=None, D=None, h0=None,
+                    angle0=None, xprev0=None, bprev0=None, nthreads: int | None = None):
+    """Sequential fp64 MIMO forward.
+
+    Shapes: X (b,L,H,P,R); logdecay, beta, gamma (b,L,H); B, C (b,L,G,N,R);
+    theta (b,L,H,N/2); D (H); h0 (b,H,N,P); angle0 (b,H,N/2);
+    xprev0 (b,H,P,R); bprev0 (b,G,N,R).  Returns Y, hT, angleT, xprevT, bprevT.
+    """
+    X, logdecay, beta, gamma = _f64(X), _f64(logdecay), _f64(beta), _f64(gamma)
+    B, C, theta, D, h0 = _f64(B), _f64(C), _f64(theta), _f64(D), _f64(h0)
+    angle0, xprev0, bprev0 = _f64(angle0), _f64(xprev0), _f64(bprev0)
+    b, L, H, P, R = X.shape
+    G, N = B.shape[2], B.shape[3]
+    if N % 2 or H % G or B.shape != (b, L, G, N, R) or C.shape != (b, L, G, N, R):
+        raise ValueError("oracle_mimo_fwd: shapes")
+    d = _MimoDims(b, L, H, P, N, G, R)
+    Y = np.zeros((b, L, H, P, R))
+    hT = np.zeros((b, H, N, P)) if h0 is None else h0.copy()
+    angleT = np.zeros((b, H, N // 2)) if angle0 is None else angle0.copy()
+    xprevT = np.zeros((b, H, P, R)) if xprev0 is None else xprev0.copy()
+    bprevT = np.zeros((b, G, N, R)) if bprev0 is None else bprev0.copy()
+    rc = _load().oracle_mimo_fwd(ctypes.byref(d), _ptr(X), _ptr(logdecay), _ptr(beta),
+                                 _ptr(gamma), _ptr(B), _ptr(C), _ptr(theta), _ptr(D), _ptr(h0),
+                                 _ptr(angle0), _ptr(xprev0), _ptr(bprev0), _ptr(Y), _ptr(hT),
+                                 _ptr(angleT), _ptr(xprevT), _ptr(bprevT),
+                                 int(nthreads or default_threads()))
+    if rc != 0:
+        raise RuntimeError(f"oracle_mimo_fwd failed with code {rc}")
+    return {"Y": Y, "hT": hT, "angleT": angleT, "xprevT": xprevT, "bprevT": bprevT}
+
+
+def oracle_mimo_step(cache, x_t, logdecay_t, beta_t, gamma_t, B_t, C_t, theta_t=None, D=None):
+    """One MIMO decode step; ``cache`` holds float64 arrays angle (b,H,N/2),
+    ssm (b,H,N,P), x_prev (b,H,P,R), b_prev (b,G,N,R), updated in place.
+    Returns y_t (b,H,P,R)."""
+    x_t, logdecay_t, beta_t, gamma_t = _f64(x_t), _f64(logdecay_t), _f64(beta_t), _f64(gamma_t)
+    B_t, C_t, theta_t, D = _f64(B_t), _f64(C_t), _f64(theta_t), _f64(D)
+    for k in ("angle", "ssm", "x_prev", "b_prev"):
+        a = cache[k]
+        if not (isinstance(a, np.ndarray) and a.dtype == np.float64 and a.flags.c_contiguous):
+            raise ValueError(f"oracle_mimo_step: cache[{k!r}] must be a C-contiguous float64 ndarray")
+    b, H, P, R = x_t.shape
+    G, N = B_t.shape[1], B_t.shape[2]
+    d = _MimoDims(b, 1, H, P, N, G, R)
+    y = np.zeros((b, H, P, R))
+    rc = _load().oracle_mimo_step(ctypes.byref(d), _ptr(x_t), _ptr(logdecay_t), _ptr(beta_t),
+                                  _ptr(gamma_t), _ptr(B_t), _ptr(C_t), _ptr(theta_t), _ptr(D),
+                                  _ptr(cache["angle"]), _ptr(cache["ssm"]), _ptr(cache["x_prev"]),
+                                  _ptr(cache["b_prev"]), _ptr(y))
+    if rc != 0:
+        raise RuntimeError(f"oracle_mimo_step failed with code {rc}")
     return y
 
 

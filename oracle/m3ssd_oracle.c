@@ -541,3 +541,201 @@ int oracle_bwd(const oracle_dims* d, const double* X, const double* logdecay, co
   free(dB_head); free(dC_head); free(dbprev_head); free(dD_bh);
   return j.status ? 2 : 0;
 }
+
+/* ---------------------------------------------------------------------------
+ * MIMO rank R ("TorchMamba" README, table "Models", row Mamba-3 MIMO: a rank-R
+ * matmul update on a shared (N, P) state; "Functional cores": mimo_loop with
+ * X (B,L,H,P,R) -> Y (B,L,H,P,R), h (B,H,N,P); "Math notes", MIMO: the B x^T
+ * outer product becomes a matmul).  Reading: B and C carry the rank axis as
+ * (b,L,G,N,R); every rank column is rotated by the same angle; the update is
+ *     h_t = a_t h_{t-1} + beta_t sum_r Bbar_{t-1,r} x_{t-1,r}^T + gamma_t sum_r Bbar_{t,r} x_{t,r}^T
+ *     y_{t,r} = Cbar_{t,r}^T h_t + D_h x_{t,r}
+ * and the cache holds x_prev (b,H,P,R) and b_prev (b,G,N,R).  At R = 1 this is
+ * the SISO recurrence above.
+ * --------------------------------------------------------------------------- */
+typedef struct {
+  int64_t batch, seqlen, nheads, headdim, dstate, ngroups, rank;
+} oracle_mimo_dims;
+
+/* column r of an (N, R) matrix rotated pairwise: out[(2i) R + r], out[(2i+1) R + r] */
+static void rotate_pairs_col(const double* v, const double* phi, int64_t n, int64_t R,
+                             double* out) {
+  for (int64_t i = 0; i < n / 2; ++i) {
+    const double c = cos(phi[i]);
+    const double s = sin(phi[i]);
+    for (int64_t r = 0; r < R; ++r) {
+      const double re = v[(2 * i) * R + r];
+      const double im = v[(2 * i + 1) * R + r];
+      out[(2 * i) * R + r] = c * re - s * im;
+      out[(2 * i + 1) * R + r] = s * re + c * im;
+    }
+  }
+}
+
+typedef struct {
+  const oracle_mimo_dims* d;
+  const double *X, *logdecay, *beta, *gamma, *B, *C, *theta, *D, *h0;
+  const double *angle0, *xprev0, *bprev0;
+  double *Y, *hT, *angleT, *xprevT, *bprevT;
+  int64_t next_pair;
+  pthread_mutex_t mu;
+  int status;
+} mimo_job;
+
+/* one MIMO token: S, phi and the previous-token buffers updated in place */
+static void mimo_token(const oracle_mimo_dims* d, int64_t h, const double* x, const double* B,
+                       const double* C, const double* theta_t, double logdecay, double be,
+                       double ga, const double* D, double* phi, double* phi_prev, double* S,
+                       double* xp, double* Bp, double* Bbar, double* Cbar, double* Bpbar,
+                       double* y) {
+  const int64_t P = d->headdim, N = d->dstate, R = d->rank, NH = N / 2;
+  if (theta_t)
+    for (int64_t i = 0; i < NH; ++i) phi[i] += theta_t[i];
+  rotate_pairs_col(B, phi, N, R, Bbar);
+  rotate_pairs_col(C, phi, N, R, Cbar);
+  rotate_pairs_col(Bp, phi_prev, N, R, Bpbar);
+  const double alpha = exp(logdecay);
+  for (int64_t n = 0; n < N; ++n)
+    for (int64_t p = 0; p < P; ++p) {
+      double ub = 0.0, ug = 0.0;
+      for (int64_t r = 0; r < R; ++r) {
+        ub += Bpbar[n * R + r] * xp[p * R + r];
+        ug += Bbar[n * R + r] * x[p * R + r];
+      }
+      S[n * P + p] = alpha * S[n * P + p] + be * ub + ga * ug;
+    }
+  const double dh = D ? D[h] : 0.0;
+  for (int64_t p = 0; p < P; ++p)
+    for (int64_t r = 0; r < R; ++r) {
+      double acc = 0.0;
+      for (int64_t n = 0; n < N; ++n) acc += Cbar[n * R + r] * S[n * P + p];
+      y[p * R + r] = acc + dh * x[p * R + r];
+    }
+  memcpy(xp, x, (size_t)(P * R) * sizeof(double));
+  memcpy(Bp, B, (size_t)(N * R) * sizeof(double));
+  memcpy(phi_prev, phi, (size_t)NH * sizeof(double));
+}
+
+static int mimo_one(mimo_job* j, int64_t b, int64_t h) {
+  const oracle_mimo_dims* d = j->d;
+  const int64_t L = d->seqlen, H = d->nheads, P = d->headdim, N = d->dstate, G = d->ngroups;
+  const int64_t R = d->rank, g = h / (H / G), NH = N / 2, bh = b * H + h;
+  double* phi = calloc((size_t)NH, sizeof(double));
+  double* phi_prev = calloc((size_t)NH, sizeof(double));
+  double* S = calloc((size_t)(N * P), sizeof(double));
+  double* xp = calloc((size_t)(P * R), sizeof(double));
+  double* Bp = calloc((size_t)(N * R), sizeof(double));
+  double* buf = malloc((size_t)(3 * N * R) * sizeof(double));
+  if (!phi || !phi_prev || !S || !xp || !Bp || !buf) {
+    free(phi); free(phi_prev); free(S); free(xp); free(Bp); free(buf);
+    return 1;
+  }
+  for (int64_t i = 0; i < NH; ++i) phi[i] = j->angle0 ? j->angle0[bh * NH + i] : 0.0;
+  memcpy(phi_prev, phi, (size_t)NH * sizeof(double));
+  if (j->h0) memcpy(S, j->h0 + bh * N * P, (size_t)(N * P) * sizeof(double));
+  if (j->xprev0) memcpy(xp, j->xprev0 + bh * P * R, (size_t)(P * R) * sizeof(double));
+  if (j->bprev0) memcpy(Bp, j->bprev0 + (b * G + g) * N * R, (size_t)(N * R) * sizeof(double));
+  for (int64_t t = 0; t < L; ++t) {
+    const int64_t th = (b * L + t) * H + h, tg = (b * L + t) * G + g;
+    mimo_token(d, h, j->X + th * P * R, j->B + tg * N * R, j->C + tg * N * R,
+               j->theta ? j->theta + th * NH : NULL, j->logdecay[th],
+               j->beta ? j->beta[th] : 0.0, j->gamma[th], j->D, phi, phi_prev, S, xp, Bp, buf,
+               buf + N * R, buf + 2 * N * R, j->Y + th * P * R);
+  }
+  if (j->hT) memcpy(j->hT + bh * N * P, S, (size_t)(N * P) * sizeof(double));
+  if (j->angleT) memcpy(j->angleT + bh * NH, phi, (size_t)NH * sizeof(double));
+  if (j->xprevT) memcpy(j->xprevT + bh * P * R, xp, (size_t)(P * R) * sizeof(double));
+  if (j->bprevT && h % (H / G) == 0)
+    memcpy(j->bprevT + (b * G + g) * N * R, Bp, (size_t)(N * R) * sizeof(double));
+  free(phi); free(phi_prev); free(S); free(xp); free(Bp); free(buf);
+  return 0;
+}
+
+static void* mimo_worker(void* arg) {
+  mimo_job* j = (mimo_job*)arg;
+  const int64_t npairs = j->d->batch * j->d->nheads;
+  for (;;) {
+    pthread_mutex_lock(&j->mu);
+    const int64_t k = j->next_pair++;
+    pthread_mutex_unlock(&j->mu);
+    if (k >= npairs) break;
+    if (mimo_one(j, k / j->d->nheads, k % j->d->nheads) != 0) {
+      pthread_mutex_lock(&j->mu);
+      j->status = 1;
+      pthread_mutex_unlock(&j->mu);
+    }
+  }
+  return NULL;
+}
+
+static int mimo_dims_ok(const oracle_mimo_dims* d) {
+  if (!d || d->rank < 1) return 0;
+  const oracle_dims s = {d->batch, d->seqlen, d->nheads, d->headdim, d->dstate, d->ngroups};
+  return dims_ok(&s);
+}
+
+/*
+ * MIMO forward.  Layouts: X, Y (b,L,H,P,R); logdecay, beta, gamma (b,L,H);
+ * B, C (b,L,G,N,R); theta (b,L,H,N/2); D (H); h0, hT (b,H,N,P);
+ * angle0, angleT (b,H,N/2); xprev0, xprevT (b,H,P,R); bprev0, bprevT (b,G,N,R).
+ * NULL conventions and return codes as oracle_fwd.
+ */
+int oracle_mimo_fwd(const oracle_mimo_dims* d, const double* X, const double* logdecay,
+                    const double* beta, const double* gamma, const double* B, const double* C,
+                    const double* theta, const double* D, const double* h0, const double* angle0,
+                    const double* xprev0, const double* bprev0, double* Y, double* hT,
+                    double* angleT, double* xprevT, double* bprevT, int nthreads) {
+  if (!mimo_dims_ok(d)) return 1;
+  if (d->batch * d->seqlen > 0 && (!X || !logdecay || !gamma || !B || !C || !Y)) return 1;
+  mimo_job j = {d, X, logdecay, beta, gamma, B, C, theta, D, h0, angle0, xprev0, bprev0,
+                Y, hT, angleT, xprevT, bprevT, 0, PTHREAD_MUTEX_INITIALIZER, 0};
+  if (nthreads < 1) nthreads = 1;
+  const int64_t npairs = d->batch * d->nheads;
+  if (nthreads > npairs) nthreads = (int)(npairs > 0 ? npairs : 1);
+  pthread_t* th = malloc((size_t)nthreads * sizeof(pthread_t));
+  int started = 0;
+  if (th)
+    for (int k = 0; k < nthreads; ++k) {
+      if (pthread_create(&th[k], NULL, mimo_worker, &j) != 0) break;
+      ++started;
+    }
+  if (started == 0) mimo_worker(&j);
+  for (int k = 0; k < started; ++k) pthread_join(th[k], NULL);
+  free(th);
+  return j.status ? 2 : 0;
+}
+
+/*
+ * One MIMO decode step on a cache (angle (b,H,N/2), ssm (b,H,N,P),
+ * x_prev (b,H,P,R), b_prev (b,G,N,R) unrotated), updated in place; x_t, y_t
+ * (b,H,P,R), B_t, C_t (b,G,N,R), logdecay_t, beta_t, gamma_t (b,H),
+ * theta_t (b,H,N/2).  b_prev is replaced after every head has used it.
+ */
+int oracle_mimo_step(const oracle_mimo_dims* d, const double* x_t, const double* logdecay_t,
+                     const double* beta_t, const double* gamma_t, const double* B_t,
+                     const double* C_t, const double* theta_t, const double* D, double* angle,
+                     double* ssm, double* x_prev, double* b_prev, double* y_t) {
+  if (!mimo_dims_ok(d)) return 1;
+  const int64_t Bt = d->batch, H = d->nheads, P = d->headdim, N = d->dstate, G = d->ngroups;
+  const int64_t R = d->rank, NH = N / 2;
+  double* phi_prev = malloc((size_t)NH * sizeof(double));
+  double* Bp = malloc((size_t)(N * R) * sizeof(double));
+  double* buf = malloc((size_t)(3 * N * R) * sizeof(double));
+  if (!phi_prev || !Bp || !buf) {
+    free(phi_prev); free(Bp); free(buf);
+    return 2;
+  }
+  for (int64_t b = 0; b < Bt; ++b)
+    for (int64_t h = 0; h < H; ++h) {
+      const int64_t bh = b * H + h, g = h / (H / G);
+      memcpy(phi_prev, angle + bh * NH, (size_t)NH * sizeof(double));
+      memcpy(Bp, b_prev + (b * G + g) * N * R, (size_t)(N * R) * sizeof(double));
+      mimo_token(d, h, x_t + bh * P * R, B_t + (b * G + g) * N * R, C_t + (b * G + g) * N * R,
+                 theta_t ? theta_t + bh * NH : NULL, logdecay_t[bh], beta_t ? beta_t[bh] : 0.0,
+                 gamma_t[bh], D, angle + bh * NH, phi_prev, ssm + bh * N * P,
+                 x_prev + bh * P * R, Bp, buf, buf + N * R, buf + 2 * N * R, y_t + bh * P * R);
+    }
+  memcpy(b_prev, B_t, (size_t)(Bt * G * N * R) * sizeof(double));
+  free(phi_prev); free(Bp); free(buf);
+  return 0;
+}

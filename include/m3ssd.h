@@ -159,6 +159,36 @@ m3ssd_status m3ssd_step(const m3ssd_dims* dims, const void* x_t, const float* lo
                         const void* C_t, const float* theta_t, const float* D,
                         const m3ssd_cache* cache, void* y_t, void* stream);
 
+/*
+ * MIMO rank R forward ("TorchMamba" README, table "Models", row Mamba-3 MIMO:
+ * a rank-R matmul update on a shared (N, P) state; "Functional cores":
+ * mimo_loop with X (B,L,H,P,R) -> Y (B,L,H,P,R), h (B,H,N,P)):
+ *   h_t = alpha_t h_{t-1} + beta_t sum_r Bbar_{t-1,r} x_{t-1,r}^T + gamma_t sum_r Bbar_{t,r} x_{t,r}^T
+ *   y_{t,r} = Cbar_{t,r}^T h_t + D x_{t,r}
+ * with every rank column of B and C rotated by the head's angle.  Layouts as
+ * m3ssd_fwd with a trailing rank axis: X, Y (b, L, H, P, R); B, C
+ * (b, L, G, N, R); extra->xprev0 / xprevT (b, H, P, R) and bprev0 / bprevT
+ * (b, G, N, R); the state h0, hT stays (b, H, N, P).  1 <= rank <= 8, N <= 256,
+ * P <= 256, N*P <= 16384 (else M3SSD_ERR_UNSUPPORTED).  Sequential fp32 state;
+ * Y rounded once to x_dtype.  No workspace, no allocation, no synchronisation.
+ */
+m3ssd_status m3ssd_mimo_fwd(const m3ssd_dims* dims, int32_t rank, const void* X,
+                            const float* logdecay, const float* beta, const float* gamma,
+                            const void* B, const void* C, const float* theta, const float* D,
+                            const float* h0, void* Y, float* hT, const m3ssd_fwd_extra* extra,
+                            void* stream);
+
+/*
+ * One MIMO decode step on a cache whose x_prev is (b, H, P, R) and b_prev
+ * (b, G, N, R) (angle and ssm as for m3ssd_step); x_t, y_t (b, H, P, R) and
+ * B_t, C_t (b, G, N, R) have dtype dims->x_dtype.  Limits as m3ssd_mimo_fwd.
+ * Two launches (the step, then b_prev <- B_t).  No allocation, no synchronisation.
+ */
+m3ssd_status m3ssd_mimo_step(const m3ssd_dims* dims, int32_t rank, const void* x_t,
+                             const float* logdecay_t, const float* beta_t, const float* gamma_t,
+                             const void* B_t, const void* C_t, const float* theta_t,
+                             const float* D, const m3ssd_cache* cache, void* y_t, void* stream);
+
 /* fp32 gradient outputs of m3ssd_bwd, each shaped like the matching input of
  * m3ssd_fwd (dB, dC, dbprev0 per group; dD per head).  dX, dlogdecay, dgamma,
  * dB, dC are required when b*L > 0; the others may be NULL (not written).  An

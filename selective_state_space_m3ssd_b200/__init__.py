@@ -82,6 +82,12 @@ def load(path: str | None = None):
         lib.m3ssd_step.argtypes = [ctypes.POINTER(Dims)] + [vp] * 8 + \
             [ctypes.POINTER(Cache), vp, vp]
         lib.m3ssd_step.restype = ctypes.c_int
+        lib.m3ssd_mimo_fwd.argtypes = [ctypes.POINTER(Dims), ctypes.c_int32] + [vp] * 11 + \
+            [ctypes.POINTER(FwdExtra), vp]
+        lib.m3ssd_mimo_fwd.restype = ctypes.c_int
+        lib.m3ssd_mimo_step.argtypes = [ctypes.POINTER(Dims), ctypes.c_int32] + [vp] * 8 + \
+            [ctypes.POINTER(Cache), vp, vp]
+        lib.m3ssd_mimo_step.restype = ctypes.c_int
         lib.m3ssd_bwd_workspace_size.argtypes = [ctypes.POINTER(Dims)]
         lib.m3ssd_bwd_workspace_size.restype = sz
         lib.m3ssd_bwd.argtypes = [ctypes.POINTER(Dims)] + [vp] * 9 + \
@@ -354,6 +360,88 @@ def step(cache: dict, x_t, logdecay_t, beta_t, gamma_t, B_t, C_t, theta_t=None, 
                            _ptr(gamma_t), _ptr(B_t), _ptr(C_t), _ptr(theta_t), _ptr(D),
                            ctypes.byref(c), _ptr(y_t), _stream_handle(dev))
     _check(st, "m3ssd_step")
+    return y_t
+
+
+def mimo_fwd(X, logdecay, beta, gamma, B, C, theta=None, D=None, h0=None, *, Y=None,
+             want_hT: bool = True, angle0=None, xprev0=None, bprev0=None,
+             want_cache: bool = False):
+    """MIMO rank-R forward through ``m3ssd_mimo_fwd``: X (b,L,H,P,R), B, C
+    (b,L,G,N,R).  Returns ``(Y, hT, cache_out)`` like :func:`fwd`, with the
+    cache's x_prev (b,H,P,R) and b_prev (b,G,N,R)."""
+    import torch
+    b, L, H, P, R = X.shape
+    G, N = B.shape[2], B.shape[3]
+    dev, f32, xd = X.device, torch.float32, X.dtype
+    _need(X, "X", device=dev)
+    for name, t, dt, shape in (("logdecay", logdecay, f32, (b, L, H)), ("beta", beta, f32, (b, L, H)),
+                               ("gamma", gamma, f32, (b, L, H)), ("B", B, xd, (b, L, G, N, R)),
+                               ("C", C, xd, (b, L, G, N, R)), ("theta", theta, f32, (b, L, H, N // 2)),
+                               ("D", D, f32, (H,)), ("h0", h0, f32, (b, H, N, P)),
+                               ("angle0", angle0, f32, (b, H, N // 2)),
+                               ("xprev0", xprev0, f32, (b, H, P, R)),
+                               ("bprev0", bprev0, f32, (b, G, N, R))):
+        _need(t, name, dt, shape, dev)
+    Y = torch.empty_like(X) if Y is None else Y
+    _need(Y, "Y", xd, (b, L, H, P, R), dev)
+    hT = torch.empty(b, H, N, P, dtype=f32, device=dev) if want_hT else None
+    cache_out = None
+    extra = None
+    if want_cache or angle0 is not None or xprev0 is not None or bprev0 is not None:
+        if want_cache:
+            cache_out = {"angle": torch.empty(b, H, N // 2, dtype=f32, device=dev),
+                         "x_prev": torch.empty(b, H, P, R, dtype=f32, device=dev),
+                         "b_prev": torch.empty(b, G, N, R, dtype=f32, device=dev)}
+        extra = FwdExtra(
+            *(None if t is None else t.data_ptr() for t in (angle0, xprev0, bprev0)),
+            *(None if cache_out is None else cache_out[k].data_ptr()
+              for k in ("angle", "x_prev", "b_prev")))
+    dims = make_dims(b, L, H, P, N, G, _xdtype(X), 0)
+    st = load().m3ssd_mimo_fwd(ctypes.byref(dims), R, _ptr(X), _ptr(logdecay), _ptr(beta),
+                               _ptr(gamma), _ptr(B), _ptr(C), _ptr(theta), _ptr(D), _ptr(h0),
+                               _ptr(Y), _ptr(hT), None if extra is None else ctypes.byref(extra),
+                               _stream_handle(dev))
+    _check(st, "m3ssd_mimo_fwd")
+    return Y, hT, cache_out
+
+
+def new_mimo_cache(batch, nheads, headdim, dstate, ngroups, rank, device):
+    """A zeroed fp32 MIMO decode cache: angle, ssm, x_prev (b,H,P,R), b_prev (b,G,N,R)."""
+    import torch
+    z = dict(dtype=torch.float32, device=device)
+    return {"angle": torch.zeros(batch, nheads, dstate // 2, **z),
+            "ssm": torch.zeros(batch, nheads, dstate, headdim, **z),
+            "x_prev": torch.zeros(batch, nheads, headdim, rank, **z),
+            "b_prev": torch.zeros(batch, ngroups, dstate, rank, **z)}
+
+
+def mimo_step(cache: dict, x_t, logdecay_t, beta_t, gamma_t, B_t, C_t, theta_t=None, D=None, *,
+              y_t=None):
+    """One MIMO decode step through ``m3ssd_mimo_step``: x_t (b,H,P,R), B_t, C_t
+    (b,G,N,R); updates ``cache`` in place and returns y_t (b,H,P,R)."""
+    import torch
+    b, H, P, R = x_t.shape
+    G, N = B_t.shape[1], B_t.shape[2]
+    dev, f32, xd = x_t.device, torch.float32, x_t.dtype
+    _need(x_t, "x_t", device=dev)
+    for name, t, dt, shape in (("logdecay_t", logdecay_t, f32, (b, H)), ("beta_t", beta_t, f32, (b, H)),
+                               ("gamma_t", gamma_t, f32, (b, H)), ("B_t", B_t, xd, (b, G, N, R)),
+                               ("C_t", C_t, xd, (b, G, N, R)), ("theta_t", theta_t, f32, (b, H, N // 2)),
+                               ("D", D, f32, (H,)),
+                               ("cache.angle", cache["angle"], f32, (b, H, N // 2)),
+                               ("cache.ssm", cache["ssm"], f32, (b, H, N, P)),
+                               ("cache.x_prev", cache["x_prev"], f32, (b, H, P, R)),
+                               ("cache.b_prev", cache["b_prev"], f32, (b, G, N, R))):
+        _need(t, name, dt, shape, dev)
+    y_t = torch.empty_like(x_t) if y_t is None else y_t
+    _need(y_t, "y_t", xd, (b, H, P, R), dev)
+    c = Cache(cache["angle"].data_ptr(), cache["ssm"].data_ptr(), cache["x_prev"].data_ptr(),
+              cache["b_prev"].data_ptr())
+    dims = make_dims(b, 1, H, P, N, G, _xdtype(x_t))
+    st = load().m3ssd_mimo_step(ctypes.byref(dims), R, _ptr(x_t), _ptr(logdecay_t), _ptr(beta_t),
+                                _ptr(gamma_t), _ptr(B_t), _ptr(C_t), _ptr(theta_t), _ptr(D),
+                                ctypes.byref(c), _ptr(y_t), _stream_handle(dev))
+    _check(st, "m3ssd_mimo_step")
     return y_t
 
 

@@ -77,6 +77,12 @@ struct BwdArgs {
 size_t bwd_workspace_bytes(int64_t b, int64_t L, int64_t H, int64_t P, int64_t N);
 cudaError_t launch_bwd_seq(const BwdArgs& a, cudaStream_t s);
 
+// MIMO rank R (1..8): layouts as the SISO ones with a trailing rank axis on X,
+// Y, B, C, x_prev, b_prev (and the extra cache inputs / outputs).
+bool mimo_shape_ok(int64_t N, int64_t P, int64_t R);
+cudaError_t launch_mimo_fwd(const FwdArgs& a, int64_t R, cudaStream_t s);
+cudaError_t launch_mimo_step(const StepArgs& a, int64_t R, cudaStream_t s);
+
 // Sequential fp32 forward: one CTA per (b, h), token by token.
 cudaError_t launch_fwd_seq(const FwdArgs& a, cudaStream_t s);
 // Chunked bf16 tensor-core forward (N = 128, P = 64).

@@ -118,6 +118,76 @@ m3ssd_status m3ssd_fwd(const m3ssd_dims* dims, const void* X, const float* logde
   return from_cuda(chunked ? m3ssd::launch_fwd_chunk(a, s) : m3ssd::launch_fwd_seq(a, s));
 }
 
+m3ssd_status m3ssd_mimo_fwd(const m3ssd_dims* dims, int32_t rank, const void* X,
+                            const float* logdecay, const float* beta, const float* gamma,
+                            const void* B, const void* C, const float* theta, const float* D,
+                            const float* h0, void* Y, float* hT, const m3ssd_fwd_extra* extra,
+                            void* stream) {
+  m3ssd_status st = check_dims(dims);
+  if (st != M3SSD_OK) return st;
+  if (dims->chunk != 0) return M3SSD_ERR_UNSUPPORTED;
+  if (rank < 1) return M3SSD_ERR_INVALID_ARG;
+  if (!m3ssd::mimo_shape_ok(dims->dstate, dims->headdim, rank)) return M3SSD_ERR_UNSUPPORTED;
+  const bool bf16 = dims->x_dtype == M3SSD_BF16;
+  const uintptr_t esz = bf16 ? 2 : 4;
+  if (dims->batch * dims->seqlen > 0 && (!X || !logdecay || !gamma || !B || !C || !Y))
+    return M3SSD_ERR_INVALID_ARG;
+  if (!aligned(X, esz) || !aligned(B, esz) || !aligned(C, esz) || !aligned(Y, esz))
+    return M3SSD_ERR_INVALID_ARG;
+  const void* f32ptrs[] = {logdecay, beta, gamma, theta, D, h0, hT};
+  for (const void* p : f32ptrs)
+    if (!aligned(p, 4)) return M3SSD_ERR_INVALID_ARG;
+  m3ssd::FwdArgs a{};
+  if (extra) {
+    if (extra->bprevT && extra->bprevT == extra->bprev0) return M3SSD_ERR_INVALID_ARG;
+    const void* eptrs[] = {extra->angle0, extra->xprev0, extra->bprev0,
+                           extra->angleT, extra->xprevT, extra->bprevT};
+    for (const void* p : eptrs)
+      if (!aligned(p, 4)) return M3SSD_ERR_INVALID_ARG;
+    a.angle0 = extra->angle0; a.xprev0 = extra->xprev0; a.bprev0 = extra->bprev0;
+    a.angleT = extra->angleT; a.xprevT = extra->xprevT; a.bprevT = extra->bprevT;
+  }
+  if (dims->batch == 0) return M3SSD_OK;
+  a.b = dims->batch; a.L = dims->seqlen; a.H = dims->nheads; a.P = dims->headdim;
+  a.N = dims->dstate; a.G = dims->ngroups; a.bf16 = bf16;
+  a.X = X; a.logdecay = logdecay; a.beta = beta; a.gamma = gamma; a.B = B; a.C = C;
+  a.theta = theta; a.D = D; a.h0 = h0; a.Y = Y; a.hT = hT;
+  return from_cuda(m3ssd::launch_mimo_fwd(a, rank, static_cast<cudaStream_t>(stream)));
+}
+
+m3ssd_status m3ssd_mimo_step(const m3ssd_dims* dims, int32_t rank, const void* x_t,
+                             const float* logdecay_t, const float* beta_t, const float* gamma_t,
+                             const void* B_t, const void* C_t, const float* theta_t,
+                             const float* D, const m3ssd_cache* cache, void* y_t, void* stream) {
+  m3ssd_status st = check_dims(dims);
+  if (st != M3SSD_OK) return st;
+  if (rank < 1) return M3SSD_ERR_INVALID_ARG;
+  if (!m3ssd::mimo_shape_ok(dims->dstate, dims->headdim, rank)) return M3SSD_ERR_UNSUPPORTED;
+  if (!cache) return M3SSD_ERR_INVALID_ARG;
+  const bool bf16 = dims->x_dtype == M3SSD_BF16;
+  const uintptr_t esz = bf16 ? 2 : 4;
+  if (dims->batch > 0) {
+    if (!x_t || !logdecay_t || !gamma_t || !B_t || !C_t || !y_t) return M3SSD_ERR_INVALID_ARG;
+    if (!cache->angle || !cache->ssm || !cache->x_prev || !cache->b_prev)
+      return M3SSD_ERR_INVALID_ARG;
+  }
+  if (!aligned(x_t, esz) || !aligned(B_t, esz) || !aligned(C_t, esz) || !aligned(y_t, esz))
+    return M3SSD_ERR_INVALID_ARG;
+  const void* f32ptrs[] = {logdecay_t, beta_t, gamma_t, theta_t, D,
+                           cache->angle, cache->ssm, cache->x_prev, cache->b_prev};
+  for (const void* p : f32ptrs)
+    if (!aligned(p, 4)) return M3SSD_ERR_INVALID_ARG;
+  if (dims->batch == 0) return M3SSD_OK;
+  m3ssd::StepArgs a{};
+  a.b = dims->batch; a.H = dims->nheads; a.P = dims->headdim; a.N = dims->dstate;
+  a.G = dims->ngroups; a.bf16 = bf16;
+  a.x_t = x_t; a.logdecay_t = logdecay_t; a.beta_t = beta_t; a.gamma_t = gamma_t;
+  a.B_t = B_t; a.C_t = C_t; a.theta_t = theta_t; a.D = D;
+  a.angle = cache->angle; a.ssm = cache->ssm; a.x_prev = cache->x_prev; a.b_prev = cache->b_prev;
+  a.y_t = y_t;
+  return from_cuda(m3ssd::launch_mimo_step(a, rank, static_cast<cudaStream_t>(stream)));
+}
+
 size_t m3ssd_bwd_workspace_size(const m3ssd_dims* dims) {
   if (check_dims(dims) != M3SSD_OK || !general_shape_ok(dims)) return 0;
   return m3ssd::bwd_workspace_bytes(dims->batch, dims->seqlen, dims->nheads, dims->headdim,

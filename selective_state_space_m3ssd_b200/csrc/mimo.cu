@@ -1,0 +1,238 @@
+// MIMO rank-R scan and decode step (fp32 state; X, B, C, Y in fp32 or bf16).
+//
+// "TorchMamba" README, table "Models", row Mamba-3 MIMO: a rank-R matmul update
+// on a shared (N, P) state; "Functional cores": mimo_loop with X (B,L,H,P,R)
+// -> Y (B,L,H,P,R) and h (B,H,N,P); "Math notes", MIMO.  With B and C carrying
+// the rank axis as (b,L,G,N,R) and every rank column rotated by the head's
+// angle:
+//   h_t = a_t h_{t-1} + beta_t sum_r Bbar_{t-1,r} x_{t-1,r}^T + gamma_t sum_r Bbar_{t,r} x_{t,r}^T
+//   y_{t,r} = Cbar_{t,r}^T h_t + D x_{t,r}
+// One CTA per (b, h).  Thread (rg, p) with p = tid % P and rg = tid / P updates
+// the state column p in rows rg, rg + NG, ... and keeps the R partial outputs of
+// that column; the NG row groups' partials are summed through shared memory.
+// Per state element a token costs 2R fused multiply-adds for the update and R
+// for the output against 8 bytes of state traffic in the decode step, so at
+// R <= 8 the step stays bound by HBM.
+#include "common.cuh"
+#include "internal.h"
+
+namespace m3ssd {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kMaxRank = 8;
+
+// Shared-memory layout of one token (floats).
+struct MimoSmem {
+  float *Bb, *Cb, *Bpb;  // N*R each: rotated B_t, C_t, B_{t-1}
+  float *xv, *xpv;       // P*R each: x_t, x_{t-1}
+  float *phi, *phip;     // N/2 each: angle of t and of t-1
+  float* red;            // NG*P*R partial outputs
+};
+
+__device__ __forceinline__ MimoSmem carve(float* base, int64_t N, int64_t P, int64_t R, int NG) {
+  MimoSmem m;
+  m.Bb = base;
+  m.Cb = m.Bb + N * R;
+  m.Bpb = m.Cb + N * R;
+  m.xv = m.Bpb + N * R;
+  m.xpv = m.xv + P * R;
+  m.phi = m.xpv + P * R;
+  m.phip = m.phi + N / 2;
+  m.red = m.phip + N / 2;
+  return m;
+}
+size_t token_smem_floats(int64_t N, int64_t P, int64_t R) {
+  const int NG = kThreads / (int)P;
+  return (size_t)(3 * N * R + 2 * P * R + N + (int64_t)NG * P * R);
+}
+
+// Columns of an (N, R) matrix v (element (n, r) at v[n R + r]) rotated pairwise by phi.
+template <typename V>
+__device__ __forceinline__ void rotate_cols(const V* v, const float* phi, int64_t N, int64_t R,
+                                            float* out) {
+  const int64_t NH = N / 2;
+  for (int64_t k = threadIdx.x; k < NH * R; k += kThreads) {
+    const int64_t i = k / R, r = k - i * R;
+    float s, c;
+    __sincosf(phi[i], &s, &c);
+    const float re = to_f32(v[(2 * i) * R + r]), im = to_f32(v[(2 * i + 1) * R + r]);
+    out[(2 * i) * R + r] = c * re - s * im;
+    out[(2 * i + 1) * R + r] = s * re + c * im;
+  }
+}
+
+// The state update and the outputs of one token, once Bb, Cb, Bpb, xv, xpv are in
+// shared memory.  S is the (N, P) state (shared or global memory); y receives
+// the (P, R) outputs in type T.
+template <typename T>
+__device__ __forceinline__ void token_update(const MimoSmem& m, float* S, int64_t N, int64_t P,
+                                             int64_t R, float a, float be, float ga, float Dh,
+                                             T* y) {
+  const int NG = kThreads / (int)P;
+  const int tid = threadIdx.x;
+  const int64_t p = tid % P, rg = tid / P;
+  if (rg < NG) {
+    float acc[kMaxRank];
+#pragma unroll
+    for (int r = 0; r < kMaxRank; ++r) acc[r] = 0.f;
+    for (int64_t n = rg; n < N; n += NG) {
+      float ub = 0.f, ug = 0.f;
+#pragma unroll
+      for (int r = 0; r < kMaxRank; ++r)
+        if (r < R) {
+          ub += m.Bpb[n * R + r] * m.xpv[p * R + r];
+          ug += m.Bb[n * R + r] * m.xv[p * R + r];
+        }
+      const float s = a * S[n * P + p] + be * ub + ga * ug;
+      S[n * P + p] = s;
+#pragma unroll
+      for (int r = 0; r < kMaxRank; ++r)
+        if (r < R) acc[r] += m.Cb[n * R + r] * s;
+    }
+#pragma unroll
+    for (int r = 0; r < kMaxRank; ++r)
+      if (r < R) m.red[(rg * P + p) * R + r] = acc[r];
+  }
+  __syncthreads();
+  for (int64_t k = tid; k < P * R; k += kThreads) {
+    float s = 0.f;
+    for (int g = 0; g < NG; ++g) s += m.red[(int64_t)g * P * R + k];
+    y[k] = from_f32<T>(s + Dh * m.xv[k]);
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads) mimo_fwd_kernel(FwdArgs a, int64_t R) {
+  extern __shared__ float smem[];
+  const int64_t H = a.H, P = a.P, N = a.N, G = a.G, L = a.L, NH = N / 2;
+  const int64_t bh = blockIdx.x, b = bh / H, h = bh % H, g = h / (H / G);
+  const int NG = kThreads / (int)P;
+  const int tid = threadIdx.x;
+  float* S = smem;
+  const MimoSmem m = carve(S + N * P, N, P, R, NG);
+  const T* X = static_cast<const T*>(a.X);
+  const T* Bg = static_cast<const T*>(a.B);
+  const T* Cg = static_cast<const T*>(a.C);
+  T* Y = static_cast<T*>(a.Y);
+  const float Dh = a.D ? a.D[h] : 0.f;
+
+  for (int64_t i = tid; i < NH; i += kThreads)
+    m.phi[i] = wrap_angle(a.angle0 ? a.angle0[bh * NH + i] : 0.f);
+  for (int64_t e = tid; e < N * P; e += kThreads) S[e] = a.h0 ? a.h0[bh * N * P + e] : 0.f;
+  __syncthreads();
+  for (int64_t t = 0; t < L; ++t) {
+    const int64_t th = (b * L + t) * H + h, tg = (b * L + t) * G + g;
+    for (int64_t k = tid; k < P * R; k += kThreads) {
+      m.xv[k] = to_f32(X[th * P * R + k]);
+      m.xpv[k] = t > 0 ? to_f32(X[(th - H) * P * R + k]) : (a.xprev0 ? a.xprev0[bh * P * R + k] : 0.f);
+    }
+    // B_{t-1} by phi_{t-1} (the cache's bprev0 for t = 0)
+    if (t > 0) {
+      rotate_cols(Bg + (tg - G) * N * R, m.phi, N, R, m.Bpb);
+    } else if (a.bprev0) {
+      rotate_cols(a.bprev0 + (b * G + g) * N * R, m.phi, N, R, m.Bpb);
+    } else {
+      for (int64_t k = tid; k < N * R; k += kThreads) m.Bpb[k] = 0.f;
+    }
+    __syncthreads();
+    for (int64_t i = tid; i < NH; i += kThreads)
+      m.phi[i] = wrap_angle(m.phi[i] + (a.theta ? a.theta[th * NH + i] : 0.f));
+    __syncthreads();
+    rotate_cols(Bg + tg * N * R, m.phi, N, R, m.Bb);
+    rotate_cols(Cg + tg * N * R, m.phi, N, R, m.Cb);
+    __syncthreads();
+    token_update<T>(m, S, N, P, R, expf(a.logdecay[th]), a.beta ? a.beta[th] : 0.f, a.gamma[th],
+                    Dh, Y + th * P * R);
+    __syncthreads();
+  }
+  if (a.hT)
+    for (int64_t e = tid; e < N * P; e += kThreads) a.hT[bh * N * P + e] = S[e];
+  if (a.angleT)
+    for (int64_t i = tid; i < NH; i += kThreads) a.angleT[bh * NH + i] = m.phi[i];
+  if (a.xprevT && L > 0)
+    for (int64_t k = tid; k < P * R; k += kThreads)
+      a.xprevT[bh * P * R + k] = to_f32(X[((b * L + L - 1) * H + h) * P * R + k]);
+  if (a.bprevT && L > 0 && h % (H / G) == 0)
+    for (int64_t k = tid; k < N * R; k += kThreads)
+      a.bprevT[(b * G + g) * N * R + k] = to_f32(Bg[((b * L + L - 1) * G + g) * N * R + k]);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads) mimo_step_kernel(StepArgs a, int64_t R) {
+  extern __shared__ float smem[];
+  const int64_t H = a.H, P = a.P, N = a.N, G = a.G, NH = N / 2;
+  const int64_t bh = blockIdx.x, b = bh / H, h = bh % H, g = h / (H / G);
+  const int NG = kThreads / (int)P;
+  const int tid = threadIdx.x;
+  const MimoSmem m = carve(smem, N, P, R, NG);
+  const T* x = static_cast<const T*>(a.x_t) + bh * P * R;
+  for (int64_t k = tid; k < P * R; k += kThreads) {
+    m.xv[k] = to_f32(x[k]);
+    m.xpv[k] = a.x_prev[bh * P * R + k];
+  }
+  for (int64_t i = tid; i < NH; i += kThreads) m.phip[i] = a.angle[bh * NH + i];
+  __syncthreads();
+  rotate_cols(a.b_prev + (b * G + g) * N * R, m.phip, N, R, m.Bpb);
+  for (int64_t i = tid; i < NH; i += kThreads)
+    m.phi[i] = wrap_angle(m.phip[i] + (a.theta_t ? a.theta_t[bh * NH + i] : 0.f));
+  __syncthreads();
+  rotate_cols(static_cast<const T*>(a.B_t) + (b * G + g) * N * R, m.phi, N, R, m.Bb);
+  rotate_cols(static_cast<const T*>(a.C_t) + (b * G + g) * N * R, m.phi, N, R, m.Cb);
+  __syncthreads();
+  token_update<T>(m, a.ssm + bh * N * P, N, P, R, expf(a.logdecay_t[bh]),
+                  a.beta_t ? a.beta_t[bh] : 0.f, a.gamma_t[bh], a.D ? a.D[h] : 0.f,
+                  static_cast<T*>(a.y_t) + bh * P * R);
+  for (int64_t i = tid; i < NH; i += kThreads) a.angle[bh * NH + i] = m.phi[i];
+  for (int64_t k = tid; k < P * R; k += kThreads) a.x_prev[bh * P * R + k] = m.xv[k];
+}
+
+// b_prev <- B_t once every head of the step has read the old value.
+template <typename T>
+__global__ void mimo_bprev_kernel(const T* B_t, float* b_prev, int64_t n) {
+  for (int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; k < n;
+       k += (int64_t)gridDim.x * blockDim.x)
+    b_prev[k] = to_f32(B_t[k]);
+}
+
+}  // namespace
+
+bool mimo_shape_ok(int64_t N, int64_t P, int64_t R) {
+  return R >= 1 && R <= kMaxRank && P <= kThreads && N <= 256 && N * P <= 16384 &&
+         sizeof(float) * ((size_t)(N * P) + token_smem_floats(N, P, R)) <= 200 * 1024;
+}
+
+cudaError_t launch_mimo_fwd(const FwdArgs& a, int64_t R, cudaStream_t s) {
+  if (a.b * a.H == 0) return cudaSuccess;
+  const size_t smem = sizeof(float) * ((size_t)(a.N * a.P) + token_smem_floats(a.N, a.P, R));
+  cudaError_t e;
+  if (a.bf16) {
+    e = cudaFuncSetAttribute(mimo_fwd_kernel<__nv_bfloat16>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    mimo_fwd_kernel<__nv_bfloat16><<<(unsigned)(a.b * a.H), kThreads, smem, s>>>(a, R);
+  } else {
+    e = cudaFuncSetAttribute(mimo_fwd_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+    if (e != cudaSuccess) return e;
+    mimo_fwd_kernel<float><<<(unsigned)(a.b * a.H), kThreads, smem, s>>>(a, R);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_mimo_step(const StepArgs& a, int64_t R, cudaStream_t s) {
+  if (a.b * a.H == 0) return cudaSuccess;
+  const size_t smem = sizeof(float) * token_smem_floats(a.N, a.P, R);
+  const int64_t nbp = a.b * a.G * a.N * R;
+  const unsigned gbp = (unsigned)((nbp + 255) / 256 < 1024 ? (nbp + 255) / 256 : 1024);
+  if (a.bf16) {
+    mimo_step_kernel<__nv_bfloat16><<<(unsigned)(a.b * a.H), kThreads, smem, s>>>(a, R);
+    mimo_bprev_kernel<<<gbp, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(a.B_t), a.b_prev, nbp);
+  } else {
+    mimo_step_kernel<float><<<(unsigned)(a.b * a.H), kThreads, smem, s>>>(a, R);
+    mimo_bprev_kernel<<<gbp, 256, 0, s>>>(static_cast<const float*>(a.B_t), a.b_prev, nbp);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace m3ssd

@@ -155,6 +155,29 @@ def test_bwd_validation(lib):
     assert _bwd(lib, _dims(batch=0), X=None, dY=None, ws=FAKE, ws_bytes=1 << 20) == m3.OK
 
 
+def test_mimo_validation(lib):
+    d = _dims()
+    def fwd(rank, dims=d, X=FAKE):
+        return lib.m3ssd_mimo_fwd(ctypes.byref(dims), rank, X, FAKE, None, FAKE, FAKE, FAKE, None,
+                                  None, None, FAKE, None, None, None)
+    assert fwd(0) == m3.ERR_INVALID_ARG
+    assert fwd(9) == m3.ERR_UNSUPPORTED
+    assert fwd(2, X=None) == m3.ERR_INVALID_ARG
+    assert fwd(2, X=ctypes.c_void_p(0x10002)) == m3.ERR_INVALID_ARG
+    assert fwd(2, dims=_dims(chunk=64)) == m3.ERR_UNSUPPORTED
+    assert fwd(2, dims=_dims(dstate=7)) == m3.ERR_INVALID_ARG
+    assert fwd(2, dims=_dims(batch=0), X=None) == m3.OK
+    c = m3.Cache(0x10000, 0x10000, 0x10000, 0x10000)
+    def step(rank, cache=c, x=FAKE):
+        return lib.m3ssd_mimo_step(ctypes.byref(d), rank, x, FAKE, None, FAKE, FAKE, FAKE, None,
+                                   None, ctypes.byref(cache) if cache else None, FAKE, None)
+    assert step(0) == m3.ERR_INVALID_ARG
+    assert step(9) == m3.ERR_UNSUPPORTED
+    assert step(2, cache=None) == m3.ERR_INVALID_ARG
+    assert step(2, x=None) == m3.ERR_INVALID_ARG
+    assert step(2, cache=m3.Cache(0x10000, None, 0x10000, 0x10000)) == m3.ERR_INVALID_ARG
+
+
 def test_wait_timeout_query_rejects_null(lib):
     assert lib.m3ssd_device_wait_timeouts(None) == m3.ERR_INVALID_ARG
 

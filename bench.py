@@ -347,6 +347,70 @@ def bench_decode(dev, rank, steps_graph_replays: int, peaks: dict):
             "gpu_launches": 2 * nsteps}
 
 
+def bench_mimo_decode(dev, rank, peaks: dict, R: int = 4, nsteps: int = 100, replays: int = 3):
+    """MIMO rank-R decode: one CUDA graph of ``nsteps`` m3ssd_mimo_step calls on
+    pre-staged synthetic per-step inputs of the decode workload's shape (fp32
+    cache and inputs), replayed ``replays`` times."""
+    import selective_state_space_m3ssd_b200 as m3
+    w = rank_workload(WORKLOADS["decode"], rank)
+    b, H, P, N, G = w.batch, w.nheads, w.headdim, w.dstate, w.ngroups
+    gen = torch.Generator(device=dev).manual_seed(w.seed + 17)
+    z = dict(device=dev, dtype=torch.float32)
+    cache = m3.new_mimo_cache(b, H, P, N, G, R, dev)
+    cache["ssm"].normal_(0, 0.3, generator=gen)
+    xs = torch.randn(nsteps, b, H, P, R, generator=gen, **z)
+    Bs = torch.randn(nsteps, b, G, N, R, generator=gen, **z) / N ** 0.5
+    Cs = torch.randn(nsteps, b, G, N, R, generator=gen, **z) / N ** 0.5
+    ths = torch.randn(nsteps, b, H, N // 2, generator=gen, **z) * 0.05
+    lds = -torch.rand(nsteps, b, H, generator=gen, **z) * 0.5
+    bes = torch.rand(nsteps, b, H, generator=gen, **z) * 0.3
+    gas = torch.rand(nsteps, b, H, generator=gen, **z) * 0.5
+    D = torch.randn(H, generator=gen, **z)
+    ys = torch.empty_like(xs)
+
+    def run_steps():
+        for t in range(nsteps):
+            m3.mimo_step(cache, xs[t], lds[t], bes[t], gas[t], Bs[t], Cs[t], ths[t], D, y_t=ys[t])
+
+    s = torch.cuda.Stream(dev)
+    s.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(s):
+        run_steps()
+    torch.cuda.current_stream(dev).wait_stream(s)
+    torch.cuda.synchronize(dev)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        run_steps()
+    g.replay()
+    torch.cuda.synchronize(dev)
+    stream = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(replays):
+        g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms_step = e0.elapsed_time(e1) / (nsteps * replays)
+    f = 4
+    step_bytes = (2 * b * H * N * P * f + 2 * b * H * (N // 2) * f + 2 * b * H * P * R * f
+                  + 2 * b * G * N * R * f + b * H * P * R * f + b * H * (N // 2) * f
+                  + 2 * b * G * N * R * f + 3 * b * H * f + H * f + b * H * P * R * f)
+    achieved = step_bytes / (ms_step / 1e3) / 1e9
+    del g
+    return {"metric": "mimo decode steps/s", "value": 1e3 / ms_step, "unit": "steps/s",
+            "ms_per_step": ms_step, "graph_steps": nsteps * replays,
+            "config": {"workload": f"MIMO rank-{R} decode b{b} H{H} P{P} N{N} fp32",
+                       "batch": b, "nheads": H, "headdim": P, "dstate": N, "rank": R,
+                       "dtype": "f32"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                         "peak_source": peaks["source"], "traffic": None,
+                         "algo_bytes_per_step": step_bytes,
+                         "flops_per_step": 2 * 3 * R * b * H * N * P,
+                         "note": "per step = MIMO step kernel + b_prev update kernel (2 launches)"},
+            "gpu_launches": 2 * nsteps * replays}
+
+
 def bench_backward(w, dev, steps, world, d, peaks):
     """The backward (m3ssd_bwd) on the forward's workload: dY, dhT synthetic,
     every gradient output written; inputs resident in HBM."""
@@ -409,6 +473,7 @@ def run_ours(args):
                       if hasattr(torch.cuda.get_device_properties(dev), "index") else local) as clk:
         fw = bench_forward(w, dev, args.steps, args.warmup, world, rank)
         dec = bench_decode(dev, rank, max(1, args.decode_replays), peaks)
+        mimo = bench_mimo_decode(dev, rank, peaks)
         bwd = None if args.no_backward else bench_backward(
             w, dev, max(1, min(args.steps, 3)), world, fw["dev_inputs"], peaks)
     e2e = bench_e2e(w, dev, max(1, min(args.steps, 5)), 1, fw["inp"], world)
@@ -430,6 +495,7 @@ def run_ours(args):
         "e2e": e2e,
         "gpu_launches": fw["launches"],
         "decode": dec,
+        "mimo_decode": mimo,
         "backward": bwd,
         "clocks": clk.summary(),
     }

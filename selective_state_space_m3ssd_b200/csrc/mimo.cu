@@ -22,6 +22,12 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kMaxRank = 8;
 
+constexpr int kVecRank = 4;
+// The float4 mapping of token_update_v4 applies.
+__host__ __device__ constexpr bool vec_ok(int64_t P, int64_t R) {
+  return P % 4 == 0 && R <= kVecRank && 4 * kThreads / P >= 1;
+}
+
 // Shared-memory layout of one token (floats).
 struct MimoSmem {
   float *Bb, *Cb, *Bpb;  // N*R each: rotated B_t, C_t, B_{t-1}
@@ -42,9 +48,10 @@ __device__ __forceinline__ MimoSmem carve(float* base, int64_t N, int64_t P, int
   m.red = m.phip + N / 2;
   return m;
 }
-size_t token_smem_floats(int64_t N, int64_t P, int64_t R) {
-  const int NG = kThreads / (int)P;
-  return (size_t)(3 * N * R + 2 * P * R + N + (int64_t)NG * P * R);
+size_t token_smem_floats(int64_t N, int64_t P, int64_t R, bool vec) {
+  // partial outputs: one set per row group of the mapping in use
+  const int64_t groups = vec ? 4 * kThreads / P : kThreads / P;
+  return (size_t)(3 * N * R + 2 * P * R + N + groups * P * R);
 }
 
 // Columns of an (N, R) matrix v (element (n, r) at v[n R + r]) rotated pairwise by phi.
@@ -102,8 +109,69 @@ __device__ __forceinline__ void token_update(const MimoSmem& m, float* S, int64_
   }
 }
 
+// The same for P % 4 == 0 and R <= 4: thread (rg, cg) owns the four columns
+// 4 cg .. 4 cg + 3 in rows rg, rg + NG4, ... (NG4 = 4 kThreads / P row groups),
+// moves the state as float4 and keeps its x_t, x_{t-1} values in registers.
 template <typename T>
-__global__ void __launch_bounds__(kThreads) mimo_fwd_kernel(FwdArgs a, int64_t R) {
+__device__ __forceinline__ void token_update_v4(const MimoSmem& m, float* S, int64_t N, int64_t P,
+                                                int64_t R, float a, float be, float ga, float Dh,
+                                                T* y) {
+  const int CG = (int)(P / 4), NG4 = kThreads / CG;
+  const int tid = threadIdx.x;
+  const int cg = tid % CG, rg = tid / CG;
+  if (rg < NG4) {
+    float xr[4][kVecRank], xpr[4][kVecRank], acc[4][kVecRank];
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+#pragma unroll
+      for (int r = 0; r < kVecRank; ++r) {
+        const bool on = r < R;
+        xr[c][r] = on ? m.xv[(4 * cg + c) * R + r] : 0.f;
+        xpr[c][r] = on ? m.xpv[(4 * cg + c) * R + r] : 0.f;
+        acc[c][r] = 0.f;
+      }
+    for (int64_t n = rg; n < N; n += NG4) {
+      float bb[kVecRank], bp[kVecRank], cc[kVecRank];
+#pragma unroll
+      for (int r = 0; r < kVecRank; ++r) {
+        const bool on = r < R;
+        bb[r] = on ? m.Bb[n * R + r] : 0.f;
+        bp[r] = on ? m.Bpb[n * R + r] : 0.f;
+        cc[r] = on ? m.Cb[n * R + r] : 0.f;
+      }
+      float4* sp = reinterpret_cast<float4*>(S + n * P + 4 * cg);
+      float4 v = *sp;
+      float* vv = reinterpret_cast<float*>(&v);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float ub = 0.f, ug = 0.f;
+#pragma unroll
+        for (int r = 0; r < kVecRank; ++r) {
+          ub = fmaf(bp[r], xpr[c][r], ub);
+          ug = fmaf(bb[r], xr[c][r], ug);
+        }
+        vv[c] = a * vv[c] + be * ub + ga * ug;
+#pragma unroll
+        for (int r = 0; r < kVecRank; ++r) acc[c][r] = fmaf(cc[r], vv[c], acc[c][r]);
+      }
+      *sp = v;
+    }
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+#pragma unroll
+      for (int r = 0; r < kVecRank; ++r)
+        if (r < R) m.red[((int64_t)rg * P + 4 * cg + c) * R + r] = acc[c][r];
+  }
+  __syncthreads();
+  for (int64_t k = tid; k < P * R; k += kThreads) {
+    float sum = 0.f;
+    for (int g2 = 0; g2 < NG4; ++g2) sum += m.red[(int64_t)g2 * P * R + k];
+    y[k] = from_f32<T>(sum + Dh * m.xv[k]);
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads) mimo_fwd_kernel(FwdArgs a, int64_t R, bool vec) {
   extern __shared__ float smem[];
   const int64_t H = a.H, P = a.P, N = a.N, G = a.G, L = a.L, NH = N / 2;
   const int64_t bh = blockIdx.x, b = bh / H, h = bh % H, g = h / (H / G);
@@ -111,6 +179,7 @@ __global__ void __launch_bounds__(kThreads) mimo_fwd_kernel(FwdArgs a, int64_t R
   const int tid = threadIdx.x;
   float* S = smem;
   const MimoSmem m = carve(S + N * P, N, P, R, NG);
+  (void)vec;
   const T* X = static_cast<const T*>(a.X);
   const T* Bg = static_cast<const T*>(a.B);
   const T* Cg = static_cast<const T*>(a.C);
@@ -142,8 +211,12 @@ __global__ void __launch_bounds__(kThreads) mimo_fwd_kernel(FwdArgs a, int64_t R
     rotate_cols(Bg + tg * N * R, m.phi, N, R, m.Bb);
     rotate_cols(Cg + tg * N * R, m.phi, N, R, m.Cb);
     __syncthreads();
-    token_update<T>(m, S, N, P, R, expf(a.logdecay[th]), a.beta ? a.beta[th] : 0.f, a.gamma[th],
-                    Dh, Y + th * P * R);
+    if (vec)
+      token_update_v4<T>(m, S, N, P, R, expf(a.logdecay[th]), a.beta ? a.beta[th] : 0.f,
+                         a.gamma[th], Dh, Y + th * P * R);
+    else
+      token_update<T>(m, S, N, P, R, expf(a.logdecay[th]), a.beta ? a.beta[th] : 0.f,
+                      a.gamma[th], Dh, Y + th * P * R);
     __syncthreads();
   }
   if (a.hT)
@@ -159,7 +232,7 @@ __global__ void __launch_bounds__(kThreads) mimo_fwd_kernel(FwdArgs a, int64_t R
 }
 
 template <typename T>
-__global__ void __launch_bounds__(kThreads) mimo_step_kernel(StepArgs a, int64_t R) {
+__global__ void __launch_bounds__(kThreads) mimo_step_kernel(StepArgs a, int64_t R, bool vec) {
   extern __shared__ float smem[];
   const int64_t H = a.H, P = a.P, N = a.N, G = a.G, NH = N / 2;
   const int64_t bh = blockIdx.x, b = bh / H, h = bh % H, g = h / (H / G);
@@ -180,9 +253,14 @@ __global__ void __launch_bounds__(kThreads) mimo_step_kernel(StepArgs a, int64_t
   rotate_cols(static_cast<const T*>(a.B_t) + (b * G + g) * N * R, m.phi, N, R, m.Bb);
   rotate_cols(static_cast<const T*>(a.C_t) + (b * G + g) * N * R, m.phi, N, R, m.Cb);
   __syncthreads();
-  token_update<T>(m, a.ssm + bh * N * P, N, P, R, expf(a.logdecay_t[bh]),
-                  a.beta_t ? a.beta_t[bh] : 0.f, a.gamma_t[bh], a.D ? a.D[h] : 0.f,
-                  static_cast<T*>(a.y_t) + bh * P * R);
+  if (vec)
+    token_update_v4<T>(m, a.ssm + bh * N * P, N, P, R, expf(a.logdecay_t[bh]),
+                       a.beta_t ? a.beta_t[bh] : 0.f, a.gamma_t[bh], a.D ? a.D[h] : 0.f,
+                       static_cast<T*>(a.y_t) + bh * P * R);
+  else
+    token_update<T>(m, a.ssm + bh * N * P, N, P, R, expf(a.logdecay_t[bh]),
+                    a.beta_t ? a.beta_t[bh] : 0.f, a.gamma_t[bh], a.D ? a.D[h] : 0.f,
+                    static_cast<T*>(a.y_t) + bh * P * R);
   for (int64_t i = tid; i < NH; i += kThreads) a.angle[bh * NH + i] = m.phi[i];
   for (int64_t k = tid; k < P * R; k += kThreads) a.x_prev[bh * P * R + k] = m.xv[k];
 }
@@ -199,37 +277,42 @@ __global__ void mimo_bprev_kernel(const T* B_t, float* b_prev, int64_t n) {
 
 bool mimo_shape_ok(int64_t N, int64_t P, int64_t R) {
   return R >= 1 && R <= kMaxRank && P <= kThreads && N <= 256 && N * P <= 16384 &&
-         sizeof(float) * ((size_t)(N * P) + token_smem_floats(N, P, R)) <= 200 * 1024;
+         sizeof(float) * ((size_t)(N * P) + token_smem_floats(N, P, R, vec_ok(P, R))) <=
+             200 * 1024 &&
+         sizeof(float) * token_smem_floats(N, P, R, false) <= 48 * 1024;
 }
 
 cudaError_t launch_mimo_fwd(const FwdArgs& a, int64_t R, cudaStream_t s) {
   if (a.b * a.H == 0) return cudaSuccess;
-  const size_t smem = sizeof(float) * ((size_t)(a.N * a.P) + token_smem_floats(a.N, a.P, R));
+  const bool vec = vec_ok(a.P, R);  // the state is in shared memory (16-byte aligned)
+  const size_t smem = sizeof(float) * ((size_t)(a.N * a.P) + token_smem_floats(a.N, a.P, R, vec));
   cudaError_t e;
   if (a.bf16) {
     e = cudaFuncSetAttribute(mimo_fwd_kernel<__nv_bfloat16>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    mimo_fwd_kernel<__nv_bfloat16><<<(unsigned)(a.b * a.H), kThreads, smem, s>>>(a, R);
+    mimo_fwd_kernel<__nv_bfloat16><<<(unsigned)(a.b * a.H), kThreads, smem, s>>>(a, R, vec);
   } else {
     e = cudaFuncSetAttribute(mimo_fwd_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem);
     if (e != cudaSuccess) return e;
-    mimo_fwd_kernel<float><<<(unsigned)(a.b * a.H), kThreads, smem, s>>>(a, R);
+    mimo_fwd_kernel<float><<<(unsigned)(a.b * a.H), kThreads, smem, s>>>(a, R, vec);
   }
   return cudaGetLastError();
 }
 
 cudaError_t launch_mimo_step(const StepArgs& a, int64_t R, cudaStream_t s) {
   if (a.b * a.H == 0) return cudaSuccess;
-  const size_t smem = sizeof(float) * token_smem_floats(a.N, a.P, R);
+  // float4 state accesses need a 16-byte aligned cache state
+  const bool vec = vec_ok(a.P, R) && (reinterpret_cast<uintptr_t>(a.ssm) & 15) == 0;
+  const size_t smem = sizeof(float) * token_smem_floats(a.N, a.P, R, vec);
   const int64_t nbp = a.b * a.G * a.N * R;
   const unsigned gbp = (unsigned)((nbp + 255) / 256 < 1024 ? (nbp + 255) / 256 : 1024);
   if (a.bf16) {
-    mimo_step_kernel<__nv_bfloat16><<<(unsigned)(a.b * a.H), kThreads, smem, s>>>(a, R);
+    mimo_step_kernel<__nv_bfloat16><<<(unsigned)(a.b * a.H), kThreads, smem, s>>>(a, R, vec);
     mimo_bprev_kernel<<<gbp, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(a.B_t), a.b_prev, nbp);
   } else {
-    mimo_step_kernel<float><<<(unsigned)(a.b * a.H), kThreads, smem, s>>>(a, R);
+    mimo_step_kernel<float><<<(unsigned)(a.b * a.H), kThreads, smem, s>>>(a, R, vec);
     mimo_bprev_kernel<<<gbp, 256, 0, s>>>(static_cast<const float*>(a.B_t), a.b_prev, nbp);
   }
   return cudaGetLastError();

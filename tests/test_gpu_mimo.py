@@ -100,3 +100,32 @@ def test_mimo_rejects_unsupported_rank():
     with pytest.raises(m3.M3SSDError):
         m3.mimo_fwd(bad, d["logdecay"], d["beta"], d["gamma"], d["B"].repeat(1, 1, 1, 1, 3),
                     d["C"].repeat(1, 1, 1, 1, 3))
+
+
+@pytest.mark.parametrize("aligned", [True, False])
+def test_mimo_decode_steps_at_wide_heads(aligned):
+    # P = 64, N = 128, R = 4: the float4 state mapping when the cache state is
+    # 16-byte aligned, the general mapping when it starts 4 bytes past that
+    inp = make_mimo(21, b=2, L=6, H=3, G=1, P=64, N=128, R=4)
+    ref_in, d = prep(inp, "bf16")
+    full = oracle.oracle_mimo_fwd(**ref_in)
+    L1 = 2
+    pre = {k: (v[:, :L1] if k in ("X", "logdecay", "beta", "gamma", "B", "C", "theta")
+               and v is not None else v) for k, v in ref_in.items()}
+    p = oracle.oracle_mimo_fwd(**pre)
+    n = p["hT"].size
+    buf = torch.zeros(n + 4, dtype=torch.float32, device="cuda")
+    ssm = buf[(0 if aligned else 1):][:n].view(p["hT"].shape)
+    ssm.copy_(torch.from_numpy(p["hT"]).float())
+    assert (ssm.data_ptr() % 16 == 0) == aligned
+    cache = {"angle": torch.from_numpy(p["angleT"]).float().cuda(), "ssm": ssm,
+             "x_prev": torch.from_numpy(p["xprevT"]).float().cuda(),
+             "b_prev": torch.from_numpy(p["bprevT"]).float().cuda()}
+    for t in range(L1, 6):
+        y = m3.mimo_step(cache, d["X"][:, t].contiguous(), d["logdecay"][:, t].contiguous(),
+                         d["beta"][:, t].contiguous(), d["gamma"][:, t].contiguous(),
+                         d["B"][:, t].contiguous(), d["C"][:, t].contiguous(),
+                         d["theta"][:, t].contiguous(), d["D"])
+        torch.cuda.synchronize()
+        assert rel_max_err_out(y.double().cpu().numpy(), full["Y"][:, t], True) <= TOL, t
+    assert rel_max_err(ssm.double().cpu().numpy(), full["hT"]) <= TOL

@@ -265,6 +265,129 @@ __global__ void __launch_bounds__(kThreads) mimo_step_kernel(StepArgs a, int64_t
   for (int64_t k = tid; k < P * R; k += kThreads) a.x_prev[bh * P * R + k] = m.xv[k];
 }
 
+// Specialised decode step for N = 128, P = 64 and R <= 4: 128 threads, thread
+// (r0, q) with q = tid % 16 and r0 = tid / 16 owning the 4-wide column slice q
+// of rows r0, r0 + 8, ...  Each thread starts the asynchronous copies of its own
+// 16 state float4 into shared memory before the rotation prologue, so the
+// state stream (32 KB per CTA) is in flight while the angles, sincos and
+// rotations are computed; it later reads back only what it copied itself.
+constexpr int kMN = 128, kMP = 64, kMThreads = 128, kMRows = kMN / (kMThreads / (kMP / 4));
+
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                   static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst))),
+               "l"(gmem_src)
+               : "memory");
+}
+
+template <typename T, int R>
+__global__ void __launch_bounds__(kMThreads) mimo_step_n128p64(StepArgs a) {
+  __shared__ float4 Sv[kMN * kMP / 4];
+  __shared__ __align__(16) float Bb[kMN * R], Cb[kMN * R], Bpb[kMN * R];
+  __shared__ __align__(16) float xs[kMP * R], xps[kMP * R];
+  __shared__ __align__(16) float red[kMThreads / 32][kMP * R];
+  const int64_t H = a.H, G = a.G;
+  const int64_t bh = blockIdx.x, b = bh / H, h = bh % H, g = h / (H / G);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int q = tid & 15, r0 = tid >> 4;
+  float4* S = reinterpret_cast<float4*>(a.ssm + bh * kMN * kMP);
+#pragma unroll
+  for (int k = 0; k < kMRows; ++k) {
+    const int e = (r0 + 8 * k) * (kMP / 4) + q;
+    cp_async16(&Sv[e], &S[e]);
+  }
+  asm volatile("cp.async.commit_group;" ::: "memory");
+
+  const int64_t gbase = (b * G + g) * kMN * R;
+  if (tid < kMN / 2) {
+    const int i = tid;
+    const float ang = a.angle[bh * (kMN / 2) + i];
+    const float ph = wrap_angle(ang + (a.theta_t ? a.theta_t[bh * (kMN / 2) + i] : 0.f));
+    float s, c, s0, c0;
+    sincosf(ph, &s, &c);
+    sincosf(ang, &s0, &c0);
+    const T* Bt = static_cast<const T*>(a.B_t) + gbase;
+    const T* Ct = static_cast<const T*>(a.C_t) + gbase;
+    const float* bp = a.b_prev + gbase;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int e0 = (2 * i) * R + r, e1 = (2 * i + 1) * R + r;
+      const float b0 = to_f32(Bt[e0]), b1 = to_f32(Bt[e1]);
+      const float c0v = to_f32(Ct[e0]), c1v = to_f32(Ct[e1]);
+      const float p0 = bp[e0], p1 = bp[e1];
+      Bb[e0] = c * b0 - s * b1;
+      Bb[e1] = s * b0 + c * b1;
+      Cb[e0] = c * c0v - s * c1v;
+      Cb[e1] = s * c0v + c * c1v;
+      Bpb[e0] = c0 * p0 - s0 * p1;
+      Bpb[e1] = s0 * p0 + c0 * p1;
+    }
+    a.angle[bh * (kMN / 2) + i] = ph;
+  } else {
+    const int p = tid - kMN / 2;
+    const T* xt = static_cast<const T*>(a.x_t) + bh * kMP * R;
+    float* xp = a.x_prev + bh * kMP * R;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const float x = to_f32(xt[p * R + r]);
+      xs[p * R + r] = x;
+      xps[p * R + r] = xp[p * R + r];
+      xp[p * R + r] = x;
+    }
+  }
+  const float alpha = expf(a.logdecay_t[bh]);
+  const float be = a.beta_t ? a.beta_t[bh] : 0.f;
+  const float ga = a.gamma_t[bh];
+  __syncthreads();
+
+  float xr[4][R], xpr[4][R], acc[4][R];
+#pragma unroll
+  for (int c = 0; c < 4; ++c)
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      xr[c][r] = ga * xs[(4 * q + c) * R + r];
+      xpr[c][r] = be * xps[(4 * q + c) * R + r];
+      acc[c][r] = 0.f;
+    }
+  asm volatile("cp.async.wait_all;" ::: "memory");
+#pragma unroll 4
+  for (int k = 0; k < kMRows; ++k) {
+    const int n = r0 + 8 * k;
+    float4 v = Sv[n * (kMP / 4) + q];
+    float* vv = reinterpret_cast<float*>(&v);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      float u = alpha * vv[c];
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        u = fmaf(Bpb[n * R + r], xpr[c][r], u);
+        u = fmaf(Bb[n * R + r], xr[c][r], u);
+      }
+      vv[c] = u;
+#pragma unroll
+      for (int r = 0; r < R; ++r) acc[c][r] = fmaf(Cb[n * R + r], u, acc[c][r]);
+    }
+    S[n * (kMP / 4) + q] = v;
+  }
+  // lanes l and l + 16 hold the same column slice
+#pragma unroll
+  for (int c = 0; c < 4; ++c)
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      acc[c][r] += __shfl_xor_sync(0xffffffffu, acc[c][r], 16);
+      if (lane < 16) red[warp][(4 * q + c) * R + r] = acc[c][r];
+    }
+  __syncthreads();
+  T* yt = static_cast<T*>(a.y_t) + bh * kMP * R;
+  const float Dh = a.D ? a.D[h] : 0.f;
+  for (int k = tid; k < kMP * R; k += kMThreads) {
+    float y = Dh * xs[k];
+#pragma unroll
+    for (int w = 0; w < kMThreads / 32; ++w) y += red[w][k];
+    yt[k] = from_f32<T>(y);
+  }
+}
+
 // b_prev <- B_t once every head of the step has read the old value.
 template <typename T>
 __global__ void mimo_bprev_kernel(const T* B_t, float* b_prev, int64_t n) {
@@ -308,6 +431,27 @@ cudaError_t launch_mimo_step(const StepArgs& a, int64_t R, cudaStream_t s) {
   const size_t smem = sizeof(float) * token_smem_floats(a.N, a.P, R, vec);
   const int64_t nbp = a.b * a.G * a.N * R;
   const unsigned gbp = (unsigned)((nbp + 255) / 256 < 1024 ? (nbp + 255) / 256 : 1024);
+  if (vec && a.N == kMN && a.P == kMP) {
+    const unsigned grid = (unsigned)(a.b * a.H);
+    if (a.bf16) {
+      switch (R) {
+        case 1: mimo_step_n128p64<__nv_bfloat16, 1><<<grid, kMThreads, 0, s>>>(a); break;
+        case 2: mimo_step_n128p64<__nv_bfloat16, 2><<<grid, kMThreads, 0, s>>>(a); break;
+        case 3: mimo_step_n128p64<__nv_bfloat16, 3><<<grid, kMThreads, 0, s>>>(a); break;
+        default: mimo_step_n128p64<__nv_bfloat16, 4><<<grid, kMThreads, 0, s>>>(a); break;
+      }
+      mimo_bprev_kernel<<<gbp, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(a.B_t), a.b_prev, nbp);
+    } else {
+      switch (R) {
+        case 1: mimo_step_n128p64<float, 1><<<grid, kMThreads, 0, s>>>(a); break;
+        case 2: mimo_step_n128p64<float, 2><<<grid, kMThreads, 0, s>>>(a); break;
+        case 3: mimo_step_n128p64<float, 3><<<grid, kMThreads, 0, s>>>(a); break;
+        default: mimo_step_n128p64<float, 4><<<grid, kMThreads, 0, s>>>(a); break;
+      }
+      mimo_bprev_kernel<<<gbp, 256, 0, s>>>(static_cast<const float*>(a.B_t), a.b_prev, nbp);
+    }
+    return cudaGetLastError();
+  }
   if (a.bf16) {
     mimo_step_kernel<__nv_bfloat16><<<(unsigned)(a.b * a.H), kThreads, smem, s>>>(a, R, vec);
     mimo_bprev_kernel<<<gbp, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(a.B_t), a.b_prev, nbp);

@@ -102,11 +102,11 @@ def test_mimo_rejects_unsupported_rank():
                     d["C"].repeat(1, 1, 1, 1, 3))
 
 
-@pytest.mark.parametrize("aligned", [True, False])
-def test_mimo_decode_steps_at_wide_heads(aligned):
-    # P = 64, N = 128, R = 4: the float4 state mapping when the cache state is
-    # 16-byte aligned, the general mapping when it starts 4 bytes past that
-    inp = make_mimo(21, b=2, L=6, H=3, G=1, P=64, N=128, R=4)
+@pytest.mark.parametrize("R,aligned", [(1, True), (2, True), (3, True), (4, True), (4, False)])
+def test_mimo_decode_steps_at_wide_heads(R, aligned):
+    # P = 64, N = 128: the specialised step when the cache state is 16-byte
+    # aligned, the general mapping when it starts 4 bytes past that
+    inp = make_mimo(21 + R, b=2, L=6, H=4, G=2, P=64, N=128, R=R)
     ref_in, d = prep(inp, "bf16")
     full = oracle.oracle_mimo_fwd(**ref_in)
     L1 = 2

@@ -363,14 +363,15 @@ __global__ void __launch_bounds__(kThreads, 2)
         chunk_params(sm.prm[(c + 1) & 1], pld, pbe, pga, lane);
         if (c + 2 < nC) load_params(c + 2);
       }
+      // descriptors of the operand tiles: an offset inside a tile only adds
+      // (offset >> 4) to the start-address field (shared addresses stay below 256 KB)
+      const uint64_t dC = tc5::desc_sw128(aC, 16, 1024), dB = tc5::desc_sw128(aB, 16, 1024);
+      const uint64_t dH = tc5::desc_sw128(aH, kAtom, 1024), dX = tc5::desc_sw128(aX, kAtom, 1024);
+      const uint64_t dWh = tc5::desc_sw128(aWh, kAtom, 1024), dWl = tc5::desc_sw128(aWl, kAtom, 1024);
+      const uint64_t dM = tc5::desc_sw128(aM, 16, 1024);
       __syncthreads();  // S3: Cbar, Bbar, W_end o Bbar ready
       if (ctrl_lead) {
         tc5::fence_after_sync();
-        // descriptors of the operand tiles: an offset inside a tile only adds
-        // (offset >> 4) to the start-address field (shared addresses stay below 256 KB)
-        const uint64_t dC = tc5::desc_sw128(aC, 16, 1024), dB = tc5::desc_sw128(aB, 16, 1024);
-        const uint64_t dH = tc5::desc_sw128(aH, kAtom, 1024), dX = tc5::desc_sw128(aX, kAtom, 1024);
-        const uint64_t dWh = tc5::desc_sw128(aWh, kAtom, 1024), dWl = tc5::desc_sw128(aWl, kAtom, 1024);
         // G = Cbar Bbar^T (both K-major), K = 128 in 8 steps of 16
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
@@ -391,24 +392,27 @@ __global__ void __launch_bounds__(kThreads, 2)
           tc5::mma_bf16(tmem + kColS, (j < 4 ? dWh : dWl) + kofs, dX + kofs, kIdescS, j > 0);
         }
         tc5::commit(&sm.mbar[1]);
+        // the Gram consumes Bbar: refill it for the next chunk before joining S4
         if (c + 1 < nC) {
-          // the Gram consumes Bbar; Y1 and S consume Cbar and W_end o Bbar (theta's space)
           if (!tc5::mbar_wait(&sm.mbar[0], par, kWaitLimitNs)) sm.err = 1;
           tma_bc(c + 1, &tm.B, aB);
-          if (!tc5::mbar_wait(&sm.mbar[1], par, kWaitLimitNs)) sm.err = 1;
-          tma_bc(c + 1, &tm.C, aC);
-          if (ROT && has_theta) tma_theta(c + 1);
         }
       }
       __syncthreads();  // S4: M ready
       if (ctrl_lead) {
         tc5::fence_after_sync();
-        const uint64_t dM = tc5::desc_sw128(aM, 16, 1024), dX = tc5::desc_sw128(aX, kAtom, 1024);
 #pragma unroll
         for (int j = 0; j < 4; ++j)
           tc5::mma_bf16(tmem + kColY2, dM + (uint64_t)(j * (32 >> 4)), dX + (uint64_t)(j * (2048 >> 4)),
                         kIdescY, j > 0);
         tc5::commit(&sm.mbar[2]);
+        // Y1 and S consume Cbar and W_end o Bbar (theta's space): refill them once
+        // those products are done, after Y2 is on its way
+        if (c + 1 < nC) {
+          if (!tc5::mbar_wait(&sm.mbar[1], par, kWaitLimitNs)) sm.err = 1;
+          tma_bc(c + 1, &tm.C, aC);
+          if (ROT && has_theta) tma_theta(c + 1);
+        }
       }
       continue;
     }
@@ -507,15 +511,17 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     tc5::fence_proxy_async();
     __syncthreads();  // S3: Cbar, Bbar, W_end o Bbar ready
-    if (ROT && tid < NH) sm.Phi[tid] = sm.nPhi[tid];
+    if (ROT && tid >= 2 * NH && tid < 3 * NH) sm.Phi[tid - 2 * NH] = sm.nPhi[tid - 2 * NH];
 
     // -- phase G: masked Gram -> M (rows 16 (warp % 4) + .., columns cb + ..) -------
     {
       // the mask depends only on the chunk scalars: compute it while the Gram runs.
       // Row t = 16 (warp % 4) + lane/4 + 8 hf lies in 8-row block kr = t / 8; column
-      // block kc = cb/8 + q.  Below the diagonal blocks the weight factorises through
+      // block kc = 2 q + warp / 4, so that every warp holds one of the two diagonal
+      // blocks of its rows.  Below the diagonal blocks the weight factorises through
       // the decay at the block's first row (both factors at most 1); the diagonal
       // block takes the direct exponential; blocks with kc > kr are zero.
+      const int cpar = warp >> 2;
       float wv[2][4][2];
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf) {
@@ -524,8 +530,8 @@ __global__ void __launch_bounds__(kThreads, 2)
         const float et = P.et[t];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          const int kc = (cb >> 3) + q;
-          const int s0 = cb + 8 * q + 2 * (lane & 3);
+          const int kc = 2 * q + cpar;
+          const int s0 = 8 * kc + 2 * (lane & 3);
           float w0 = 0.f, w1 = 0.f;
           if (kc < kr) {
             const float2 f = *reinterpret_cast<const float2*>(&P.fs[fs_index(kr, s0)]);
@@ -544,18 +550,20 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
       if (!tc5::mbar_wait(&sm.mbar[0], par, kWaitLimitNs)) sm.err = 1;
       tc5::fence_after_sync();
-      uint32_t gr[16];
-      tc5::ld_16x256b_x4(tmem + tlane + kColG + (uint32_t)cb, gr);
+      uint32_t gr[4][4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        tc5::ld_16x256b_x1(tmem + tlane + kColG + (uint32_t)(8 * (2 * q + cpar)), gr[q]);
       tc5::wait_ld();
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf) {
         const int t = 16 * (warp & 3) + (lane >> 2) + 8 * hf;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          const int s0 = cb + 8 * q + 2 * (lane & 3);
+          const int s0 = 8 * (2 * q + cpar) + 2 * (lane & 3);
           *reinterpret_cast<uint32_t*>(sm.M + off1(t, s0)) =
-              pack_bf16(__uint_as_float(gr[4 * q + 2 * hf]) * wv[hf][q][0],
-                        __uint_as_float(gr[4 * q + 2 * hf + 1]) * wv[hf][q][1]);
+              pack_bf16(__uint_as_float(gr[q][2 * hf]) * wv[hf][q][0],
+                        __uint_as_float(gr[q][2 * hf + 1]) * wv[hf][q][1]);
         }
       }
     }

@@ -197,6 +197,13 @@ __device__ __forceinline__ void ld_32x32b_x32(uint32_t taddr, uint32_t (&r)[32])
       : "r"(taddr));
 }
 // 16x256b.x2: as x4 with g = 0..1 (r[4g .. 4g+3]).
+// 16x256b.x1: thread t gets lanes base + t / 4 (r[0], r[1]) and base + 8 + t / 4
+// (r[2], r[3]), 32-bit columns c + 2 (t % 4) and c + 2 (t % 4) + 1.
+__device__ __forceinline__ void ld_16x256b_x1(uint32_t taddr, uint32_t (&r)[4]) {
+  asm volatile("tcgen05.ld.sync.aligned.16x256b.x1.b32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(taddr));
+}
 __device__ __forceinline__ void ld_16x256b_x2(uint32_t taddr, uint32_t (&r)[8]) {
   asm volatile("tcgen05.ld.sync.aligned.16x256b.x2.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),

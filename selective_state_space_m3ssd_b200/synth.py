@@ -153,3 +153,68 @@ def slice_inputs(inp: dict, b: slice | int, t: slice | int | None = None, heads=
         else:
             out[k] = v
     return out
+
+
+# ---- the Mamba-3 SISO block around the scan -----------------------------------
+
+@dataclass(frozen=True)
+class BlockShape:
+    name: str
+    batch: int
+    seqlen: int
+    d_model: int
+    nheads: int
+    headdim: int
+    dstate: int
+    ngroups: int
+    seed: int
+
+    def with_(self, **kw) -> "BlockShape":
+        return replace(self, **kw)
+
+    @property
+    def in_proj_width(self) -> int:
+        H, P, N, G = self.nheads, self.headdim, self.dstate, self.ngroups
+        return 2 * H * P + 2 * G * N + 2 * H + H * (N // 2)
+
+
+# The block at the model size of the full siso workload: d_model 1024, expand 2
+# (32 heads of 64), N = 128, one B/C group.
+BLOCKS = {
+    "small": BlockShape("siso block b2 L70 d_model 32 H4 P8 N8 G2", 2, 70, 32, 4, 8, 8, 2, 2000),
+    "model": BlockShape("siso block b8 L4096 d_model 1024 H32 P64 N128 G1", 8, 4096, 1024, 32, 64,
+                        128, 1, 2001),
+}
+
+
+def make_block(s: BlockShape, device: str | torch.device = "cpu") -> tuple[torch.Tensor, dict]:
+    """Random-init weights of the block and one input sequence, seeded by ``s.seed``.
+
+    u (b, L, d_model) ~ N(0, 1); W_in (width, d_model) ~ N(0, 1/d_model) and
+    W_out (d_model, H P) ~ N(0, 1/(H P)), all three rounded to bf16 once;
+    dt_bias ~ U(-4, -2), A_log = log U(1, 16), D ~ N(0, 1) per head; the norm
+    weights (N) and the head-specific B/C biases (H, N) ~ U(0.5, 1.5) (the pages
+    initialise the biases to ones; random values exercise them); eps = 1e-6.
+    """
+    g = torch.Generator().manual_seed(s.seed)
+    b, L, dm, H, P, N = s.batch, s.seqlen, s.d_model, s.nheads, s.headdim, s.dstate
+    bf = torch.bfloat16
+    u = torch.randn(b, L, dm, generator=g).to(bf)
+    W_in = (torch.randn(s.in_proj_width, dm, generator=g) / math.sqrt(dm)).to(bf)
+    W_out = (torch.randn(dm, H * P, generator=g) / math.sqrt(H * P)).to(bf)
+    wts = {
+        "W_in": W_in,
+        "W_out": W_out,
+        "dt_bias": torch.rand(H, generator=g) * 2.0 - 4.0,
+        "A_log": torch.log(torch.rand(H, generator=g) * 15.0 + 1.0),
+        "D": torch.randn(H, generator=g),
+        "B_norm_w": torch.rand(N, generator=g) + 0.5,
+        "C_norm_w": torch.rand(N, generator=g) + 0.5,
+        "B_bias": torch.rand(H, N, generator=g) + 0.5,
+        "C_bias": torch.rand(H, N, generator=g) + 0.5,
+        "eps": 1e-6,
+    }
+    if str(device) != "cpu":
+        u = u.to(device)
+        wts = {k: (v.to(device) if isinstance(v, torch.Tensor) else v) for k, v in wts.items()}
+    return u, wts

@@ -62,8 +62,9 @@ def load_peaks() -> dict:
     if os.path.exists(p):
         with open(p) as f:
             d = json.load(f)
-        return {"hbm_gbs": float(d["hbm_gbs"]), "source": "measured"}
-    return {"hbm_gbs": 6650.0, "source": "fallback"}
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
 
 
 def src_sha(path: str) -> str:
@@ -411,6 +412,56 @@ def bench_mimo_decode(dev, rank, peaks: dict, R: int = 4, nsteps: int = 100, rep
             "gpu_launches": 2 * nsteps * replays}
 
 
+def bench_block(dev, rank, peaks: dict, steps: int = 5, warmup: int = 3):
+    """The Mamba-3 SISO block forward (m3ssd_block_fwd: in_proj, prep, scan, gate,
+    out_proj) at model size d_model 1024, b8 L4096, random-init weights;
+    inputs and weights resident in HBM (their sizes exceed L2)."""
+    import selective_state_space_m3ssd_b200 as m3
+    from selective_state_space_m3ssd_b200.synth import BLOCKS, make_block
+    s = BLOCKS["model"].with_(seed=BLOCKS["model"].seed + 7919 * rank)
+    u, wts = make_block(s, device=dev)
+    out = torch.empty_like(u)
+    dims = m3.BlockDims(s.batch, s.seqlen, s.d_model, s.nheads, s.headdim, s.dstate, s.ngroups)
+    ws = torch.empty(m3.block_workspace_size(dims), dtype=torch.uint8, device=dev)
+    for _ in range(warmup):
+        m3.block_fwd(u, wts, out=out, workspace=ws)
+    torch.cuda.synchronize(dev)
+    stream = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        m3.block_fwd(u, wts, out=out, workspace=ws)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / steps
+    M, dm, H, P, N, G = s.batch * s.seqlen, s.d_model, s.nheads, s.headdim, s.dstate, s.ngroups
+    HP, width = H * P, s.in_proj_width
+    # per phase, the least time its own work allows: the two GEMMs at the bf16
+    # peak or their operand bytes at HBM bandwidth, whichever is larger; the
+    # prep, scan and gate kernels by the bytes they must move
+    bw, pt = peaks["hbm_gbs"] * 1e9, peaks["bf16_tflops"] * 1e12
+    t_in = max(2.0 * M * dm * width / pt, (M * dm * 2 + width * dm * 2 + M * width * 4) / bw)
+    t_out = max(2.0 * M * HP * dm / pt, (M * HP * 2 + dm * HP * 2 + M * dm * 2) / bw)
+    prep_b = M * (width * 4 + HP * 2 + 2 * H * N * 2 + 3 * H * 4 + H * (N // 2) * 4)
+    scan_b = M * (2 * HP * 2 + 3 * H * 4 + 2 * H * N * 2 + H * (N // 2) * 4)
+    gate_b = M * HP * (2 + 4 + 2)
+    t_lb = t_in + t_out + (prep_b + scan_b + gate_b) / bw
+    return {"metric": "block Mtokens/s (fwd)", "value": M / (ms / 1e3) / 1e6, "unit": "Mtokens/s",
+            "ms_per_step": ms, "steps": steps,
+            "config": {"workload": s.name, "batch": s.batch, "seqlen": s.seqlen, "d_model": dm,
+                       "nheads": H, "headdim": P, "dstate": N, "ngroups": G, "dtype": "bf16",
+                       "weights": "random init"},
+            "roofline": {"bound": "mixed", "t_lower_bound_ms": t_lb * 1e3,
+                         "frac": t_lb * 1e3 / ms, "peak_hbm_gbs": peaks["hbm_gbs"],
+                         "peak_bf16_tflops": peaks["bf16_tflops"], "peak_source": peaks["source"],
+                         "gemm_tflop_per_step": 2.0 * M * (dm * width + HP * dm) / 1e12,
+                         "note": "sum over phases of max(flops / bf16 peak, bytes / HBM) for the "
+                                 "GEMMs and bytes / HBM for prep, scan (one B/C per head) and gate"},
+            "gpu_launches": 3 * steps,
+            "library_launches": 2 * steps,
+            "note": "own kernels per call: prep, scan, gate; cuBLASLt: in_proj, out_proj"}
+
+
 def bench_backward(w, dev, steps, world, d, peaks):
     """The backward (m3ssd_bwd) on the forward's workload: dY, dhT synthetic,
     every gradient output written; inputs resident in HBM."""
@@ -474,6 +525,7 @@ def run_ours(args):
         fw = bench_forward(w, dev, args.steps, args.warmup, world, rank)
         dec = bench_decode(dev, rank, max(1, args.decode_replays), peaks)
         mimo = bench_mimo_decode(dev, rank, peaks)
+        blk = None if args.no_block else bench_block(dev, rank, peaks)
         bwd = None if args.no_backward else bench_backward(
             w, dev, max(1, min(args.steps, 3)), world, fw["dev_inputs"], peaks)
     e2e = bench_e2e(w, dev, max(1, min(args.steps, 5)), 1, fw["inp"], world)
@@ -496,6 +548,7 @@ def run_ours(args):
         "gpu_launches": fw["launches"],
         "decode": dec,
         "mimo_decode": mimo,
+        "block": blk,
         "backward": bwd,
         "clocks": clk.summary(),
     }
@@ -554,6 +607,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--decode-replays", type=int, default=3,
                     help="replays of the 1000-step decode graph in the timed region")
+    ap.add_argument("--no-block", action="store_true",
+                    help="skip the Mamba-3 SISO block measurement")
     ap.add_argument("--no-backward", action="store_true",
                     help="skip the backward measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true",

@@ -257,6 +257,78 @@ m3ssd_status m3ssd_bwd_noalloc(const m3ssd_dims* dims, const void* X, const floa
                                const float* h0, const m3ssd_fwd_extra* extra, const void* dY,
                                const float* dhT, const m3ssd_bwd_grads* grads, void* stream);
 
+/*
+ * The Mamba-3 SISO block around the scan ("VikramLex/mamba3-minimal" README,
+ * "Architecture", the Mamba3 SSM box; "TorchMamba" README, "API reference",
+ * Mamba3SisoBlock with forward / prefill / step and its cache):
+ *
+ *   zx = u W_in^T                       in_proj, no bias
+ *   [z | x | B | C | dt | lam | theta] = zx   (widths H P, H P, G N, G N, H, H, H N/2;
+ *                                              heads outermost inside each part)
+ *   Delta = softplus(dt + dt_bias), logdecay = -exp(A_log) Delta,
+ *   lambda = sigmoid(lam), gamma = lambda Delta, beta = (1 - lambda) Delta exp(logdecay),
+ *   theta_dt = Delta theta
+ *   B'_h = B_g / sqrt(mean_n B_g^2 + eps) * B_norm_w + B_bias[h]   (QK-norm, then the
+ *   C'_h likewise                                                   head-specific BC bias)
+ *   y = scan(x, logdecay, beta, gamma, B', C', theta_dt, D)        (the SISO scan above,
+ *                                                                    one B/C per head)
+ *   out = (y * SiLU(z)) W_out^T          out_proj, no bias
+ *
+ * The projections are plain GEMMs run by cuBLASLt (bf16 operands, fp32
+ * accumulation; in_proj writes fp32, out_proj bf16); the rest runs in this
+ * library's kernels.  u and out are bf16.  The block cache is an m3ssd_cache
+ * whose b_prev is per HEAD: (b, H, N) holding B'_{t-1} unrotated.
+ */
+typedef struct {
+  int64_t batch;    /* b >= 0 */
+  int64_t seqlen;   /* L >= 0 (ignored by m3ssd_block_step) */
+  int64_t d_model;  /* >= 1, a multiple of 8 */
+  int64_t nheads;   /* H >= 1 */
+  int64_t headdim;  /* P >= 1, H * P a multiple of 8 */
+  int64_t dstate;   /* N >= 2, even */
+  int64_t ngroups;  /* G >= 1, H % G == 0 */
+} m3ssd_block_dims;
+
+typedef struct {
+  const void* W_in;       /* (2HP + 2GN + 2H + H N/2, d_model) bf16, row-major */
+  const void* W_out;      /* (d_model, H P) bf16, row-major */
+  const float* dt_bias;   /* (H) */
+  const float* A_log;     /* (H) */
+  const float* D;         /* (H), may be NULL (zero) */
+  const float* B_norm_w;  /* (N) */
+  const float* C_norm_w;  /* (N) */
+  const float* B_bias;    /* (H, N) */
+  const float* C_bias;    /* (H, N) */
+  float eps;              /* >= 0 */
+} m3ssd_block_weights;
+
+/* Bytes of device workspace m3ssd_block_fwd needs for these dims (with
+ * seqlen = 1 it also covers m3ssd_block_step); 0 for invalid dims. */
+size_t m3ssd_block_workspace_size(const m3ssd_block_dims* dims);
+
+/*
+ * Block forward over a sequence (Mamba3SisoBlock.forward; with cache_out it is
+ * prefill).  u, out: (b, L, d_model) bf16.  cache_in (may be NULL: start from
+ * zero) is the state the sequence continues from; cache_out (may be NULL) gets
+ * the state after the last token and may be the same object as cache_in.
+ * workspace: workspace_bytes >= m3ssd_block_workspace_size(dims), 256-byte
+ * aligned, not read afterwards.  Errors as m3ssd_fwd; a cuBLASLt failure
+ * returns M3SSD_ERR_CUDA.
+ */
+m3ssd_status m3ssd_block_fwd(const m3ssd_block_dims* dims, const m3ssd_block_weights* w,
+                             const void* u, void* out, const m3ssd_cache* cache_in,
+                             const m3ssd_cache* cache_out, void* workspace,
+                             size_t workspace_bytes, void* stream);
+
+/*
+ * One decode step of the block (Mamba3SisoBlock.step): u_t, out_t (b, d_model)
+ * bf16; cache (required) is advanced in place.  workspace as for
+ * m3ssd_block_fwd with seqlen = 1.  Capturable in a CUDA graph.
+ */
+m3ssd_status m3ssd_block_step(const m3ssd_block_dims* dims, const m3ssd_block_weights* w,
+                              const void* u_t, void* out_t, const m3ssd_cache* cache,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
 /* Number of bounded device-side waits of the chunked forward that ran out
  * (each makes its CTA stop and leave its outputs unwritten) since the last
  * call; the count is then reset.  This call synchronises the current device

@@ -30,6 +30,14 @@ Readings where the pages are silent (each is listed in the design notes):
     applied per group; the head bias is added after it, so each head gets its
     own B and C (the scan runs with G = H) and the cache's b_prev is per head.
 
+Storage precision: the pages' numerics policy ("TorchMamba" README,
+"Behavioral notes": bf16 computes in fp32 and each output is downcast to the
+input dtype) makes the tensors a bf16 block hands from one step to the next
+bf16.  ``store`` (default: none) is applied to exactly those hand-offs -- x,
+B', C' (the scan's bf16 inputs), the scan output y and the gated product
+(out_proj's input) -- so that a test can compare against a device path that
+stores them in bf16; everything else stays fp64.
+
 Numerical pins: ``tests/test_oracle_block.py`` (closed forms for one and two
 tokens, the scale invariance of the norm, forward == prefill + steps, and
 planted mistakes).
@@ -75,7 +83,11 @@ def bc_norm(v, w, eps):
     return v / np.sqrt(np.mean(v * v, axis=-1, keepdims=True) + eps) * w
 
 
-def scan_inputs(u, wts, H, P, N, G):
+def _keep(v):
+    return v
+
+
+def scan_inputs(u, wts, H, P, N, G, store=_keep):
     """Steps 1-2 of the block: the scan's inputs from the block input u (..., d_model)."""
     f = lambda k: np.asarray(wts[k], dtype=np.float64)
     zx = np.asarray(u, dtype=np.float64) @ f("W_in").T
@@ -91,8 +103,8 @@ def scan_inputs(u, wts, H, P, N, G):
     grp = np.arange(H) // (H // G)
     Bh = bc_norm(s["B"], f("B_norm_w"), eps)[..., grp, :] + f("B_bias")
     Ch = bc_norm(s["C"], f("C_norm_w"), eps)[..., grp, :] + f("C_bias")
-    return {"z": s["z"], "X": s["x"], "logdecay": logdecay, "beta": beta, "gamma": gamma,
-            "B": Bh, "C": Ch, "theta": theta}
+    return {"z": s["z"], "X": store(s["x"]), "logdecay": logdecay, "beta": beta, "gamma": gamma,
+            "B": store(Bh), "C": store(Ch), "theta": theta}
 
 
 def new_block_cache(b, H, P, N):
@@ -102,31 +114,32 @@ def new_block_cache(b, H, P, N):
             "x_prev": np.zeros((b, H, P)), "b_prev": np.zeros((b, H, N))}
 
 
-def oracle_block_fwd(u, wts, H, P, N, G, cache=None):
+def oracle_block_fwd(u, wts, H, P, N, G, cache=None, store=_keep):
     """Block forward over a sequence: u (b, L, d_model) -> out (b, L, d_model).
 
     ``cache`` (optional, a dict as from :func:`new_block_cache`) is the state
-    the sequence continues from.  Returns (out, cache after the last token)."""
+    the sequence continues from; ``store`` rounds the bf16 hand-offs (see the
+    module notes).  Returns (out, cache after the last token)."""
     u = np.asarray(u, dtype=np.float64)
     b = u.shape[0]
-    si = scan_inputs(u, wts, H, P, N, G)
+    si = scan_inputs(u, wts, H, P, N, G, store)
     c = cache if cache is not None else new_block_cache(b, H, P, N)
     r = oracle_fwd(si["X"], si["logdecay"], si["beta"], si["gamma"], si["B"], si["C"],
                    si["theta"], np.asarray(wts["D"], dtype=np.float64), c["ssm"],
                    angle0=c["angle"], xprev0=c["x_prev"], bprev0=c["b_prev"])
-    gated = r["Y"] * silu(si["z"])
+    gated = store(store(r["Y"]) * silu(si["z"]))
     out = gated.reshape(gated.shape[:2] + (H * P,)) @ np.asarray(wts["W_out"], dtype=np.float64).T
     return out, {"angle": r["angleT"], "ssm": r["hT"], "x_prev": r["xprevT"],
                  "b_prev": r["bprevT"]}
 
 
-def oracle_block_step(u_t, wts, H, P, N, G, cache):
+def oracle_block_step(u_t, wts, H, P, N, G, cache, store=_keep):
     """One decode step of the block: u_t (b, d_model) -> out_t (b, d_model);
     ``cache`` (float64 arrays) is updated in place."""
     u_t = np.asarray(u_t, dtype=np.float64)
-    si = scan_inputs(u_t, wts, H, P, N, G)
+    si = scan_inputs(u_t, wts, H, P, N, G, store)
     y = oracle_step(cache, si["X"], si["logdecay"], si["beta"], si["gamma"], si["B"], si["C"],
                     si["theta"], np.asarray(wts["D"], dtype=np.float64))
-    gated = y * silu(si["z"])
+    gated = store(store(y) * silu(si["z"]))
     return gated.reshape(gated.shape[:1] + (H * P,)) @ np.asarray(wts["W_out"],
                                                                   dtype=np.float64).T

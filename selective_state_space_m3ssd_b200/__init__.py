@@ -62,6 +62,19 @@ class Cache(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in ("angle", "ssm", "x_prev", "b_prev")]
 
 
+class BlockDims(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int64) for n in
+                ("batch", "seqlen", "d_model", "nheads", "headdim", "dstate", "ngroups")]
+
+
+BLOCK_WEIGHT_NAMES = ("W_in", "W_out", "dt_bias", "A_log", "D", "B_norm_w", "C_norm_w",
+                      "B_bias", "C_bias")
+
+
+class BlockWeights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in BLOCK_WEIGHT_NAMES] + [("eps", ctypes.c_float)]
+
+
 def load(path: str | None = None):
     """Load ``libm3ssd.so`` (once) and declare the C signatures."""
     global _lib
@@ -96,6 +109,15 @@ def load(path: str | None = None):
         lib.m3ssd_bwd_noalloc.argtypes = [ctypes.POINTER(Dims)] + [vp] * 9 + \
             [ctypes.POINTER(FwdExtra), vp, vp, ctypes.POINTER(BwdGrads), vp]
         lib.m3ssd_bwd_noalloc.restype = ctypes.c_int
+        lib.m3ssd_block_workspace_size.argtypes = [ctypes.POINTER(BlockDims)]
+        lib.m3ssd_block_workspace_size.restype = sz
+        lib.m3ssd_block_fwd.argtypes = [ctypes.POINTER(BlockDims), ctypes.POINTER(BlockWeights),
+                                        vp, vp, ctypes.POINTER(Cache), ctypes.POINTER(Cache),
+                                        vp, sz, vp]
+        lib.m3ssd_block_fwd.restype = ctypes.c_int
+        lib.m3ssd_block_step.argtypes = [ctypes.POINTER(BlockDims), ctypes.POINTER(BlockWeights),
+                                         vp, vp, ctypes.POINTER(Cache), vp, sz, vp]
+        lib.m3ssd_block_step.restype = ctypes.c_int
         lib.m3ssd_status_string.argtypes = [ctypes.c_int]
         lib.m3ssd_status_string.restype = ctypes.c_char_p
         lib.m3ssd_abi_version.argtypes = []
@@ -443,6 +465,108 @@ def mimo_step(cache: dict, x_t, logdecay_t, beta_t, gamma_t, B_t, C_t, theta_t=N
                                 ctypes.byref(c), _ptr(y_t), _stream_handle(dev))
     _check(st, "m3ssd_mimo_step")
     return y_t
+
+
+# ---- the Mamba-3 SISO block around the scan --------------------------------------
+
+def block_in_proj_width(nheads, headdim, dstate, ngroups) -> int:
+    """Rows of W_in: z, x (H P each), B, C (G N each), dt, lam (H each), theta (H N/2)."""
+    return 2 * nheads * headdim + 2 * ngroups * dstate + 2 * nheads + nheads * (dstate // 2)
+
+
+def _block_args(u, wts, seqlen):
+    import torch
+    b, dm = u.shape[0], u.shape[-1]
+    H = wts["A_log"].shape[0]
+    N = wts["B_norm_w"].shape[0]
+    HP = wts["W_out"].shape[1]
+    if HP % H:
+        raise ValueError("W_out's columns must be H * P")
+    P = HP // H
+    width = wts["W_in"].shape[0]
+    rest = width - 2 * HP - 2 * H - H * (N // 2)
+    if rest <= 0 or rest % (2 * N):
+        raise ValueError("W_in's rows do not match any group count")
+    G = rest // (2 * N)
+    dev = u.device
+    f32, bf = torch.float32, torch.bfloat16
+    _need(u, "u", bf, device=dev)
+    _need(wts["W_in"], "W_in", bf, (width, dm), dev)
+    _need(wts["W_out"], "W_out", bf, (dm, HP), dev)
+    for k, shape in (("dt_bias", (H,)), ("A_log", (H,)), ("B_norm_w", (N,)), ("C_norm_w", (N,)),
+                     ("B_bias", (H, N)), ("C_bias", (H, N))):
+        _need(wts[k], k, f32, shape, dev)
+    _need(wts.get("D"), "D", f32, (H,), dev)
+    dims = BlockDims(b, seqlen, dm, H, P, N, G)
+    w = BlockWeights(*[(None if wts.get(k) is None else wts[k].data_ptr())
+                       for k in BLOCK_WEIGHT_NAMES], float(wts.get("eps", 1e-6)))
+    return dims, w, (H, P, N, G)
+
+
+def new_block_cache(batch, nheads, headdim, dstate, device):
+    """A zeroed block cache: angle (b,H,N/2), ssm (b,H,N,P), x_prev (b,H,P) and
+    the per-head b_prev (b,H,N), all fp32."""
+    return new_cache(batch, nheads, headdim, dstate, nheads, device)
+
+
+def _cache_struct(cache, b, H, P, N, dev, name):
+    import torch
+    f32 = torch.float32
+    _need(cache["angle"], name + ".angle", f32, (b, H, N // 2), dev)
+    _need(cache["ssm"], name + ".ssm", f32, (b, H, N, P), dev)
+    _need(cache["x_prev"], name + ".x_prev", f32, (b, H, P), dev)
+    _need(cache["b_prev"], name + ".b_prev", f32, (b, H, N), dev)
+    return Cache(cache["angle"].data_ptr(), cache["ssm"].data_ptr(), cache["x_prev"].data_ptr(),
+                 cache["b_prev"].data_ptr())
+
+
+def block_workspace_size(dims: BlockDims) -> int:
+    return int(load().m3ssd_block_workspace_size(ctypes.byref(dims)))
+
+
+def block_fwd(u, wts: dict, *, cache_in=None, cache_out=None, out=None, workspace=None):
+    """Forward of the Mamba-3 SISO block through ``m3ssd_block_fwd``: u (b, L,
+    d_model) bf16 -> out (b, L, d_model) bf16.  ``cache_in`` / ``cache_out``
+    (dicts as from :func:`new_block_cache`, may be the same dict) continue from
+    and hand back the decode state.  ``workspace`` (uint8, 256-byte aligned) is
+    allocated by torch when not given."""
+    import torch
+    b, L, dm = u.shape
+    dims, w, (H, P, N, G) = _block_args(u, wts, L)
+    dev = u.device
+    out = torch.empty_like(u) if out is None else out
+    _need(out, "out", torch.bfloat16, (b, L, dm), dev)
+    ci = None if cache_in is None else _cache_struct(cache_in, b, H, P, N, dev, "cache_in")
+    co = None if cache_out is None else _cache_struct(cache_out, b, H, P, N, dev, "cache_out")
+    need = block_workspace_size(dims)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    st = load().m3ssd_block_fwd(ctypes.byref(dims), ctypes.byref(w), _ptr(u), _ptr(out),
+                                None if ci is None else ctypes.byref(ci),
+                                None if co is None else ctypes.byref(co), _ptr(workspace),
+                                workspace.numel(), _stream_handle(dev))
+    _check(st, "m3ssd_block_fwd")
+    return out
+
+
+def block_step(cache: dict, u_t, wts: dict, *, out_t=None, workspace=None):
+    """One decode step of the block through ``m3ssd_block_step``: u_t (b,
+    d_model) bf16 -> out_t; ``cache`` is advanced in place."""
+    import torch
+    b, dm = u_t.shape
+    dims, w, (H, P, N, G) = _block_args(u_t, wts, 1)
+    dev = u_t.device
+    out_t = torch.empty_like(u_t) if out_t is None else out_t
+    _need(out_t, "out_t", torch.bfloat16, (b, dm), dev)
+    c = _cache_struct(cache, b, H, P, N, dev, "cache")
+    need = block_workspace_size(dims)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    st = load().m3ssd_block_step(ctypes.byref(dims), ctypes.byref(w), _ptr(u_t), _ptr(out_t),
+                                 ctypes.byref(c), _ptr(workspace), workspace.numel(),
+                                 _stream_handle(dev))
+    _check(st, "m3ssd_block_step")
+    return out_t
 
 
 class PreparedFwd:

@@ -3,7 +3,8 @@
 ``python -m selective_state_space_m3ssd_b200.build [--force] [--verbose]``
 compiles every ``csrc/*.cu`` to an object under ``_build/`` (in parallel) and
 links them into ``selective_state_space_m3ssd_b200/libm3ssd.so``.  The CUDA
-runtime is linked statically, so the library needs only the driver at run time.
+runtime is linked statically; cuBLASLt (the block's two projections) is the
+one shared library it loads, from the toolkit's lib64.
 """
 from __future__ import annotations
 
@@ -24,6 +25,15 @@ HEADER = os.path.join(ROOT, "include", "m3ssd.h")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2",
                 "--expt-relaxed-constexpr", "-I", os.path.join(ROOT, "include")]
+
+
+def _cuda_lib() -> str:
+    return os.path.join(os.environ.get("CUDA_HOME", "/usr/local/cuda"), "lib64")
+
+
+# cuBLASLt runs the block's two projections (plain GEMMs); it is the only
+# library linked dynamically, found through the toolkit's lib64 at run time.
+LINK = ["-L" + _cuda_lib(), "-lcublasLt", "-Xlinker", "-rpath," + _cuda_lib()]
 
 
 def nvcc() -> str:
@@ -65,7 +75,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
     with cf.ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
         objs = list(ex.map(lambda s: _compile(s, verbose), sources()))
     tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc()] + ARCH + ["-shared", "-cudart", "static", "-o", tmp] + objs
+    cmd = [nvcc()] + ARCH + ["-shared", "-cudart", "static", "-o", tmp] + objs + LINK
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stderr}")

@@ -1,0 +1,375 @@
+// The Mamba-3 SISO block around the scan.
+//
+// "VikramLex/mamba3-minimal" README, "Architecture" (the Mamba3 SSM box:
+// in_proj -> (z, x, B, C, Delta, lambda, theta); B, C: QK-norm -> +bias ->
+// RoPE; trapezoidal SSD; y + D x -> y * SiLU(z) -> out) and "TorchMamba"
+// README, "API reference" (Mamba3SisoBlock with forward / prefill / step and
+// Mamba3SisoCache).  The two projections are plain GEMMs and run in cuBLASLt
+// (bf16 operands, fp32 accumulation); everything between them runs here:
+//
+//   block_prep_kernel   one CTA per token: splits the fp32 in_proj row, writes x
+//                       (bf16), the per-head B' and C' (QK-norm of the group's
+//                       vector times the norm weight plus the head's bias, bf16),
+//                       logdecay, beta, gamma (fp32) and theta_dt (fp32);
+//   m3ssd_fwd / m3ssd_step of this library on those tensors (one B/C per head);
+//   block_gate_kernel   y * SiLU(z) (bf16), the input of out_proj.
+#include <cublasLt.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <mutex>
+
+#include "../../include/m3ssd.h"
+#include "common.cuh"
+
+namespace m3ssd {
+namespace {
+
+constexpr size_t kLtWorkspace = size_t(32) << 20;
+constexpr int kPrepThreads = 256;
+
+size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
+
+int64_t in_proj_width(const m3ssd_block_dims* d) {
+  return 2 * d->nheads * d->headdim + 2 * d->ngroups * d->dstate + 2 * d->nheads +
+         d->nheads * (d->dstate / 2);
+}
+
+// Workspace regions (byte offsets) for M tokens.
+struct BlockWs {
+  size_t zx, x, B, C, ld, be, ga, th, y, bp, lt, total;
+};
+BlockWs block_ws(const m3ssd_block_dims* d, int64_t M) {
+  const size_t H = (size_t)d->nheads, P = (size_t)d->headdim, N = (size_t)d->dstate;
+  const size_t m = (size_t)M;
+  BlockWs w{};
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t r = o;
+    o += al256(bytes);
+    return r;
+  };
+  w.zx = take(m * (size_t)in_proj_width(d) * 4);
+  w.x = take(m * H * P * 2);   // x, then y * SiLU(z)
+  w.B = take(m * H * N * 2);
+  w.C = take(m * H * N * 2);
+  w.ld = take(m * H * 4);
+  w.be = take(m * H * 4);
+  w.ga = take(m * H * 4);
+  w.th = take(m * H * (N / 2) * 4);
+  w.y = take(m * H * P * 2);
+  w.bp = take((size_t)d->batch * H * N * 4);  // copy of the incoming b_prev
+  w.lt = take(kLtWorkspace);
+  w.total = o;
+  return w;
+}
+
+struct PrepArgs {
+  int64_t M, H, P, N, G, width;
+  const float* zx;
+  const float* dt_bias;
+  const float* A_log;
+  const float* Bw;
+  const float* Cw;
+  const float* Bbias;
+  const float* Cbias;
+  float eps;
+  __nv_bfloat16* X;
+  __nv_bfloat16* B;
+  __nv_bfloat16* C;
+  float* ld;
+  float* be;
+  float* ga;
+  float* th;
+};
+
+__device__ __forceinline__ float softplus_f(float v) { return v > 20.f ? v : log1pf(expf(v)); }
+
+// One CTA per token.  Shared memory: 2G inverse RMS values (B groups, then C
+// groups) and the H step sizes Delta.
+__global__ void __launch_bounds__(kPrepThreads) block_prep_kernel(PrepArgs a) {
+  extern __shared__ float sh[];
+  const int64_t tok = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int H = (int)a.H, P = (int)a.P, N = (int)a.N, G = (int)a.G, NH = N / 2;
+  const int HP = H * P, GN = G * N;
+  const int oB = 2 * HP, oC = oB + GN, odt = oC + GN, olam = odt + H, oth = olam + H;
+  const float* row = a.zx + tok * a.width;
+  float* inv = sh;
+  float* delta = sh + 2 * G;
+
+  for (int j = warp; j < 2 * G; j += kPrepThreads / 32) {
+    const float* v = row + (j < G ? oB + j * N : oC + (j - G) * N);
+    float ss = 0.f;
+    for (int n = lane; n < N; n += 32) ss = fmaf(v[n], v[n], ss);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if (lane == 0) inv[j] = 1.f / sqrtf(ss / (float)N + a.eps);
+  }
+  for (int h = tid; h < H; h += kPrepThreads) {
+    const float dl = softplus_f(row[odt + h] + a.dt_bias[h]);
+    const float lg = -expf(a.A_log[h]) * dl;
+    const float lam = 1.f / (1.f + expf(-row[olam + h]));
+    a.ld[tok * H + h] = lg;
+    a.ga[tok * H + h] = lam * dl;
+    a.be[tok * H + h] = (1.f - lam) * dl * expf(lg);
+    delta[h] = dl;
+  }
+  for (int k = tid; k < HP; k += kPrepThreads) a.X[tok * HP + k] = __float2bfloat16_rn(row[HP + k]);
+  __syncthreads();
+  const int hpg = H / G;
+  for (int k = tid; k < H * N; k += kPrepThreads) {
+    const int h = k / N, n = k - h * N, g = h / hpg;
+    a.B[tok * H * N + k] = __float2bfloat16_rn(fmaf(row[oB + g * N + n] * inv[g], a.Bw[n], a.Bbias[k]));
+    a.C[tok * H * N + k] =
+        __float2bfloat16_rn(fmaf(row[oC + g * N + n] * inv[G + g], a.Cw[n], a.Cbias[k]));
+  }
+  for (int k = tid; k < H * NH; k += kPrepThreads) a.th[tok * H * NH + k] = delta[k / NH] * row[oth + k];
+}
+
+// y * SiLU(z), z read from the fp32 in_proj rows.
+__global__ void block_gate_kernel(const __nv_bfloat16* __restrict__ y, const float* __restrict__ zx,
+                                  int64_t width, int64_t HP, int64_t M,
+                                  __nv_bfloat16* __restrict__ out) {
+  const int64_t n = M * HP, stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) {
+    const int64_t tok = i / HP, k = i - tok * HP;
+    const float z = zx[tok * width + k];
+    out[i] = __float2bfloat16_rn(__bfloat162float(y[i]) * z / (1.f + expf(-z)));
+  }
+}
+
+cublasLtHandle_t lt_handle() {
+  static std::once_flag once;
+  static cublasLtHandle_t h = nullptr;
+  std::call_once(once, [] {
+    if (cublasLtCreate(&h) != CUBLAS_STATUS_SUCCESS) h = nullptr;
+  });
+  return h;
+}
+
+// D (M x Nout, row-major, type dt) = A (M x K, bf16, row-major) W^T, with W
+// (Nout x K, bf16, row-major) -- in cuBLASLt's column-major terms
+// D^T = op_T(W) A^T.  Returns false if cuBLASLt refuses or fails.
+bool gemm_bf16(int64_t M, int64_t Nout, int64_t K, const void* A, const void* W, void* D,
+               cudaDataType_t dt, void* ws, size_t ws_bytes, cudaStream_t s) {
+  cublasLtHandle_t h = lt_handle();
+  if (!h) return false;
+  cublasLtMatmulDesc_t op = nullptr;
+  cublasLtMatrixLayout_t la = nullptr, lb = nullptr, lc = nullptr;
+  cublasLtMatmulPreference_t pref = nullptr;
+  bool ok = false;
+  do {
+    if (cublasLtMatmulDescCreate(&op, CUBLAS_COMPUTE_32F, CUDA_R_32F) != CUBLAS_STATUS_SUCCESS) break;
+    const cublasOperation_t ta = CUBLAS_OP_T, tb = CUBLAS_OP_N;
+    if (cublasLtMatmulDescSetAttribute(op, CUBLASLT_MATMUL_DESC_TRANSA, &ta, sizeof(ta)) !=
+            CUBLAS_STATUS_SUCCESS ||
+        cublasLtMatmulDescSetAttribute(op, CUBLASLT_MATMUL_DESC_TRANSB, &tb, sizeof(tb)) !=
+            CUBLAS_STATUS_SUCCESS)
+      break;
+    if (cublasLtMatrixLayoutCreate(&la, CUDA_R_16BF, (uint64_t)K, (uint64_t)Nout, K) !=
+            CUBLAS_STATUS_SUCCESS ||
+        cublasLtMatrixLayoutCreate(&lb, CUDA_R_16BF, (uint64_t)K, (uint64_t)M, K) !=
+            CUBLAS_STATUS_SUCCESS ||
+        cublasLtMatrixLayoutCreate(&lc, dt, (uint64_t)Nout, (uint64_t)M, Nout) !=
+            CUBLAS_STATUS_SUCCESS)
+      break;
+    if (cublasLtMatmulPreferenceCreate(&pref) != CUBLAS_STATUS_SUCCESS) break;
+    if (cublasLtMatmulPreferenceSetAttribute(pref, CUBLASLT_MATMUL_PREF_MAX_WORKSPACE_BYTES,
+                                             &ws_bytes, sizeof(ws_bytes)) != CUBLAS_STATUS_SUCCESS)
+      break;
+    cublasLtMatmulHeuristicResult_t res{};
+    int found = 0;
+    if (cublasLtMatmulAlgoGetHeuristic(h, op, la, lb, lc, lc, pref, 1, &res, &found) !=
+            CUBLAS_STATUS_SUCCESS ||
+        found == 0)
+      break;
+    const float alpha = 1.f, beta = 0.f;
+    if (cublasLtMatmul(h, op, &alpha, W, la, A, lb, &beta, D, lc, D, lc, &res.algo, ws, ws_bytes,
+                       s) != CUBLAS_STATUS_SUCCESS)
+      break;
+    ok = true;
+  } while (false);
+  if (pref) cublasLtMatmulPreferenceDestroy(pref);
+  if (lc) cublasLtMatrixLayoutDestroy(lc);
+  if (lb) cublasLtMatrixLayoutDestroy(lb);
+  if (la) cublasLtMatrixLayoutDestroy(la);
+  if (op) cublasLtMatmulDescDestroy(op);
+  return ok;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+m3ssd_status check_block(const m3ssd_block_dims* d, const m3ssd_block_weights* w) {
+  if (!d || !w) return M3SSD_ERR_INVALID_ARG;
+  if (d->batch < 0 || d->seqlen < 0 || d->d_model < 1 || d->nheads < 1 || d->headdim < 1 ||
+      d->ngroups < 1)
+    return M3SSD_ERR_INVALID_ARG;
+  if (d->dstate < 2 || d->dstate % 2 != 0 || d->nheads % d->ngroups != 0)
+    return M3SSD_ERR_INVALID_ARG;
+  if (d->d_model % 8 != 0 || (d->nheads * d->headdim) % 8 != 0) return M3SSD_ERR_UNSUPPORTED;
+  if (!(w->eps >= 0.f)) return M3SSD_ERR_INVALID_ARG;
+  if (!w->W_in || !w->W_out || !w->dt_bias || !w->A_log || !w->B_norm_w || !w->C_norm_w ||
+      !w->B_bias || !w->C_bias)
+    return M3SSD_ERR_INVALID_ARG;
+  if (!aligned(w->W_in, 16) || !aligned(w->W_out, 16)) return M3SSD_ERR_INVALID_ARG;
+  const void* f32[] = {w->dt_bias, w->A_log, w->D, w->B_norm_w, w->C_norm_w, w->B_bias, w->C_bias};
+  for (const void* p : f32)
+    if (!aligned(p, 4)) return M3SSD_ERR_INVALID_ARG;
+  if (d->batch * d->seqlen > INT32_MAX) return M3SSD_ERR_UNSUPPORTED;
+  return M3SSD_OK;
+}
+
+m3ssd_dims scan_dims(const m3ssd_block_dims* d, int64_t L) {
+  m3ssd_dims s{};
+  s.batch = d->batch;
+  s.seqlen = L;
+  s.nheads = d->nheads;
+  s.headdim = d->headdim;
+  s.dstate = d->dstate;
+  s.ngroups = d->nheads;  // one B'/C' per head (the bias is head-specific)
+  s.chunk = 0;
+  s.x_dtype = M3SSD_BF16;
+  return s;
+}
+
+// in_proj, the prep kernel; returns the scan inputs' pointers through ws.
+m3ssd_status front(const m3ssd_block_dims* d, const m3ssd_block_weights* w, const void* u,
+                   int64_t M, char* base, const BlockWs& ws, cudaStream_t s) {
+  const int64_t width = in_proj_width(d);
+  if (!gemm_bf16(M, width, d->d_model, u, w->W_in, base + ws.zx, CUDA_R_32F, base + ws.lt,
+                 kLtWorkspace, s))
+    return M3SSD_ERR_CUDA;
+  PrepArgs a{};
+  a.M = M; a.H = d->nheads; a.P = d->headdim; a.N = d->dstate; a.G = d->ngroups; a.width = width;
+  a.zx = reinterpret_cast<const float*>(base + ws.zx);
+  a.dt_bias = w->dt_bias; a.A_log = w->A_log; a.Bw = w->B_norm_w; a.Cw = w->C_norm_w;
+  a.Bbias = w->B_bias; a.Cbias = w->C_bias; a.eps = w->eps;
+  a.X = reinterpret_cast<__nv_bfloat16*>(base + ws.x);
+  a.B = reinterpret_cast<__nv_bfloat16*>(base + ws.B);
+  a.C = reinterpret_cast<__nv_bfloat16*>(base + ws.C);
+  a.ld = reinterpret_cast<float*>(base + ws.ld);
+  a.be = reinterpret_cast<float*>(base + ws.be);
+  a.ga = reinterpret_cast<float*>(base + ws.ga);
+  a.th = reinterpret_cast<float*>(base + ws.th);
+  const size_t smem = sizeof(float) * (size_t)(2 * d->ngroups + d->nheads);
+  if (smem > 48 * 1024) return M3SSD_ERR_UNSUPPORTED;
+  block_prep_kernel<<<(unsigned)M, kPrepThreads, smem, s>>>(a);
+  return cudaGetLastError() == cudaSuccess ? M3SSD_OK : M3SSD_ERR_CUDA;
+}
+
+// y * SiLU(z) into the x region, then out_proj.
+m3ssd_status back(const m3ssd_block_dims* d, const m3ssd_block_weights* w, int64_t M, char* base,
+                  const BlockWs& ws, void* out, cudaStream_t s) {
+  const int64_t HP = d->nheads * d->headdim;
+  const int64_t n = M * HP;
+  const unsigned grid = (unsigned)((n + 255) / 256 < 148 * 16 ? (n + 255) / 256 : 148 * 16);
+  block_gate_kernel<<<grid, 256, 0, s>>>(reinterpret_cast<const __nv_bfloat16*>(base + ws.y),
+                                         reinterpret_cast<const float*>(base + ws.zx),
+                                         in_proj_width(d), HP, M,
+                                         reinterpret_cast<__nv_bfloat16*>(base + ws.x));
+  if (cudaGetLastError() != cudaSuccess) return M3SSD_ERR_CUDA;
+  if (!gemm_bf16(M, d->d_model, HP, base + ws.x, w->W_out, out, CUDA_R_16BF, base + ws.lt,
+                 kLtWorkspace, s))
+    return M3SSD_ERR_CUDA;
+  return M3SSD_OK;
+}
+
+}  // namespace
+}  // namespace m3ssd
+
+extern "C" {
+
+size_t m3ssd_block_workspace_size(const m3ssd_block_dims* dims) {
+  if (!dims || dims->batch < 0 || dims->seqlen < 0 || dims->nheads < 1 || dims->headdim < 1 ||
+      dims->dstate < 2 || dims->ngroups < 1)
+    return 0;
+  const int64_t L = dims->seqlen > 0 ? dims->seqlen : 1;
+  return m3ssd::block_ws(dims, dims->batch * L).total;
+}
+
+m3ssd_status m3ssd_block_fwd(const m3ssd_block_dims* dims, const m3ssd_block_weights* w,
+                             const void* u, void* out, const m3ssd_cache* cache_in,
+                             const m3ssd_cache* cache_out, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+  using namespace m3ssd;
+  m3ssd_status st = check_block(dims, w);
+  if (st != M3SSD_OK) return st;
+  const int64_t M = dims->batch * dims->seqlen;
+  if (M > 0 && (!u || !out || !aligned(u, 16) || !aligned(out, 16))) return M3SSD_ERR_INVALID_ARG;
+  if (cache_in && (!cache_in->angle || !cache_in->ssm || !cache_in->x_prev || !cache_in->b_prev))
+    return M3SSD_ERR_INVALID_ARG;
+  if (cache_out &&
+      (!cache_out->angle || !cache_out->ssm || !cache_out->x_prev || !cache_out->b_prev))
+    return M3SSD_ERR_INVALID_ARG;
+  const size_t need = m3ssd_block_workspace_size(dims);
+  if (workspace_bytes < need || !workspace || !aligned(workspace, 256)) return M3SSD_ERR_WORKSPACE;
+  if (dims->batch == 0) return M3SSD_OK;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const BlockWs ws = block_ws(dims, M > 0 ? M : dims->batch);
+  char* base = static_cast<char*>(workspace);
+  if (M > 0) {
+    st = front(dims, w, u, M, base, ws, s);
+    if (st != M3SSD_OK) return st;
+  }
+  // the scan; the incoming b_prev is copied first, so that the outgoing one may
+  // overwrite the same buffer
+  const m3ssd_dims sd = scan_dims(dims, dims->seqlen);
+  m3ssd_fwd_extra ex{};
+  if (cache_in) {
+    const size_t bytes = (size_t)dims->batch * dims->nheads * dims->dstate * sizeof(float);
+    if (cudaMemcpyAsync(base + ws.bp, cache_in->b_prev, bytes, cudaMemcpyDeviceToDevice, s) !=
+        cudaSuccess)
+      return M3SSD_ERR_CUDA;
+    ex.angle0 = cache_in->angle;
+    ex.xprev0 = cache_in->x_prev;
+    ex.bprev0 = reinterpret_cast<const float*>(base + ws.bp);
+  }
+  if (cache_out) {
+    ex.angleT = cache_out->angle;
+    ex.xprevT = cache_out->x_prev;
+    ex.bprevT = cache_out->b_prev;
+  }
+  st = m3ssd_fwd(&sd, base + ws.x, reinterpret_cast<const float*>(base + ws.ld),
+                 reinterpret_cast<const float*>(base + ws.be),
+                 reinterpret_cast<const float*>(base + ws.ga), base + ws.B, base + ws.C,
+                 reinterpret_cast<const float*>(base + ws.th), w->D,
+                 cache_in ? cache_in->ssm : nullptr, base + ws.y,
+                 cache_out ? cache_out->ssm : nullptr, &ex, nullptr, 0, stream);
+  if (st != M3SSD_OK || M == 0) return st;
+  return back(dims, w, M, base, ws, out, s);
+}
+
+m3ssd_status m3ssd_block_step(const m3ssd_block_dims* dims, const m3ssd_block_weights* w,
+                              const void* u_t, void* out_t, const m3ssd_cache* cache,
+                              void* workspace, size_t workspace_bytes, void* stream) {
+  using namespace m3ssd;
+  m3ssd_status st = check_block(dims, w);
+  if (st != M3SSD_OK) return st;
+  if (!cache || !cache->angle || !cache->ssm || !cache->x_prev || !cache->b_prev)
+    return M3SSD_ERR_INVALID_ARG;
+  const int64_t M = dims->batch;
+  if (M > 0 && (!u_t || !out_t || !aligned(u_t, 16) || !aligned(out_t, 16)))
+    return M3SSD_ERR_INVALID_ARG;
+  m3ssd_block_dims one = *dims;
+  one.seqlen = 1;
+  const size_t need = m3ssd_block_workspace_size(&one);
+  if (workspace_bytes < need || !workspace || !aligned(workspace, 256)) return M3SSD_ERR_WORKSPACE;
+  if (M == 0) return M3SSD_OK;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const BlockWs ws = block_ws(&one, M);
+  char* base = static_cast<char*>(workspace);
+  st = front(&one, w, u_t, M, base, ws, s);
+  if (st != M3SSD_OK) return st;
+  const m3ssd_dims sd = scan_dims(&one, 1);
+  st = m3ssd_step(&sd, base + ws.x, reinterpret_cast<const float*>(base + ws.ld),
+                  reinterpret_cast<const float*>(base + ws.be),
+                  reinterpret_cast<const float*>(base + ws.ga), base + ws.B, base + ws.C,
+                  reinterpret_cast<const float*>(base + ws.th), w->D, cache, base + ws.y, stream);
+  if (st != M3SSD_OK) return st;
+  return back(&one, w, M, base, ws, out_t, s);
+}
+
+}  // extern "C"

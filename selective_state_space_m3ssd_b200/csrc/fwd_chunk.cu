@@ -120,7 +120,7 @@ struct Smem {
   float segtot[8][NH];
   float Phi[NH];               // absolute angle at the chunk start, in [-pi, pi]
   float nPhi[NH];              // the same for the next chunk
-  uint64_t mbar[3];
+  uint64_t mbar[4];            // G done; Y1 (and S) done; Y2 done; S done
   uint64_t lmbar;              // TMA loads of the next chunk
   uint32_t tmem;
   uint32_t err;
@@ -278,6 +278,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     tc5::mbar_init(&sm.mbar[0], 1);
     tc5::mbar_init(&sm.mbar[1], 1);
     tc5::mbar_init(&sm.mbar[2], 1);
+    tc5::mbar_init(&sm.mbar[3], 1);
     tc5::mbar_init(&sm.lmbar, 1);
     tc5::fence_mbar_init();
     sm.err = 0;
@@ -368,7 +369,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       const uint64_t dC = tc5::desc_sw128(aC, 16, 1024), dB = tc5::desc_sw128(aB, 16, 1024);
       const uint64_t dH = tc5::desc_sw128(aH, kAtom, 1024), dX = tc5::desc_sw128(aX, kAtom, 1024);
       const uint64_t dWh = tc5::desc_sw128(aWh, kAtom, 1024), dWl = tc5::desc_sw128(aWl, kAtom, 1024);
-      const uint64_t dM = tc5::desc_sw128(aM, 16, 1024);
+      const uint64_t dM = tc5::desc_sw128(aM, 16, 1024), dMl = tc5::desc_sw128(aWl, 16, 1024);
       __syncthreads();  // S3: Cbar, Bbar, W_end o Bbar ready
       if (ctrl_lead) {
         tc5::fence_after_sync();
@@ -379,17 +380,19 @@ __global__ void __launch_bounds__(kThreads, 2)
           tc5::mma_bf16(tmem + kColG, dC + ko, dB + ko, kIdescG, j > 0);
         }
         tc5::commit(&sm.mbar[0]);
+        // S = (W_end o Bbar)^T X with the operand in two parts (A and B MN-major), K = 64;
+        // once it is done the residual tile's space takes the residual of the masked Gram
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const uint64_t kofs = (uint64_t)((j & 3) * (2048 >> 4));
+          tc5::mma_bf16(tmem + kColS, (j < 4 ? dWh : dWl) + kofs, dX + kofs, kIdescS, j > 0);
+        }
+        tc5::commit(&sm.mbar[3]);
         // Y1 = Cbar h (h MN-major: K = n, rows of 128 B)
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const uint64_t ko = (uint64_t)(((j >> 2) * kAtom + (j & 3) * 32) >> 4);
           tc5::mma_bf16(tmem + kColY1, dC + ko, dH + (uint64_t)(j * (2048 >> 4)), kIdescY, j > 0);
-        }
-        // S = (W_end o Bbar)^T X with the operand in two parts (A and B MN-major), K = 64
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const uint64_t kofs = (uint64_t)((j & 3) * (2048 >> 4));
-          tc5::mma_bf16(tmem + kColS, (j < 4 ? dWh : dWl) + kofs, dX + kofs, kIdescS, j > 0);
         }
         tc5::commit(&sm.mbar[1]);
         // the Gram consumes Bbar: refill it for the next chunk before joining S4
@@ -401,10 +404,11 @@ __global__ void __launch_bounds__(kThreads, 2)
       __syncthreads();  // S4: M ready
       if (ctrl_lead) {
         tc5::fence_after_sync();
+        // Y2 = M X with M in a bf16 high part and a bf16 residual
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
-          tc5::mma_bf16(tmem + kColY2, dM + (uint64_t)(j * (32 >> 4)), dX + (uint64_t)(j * (2048 >> 4)),
-                        kIdescY, j > 0);
+        for (int j = 0; j < 8; ++j)
+          tc5::mma_bf16(tmem + kColY2, (j < 4 ? dM : dMl) + (uint64_t)((j & 3) * (32 >> 4)),
+                        dX + (uint64_t)((j & 3) * (2048 >> 4)), kIdescY, j > 0);
         tc5::commit(&sm.mbar[2]);
         // Y1 and S consume Cbar and W_end o Bbar (theta's space): refill them once
         // those products are done, after Y2 is on its way
@@ -555,16 +559,30 @@ __global__ void __launch_bounds__(kThreads, 2)
       for (int q = 0; q < 4; ++q)
         tc5::ld_16x256b_x1(tmem + tlane + kColG + (uint32_t)(8 * (2 * q + cpar)), gr[q]);
       tc5::wait_ld();
+      // M = W o G in a bf16 high part (to M now) and a bf16 residual (to the
+      // residual tile once S, its previous reader, is done)
+      uint32_t mlo[2][4];
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf) {
         const int t = 16 * (warp & 3) + (lane >> 2) + 8 * hf;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const int s0 = 8 * (2 * q + cpar) + 2 * (lane & 3);
-          *reinterpret_cast<uint32_t*>(sm.M + off1(t, s0)) =
-              pack_bf16(__uint_as_float(gr[q][2 * hf]) * wv[hf][q][0],
-                        __uint_as_float(gr[q][2 * hf + 1]) * wv[hf][q][1]);
+          const float m0 = __uint_as_float(gr[q][2 * hf]) * wv[hf][q][0];
+          const float m1 = __uint_as_float(gr[q][2 * hf + 1]) * wv[hf][q][1];
+          const uint32_t hi = pack_bf16(m0, m1);
+          *reinterpret_cast<uint32_t*>(sm.M + off1(t, s0)) = hi;
+          mlo[hf][q] = pack_bf16(m0 - __uint_as_float(hi << 16), m1 - __uint_as_float(hi & 0xffff0000u));
         }
+      }
+      if (!tc5::mbar_wait(&sm.mbar[3], par, kWaitLimitNs)) sm.err = 1;
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        const int t = 16 * (warp & 3) + (lane >> 2) + 8 * hf;
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          *reinterpret_cast<uint32_t*>(sm.bw_lo + off1(t, 8 * (2 * q + cpar) + 2 * (lane & 3))) =
+              mlo[hf][q];
       }
     }
     tc5::fence_proxy_async();

@@ -34,6 +34,20 @@ def rel_max_err_out(got, ref, out_bf16: bool) -> float:
     return float(np.max(err)) / max(rms, 1e-30)
 
 
+def rel_close_err(got, ref, rtol: float, out_bf16: bool) -> float:
+    """max over elements of (|got - ref| - rtol |ref|), beyond the final bf16
+    rounding as in rel_max_err_out, over RMS(ref): an allclose-style metric
+    (absolute bar in units of the RMS, relative slack per element) for
+    heavy-tailed outputs."""
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    err = np.abs(got - ref) - rtol * np.abs(ref)
+    if out_bf16:
+        err = err - bf16_half_ulp(np.maximum(np.abs(got), np.abs(ref)))
+    rms = float(np.sqrt(np.mean(ref ** 2)))
+    return float(max(np.max(err), 0.0)) / max(rms, 1e-30)
+
+
 def rms_rel_err(got, ref) -> float:
     """RMS(got - ref) / RMS(ref)."""
     got = np.asarray(got, dtype=np.float64)

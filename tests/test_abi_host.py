@@ -187,3 +187,51 @@ def test_python_binding_raises_value_error_on_invalid_args(lib):
         m3._check(m3.ERR_INVALID_ARG, "m3ssd_fwd")
     with pytest.raises(m3.M3SSDError):
         m3._check(m3.ERR_UNSUPPORTED, "m3ssd_fwd")
+
+
+def _block_dims(**kw):
+    v = dict(batch=2, seqlen=16, d_model=64, nheads=4, headdim=16, dstate=16, ngroups=2)
+    v.update(kw)
+    return m3.BlockDims(**v)
+
+
+def _block_weights(**kw):
+    v = {n: 0x10000 for n in m3.BLOCK_WEIGHT_NAMES}
+    v.update(kw)
+    return m3.BlockWeights(*[v[n] for n in m3.BLOCK_WEIGHT_NAMES], 1e-6)
+
+
+def test_block_validation(lib):
+    d, w = _block_dims(), _block_weights()
+    need = lib.m3ssd_block_workspace_size(ctypes.byref(d))
+    assert need > 0
+    assert lib.m3ssd_block_workspace_size(None) == 0
+    assert lib.m3ssd_block_workspace_size(ctypes.byref(_block_dims(nheads=0))) == 0
+
+    def fwd(dims=d, wts=w, u=FAKE, ws=FAKE, ws_bytes=need, cin=None):
+        return lib.m3ssd_block_fwd(ctypes.byref(dims) if dims else None,
+                                   ctypes.byref(wts) if wts else None, u, FAKE,
+                                   ctypes.byref(cin) if cin else None, None, ws, ws_bytes, None)
+    assert fwd(dims=None) == m3.ERR_INVALID_ARG
+    assert fwd(wts=None) == m3.ERR_INVALID_ARG
+    assert fwd(dims=_block_dims(d_model=60)) == m3.ERR_UNSUPPORTED
+    assert fwd(dims=_block_dims(dstate=15)) == m3.ERR_INVALID_ARG
+    assert fwd(dims=_block_dims(nheads=3)) == m3.ERR_INVALID_ARG   # H % G != 0
+    assert fwd(wts=_block_weights(W_in=None)) == m3.ERR_INVALID_ARG
+    assert fwd(wts=_block_weights(B_bias=None)) == m3.ERR_INVALID_ARG
+    assert fwd(wts=_block_weights(W_out=0x10008)) == m3.ERR_INVALID_ARG   # not 16-byte aligned
+    assert fwd(u=None) == m3.ERR_INVALID_ARG
+    assert fwd(ws_bytes=need - 1) == m3.ERR_WORKSPACE
+    assert fwd(ws=ctypes.c_void_p(0x10010)) == m3.ERR_WORKSPACE
+    assert fwd(cin=m3.Cache(0x10000, None, 0x10000, 0x10000)) == m3.ERR_INVALID_ARG
+    d0 = _block_dims(batch=0)
+    assert fwd(dims=d0, u=None, ws_bytes=lib.m3ssd_block_workspace_size(ctypes.byref(d0))) == m3.OK
+
+    c = m3.Cache(0x10000, 0x10000, 0x10000, 0x10000)
+    def step(cache=c, dims=d, ws_bytes=need):
+        return lib.m3ssd_block_step(ctypes.byref(dims), ctypes.byref(w), FAKE, FAKE,
+                                    ctypes.byref(cache) if cache else None, FAKE, ws_bytes, None)
+    assert step(cache=None) == m3.ERR_INVALID_ARG
+    assert step(cache=m3.Cache(0x10000, 0x10000, None, 0x10000)) == m3.ERR_INVALID_ARG
+    assert step(ws_bytes=16) == m3.ERR_WORKSPACE
+    assert step(dims=_block_dims(batch=0)) == m3.OK

@@ -21,14 +21,19 @@
 // form one mask ("TorchMamba" README: "the parallel mask is L = 1SS @ band").
 //
 // Tensor-core work per chunk (tcgen05.mma kind::f16, bf16 in, fp32 in TMEM),
-// issued by one thread and tracked by three mbarriers (G done; Y1 and S done;
-// Y2 done) so each input buffer is refilled as soon as its last reader finishes:
+// issued by one thread in this order and tracked by four mbarriers (G done; S
+// done; Y1 done; Y2 done) so each buffer is reused as soon as its last reader
+// finishes:
 //   G  = Cbar Bbar^T                 M=64  N=64 K=128   (TMEM cols   0..63)
-//   Y1 = Cbar h_bf16                 M=64  N=64 K=128   (TMEM cols  64..127)
 //   S  = (W_end o Bbar)^T X          M=128 N=64 K=64 x2 (TMEM cols 192..255), the
 //        operand split into a bf16 high part and a bf16 residual, so the state
 //        update carries one rounding of ~2^-17 (X itself is exact bf16)
-//   Y2 = (W o G) X                   M=64  N=64 K=64    (TMEM cols 128..191)
+//   Y1 = Cbar h_bf16                 M=64  N=64 K=128   (TMEM cols  64..127)
+//   Y2 = (W o G) X                   M=64  N=64 K=64 x2 (TMEM cols 128..191), the
+//        masked Gram likewise split into a high part and a residual (the
+//        residual takes the space of W_end o Bbar's residual once S is done),
+//        so that large diagonal terms gamma_r (Cbar_r . Bbar_r) x_r keep fp32-
+//        level precision
 // and y = exp(cs) Y1 + Y2 + D x, h = exp(cs_63) h + S on the SIMT pipes, where the
 // decay/angle cumsums, sincos, rotations and the mask also run.  Operand tiles
 // live in shared memory in the 128-byte-swizzled canonical layouts: K-major rows

@@ -599,6 +599,32 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_profile(args):
+    """One kernel family alone, for ncu: the forward on the siso workload at
+    batch 2 (146 MB of inputs, above L2; a small case for full-section
+    captures), or the block at its model size (for launch lists only).  Prints
+    one summary line; not a bench line."""
+    import selective_state_space_m3ssd_b200 as m3
+    from selective_state_space_m3ssd_b200 import build as m3build
+    m3build.build()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    if args.profile == "forward":
+        w = WORKLOADS[FWD_KEY].with_(batch=2)
+        fw = bench_forward(w, dev, args.steps, args.warmup, 1, 0)
+        print(json.dumps({"profile": "forward", "workload": w.name.replace("b8", "b2"),
+                          "ms_per_step": fw["ms_per_step"], "launches": fw["launches"]}))
+    else:
+        from selective_state_space_m3ssd_b200.synth import BLOCKS, make_block
+        s = BLOCKS["model"]
+        u, wts = make_block(s, device=dev)
+        out = torch.empty_like(u)
+        for _ in range(args.warmup + args.steps):
+            m3.block_fwd(u, wts, out=out)
+        torch.cuda.synchronize(dev)
+        print(json.dumps({"profile": "block", "workload": s.name}))
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -613,10 +639,14 @@ def main():
                     help="skip the backward measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="omit the oracle timing (it never runs inside a GPU timed region)")
+    ap.add_argument("--profile", choices=["forward", "block"],
+                    help="run only a small case of one kernel family (for ncu captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
-    if args.impl == "reference":
+    if args.profile:
+        run_profile(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)

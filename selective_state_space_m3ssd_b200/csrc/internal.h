@@ -76,6 +76,12 @@ struct BwdArgs {
 // block per sequence, and per-head shares of the group-summed gradients.
 size_t bwd_workspace_bytes(int64_t b, int64_t L, int64_t H, int64_t P, int64_t N);
 cudaError_t launch_bwd_seq(const BwdArgs& a, cudaStream_t s);
+// The backward with the state's columns split across CTAs (N = 128, P a
+// multiple of 16): checkpoints and block states per (b, h, column slice), and
+// per-slice partials of the column-summed gradients.
+bool bwd_split_supported(int64_t N, int64_t P);
+size_t bwd_split_workspace_bytes(int64_t b, int64_t L, int64_t H, int64_t P);
+cudaError_t launch_bwd_split(const BwdArgs& a, cudaStream_t s);
 
 // MIMO rank R (1..8): layouts as the SISO ones with a trailing rank axis on X,
 // Y, B, C, x_prev, b_prev (and the extra cache inputs / outputs).

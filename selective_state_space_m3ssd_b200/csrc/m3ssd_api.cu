@@ -190,6 +190,9 @@ m3ssd_status m3ssd_mimo_step(const m3ssd_dims* dims, int32_t rank, const void* x
 
 size_t m3ssd_bwd_workspace_size(const m3ssd_dims* dims) {
   if (check_dims(dims) != M3SSD_OK || !general_shape_ok(dims)) return 0;
+  if (m3ssd::bwd_split_supported(dims->dstate, dims->headdim))
+    return m3ssd::bwd_split_workspace_bytes(dims->batch, dims->seqlen, dims->nheads,
+                                            dims->headdim);
   return m3ssd::bwd_workspace_bytes(dims->batch, dims->seqlen, dims->nheads, dims->headdim,
                                     dims->dstate);
 }
@@ -236,7 +239,9 @@ m3ssd_status m3ssd_bwd(const m3ssd_dims* dims, const void* X, const float* logde
   a.dgamma = grads->dgamma; a.dB = grads->dB; a.dC = grads->dC; a.dtheta = grads->dtheta;
   a.dD = grads->dD; a.dh0 = grads->dh0; a.dangle0 = grads->dangle0; a.dxprev0 = grads->dxprev0;
   a.dbprev0 = grads->dbprev0; a.workspace = workspace;
-  return from_cuda(m3ssd::launch_bwd_seq(a, static_cast<cudaStream_t>(stream)));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return from_cuda(m3ssd::bwd_split_supported(a.N, a.P) ? m3ssd::launch_bwd_split(a, s)
+                                                         : m3ssd::launch_bwd_seq(a, s));
 }
 
 m3ssd_status m3ssd_step(const m3ssd_dims* dims, const void* x_t, const float* logdecay_t,

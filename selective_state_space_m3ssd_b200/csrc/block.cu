@@ -85,6 +85,16 @@ struct PrepArgs {
 
 __device__ __forceinline__ float softplus_f(float v) { return v > 20.f ? v : log1pf(expf(v)); }
 
+// two floats as bf16 (round to nearest even), the first in the low half
+__device__ __forceinline__ uint32_t pack2_bf16(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+bool vec_shape(int64_t H, int64_t P, int64_t N, int64_t G) {
+  return (H * P) % 8 == 0 && (G * N) % 4 == 0 && H % 4 == 0 && N % 8 == 0;
+}
+
 // One CTA per token.  Shared memory: 2G inverse RMS values (B groups, then C
 // groups) and the H step sizes Delta.
 __global__ void __launch_bounds__(kPrepThreads) block_prep_kernel(PrepArgs a) {
@@ -125,6 +135,98 @@ __global__ void __launch_bounds__(kPrepThreads) block_prep_kernel(PrepArgs a) {
         __float2bfloat16_rn(fmaf(row[oC + g * N + n] * inv[G + g], a.Cw[n], a.Cbias[k]));
   }
   for (int k = tid; k < H * NH; k += kPrepThreads) a.th[tok * H * NH + k] = delta[k / NH] * row[oth + k];
+}
+
+// The same with 16-byte accesses, for shapes whose row parts are multiples of
+// four floats and eight bf16 (H P % 8, G N % 4, H % 4, N % 8).
+__global__ void __launch_bounds__(kPrepThreads) block_prep_vec_kernel(PrepArgs a) {
+  extern __shared__ float sh[];
+  const int64_t tok = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int H = (int)a.H, P = (int)a.P, N = (int)a.N, G = (int)a.G, NH = N / 2;
+  const int HP = H * P, GN = G * N;
+  const int oB = 2 * HP, oC = oB + GN, odt = oC + GN, olam = odt + H, oth = olam + H;
+  const float* row = a.zx + tok * a.width;
+  float* inv = sh;
+  float* delta = sh + 2 * G;
+
+  for (int j = warp; j < 2 * G; j += kPrepThreads / 32) {
+    const float* v = row + (j < G ? oB + j * N : oC + (j - G) * N);
+    float ss = 0.f;
+    for (int n = 4 * lane; n < N; n += 128) {
+      const float4 q = *reinterpret_cast<const float4*>(v + n);
+      ss = fmaf(q.x, q.x, fmaf(q.y, q.y, fmaf(q.z, q.z, fmaf(q.w, q.w, ss))));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if (lane == 0) inv[j] = 1.f / sqrtf(ss / (float)N + a.eps);
+  }
+  for (int h = tid; h < H; h += kPrepThreads) {
+    const float dl = softplus_f(row[odt + h] + a.dt_bias[h]);
+    const float lg = -expf(a.A_log[h]) * dl;
+    const float lam = 1.f / (1.f + expf(-row[olam + h]));
+    a.ld[tok * H + h] = lg;
+    a.ga[tok * H + h] = lam * dl;
+    a.be[tok * H + h] = (1.f - lam) * dl * expf(lg);
+    delta[h] = dl;
+  }
+  for (int k = tid; k < HP / 8; k += kPrepThreads) {
+    const float4 u = *reinterpret_cast<const float4*>(row + HP + 8 * k);
+    const float4 v = *reinterpret_cast<const float4*>(row + HP + 8 * k + 4);
+    uint4 o;
+    o.x = pack2_bf16(u.x, u.y); o.y = pack2_bf16(u.z, u.w);
+    o.z = pack2_bf16(v.x, v.y); o.w = pack2_bf16(v.z, v.w);
+    *reinterpret_cast<uint4*>(a.X + tok * HP + 8 * k) = o;
+  }
+  __syncthreads();
+  const int NQ = N / 4, hpg = H / G;
+  for (int k = tid; k < H * NQ; k += kPrepThreads) {
+    const int h = k / NQ, n = 4 * (k - h * NQ), g = h / hpg;
+    const float4 bv = *reinterpret_cast<const float4*>(row + oB + g * N + n);
+    const float4 cv = *reinterpret_cast<const float4*>(row + oC + g * N + n);
+    const float4 bw = *reinterpret_cast<const float4*>(a.Bw + n);
+    const float4 cw = *reinterpret_cast<const float4*>(a.Cw + n);
+    const float4 bb = *reinterpret_cast<const float4*>(a.Bbias + h * N + n);
+    const float4 cb = *reinterpret_cast<const float4*>(a.Cbias + h * N + n);
+    const float ib = inv[g], ic = inv[G + g];
+    uint2 ob, oc;
+    ob.x = pack2_bf16(fmaf(bv.x * ib, bw.x, bb.x), fmaf(bv.y * ib, bw.y, bb.y));
+    ob.y = pack2_bf16(fmaf(bv.z * ib, bw.z, bb.z), fmaf(bv.w * ib, bw.w, bb.w));
+    oc.x = pack2_bf16(fmaf(cv.x * ic, cw.x, cb.x), fmaf(cv.y * ic, cw.y, cb.y));
+    oc.y = pack2_bf16(fmaf(cv.z * ic, cw.z, cb.z), fmaf(cv.w * ic, cw.w, cb.w));
+    *reinterpret_cast<uint2*>(a.B + tok * H * N + h * N + n) = ob;
+    *reinterpret_cast<uint2*>(a.C + tok * H * N + h * N + n) = oc;
+  }
+  for (int k = tid; k < H * NH / 4; k += kPrepThreads) {
+    const float d = delta[(4 * k) / NH];
+    const float4 v = *reinterpret_cast<const float4*>(row + oth + 4 * k);
+    *reinterpret_cast<float4*>(a.th + tok * H * NH + 4 * k) =
+        make_float4(d * v.x, d * v.y, d * v.z, d * v.w);
+  }
+}
+
+// y * SiLU(z), z read from the fp32 in_proj rows, eight elements a thread
+// (H P % 8 == 0, in_proj width % 4 == 0).
+__global__ void block_gate_vec_kernel(const __nv_bfloat16* __restrict__ y,
+                                      const float* __restrict__ zx, int64_t width, int64_t HP,
+                                      int64_t M, __nv_bfloat16* __restrict__ out) {
+  const int64_t n8 = M * HP / 8, stride = (int64_t)gridDim.x * blockDim.x, hp8 = HP / 8;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8; i += stride) {
+    const int64_t tok = i / hp8, k = 8 * (i - tok * hp8);
+    const uint4 yv = *reinterpret_cast<const uint4*>(y + 8 * i);
+    const float4 z0 = *reinterpret_cast<const float4*>(zx + tok * width + k);
+    const float4 z1 = *reinterpret_cast<const float4*>(zx + tok * width + k + 4);
+    const uint32_t yw[4] = {yv.x, yv.y, yv.z, yv.w};
+    const float z[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float y0 = __uint_as_float(yw[j] << 16), y1 = __uint_as_float(yw[j] & 0xffff0000u);
+      o[j] = pack2_bf16(y0 * z[2 * j] / (1.f + expf(-z[2 * j])),
+                        y1 * z[2 * j + 1] / (1.f + expf(-z[2 * j + 1])));
+    }
+    *reinterpret_cast<uint4*>(out + 8 * i) = make_uint4(o[0], o[1], o[2], o[3]);
+  }
 }
 
 // y * SiLU(z), z read from the fp32 in_proj rows.
@@ -254,7 +356,12 @@ m3ssd_status front(const m3ssd_block_dims* d, const m3ssd_block_weights* w, cons
   a.th = reinterpret_cast<float*>(base + ws.th);
   const size_t smem = sizeof(float) * (size_t)(2 * d->ngroups + d->nheads);
   if (smem > 48 * 1024) return M3SSD_ERR_UNSUPPORTED;
-  block_prep_kernel<<<(unsigned)M, kPrepThreads, smem, s>>>(a);
+  const bool w16 = aligned(a.Bw, 16) && aligned(a.Cw, 16) && aligned(a.Bbias, 16) &&
+                   aligned(a.Cbias, 16);
+  if (w16 && vec_shape(a.H, a.P, a.N, a.G))
+    block_prep_vec_kernel<<<(unsigned)M, kPrepThreads, smem, s>>>(a);
+  else
+    block_prep_kernel<<<(unsigned)M, kPrepThreads, smem, s>>>(a);
   return cudaGetLastError() == cudaSuccess ? M3SSD_OK : M3SSD_ERR_CUDA;
 }
 
@@ -263,11 +370,18 @@ m3ssd_status back(const m3ssd_block_dims* d, const m3ssd_block_weights* w, int64
                   const BlockWs& ws, void* out, cudaStream_t s) {
   const int64_t HP = d->nheads * d->headdim;
   const int64_t n = M * HP;
-  const unsigned grid = (unsigned)((n + 255) / 256 < 148 * 16 ? (n + 255) / 256 : 148 * 16);
-  block_gate_kernel<<<grid, 256, 0, s>>>(reinterpret_cast<const __nv_bfloat16*>(base + ws.y),
-                                         reinterpret_cast<const float*>(base + ws.zx),
-                                         in_proj_width(d), HP, M,
-                                         reinterpret_cast<__nv_bfloat16*>(base + ws.x));
+  const int64_t width = in_proj_width(d);
+  const auto* yp = reinterpret_cast<const __nv_bfloat16*>(base + ws.y);
+  const auto* zp = reinterpret_cast<const float*>(base + ws.zx);
+  auto* gp = reinterpret_cast<__nv_bfloat16*>(base + ws.x);
+  if (HP % 8 == 0 && width % 4 == 0) {
+    const int64_t n8 = n / 8;
+    const unsigned grid = (unsigned)((n8 + 255) / 256 < 148 * 16 ? (n8 + 255) / 256 : 148 * 16);
+    block_gate_vec_kernel<<<grid, 256, 0, s>>>(yp, zp, width, HP, M, gp);
+  } else {
+    const unsigned grid = (unsigned)((n + 255) / 256 < 148 * 16 ? (n + 255) / 256 : 148 * 16);
+    block_gate_kernel<<<grid, 256, 0, s>>>(yp, zp, width, HP, M, gp);
+  }
   if (cudaGetLastError() != cudaSuccess) return M3SSD_ERR_CUDA;
   if (!gemm_bf16(M, d->d_model, HP, base + ws.x, w->W_out, out, CUDA_R_16BF, base + ws.lt,
                  kLtWorkspace, s))

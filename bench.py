@@ -602,7 +602,8 @@ def run_reference(args):
 def run_profile(args):
     """One kernel family alone, for ncu: the forward on the siso workload at
     batch 2 (146 MB of inputs, above L2; a small case for full-section
-    captures), or the block at its model size (for launch lists only).  Prints
+    captures), the backward on one batch row at L = 1024 (a small case), or
+    the block at its model size (for launch lists only).  Prints
     one summary line; not a bench line."""
     import selective_state_space_m3ssd_b200 as m3
     from selective_state_space_m3ssd_b200 import build as m3build
@@ -614,6 +615,20 @@ def run_profile(args):
         fw = bench_forward(w, dev, args.steps, args.warmup, 1, 0)
         print(json.dumps({"profile": "forward", "workload": w.name.replace("b8", "b2"),
                           "ms_per_step": fw["ms_per_step"], "launches": fw["launches"]}))
+    elif args.profile == "backward":
+        # one (b, h) sequence group of the forward's workload: 32 heads x 4 column
+        # slices = 128 CTAs, L = 1024
+        w = WORKLOADS[FWD_KEY].with_(batch=1, seqlen=1024)
+        inp = make_inputs(w)
+        d = {k: (None if v is None else v.to(dev)) for k, v in inp.items()}
+        dY = torch.randn(tuple(d["X"].shape), generator=torch.Generator().manual_seed(7)).to(
+            d["X"].dtype).to(dev)
+        args_ = [d.get(k) for k in ("X", "logdecay", "beta", "gamma", "B", "C", "theta", "D",
+                                    "h0")]
+        for _ in range(args.warmup + args.steps):
+            m3.bwd(*args_, dY=dY)
+        torch.cuda.synchronize(dev)
+        print(json.dumps({"profile": "backward", "workload": "siso shape b1 L1024 H32 P64 N128"}))
     else:
         from selective_state_space_m3ssd_b200.synth import BLOCKS, make_block
         s = BLOCKS["model"]
@@ -639,7 +654,7 @@ def main():
                     help="skip the backward measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="omit the oracle timing (it never runs inside a GPU timed region)")
-    ap.add_argument("--profile", choices=["forward", "block"],
+    ap.add_argument("--profile", choices=["forward", "block", "backward"],
                     help="run only a small case of one kernel family (for ncu captures)")
     args = ap.parse_args()
     if args.warmup < 3:

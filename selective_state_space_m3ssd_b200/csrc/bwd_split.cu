@@ -72,13 +72,15 @@ __device__ __forceinline__ float ld(const T* p, int64_t i) {
 template <typename T>
 __global__ void __launch_bounds__(kT, 4) bwd_split_kernel(BwdArgs a, SplitWs ws) {
   __shared__ float Bb[3][kN];     // Bbar of tokens, three-deep so one barrier a token suffices
-  __shared__ float xs[3][kPS];    // x slices, likewise
+  __shared__ __align__(16) float xs[3][kPS];    // x slices, likewise
   __shared__ float Cb[kN], Bpb[kN], rcv[kN], rxv[kN], rxpv[kN];
-  __shared__ float xv[kPS], xpv[kPS], dyv[kPS];
+  __shared__ __align__(16) float xv[kPS];
+  __shared__ __align__(16) float xpv[kPS];
+  __shared__ __align__(16) float dyv[kPS];
   __shared__ float gvS[kN * kPad];
   __shared__ float phiB[(kK + 1) * kNH];
   __shared__ float colp[4][2][kPS];
-  __shared__ float red[kT / 32];
+  __shared__ float red[3][kT / 32];  // per warp: <g, h_{t-1}>, Bbar_t . g x_t, Bbar_{t-1} . g x_{t-1}
 
   const int64_t H = a.H, P = a.P, G = a.G, L = a.L;
   const int S = (int)(P / kPS);
@@ -185,9 +187,9 @@ __global__ void __launch_bounds__(kT, 4) bwd_split_kernel(BwdArgs a, SplitWs ws)
 #pragma unroll
   for (int p = 0; p < kPS; ++p) gS[p] = a.dhT ? a.dhT[(bh * kN + n) * P + p0 + p] : 0.f;
   float apend = 1.f;
-  float dxc = 0.f;                      // threads < kPS: gradient of x_{t-1} carried back
+  float dxc = 0.f;                      // lanes < kPS of warp 0: gradient of x_{t-1} carried back
   float dbc0 = 0.f, dbc1 = 0.f, dphc = 0.f, rth = 0.f;  // rotation threads: carries of pair ri
-  float dDacc = 0.f;                    // warp 1 lane 0: running y . x
+  float dDacc = 0.f;                    // thread 0: running dy . x
 
   for (int64_t k = nblk - 1; k >= 0; --k) {
     const int64_t t0 = k * kK, t1 = (t0 + kK < L) ? t0 + kK : L;
@@ -261,26 +263,45 @@ __global__ void __launch_bounds__(kT, 4) bwd_split_kernel(BwdArgs a, SplitWs ws)
       const float be = a.beta ? a.beta[th] : 0.f, ga = a.gamma[th];
       __syncthreads();  // (1)
 
-      // phase B: this row's element pass
+      // phase B: this row's element pass, and its shares of <g, h_{t-1}>,
+      // dgamma = Bbar_t . (g x_t) and dbeta = Bbar_{t-1} . (g x_{t-1})
       {
         const float cn = Cb[n];
         float rc = 0.f, rx = 0.f, rxp = 0.f, da = 0.f;
 #pragma unroll
-        for (int p = 0; p < kPS; ++p) {
-          const float gv = fmaf(apend, gS[p], cn * dyv[p]);
-          rc = fmaf(St[p], dyv[p], rc);
-          da = fmaf(gv, Sp[p], da);
-          rx = fmaf(gv, xv[p], rx);
-          rxp = fmaf(gv, xpv[p], rxp);
-          gS[p] = gv;
-          gvS[n * kPad + p] = gv;
+        for (int p = 0; p < kPS; p += 4) {
+          const float4 dy4 = *reinterpret_cast<const float4*>(dyv + p);
+          const float4 x4 = *reinterpret_cast<const float4*>(xv + p);
+          const float4 xp4 = *reinterpret_cast<const float4*>(xpv + p);
+          const float dy[4] = {dy4.x, dy4.y, dy4.z, dy4.w};
+          const float xx[4] = {x4.x, x4.y, x4.z, x4.w};
+          const float xp[4] = {xp4.x, xp4.y, xp4.z, xp4.w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float gv = fmaf(apend, gS[p + q], cn * dy[q]);
+            rc = fmaf(St[p + q], dy[q], rc);
+            da = fmaf(gv, Sp[p + q], da);
+            rx = fmaf(gv, xx[q], rx);
+            rxp = fmaf(gv, xp[q], rxp);
+            gS[p + q] = gv;
+            gvS[n * kPad + p + q] = gv;
+          }
         }
         rcv[n] = rc;
         rxv[n] = rx;
         rxpv[n] = rxp;
+        float sg = Bb[0][n] * rx, sb = Bpb[n] * rxp;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) da += __shfl_xor_sync(0xffffffffu, da, o);
-        if (lane == 0) red[warp] = da;
+        for (int o = 16; o > 0; o >>= 1) {
+          da += __shfl_xor_sync(0xffffffffu, da, o);
+          sg += __shfl_xor_sync(0xffffffffu, sg, o);
+          sb += __shfl_xor_sync(0xffffffffu, sb, o);
+        }
+        if (lane == 0) {
+          red[0][warp] = da;
+          red[1][warp] = sg;
+          red[2][warp] = sb;
+        }
       }
       __syncthreads();  // (2)
 
@@ -288,38 +309,35 @@ __global__ void __launch_bounds__(kT, 4) bwd_split_kernel(BwdArgs a, SplitWs ws)
       {
         const int p = tid & (kPS - 1), which = (tid >> 4) & 1, q = tid >> 5;
         const float* v = which ? Bpb : Bb[0];
-        float acc = 0.f;
+        float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll 8
-        for (int r = 32 * q; r < 32 * q + 32; ++r) acc = fmaf(gvS[r * kPad + p], v[r], acc);
-        colp[q][which][p] = acc;
+        for (int r = 32 * q; r < 32 * q + 32; r += 2) {
+          acc0 = fmaf(gvS[r * kPad + p], v[r], acc0);
+          acc1 = fmaf(gvS[(r + 1) * kPad + p], v[r + 1], acc1);
+        }
+        colp[q][which][p] = acc0 + acc1;
       }
       __syncthreads();  // (3)
 
       // phase D: dX, the scalar partials, and the rotation adjoints
-      if (tid < kPS) {
-        const float pb = colp[0][0][tid] + colp[1][0][tid] + colp[2][0][tid] + colp[3][0][tid];
-        const float pbp = colp[0][1][tid] + colp[1][1][tid] + colp[2][1][tid] + colp[3][1][tid];
-        a.dX[th * P + p0 + tid] = dxc + Dh * dyv[tid] + ga * pb;
-        dxc = be * pbp;
-      } else if (warp == 1) {
-        float sg = 0.f, sb = 0.f;
-        for (int r = lane; r < kN; r += 32) {
-          sg = fmaf(Bb[0][r], rxv[r], sg);
-          sb = fmaf(Bpb[r], rxpv[r], sb);
+      if (warp == 0) {
+        // lanes < kPS: dX of their column; lanes 0..2: the token's scalar partials
+        float sd = 0.f;
+        if (lane < kPS) {
+          const float pb = colp[0][0][lane] + colp[1][0][lane] + colp[2][0][lane] + colp[3][0][lane];
+          const float pbp =
+              colp[0][1][lane] + colp[1][1][lane] + colp[2][1][lane] + colp[3][1][lane];
+          a.dX[th * P + p0 + lane] = dxc + Dh * dyv[lane] + ga * pb;
+          dxc = be * pbp;
+          sd = dyv[lane] * xv[lane];
         }
-        float sd = lane < kPS ? dyv[lane] * xv[lane] : 0.f;
+        if (lane < 3) {
+          const float v = red[lane][0] + red[lane][1] + red[lane][2] + red[lane][3];
+          dScal[th * 3 + lane] = lane == 0 ? at * v : v;
+        }
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-          sg += __shfl_xor_sync(0xffffffffu, sg, o);
-          sb += __shfl_xor_sync(0xffffffffu, sb, o);
-          sd += __shfl_xor_sync(0xffffffffu, sd, o);
-        }
-        if (lane == 0) {
-          dScal[th * 3 + 1] = sg;
-          dScal[th * 3 + 2] = sb;
-          dScal[th * 3 + 0] = at * (red[0] + red[1] + red[2] + red[3]);
-          dDacc += sd;
-        }
+        for (int o = 8; o > 0; o >>= 1) sd += __shfl_xor_sync(0xffffffffu, sd, o);
+        if (lane == 0) dDacc += sd;
       } else if (rot) {
         const float d0 = ga * rxv[2 * ri], d1 = ga * rxv[2 * ri + 1];
         const float e0 = rcv[2 * ri], e1 = rcv[2 * ri + 1];
@@ -352,7 +370,7 @@ __global__ void __launch_bounds__(kT, 4) bwd_split_kernel(BwdArgs a, SplitWs ws)
     dbpp[bh * kN + 2 * ri + 1] = dbc1;
     dAngp[bh * kNH + ri] = rth + dphc;
   }
-  if (warp == 1 && lane == 0) dDp[bh] = dDacc;
+  if (tid == 0) dDp[bh] = dDacc;
 }
 
 // Sums of the slice partials (and of the heads of a group, and of the batch for

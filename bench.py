@@ -469,8 +469,8 @@ def bench_block(dev, rank, peaks: dict, steps: int = 5, warmup: int = 3):
     bw, pt = peaks["hbm_gbs"] * 1e9, peaks["bf16_tflops"] * 1e12
     t_in = max(2.0 * M * dm * width / pt, (M * dm * 2 + width * dm * 2 + M * width * 4) / bw)
     t_out = max(2.0 * M * HP * dm / pt, (M * HP * 2 + dm * HP * 2 + M * dm * 2) / bw)
-    prep_b = M * (width * 4 + HP * 2 + 2 * H * N * 2 + 3 * H * 4 + H * (N // 2) * 4)
-    scan_b = M * (2 * HP * 2 + 3 * H * 4 + 2 * H * N * 2 + H * (N // 2) * 4)
+    prep_b = M * (width * 4 + HP * 2 + 2 * G * N * 2 + 3 * H * 4 + H * (N // 2) * 4)
+    scan_b = M * (2 * HP * 2 + 3 * H * 4 + 2 * G * N * 2 + H * (N // 2) * 4)
     gate_b = M * HP * (2 + 4 + 2)
     t_lb = t_in + t_out + (prep_b + scan_b + gate_b) / bw
     return {"metric": "block Mtokens/s (fwd)", "value": M / (ms / 1e3) / 1e6, "unit": "Mtokens/s",
@@ -483,7 +483,7 @@ def bench_block(dev, rank, peaks: dict, steps: int = 5, warmup: int = 3):
                          "peak_bf16_tflops": peaks["bf16_tflops"], "peak_source": peaks["source"],
                          "gemm_tflop_per_step": 2.0 * M * (dm * width + HP * dm) / 1e12,
                          "note": "sum over phases of max(flops / bf16 peak, bytes / HBM) for the "
-                                 "GEMMs and bytes / HBM for prep, scan (one B/C per head) and gate"},
+                                 "GEMMs and bytes / HBM for prep, scan (B, C per group, head bias applied inside) and gate"},
             "gpu_launches": 3 * steps,
             "library_launches": 2 * steps,
             "note": "own kernels per call: prep, scan, gate; cuBLASLt: in_proj, out_proj"}

@@ -276,8 +276,10 @@ m3ssd_status m3ssd_bwd_noalloc(const m3ssd_dims* dims, const void* X, const floa
  *
  * The projections are plain GEMMs run by cuBLASLt (bf16 operands, fp32
  * accumulation; in_proj writes fp32, out_proj bf16); the rest runs in this
- * library's kernels.  u and out are bf16.  The block cache is an m3ssd_cache
- * whose b_prev is per HEAD: (b, H, N) holding B'_{t-1} unrotated.
+ * library's kernels, the head biases inside the scan (added in fp32 before the
+ * rotation).  u and out are bf16.  The block cache is an m3ssd_cache with
+ * b_prev (b, G, N) holding the QK-normed group vector B_{t-1} (times its norm
+ * weight, without the head bias) unrotated; the bias is added at use.
  */
 typedef struct {
   int64_t batch;    /* b >= 0 */

@@ -34,9 +34,10 @@ Storage precision: the pages' numerics policy ("TorchMamba" README,
 "Behavioral notes": bf16 computes in fp32 and each output is downcast to the
 input dtype) makes the tensors a bf16 block hands from one step to the next
 bf16.  ``store`` (default: none) is applied to exactly those hand-offs -- x,
-B', C' (the scan's bf16 inputs), the scan output y and the gated product
-(out_proj's input) -- so that a test can compare against a device path that
-stores them in bf16; everything else stays fp64.
+the QK-normed group vectors of B and C (the scan's bf16 inputs; the head bias
+is added after them), the scan output y and the gated product (out_proj's
+input) -- so that a test can compare against a device path that stores them
+in bf16; everything else stays fp64.
 
 Numerical pins: ``tests/test_oracle_block.py`` (closed forms for one and two
 tokens, the scale invariance of the norm, forward == prefill + steps, and
@@ -101,10 +102,10 @@ def scan_inputs(u, wts, H, P, N, G, store=_keep):
     theta = delta[..., None] * s["theta"]
     eps = float(wts["eps"])
     grp = np.arange(H) // (H // G)
-    Bh = bc_norm(s["B"], f("B_norm_w"), eps)[..., grp, :] + f("B_bias")
-    Ch = bc_norm(s["C"], f("C_norm_w"), eps)[..., grp, :] + f("C_bias")
+    Bh = store(bc_norm(s["B"], f("B_norm_w"), eps))[..., grp, :] + f("B_bias")
+    Ch = store(bc_norm(s["C"], f("C_norm_w"), eps))[..., grp, :] + f("C_bias")
     return {"z": s["z"], "X": store(s["x"]), "logdecay": logdecay, "beta": beta, "gamma": gamma,
-            "B": store(Bh), "C": store(Ch), "theta": theta}
+            "B": Bh, "C": Ch, "theta": theta}
 
 
 def new_block_cache(b, H, P, N):

@@ -503,19 +503,19 @@ def _block_args(u, wts, seqlen):
     return dims, w, (H, P, N, G)
 
 
-def new_block_cache(batch, nheads, headdim, dstate, device):
+def new_block_cache(batch, nheads, headdim, dstate, ngroups, device):
     """A zeroed block cache: angle (b,H,N/2), ssm (b,H,N,P), x_prev (b,H,P) and
-    the per-head b_prev (b,H,N), all fp32."""
-    return new_cache(batch, nheads, headdim, dstate, nheads, device)
+    b_prev (b,G,N) (the normed group vector, the head bias added at use), all fp32."""
+    return new_cache(batch, nheads, headdim, dstate, ngroups, device)
 
 
-def _cache_struct(cache, b, H, P, N, dev, name):
+def _cache_struct(cache, b, H, P, N, G, dev, name):
     import torch
     f32 = torch.float32
     _need(cache["angle"], name + ".angle", f32, (b, H, N // 2), dev)
     _need(cache["ssm"], name + ".ssm", f32, (b, H, N, P), dev)
     _need(cache["x_prev"], name + ".x_prev", f32, (b, H, P), dev)
-    _need(cache["b_prev"], name + ".b_prev", f32, (b, H, N), dev)
+    _need(cache["b_prev"], name + ".b_prev", f32, (b, G, N), dev)
     return Cache(cache["angle"].data_ptr(), cache["ssm"].data_ptr(), cache["x_prev"].data_ptr(),
                  cache["b_prev"].data_ptr())
 
@@ -536,8 +536,8 @@ def block_fwd(u, wts: dict, *, cache_in=None, cache_out=None, out=None, workspac
     dev = u.device
     out = torch.empty_like(u) if out is None else out
     _need(out, "out", torch.bfloat16, (b, L, dm), dev)
-    ci = None if cache_in is None else _cache_struct(cache_in, b, H, P, N, dev, "cache_in")
-    co = None if cache_out is None else _cache_struct(cache_out, b, H, P, N, dev, "cache_out")
+    ci = None if cache_in is None else _cache_struct(cache_in, b, H, P, N, G, dev, "cache_in")
+    co = None if cache_out is None else _cache_struct(cache_out, b, H, P, N, G, dev, "cache_out")
     need = block_workspace_size(dims)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
@@ -558,7 +558,7 @@ def block_step(cache: dict, u_t, wts: dict, *, out_t=None, workspace=None):
     dev = u_t.device
     out_t = torch.empty_like(u_t) if out_t is None else out_t
     _need(out_t, "out_t", torch.bfloat16, (b, dm), dev)
-    c = _cache_struct(cache, b, H, P, N, dev, "cache")
+    c = _cache_struct(cache, b, H, P, N, G, dev, "cache")
     need = block_workspace_size(dims)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)

@@ -8,10 +8,11 @@
 // (bf16 operands, fp32 accumulation); everything between them runs here:
 //
 //   block_prep_kernel   one CTA per token: splits the fp32 in_proj row, writes x
-//                       (bf16), the per-head B' and C' (QK-norm of the group's
-//                       vector times the norm weight plus the head's bias, bf16),
-//                       logdecay, beta, gamma (fp32) and theta_dt (fp32);
-//   m3ssd_fwd / m3ssd_step of this library on those tensors (one B/C per head);
+//                       (bf16), the QK-normed B and C of each group times the
+//                       norm weight (bf16), logdecay, beta, gamma (fp32) and
+//                       theta_dt (fp32);
+//   the scan's forward / step kernels on those tensors, which add the head's
+//   B and C biases in fp32 before rotating (no per-head copy of B and C);
 //   block_gate_kernel   y * SiLU(z) (bf16), the input of out_proj.
 #include <cublasLt.h>
 #include <cuda_runtime.h>
@@ -21,6 +22,7 @@
 
 #include "../../include/m3ssd.h"
 #include "common.cuh"
+#include "internal.h"
 
 namespace m3ssd {
 namespace {
@@ -51,14 +53,15 @@ BlockWs block_ws(const m3ssd_block_dims* d, int64_t M) {
   };
   w.zx = take(m * (size_t)in_proj_width(d) * 4);
   w.x = take(m * H * P * 2);   // x, then y * SiLU(z)
-  w.B = take(m * H * N * 2);
-  w.C = take(m * H * N * 2);
+  const size_t G = (size_t)d->ngroups;
+  w.B = take(m * G * N * 2);
+  w.C = take(m * G * N * 2);
   w.ld = take(m * H * 4);
   w.be = take(m * H * 4);
   w.ga = take(m * H * 4);
   w.th = take(m * H * (N / 2) * 4);
   w.y = take(m * H * P * 2);
-  w.bp = take((size_t)d->batch * H * N * 4);  // copy of the incoming b_prev
+  w.bp = take((size_t)d->batch * G * N * 4);  // copy of the incoming b_prev
   w.lt = take(kLtWorkspace);
   w.total = o;
   return w;
@@ -127,12 +130,10 @@ __global__ void __launch_bounds__(kPrepThreads) block_prep_kernel(PrepArgs a) {
   }
   for (int k = tid; k < HP; k += kPrepThreads) a.X[tok * HP + k] = __float2bfloat16_rn(row[HP + k]);
   __syncthreads();
-  const int hpg = H / G;
-  for (int k = tid; k < H * N; k += kPrepThreads) {
-    const int h = k / N, n = k - h * N, g = h / hpg;
-    a.B[tok * H * N + k] = __float2bfloat16_rn(fmaf(row[oB + g * N + n] * inv[g], a.Bw[n], a.Bbias[k]));
-    a.C[tok * H * N + k] =
-        __float2bfloat16_rn(fmaf(row[oC + g * N + n] * inv[G + g], a.Cw[n], a.Cbias[k]));
+  for (int k = tid; k < G * N; k += kPrepThreads) {
+    const int g = k / N, n = k - g * N;
+    a.B[tok * G * N + k] = __float2bfloat16_rn(row[oB + k] * inv[g] * a.Bw[n]);
+    a.C[tok * G * N + k] = __float2bfloat16_rn(row[oC + k] * inv[G + g] * a.Cw[n]);
   }
   for (int k = tid; k < H * NH; k += kPrepThreads) a.th[tok * H * NH + k] = delta[k / NH] * row[oth + k];
 }
@@ -179,23 +180,21 @@ __global__ void __launch_bounds__(kPrepThreads) block_prep_vec_kernel(PrepArgs a
     *reinterpret_cast<uint4*>(a.X + tok * HP + 8 * k) = o;
   }
   __syncthreads();
-  const int NQ = N / 4, hpg = H / G;
-  for (int k = tid; k < H * NQ; k += kPrepThreads) {
-    const int h = k / NQ, n = 4 * (k - h * NQ), g = h / hpg;
+  const int NQ = N / 4;
+  for (int k = tid; k < G * NQ; k += kPrepThreads) {
+    const int g = k / NQ, n = 4 * (k - g * NQ);
     const float4 bv = *reinterpret_cast<const float4*>(row + oB + g * N + n);
     const float4 cv = *reinterpret_cast<const float4*>(row + oC + g * N + n);
     const float4 bw = *reinterpret_cast<const float4*>(a.Bw + n);
     const float4 cw = *reinterpret_cast<const float4*>(a.Cw + n);
-    const float4 bb = *reinterpret_cast<const float4*>(a.Bbias + h * N + n);
-    const float4 cb = *reinterpret_cast<const float4*>(a.Cbias + h * N + n);
     const float ib = inv[g], ic = inv[G + g];
     uint2 ob, oc;
-    ob.x = pack2_bf16(fmaf(bv.x * ib, bw.x, bb.x), fmaf(bv.y * ib, bw.y, bb.y));
-    ob.y = pack2_bf16(fmaf(bv.z * ib, bw.z, bb.z), fmaf(bv.w * ib, bw.w, bb.w));
-    oc.x = pack2_bf16(fmaf(cv.x * ic, cw.x, cb.x), fmaf(cv.y * ic, cw.y, cb.y));
-    oc.y = pack2_bf16(fmaf(cv.z * ic, cw.z, cb.z), fmaf(cv.w * ic, cw.w, cb.w));
-    *reinterpret_cast<uint2*>(a.B + tok * H * N + h * N + n) = ob;
-    *reinterpret_cast<uint2*>(a.C + tok * H * N + h * N + n) = oc;
+    ob.x = pack2_bf16(bv.x * ib * bw.x, bv.y * ib * bw.y);
+    ob.y = pack2_bf16(bv.z * ib * bw.z, bv.w * ib * bw.w);
+    oc.x = pack2_bf16(cv.x * ic * cw.x, cv.y * ic * cw.y);
+    oc.y = pack2_bf16(cv.z * ic * cw.z, cv.w * ic * cw.w);
+    *reinterpret_cast<uint2*>(a.B + tok * G * N + g * N + n) = ob;
+    *reinterpret_cast<uint2*>(a.C + tok * G * N + g * N + n) = oc;
   }
   for (int k = tid; k < H * NH / 4; k += kPrepThreads) {
     const float d = delta[(4 * k) / NH];
@@ -322,17 +321,9 @@ m3ssd_status check_block(const m3ssd_block_dims* d, const m3ssd_block_weights* w
   return M3SSD_OK;
 }
 
-m3ssd_dims scan_dims(const m3ssd_block_dims* d, int64_t L) {
-  m3ssd_dims s{};
-  s.batch = d->batch;
-  s.seqlen = L;
-  s.nheads = d->nheads;
-  s.headdim = d->headdim;
-  s.dstate = d->dstate;
-  s.ngroups = d->nheads;  // one B'/C' per head (the bias is head-specific)
-  s.chunk = 0;
-  s.x_dtype = M3SSD_BF16;
-  return s;
+// The scan's shapes its sequential and step kernels keep in one CTA.
+bool scan_shape_ok(const m3ssd_block_dims* d) {
+  return d->dstate <= 256 && d->headdim <= 256 && d->dstate * d->headdim <= 16384;
 }
 
 // in_proj, the prep kernel; returns the scan inputs' pointers through ws.
@@ -356,8 +347,7 @@ m3ssd_status front(const m3ssd_block_dims* d, const m3ssd_block_weights* w, cons
   a.th = reinterpret_cast<float*>(base + ws.th);
   const size_t smem = sizeof(float) * (size_t)(2 * d->ngroups + d->nheads);
   if (smem > 48 * 1024) return M3SSD_ERR_UNSUPPORTED;
-  const bool w16 = aligned(a.Bw, 16) && aligned(a.Cw, 16) && aligned(a.Bbias, 16) &&
-                   aligned(a.Cbias, 16);
+  const bool w16 = aligned(a.Bw, 16) && aligned(a.Cw, 16);
   if (w16 && vec_shape(a.H, a.P, a.N, a.G))
     block_prep_vec_kernel<<<(unsigned)M, kPrepThreads, smem, s>>>(a);
   else
@@ -416,6 +406,10 @@ m3ssd_status m3ssd_block_fwd(const m3ssd_block_dims* dims, const m3ssd_block_wei
   if (cache_out &&
       (!cache_out->angle || !cache_out->ssm || !cache_out->x_prev || !cache_out->b_prev))
     return M3SSD_ERR_INVALID_ARG;
+  for (const m3ssd_cache* c : {cache_in, cache_out})
+    if (c && !(aligned(c->angle, 4) && aligned(c->ssm, 4) && aligned(c->x_prev, 4) &&
+               aligned(c->b_prev, 4)))
+      return M3SSD_ERR_INVALID_ARG;
   const size_t need = m3ssd_block_workspace_size(dims);
   if (workspace_bytes < need || !workspace || !aligned(workspace, 256)) return M3SSD_ERR_WORKSPACE;
   if (dims->batch == 0) return M3SSD_OK;
@@ -427,31 +421,46 @@ m3ssd_status m3ssd_block_fwd(const m3ssd_block_dims* dims, const m3ssd_block_wei
     st = front(dims, w, u, M, base, ws, s);
     if (st != M3SSD_OK) return st;
   }
-  // the scan; the incoming b_prev is copied first, so that the outgoing one may
-  // overwrite the same buffer
-  const m3ssd_dims sd = scan_dims(dims, dims->seqlen);
-  m3ssd_fwd_extra ex{};
+  // the scan, with the head biases of B and C applied inside it; the incoming
+  // b_prev is copied first, so that the outgoing one may overwrite the same buffer
+  FwdArgs a{};
+  a.b = dims->batch; a.L = dims->seqlen; a.H = dims->nheads; a.P = dims->headdim;
+  a.N = dims->dstate; a.G = dims->ngroups; a.chunk = 0; a.bf16 = true;
+  a.X = base + ws.x;
+  a.logdecay = reinterpret_cast<const float*>(base + ws.ld);
+  a.beta = reinterpret_cast<const float*>(base + ws.be);
+  a.gamma = reinterpret_cast<const float*>(base + ws.ga);
+  a.B = base + ws.B;
+  a.C = base + ws.C;
+  a.theta = reinterpret_cast<const float*>(base + ws.th);
+  a.D = w->D;
+  a.Bbias = w->B_bias;
+  a.Cbias = w->C_bias;
+  a.Y = base + ws.y;
   if (cache_in) {
-    const size_t bytes = (size_t)dims->batch * dims->nheads * dims->dstate * sizeof(float);
+    const size_t bytes = (size_t)dims->batch * dims->ngroups * dims->dstate * sizeof(float);
     if (cudaMemcpyAsync(base + ws.bp, cache_in->b_prev, bytes, cudaMemcpyDeviceToDevice, s) !=
         cudaSuccess)
       return M3SSD_ERR_CUDA;
-    ex.angle0 = cache_in->angle;
-    ex.xprev0 = cache_in->x_prev;
-    ex.bprev0 = reinterpret_cast<const float*>(base + ws.bp);
+    a.h0 = cache_in->ssm;
+    a.angle0 = cache_in->angle;
+    a.xprev0 = cache_in->x_prev;
+    a.bprev0 = reinterpret_cast<const float*>(base + ws.bp);
   }
   if (cache_out) {
-    ex.angleT = cache_out->angle;
-    ex.xprevT = cache_out->x_prev;
-    ex.bprevT = cache_out->b_prev;
+    a.hT = cache_out->ssm;
+    a.angleT = cache_out->angle;
+    a.xprevT = cache_out->x_prev;
+    a.bprevT = cache_out->b_prev;
   }
-  st = m3ssd_fwd(&sd, base + ws.x, reinterpret_cast<const float*>(base + ws.ld),
-                 reinterpret_cast<const float*>(base + ws.be),
-                 reinterpret_cast<const float*>(base + ws.ga), base + ws.B, base + ws.C,
-                 reinterpret_cast<const float*>(base + ws.th), w->D,
-                 cache_in ? cache_in->ssm : nullptr, base + ws.y,
-                 cache_out ? cache_out->ssm : nullptr, &ex, nullptr, 0, stream);
-  if (st != M3SSD_OK || M == 0) return st;
+  const bool chunked = fwd_chunk_supported(a);
+  if (!chunked && !scan_shape_ok(dims)) return M3SSD_ERR_UNSUPPORTED;
+  const cudaError_t e = chunked ? launch_fwd_chunk(a, s) : launch_fwd_seq(a, s);
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    return M3SSD_ERR_CUDA;
+  }
+  if (M == 0) return M3SSD_OK;
   return back(dims, w, M, base, ws, out, s);
 }
 
@@ -462,6 +471,9 @@ m3ssd_status m3ssd_block_step(const m3ssd_block_dims* dims, const m3ssd_block_we
   m3ssd_status st = check_block(dims, w);
   if (st != M3SSD_OK) return st;
   if (!cache || !cache->angle || !cache->ssm || !cache->x_prev || !cache->b_prev)
+    return M3SSD_ERR_INVALID_ARG;
+  if (!(aligned(cache->angle, 4) && aligned(cache->ssm, 4) && aligned(cache->x_prev, 4) &&
+        aligned(cache->b_prev, 4)))
     return M3SSD_ERR_INVALID_ARG;
   const int64_t M = dims->batch;
   if (M > 0 && (!u_t || !out_t || !aligned(u_t, 16) || !aligned(out_t, 16)))
@@ -477,12 +489,26 @@ m3ssd_status m3ssd_block_step(const m3ssd_block_dims* dims, const m3ssd_block_we
   char* base = static_cast<char*>(workspace);
   st = front(&one, w, u_t, M, base, ws, s);
   if (st != M3SSD_OK) return st;
-  const m3ssd_dims sd = scan_dims(&one, 1);
-  st = m3ssd_step(&sd, base + ws.x, reinterpret_cast<const float*>(base + ws.ld),
-                  reinterpret_cast<const float*>(base + ws.be),
-                  reinterpret_cast<const float*>(base + ws.ga), base + ws.B, base + ws.C,
-                  reinterpret_cast<const float*>(base + ws.th), w->D, cache, base + ws.y, stream);
-  if (st != M3SSD_OK) return st;
+  StepArgs a{};
+  a.b = M; a.H = dims->nheads; a.P = dims->headdim; a.N = dims->dstate; a.G = dims->ngroups;
+  a.bf16 = true;
+  a.x_t = base + ws.x;
+  a.logdecay_t = reinterpret_cast<const float*>(base + ws.ld);
+  a.beta_t = reinterpret_cast<const float*>(base + ws.be);
+  a.gamma_t = reinterpret_cast<const float*>(base + ws.ga);
+  a.B_t = base + ws.B;
+  a.C_t = base + ws.C;
+  a.theta_t = reinterpret_cast<const float*>(base + ws.th);
+  a.D = w->D;
+  a.angle = cache->angle; a.ssm = cache->ssm; a.x_prev = cache->x_prev; a.b_prev = cache->b_prev;
+  a.y_t = base + ws.y;
+  a.Bbias = w->B_bias;
+  a.Cbias = w->C_bias;
+  if (!scan_shape_ok(&one)) return M3SSD_ERR_UNSUPPORTED;
+  if (launch_step(a, s) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return M3SSD_ERR_CUDA;
+  }
   return back(&one, w, M, base, ws, out_t, s);
 }
 

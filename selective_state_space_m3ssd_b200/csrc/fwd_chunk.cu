@@ -338,6 +338,20 @@ __global__ void __launch_bounds__(kThreads, 2)
   __syncthreads();
   tc5::fence_after_sync();
   const uint32_t tmem = sm.tmem;
+  // head biases of B and C for this thread's elements 4 lane .. 4 lane + 3 of a
+  // row (real parts: elements 4 lane, 4 lane + 2; imaginary: 4 lane + 1, 4 lane + 3)
+  const bool has_bbias = a.Bbias != nullptr, has_cbias = a.Cbias != nullptr;
+  float2 bbr = make_float2(0.f, 0.f), bbi = bbr, cbr = bbr, cbi = bbr;
+  if (has_bbias && !ctrl) {
+    const float4 v = *reinterpret_cast<const float4*>(a.Bbias + h * NS + 4 * lane);
+    bbr = make_float2(v.x, v.z);
+    bbi = make_float2(v.y, v.w);
+  }
+  if (has_cbias && !ctrl) {
+    const float4 v = *reinterpret_cast<const float4*>(a.Cbias + h * NS + 4 * lane);
+    cbr = make_float2(v.x, v.z);
+    cbi = make_float2(v.y, v.w);
+  }
   // this warp's TMEM lane quarter (rows of the M=64 and M=128 accumulators)
   const uint32_t tlane = (uint32_t)(32 * (warp & 3)) << 16;
 
@@ -478,12 +492,20 @@ __global__ void __launch_bounds__(kThreads, 2)
         float2 bre = make_float2(__uint_as_float(bw2.x << 16), __uint_as_float(bw2.y << 16));
         float2 bim = make_float2(__uint_as_float(bw2.x & 0xffff0000u),
                                  __uint_as_float(bw2.y & 0xffff0000u));
+        if (has_bbias) {
+          bre = __fadd2_rn(bre, bbr);
+          bim = __fadd2_rn(bim, bbi);
+        }
         if (ROT) {
           uint2* pc = reinterpret_cast<uint2*>(sm.C + o);
           const uint2 cw2 = *pc;
-          const float2 cre = make_float2(__uint_as_float(cw2.x << 16), __uint_as_float(cw2.y << 16));
-          const float2 cim = make_float2(__uint_as_float(cw2.x & 0xffff0000u),
-                                         __uint_as_float(cw2.y & 0xffff0000u));
+          float2 cre = make_float2(__uint_as_float(cw2.x << 16), __uint_as_float(cw2.y << 16));
+          float2 cim = make_float2(__uint_as_float(cw2.x & 0xffff0000u),
+                                   __uint_as_float(cw2.y & 0xffff0000u));
+          if (has_cbias) {
+            cre = __fadd2_rn(cre, cbr);
+            cim = __fadd2_rn(cim, cbi);
+          }
           const float2 ang = __fadd2_rn(psi[k], base);
           float s0, c0, s1, c1;
           __sincosf(ang.x, &s0, &c0);
@@ -720,12 +742,14 @@ bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 bool fwd_chunk_supported(const FwdArgs& a) {
   return a.bf16 && a.N == NS && a.P == PD && a.L > 0 && (a.chunk == 0 || a.chunk == Q) &&
          al16(a.X) && al16(a.B) && al16(a.C) && al16(a.Y) && al16(a.theta) && al16(a.h0) &&
-         al16(a.hT) && al16(a.logdecay);
+         al16(a.hT) && al16(a.logdecay) && al16(a.Bbias) && al16(a.Cbias);
 }
 
 cudaError_t launch_fwd_chunk(const FwdArgs& a, cudaStream_t s) {
   if (a.b * a.H == 0) return cudaSuccess;
-  if (a.theta != nullptr || a.angle0 != nullptr) return launch_variant<true>(a, s);
+  // the rotation phase also applies the head biases of B and C
+  if (a.theta != nullptr || a.angle0 != nullptr || a.Bbias != nullptr || a.Cbias != nullptr)
+    return launch_variant<true>(a, s);
   return launch_variant<false>(a, s);
 }
 

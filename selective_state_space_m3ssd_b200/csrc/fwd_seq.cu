@@ -49,8 +49,10 @@ __global__ void __launch_bounds__(kThreads) fwd_seq_kernel(FwdArgs a) {
     phi[i] = ph;
     float s, c;
     sincosf(ph, &s, &c);
-    const float b0 = a.bprev0 ? a.bprev0[(b * G + g) * N + 2 * i] : 0.f;
-    const float b1 = a.bprev0 ? a.bprev0[(b * G + g) * N + 2 * i + 1] : 0.f;
+    const float b0 = (a.bprev0 ? a.bprev0[(b * G + g) * N + 2 * i] : 0.f) +
+                     (a.Bbias ? a.Bbias[h * N + 2 * i] : 0.f);
+    const float b1 = (a.bprev0 ? a.bprev0[(b * G + g) * N + 2 * i + 1] : 0.f) +
+                     (a.Bbias ? a.Bbias[h * N + 2 * i + 1] : 0.f);
     const float2 r = rot2(c, s, b0, b1);
     Bbuf[N + 2 * i] = r.x;
     Bbuf[N + 2 * i + 1] = r.y;
@@ -72,8 +74,18 @@ __global__ void __launch_bounds__(kThreads) fwd_seq_kernel(FwdArgs a) {
       phi[i] = ph;
       float s, c;
       sincosf(ph, &s, &c);
-      const float2 rb = rot2(c, s, to_f32(Bm[tg * N + 2 * i]), to_f32(Bm[tg * N + 2 * i + 1]));
-      const float2 rc = rot2(c, s, to_f32(Cm[tg * N + 2 * i]), to_f32(Cm[tg * N + 2 * i + 1]));
+      float b0 = to_f32(Bm[tg * N + 2 * i]), b1 = to_f32(Bm[tg * N + 2 * i + 1]);
+      float c0 = to_f32(Cm[tg * N + 2 * i]), c1 = to_f32(Cm[tg * N + 2 * i + 1]);
+      if (a.Bbias) {
+        b0 += a.Bbias[h * N + 2 * i];
+        b1 += a.Bbias[h * N + 2 * i + 1];
+      }
+      if (a.Cbias) {
+        c0 += a.Cbias[h * N + 2 * i];
+        c1 += a.Cbias[h * N + 2 * i + 1];
+      }
+      const float2 rb = rot2(c, s, b0, b1);
+      const float2 rc = rot2(c, s, c0, c1);
       Bc[2 * i] = rb.x;
       Bc[2 * i + 1] = rb.y;
       Cb[2 * i] = rc.x;

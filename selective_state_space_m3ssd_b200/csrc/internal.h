@@ -28,6 +28,12 @@ struct FwdArgs {
   float* angleT;       // nullable
   float* xprevT;       // nullable
   float* bprevT;       // nullable
+  // Head-specific additive biases of B and C, (H, N) fp32, nullable: every use
+  // of B (including the cache's bprev0) reads B + Bbias[h], likewise C.  Used by
+  // the block (its QK-normed B, C per group plus a bias per head); the public
+  // scan entry points leave them NULL.
+  const float* Bbias;
+  const float* Cbias;
 };
 
 struct StepArgs {
@@ -46,6 +52,8 @@ struct StepArgs {
   float* x_prev;
   float* b_prev;
   void* y_t;
+  const float* Bbias;  // nullable, as in FwdArgs
+  const float* Cbias;  // nullable
 };
 
 // Everything one backward launch needs (gradients are fp32; the nullable

@@ -68,9 +68,20 @@ __global__ void __launch_bounds__(kThreads) step_kernel(StepArgs a) {
     float s, c, s0, c0;
     sincosf(ph, &s, &c);
     sincosf(ang, &s0, &c0);
-    const float2 rb = rot2(c, s, to_f32(Bt[2 * i]), to_f32(Bt[2 * i + 1]));
-    const float2 rc = rot2(c, s, to_f32(Ct[2 * i]), to_f32(Ct[2 * i + 1]));
-    const float2 rp = rot2(c0, s0, bprev[2 * i], bprev[2 * i + 1]);
+    float bx = to_f32(Bt[2 * i]), by = to_f32(Bt[2 * i + 1]);
+    float cx = to_f32(Ct[2 * i]), cy = to_f32(Ct[2 * i + 1]);
+    float px = bprev[2 * i], py = bprev[2 * i + 1];
+    if (a.Bbias) {
+      const float u0 = a.Bbias[h * N + 2 * i], u1 = a.Bbias[h * N + 2 * i + 1];
+      bx += u0; by += u1; px += u0; py += u1;
+    }
+    if (a.Cbias) {
+      cx += a.Cbias[h * N + 2 * i];
+      cy += a.Cbias[h * N + 2 * i + 1];
+    }
+    const float2 rb = rot2(c, s, bx, by);
+    const float2 rc = rot2(c, s, cx, cy);
+    const float2 rp = rot2(c0, s0, px, py);
     Bb[2 * i] = rb.x; Bb[2 * i + 1] = rb.y;
     Cb[2 * i] = rc.x; Cb[2 * i + 1] = rc.y;
     Bpb[2 * i] = rp.x; Bpb[2 * i + 1] = rp.y;
@@ -167,9 +178,20 @@ __global__ void __launch_bounds__(kThreads128) step_kernel_n128p64(StepArgs a) {
     float s, c, s0, c0;
     sincosf(ph, &s, &c);
     sincosf(ang, &s0, &c0);
-    const float2 rb = rot2(c, s, to_f32(Bt[2 * i]), to_f32(Bt[2 * i + 1]));
-    const float2 rc = rot2(c, s, to_f32(Ct[2 * i]), to_f32(Ct[2 * i + 1]));
-    const float2 rp = rot2(c0, s0, bprev[2 * i], bprev[2 * i + 1]);
+    float bx = to_f32(Bt[2 * i]), by = to_f32(Bt[2 * i + 1]);
+    float cx = to_f32(Ct[2 * i]), cy = to_f32(Ct[2 * i + 1]);
+    float px = bprev[2 * i], py = bprev[2 * i + 1];
+    if (a.Bbias) {
+      const float u0 = a.Bbias[h * kN + 2 * i], u1 = a.Bbias[h * kN + 2 * i + 1];
+      bx += u0; by += u1; px += u0; py += u1;
+    }
+    if (a.Cbias) {
+      cx += a.Cbias[h * kN + 2 * i];
+      cy += a.Cbias[h * kN + 2 * i + 1];
+    }
+    const float2 rb = rot2(c, s, bx, by);
+    const float2 rc = rot2(c, s, cx, cy);
+    const float2 rp = rot2(c0, s0, px, py);
     Bb[2 * i] = rb.x; Bb[2 * i + 1] = rb.y;
     Cb[2 * i] = rc.x; Cb[2 * i + 1] = rc.y;
     Bpb[2 * i] = rp.x; Bpb[2 * i + 1] = rp.y;

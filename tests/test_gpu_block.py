@@ -86,7 +86,7 @@ def test_block_prefill_then_steps_match_the_forward(name):
     ref, ref_cache = ob.oracle_block_fwd(u.double().numpy(), _np(w), H, P, N, G,
                                          store=bf16_store)
     L1 = s.seqlen - 6
-    cache = m3.new_block_cache(s.batch, H, P, N, "cuda")
+    cache = m3.new_block_cache(s.batch, H, P, N, G, "cuda")
     pre = m3.block_fwd(ud[:, :L1].contiguous(), wd, cache_out=cache)
     torch.cuda.synchronize()
     check(pre, ref[:, :L1])
@@ -104,7 +104,7 @@ def test_block_fwd_continues_from_its_own_cache_in_place():
     s, u, w, ud, wd = setup("small_g2", seed=9)
     H, P, N, G = s.nheads, s.headdim, s.dstate, s.ngroups
     ref, _ = ob.oracle_block_fwd(u.double().numpy(), _np(w), H, P, N, G, store=bf16_store)
-    cache = m3.new_block_cache(s.batch, H, P, N, "cuda")
+    cache = m3.new_block_cache(s.batch, H, P, N, G, "cuda")
     m3.block_fwd(ud[:, :33].contiguous(), wd, cache_out=cache)
     tail = m3.block_fwd(ud[:, 33:].contiguous(), wd, cache_in=cache, cache_out=cache)
     torch.cuda.synchronize()

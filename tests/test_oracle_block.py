@@ -162,10 +162,11 @@ def test_block_cache_continues_a_sequence():
 MUTATIONS = {
     "gate by sigmoid instead of SiLU": ("return v * sigmoid(v)", "return sigmoid(v)"),
     "head bias before the norm": (
-        'Bh = bc_norm(s["B"], f("B_norm_w"), eps)[..., grp, :] + f("B_bias")',
-        'Bh = bc_norm(s["B"][..., grp, :] + f("B_bias"), f("B_norm_w"), eps)'),
-    "norm dropped on C": ('Ch = bc_norm(s["C"], f("C_norm_w"), eps)[..., grp, :] + f("C_bias")',
-                          'Ch = s["C"][..., grp, :] * f("C_norm_w") + f("C_bias")'),
+        'Bh = store(bc_norm(s["B"], f("B_norm_w"), eps))[..., grp, :] + f("B_bias")',
+        'Bh = store(bc_norm(s["B"][..., grp, :] + f("B_bias"), f("B_norm_w"), eps))'),
+    "norm dropped on C": (
+        'Ch = store(bc_norm(s["C"], f("C_norm_w"), eps))[..., grp, :] + f("C_bias")',
+        'Ch = store(s["C"] * f("C_norm_w"))[..., grp, :] + f("C_bias")'),
     "dt bias dropped": ('delta = softplus(s["dt"] + f("dt_bias"))', 'delta = softplus(s["dt"])'),
     "angle not scaled by the step": ('theta = delta[..., None] * s["theta"]',
                                      'theta = s["theta"]'),

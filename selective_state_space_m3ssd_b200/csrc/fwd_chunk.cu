@@ -218,7 +218,7 @@ struct TmaMaps {
   CUtensorMap X;      // bf16 (p, head, token, batch), box 64 x 1 x 64 x 1, 128-byte swizzle
 };
 
-template <bool ROT>
+template <bool ROT, bool BIAS>
 __global__ void __launch_bounds__(kThreads, 2)
     fwd_chunk_kernel(FwdArgs a, const __grid_constant__ TmaMaps tm) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -340,7 +340,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   const uint32_t tmem = sm.tmem;
   // head biases of B and C for this thread's elements 4 lane .. 4 lane + 3 of a
   // row (real parts: elements 4 lane, 4 lane + 2; imaginary: 4 lane + 1, 4 lane + 3)
-  const bool has_bbias = a.Bbias != nullptr, has_cbias = a.Cbias != nullptr;
+  const bool has_bbias = BIAS && a.Bbias != nullptr, has_cbias = BIAS && a.Cbias != nullptr;
   float2 bbr = make_float2(0.f, 0.f), bbi = bbr, cbr = bbr, cbi = bbr;
   if (has_bbias && !ctrl) {
     const float4 v = *reinterpret_cast<const float4*>(a.Bbias + h * NS + 4 * lane);
@@ -712,7 +712,7 @@ bool encode_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool ROT>
+template <bool ROT, bool BIAS>
 cudaError_t launch_variant(const FwdArgs& a, cudaStream_t s) {
   TmaMaps tm;
   memset(&tm, 0, sizeof(tm));
@@ -728,10 +728,10 @@ cudaError_t launch_variant(const FwdArgs& a, cudaStream_t s) {
                     CU_TENSOR_MAP_SWIZZLE_NONE);
   if (!ok) return cudaErrorInvalidValue;
   const size_t smem = sizeof(Smem) + 1024;
-  cudaError_t e = cudaFuncSetAttribute(fwd_chunk_kernel<ROT>,
+  cudaError_t e = cudaFuncSetAttribute(fwd_chunk_kernel<ROT, BIAS>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  fwd_chunk_kernel<ROT><<<(unsigned)(a.b * a.H), kThreads, smem, s>>>(a, tm);
+  fwd_chunk_kernel<ROT, BIAS><<<(unsigned)(a.b * a.H), kThreads, smem, s>>>(a, tm);
   return cudaGetLastError();
 }
 
@@ -747,10 +747,11 @@ bool fwd_chunk_supported(const FwdArgs& a) {
 
 cudaError_t launch_fwd_chunk(const FwdArgs& a, cudaStream_t s) {
   if (a.b * a.H == 0) return cudaSuccess;
-  // the rotation phase also applies the head biases of B and C
-  if (a.theta != nullptr || a.angle0 != nullptr || a.Bbias != nullptr || a.Cbias != nullptr)
-    return launch_variant<true>(a, s);
-  return launch_variant<false>(a, s);
+  // the rotation phase also applies the head biases of B and C (its own variant,
+  // so that the plain scan's kernel carries none of it)
+  if (a.Bbias != nullptr || a.Cbias != nullptr) return launch_variant<true, true>(a, s);
+  if (a.theta != nullptr || a.angle0 != nullptr) return launch_variant<true, false>(a, s);
+  return launch_variant<false, false>(a, s);
 }
 
 cudaError_t read_and_clear_wait_timeouts(unsigned int* count) {

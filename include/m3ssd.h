@@ -228,12 +228,16 @@ size_t m3ssd_bwd_workspace_size(const m3ssd_dims* dims);
  * fp32, NULL = 0), and writes the fp32 gradients in *grads.  The cache outputs
  * angleT, xprevT and bprevT take no upstream gradient.
  *
- * The sequential backward recomputes the forward in fp32 from state
- * checkpoints; group-shared gradients are summed over heads in a fixed
+ * The backward recomputes the forward in fp32 from state checkpoints.  At
+ * N = 128 with P a multiple of 16 it splits each sequence over P/16 CTAs of
+ * 16 state columns and sums the per-slice partials of the column-mixing
+ * gradients afterwards; other shapes run one CTA per sequence.  Either way
+ * every sum (over slices, the heads of a group, the batch) runs in a fixed
  * order, so results are deterministic.  Limits as the sequential forward:
  * N <= 256, P <= 256, N*P <= 16384 (else M3SSD_ERR_UNSUPPORTED).  workspace
  * must hold m3ssd_bwd_workspace_size(dims) bytes, 256-byte aligned (else
- * M3SSD_ERR_WORKSPACE).  No allocation, no synchronisation.
+ * M3SSD_ERR_WORKSPACE); the size depends on the path.  No allocation, no
+ * synchronisation.
  */
 m3ssd_status m3ssd_bwd(const m3ssd_dims* dims, const void* X, const float* logdecay,
                        const float* beta, const float* gamma, const void* B, const void* C,

@@ -109,3 +109,17 @@ def test_block_fwd_continues_from_its_own_cache_in_place():
     tail = m3.block_fwd(ud[:, 33:].contiguous(), wd, cache_in=cache, cache_out=cache)
     torch.cuda.synchronize()
     check(tail, ref[:, 33:])
+
+
+def test_block_at_model_size_one_batch_row():
+    # the block in the configuration the benchmark times (b8 L4096 d_model 1024,
+    # H32 P64 N128 G1): batch row 3 against the oracle with the same hand-offs
+    s = BLOCKS["model"]
+    u, w = make_block(s)
+    wd = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in w.items()}
+    out = m3.block_fwd(u.cuda(), wd)
+    torch.cuda.synchronize()
+    bi = 3
+    ref, _ = ob.oracle_block_fwd(u[bi:bi + 1].double().numpy(), _np(w), s.nheads, s.headdim,
+                                 s.dstate, s.ngroups, store=bf16_store)
+    check(out[bi:bi + 1], ref)

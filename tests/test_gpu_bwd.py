@@ -149,3 +149,25 @@ def test_bwd_split_is_deterministic():
     torch.cuda.synchronize()
     for k in g1:
         assert torch.equal(g1[k], g2[k]), k
+
+
+def test_bwd_full_siso_workload_one_batch_row():
+    # the backward in the launch configuration the benchmark times (b8 L4096 H32
+    # P64 N128 bf16, column-split kernel), checked on batch row 5: every gradient
+    # of its 32 heads, and dB / dC of its one group, which sum over those heads
+    from selective_state_space_m3ssd_b200.synth import slice_inputs
+    w = WORKLOADS["siso"]
+    inp = make_inputs(w)
+    gen = torch.Generator().manual_seed(123)
+    dY = torch.randn(inp["X"].shape, generator=gen).to(inp["X"].dtype)
+    dhT = torch.randn(w.batch, w.nheads, w.dstate, w.headdim, generator=gen) * 0.1
+    d = to_dev(inp)
+    got = m3.bwd(*(d.get(k) for k in ARGS), dY=dY.cuda(), dhT=dhT.cuda())
+    torch.cuda.synchronize()
+    bi = 5
+    sub = slice_inputs(inp, b=bi)
+    ref = oracle.oracle_bwd(**sub, dY=dY[bi:bi + 1], dhT=dhT[bi:bi + 1])
+    per_batch = {"dX", "dlogdecay", "dbeta", "dgamma", "dB", "dC", "dtheta", "dh0"}
+    for k in per_batch:
+        g = np64(got[k][bi:bi + 1])
+        assert rel_max_err(g, ref[k]) <= TOL, (k, rel_max_err(g, ref[k]))

@@ -643,8 +643,8 @@ def run_profile(args):
         print(json.dumps({"profile": "forward", "workload": w.name.replace("b8", "b2"),
                           "ms_per_step": fw["ms_per_step"], "launches": fw["launches"]}))
     elif args.profile == "backward":
-        # one (b, h) sequence group of the forward's workload: 32 heads x 4 column
-        # slices = 128 CTAs, L = 1024
+        # one batch row of the forward's workload at L = 1024: 32 (b, h) CTAs of
+        # the chunked backward
         w = WORKLOADS[FWD_KEY].with_(batch=1, seqlen=1024)
         inp = make_inputs(w)
         d = {k: (None if v is None else v.to(dev)) for k, v in inp.items()}

@@ -1,0 +1,817 @@
+// Chunked backward of the Mamba-3 SISO scan in fp32 (N = 128, P = 64, bf16 or
+// fp32 inputs), one CTA of 512 threads per (b, h).
+//
+// The recurrence ("TorchMamba" README, "Math notes", M3 SISO) over a chunk of
+// Q = 64 rows -- row 0 the token before the chunk (t0 - 1, the carry-in of the
+// trapezoid's beta term), rows 1..63 the chunk's tokens -- reads, with the
+// chunk-local decay sums cs_r (cs_0 = 0), cv_u = gamma_u alpha_{u+1} + beta_{u+1}
+// (gamma_0 := 0), W(r,u<r) = exp(cs_r - cs_{u+1}) cv_u, W(r,r) = gamma_r and
+// W_end(u) = W(63,u):
+//   y_r   = exp(cs_r) Cbar_r . h_prev + sum_u W(r,u) (Cbar_r . Bbar_u) x_u + D x_r
+//   h_end = exp(cs_63) h_prev + sum_u W_end(u) Bbar_u x_u^T.
+// Its adjoint, chunk by chunk in reverse with g = dL/dh_end, E = dY X^T,
+// G = Cbar Bbar^T, M = W o G, WE = W o E:
+//   dh_prev = exp(cs_63) g + Cbar^T (exp(cs) o dY)
+//   dX      = M^T dY + W_end o (Bbar g) + D dY            (row 0 goes to the previous chunk)
+//   dCbar   = exp(cs) o (dY h_prev^T) + WE Bbar
+//   dBbar   = WE^T Cbar + W_end o (X g^T)                 (row 0 goes to the previous chunk)
+//   dW = G o E, dW_end(u) = x_u . (Bbar_u g)   -> decay sums, cv, gamma, beta, logdecay,
+// plus exp(cs_r)'s own terms (Cbar_r . h_prev dy_r and <g, h_prev> at r = 63),
+// and the rotation adjoints dv = R(phi)^T dvbar, dphi_i, dtheta = suffix sums of dphi.
+//
+// Pass 1 walks the chunks forward and stores each chunk's starting state and
+// angle in the workspace.  Pass 2 walks them in reverse; every product is a
+// register-tiled loop over fp32 shared-memory tiles, and every cross-thread sum
+// runs in a fixed order (warp shuffles, then fixed-order shared-memory sums), so
+// the result does not depend on scheduling.  The group-shared dB, dC, dbprev0 and
+// dD are written per head and summed by a second kernel.
+#include "common.cuh"
+#include "internal.h"
+
+namespace m3ssd {
+namespace {
+
+constexpr int kQ = 64, QT = kQ - 1, kN = 128, kNH = kN / 2, kP = 64, kT = 512;
+constexpr int SB = kN + 4;  // row stride of the Bbar / Cbar tiles (floats)
+constexpr int SX = kP + 4;  // row stride of the 64-wide tiles
+
+size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct ChunkWs {
+  size_t hs, phs, dBh, dCh, dbph, dDbh, total;
+};
+ChunkWs chunk_ws_layout(int64_t b, int64_t L, int64_t H) {
+  const size_t bh = (size_t)(b * H), nC = (size_t)((L + QT - 1) / QT);
+  ChunkWs w{};
+  size_t o = 0;
+  auto take = [&](size_t floats) {
+    const size_t r = o;
+    o += al256(floats * sizeof(float));
+    return r;
+  };
+  w.hs = take(bh * (nC > 0 ? nC : 1) * kN * kP);
+  w.phs = take(bh * (nC > 0 ? nC : 1) * kNH);
+  w.dBh = take((size_t)(b * L * H) * kN);
+  w.dCh = take((size_t)(b * L * H) * kN);
+  w.dbph = take(bh * kN);
+  w.dDbh = take(bh);
+  w.total = o;
+  return w;
+}
+
+// Shared memory (floats).
+struct Sm {
+  float Bb[kQ * SB];   // B (raw), then Bbar (and W_end o Bbar in pass 1)
+  float Cb[kQ * SB];   // C, then Cbar
+  float Xs[kQ * SX];   // x rows
+  float Ys[kQ * SX];   // dy rows
+  float Hp[kP * SB];   // h_prev, transposed: (p, n)
+  float Gs[kP * SB];   // g = dL/dh_end, transposed: (p, n)
+  float Gm[kQ * SX];   // G, then M, then dphi
+  float Em[kQ * SX];   // E, then WE
+  float Vt[kQ * SX];   // theta (r, i), then the angles phi (r, i)
+  float cs[kQ], al[kQ], ga[kQ], be[kQ], cv[kQ], ecs[kQ], wend[kQ];
+  float dcsA[kQ], dcsB[kQ], dcv[kQ], dga[kQ], dwend[kQ], dcsY[kQ];
+  float red[kT / 32 * 4];
+  float phi0[kNH];     // angle at the chunk start (phi of row 0)
+  float cdx[2][kP];    // dX of row 0 of a chunk (carried back), by chunk parity
+  float cdb[2][kN];    // dBbar of row 0 of a chunk, by chunk parity
+  float run[kNH];      // sum of dphi over all later tokens
+  float misc[8];
+};
+static_assert(sizeof(Sm) <= 232448, "one CTA's shared memory");
+
+template <typename T>
+__device__ __forceinline__ float ld(const T* p, int64_t i) {
+  return to_f32(p[i]);
+}
+
+__device__ __forceinline__ float acc4(float acc, const float4 a, const float4 b) {
+  return fmaf(a.w, b.w, fmaf(a.z, b.z, fmaf(a.y, b.y, fmaf(a.x, b.x, acc))));
+}
+__device__ __forceinline__ float4 ld4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+__device__ __forceinline__ float2 ld2(const float* p) { return *reinterpret_cast<const float2*>(p); }
+__device__ __forceinline__ float comp(const float4 v, int m) {
+  return m == 0 ? v.x : m == 1 ? v.y : m == 2 ? v.z : v.w;
+}
+// sum over the 16 lanes of a half-warp (fixed order)
+__device__ __forceinline__ float half_sum(float v) {
+#pragma unroll
+  for (int o = 1; o < 16; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Sum of v over the CTA in a fixed order (warp shuffles, then warp 0 adds the
+// 16 warp sums in order); every thread gets the result.
+__device__ __forceinline__ float block_sum(float v, float* red, float* out) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float s = 0.f;
+    for (int w = 0; w < kT / 32; ++w) s += red[w];
+    *out = s;
+  }
+  __syncthreads();
+  return *out;
+}
+
+static_assert(kNH == kP, "theta rows share the x-row loop");
+
+template <typename T>
+__global__ void __launch_bounds__(kT, 1) bwd_chunk_kernel(BwdArgs a, ChunkWs ws) {
+  extern __shared__ __align__(16) unsigned char smraw[];
+  Sm& sm = *reinterpret_cast<Sm*>(smraw);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t H = a.H, G = a.G, L = a.L;
+  const int64_t bh = blockIdx.x, b = bh / H, h = bh % H, g = h / (H / G);
+  const int nC = (int)((L + QT - 1) / QT);
+  const T* X = static_cast<const T*>(a.X);
+  const T* Bg = static_cast<const T*>(a.B);
+  const T* Cg = static_cast<const T*>(a.C);
+  const T* dY = static_cast<const T*>(a.dY);
+  const float Dh = a.D ? a.D[h] : 0.f;
+  char* wsb = static_cast<char*>(a.workspace);
+  float* hs_ws = reinterpret_cast<float*>(wsb + ws.hs) + bh * (int64_t)nC * kN * kP;
+  float* ph_ws = reinterpret_cast<float*>(wsb + ws.phs) + bh * (int64_t)nC * kNH;
+  float* dBh = reinterpret_cast<float*>(wsb + ws.dBh);
+  float* dCh = reinterpret_cast<float*>(wsb + ws.dCh);
+  float* dbph = reinterpret_cast<float*>(wsb + ws.dbph);
+  float* dDbh = reinterpret_cast<float*>(wsb + ws.dDbh);
+
+  // ---- the inputs of chunk c: rows r <-> tokens t0 - 1 + r -------------------
+  auto load_chunk = [&](int c, bool bwd) {
+    const int64_t t0 = (int64_t)c * QT - 1;
+    for (int e = tid; e < kQ * kP; e += kT) {
+      const int r = e >> 6, p = e & 63;
+      const int64_t t = t0 + r;
+      const bool own = r > 0 && t < L;
+      float xv = 0.f;
+      if (t >= 0 && t < L)
+        xv = ld(X, ((b * L + t) * H + h) * kP + p);
+      else if (t == -1 && a.xprev0)
+        xv = a.xprev0[bh * kP + p];
+      sm.Xs[r * SX + p] = xv;
+      if (bwd) sm.Ys[r * SX + p] = own ? ld(dY, ((b * L + t) * H + h) * kP + p) : 0.f;
+      sm.Vt[r * SX + p] = (own && a.theta) ? a.theta[((b * L + t) * H + h) * kNH + p] : 0.f;
+    }
+    for (int e = tid; e < kQ * kN; e += kT) {
+      const int r = e >> 7, n = e & 127;
+      const int64_t t = t0 + r;
+      float bv = 0.f, cw = 0.f;
+      if (t >= 0 && t < L) {
+        const int64_t o = ((b * L + t) * G + g) * kN + n;
+        bv = ld(Bg, o);
+        if (bwd && r > 0) cw = ld(Cg, o);
+      } else if (t == -1 && a.bprev0) {
+        bv = a.bprev0[(b * G + g) * kN + n];
+      }
+      sm.Bb[r * SB + n] = bv;
+      if (bwd) sm.Cb[r * SB + n] = cw;
+    }
+    if (tid < kQ) {
+      const int r = tid;
+      const int64_t t = t0 + r;
+      const bool own = r > 0 && t < L;
+      const int64_t th = (b * L + (own ? t : 0)) * H + h;
+      sm.cs[r] = own ? a.logdecay[th] : 0.f;  // the raw logdecay until chunk_scalars
+      sm.ga[r] = own ? a.gamma[th] : 0.f;
+      sm.be[r] = (own && a.beta) ? a.beta[th] : 0.f;
+    }
+  };
+
+  // ---- chunk scalars: cs (inclusive sums of logdecay), alpha, exp(cs), cv, W_end
+  auto chunk_scalars = [&]() {
+    if (warp == 0) {
+      const float l0 = sm.cs[lane], l1 = sm.cs[lane + 32];
+      float s0 = l0, s1 = l1;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const float v0 = __shfl_up_sync(0xffffffffu, s0, o);
+        const float v1 = __shfl_up_sync(0xffffffffu, s1, o);
+        if (lane >= o) {
+          s0 += v0;
+          s1 += v1;
+        }
+      }
+      s1 += __shfl_sync(0xffffffffu, s0, 31);
+      sm.al[lane] = expf(l0);
+      sm.al[lane + 32] = expf(l1);
+      sm.cs[lane] = s0;
+      sm.cs[lane + 32] = s1;
+    }
+    __syncthreads();
+    if (tid < kQ) {
+      const int r = tid;
+      sm.ecs[r] = expf(sm.cs[r]);
+      sm.cv[r] = r < kQ - 1 ? sm.ga[r] * sm.al[r + 1] + sm.be[r + 1] : 0.f;
+    }
+    __syncthreads();
+    if (tid < kQ) {
+      const int u = tid;
+      sm.wend[u] = u < kQ - 1 ? expf(sm.cs[kQ - 1] - sm.cs[u + 1]) * sm.cv[u] : sm.ga[kQ - 1];
+    }
+    __syncthreads();
+  };
+
+  // ---- angles phi(r, i) = phi0[i] + sum_{k <= r} theta(k, i) in Vt, then the
+  // rotations of B (and C) in place
+  auto angles_rotate = [&](bool rot_c) {
+    {
+      const int i = tid & 63, grp = tid >> 6;
+      float run_ = 0.f;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int r = 8 * grp + k;
+        run_ += sm.Vt[r * SX + i];
+        sm.Vt[r * SX + i] = run_;
+      }
+      sm.Gm[grp * SX + i] = run_;  // segment totals (the Gram tile is free here)
+      __syncthreads();
+      float base = sm.phi0[i];
+      for (int q = 0; q < grp; ++q) base += sm.Gm[q * SX + i];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) sm.Vt[(8 * grp + k) * SX + i] += base;
+      __syncthreads();
+    }
+    for (int e = tid; e < kQ * kNH; e += kT) {
+      const int r = e >> 6, i = e & 63;
+      float sn, cs_;
+      fast_sincos(sm.Vt[r * SX + i], &sn, &cs_);
+      float* bp = &sm.Bb[r * SB + 2 * i];
+      const float b0 = bp[0], b1 = bp[1];
+      bp[0] = cs_ * b0 - sn * b1;
+      bp[1] = sn * b0 + cs_ * b1;
+      if (rot_c) {
+        float* cp = &sm.Cb[r * SB + 2 * i];
+        const float c0 = cp[0], c1 = cp[1];
+        cp[0] = cs_ * c0 - sn * c1;
+        cp[1] = sn * c0 + cs_ * c1;
+      }
+    }
+    __syncthreads();
+  };
+
+  // ---- pass 1: the state and the angle at every chunk start -----------------
+  // state tile of a thread: n in nq .. nq + 3, p in cq + 16 j
+  const int cq = tid & 15, nq = 4 * (tid >> 4);
+  {
+    float hreg[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        hreg[i][j] = a.h0 ? a.h0[(bh * kN + nq + i) * kP + cq + 16 * j] : 0.f;
+    if (tid < kNH) sm.phi0[tid] = wrap_angle(a.angle0 ? a.angle0[bh * kNH + tid] : 0.f);
+    __syncthreads();
+    for (int c = 0; c < nC; ++c) {
+      float* hw = hs_ws + (int64_t)c * kN * kP;
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) hw[(nq + i) * kP + cq + 16 * j] = hreg[i][j];
+      if (tid < kNH) ph_ws[(int64_t)c * kNH + tid] = sm.phi0[tid];
+      load_chunk(c, false);
+      __syncthreads();
+      chunk_scalars();
+      angles_rotate(false);
+      const float eE = sm.ecs[kQ - 1];
+      float acc[4][4] = {};
+      for (int u = 0; u < kQ; ++u) {
+        const float w = sm.wend[u];
+        const float4 bv = *reinterpret_cast<const float4*>(&sm.Bb[u * SB + nq]);
+        const float bw[4] = {w * bv.x, w * bv.y, w * bv.z, w * bv.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float xv = sm.Xs[u * SX + cq + 16 * j];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) acc[i][j] = fmaf(bw[i], xv, acc[i][j]);
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) hreg[i][j] = fmaf(eE, hreg[i][j], acc[i][j]);
+      __syncthreads();  // every read of this chunk's tiles is done
+      if (tid < kNH) sm.phi0[tid] = wrap_angle(sm.Vt[(kQ - 1) * SX + tid]);
+      __syncthreads();
+    }
+  }
+
+  // ---- pass 2: the chunks in reverse --------------------------------------
+  // tiles of 64-row products: rows r0 = 2 rq, r1 = r0 + 1; the rows of a warp
+  // are 4 warp .. 4 warp + 3, which bounds the triangular loops warp-uniformly
+  const int rq = tid >> 4, r0 = 2 * rq, r1 = r0 + 1;
+  const int wlo = 4 * warp, whi = 4 * warp + 3;
+  if (tid < kNH) sm.run[tid] = 0.f;
+  if (tid < kP) {
+    sm.cdx[0][tid] = 0.f;
+    sm.cdx[1][tid] = 0.f;
+  }
+  if (tid < kN) {
+    sm.cdb[0][tid] = 0.f;
+    sm.cdb[1][tid] = 0.f;
+  }
+  for (int e = tid; e < kN * kP; e += kT) {
+    const int n = e >> 6, p = e & 63;
+    sm.Gs[p * SB + n] = a.dhT ? a.dhT[(bh * kN + n) * kP + p] : 0.f;
+  }
+  float dDacc = 0.f;
+  __syncthreads();
+
+  for (int c = nC - 1; c >= 0; --c) {
+    const int cur = c & 1, nxt = cur ^ 1;
+    const int64_t t0 = (int64_t)c * QT - 1;  // token of row 0
+    auto own = [&](int r) { return r > 0 && t0 + r < L; };
+    {
+      const float* hw = hs_ws + (int64_t)c * kN * kP;
+      for (int e = tid; e < kN * kP; e += kT) {
+        const int n = e >> 6, p = e & 63;
+        sm.Hp[p * SB + n] = hw[e];
+      }
+      if (tid < kNH) sm.phi0[tid] = ph_ws[(int64_t)c * kNH + tid];
+    }
+    load_chunk(c, true);
+    __syncthreads();
+    chunk_scalars();
+    angles_rotate(true);
+
+    // -- G = Cbar Bbar^T and E = dY X^T on the lower triangle, then the mask
+    //    gradients of dW = G o E, M = W o G and WE = W o E
+    {
+      float gt[2][4], et[2][4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) gt[0][j] = gt[1][j] = et[0][j] = et[1][j] = 0.f;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (16 * j > whi) break;
+        const int u = cq + 16 * j;
+        for (int k = 0; k < kN; k += 4) {
+          const float4 bv = ld4(&sm.Bb[u * SB + k]);
+          gt[0][j] = acc4(gt[0][j], ld4(&sm.Cb[r0 * SB + k]), bv);
+          gt[1][j] = acc4(gt[1][j], ld4(&sm.Cb[r1 * SB + k]), bv);
+        }
+        for (int k = 0; k < kP; k += 4) {
+          const float4 xv = ld4(&sm.Xs[u * SX + k]);
+          et[0][j] = acc4(et[0][j], ld4(&sm.Ys[r0 * SX + k]), xv);
+          et[1][j] = acc4(et[1][j], ld4(&sm.Ys[r1 * SX + k]), xv);
+        }
+      }
+      float rowA[2] = {0.f, 0.f}, colB[4] = {0.f, 0.f, 0.f, 0.f}, colV[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const int r = r0 + i;
+        const float csr = sm.cs[r];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int u = cq + 16 * j;
+          const float dW = gt[i][j] * et[i][j];
+          float w = 0.f;
+          if (u < r) {
+            const float ex = expf(csr - sm.cs[u + 1]);
+            w = ex * sm.cv[u];
+            rowA[i] = fmaf(dW, w, rowA[i]);
+            colB[j] = fmaf(dW, w, colB[j]);
+            colV[j] = fmaf(dW, ex, colV[j]);
+          } else if (u == r) {
+            w = sm.ga[r];
+            sm.dga[r] = dW;
+          }
+          gt[i][j] *= w;  // M
+          et[i][j] *= w;  // WE
+        }
+        rowA[i] = half_sum(rowA[i]);
+      }
+      if (cq == 0) {
+        sm.dcsA[r0] = rowA[0];
+        sm.dcsA[r1] = rowA[1];
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        colB[j] += __shfl_xor_sync(0xffffffffu, colB[j], 16);
+        colV[j] += __shfl_xor_sync(0xffffffffu, colV[j], 16);
+      }
+      if (lane < 16) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          sm.Gm[warp * SX + cq + 16 * j] = colB[j];
+          sm.Em[warp * SX + cq + 16 * j] = colV[j];
+        }
+      }
+      __syncthreads();
+      if (tid < 2 * kQ) {
+        const int u = tid & 63;
+        const float* src = tid < kQ ? sm.Gm : sm.Em;
+        float s = 0.f;
+        for (int w = 0; w < kT / 32; ++w) s += src[w * SX + u];
+        (tid < kQ ? sm.dcsB : sm.dcv)[u] = s;
+      }
+      __syncthreads();
+#pragma unroll
+      for (int i = 0; i < 2; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          sm.Gm[(r0 + i) * SX + cq + 16 * j] = gt[i][j];
+          sm.Em[(r0 + i) * SX + cq + 16 * j] = et[i][j];
+        }
+      __syncthreads();
+    }
+
+    // -- dX = M^T dY + W_end o (Bbar g) + D dY, and dW_end(u) = x_u . (Bbar_u g)
+    {
+      float vt[2][4], xt[2][4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) vt[0][j] = vt[1][j] = xt[0][j] = xt[1][j] = 0.f;
+      for (int n = 0; n < kN; n += 4) {
+        const float4 b0 = ld4(&sm.Bb[r0 * SB + n]), b1 = ld4(&sm.Bb[r1 * SB + n]);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float4 gv = ld4(&sm.Gs[(cq + 16 * j) * SB + n]);
+          vt[0][j] = acc4(vt[0][j], b0, gv);
+          vt[1][j] = acc4(vt[1][j], b1, gv);
+        }
+      }
+      for (int r = wlo; r < kQ; ++r) {  // M(r, u) = 0 for r < u
+        const float2 m = ld2(&sm.Gm[r * SX + r0]);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float y = sm.Ys[r * SX + cq + 16 * j];
+          xt[0][j] = fmaf(m.x, y, xt[0][j]);
+          xt[1][j] = fmaf(m.y, y, xt[1][j]);
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const int u = r0 + i;
+        const float we = sm.wend[u];
+        float dwe = 0.f;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int p = cq + 16 * j;
+          const float xv = sm.Xs[u * SX + p], yv = sm.Ys[u * SX + p];
+          dwe = fmaf(xv, vt[i][j], dwe);
+          dDacc = fmaf(yv, xv, dDacc);
+          float dx = xt[i][j] + fmaf(we, vt[i][j], Dh * yv);
+          if (u == kQ - 1) dx += sm.cdx[nxt][p];
+          if (u == 0)
+            sm.cdx[cur][p] = dx;
+          else if (own(u))
+            a.dX[((b * L + t0 + u) * H + h) * kP + p] = dx;
+        }
+        dwe = half_sum(dwe);
+        if (cq == 0) sm.dwend[u] = dwe;
+      }
+    }
+    __syncthreads();  // M is dead: the Gram tile takes dphi next
+
+    // -- dCbar = exp(cs) o (dY h_prev^T) + WE Bbar, then its rotation adjoint;
+    //    columns 4 cq + 64 (k / 4) + k % 4 of rows r0, r1
+    {
+      float ac[2][8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) ac[0][k] = ac[1][k] = 0.f;
+      for (int p = 0; p < kP; p += 4) {
+        const float4 y0 = ld4(&sm.Ys[r0 * SX + p]), y1 = ld4(&sm.Ys[r1 * SX + p]);
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          const float4 h0 = ld4(&sm.Hp[(p + m) * SB + 4 * cq]);
+          const float4 h1 = ld4(&sm.Hp[(p + m) * SB + 4 * cq + 64]);
+          const float hv[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+          const float ya = comp(y0, m), yb = comp(y1, m);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            ac[0][k] = fmaf(ya, hv[k], ac[0][k]);
+            ac[1][k] = fmaf(yb, hv[k], ac[1][k]);
+          }
+        }
+      }
+      // exp(cs_r) Cbar_r . (dY h_prev^T)_r: the h_prev term of d cs_r
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const int r = r0 + i;
+        const float4 c0 = ld4(&sm.Cb[r * SB + 4 * cq]), c1 = ld4(&sm.Cb[r * SB + 4 * cq + 64]);
+        const float cv8[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+        float s = 0.f;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) s = fmaf(cv8[k], ac[i][k], s);
+        s = half_sum(s);
+        const float e = sm.ecs[r];
+        if (cq == 0) sm.dcsY[r] = e * s;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) ac[i][k] *= e;
+      }
+      for (int u = 0; u <= whi; u += 4) {  // WE(r, u) = 0 for u > r
+        const float4 w0 = ld4(&sm.Em[r0 * SX + u]), w1 = ld4(&sm.Em[r1 * SX + u]);
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          const float4 b0 = ld4(&sm.Bb[(u + m) * SB + 4 * cq]);
+          const float4 b1 = ld4(&sm.Bb[(u + m) * SB + 4 * cq + 64]);
+          const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+          const float wa = comp(w0, m), wb = comp(w1, m);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            ac[0][k] = fmaf(wa, bv[k], ac[0][k]);
+            ac[1][k] = fmaf(wb, bv[k], ac[1][k]);
+          }
+        }
+      }
+      // dC = R(phi)^T dCbar; dphi_i = Cbar x dCbar (the B part is added below)
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const int r = r0 + i;
+        const bool ok = own(r);
+        const int64_t ro = ((b * L + (ok ? t0 + r : 0)) * H + h) * kN;
+#pragma unroll
+        for (int k = 0; k < 8; k += 2) {
+          const int n = 4 * cq + 64 * (k >> 2) + (k & 3), pi = n >> 1;
+          float sn, cs_;
+          fast_sincos(sm.Vt[r * SX + pi], &sn, &cs_);
+          const float d0 = ac[i][k], d1 = ac[i][k + 1];
+          const float v0 = sm.Cb[r * SB + n], v1 = sm.Cb[r * SB + n + 1];
+          sm.Gm[r * SX + pi] = ok ? fmaf(d1, v0, -d0 * v1) : 0.f;
+          if (ok)
+            *reinterpret_cast<float2*>(&dCh[ro + n]) =
+                make_float2(fmaf(cs_, d0, sn * d1), fmaf(cs_, d1, -sn * d0));
+        }
+      }
+    }
+
+    // -- dBbar = WE^T Cbar + W_end o (X g^T), the carries of row 0 (this
+    //    chunk's carry-in token) and into row 63, then the rotation adjoint
+    {
+      float bb[2][8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) bb[0][k] = bb[1][k] = 0.f;
+      for (int p = 0; p < kP; p += 4) {
+        const float4 x0 = ld4(&sm.Xs[r0 * SX + p]), x1 = ld4(&sm.Xs[r1 * SX + p]);
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          const float4 g0 = ld4(&sm.Gs[(p + m) * SB + 4 * cq]);
+          const float4 g1 = ld4(&sm.Gs[(p + m) * SB + 4 * cq + 64]);
+          const float gv[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+          const float xa = comp(x0, m), xb = comp(x1, m);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            bb[0][k] = fmaf(xa, gv[k], bb[0][k]);
+            bb[1][k] = fmaf(xb, gv[k], bb[1][k]);
+          }
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const float we = sm.wend[r0 + i];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) bb[i][k] *= we;
+      }
+      for (int r = wlo; r < kQ; ++r) {  // WE(r, u) = 0 for r < u
+        const float2 w = ld2(&sm.Em[r * SX + r0]);
+        const float4 c0 = ld4(&sm.Cb[r * SB + 4 * cq]), c1 = ld4(&sm.Cb[r * SB + 4 * cq + 64]);
+        const float cv8[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          bb[0][k] = fmaf(w.x, cv8[k], bb[0][k]);
+          bb[1][k] = fmaf(w.y, cv8[k], bb[1][k]);
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const int r = r0 + i;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int n = 4 * cq + 64 * (k >> 2) + (k & 3);
+          if (r == kQ - 1) bb[i][k] += sm.cdb[nxt][n];
+          if (r == 0) sm.cdb[cur][n] = bb[i][k];
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const int r = r0 + i;
+        if (!own(r)) continue;
+        const int64_t ro = ((b * L + t0 + r) * H + h) * kN;
+#pragma unroll
+        for (int k = 0; k < 8; k += 2) {
+          const int n = 4 * cq + 64 * (k >> 2) + (k & 3), pi = n >> 1;
+          float sn, cs_;
+          fast_sincos(sm.Vt[r * SX + pi], &sn, &cs_);
+          const float d0 = bb[i][k], d1 = bb[i][k + 1];
+          const float v0 = sm.Bb[r * SB + n], v1 = sm.Bb[r * SB + n + 1];
+          sm.Gm[r * SX + pi] += fmaf(d1, v0, -d0 * v1);
+          *reinterpret_cast<float2*>(&dBh[ro + n]) =
+              make_float2(fmaf(cs_, d0, sn * d1), fmaf(cs_, d1, -sn * d0));
+        }
+      }
+    }
+
+    // -- dh_prev = exp(cs_63) g + Cbar^T (exp(cs) o dY) and <g, h_prev>
+    float dh[4][4];
+    {
+      const float eE = sm.ecs[kQ - 1];
+      float ghp = 0.f;
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int o = (cq + 16 * j) * SB + nq + i;
+          const float gv = sm.Gs[o];
+          ghp = fmaf(gv, sm.Hp[o], ghp);
+          dh[i][j] = eE * gv;
+        }
+      for (int r = 1; r < kQ; ++r) {
+        const float e = sm.ecs[r];
+        const float4 cv = ld4(&sm.Cb[r * SB + nq]);
+        const float cw[4] = {e * cv.x, e * cv.y, e * cv.z, e * cv.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float y = sm.Ys[r * SX + cq + 16 * j];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) dh[i][j] = fmaf(cw[i], y, dh[i][j]);
+        }
+      }
+      block_sum(ghp, sm.red, &sm.misc[0]);  // ends with a barrier: g is free
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) sm.Gs[(cq + 16 * j) * SB + nq + i] = dh[i][j];
+
+    // -- the scalar chain: decay sums -> cv -> gamma, beta, logdecay
+    if (warp == 0) {
+      const float eE = sm.ecs[kQ - 1];
+      float endsum = 0.f;
+      float dcsv[2];
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int u = lane + 32 * k;
+        if (u < kQ - 1) endsum = fmaf(sm.dwend[u], sm.wend[u], endsum);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) endsum += __shfl_xor_sync(0xffffffffu, endsum, o);
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int r = lane + 32 * k;
+        float d = sm.dcsA[r] + sm.dcsY[r];
+        if (r >= 1) d -= sm.dcsB[r - 1] + sm.dwend[r - 1] * sm.wend[r - 1];
+        if (r == kQ - 1) d += endsum + eE * sm.misc[0];
+        dcsv[k] = d;
+        if (r < kQ - 1) sm.dcv[r] = fmaf(sm.dwend[r], expf(sm.cs[kQ - 1] - sm.cs[r + 1]), sm.dcv[r]);
+      }
+      __syncwarp();
+      // suffix sums of dcs over the chunk's rows
+      float s1 = dcsv[1], s0 = dcsv[0];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const float v1 = __shfl_down_sync(0xffffffffu, s1, o);
+        const float v0 = __shfl_down_sync(0xffffffffu, s0, o);
+        if (lane + o < 32) {
+          s1 += v1;
+          s0 += v0;
+        }
+      }
+      s0 += __shfl_sync(0xffffffffu, s1, 0);
+      const float suf[2] = {s0, s1};
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int r = lane + 32 * k;
+        if (!own(r)) continue;
+        const float dcvp = sm.dcv[r - 1];
+        float dg = sm.dga[r];
+        if (r == kQ - 1) dg += sm.dwend[kQ - 1];
+        if (r < kQ - 1) dg = fmaf(sm.dcv[r], sm.al[r + 1], dg);
+        const float dal = dcvp * sm.ga[r - 1];
+        const int64_t th = (b * L + t0 + r) * H + h;
+        a.dlogdecay[th] = fmaf(sm.al[r], dal, suf[k]);
+        a.dgamma[th] = dg;
+        if (a.dbeta) a.dbeta[th] = dcvp;
+      }
+    }
+
+    // -- dtheta: suffix sums of dphi over the tokens after, in 8-row segments
+    {
+      const int i = tid & 63, grp = tid >> 6;
+      float tmp[8];
+      float s = 0.f;
+#pragma unroll
+      for (int k = 7; k >= 0; --k) {
+        s += sm.Gm[(8 * grp + k) * SX + i];
+        tmp[k] = s;
+      }
+      sm.Em[grp * SX + i] = s;
+      __syncthreads();
+      float base = sm.run[i];
+      for (int q = 7; q > grp; --q) base += sm.Em[q * SX + i];
+      if (a.dtheta) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int r = 8 * grp + k;
+          if (own(r)) a.dtheta[((b * L + t0 + r) * H + h) * kNH + i] = base + tmp[k];
+        }
+      }
+      __syncthreads();
+      if (grp == 0) sm.run[i] = base + tmp[0];
+      __syncthreads();
+    }
+  }
+
+  // ---- the cache token before the sequence: dh0, dxprev0, dbprev0, dangle0, dD
+  if (a.dh0)
+    for (int e = tid; e < kN * kP; e += kT) {
+      const int n = e >> 6, p = e & 63;
+      a.dh0[(bh * kN + n) * kP + p] = sm.Gs[p * SB + n];
+    }
+  if (a.dxprev0 && tid < kP) a.dxprev0[bh * kP + tid] = sm.cdx[0][tid];
+  if (tid < kNH) {
+    const int i = tid;
+    float sn, cs_;
+    fast_sincos(sm.phi0[i], &sn, &cs_);
+    const float d0 = sm.cdb[0][2 * i], d1 = sm.cdb[0][2 * i + 1];
+    float v0 = 0.f, v1 = 0.f;
+    if (a.bprev0) {
+      v0 = a.bprev0[(b * G + g) * kN + 2 * i];
+      v1 = a.bprev0[(b * G + g) * kN + 2 * i + 1];
+    }
+    const float vb0 = cs_ * v0 - sn * v1, vb1 = sn * v0 + cs_ * v1;
+    dbph[bh * kN + 2 * i] = fmaf(cs_, d0, sn * d1);
+    dbph[bh * kN + 2 * i + 1] = fmaf(cs_, d1, -sn * d0);
+    if (a.dangle0) a.dangle0[bh * kNH + i] = sm.run[i] + fmaf(d1, vb0, -d0 * vb1);
+  }
+  const float dDs = block_sum(dDacc, sm.red, &sm.misc[1]);
+  if (tid == 0) dDbh[bh] = dDs;
+}
+
+// Sums over the heads of a group (dB, dC, dbprev0) and over the batch (dD),
+// each in a fixed order.
+__global__ void bwd_chunk_reduce_kernel(BwdArgs a, ChunkWs ws) {
+  const int64_t H = a.H, G = a.G, hpg = H / G;
+  const char* wsb = static_cast<const char*>(a.workspace);
+  const float* dBh = reinterpret_cast<const float*>(wsb + ws.dBh);
+  const float* dCh = reinterpret_cast<const float*>(wsb + ws.dCh);
+  const float* dbph = reinterpret_cast<const float*>(wsb + ws.dbph);
+  const float* dDbh = reinterpret_cast<const float*>(wsb + ws.dDbh);
+  const int64_t nBC = a.b * a.L * G * kN, nbp = a.b * G * kN;
+  const int64_t total = nBC + nbp + H;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += stride) {
+    int64_t r = i;
+    if (r < nBC) {  // dB, dC: (b, L, G, N)
+      const int64_t nn = r % kN, row = r / kN, gg = row % G, bt = row / G;
+      float sb = 0.f, sc = 0.f;
+      for (int64_t q = 0; q < hpg; ++q) {
+        const int64_t src = (bt * H + gg * hpg + q) * kN + nn;
+        sb += dBh[src];
+        sc += dCh[src];
+      }
+      a.dB[r] = sb;
+      a.dC[r] = sc;
+      continue;
+    }
+    r -= nBC;
+    if (r < nbp) {  // dbprev0: (b, G, N)
+      const int64_t nn = r % kN, row = r / kN, gg = row % G, bb = row / G;
+      float v = 0.f;
+      for (int64_t q = 0; q < hpg; ++q) v += dbph[(bb * H + gg * hpg + q) * kN + nn];
+      if (a.dbprev0) a.dbprev0[r] = v;
+      continue;
+    }
+    r -= nbp;
+    float v = 0.f;  // dD: (H)
+    for (int64_t bb = 0; bb < a.b; ++bb) v += dDbh[bb * H + r];
+    if (a.dD) a.dD[r] = v;
+  }
+}
+
+}  // namespace
+
+bool bwd_chunk_supported(int64_t N, int64_t P) { return N == kN && P == kP; }
+
+size_t bwd_chunk_workspace_bytes(int64_t b, int64_t L, int64_t H) {
+  return chunk_ws_layout(b, L, H).total;
+}
+
+cudaError_t launch_bwd_chunk(const BwdArgs& a, cudaStream_t s) {
+  if (a.b * a.H == 0) return cudaSuccess;
+  const ChunkWs ws = chunk_ws_layout(a.b, a.L, a.H);
+  const int smem = (int)sizeof(Sm);
+  cudaError_t e;
+  if (a.bf16) {
+    e = cudaFuncSetAttribute(bwd_chunk_kernel<__nv_bfloat16>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    bwd_chunk_kernel<__nv_bfloat16><<<(unsigned)(a.b * a.H), kT, smem, s>>>(a, ws);
+  } else {
+    e = cudaFuncSetAttribute(bwd_chunk_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem);
+    if (e != cudaSuccess) return e;
+    bwd_chunk_kernel<float><<<(unsigned)(a.b * a.H), kT, smem, s>>>(a, ws);
+  }
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int64_t total = a.b * a.L * a.G * kN + a.b * a.G * kN + a.H;
+  const int64_t blocks = (total + 255) / 256;
+  const unsigned rg = (unsigned)(blocks < 148 * 32 ? (blocks > 0 ? blocks : 1) : 148 * 32);
+  bwd_chunk_reduce_kernel<<<rg, 256, 0, s>>>(a, ws);
+  return cudaGetLastError();
+}
+
+}  // namespace m3ssd

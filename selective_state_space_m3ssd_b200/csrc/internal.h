@@ -90,6 +90,12 @@ cudaError_t launch_bwd_seq(const BwdArgs& a, cudaStream_t s);
 bool bwd_split_supported(int64_t N, int64_t P);
 size_t bwd_split_workspace_bytes(int64_t b, int64_t L, int64_t H, int64_t P);
 cudaError_t launch_bwd_split(const BwdArgs& a, cudaStream_t s);
+// The chunked backward (N = 128, P = 64): one CTA per (b, h) walks chunks of 63
+// tokens, forward for the chunk-start states, then in reverse; per-head shares
+// of the group-summed gradients in the workspace.
+bool bwd_chunk_supported(int64_t N, int64_t P);
+size_t bwd_chunk_workspace_bytes(int64_t b, int64_t L, int64_t H);
+cudaError_t launch_bwd_chunk(const BwdArgs& a, cudaStream_t s);
 
 // MIMO rank R (1..8): layouts as the SISO ones with a trailing rank axis on X,
 // Y, B, C, x_prev, b_prev (and the extra cache inputs / outputs).

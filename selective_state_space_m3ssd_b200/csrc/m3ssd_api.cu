@@ -190,6 +190,8 @@ m3ssd_status m3ssd_mimo_step(const m3ssd_dims* dims, int32_t rank, const void* x
 
 size_t m3ssd_bwd_workspace_size(const m3ssd_dims* dims) {
   if (check_dims(dims) != M3SSD_OK || !general_shape_ok(dims)) return 0;
+  if (m3ssd::bwd_chunk_supported(dims->dstate, dims->headdim))
+    return m3ssd::bwd_chunk_workspace_bytes(dims->batch, dims->seqlen, dims->nheads);
   if (m3ssd::bwd_split_supported(dims->dstate, dims->headdim))
     return m3ssd::bwd_split_workspace_bytes(dims->batch, dims->seqlen, dims->nheads,
                                             dims->headdim);
@@ -240,6 +242,7 @@ m3ssd_status m3ssd_bwd(const m3ssd_dims* dims, const void* X, const float* logde
   a.dD = grads->dD; a.dh0 = grads->dh0; a.dangle0 = grads->dangle0; a.dxprev0 = grads->dxprev0;
   a.dbprev0 = grads->dbprev0; a.workspace = workspace;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (m3ssd::bwd_chunk_supported(a.N, a.P)) return from_cuda(m3ssd::launch_bwd_chunk(a, s));
   return from_cuda(m3ssd::bwd_split_supported(a.N, a.P) ? m3ssd::launch_bwd_split(a, s)
                                                          : m3ssd::launch_bwd_seq(a, s));
 }

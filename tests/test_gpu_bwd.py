@@ -151,9 +151,56 @@ def test_bwd_split_is_deterministic():
         assert torch.equal(g1[k], g2[k]), k
 
 
+# N = 128 and P = 64: the chunked backward (one CTA per (b, h), chunks of 63
+# tokens plus the carry-in row, forward pass for the chunk-start states, then
+# the chunks in reverse; group sums in a second kernel)
+CHUNK = WORKLOADS["siso"].with_(batch=2, nheads=4, ngroups=2, seed=131)
+
+
+@pytest.mark.parametrize("L", [1, 2, 62, 63, 64, 126, 127, 200])
+def test_bwd_chunk_lengths(L):
+    inp = with_cache_inputs(make_inputs(CHUNK.with_(seqlen=L, dtype="f32")), seed=L)
+    dY, dhT = upstream(inp, 60 + L)
+    got, ref = run_both(inp, dY, dhT)
+    check_all(got, ref)
+
+
+@pytest.mark.parametrize("variant", ["no_beta", "no_theta", "no_cache", "no_dhT", "one_group",
+                                     "bf16"])
+def test_bwd_chunk_paths(variant):
+    w = CHUNK.with_(seqlen=150, dtype="f32")
+    if variant == "no_beta":
+        w = w.with_(has_beta=False)
+    if variant == "no_theta":
+        w = w.with_(has_theta=False)
+    if variant == "one_group":
+        w = w.with_(ngroups=1)
+    if variant == "bf16":
+        w = w.with_(dtype="bf16")
+    inp = make_inputs(w)
+    if variant != "no_cache":
+        inp = with_cache_inputs(inp, seed=12)
+    dY, dhT = upstream(inp, 7, with_dhT=variant != "no_dhT")
+    got, ref = run_both(inp, dY, dhT)
+    check_all(got, ref)
+
+
+def test_bwd_chunk_is_deterministic():
+    inp = with_cache_inputs(make_inputs(CHUNK.with_(seqlen=140)), seed=4)
+    dY, dhT = upstream(inp, 23)
+    d = to_dev(inp)
+    args = [d.get(k) for k in ARGS]
+    extra = dict(angle0=d.get("angle0"), xprev0=d.get("xprev0"), bprev0=d.get("bprev0"))
+    g1 = m3.bwd(*args, dY=dY.cuda(), dhT=dhT.cuda(), **extra)
+    g2 = m3.bwd(*args, dY=dY.cuda(), dhT=dhT.cuda(), **extra)
+    torch.cuda.synchronize()
+    for k in g1:
+        assert torch.equal(g1[k], g2[k]), k
+
+
 def test_bwd_full_siso_workload_one_batch_row():
     # the backward in the launch configuration the benchmark times (b8 L4096 H32
-    # P64 N128 bf16, column-split kernel), checked on batch row 5: every gradient
+    # P64 N128 bf16, chunked kernel), checked on batch row 5: every gradient
     # of its 32 heads, and dB / dC of its one group, which sum over those heads
     from selective_state_space_m3ssd_b200.synth import slice_inputs
     w = WORKLOADS["siso"]

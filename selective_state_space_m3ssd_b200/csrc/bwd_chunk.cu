@@ -59,7 +59,7 @@ ChunkWs chunk_ws_layout(int64_t b, int64_t L, int64_t H) {
   return w;
 }
 
-// Shared memory (floats).
+// Shared memory (floats).  The workspace holds each chunk-start state as (p, n).
 struct Sm {
   float Bb[kQ * SB];   // B (raw), then Bbar (and W_end o Bbar in pass 1)
   float Cb[kQ * SB];   // C, then Cbar
@@ -81,9 +81,47 @@ struct Sm {
 };
 static_assert(sizeof(Sm) <= 232448, "one CTA's shared memory");
 
-template <typename T>
-__device__ __forceinline__ float ld(const T* p, int64_t i) {
-  return to_f32(p[i]);
+// n consecutive elements from p into out (fp32), in 16-byte loads when vec
+template <int n>
+__device__ __forceinline__ void ldn(const float* p, bool vec, float* out) {
+  if (vec) {
+#pragma unroll
+    for (int k = 0; k < n / 4; ++k) {
+      const float4 v = *reinterpret_cast<const float4*>(p + 4 * k);
+      out[4 * k] = v.x;
+      out[4 * k + 1] = v.y;
+      out[4 * k + 2] = v.z;
+      out[4 * k + 3] = v.w;
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < n; ++k) out[k] = p[k];
+  }
+}
+template <int n>
+__device__ __forceinline__ void ldn(const __nv_bfloat16* p, bool vec, float* out) {
+  if (vec) {
+#pragma unroll
+    for (int k = 0; k < n / 8; ++k) {
+      const uint4 raw = *reinterpret_cast<const uint4*>(p + 8 * k);
+      const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[q]));
+        out[8 * k + 2 * q] = f.x;
+        out[8 * k + 2 * q + 1] = f.y;
+      }
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < n; ++k) out[k] = __bfloat162float(p[k]);
+  }
+}
+template <int n>
+__device__ __forceinline__ void stn(float* dst, const float* v) {
+#pragma unroll
+  for (int k = 0; k < n / 4; ++k)
+    *reinterpret_cast<float4*>(dst + 4 * k) = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
 }
 
 __device__ __forceinline__ float acc4(float acc, const float4 a, const float4 b) {
@@ -142,43 +180,55 @@ __global__ void __launch_bounds__(kT, 1) bwd_chunk_kernel(BwdArgs a, ChunkWs ws)
   float* dDbh = reinterpret_cast<float*>(wsb + ws.dDbh);
 
   // ---- the inputs of chunk c: rows r <-> tokens t0 - 1 + r -------------------
+  // 16-byte loads where every base pointer allows them (rows are whole multiples)
+  const bool vec = ((reinterpret_cast<uintptr_t>(X) | reinterpret_cast<uintptr_t>(Bg) |
+                     reinterpret_cast<uintptr_t>(Cg) | reinterpret_cast<uintptr_t>(dY) |
+                     reinterpret_cast<uintptr_t>(a.theta)) & 15) == 0;
   auto load_chunk = [&](int c, bool bwd) {
     const int64_t t0 = (int64_t)c * QT - 1;
-    for (int e = tid; e < kQ * kP; e += kT) {
-      const int r = e >> 6, p = e & 63;
-      const int64_t t = t0 + r;
-      const bool own = r > 0 && t < L;
-      float xv = 0.f;
-      if (t >= 0 && t < L)
-        xv = ld(X, ((b * L + t) * H + h) * kP + p);
-      else if (t == -1 && a.xprev0)
-        xv = a.xprev0[bh * kP + p];
-      sm.Xs[r * SX + p] = xv;
-      if (bwd) sm.Ys[r * SX + p] = own ? ld(dY, ((b * L + t) * H + h) * kP + p) : 0.f;
-      sm.Vt[r * SX + p] = (own && a.theta) ? a.theta[((b * L + t) * H + h) * kNH + p] : 0.f;
+    const int r = tid >> 3, sg = tid & 7;  // row r, columns 8 sg .. (16 sg .. for N)
+    const int64_t t = t0 + r;
+    const bool in = t >= 0 && t < L, own = r > 0 && t < L;
+    const int64_t th = (b * L + (in ? t : 0)) * H + h, tg = (b * L + (in ? t : 0)) * G + g;
+    float xv[8], yv[8], tv[8], bv[16], cv[16];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) xv[k] = yv[k] = tv[k] = 0.f;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) bv[k] = cv[k] = 0.f;
+    if (in) {
+      ldn<8>(X + th * kP + 8 * sg, vec, xv);
+      ldn<16>(Bg + tg * kN + 16 * sg, vec, bv);
+    } else if (t == -1) {
+      if (a.xprev0) ldn<8>(a.xprev0 + bh * kP + 8 * sg, false, xv);
+      if (a.bprev0) ldn<16>(a.bprev0 + (b * G + g) * kN + 16 * sg, false, bv);
     }
-    for (int e = tid; e < kQ * kN; e += kT) {
-      const int r = e >> 7, n = e & 127;
-      const int64_t t = t0 + r;
-      float bv = 0.f, cw = 0.f;
-      if (t >= 0 && t < L) {
-        const int64_t o = ((b * L + t) * G + g) * kN + n;
-        bv = ld(Bg, o);
-        if (bwd && r > 0) cw = ld(Cg, o);
-      } else if (t == -1 && a.bprev0) {
-        bv = a.bprev0[(b * G + g) * kN + n];
+    if (own && a.theta) ldn<8>(a.theta + th * kNH + 8 * sg, vec, tv);
+    if (bwd && own) {
+      ldn<8>(dY + th * kP + 8 * sg, vec, yv);
+      ldn<16>(Cg + tg * kN + 16 * sg, vec, cv);
+    }
+    float sc[3] = {0.f, 0.f, 0.f};
+    if (tid < kQ) {
+      const int rr = tid;
+      const int64_t tt = t0 + rr;
+      if (rr > 0 && tt < L) {
+        const int64_t ts = (b * L + tt) * H + h;
+        sc[0] = a.logdecay[ts];
+        sc[1] = a.gamma[ts];
+        sc[2] = a.beta ? a.beta[ts] : 0.f;
       }
-      sm.Bb[r * SB + n] = bv;
-      if (bwd) sm.Cb[r * SB + n] = cw;
+    }
+    stn<8>(&sm.Xs[r * SX + 8 * sg], xv);
+    stn<8>(&sm.Vt[r * SX + 8 * sg], tv);
+    stn<16>(&sm.Bb[r * SB + 16 * sg], bv);
+    if (bwd) {
+      stn<8>(&sm.Ys[r * SX + 8 * sg], yv);
+      stn<16>(&sm.Cb[r * SB + 16 * sg], cv);
     }
     if (tid < kQ) {
-      const int r = tid;
-      const int64_t t = t0 + r;
-      const bool own = r > 0 && t < L;
-      const int64_t th = (b * L + (own ? t : 0)) * H + h;
-      sm.cs[r] = own ? a.logdecay[th] : 0.f;  // the raw logdecay until chunk_scalars
-      sm.ga[r] = own ? a.gamma[th] : 0.f;
-      sm.be[r] = (own && a.beta) ? a.beta[th] : 0.f;
+      sm.cs[tid] = sc[0];  // the raw logdecay until chunk_scalars
+      sm.ga[tid] = sc[1];
+      sm.be[tid] = sc[2];
     }
   };
 
@@ -267,11 +317,11 @@ __global__ void __launch_bounds__(kT, 1) bwd_chunk_kernel(BwdArgs a, ChunkWs ws)
     if (tid < kNH) sm.phi0[tid] = wrap_angle(a.angle0 ? a.angle0[bh * kNH + tid] : 0.f);
     __syncthreads();
     for (int c = 0; c < nC; ++c) {
-      float* hw = hs_ws + (int64_t)c * kN * kP;
+      float* hw = hs_ws + (int64_t)c * kN * kP;  // (p, n)
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) hw[(nq + i) * kP + cq + 16 * j] = hreg[i][j];
+      for (int j = 0; j < 4; ++j)
+        *reinterpret_cast<float4*>(&hw[(cq + 16 * j) * kN + nq]) =
+            make_float4(hreg[0][j], hreg[1][j], hreg[2][j], hreg[3][j]);
       if (tid < kNH) ph_ws[(int64_t)c * kNH + tid] = sm.phi0[tid];
       load_chunk(c, false);
       __syncthreads();
@@ -325,15 +375,22 @@ __global__ void __launch_bounds__(kT, 1) bwd_chunk_kernel(BwdArgs a, ChunkWs ws)
     const int cur = c & 1, nxt = cur ^ 1;
     const int64_t t0 = (int64_t)c * QT - 1;  // token of row 0
     auto own = [&](int r) { return r > 0 && t0 + r < L; };
+    float4 hpv[4];  // the chunk-start state, (p, n) float4s
     {
       const float* hw = hs_ws + (int64_t)c * kN * kP;
-      for (int e = tid; e < kN * kP; e += kT) {
-        const int n = e >> 6, p = e & 63;
-        sm.Hp[p * SB + n] = hw[e];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int idx = tid + kT * k;
+        hpv[k] = *reinterpret_cast<const float4*>(&hw[(idx >> 5) * kN + 4 * (idx & 31)]);
       }
       if (tid < kNH) sm.phi0[tid] = ph_ws[(int64_t)c * kNH + tid];
     }
     load_chunk(c, true);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int idx = tid + kT * k;
+      *reinterpret_cast<float4*>(&sm.Hp[(idx >> 5) * SB + 4 * (idx & 31)]) = hpv[k];
+    }
     __syncthreads();
     chunk_scalars();
     angles_rotate(true);
@@ -344,20 +401,29 @@ __global__ void __launch_bounds__(kT, 1) bwd_chunk_kernel(BwdArgs a, ChunkWs ws)
       float gt[2][4], et[2][4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) gt[0][j] = gt[1][j] = et[0][j] = et[1][j] = 0.f;
+      // columns past the warp's last row are masked out (warp-uniform test)
+      const int nj = whi / 16 + 1;
+#pragma unroll 2
+      for (int k = 0; k < kN; k += 4) {
+        const float4 c0 = ld4(&sm.Cb[r0 * SB + k]), c1 = ld4(&sm.Cb[r1 * SB + k]);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        if (16 * j > whi) break;
-        const int u = cq + 16 * j;
-        for (int k = 0; k < kN; k += 4) {
-          const float4 bv = ld4(&sm.Bb[u * SB + k]);
-          gt[0][j] = acc4(gt[0][j], ld4(&sm.Cb[r0 * SB + k]), bv);
-          gt[1][j] = acc4(gt[1][j], ld4(&sm.Cb[r1 * SB + k]), bv);
-        }
-        for (int k = 0; k < kP; k += 4) {
-          const float4 xv = ld4(&sm.Xs[u * SX + k]);
-          et[0][j] = acc4(et[0][j], ld4(&sm.Ys[r0 * SX + k]), xv);
-          et[1][j] = acc4(et[1][j], ld4(&sm.Ys[r1 * SX + k]), xv);
-        }
+        for (int j = 0; j < 4; ++j)
+          if (j < nj) {
+            const float4 bv = ld4(&sm.Bb[(cq + 16 * j) * SB + k]);
+            gt[0][j] = acc4(gt[0][j], c0, bv);
+            gt[1][j] = acc4(gt[1][j], c1, bv);
+          }
+      }
+#pragma unroll 2
+      for (int k = 0; k < kP; k += 4) {
+        const float4 y0 = ld4(&sm.Ys[r0 * SX + k]), y1 = ld4(&sm.Ys[r1 * SX + k]);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (j < nj) {
+            const float4 xv = ld4(&sm.Xs[(cq + 16 * j) * SX + k]);
+            et[0][j] = acc4(et[0][j], y0, xv);
+            et[1][j] = acc4(et[1][j], y1, xv);
+          }
       }
       float rowA[2] = {0.f, 0.f}, colB[4] = {0.f, 0.f, 0.f, 0.f}, colV[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll

@@ -185,6 +185,31 @@ def test_bwd_chunk_paths(variant):
     check_all(got, ref)
 
 
+def _offset_copy(t):
+    # the same values at an address one element past a 16-byte boundary
+    flat = torch.empty(t.numel() + 1, dtype=t.dtype, device=t.device)
+    v = flat[1:].view(t.shape)
+    v.copy_(t)
+    return v
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_bwd_chunk_unaligned_inputs(dtype):
+    # X, B, C, theta and dY off the 16-byte grid: the element-wise load path
+    inp = with_cache_inputs(make_inputs(CHUNK.with_(seqlen=90, dtype=dtype)), seed=5)
+    dY, dhT = upstream(inp, 24)
+    ref = oracle.oracle_bwd(**inp, dY=dY, dhT=dhT)
+    d = to_dev(inp)
+    for k in ("X", "B", "C", "theta"):
+        d[k] = _offset_copy(d[k])
+    dYd = _offset_copy(dY.cuda())
+    assert dYd.data_ptr() % 16 != 0
+    got = m3.bwd(*(d.get(k) for k in ARGS), dY=dYd, dhT=dhT.cuda(), angle0=d.get("angle0"),
+                 xprev0=d.get("xprev0"), bprev0=d.get("bprev0"))
+    torch.cuda.synchronize()
+    check_all({k: np64(v) for k, v in got.items()}, ref)
+
+
 def test_bwd_chunk_is_deterministic():
     inp = with_cache_inputs(make_inputs(CHUNK.with_(seqlen=140)), seed=4)
     dY, dhT = upstream(inp, 23)

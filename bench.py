@@ -63,7 +63,7 @@ def load_peaks() -> dict:
         with open(p) as f:
             d = json.load(f)
         return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
-                "source": "measured"}
+                "sm_max_mhz": float(d.get("sm_max_mhz", 1965.0)), "source": "measured"}
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
 
 
@@ -515,14 +515,34 @@ def bench_backward(w, dev, steps, world, d, peaks):
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         ms = float(t.item())
     algo = nbytes(*args, dY, dhT, *grads.values())
-    achieved = algo / (ms / 1e3) / 1e9
+    flops = bwd_chunk_flops(w.batch, w.seqlen, w.nheads) * world
+    tflops = flops / (ms / 1e3) / 1e12
+    peak = fp32_simt_tflops(peaks)
     return {"metric": "bwd Mtokens/s", "value": w.batch * w.seqlen * world / (ms / 1e3) / 1e6,
             "unit": "Mtokens/s", "ms_per_step": ms, "steps": steps,
-            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
-                         "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
-                         "algo_bytes_per_step": algo, "traffic": None,
-                         "peak_source": peaks["source"]},
-            "kernel": "bwd_seq_kernel + bwd_reduce_kernel (sequential fp32, 2 launches)"}
+            "roofline": {"bound": "alu", "achieved": tflops, "peak": peak, "unit": "TFLOP/s",
+                         "frac": tflops / peak, "algo_flops_per_step": flops, "traffic": None,
+                         "peak_source": "148 SMs x 128 fp32 lanes x 2 FLOP x max SM clock"},
+            "hbm": {"algo_bytes_per_step": algo, "achieved_gbs": algo / (ms / 1e3) / 1e9,
+                    "frac": algo / (ms / 1e3) / 1e9 / peaks["hbm_gbs"]},
+            "kernel": "bwd_chunk_kernel + bwd_chunk_reduce_kernel (chunked fp32, 2 launches)"}
+
+
+def bwd_chunk_flops(b: int, L: int, H: int, N: int = 128, P: int = 64, Q: int = 64) -> int:
+    """Product FLOPs of the chunked backward per call: per chunk of Q rows, the
+    state pass's (W_end o Bbar)^T X (2 N P Q), then G = Cbar Bbar^T and
+    E = dY X^T on their lower triangles (Q^2 N + Q^2 P), Bbar g (2 Q N P),
+    M^T dY (Q^2 P), dY h^T (2 Q N P), WE Bbar and WE^T Cbar (2 Q^2 N),
+    X g^T (2 Q N P) and Cbar^T (exp(cs) dY) (2 N P Q)."""
+    per_chunk = 2 * N * P * Q + Q * Q * N + Q * Q * P + 2 * Q * N * P + Q * Q * P + \
+        2 * Q * N * P + 2 * Q * Q * N + 2 * Q * N * P + 2 * N * P * Q
+    return b * H * -(-L // (Q - 1)) * per_chunk
+
+
+def fp32_simt_tflops(peaks: dict) -> float:
+    """fp32 FMA peak of the SIMT pipes: 148 SMs x 128 lanes x 2 FLOP at the
+    maximum SM clock (from the measured-peaks record, else 1,965 MHz)."""
+    return 148 * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
 
 
 def run_ours(args):

@@ -124,8 +124,13 @@ __device__ __forceinline__ void stn(float* dst, const float* v) {
     *reinterpret_cast<float4*>(dst + 4 * k) = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
 }
 
-__device__ __forceinline__ float acc4(float acc, const float4 a, const float4 b) {
-  return fmaf(a.w, b.w, fmaf(a.z, b.z, fmaf(a.y, b.y, fmaf(a.x, b.x, acc))));
+// Packed fp32 pairs (two FMAs an instruction on sm_100).
+__device__ __forceinline__ float2 lo2(const float4 v) { return make_float2(v.x, v.y); }
+__device__ __forceinline__ float2 hi2(const float4 v) { return make_float2(v.z, v.w); }
+__device__ __forceinline__ float2 bc2(float v) { return make_float2(v, v); }
+// a . b over four terms, accumulated as two partial sums in the lanes of acc
+__device__ __forceinline__ float2 acc4(float2 acc, const float4 a, const float4 b) {
+  return __ffma2_rn(hi2(a), hi2(b), __ffma2_rn(lo2(a), lo2(b), acc));
 }
 __device__ __forceinline__ float4 ld4(const float* p) { return *reinterpret_cast<const float4*>(p); }
 __device__ __forceinline__ float2 ld2(const float* p) { return *reinterpret_cast<const float2*>(p); }
@@ -328,22 +333,27 @@ __global__ void __launch_bounds__(kT, 1) bwd_chunk_kernel(BwdArgs a, ChunkWs ws)
       chunk_scalars();
       angles_rotate(false);
       const float eE = sm.ecs[kQ - 1];
-      float acc[4][4] = {};
+      float2 acc[2][4];  // rows (nq + 2 ii, nq + 2 ii + 1), column cq + 16 j
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[0][j] = acc[1][j] = make_float2(0.f, 0.f);
       for (int u = 0; u < kQ; ++u) {
-        const float w = sm.wend[u];
-        const float4 bv = *reinterpret_cast<const float4*>(&sm.Bb[u * SB + nq]);
-        const float bw[4] = {w * bv.x, w * bv.y, w * bv.z, w * bv.w};
+        const float2 w = bc2(sm.wend[u]);
+        const float4 bv = ld4(&sm.Bb[u * SB + nq]);
+        const float2 bw0 = __fmul2_rn(w, lo2(bv)), bw1 = __fmul2_rn(w, hi2(bv));
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          const float xv = sm.Xs[u * SX + cq + 16 * j];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) acc[i][j] = fmaf(bw[i], xv, acc[i][j]);
+          const float2 xv = bc2(sm.Xs[u * SX + cq + 16 * j]);
+          acc[0][j] = __ffma2_rn(bw0, xv, acc[0][j]);
+          acc[1][j] = __ffma2_rn(bw1, xv, acc[1][j]);
         }
       }
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) hreg[i][j] = fmaf(eE, hreg[i][j], acc[i][j]);
+      for (int j = 0; j < 4; ++j) {
+        hreg[0][j] = fmaf(eE, hreg[0][j], acc[0][j].x);
+        hreg[1][j] = fmaf(eE, hreg[1][j], acc[0][j].y);
+        hreg[2][j] = fmaf(eE, hreg[2][j], acc[1][j].x);
+        hreg[3][j] = fmaf(eE, hreg[3][j], acc[1][j].y);
+      }
       __syncthreads();  // every read of this chunk's tiles is done
       if (tid < kNH) sm.phi0[tid] = wrap_angle(sm.Vt[(kQ - 1) * SX + tid]);
       __syncthreads();
@@ -398,9 +408,9 @@ __global__ void __launch_bounds__(kT, 1) bwd_chunk_kernel(BwdArgs a, ChunkWs ws)
     // -- G = Cbar Bbar^T and E = dY X^T on the lower triangle, then the mask
     //    gradients of dW = G o E, M = W o G and WE = W o E
     {
-      float gt[2][4], et[2][4];
+      float2 gp[2][4], ep[2][4];  // two partial sums each
 #pragma unroll
-      for (int j = 0; j < 4; ++j) gt[0][j] = gt[1][j] = et[0][j] = et[1][j] = 0.f;
+      for (int j = 0; j < 4; ++j) gp[0][j] = gp[1][j] = ep[0][j] = ep[1][j] = make_float2(0.f, 0.f);
       // columns past the warp's last row are masked out (warp-uniform test)
       const int nj = whi / 16 + 1;
 #pragma unroll 2
@@ -410,8 +420,8 @@ __global__ void __launch_bounds__(kT, 1) bwd_chunk_kernel(BwdArgs a, ChunkWs ws)
         for (int j = 0; j < 4; ++j)
           if (j < nj) {
             const float4 bv = ld4(&sm.Bb[(cq + 16 * j) * SB + k]);
-            gt[0][j] = acc4(gt[0][j], c0, bv);
-            gt[1][j] = acc4(gt[1][j], c1, bv);
+            gp[0][j] = acc4(gp[0][j], c0, bv);
+            gp[1][j] = acc4(gp[1][j], c1, bv);
           }
       }
 #pragma unroll 2
@@ -421,10 +431,18 @@ __global__ void __launch_bounds__(kT, 1) bwd_chunk_kernel(BwdArgs a, ChunkWs ws)
         for (int j = 0; j < 4; ++j)
           if (j < nj) {
             const float4 xv = ld4(&sm.Xs[(cq + 16 * j) * SX + k]);
-            et[0][j] = acc4(et[0][j], y0, xv);
-            et[1][j] = acc4(et[1][j], y1, xv);
+            ep[0][j] = acc4(ep[0][j], y0, xv);
+            ep[1][j] = acc4(ep[1][j], y1, xv);
           }
       }
+      float gt[2][4], et[2][4];
+#pragma unroll
+      for (int i = 0; i < 2; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          gt[i][j] = gp[i][j].x + gp[i][j].y;
+          et[i][j] = ep[i][j].x + ep[i][j].y;
+        }
       float rowA[2] = {0.f, 0.f}, colB[4] = {0.f, 0.f, 0.f, 0.f}, colV[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
@@ -488,24 +506,33 @@ __global__ void __launch_bounds__(kT, 1) bwd_chunk_kernel(BwdArgs a, ChunkWs ws)
     // -- dX = M^T dY + W_end o (Bbar g) + D dY, and dW_end(u) = x_u . (Bbar_u g)
     {
       float vt[2][4], xt[2][4];
+      {
+        float2 vp[2][4];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) vt[0][j] = vt[1][j] = xt[0][j] = xt[1][j] = 0.f;
-      for (int n = 0; n < kN; n += 4) {
-        const float4 b0 = ld4(&sm.Bb[r0 * SB + n]), b1 = ld4(&sm.Bb[r1 * SB + n]);
+        for (int j = 0; j < 4; ++j) vp[0][j] = vp[1][j] = make_float2(0.f, 0.f);
+        for (int n = 0; n < kN; n += 4) {
+          const float4 b0 = ld4(&sm.Bb[r0 * SB + n]), b1 = ld4(&sm.Bb[r1 * SB + n]);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const float4 gv = ld4(&sm.Gs[(cq + 16 * j) * SB + n]);
-          vt[0][j] = acc4(vt[0][j], b0, gv);
-          vt[1][j] = acc4(vt[1][j], b1, gv);
+          for (int j = 0; j < 4; ++j) {
+            const float4 gv = ld4(&sm.Gs[(cq + 16 * j) * SB + n]);
+            vp[0][j] = acc4(vp[0][j], b0, gv);
+            vp[1][j] = acc4(vp[1][j], b1, gv);
+          }
         }
-      }
-      for (int r = wlo; r < kQ; ++r) {  // M(r, u) = 0 for r < u
-        const float2 m = ld2(&sm.Gm[r * SX + r0]);
+        float2 xp[4];  // (row r0, row r1) pairs
+#pragma unroll
+        for (int j = 0; j < 4; ++j) xp[j] = make_float2(0.f, 0.f);
+        for (int r = wlo; r < kQ; ++r) {  // M(r, u) = 0 for r < u
+          const float2 m = ld2(&sm.Gm[r * SX + r0]);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) xp[j] = __ffma2_rn(m, bc2(sm.Ys[r * SX + cq + 16 * j]), xp[j]);
+        }
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          const float y = sm.Ys[r * SX + cq + 16 * j];
-          xt[0][j] = fmaf(m.x, y, xt[0][j]);
-          xt[1][j] = fmaf(m.y, y, xt[1][j]);
+          vt[0][j] = vp[0][j].x + vp[0][j].y;
+          vt[1][j] = vp[1][j].x + vp[1][j].y;
+          xt[0][j] = xp[j].x;
+          xt[1][j] = xp[j].y;
         }
       }
 #pragma unroll
@@ -535,21 +562,21 @@ __global__ void __launch_bounds__(kT, 1) bwd_chunk_kernel(BwdArgs a, ChunkWs ws)
     // -- dCbar = exp(cs) o (dY h_prev^T) + WE Bbar, then its rotation adjoint;
     //    columns 4 cq + 64 (k / 4) + k % 4 of rows r0, r1
     {
-      float ac[2][8];
+      float2 ac[2][4];  // column pairs (n, n + 1) of rows r0, r1
 #pragma unroll
-      for (int k = 0; k < 8; ++k) ac[0][k] = ac[1][k] = 0.f;
+      for (int q = 0; q < 4; ++q) ac[0][q] = ac[1][q] = make_float2(0.f, 0.f);
       for (int p = 0; p < kP; p += 4) {
         const float4 y0 = ld4(&sm.Ys[r0 * SX + p]), y1 = ld4(&sm.Ys[r1 * SX + p]);
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
           const float4 h0 = ld4(&sm.Hp[(p + m) * SB + 4 * cq]);
           const float4 h1 = ld4(&sm.Hp[(p + m) * SB + 4 * cq + 64]);
-          const float hv[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
-          const float ya = comp(y0, m), yb = comp(y1, m);
+          const float2 hv[4] = {lo2(h0), hi2(h0), lo2(h1), hi2(h1)};
+          const float2 ya = bc2(comp(y0, m)), yb = bc2(comp(y1, m));
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            ac[0][k] = fmaf(ya, hv[k], ac[0][k]);
-            ac[1][k] = fmaf(yb, hv[k], ac[1][k]);
+          for (int q = 0; q < 4; ++q) {
+            ac[0][q] = __ffma2_rn(ya, hv[q], ac[0][q]);
+            ac[1][q] = __ffma2_rn(yb, hv[q], ac[1][q]);
           }
         }
       }
@@ -558,15 +585,15 @@ __global__ void __launch_bounds__(kT, 1) bwd_chunk_kernel(BwdArgs a, ChunkWs ws)
       for (int i = 0; i < 2; ++i) {
         const int r = r0 + i;
         const float4 c0 = ld4(&sm.Cb[r * SB + 4 * cq]), c1 = ld4(&sm.Cb[r * SB + 4 * cq + 64]);
-        const float cv8[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-        float s = 0.f;
+        const float2 cv[4] = {lo2(c0), hi2(c0), lo2(c1), hi2(c1)};
+        float2 s2 = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) s = fmaf(cv8[k], ac[i][k], s);
-        s = half_sum(s);
+        for (int q = 0; q < 4; ++q) s2 = __ffma2_rn(cv[q], ac[i][q], s2);
+        const float s = half_sum(s2.x + s2.y);
         const float e = sm.ecs[r];
         if (cq == 0) sm.dcsY[r] = e * s;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) ac[i][k] *= e;
+        for (int q = 0; q < 4; ++q) ac[i][q] = __fmul2_rn(bc2(e), ac[i][q]);
       }
       for (int u = 0; u <= whi; u += 4) {  // WE(r, u) = 0 for u > r
         const float4 w0 = ld4(&sm.Em[r0 * SX + u]), w1 = ld4(&sm.Em[r1 * SX + u]);
@@ -574,12 +601,12 @@ __global__ void __launch_bounds__(kT, 1) bwd_chunk_kernel(BwdArgs a, ChunkWs ws)
         for (int m = 0; m < 4; ++m) {
           const float4 b0 = ld4(&sm.Bb[(u + m) * SB + 4 * cq]);
           const float4 b1 = ld4(&sm.Bb[(u + m) * SB + 4 * cq + 64]);
-          const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-          const float wa = comp(w0, m), wb = comp(w1, m);
+          const float2 bv[4] = {lo2(b0), hi2(b0), lo2(b1), hi2(b1)};
+          const float2 wa = bc2(comp(w0, m)), wb = bc2(comp(w1, m));
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            ac[0][k] = fmaf(wa, bv[k], ac[0][k]);
-            ac[1][k] = fmaf(wb, bv[k], ac[1][k]);
+          for (int q = 0; q < 4; ++q) {
+            ac[0][q] = __ffma2_rn(wa, bv[q], ac[0][q]);
+            ac[1][q] = __ffma2_rn(wb, bv[q], ac[1][q]);
           }
         }
       }
@@ -594,7 +621,7 @@ __global__ void __launch_bounds__(kT, 1) bwd_chunk_kernel(BwdArgs a, ChunkWs ws)
           const int n = 4 * cq + 64 * (k >> 2) + (k & 3), pi = n >> 1;
           float sn, cs_;
           fast_sincos(sm.Vt[r * SX + pi], &sn, &cs_);
-          const float d0 = ac[i][k], d1 = ac[i][k + 1];
+          const float d0 = ac[i][k >> 1].x, d1 = ac[i][k >> 1].y;
           const float v0 = sm.Cb[r * SB + n], v1 = sm.Cb[r * SB + n + 1];
           sm.Gm[r * SX + pi] = ok ? fmaf(d1, v0, -d0 * v1) : 0.f;
           if (ok)
@@ -607,46 +634,49 @@ __global__ void __launch_bounds__(kT, 1) bwd_chunk_kernel(BwdArgs a, ChunkWs ws)
     // -- dBbar = WE^T Cbar + W_end o (X g^T), the carries of row 0 (this
     //    chunk's carry-in token) and into row 63, then the rotation adjoint
     {
-      float bb[2][8];
+      float2 bp[2][4];  // column pairs (n, n + 1) of rows r0, r1
 #pragma unroll
-      for (int k = 0; k < 8; ++k) bb[0][k] = bb[1][k] = 0.f;
+      for (int q = 0; q < 4; ++q) bp[0][q] = bp[1][q] = make_float2(0.f, 0.f);
       for (int p = 0; p < kP; p += 4) {
         const float4 x0 = ld4(&sm.Xs[r0 * SX + p]), x1 = ld4(&sm.Xs[r1 * SX + p]);
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
           const float4 g0 = ld4(&sm.Gs[(p + m) * SB + 4 * cq]);
           const float4 g1 = ld4(&sm.Gs[(p + m) * SB + 4 * cq + 64]);
-          const float gv[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-          const float xa = comp(x0, m), xb = comp(x1, m);
+          const float2 gv[4] = {lo2(g0), hi2(g0), lo2(g1), hi2(g1)};
+          const float2 xa = bc2(comp(x0, m)), xb = bc2(comp(x1, m));
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            bb[0][k] = fmaf(xa, gv[k], bb[0][k]);
-            bb[1][k] = fmaf(xb, gv[k], bb[1][k]);
+          for (int q = 0; q < 4; ++q) {
+            bp[0][q] = __ffma2_rn(xa, gv[q], bp[0][q]);
+            bp[1][q] = __ffma2_rn(xb, gv[q], bp[1][q]);
           }
         }
       }
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
-        const float we = sm.wend[r0 + i];
+        const float2 we = bc2(sm.wend[r0 + i]);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) bb[i][k] *= we;
+        for (int q = 0; q < 4; ++q) bp[i][q] = __fmul2_rn(we, bp[i][q]);
       }
       for (int r = wlo; r < kQ; ++r) {  // WE(r, u) = 0 for r < u
         const float2 w = ld2(&sm.Em[r * SX + r0]);
         const float4 c0 = ld4(&sm.Cb[r * SB + 4 * cq]), c1 = ld4(&sm.Cb[r * SB + 4 * cq + 64]);
-        const float cv8[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+        const float2 cv[4] = {lo2(c0), hi2(c0), lo2(c1), hi2(c1)};
+        const float2 wa = bc2(w.x), wb = bc2(w.y);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          bb[0][k] = fmaf(w.x, cv8[k], bb[0][k]);
-          bb[1][k] = fmaf(w.y, cv8[k], bb[1][k]);
+        for (int q = 0; q < 4; ++q) {
+          bp[0][q] = __ffma2_rn(wa, cv[q], bp[0][q]);
+          bp[1][q] = __ffma2_rn(wb, cv[q], bp[1][q]);
         }
       }
+      float bb[2][8];
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
         const int r = r0 + i;
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const int n = 4 * cq + 64 * (k >> 2) + (k & 3);
+          bb[i][k] = (k & 1) ? bp[i][k >> 1].y : bp[i][k >> 1].x;
           if (r == kQ - 1) bb[i][k] += sm.cdb[nxt][n];
           if (r == 0) sm.cdb[cur][n] = bb[i][k];
         }
@@ -684,16 +714,26 @@ __global__ void __launch_bounds__(kT, 1) bwd_chunk_kernel(BwdArgs a, ChunkWs ws)
           ghp = fmaf(gv, sm.Hp[o], ghp);
           dh[i][j] = eE * gv;
         }
+      float2 dp[2][4];  // rows (nq + 2 ii, nq + 2 ii + 1), column cq + 16 j
+#pragma unroll
+      for (int j = 0; j < 4; ++j) dp[0][j] = dp[1][j] = make_float2(0.f, 0.f);
       for (int r = 1; r < kQ; ++r) {
-        const float e = sm.ecs[r];
+        const float2 e = bc2(sm.ecs[r]);
         const float4 cv = ld4(&sm.Cb[r * SB + nq]);
-        const float cw[4] = {e * cv.x, e * cv.y, e * cv.z, e * cv.w};
+        const float2 cw0 = __fmul2_rn(e, lo2(cv)), cw1 = __fmul2_rn(e, hi2(cv));
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          const float y = sm.Ys[r * SX + cq + 16 * j];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) dh[i][j] = fmaf(cw[i], y, dh[i][j]);
+          const float2 y = bc2(sm.Ys[r * SX + cq + 16 * j]);
+          dp[0][j] = __ffma2_rn(cw0, y, dp[0][j]);
+          dp[1][j] = __ffma2_rn(cw1, y, dp[1][j]);
         }
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        dh[0][j] += dp[0][j].x;
+        dh[1][j] += dp[0][j].y;
+        dh[2][j] += dp[1][j].x;
+        dh[3][j] += dp[1][j].y;
       }
       block_sum(ghp, sm.red, &sm.misc[0]);  // ends with a barrier: g is free
     }

@@ -117,6 +117,36 @@ __device__ __forceinline__ void ldn(const __nv_bfloat16* p, bool vec, float* out
     for (int k = 0; k < n; ++k) out[k] = __bfloat162float(p[k]);
   }
 }
+// 16 bytes from global to shared memory without a register round trip; the
+// destination is zero-filled when !full (nothing is read then)
+__device__ __forceinline__ void cp16(float* smem_dst, const void* gmem_src, bool full) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(
+                   (uint32_t)__cvta_generic_to_shared(smem_dst)),
+               "l"(gmem_src), "r"(full ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// 8 elements held as raw 16-byte vectors (one for bf16, two for fp32) to fp32
+__device__ __forceinline__ void unpack8(const uint4* v, float* out, const __nv_bfloat16*) {
+  const uint32_t w[4] = {v[0].x, v[0].y, v[0].z, v[0].w};
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[q]));
+    out[2 * q] = f.x;
+    out[2 * q + 1] = f.y;
+  }
+}
+__device__ __forceinline__ void unpack8(const uint4* v, float* out, const float*) {
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    out[4 * k] = __uint_as_float(v[k].x);
+    out[4 * k + 1] = __uint_as_float(v[k].y);
+    out[4 * k + 2] = __uint_as_float(v[k].z);
+    out[4 * k + 3] = __uint_as_float(v[k].w);
+  }
+}
 template <int n>
 __device__ __forceinline__ void stn(float* dst, const float* v) {
 #pragma unroll
@@ -237,6 +267,138 @@ __global__ void __launch_bounds__(kT, 1) bwd_chunk_kernel(BwdArgs a, ChunkWs ws)
     }
   };
 
+  // ---- the same inputs in two steps when every pointer allows 16-byte loads:
+  // fetch() issues the loads into registers a phase ahead, commit() converts
+  // and stores them (the chunk-start state and angle too, for the reverse pass)
+  constexpr int kXV = (int)sizeof(T) / 2;  // 16-byte vectors in 8 elements
+  // fp32 inputs need no conversion: the reverse pass copies them asynchronously
+  constexpr bool kRaw = sizeof(T) == 4;
+  struct Fetch {
+    uint4 x[kXV], y[kXV], bq[2 * kXV], cq[2 * kXV];
+    float4 th[2];
+    float sc[3], ph;
+  };
+  auto fetch = [&](int c, bool bwd, Fetch& f) {
+    const int64_t t0 = (int64_t)c * QT - 1;
+    const int r = tid >> 3, sg = tid & 7;
+    const int64_t t = t0 + r;
+    const bool in = t >= 0 && t < L, own = r > 0 && t < L;
+    const int64_t th = (b * L + (in ? t : 0)) * H + h, tg = (b * L + (in ? t : 0)) * G + g;
+    const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
+    const float4 zf = make_float4(0.f, 0.f, 0.f, 0.f);
+    const uint4* xs = reinterpret_cast<const uint4*>(X + th * kP + 8 * sg);
+    const uint4* bs = reinterpret_cast<const uint4*>(Bg + tg * kN + 16 * sg);
+    if (!(kRaw && bwd)) {
+#pragma unroll
+      for (int k = 0; k < kXV; ++k) f.x[k] = in ? xs[k] : z4;
+#pragma unroll
+      for (int k = 0; k < 2 * kXV; ++k) f.bq[k] = in ? bs[k] : z4;
+    }
+    if (!bwd) {
+      const float4* ts = reinterpret_cast<const float4*>(a.theta + th * kNH + 8 * sg);
+      f.th[0] = (own && a.theta) ? ts[0] : zf;
+      f.th[1] = (own && a.theta) ? ts[1] : zf;
+    }
+    if (bwd) {
+      if (!kRaw) {
+        const uint4* ys = reinterpret_cast<const uint4*>(dY + th * kP + 8 * sg);
+        const uint4* cs_ = reinterpret_cast<const uint4*>(Cg + tg * kN + 16 * sg);
+#pragma unroll
+        for (int k = 0; k < kXV; ++k) f.y[k] = own ? ys[k] : z4;
+#pragma unroll
+        for (int k = 0; k < 2 * kXV; ++k) f.cq[k] = own ? cs_[k] : z4;
+      }
+      f.ph = tid < kNH ? ph_ws[(int64_t)c * kNH + tid] : 0.f;
+    }
+    f.sc[0] = f.sc[1] = f.sc[2] = 0.f;
+    if (tid < kQ && tid > 0 && t0 + tid < L) {
+      const int64_t ts2 = (b * L + t0 + tid) * H + h;
+      f.sc[0] = a.logdecay[ts2];
+      f.sc[1] = a.gamma[ts2];
+      f.sc[2] = a.beta ? a.beta[ts2] : 0.f;
+    }
+  };
+  auto commit = [&](int c, bool bwd, const Fetch& f) {
+    const int64_t t0 = (int64_t)c * QT - 1;
+    const int r = tid >> 3, sg = tid & 7;
+    float xv[8], bv[16];
+    const bool carry = t0 + r == -1;  // the cache's carry-in token (fp32)
+    if (!(kRaw && bwd) || carry) {
+      unpack8(f.x, xv, X);
+      unpack8(f.bq, bv, Bg);
+      unpack8(f.bq + kXV, bv + 8, Bg);
+      if (carry) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) xv[k] = a.xprev0 ? a.xprev0[bh * kP + 8 * sg + k] : 0.f;
+#pragma unroll
+        for (int k = 0; k < 16; ++k)
+          bv[k] = a.bprev0 ? a.bprev0[(b * G + g) * kN + 16 * sg + k] : 0.f;
+      }
+      stn<8>(&sm.Xs[r * SX + 8 * sg], xv);
+      stn<16>(&sm.Bb[r * SB + 16 * sg], bv);
+    }
+    if (!bwd) {
+      *reinterpret_cast<float4*>(&sm.Vt[r * SX + 8 * sg]) = f.th[0];
+      *reinterpret_cast<float4*>(&sm.Vt[r * SX + 8 * sg + 4]) = f.th[1];
+    } else {
+      if (!kRaw) {
+        float yv[8], cv[16];
+        unpack8(f.y, yv, dY);
+        unpack8(f.cq, cv, Cg);
+        unpack8(f.cq + kXV, cv + 8, Cg);
+        stn<8>(&sm.Ys[r * SX + 8 * sg], yv);
+        stn<16>(&sm.Cb[r * SB + 16 * sg], cv);
+      }
+      if (tid < kNH) sm.phi0[tid] = f.ph;
+    }
+    if (tid < kQ) {
+      sm.cs[tid] = f.sc[0];  // the raw logdecay until chunk_scalars
+      sm.ga[tid] = f.sc[1];
+      sm.be[tid] = f.sc[2];
+    }
+  };
+
+  // the reverse pass's theta rows and chunk-start state (16-byte asynchronous
+  // copies into tiles that are free from the dh_prev phase on)
+  auto async_copy = [&](int c) {
+    const int64_t t0 = (int64_t)c * QT - 1;
+    const float* hw = hs_ws + (int64_t)c * kN * kP;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int e = tid + kT * k, p = e >> 5, n4 = 4 * (e & 31);
+      cp16(&sm.Hp[p * SB + n4], hw + p * kN + n4, true);
+    }
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int e = tid + kT * k, r = e >> 4, i4 = 4 * (e & 15);
+      const int64_t t = t0 + r;
+      const bool ok = a.theta && r > 0 && t < L;
+      const float* src = ok ? a.theta + ((b * L + t) * H + h) * kNH + i4 : hw;
+      cp16(&sm.Vt[r * SX + i4], src, ok);
+    }
+    if (kRaw) {
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {  // X, dY: 64 rows of 16 vectors
+        const int e = tid + kT * k, r = e >> 4, p4 = 4 * (e & 15);
+        const int64_t t = t0 + r;
+        const bool in = t >= 0 && t < L, own = r > 0 && t < L;
+        const int64_t th = ((b * L + (in ? t : 0)) * H + h) * kP + p4;
+        cp16(&sm.Xs[r * SX + p4], X + th, in);
+        cp16(&sm.Ys[r * SX + p4], dY + th, own);
+      }
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {  // B, C: 64 rows of 32 vectors
+        const int e = tid + kT * k, r = e >> 5, n4 = 4 * (e & 31);
+        const int64_t t = t0 + r;
+        const bool in = t >= 0 && t < L, own = r > 0 && t < L;
+        const int64_t tg = ((b * L + (in ? t : 0)) * G + g) * kN + n4;
+        cp16(&sm.Bb[r * SB + n4], Bg + tg, in);
+        cp16(&sm.Cb[r * SB + n4], Cg + tg, own);
+      }
+    }
+    cp_commit();
+  };
+
   // ---- chunk scalars: cs (inclusive sums of logdecay), alpha, exp(cs), cv, W_end
   auto chunk_scalars = [&]() {
     if (warp == 0) {
@@ -320,6 +482,8 @@ __global__ void __launch_bounds__(kT, 1) bwd_chunk_kernel(BwdArgs a, ChunkWs ws)
       for (int j = 0; j < 4; ++j)
         hreg[i][j] = a.h0 ? a.h0[(bh * kN + nq + i) * kP + cq + 16 * j] : 0.f;
     if (tid < kNH) sm.phi0[tid] = wrap_angle(a.angle0 ? a.angle0[bh * kNH + tid] : 0.f);
+    Fetch f;
+    if (vec && nC > 0) fetch(0, false, f);
     __syncthreads();
     for (int c = 0; c < nC; ++c) {
       float* hw = hs_ws + (int64_t)c * kN * kP;  // (p, n)
@@ -328,10 +492,15 @@ __global__ void __launch_bounds__(kT, 1) bwd_chunk_kernel(BwdArgs a, ChunkWs ws)
         *reinterpret_cast<float4*>(&hw[(cq + 16 * j) * kN + nq]) =
             make_float4(hreg[0][j], hreg[1][j], hreg[2][j], hreg[3][j]);
       if (tid < kNH) ph_ws[(int64_t)c * kNH + tid] = sm.phi0[tid];
-      load_chunk(c, false);
+      if (vec)
+        commit(c, false, f);
+      else
+        load_chunk(c, false);
+      f = Fetch{};  // consumed: nothing stays live across the chunk's compute
       __syncthreads();
       chunk_scalars();
       angles_rotate(false);
+      if (vec && c + 1 < nC) fetch(c + 1, false, f);
       const float eE = sm.ecs[kQ - 1];
       float2 acc[2][4];  // rows (nq + 2 ii, nq + 2 ii + 1), column cq + 16 j
 #pragma unroll
@@ -379,14 +548,23 @@ __global__ void __launch_bounds__(kT, 1) bwd_chunk_kernel(BwdArgs a, ChunkWs ws)
     sm.Gs[p * SB + n] = a.dhT ? a.dhT[(bh * kN + n) * kP + p] : 0.f;
   }
   float dDacc = 0.f;
+  Fetch f;
+  if (vec && nC > 0) {
+    fetch(nC - 1, true, f);
+    async_copy(nC - 1);
+  }
   __syncthreads();
 
   for (int c = nC - 1; c >= 0; --c) {
     const int cur = c & 1, nxt = cur ^ 1;
     const int64_t t0 = (int64_t)c * QT - 1;  // token of row 0
     auto own = [&](int r) { return r > 0 && t0 + r < L; };
-    float4 hpv[4];  // the chunk-start state, (p, n) float4s
-    {
+    if (vec) {
+      cp_wait_all();  // before commit: the carry-in row overwrites a zero-filled copy
+      commit(c, true, f);
+      f = Fetch{};  // consumed: nothing stays live across the chunk's compute
+    } else {
+      float4 hpv[4];  // the chunk-start state, (p, n) float4s
       const float* hw = hs_ws + (int64_t)c * kN * kP;
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
@@ -394,12 +572,12 @@ __global__ void __launch_bounds__(kT, 1) bwd_chunk_kernel(BwdArgs a, ChunkWs ws)
         hpv[k] = *reinterpret_cast<const float4*>(&hw[(idx >> 5) * kN + 4 * (idx & 31)]);
       }
       if (tid < kNH) sm.phi0[tid] = ph_ws[(int64_t)c * kNH + tid];
-    }
-    load_chunk(c, true);
+      load_chunk(c, true);
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int idx = tid + kT * k;
-      *reinterpret_cast<float4*>(&sm.Hp[(idx >> 5) * SB + 4 * (idx & 31)]) = hpv[k];
+      for (int k = 0; k < 4; ++k) {
+        const int idx = tid + kT * k;
+        *reinterpret_cast<float4*>(&sm.Hp[(idx >> 5) * SB + 4 * (idx & 31)]) = hpv[k];
+      }
     }
     __syncthreads();
     chunk_scalars();
@@ -741,6 +919,11 @@ __global__ void __launch_bounds__(kT, 1) bwd_chunk_kernel(BwdArgs a, ChunkWs ws)
     for (int i = 0; i < 4; ++i)
 #pragma unroll
       for (int j = 0; j < 4; ++j) sm.Gs[(cq + 16 * j) * SB + nq + i] = dh[i][j];
+
+    if (vec && c > 0) {  // the inputs of chunk c - 1
+      fetch(c - 1, true, f);
+      async_copy(c - 1);
+    }
 
     // -- the scalar chain: decay sums -> cv -> gamma, beta, logdecay
     if (warp == 0) {

@@ -210,10 +210,12 @@ typedef struct {
 } m3ssd_bwd_grads;
 
 /* Bytes of device workspace m3ssd_bwd needs for these dims (0 for invalid
- * dims).  It holds a state checkpoint every 64 tokens of every sequence, the
- * states of one 64-token block per sequence, and per-head shares of the
- * group-summed gradients: about 4 (b H ceil(L/64) (N P + N/2) + b H 65 N P +
- * 2 b L H N) bytes. */
+ * dims); the size depends on the path.  At N = 128, P = 64 it holds every
+ * chunk-start state and angle (chunks of 63 tokens) and per-head shares of
+ * the group-summed gradients: about 4 (b H ceil(L/63) (N P + N/2) +
+ * 2 b L H N) bytes.  Other shapes keep a state checkpoint every 16 or 64
+ * tokens, the states of one block per sequence and the same per-head (or
+ * per-slice) shares. */
 size_t m3ssd_bwd_workspace_size(const m3ssd_dims* dims);
 
 /*
@@ -228,12 +230,15 @@ size_t m3ssd_bwd_workspace_size(const m3ssd_dims* dims);
  * fp32, NULL = 0), and writes the fp32 gradients in *grads.  The cache outputs
  * angleT, xprevT and bprevT take no upstream gradient.
  *
- * The backward recomputes the forward in fp32 from state checkpoints.  At
- * N = 128 with P a multiple of 16 it splits each sequence over P/16 CTAs of
- * 16 state columns and sums the per-slice partials of the column-mixing
- * gradients afterwards; other shapes run one CTA per sequence.  Either way
- * every sum (over slices, the heads of a group, the batch) runs in a fixed
- * order, so results are deterministic.  Limits as the sequential forward:
+ * The backward recomputes the forward in fp32.  At N = 128, P = 64 it works
+ * chunk by chunk (one CTA per sequence: a forward pass stores the state and
+ * angle at every chunk start, then each chunk's adjoint is a set of fp32
+ * products in shared memory, walking the chunks in reverse).  At N = 128 with
+ * another P a multiple of 16 it splits each sequence over P/16 CTAs of 16
+ * state columns and sums the per-slice partials of the column-mixing
+ * gradients afterwards; other shapes run one CTA per sequence token by
+ * token.  Every sum (over slices, the heads of a group, the batch) runs in a
+ * fixed order, so results are deterministic.  Limits as the sequential forward:
  * N <= 256, P <= 256, N*P <= 16384 (else M3SSD_ERR_UNSUPPORTED).  workspace
  * must hold m3ssd_bwd_workspace_size(dims) bytes, 256-byte aligned (else
  * M3SSD_ERR_WORKSPACE); the size depends on the path.  No allocation, no

@@ -340,34 +340,86 @@ __global__ void __launch_bounds__(kMThreads) mimo_step_n128p64(StepArgs a) {
   const float ga = a.gamma_t[bh];
   __syncthreads();
 
-  float xr[4][R], xpr[4][R], acc[4][R];
+  float acc[4][R];
+  if constexpr (R % 2 == 0) {
+    // packed fp32 pairs over the rank index r (two FMAs an instruction)
+    constexpr int R2 = R / 2;
+    float2 xr[4][R2], xpr[4][R2], ac2[4][R2];
 #pragma unroll
-  for (int c = 0; c < 4; ++c)
+    for (int c = 0; c < 4; ++c)
 #pragma unroll
-    for (int r = 0; r < R; ++r) {
-      xr[c][r] = ga * xs[(4 * q + c) * R + r];
-      xpr[c][r] = be * xps[(4 * q + c) * R + r];
-      acc[c][r] = 0.f;
-    }
-  asm volatile("cp.async.wait_all;" ::: "memory");
+      for (int j = 0; j < R2; ++j) {
+        const int e = (4 * q + c) * R + 2 * j;
+        xr[c][j] = make_float2(ga * xs[e], ga * xs[e + 1]);
+        xpr[c][j] = make_float2(be * xps[e], be * xps[e + 1]);
+        ac2[c][j] = make_float2(0.f, 0.f);
+      }
+    asm volatile("cp.async.wait_all;" ::: "memory");
 #pragma unroll 4
-  for (int k = 0; k < kMRows; ++k) {
-    const int n = r0 + 8 * k;
-    float4 v = Sv[n * (kMP / 4) + q];
-    float* vv = reinterpret_cast<float*>(&v);
+    for (int k = 0; k < kMRows; ++k) {
+      const int n = r0 + 8 * k;
+      float4 v = Sv[n * (kMP / 4) + q];
+      float* vv = reinterpret_cast<float*>(&v);
+      float2 bpv[R2], bv[R2], cv[R2];
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      float u = alpha * vv[c];
+      for (int j = 0; j < R2; ++j) {
+        bpv[j] = *reinterpret_cast<const float2*>(&Bpb[n * R + 2 * j]);
+        bv[j] = *reinterpret_cast<const float2*>(&Bb[n * R + 2 * j]);
+        cv[j] = *reinterpret_cast<const float2*>(&Cb[n * R + 2 * j]);
+      }
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float2 s2 = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int j = 0; j < R2; ++j) {
+          s2 = __ffma2_rn(bpv[j], xpr[c][j], s2);
+          s2 = __ffma2_rn(bv[j], xr[c][j], s2);
+        }
+        const float u = fmaf(alpha, vv[c], s2.x + s2.y);
+        vv[c] = u;
+        const float2 u2 = make_float2(u, u);
+#pragma unroll
+        for (int j = 0; j < R2; ++j) ac2[c][j] = __ffma2_rn(cv[j], u2, ac2[c][j]);
+      }
+      S[n * (kMP / 4) + q] = v;
+    }
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+#pragma unroll
+      for (int j = 0; j < R2; ++j) {
+        acc[c][2 * j] = ac2[c][j].x;
+        acc[c][2 * j + 1] = ac2[c][j].y;
+      }
+  } else {
+    float xr[4][R], xpr[4][R];
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
 #pragma unroll
       for (int r = 0; r < R; ++r) {
-        u = fmaf(Bpb[n * R + r], xpr[c][r], u);
-        u = fmaf(Bb[n * R + r], xr[c][r], u);
+        xr[c][r] = ga * xs[(4 * q + c) * R + r];
+        xpr[c][r] = be * xps[(4 * q + c) * R + r];
+        acc[c][r] = 0.f;
       }
-      vv[c] = u;
+    asm volatile("cp.async.wait_all;" ::: "memory");
+#pragma unroll 4
+    for (int k = 0; k < kMRows; ++k) {
+      const int n = r0 + 8 * k;
+      float4 v = Sv[n * (kMP / 4) + q];
+      float* vv = reinterpret_cast<float*>(&v);
 #pragma unroll
-      for (int r = 0; r < R; ++r) acc[c][r] = fmaf(Cb[n * R + r], u, acc[c][r]);
+      for (int c = 0; c < 4; ++c) {
+        float u = alpha * vv[c];
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          u = fmaf(Bpb[n * R + r], xpr[c][r], u);
+          u = fmaf(Bb[n * R + r], xr[c][r], u);
+        }
+        vv[c] = u;
+#pragma unroll
+        for (int r = 0; r < R; ++r) acc[c][r] = fmaf(Cb[n * R + r], u, acc[c][r]);
+      }
+      S[n * (kMP / 4) + q] = v;
     }
-    S[n * (kMP / 4) + q] = v;
   }
   // lanes l and l + 16 hold the same column slice
 #pragma unroll

@@ -284,7 +284,7 @@ m3ssd_status m3ssd_bwd_noalloc(const m3ssd_dims* dims, const void* X, const floa
  *   out = (y * SiLU(z)) W_out^T          out_proj, no bias
  *
  * The projections are plain GEMMs run by cuBLASLt (bf16 operands, fp32
- * accumulation; in_proj writes fp32, out_proj bf16); the rest runs in this
+ * accumulation, bf16 outputs); the rest runs in this
  * library's kernels, the head biases inside the scan (added in fp32 before the
  * rotation).  u and out are bf16.  The block cache is an m3ssd_cache with
  * b_prev (b, G, N) holding the QK-normed group vector B_{t-1} (times its norm

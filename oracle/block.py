@@ -33,11 +33,12 @@ Readings where the pages are silent (each is listed in the design notes):
 Storage precision: the pages' numerics policy ("TorchMamba" README,
 "Behavioral notes": bf16 computes in fp32 and each output is downcast to the
 input dtype) makes the tensors a bf16 block hands from one step to the next
-bf16.  ``store`` (default: none) is applied to exactly those hand-offs -- x,
-the QK-normed group vectors of B and C (the scan's bf16 inputs; the head bias
-is added after them), the scan output y and the gated product (out_proj's
-input) -- so that a test can compare against a device path that stores them
-in bf16; everything else stays fp64.
+bf16.  ``store`` (default: none) is applied to exactly those hand-offs -- the
+in_proj output (z, x, B, C, dt, lam, theta), the QK-normed group vectors of B
+and C (the scan's bf16 inputs; the head bias is added after them), the scan
+output y and the gated product (out_proj's input) -- so that a test can
+compare against a device path that stores them in bf16; everything else stays
+fp64.
 
 Numerical pins: ``tests/test_oracle_block.py`` (closed forms for one and two
 tokens, the scale invariance of the norm, forward == prefill + steps, and
@@ -91,7 +92,7 @@ def _keep(v):
 def scan_inputs(u, wts, H, P, N, G, store=_keep):
     """Steps 1-2 of the block: the scan's inputs from the block input u (..., d_model)."""
     f = lambda k: np.asarray(wts[k], dtype=np.float64)
-    zx = np.asarray(u, dtype=np.float64) @ f("W_in").T
+    zx = store(np.asarray(u, dtype=np.float64) @ f("W_in").T)
     s = _split(zx, H, P, N, G)
     delta = softplus(s["dt"] + f("dt_bias"))
     A = -np.exp(f("A_log"))

@@ -7,8 +7,8 @@
 // Mamba3SisoCache).  The two projections are plain GEMMs and run in cuBLASLt
 // (bf16 operands, fp32 accumulation); everything between them runs here:
 //
-//   block_prep_kernel   one CTA per token: splits the fp32 in_proj row, writes x
-//                       (bf16), the QK-normed B and C of each group times the
+//   block_prep_kernel   one CTA per token: splits the bf16 in_proj row, copies x
+//                       (bf16), writes the QK-normed B and C of each group times the
 //                       norm weight (bf16), logdecay, beta, gamma (fp32) and
 //                       theta_dt (fp32);
 //   the scan's forward / step kernels on those tensors, which add the head's
@@ -51,7 +51,7 @@ BlockWs block_ws(const m3ssd_block_dims* d, int64_t M) {
     o += al256(bytes);
     return r;
   };
-  w.zx = take(m * (size_t)in_proj_width(d) * 4);
+  w.zx = take(m * (size_t)in_proj_width(d) * 2);  // bf16 in_proj output
   w.x = take(m * H * P * 2);   // x, then y * SiLU(z)
   const size_t G = (size_t)d->ngroups;
   w.B = take(m * G * N * 2);
@@ -69,7 +69,7 @@ BlockWs block_ws(const m3ssd_block_dims* d, int64_t M) {
 
 struct PrepArgs {
   int64_t M, H, P, N, G, width;
-  const float* zx;
+  const __nv_bfloat16* zx;
   const float* dt_bias;
   const float* A_log;
   const float* Bw;
@@ -94,8 +94,16 @@ __device__ __forceinline__ uint32_t pack2_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-bool vec_shape(int64_t H, int64_t P, int64_t N, int64_t G) {
-  return (H * P) % 8 == 0 && (G * N) % 4 == 0 && H % 4 == 0 && N % 8 == 0;
+bool vec_shape(int64_t H, int64_t P, int64_t N, int64_t G, int64_t width) {
+  return (H * P) % 8 == 0 && (G * N) % 4 == 0 && H % 4 == 0 && N % 8 == 0 && width % 8 == 0;
+}
+
+__device__ __forceinline__ float bf(const __nv_bfloat16 v) { return __bfloat162float(v); }
+// four bf16 (8 bytes) to fp32
+__device__ __forceinline__ float4 ld4_bf16(const __nv_bfloat16* p) {
+  const uint2 w = *reinterpret_cast<const uint2*>(p);
+  return make_float4(__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xffff0000u),
+                     __uint_as_float(w.y << 16), __uint_as_float(w.y & 0xffff0000u));
 }
 
 // One CTA per token.  Shared memory: 2G inverse RMS values (B groups, then C
@@ -107,35 +115,36 @@ __global__ void __launch_bounds__(kPrepThreads) block_prep_kernel(PrepArgs a) {
   const int H = (int)a.H, P = (int)a.P, N = (int)a.N, G = (int)a.G, NH = N / 2;
   const int HP = H * P, GN = G * N;
   const int oB = 2 * HP, oC = oB + GN, odt = oC + GN, olam = odt + H, oth = olam + H;
-  const float* row = a.zx + tok * a.width;
+  const __nv_bfloat16* row = a.zx + tok * a.width;
   float* inv = sh;
   float* delta = sh + 2 * G;
 
   for (int j = warp; j < 2 * G; j += kPrepThreads / 32) {
-    const float* v = row + (j < G ? oB + j * N : oC + (j - G) * N);
+    const __nv_bfloat16* v = row + (j < G ? oB + j * N : oC + (j - G) * N);
     float ss = 0.f;
-    for (int n = lane; n < N; n += 32) ss = fmaf(v[n], v[n], ss);
+    for (int n = lane; n < N; n += 32) ss = fmaf(bf(v[n]), bf(v[n]), ss);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
     if (lane == 0) inv[j] = 1.f / sqrtf(ss / (float)N + a.eps);
   }
   for (int h = tid; h < H; h += kPrepThreads) {
-    const float dl = softplus_f(row[odt + h] + a.dt_bias[h]);
+    const float dl = softplus_f(bf(row[odt + h]) + a.dt_bias[h]);
     const float lg = -expf(a.A_log[h]) * dl;
-    const float lam = 1.f / (1.f + expf(-row[olam + h]));
+    const float lam = 1.f / (1.f + expf(-bf(row[olam + h])));
     a.ld[tok * H + h] = lg;
     a.ga[tok * H + h] = lam * dl;
     a.be[tok * H + h] = (1.f - lam) * dl * expf(lg);
     delta[h] = dl;
   }
-  for (int k = tid; k < HP; k += kPrepThreads) a.X[tok * HP + k] = __float2bfloat16_rn(row[HP + k]);
+  for (int k = tid; k < HP; k += kPrepThreads) a.X[tok * HP + k] = row[HP + k];
   __syncthreads();
   for (int k = tid; k < G * N; k += kPrepThreads) {
     const int g = k / N, n = k - g * N;
-    a.B[tok * G * N + k] = __float2bfloat16_rn(row[oB + k] * inv[g] * a.Bw[n]);
-    a.C[tok * G * N + k] = __float2bfloat16_rn(row[oC + k] * inv[G + g] * a.Cw[n]);
+    a.B[tok * G * N + k] = __float2bfloat16_rn(bf(row[oB + k]) * inv[g] * a.Bw[n]);
+    a.C[tok * G * N + k] = __float2bfloat16_rn(bf(row[oC + k]) * inv[G + g] * a.Cw[n]);
   }
-  for (int k = tid; k < H * NH; k += kPrepThreads) a.th[tok * H * NH + k] = delta[k / NH] * row[oth + k];
+  for (int k = tid; k < H * NH; k += kPrepThreads)
+    a.th[tok * H * NH + k] = delta[k / NH] * bf(row[oth + k]);
 }
 
 // The same with 16-byte accesses, for shapes whose row parts are multiples of
@@ -147,15 +156,15 @@ __global__ void __launch_bounds__(kPrepThreads) block_prep_vec_kernel(PrepArgs a
   const int H = (int)a.H, P = (int)a.P, N = (int)a.N, G = (int)a.G, NH = N / 2;
   const int HP = H * P, GN = G * N;
   const int oB = 2 * HP, oC = oB + GN, odt = oC + GN, olam = odt + H, oth = olam + H;
-  const float* row = a.zx + tok * a.width;
+  const __nv_bfloat16* row = a.zx + tok * a.width;
   float* inv = sh;
   float* delta = sh + 2 * G;
 
   for (int j = warp; j < 2 * G; j += kPrepThreads / 32) {
-    const float* v = row + (j < G ? oB + j * N : oC + (j - G) * N);
+    const __nv_bfloat16* v = row + (j < G ? oB + j * N : oC + (j - G) * N);
     float ss = 0.f;
     for (int n = 4 * lane; n < N; n += 128) {
-      const float4 q = *reinterpret_cast<const float4*>(v + n);
+      const float4 q = ld4_bf16(v + n);
       ss = fmaf(q.x, q.x, fmaf(q.y, q.y, fmaf(q.z, q.z, fmaf(q.w, q.w, ss))));
     }
 #pragma unroll
@@ -163,28 +172,23 @@ __global__ void __launch_bounds__(kPrepThreads) block_prep_vec_kernel(PrepArgs a
     if (lane == 0) inv[j] = 1.f / sqrtf(ss / (float)N + a.eps);
   }
   for (int h = tid; h < H; h += kPrepThreads) {
-    const float dl = softplus_f(row[odt + h] + a.dt_bias[h]);
+    const float dl = softplus_f(bf(row[odt + h]) + a.dt_bias[h]);
     const float lg = -expf(a.A_log[h]) * dl;
-    const float lam = 1.f / (1.f + expf(-row[olam + h]));
+    const float lam = 1.f / (1.f + expf(-bf(row[olam + h])));
     a.ld[tok * H + h] = lg;
     a.ga[tok * H + h] = lam * dl;
     a.be[tok * H + h] = (1.f - lam) * dl * expf(lg);
     delta[h] = dl;
   }
-  for (int k = tid; k < HP / 8; k += kPrepThreads) {
-    const float4 u = *reinterpret_cast<const float4*>(row + HP + 8 * k);
-    const float4 v = *reinterpret_cast<const float4*>(row + HP + 8 * k + 4);
-    uint4 o;
-    o.x = pack2_bf16(u.x, u.y); o.y = pack2_bf16(u.z, u.w);
-    o.z = pack2_bf16(v.x, v.y); o.w = pack2_bf16(v.z, v.w);
-    *reinterpret_cast<uint4*>(a.X + tok * HP + 8 * k) = o;
-  }
+  for (int k = tid; k < HP / 8; k += kPrepThreads)
+    *reinterpret_cast<uint4*>(a.X + tok * HP + 8 * k) =
+        *reinterpret_cast<const uint4*>(row + HP + 8 * k);
   __syncthreads();
   const int NQ = N / 4;
   for (int k = tid; k < G * NQ; k += kPrepThreads) {
     const int g = k / NQ, n = 4 * (k - g * NQ);
-    const float4 bv = *reinterpret_cast<const float4*>(row + oB + g * N + n);
-    const float4 cv = *reinterpret_cast<const float4*>(row + oC + g * N + n);
+    const float4 bv = ld4_bf16(row + oB + g * N + n);
+    const float4 cv = ld4_bf16(row + oC + g * N + n);
     const float4 bw = *reinterpret_cast<const float4*>(a.Bw + n);
     const float4 cw = *reinterpret_cast<const float4*>(a.Cw + n);
     const float ib = inv[g], ic = inv[G + g];
@@ -198,23 +202,24 @@ __global__ void __launch_bounds__(kPrepThreads) block_prep_vec_kernel(PrepArgs a
   }
   for (int k = tid; k < H * NH / 4; k += kPrepThreads) {
     const float d = delta[(4 * k) / NH];
-    const float4 v = *reinterpret_cast<const float4*>(row + oth + 4 * k);
+    const float4 v = ld4_bf16(row + oth + 4 * k);
     *reinterpret_cast<float4*>(a.th + tok * H * NH + 4 * k) =
         make_float4(d * v.x, d * v.y, d * v.z, d * v.w);
   }
 }
 
-// y * SiLU(z), z read from the fp32 in_proj rows, eight elements a thread
-// (H P % 8 == 0, in_proj width % 4 == 0).
+// y * SiLU(z), z read from the bf16 in_proj rows, eight elements a thread
+// (H P % 8 == 0, in_proj width % 8 == 0).
 __global__ void block_gate_vec_kernel(const __nv_bfloat16* __restrict__ y,
-                                      const float* __restrict__ zx, int64_t width, int64_t HP,
+                                      const __nv_bfloat16* __restrict__ zx, int64_t width,
+                                      int64_t HP,
                                       int64_t M, __nv_bfloat16* __restrict__ out) {
   const int64_t n8 = M * HP / 8, stride = (int64_t)gridDim.x * blockDim.x, hp8 = HP / 8;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8; i += stride) {
     const int64_t tok = i / hp8, k = 8 * (i - tok * hp8);
     const uint4 yv = *reinterpret_cast<const uint4*>(y + 8 * i);
-    const float4 z0 = *reinterpret_cast<const float4*>(zx + tok * width + k);
-    const float4 z1 = *reinterpret_cast<const float4*>(zx + tok * width + k + 4);
+    const float4 z0 = ld4_bf16(zx + tok * width + k);
+    const float4 z1 = ld4_bf16(zx + tok * width + k + 4);
     const uint32_t yw[4] = {yv.x, yv.y, yv.z, yv.w};
     const float z[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
     uint32_t o[4];
@@ -228,14 +233,14 @@ __global__ void block_gate_vec_kernel(const __nv_bfloat16* __restrict__ y,
   }
 }
 
-// y * SiLU(z), z read from the fp32 in_proj rows.
-__global__ void block_gate_kernel(const __nv_bfloat16* __restrict__ y, const float* __restrict__ zx,
-                                  int64_t width, int64_t HP, int64_t M,
-                                  __nv_bfloat16* __restrict__ out) {
+// y * SiLU(z), z read from the bf16 in_proj rows.
+__global__ void block_gate_kernel(const __nv_bfloat16* __restrict__ y,
+                                  const __nv_bfloat16* __restrict__ zx, int64_t width, int64_t HP,
+                                  int64_t M, __nv_bfloat16* __restrict__ out) {
   const int64_t n = M * HP, stride = (int64_t)gridDim.x * blockDim.x;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) {
     const int64_t tok = i / HP, k = i - tok * HP;
-    const float z = zx[tok * width + k];
+    const float z = __bfloat162float(zx[tok * width + k]);
     out[i] = __float2bfloat16_rn(__bfloat162float(y[i]) * z / (1.f + expf(-z)));
   }
 }
@@ -330,12 +335,12 @@ bool scan_shape_ok(const m3ssd_block_dims* d) {
 m3ssd_status front(const m3ssd_block_dims* d, const m3ssd_block_weights* w, const void* u,
                    int64_t M, char* base, const BlockWs& ws, cudaStream_t s) {
   const int64_t width = in_proj_width(d);
-  if (!gemm_bf16(M, width, d->d_model, u, w->W_in, base + ws.zx, CUDA_R_32F, base + ws.lt,
+  if (!gemm_bf16(M, width, d->d_model, u, w->W_in, base + ws.zx, CUDA_R_16BF, base + ws.lt,
                  kLtWorkspace, s))
     return M3SSD_ERR_CUDA;
   PrepArgs a{};
   a.M = M; a.H = d->nheads; a.P = d->headdim; a.N = d->dstate; a.G = d->ngroups; a.width = width;
-  a.zx = reinterpret_cast<const float*>(base + ws.zx);
+  a.zx = reinterpret_cast<const __nv_bfloat16*>(base + ws.zx);
   a.dt_bias = w->dt_bias; a.A_log = w->A_log; a.Bw = w->B_norm_w; a.Cw = w->C_norm_w;
   a.Bbias = w->B_bias; a.Cbias = w->C_bias; a.eps = w->eps;
   a.X = reinterpret_cast<__nv_bfloat16*>(base + ws.x);
@@ -348,7 +353,7 @@ m3ssd_status front(const m3ssd_block_dims* d, const m3ssd_block_weights* w, cons
   const size_t smem = sizeof(float) * (size_t)(2 * d->ngroups + d->nheads);
   if (smem > 48 * 1024) return M3SSD_ERR_UNSUPPORTED;
   const bool w16 = aligned(a.Bw, 16) && aligned(a.Cw, 16);
-  if (w16 && vec_shape(a.H, a.P, a.N, a.G))
+  if (w16 && vec_shape(a.H, a.P, a.N, a.G, width))
     block_prep_vec_kernel<<<(unsigned)M, kPrepThreads, smem, s>>>(a);
   else
     block_prep_kernel<<<(unsigned)M, kPrepThreads, smem, s>>>(a);
@@ -362,9 +367,9 @@ m3ssd_status back(const m3ssd_block_dims* d, const m3ssd_block_weights* w, int64
   const int64_t n = M * HP;
   const int64_t width = in_proj_width(d);
   const auto* yp = reinterpret_cast<const __nv_bfloat16*>(base + ws.y);
-  const auto* zp = reinterpret_cast<const float*>(base + ws.zx);
+  const auto* zp = reinterpret_cast<const __nv_bfloat16*>(base + ws.zx);
   auto* gp = reinterpret_cast<__nv_bfloat16*>(base + ws.x);
-  if (HP % 8 == 0 && width % 4 == 0) {
+  if (HP % 8 == 0 && width % 8 == 0) {
     const int64_t n8 = n / 8;
     const unsigned grid = (unsigned)((n8 + 255) / 256 < 148 * 16 ? (n8 + 255) / 256 : 148 * 16);
     block_gate_vec_kernel<<<grid, 256, 0, s>>>(yp, zp, width, HP, M, gp);

@@ -1,12 +1,13 @@
 """The Mamba-3 SISO block through the C ABI (m3ssd_block_fwd / m3ssd_block_step)
 against the fp64 block oracle on the same seeded bf16 input and weights.
 
-The block's bf16 hand-offs (x, the per-head B' and C', the scan output y and
-the gated y * SiLU(z) that out_proj reads) are rounded to bf16 on both sides
-(the oracle's ``store`` hook, following the pages' policy that a bf16 op
-downcasts its output).  With the fp32 sequential scan in between, the two
-sides then agree to the final output rounding (the general-shape cases below
-show it); the chunked scan adds its bf16 tensor-core operands.
+The block's bf16 hand-offs (the in_proj output z, x, B, C, dt, lam, theta, the
+normed group vectors of B and C, the scan output y and the gated y * SiLU(z)
+that out_proj reads) are rounded to bf16 on both sides (the oracle's ``store``
+hook, following the pages' policy that a bf16 op downcasts its output).  With
+the fp32 sequential scan in between, the two sides then agree to the final
+output rounding (the general-shape cases below show it); the chunked scan adds
+its bf16 tensor-core operands.
 
 Bars (the pages state none for the block; derived here):
   - per element, |gpu - oracle| beyond the final bf16 rounding is at most
@@ -16,10 +17,12 @@ Bars (the pages state none for the block; derived here):
     of the bf16 values it was built from -- a hand-off can land one bf16 ulp
     (2^-8) away from the oracle's rounding, and the chunked scan's operands
     carry 2^-9 each;
-  - against the unrounded fp64 oracle, the RMS error is at most 5e-3: five
-    bf16 hand-offs and the final rounding, each an independent relative error
-    of RMS 2^-9 / sqrt(3) ~ 1.1e-3, give about 2.7e-3, and the chunked scan's
-    own operands about 1.5e-3 more.
+  - against the unrounded fp64 oracle, the RMS error is at most 8e-3: each
+    stage on the path (in_proj output, normed B and C, the scan's bf16
+    operands, y, the gated product, the output) adds a relative rounding error
+    of RMS 2^-9 / sqrt(3) ~ 1.1e-3, and the stages are not independent (a
+    rounded dt or lam shifts the decay of every later state), so the bar takes
+    their plain sum over seven stages, 7.9e-3, rather than the root-sum-square.
 """
 import numpy as np
 import pytest
@@ -31,7 +34,7 @@ from selective_state_space_m3ssd_b200.synth import BLOCKS, make_block
 from tests.gpu_util import rel_close_err, rms_rel_err
 
 pytestmark = pytest.mark.gpu
-TOL_ABS, RTOL, TOL_RMS_EXACT = 2e-2, 2.0 ** -7, 5e-3
+TOL_ABS, RTOL, TOL_RMS_EXACT = 2e-2, 2.0 ** -7, 8e-3
 
 
 def bf16_store(a):

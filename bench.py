@@ -228,6 +228,26 @@ def bench_forward(w, dev, steps, warmup, world, rank):
             "dev_inputs": d, "call": call, "launches": steps}
 
 
+def forward_leg(key, dev, steps, warmup, world, rank, peaks):
+    """The forward on another of the scan workloads (its own inputs, HBM roofline
+    on its own algorithmic bytes); a side figure, not the headline."""
+    w = rank_workload(WORKLOADS[key], rank)
+    fw = bench_forward(w, dev, steps, warmup, world, rank)
+    achieved = fw["algo_bytes"] / (fw["ms_per_step"] / 1e3) / 1e9
+    out = {"metric": "scan Mtokens/s (fwd)",
+           "value": w.batch * w.seqlen * world / (fw["ms_per_step"] / 1e3) / 1e6,
+           "unit": "Mtokens/s", "ms_per_step": fw["ms_per_step"], "steps": steps,
+           "config": fwd_config(w),
+           "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                        "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                        "algo_bytes_per_launch": fw["algo_bytes"], "traffic": None,
+                        "peak_source": peaks["source"]},
+           "gpu_launches": fw["launches"]}
+    del fw
+    torch.cuda.empty_cache()
+    return out
+
+
 def bench_e2e(w, dev, steps, warmup, inp_cpu, world):
     """Same metric through host buffers: every step copies all inputs from pinned
     host memory (H2D), calls the C-ABI forward and copies Y and hT back (D2H),
@@ -576,6 +596,9 @@ def run_ours(args):
         blk = None if args.no_block else bench_block(dev, rank, peaks)
         bwd = None if args.no_backward else bench_backward(
             w, dev, max(1, min(args.steps, 3)), world, fw["dev_inputs"], peaks)
+        others = {} if args.no_other_workloads else {
+            k: forward_leg(k, dev, min(args.steps, 10), args.warmup, world, rank, peaks)
+            for k in ("ssd", "long")}
     e2e = bench_e2e(w, dev, max(1, min(args.steps, 10)), 3, fw["inp"], world)
 
     tokens = w.batch * w.seqlen * args.steps * world
@@ -598,6 +621,8 @@ def run_ours(args):
         "mimo_decode": mimo,
         "block": blk,
         "backward": bwd,
+        "ssd_forward": others.get("ssd"),
+        "long_forward": others.get("long"),
         "clocks": clk.summary(),
     }
     if world > 1:
@@ -700,6 +725,8 @@ def main():
                     help="skip the Mamba-3 SISO block measurement")
     ap.add_argument("--no-backward", action="store_true",
                     help="skip the backward measurement")
+    ap.add_argument("--no-other-workloads", action="store_true",
+                    help="skip the forward on the ssd and long workloads (side figures)")
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="omit the oracle timing (it never runs inside a GPU timed region)")
     ap.add_argument("--profile", choices=["forward", "block", "backward"],

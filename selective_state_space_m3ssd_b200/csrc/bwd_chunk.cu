@@ -19,12 +19,16 @@
 // plus exp(cs_r)'s own terms (Cbar_r . h_prev dy_r and <g, h_prev> at r = 63),
 // and the rotation adjoints dv = R(phi)^T dvbar, dphi_i, dtheta = suffix sums of dphi.
 //
-// Pass 1 walks the chunks forward and stores each chunk's starting state and
-// angle in the workspace.  Pass 2 walks them in reverse; every product is a
-// register-tiled loop over fp32 shared-memory tiles, and every cross-thread sum
-// runs in a fixed order (warp shuffles, then fixed-order shared-memory sums), so
-// the result does not depend on scheduling.  The group-shared dB, dC, dbprev0 and
-// dD are written per head and summed by a second kernel.
+// Pass 1 walks the chunks forward and stores each chunk's starting state (fp32,
+// as (p, n)) and angle in the workspace.  Pass 2 walks them in reverse; every
+// product is a register-tiled loop over fp32 shared-memory tiles in packed fp32
+// pairs, the products with a zero triangle skip it warp by warp, and every
+// cross-thread sum runs in a fixed order (warp shuffles, then fixed-order
+// shared-memory sums), so the result does not depend on scheduling.  The next
+// chunk's inputs are fetched a phase ahead: into registers in pass 1, by
+// cp.async into the tiles already free in pass 2 (16-byte aligned inputs; an
+// element-wise path otherwise).  The group-shared dB, dC, dbprev0 and dD are
+// written per head and summed by a second kernel.
 #include "common.cuh"
 #include "internal.h"
 

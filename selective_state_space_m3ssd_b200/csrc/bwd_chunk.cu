@@ -33,17 +33,16 @@
 #include "internal.h"
 
 namespace m3ssd {
+
 namespace {
 
 constexpr int kQ = 64, QT = kQ - 1, kN = 128, kNH = kN / 2, kP = 64, kT = 512;
 constexpr int SB = kN + 4;  // row stride of the Bbar / Cbar tiles (floats)
 constexpr int SX = kP + 4;  // row stride of the 64-wide tiles
-
 size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
 
-struct ChunkWs {
-  size_t hs, phs, dBh, dCh, dbph, dDbh, total;
-};
+}  // namespace
+
 ChunkWs chunk_ws_layout(int64_t b, int64_t L, int64_t H) {
   const size_t bh = (size_t)(b * H), nC = (size_t)((L + QT - 1) / QT);
   ChunkWs w{};
@@ -62,6 +61,8 @@ ChunkWs chunk_ws_layout(int64_t b, int64_t L, int64_t H) {
   w.total = o;
   return w;
 }
+
+namespace {
 
 // Shared memory (floats).  The workspace holds each chunk-start state as (p, n).
 struct Sm {
@@ -1100,6 +1101,11 @@ cudaError_t launch_bwd_chunk(const BwdArgs& a, cudaStream_t s) {
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  return launch_bwd_chunk_reduce(a, s);
+}
+
+cudaError_t launch_bwd_chunk_reduce(const BwdArgs& a, cudaStream_t s) {
+  const ChunkWs ws = chunk_ws_layout(a.b, a.L, a.H);
   const int64_t total = a.b * a.L * a.G * kN + a.b * a.G * kN + a.H;
   const int64_t blocks = (total + 255) / 256;
   const unsigned rg = (unsigned)(blocks < 148 * 32 ? (blocks > 0 ? blocks : 1) : 148 * 32);

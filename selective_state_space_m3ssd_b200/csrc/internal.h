@@ -94,6 +94,15 @@ cudaError_t launch_bwd_split(const BwdArgs& a, cudaStream_t s);
 // tokens, forward for the chunk-start states, then in reverse; per-head shares
 // of the group-summed gradients in the workspace.
 bool bwd_chunk_supported(int64_t N, int64_t P);
+// Workspace regions of the chunked backwards (byte offsets): chunk-start
+// states (fp32, (p, n) per chunk) and angles, per-head dB and dC shares,
+// per-head dbprev0 shares and per-(b, h) dD partials.
+struct ChunkWs {
+  size_t hs, phs, dBh, dCh, dbph, dDbh, total;
+};
+ChunkWs chunk_ws_layout(int64_t b, int64_t L, int64_t H);
+// Sums the per-head shares into dB, dC, dbprev0 and dD, in a fixed order.
+cudaError_t launch_bwd_chunk_reduce(const BwdArgs& a, cudaStream_t s);
 size_t bwd_chunk_workspace_bytes(int64_t b, int64_t L, int64_t H);
 cudaError_t launch_bwd_chunk(const BwdArgs& a, cudaStream_t s);
 

@@ -340,9 +340,10 @@ m3ssd_status m3ssd_block_step(const m3ssd_block_dims* dims, const m3ssd_block_we
                               const void* u_t, void* out_t, const m3ssd_cache* cache,
                               void* workspace, size_t workspace_bytes, void* stream);
 
-/* Number of bounded device-side waits of the chunked forward that ran out
- * (each makes its CTA stop and leave its outputs unwritten) since the last
- * call; the count is then reset.  This call synchronises the current device
+/* Number of bounded device-side waits of the chunked forward and of the
+ * tensor-core backward that ran out since the last call (the forward's CTA
+ * then stops and leaves its outputs unwritten; the backward's CTA skips its
+ * remaining waits and leaves its outputs undefined); the count is then reset.  This call synchronises the current device
  * and must not be captured in a CUDA graph.  Returns M3SSD_ERR_INVALID_ARG for
  * a NULL pointer and M3SSD_ERR_CUDA if the device cannot be read. */
 m3ssd_status m3ssd_device_wait_timeouts(uint32_t* count);

@@ -103,6 +103,11 @@ struct ChunkWs {
 ChunkWs chunk_ws_layout(int64_t b, int64_t L, int64_t H);
 // Sums the per-head shares into dB, dC, dbprev0 and dD, in a fixed order.
 cudaError_t launch_bwd_chunk_reduce(const BwdArgs& a, cudaStream_t s);
+// The chunked backward on the tensor cores (bf16 X, B, C, dY; N = 128, P = 64;
+// 16-byte aligned X, B, C, dY and theta); same workspace as the fp32 one.
+bool bwd_tc_supported(const BwdArgs& a);
+cudaError_t launch_bwd_tc(const BwdArgs& a, cudaStream_t s);
+cudaError_t read_and_clear_bwd_wait_timeouts(unsigned int* count);
 size_t bwd_chunk_workspace_bytes(int64_t b, int64_t L, int64_t H);
 cudaError_t launch_bwd_chunk(const BwdArgs& a, cudaStream_t s);
 

@@ -61,9 +61,10 @@ const char* m3ssd_status_string(m3ssd_status s) {
 
 m3ssd_status m3ssd_device_wait_timeouts(uint32_t* count) {
   if (!count) return M3SSD_ERR_INVALID_ARG;
-  unsigned int n = 0;
-  const m3ssd_status st = from_cuda(m3ssd::read_and_clear_wait_timeouts(&n));
-  *count = n;
+  unsigned int n = 0, nb = 0;
+  m3ssd_status st = from_cuda(m3ssd::read_and_clear_wait_timeouts(&n));
+  if (st == M3SSD_OK) st = from_cuda(m3ssd::read_and_clear_bwd_wait_timeouts(&nb));
+  *count = n + nb;
   return st;
 }
 
@@ -242,7 +243,9 @@ m3ssd_status m3ssd_bwd(const m3ssd_dims* dims, const void* X, const float* logde
   a.dD = grads->dD; a.dh0 = grads->dh0; a.dangle0 = grads->dangle0; a.dxprev0 = grads->dxprev0;
   a.dbprev0 = grads->dbprev0; a.workspace = workspace;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (m3ssd::bwd_chunk_supported(a.N, a.P)) return from_cuda(m3ssd::launch_bwd_chunk(a, s));
+  if (m3ssd::bwd_chunk_supported(a.N, a.P))
+    return from_cuda(m3ssd::bwd_tc_supported(a) ? m3ssd::launch_bwd_tc(a, s)
+                                                : m3ssd::launch_bwd_chunk(a, s));
   return from_cuda(m3ssd::bwd_split_supported(a.N, a.P) ? m3ssd::launch_bwd_split(a, s)
                                                          : m3ssd::launch_bwd_seq(a, s));
 }

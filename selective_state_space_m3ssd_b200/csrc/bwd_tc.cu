@@ -11,8 +11,9 @@
 // and the mask, decay, rotation and angle gradients, as there.  Every product
 // runs as tcgen05 MMAs (kind::f16, bf16 operands, fp32 accumulators in TMEM):
 // each fp32 operand is split into a bf16 high part and a bf16 residual, and a
-// product takes all four part products, so each operand carries only its split
-// residual (2^-17 of it); X and dY are bf16 already and enter once.  Operand tiles sit in shared memory in the
+// product takes the part products hi x hi, hi x lo, lo x hi and, where the
+// result feeds the suffix sums of dtheta, lo x lo; X and dY are bf16 already and
+// enter once.  Operand tiles sit in shared memory in the
 // 128-byte-swizzled canonical layout, K-major or MN-major as each product
 // needs (the same tile serves both ways).  TMEM columns: G | E (then V | M^T dY)
 // | Cbar h_prev | dh_prev | dCbar | dBbar.
@@ -84,6 +85,16 @@ __device__ __forceinline__ float col_sum8(float v) {  // over lanes differing in
   return v;
 }
 
+// 16 bytes global -> shared without a register round trip; zero-filled (and
+// nothing read) when !full
+__device__ __forceinline__ void cp16(void* smem_dst, const void* gmem_src, bool full) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(tc5::saddr(smem_dst)),
+               "l"(gmem_src), "r"(full ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 struct SmT {
   uint8_t Bh[kT2], Bl[kT2];      // Bbar (u, n)
   uint8_t Ch[kT2], Cl[kT2];      // Cbar (r, n)
@@ -146,17 +157,20 @@ constexpr uint32_t kI128S = tc5::idesc_bf16(128, 64, true, true);
 constexpr uint32_t kIN128 = tc5::idesc_bf16(64, 128, false, true);
 constexpr uint32_t kIN128mn = tc5::idesc_bf16(64, 128, true, true);
 
-// (hi + lo) x (hi + lo) of a product whose K steps run over `steps`: all four
-// part products, so the only error left is the residual of each split (2^-17
-// of an operand).
+// (hi + lo) x (hi + lo) of a product whose K steps run over `steps`.  `full`
+// takes all four part products; otherwise the lo x lo part (at most 2^-16 of a
+// product term) is dropped.  Dropping it is a biased error, which the suffix
+// sums over later tokens (dtheta) collect: the products that feed dCbar,
+// dBbar and dh_prev take it, the others (G, Cbar h_prev, Bbar g) do not.
 template <typename FA, typename FB>
-__device__ __forceinline__ void mma4(uint32_t d, uint32_t ah, uint32_t al, uint32_t bh,
-                                     uint32_t bl, uint32_t idesc, int steps, bool acc, FA da,
-                                     FB db) {
+__device__ __forceinline__ void mma_split(uint32_t d, uint32_t ah, uint32_t al, uint32_t bh,
+                                          uint32_t bl, uint32_t idesc, int steps, bool acc,
+                                          bool full, FA da, FB db) {
   for (int j = 0; j < steps; ++j) tc5::mma_bf16(d, da(ah, j), db(bh, j), idesc, acc || j > 0);
   for (int j = 0; j < steps; ++j) tc5::mma_bf16(d, da(ah, j), db(bl, j), idesc, true);
   for (int j = 0; j < steps; ++j) tc5::mma_bf16(d, da(al, j), db(bh, j), idesc, true);
-  for (int j = 0; j < steps; ++j) tc5::mma_bf16(d, da(al, j), db(bl, j), idesc, true);
+  if (full)
+    for (int j = 0; j < steps; ++j) tc5::mma_bf16(d, da(al, j), db(bl, j), idesc, true);
 }
 
 __global__ void __launch_bounds__(kT, 1) bwd_tc_kernel(BwdArgs a, ChunkWs ws) {
@@ -221,35 +235,28 @@ __global__ void __launch_bounds__(kT, 1) bwd_tc_kernel(BwdArgs a, ChunkWs ws) {
     tc5::fence_after_sync();
   };
 
-  // ---- the inputs of chunk c: rows r <-> tokens t0 - 1 + r -------------------
-  // thread (r = tid / 8, sg = tid % 8): X, dY columns 8 sg .., theta pairs
-  // 8 sg .., B and C columns 16 sg .. (B and C stay in registers until the
-  // rotation, which the same thread does)
+  // ---- the state pass's inputs of chunk c: rows r <-> tokens t0 - 1 + r ------
+  // thread (r = tid / 8, sg = tid % 8): X columns 8 sg .., theta pairs 8 sg ..,
+  // B columns 16 sg .. (B stays in registers until the rotation, which the same
+  // thread does)
   const int lr = tid >> 3, sg = tid & 7;
   float braw[16], craw[16], xf8[8], yf8[8];
-  auto load_chunk = [&](int c, bool bwd) {
+  auto load_chunk = [&](int c) {
     const int64_t t0 = (int64_t)c * QT - 1;
     const int64_t t = t0 + lr;
     const bool in = t >= 0 && t < L, own = lr > 0 && t < L;
     const int64_t th = (b * L + (in ? t : 0)) * H + h, tg = (b * L + (in ? t : 0)) * G + g;
-    uint4 xv = make_uint4(0u, 0u, 0u, 0u), yv = xv;
-    uint4 bv[2] = {xv, xv}, cvv[2] = {xv, xv};
+    uint4 xv = make_uint4(0u, 0u, 0u, 0u);
+    uint4 bv[2] = {xv, xv};
     float4 tv0 = make_float4(0.f, 0.f, 0.f, 0.f), tv1 = tv0;
     if (in) {
       xv = *reinterpret_cast<const uint4*>(X + th * kP + 8 * sg);
       bv[0] = *reinterpret_cast<const uint4*>(Bg + tg * kN + 16 * sg);
       bv[1] = *reinterpret_cast<const uint4*>(Bg + tg * kN + 16 * sg + 8);
     }
-    if (own) {
-      if (a.theta) {
-        tv0 = *reinterpret_cast<const float4*>(a.theta + th * kNH + 8 * sg);
-        tv1 = *reinterpret_cast<const float4*>(a.theta + th * kNH + 8 * sg + 4);
-      }
-      if (bwd) {
-        yv = *reinterpret_cast<const uint4*>(dY + th * kP + 8 * sg);
-        cvv[0] = *reinterpret_cast<const uint4*>(Cg + tg * kN + 16 * sg);
-        cvv[1] = *reinterpret_cast<const uint4*>(Cg + tg * kN + 16 * sg + 8);
-      }
+    if (own && a.theta) {
+      tv0 = *reinterpret_cast<const float4*>(a.theta + th * kNH + 8 * sg);
+      tv1 = *reinterpret_cast<const float4*>(a.theta + th * kNH + 8 * sg + 4);
     }
     float sc[3] = {0.f, 0.f, 0.f};
     if (tid < kQ && tid > 0 && t0 + tid < L) {
@@ -261,29 +268,15 @@ __global__ void __launch_bounds__(kT, 1) bwd_tc_kernel(BwdArgs a, ChunkWs ws) {
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
       const uint32_t w4[4] = {bv[k].x, bv[k].y, bv[k].z, bv[k].w};
-      const uint32_t c4[4] = {cvv[k].x, cvv[k].y, cvv[k].z, cvv[k].w};
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        const float2 fb = unpack_bf16(w4[q]), fc = unpack_bf16(c4[q]);
+        const float2 fb = unpack_bf16(w4[q]);
         braw[8 * k + 2 * q] = fb.x;
         braw[8 * k + 2 * q + 1] = fb.y;
-        craw[8 * k + 2 * q] = fc.x;
-        craw[8 * k + 2 * q + 1] = fc.y;
-      }
-    }
-    {
-      const uint32_t x4[4] = {xv.x, xv.y, xv.z, xv.w}, y4[4] = {yv.x, yv.y, yv.z, yv.w};
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float2 fx = unpack_bf16(x4[q]), fy = unpack_bf16(y4[q]);
-        xf8[2 * q] = fx.x;
-        xf8[2 * q + 1] = fx.y;
-        yf8[2 * q] = fy.x;
-        yf8[2 * q + 1] = fy.y;
       }
     }
     if (t == -1) {  // the cache's carry-in token, fp32: X as a high part and a residual
-      float* xf = xf8;
+      float xf[8];
 #pragma unroll
       for (int k = 0; k < 8; ++k) xf[k] = a.xprev0 ? a.xprev0[bh * kP + 8 * sg + k] : 0.f;
 #pragma unroll
@@ -295,7 +288,6 @@ __global__ void __launch_bounds__(kT, 1) bwd_tc_kernel(BwdArgs a, ChunkWs ws) {
       *reinterpret_cast<uint4*>(sm.Xl + off1(0, 8 * sg)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
     }
     *reinterpret_cast<uint4*>(sm.X + off1(lr, 8 * sg)) = xv;
-    if (bwd) *reinterpret_cast<uint4*>(sm.Y + off1(lr, 8 * sg)) = yv;
     *reinterpret_cast<float4*>(&sm.Vt[lr * kNH + 8 * sg]) = tv0;
     *reinterpret_cast<float4*>(&sm.Vt[lr * kNH + 8 * sg + 4]) = tv1;
     if (tid < kQ) {
@@ -415,6 +407,91 @@ __global__ void __launch_bounds__(kT, 1) bwd_tc_kernel(BwdArgs a, ChunkWs ws) {
     }
   };
 
+  // ---- the reverse pass's inputs one chunk ahead: X, dY, theta and raw B, C
+  // rows by cp.async into their tiles (free from the end of the previous
+  // chunk's epilogue on), the chunk-start state, scalars and angle into
+  // registers; commit_chunk() lands them
+  struct Pre {
+    float hp[16];
+    float sc[3];
+    float ph;
+  };
+  auto fetch_chunk = [&](int c, Pre& f) {
+    const int64_t t0 = (int64_t)c * QT - 1;
+    const int64_t t = t0 + lr;
+    const bool in = t >= 0 && t < L, own = lr > 0 && t < L;
+    const int64_t th = (b * L + (in ? t : 0)) * H + h, tg = (b * L + (in ? t : 0)) * G + g;
+    cp16(sm.X + off1(lr, 8 * sg), X + th * kP + 8 * sg, in);
+    cp16(sm.Y + off1(lr, 8 * sg), dY + th * kP + 8 * sg, own);
+    const bool th_ok = own && a.theta != nullptr;
+    const float* tsrc = th_ok ? a.theta + th * kNH + 8 * sg : reinterpret_cast<const float*>(X);
+    cp16(&sm.Vt[lr * kNH + 8 * sg], tsrc, th_ok);
+    cp16(&sm.Vt[lr * kNH + 8 * sg + 4], th_ok ? tsrc + 4 : tsrc, th_ok);
+    cp16(sm.Bh + off2(lr, 16 * sg), Bg + tg * kN + 16 * sg, in);
+    cp16(sm.Bh + off2(lr, 16 * sg + 8), Bg + tg * kN + 16 * sg + 8, in);
+    cp16(sm.Ch + off2(lr, 16 * sg), Cg + tg * kN + 16 * sg, own);
+    cp16(sm.Ch + off2(lr, 16 * sg + 8), Cg + tg * kN + 16 * sg + 8, own);
+    cp_commit();
+    const float* hw = hs_ws + (int64_t)c * kN * kP;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) f.hp[j] = hw[(16 * q4 + j) * kN + nrow];
+    f.sc[0] = f.sc[1] = f.sc[2] = 0.f;
+    f.ph = 0.f;
+    if (tid < kQ) {
+      if (tid > 0 && t0 + tid < L) {
+        const int64_t ts = (b * L + t0 + tid) * H + h;
+        f.sc[0] = a.logdecay[ts];
+        f.sc[1] = a.gamma[ts];
+        f.sc[2] = a.beta ? a.beta[ts] : 0.f;
+      }
+      if (tid < kNH) f.ph = ph_ws[(int64_t)c * kNH + tid];
+    }
+  };
+  auto commit_chunk = [&](int c, const Pre& f) {
+    cp_wait_all();
+    __syncthreads();  // every thread's copies have landed
+    const int64_t t0 = (int64_t)c * QT - 1;
+    // this thread's raw B, C (16 columns) and x, dy (8 columns) in fp32
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int n = 16 * sg + 2 * q;
+      const float2 fb = unpack_bf16(*reinterpret_cast<const uint32_t*>(sm.Bh + off2(lr, n)));
+      const float2 fc = unpack_bf16(*reinterpret_cast<const uint32_t*>(sm.Ch + off2(lr, n)));
+      braw[2 * q] = fb.x;
+      braw[2 * q + 1] = fb.y;
+      craw[2 * q] = fc.x;
+      craw[2 * q + 1] = fc.y;
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int p = 8 * sg + 2 * q;
+      const float2 fx = unpack_bf16(*reinterpret_cast<const uint32_t*>(sm.X + off1(lr, p)));
+      const float2 fy = unpack_bf16(*reinterpret_cast<const uint32_t*>(sm.Y + off1(lr, p)));
+      xf8[2 * q] = fx.x;
+      xf8[2 * q + 1] = fx.y;
+      yf8[2 * q] = fy.x;
+      yf8[2 * q + 1] = fy.y;
+    }
+    if (t0 + lr == -1) {  // the cache's carry-in token, fp32
+#pragma unroll
+      for (int k = 0; k < 8; ++k) xf8[k] = a.xprev0 ? a.xprev0[bh * kP + 8 * sg + k] : 0.f;
+#pragma unroll
+      for (int k = 0; k < 16; ++k) braw[k] = a.bprev0 ? a.bprev0[(b * G + g) * kN + 16 * sg + k] : 0.f;
+      uint32_t hi[4], lo[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) split2(xf8[2 * q], xf8[2 * q + 1], hi[q], lo[q]);
+      *reinterpret_cast<uint4*>(sm.X + off1(0, 8 * sg)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+      *reinterpret_cast<uint4*>(sm.Xl + off1(0, 8 * sg)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+    }
+    store_pn(sm.Hh, sm.Hl, f.hp);
+    if (tid < kQ) {
+      sm.cs[tid] = f.sc[0];  // the raw logdecay until chunk_scalars
+      sm.ga[tid] = f.sc[1];
+      sm.be[tid] = f.sc[2];
+      if (tid < kNH) sm.phi0[tid] = f.ph;
+    }
+  };
+
   const auto K2 = [](uint32_t ad, int j) { return dk2(ad, j); };
   const auto K1 = [](uint32_t ad, int j) { return dk1(ad, j); };
   const auto MN = [](uint32_t ad, int j) { return dmn(ad, j); };
@@ -429,7 +506,7 @@ __global__ void __launch_bounds__(kT, 1) bwd_tc_kernel(BwdArgs a, ChunkWs ws) {
 #pragma unroll
     for (int j = 0; j < 16; ++j) hw[(16 * q4 + j) * kN + nrow] = hreg[j];
     if (tid < kNH) ph_ws[(int64_t)c * kNH + tid] = sm.phi0[tid];
-    load_chunk(c, false);
+    load_chunk(c);
     __syncthreads();
     chunk_scalars();
     angles();
@@ -466,6 +543,8 @@ __global__ void __launch_bounds__(kT, 1) bwd_tc_kernel(BwdArgs a, ChunkWs ws) {
   if (tid < kP) sm.cdx[0][tid] = sm.cdx[1][tid] = 0.f;
   if (tid < kN) sm.cdb[0][tid] = sm.cdb[1][tid] = 0.f;
   float dDacc = 0.f;
+  Pre f;
+  if (nC > 0) fetch_chunk(nC - 1, f);
   __syncthreads();
 
   for (int c = nC - 1; c >= 0; --c) {
@@ -473,14 +552,9 @@ __global__ void __launch_bounds__(kT, 1) bwd_tc_kernel(BwdArgs a, ChunkWs ws) {
     const int64_t t0 = (int64_t)c * QT - 1;
     auto own = [&](int r) { return r > 0 && t0 + r < L; };
     float hpr[16];
-    {
-      const float* hw = hs_ws + (int64_t)c * kN * kP;
 #pragma unroll
-      for (int j = 0; j < 16; ++j) hpr[j] = hw[(16 * q4 + j) * kN + nrow];
-      if (tid < kNH) sm.phi0[tid] = ph_ws[(int64_t)c * kNH + tid];
-    }
-    load_chunk(c, true);
-    store_pn(sm.Hh, sm.Hl, hpr);
+    for (int j = 0; j < 16; ++j) hpr[j] = f.hp[j];
+    commit_chunk(c, f);
     __syncthreads();
     chunk_scalars();
     angles();
@@ -489,15 +563,15 @@ __global__ void __launch_bounds__(kT, 1) bwd_tc_kernel(BwdArgs a, ChunkWs ws) {
 
     // -- stage 1
     if (tid == 0) {
-      mma4(tmem + kColG, aCh, aCl, aBh, aBl, kI64, 8, false, K2, K2);  // G = Cbar Bbar^T
+      mma_split(tmem + kColG, aCh, aCl, aBh, aBl, kI64, 8, false, false, K2, K2);  // G
       for (int j = 0; j < 4; ++j) tc5::mma_bf16(tmem + kColE, dk1(aY, j), dk1(aX, j), kI64, j > 0);
       if (c == 0 && has_xl)
         for (int j = 0; j < 4; ++j) tc5::mma_bf16(tmem + kColE, dk1(aY, j), dk1(aXl, j), kI64, true);
       tc5::commit(&sm.mbar[0]);                                          // G, E
-      mma4(tmem + kColY, aCh, aCl, aHh, aHl, kI64, 8, false, K2, K2);    // Cbar h_prev
-      mma4(tmem + kColDH, aCh, aCl, aEh, aEl, kI128S, 4, false, MN, MN); // Cbar^T (e^cs dY)
-      mma4(tmem + kColDB, aWh, aWl, aGh, aGl, kIN128, 4, false, K1, MN); // (W_end X) g^T
-      mma4(tmem + kColDC, aEh, aEl, aHh, aHl, kIN128, 4, false, K1, MN); // (e^cs dY) h_prev^T
+      mma_split(tmem + kColY, aCh, aCl, aHh, aHl, kI64, 8, false, false, K2, K2);    // Cbar h_prev
+      mma_split(tmem + kColDH, aCh, aCl, aEh, aEl, kI128S, 4, false, true, MN, MN); // Cbar^T e^cs dY
+      mma_split(tmem + kColDB, aWh, aWl, aGh, aGl, kIN128, 4, false, true, K1, MN); // (W_end X) g^T
+      mma_split(tmem + kColDC, aEh, aEl, aHh, aHl, kIN128, 4, false, true, K1, MN); // e^cs dY h_prev^T
       tc5::commit(&sm.mbar[1]);
     }
 
@@ -618,11 +692,11 @@ __global__ void __launch_bounds__(kT, 1) bwd_tc_kernel(BwdArgs a, ChunkWs ws) {
 
     // -- stage 2
     if (tid == 0) {
-      mma4(tmem + kColG, aBh, aBl, aGh, aGl, kI64, 8, false, K2, K2);  // Bbar g
+      mma_split(tmem + kColG, aBh, aBl, aGh, aGl, kI64, 8, false, false, K2, K2);  // Bbar g
       for (int j = 0; j < 4; ++j) tc5::mma_bf16(tmem + kColE, dmn(aEh, j), dmn(aY, j), kI64mn, j > 0);
       for (int j = 0; j < 4; ++j) tc5::mma_bf16(tmem + kColE, dmn(aEl, j), dmn(aY, j), kI64mn, true);
-      mma4(tmem + kColDC, aWh, aWl, aBh, aBl, kIN128, 4, true, K1, MN);    // += WE Bbar
-      mma4(tmem + kColDB, aWh, aWl, aCh, aCl, kIN128mn, 4, true, MN, MN);  // += WE^T Cbar
+      mma_split(tmem + kColDC, aWh, aWl, aBh, aBl, kIN128, 4, true, true, K1, MN);    // += WE Bbar
+      mma_split(tmem + kColDB, aWh, aWl, aCh, aCl, kIN128mn, 4, true, true, MN, MN);  // += WE^T Cbar
       tc5::commit(&sm.mbar[2]);
     }
     block_sum(ghp, sm.red, &sm.misc[0]);
@@ -715,10 +789,12 @@ __global__ void __launch_bounds__(kT, 1) bwd_tc_kernel(BwdArgs a, ChunkWs ws) {
         }
       }
     }
-    store_pn(sm.Gh, sm.Gl, greg);  // the next (earlier) chunk's g
     tc5::fence_before_sync();
-    __syncthreads();
+    __syncthreads();  // the tiles of X, dY, theta and B, C are read: fetch the next chunk
     tc5::fence_after_sync();
+    if (c > 0) fetch_chunk(c - 1, f);
+    store_pn(sm.Gh, sm.Gl, greg);  // the next (earlier) chunk's g
+    __syncthreads();
 
     // -- the scalar chain: decay sums -> cv -> gamma, beta, logdecay (warp 0)
     if (warp == 0) {

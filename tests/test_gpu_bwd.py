@@ -11,12 +11,13 @@ of order 1e-6 of a gradient's scale, a few 1e-5 over a few hundred tokens.
 
 The tensor-core chunked kernel (bf16 inputs, N = 128, P = 64): bar 1e-3.  Each
 fp32 operand enters its products as a bf16 high part plus a bf16 residual, whose
-own rounding leaves at most 2^-18 of the element, and all four part products
-are taken: a product term carries up to 2^-17 relative error, about 16 times the
-fp32 kernels'.  The gradients are heavy-tailed (max / RMS up to about 16), so an
+own rounding leaves at most 2^-18 of the element; the products take
+hi x hi + hi x lo + lo x hi, and lo x lo too where they feed dtheta's suffix
+sums: a product term carries up to about 2^-16 relative error, some 30 times
+the fp32 kernels'.  The gradients are heavy-tailed (max / RMS up to about 16), so an
 element's error reaches about 1e-4 of the RMS, and dtheta and dlogdecay, suffix
 sums over every later token, collect the errors of all later chunks (measured
-3.2e-4 at L = 4096, under 1.6e-4 at L <= 400).
+3.2e-4 at L = 4096 for dtheta, under 1.6e-4 at L <= 400).
 """
 import numpy as np
 import pytest

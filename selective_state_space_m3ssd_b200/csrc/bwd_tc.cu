@@ -235,47 +235,57 @@ __global__ void __launch_bounds__(kT, 1) bwd_tc_kernel(BwdArgs a, ChunkWs ws) {
     tc5::fence_after_sync();
   };
 
-  // ---- the state pass's inputs of chunk c: rows r <-> tokens t0 - 1 + r ------
-  // thread (r = tid / 8, sg = tid % 8): X columns 8 sg .., theta pairs 8 sg ..,
-  // B columns 16 sg .. (B stays in registers until the rotation, which the same
-  // thread does)
+  // ---- the state pass's inputs, one chunk ahead: theta and raw B rows by
+  // cp.async once the rotation has read the previous ones, X once the state
+  // product has; thread (r = tid / 8, sg = tid % 8) owns X columns 8 sg ..,
+  // theta pairs 8 sg .. and B columns 16 sg .. of row r
   const int lr = tid >> 3, sg = tid & 7;
   float braw[16], craw[16], xf8[8], yf8[8];
-  auto load_chunk = [&](int c) {
+  float sc1[3] = {0.f, 0.f, 0.f};  // logdecay, gamma, beta of row tid (tid < 64)
+  auto rows_of = [&](int c, int64_t& th, int64_t& tg, bool& in, bool& own) {
+    const int64_t t = (int64_t)c * QT - 1 + lr;
+    in = t >= 0 && t < L;
+    own = lr > 0 && t < L;
+    th = (b * L + (in ? t : 0)) * H + h;
+    tg = (b * L + (in ? t : 0)) * G + g;
+  };
+  auto fetch1_tb = [&](int c) {  // theta, raw B, the scalars
+    int64_t th, tg;
+    bool in, own;
+    rows_of(c, th, tg, in, own);
+    const bool th_ok = own && a.theta != nullptr;
+    const float* tsrc = th_ok ? a.theta + th * kNH + 8 * sg : reinterpret_cast<const float*>(X);
+    cp16(&sm.Vt[lr * kNH + 8 * sg], tsrc, th_ok);
+    cp16(&sm.Vt[lr * kNH + 8 * sg + 4], th_ok ? tsrc + 4 : tsrc, th_ok);
+    cp16(sm.Bh + off2(lr, 16 * sg), Bg + tg * kN + 16 * sg, in);
+    cp16(sm.Bh + off2(lr, 16 * sg + 8), Bg + tg * kN + 16 * sg + 8, in);
+    cp_commit();
     const int64_t t0 = (int64_t)c * QT - 1;
-    const int64_t t = t0 + lr;
-    const bool in = t >= 0 && t < L, own = lr > 0 && t < L;
-    const int64_t th = (b * L + (in ? t : 0)) * H + h, tg = (b * L + (in ? t : 0)) * G + g;
-    uint4 xv = make_uint4(0u, 0u, 0u, 0u);
-    uint4 bv[2] = {xv, xv};
-    float4 tv0 = make_float4(0.f, 0.f, 0.f, 0.f), tv1 = tv0;
-    if (in) {
-      xv = *reinterpret_cast<const uint4*>(X + th * kP + 8 * sg);
-      bv[0] = *reinterpret_cast<const uint4*>(Bg + tg * kN + 16 * sg);
-      bv[1] = *reinterpret_cast<const uint4*>(Bg + tg * kN + 16 * sg + 8);
-    }
-    if (own && a.theta) {
-      tv0 = *reinterpret_cast<const float4*>(a.theta + th * kNH + 8 * sg);
-      tv1 = *reinterpret_cast<const float4*>(a.theta + th * kNH + 8 * sg + 4);
-    }
-    float sc[3] = {0.f, 0.f, 0.f};
+    sc1[0] = sc1[1] = sc1[2] = 0.f;
     if (tid < kQ && tid > 0 && t0 + tid < L) {
       const int64_t ts = (b * L + t0 + tid) * H + h;
-      sc[0] = a.logdecay[ts];
-      sc[1] = a.gamma[ts];
-      sc[2] = a.beta ? a.beta[ts] : 0.f;
+      sc1[0] = a.logdecay[ts];
+      sc1[1] = a.gamma[ts];
+      sc1[2] = a.beta ? a.beta[ts] : 0.f;
     }
+  };
+  auto fetch1_x = [&](int c) {
+    int64_t th, tg;
+    bool in, own;
+    rows_of(c, th, tg, in, own);
+    cp16(sm.X + off1(lr, 8 * sg), X + th * kP + 8 * sg, in);
+    cp_commit();
+  };
+  auto commit1 = [&](int c) {
+    cp_wait_all();
+    __syncthreads();  // every thread's copies have landed
 #pragma unroll
-    for (int k = 0; k < 2; ++k) {
-      const uint32_t w4[4] = {bv[k].x, bv[k].y, bv[k].z, bv[k].w};
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float2 fb = unpack_bf16(w4[q]);
-        braw[8 * k + 2 * q] = fb.x;
-        braw[8 * k + 2 * q + 1] = fb.y;
-      }
+    for (int q = 0; q < 8; ++q) {
+      const float2 fb = unpack_bf16(*reinterpret_cast<const uint32_t*>(sm.Bh + off2(lr, 16 * sg + 2 * q)));
+      braw[2 * q] = fb.x;
+      braw[2 * q + 1] = fb.y;
     }
-    if (t == -1) {  // the cache's carry-in token, fp32: X as a high part and a residual
+    if ((int64_t)c * QT - 1 + lr == -1) {  // the cache's carry-in token, fp32
       float xf[8];
 #pragma unroll
       for (int k = 0; k < 8; ++k) xf[k] = a.xprev0 ? a.xprev0[bh * kP + 8 * sg + k] : 0.f;
@@ -284,16 +294,13 @@ __global__ void __launch_bounds__(kT, 1) bwd_tc_kernel(BwdArgs a, ChunkWs ws) {
       uint32_t hi[4], lo[4];
 #pragma unroll
       for (int q = 0; q < 4; ++q) split2(xf[2 * q], xf[2 * q + 1], hi[q], lo[q]);
-      xv = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+      *reinterpret_cast<uint4*>(sm.X + off1(0, 8 * sg)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
       *reinterpret_cast<uint4*>(sm.Xl + off1(0, 8 * sg)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
     }
-    *reinterpret_cast<uint4*>(sm.X + off1(lr, 8 * sg)) = xv;
-    *reinterpret_cast<float4*>(&sm.Vt[lr * kNH + 8 * sg]) = tv0;
-    *reinterpret_cast<float4*>(&sm.Vt[lr * kNH + 8 * sg + 4]) = tv1;
     if (tid < kQ) {
-      sm.cs[tid] = sc[0];  // the raw logdecay until chunk_scalars
-      sm.ga[tid] = sc[1];
-      sm.be[tid] = sc[2];
+      sm.cs[tid] = sc1[0];  // the raw logdecay until chunk_scalars
+      sm.ga[tid] = sc1[1];
+      sm.be[tid] = sc1[2];
     }
   };
 
@@ -501,17 +508,23 @@ __global__ void __launch_bounds__(kT, 1) bwd_tc_kernel(BwdArgs a, ChunkWs ws) {
   float hreg[16];  // h rows nrow, columns 16 q4 + j
 #pragma unroll
   for (int j = 0; j < 16; ++j) hreg[j] = a.h0 ? a.h0[(bh * kN + nrow) * kP + 16 * q4 + j] : 0.f;
+  if (nC > 0) {
+    fetch1_tb(0);
+    fetch1_x(0);
+  }
   for (int c = 0; c < nC; ++c) {
     float* hw = hs_ws + (int64_t)c * kN * kP;  // (p, n)
 #pragma unroll
     for (int j = 0; j < 16; ++j) hw[(16 * q4 + j) * kN + nrow] = hreg[j];
     if (tid < kNH) ph_ws[(int64_t)c * kNH + tid] = sm.phi0[tid];
-    load_chunk(c);
+    commit1(c);
     __syncthreads();
     chunk_scalars();
     angles();
+    const float nphi = tid < kNH ? wrap_angle(sm.Vt[(kQ - 1) * kNH + tid]) : 0.f;
     rotate(false);
-    mma_fence_sync();
+    mma_fence_sync();  // the rotation has read theta and B: the next ones may land
+    if (c + 1 < nC) fetch1_tb(c + 1);
     if (tid == 0) {
       // S = (W_end o Bbar)^T X: A MN-major (M = n), B MN-major (N = p), K = u
       for (int j = 0; j < 4; ++j) tc5::mma_bf16(tmem + kColG, dmn(aGh, j), dmn(aX, j), kI128S, j > 0);
@@ -521,6 +534,7 @@ __global__ void __launch_bounds__(kT, 1) bwd_tc_kernel(BwdArgs a, ChunkWs ws) {
       tc5::commit(&sm.mbar[0]);
     }
     wait_bar(0);
+    if (c + 1 < nC) fetch1_x(c + 1);  // the state product has read X
     uint32_t sv[16];
     tc5::ld_32x32b_x16(tmem + tl + kColG + (uint32_t)(16 * q4), sv);
     tc5::wait_ld();
@@ -528,10 +542,9 @@ __global__ void __launch_bounds__(kT, 1) bwd_tc_kernel(BwdArgs a, ChunkWs ws) {
 #pragma unroll
     for (int j = 0; j < 16; ++j) hreg[j] = fmaf(eE, hreg[j], __uint_as_float(sv[j]));
     tc5::fence_before_sync();
-    __syncthreads();  // every read of this chunk's tiles and columns is done
+    __syncthreads();  // every read of this chunk's scalars and columns is done
     tc5::fence_after_sync();
-    if (tid < kNH) sm.phi0[tid] = wrap_angle(sm.Vt[(kQ - 1) * kNH + tid]);
-    __syncthreads();
+    if (tid < kNH) sm.phi0[tid] = nphi;
   }
 
   // ---- pass 2: the chunks in reverse --------------------------------------

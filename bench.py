@@ -537,16 +537,32 @@ def bench_backward(w, dev, steps, world, d, peaks):
         ms = float(t.item())
     algo = nbytes(*args, dY, dhT, *grads.values())
     flops = bwd_chunk_flops(w.batch, w.seqlen, w.nheads) * world
+    executed = bwd_tc_mma_flops(w.batch, w.seqlen, w.nheads) * world
     tflops = flops / (ms / 1e3) / 1e12
-    peak = fp32_simt_tflops(peaks)
+    peak = peaks["bf16_tflops"]
     return {"metric": "bwd Mtokens/s", "value": w.batch * w.seqlen * world / (ms / 1e3) / 1e6,
             "unit": "Mtokens/s", "ms_per_step": ms, "steps": steps,
-            "roofline": {"bound": "alu", "achieved": tflops, "peak": peak, "unit": "TFLOP/s",
+            "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak, "unit": "TFLOP/s",
                          "frac": tflops / peak, "algo_flops_per_step": flops, "traffic": None,
-                         "peak_source": "148 SMs x 128 fp32 lanes x 2 FLOP x max SM clock"},
+                         "executed_mma_flops_per_step": executed,
+                         "executed_frac": executed / (ms / 1e3) / 1e12 / peak,
+                         "peak_source": peaks["source"] + " bf16 dense"},
             "hbm": {"algo_bytes_per_step": algo, "achieved_gbs": algo / (ms / 1e3) / 1e9,
                     "frac": algo / (ms / 1e3) / 1e9 / peaks["hbm_gbs"]},
-            "kernel": "bwd_chunk_kernel + bwd_chunk_reduce_kernel (chunked fp32, 2 launches)"}
+            "kernel": "bwd_tc_kernel + bwd_chunk_reduce_kernel (tcgen05 chunked backward, "
+                      "2 launches)"}
+
+
+def bwd_tc_mma_flops(b: int, L: int, H: int, N: int = 128, P: int = 64, Q: int = 64) -> int:
+    """FLOPs the tensor-core backward's MMAs execute per call: every fp32
+    operand split into two bf16 parts, three part products (four where they
+    feed dtheta's suffix sums and dh_prev), X and dY exact; per chunk: G, Cbar
+    h_prev and Bbar g at three parts (2 Q^2 N, 2 Q P N, 2 Q N P each), E and
+    M^T dY at one and two (2 Q^2 P each), dh_prev, the two halves of dCbar and
+    dBbar at four (2 N P Q, 2 Q N P and 2 Q^2 N), and the state pass at two."""
+    per_chunk = 3 * (2 * Q * Q * N + 2 * Q * P * N + 2 * Q * N * P) + 2 * Q * Q * P * (1 + 2) + \
+        4 * (2 * N * P * Q + 2 * 2 * Q * N * P + 2 * 2 * Q * Q * N) + 2 * (2 * N * P * Q)
+    return b * H * -(-L // (Q - 1)) * per_chunk
 
 
 def bwd_chunk_flops(b: int, L: int, H: int, N: int = 128, P: int = 64, Q: int = 64) -> int:

@@ -230,10 +230,13 @@ size_t m3ssd_bwd_workspace_size(const m3ssd_dims* dims);
  * fp32, NULL = 0), and writes the fp32 gradients in *grads.  The cache outputs
  * angleT, xprevT and bprevT take no upstream gradient.
  *
- * The backward recomputes the forward in fp32.  At N = 128, P = 64 it works
- * chunk by chunk (one CTA per sequence: a forward pass stores the state and
- * angle at every chunk start, then each chunk's adjoint is a set of fp32
- * products in shared memory, walking the chunks in reverse).  At N = 128 with
+ * The backward recomputes the forward.  At N = 128, P = 64 it works chunk by
+ * chunk (one CTA per sequence: a forward pass stores the state and angle at
+ * every chunk start, then each chunk's adjoint is a set of products, walking
+ * the chunks in reverse): with bf16 X, B, C, dY (16-byte aligned, as theta)
+ * the products run on the tensor cores with every fp32 operand split into a
+ * bf16 high part and residual (about 2^-16 relative error per product term;
+ * gradients within about 1e-3 of their RMS at L = 4096), otherwise in fp32.  At N = 128 with
  * another P a multiple of 16 it splits each sequence over P/16 CTAs of 16
  * state columns and sums the per-slice partials of the column-mixing
  * gradients afterwards; other shapes run one CTA per sequence token by

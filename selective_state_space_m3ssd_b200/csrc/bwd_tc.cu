@@ -98,8 +98,8 @@ __device__ __forceinline__ void cp_wait_all() { asm volatile("cp.async.wait_all;
 struct SmT {
   uint8_t Bh[kT2], Bl[kT2];      // Bbar (u, n)
   uint8_t Ch[kT2], Cl[kT2];      // Cbar (r, n)
-  uint8_t Gh[kT2], Gl[kT2];      // g (p, n); in pass 1 W_end o Bbar (u, n)
-  uint8_t Hh[kT2], Hl[kT2];      // h_prev (p, n)
+  uint8_t Gh[kT2], Gl[kT2];      // g (n, p); in pass 1 W_end o Bbar (u, n)
+  uint8_t Hh[kT2], Hl[kT2];      // h_prev (n, p)
   uint8_t X[kT1], Xl[kT1];       // X (u, p); Xl: residual of the cache's fp32 carry-in row
   uint8_t Y[kT1];                // dY (r, p)
   uint8_t EYh[kT1], EYl[kT1];    // exp(cs) o dY (r, p); then M (r, u); then dphi (fp32)
@@ -155,6 +155,8 @@ constexpr uint32_t kI64 = tc5::idesc_bf16(64, 64, false, false);
 constexpr uint32_t kI64mn = tc5::idesc_bf16(64, 64, true, true);
 constexpr uint32_t kI128S = tc5::idesc_bf16(128, 64, true, true);
 constexpr uint32_t kIN128 = tc5::idesc_bf16(64, 128, false, true);
+constexpr uint32_t kIN128k = tc5::idesc_bf16(64, 128, false, false);
+constexpr uint32_t kI64kmn = tc5::idesc_bf16(64, 64, false, true);
 constexpr uint32_t kIN128mn = tc5::idesc_bf16(64, 128, true, true);
 
 // (hi + lo) x (hi + lo) of a product whose K steps run over `steps`.  `full`
@@ -363,54 +365,65 @@ __global__ void __launch_bounds__(kT, 1) bwd_tc_kernel(BwdArgs a, ChunkWs ws) {
   auto st32 = [](uint8_t* base, uint32_t off, uint32_t v) {
     *reinterpret_cast<uint32_t*>(base + off) = v;
   };
+  auto st128 = [](uint8_t* base, uint32_t off, const uint32_t* v) {
+    *reinterpret_cast<uint4*>(base + off) = make_uint4(v[0], v[1], v[2], v[3]);
+  };
   auto rotate = [&](bool bwd) {
     const int r = lr;
     const float we = sm.wend[r];
+    uint32_t bh_[8], bl_[8], ch_[8], cl_[8];  // 16 columns 16 sg .. as bf16 pairs
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
-      const int i = 8 * sg + k, n = 2 * i;
+      const int i = 8 * sg + k;
       float sn, cs_;
       fast_sincos(sm.Vt[r * kNH + i], &sn, &cs_);
       const float b0 = braw[2 * k], b1 = braw[2 * k + 1];
       const float bb0 = cs_ * b0 - sn * b1, bb1 = sn * b0 + cs_ * b1;
-      uint32_t hi, lo;
       if (!bwd) {
-        split2(we * bb0, we * bb1, hi, lo);
-        st32(sm.Gh, off2(r, n), hi);
-        st32(sm.Gl, off2(r, n), lo);
+        split2(we * bb0, we * bb1, bh_[k], bl_[k]);
       } else {
-        split2(bb0, bb1, hi, lo);
-        st32(sm.Bh, off2(r, n), hi);
-        st32(sm.Bl, off2(r, n), lo);
+        split2(bb0, bb1, bh_[k], bl_[k]);
         const float c0 = craw[2 * k], c1 = craw[2 * k + 1];
-        split2(cs_ * c0 - sn * c1, sn * c0 + cs_ * c1, hi, lo);
-        st32(sm.Ch, off2(r, n), hi);
-        st32(sm.Cl, off2(r, n), lo);
+        split2(cs_ * c0 - sn * c1, sn * c0 + cs_ * c1, ch_[k], cl_[k]);
+      }
+    }
+    uint8_t* th_ = bwd ? sm.Bh : sm.Gh;
+    uint8_t* tl_ = bwd ? sm.Bl : sm.Gl;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const uint32_t o = off2(r, 16 * sg + 8 * half);  // a 16-byte chunk of 8 columns
+      st128(th_, o, bh_ + 4 * half);
+      st128(tl_, o, bl_ + 4 * half);
+      if (bwd) {
+        st128(sm.Ch, o, ch_ + 4 * half);
+        st128(sm.Cl, o, cl_ + 4 * half);
       }
     }
     if (bwd) {
       const float e = sm.ecs[r];
+      uint32_t eh[4], el[4], xh[4], xl[4];
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        const int p = 8 * sg + 2 * q;
-        uint32_t hi, lo;
-        split2(e * yf8[2 * q], e * yf8[2 * q + 1], hi, lo);
-        st32(sm.EYh, off1(r, p), hi);
-        st32(sm.EYl, off1(r, p), lo);
-        split2(we * xf8[2 * q], we * xf8[2 * q + 1], hi, lo);
-        st32(sm.WXh, off1(r, p), hi);
-        st32(sm.WXl, off1(r, p), lo);
+        split2(e * yf8[2 * q], e * yf8[2 * q + 1], eh[q], el[q]);
+        split2(we * xf8[2 * q], we * xf8[2 * q + 1], xh[q], xl[q]);
       }
+      const uint32_t o = off1(r, 8 * sg);
+      st128(sm.EYh, o, eh);
+      st128(sm.EYl, o, el);
+      st128(sm.WXh, o, xh);
+      st128(sm.WXl, o, xl);
     }
   };
-  // a (p, n) tile pair from the thread's 16 values (rows 16 q4 + j, column nrow)
-  auto store_pn = [&](uint8_t* hi_t, uint8_t* lo_t, const float* v) {
+  // an (n, p) tile pair from the thread's 16 values (row nrow, columns 16 q4 ..)
+  auto store_np = [&](uint8_t* hi_t, uint8_t* lo_t, const float* v) {
+    uint32_t hv[8], lv[8];
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      const bf16 hv = __float2bfloat16_rn(v[j]);
-      *reinterpret_cast<bf16*>(hi_t + off2(16 * q4 + j, nrow)) = hv;
-      *reinterpret_cast<bf16*>(lo_t + off2(16 * q4 + j, nrow)) =
-          __float2bfloat16_rn(v[j] - __bfloat162float(hv));
+    for (int q = 0; q < 8; ++q) split2(v[2 * q], v[2 * q + 1], hv[q], lv[q]);
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const uint32_t o = off1(nrow, 16 * q4 + 8 * half);
+      st128(hi_t, o, hv + 4 * half);
+      st128(lo_t, o, lv + 4 * half);
     }
   };
 
@@ -490,7 +503,7 @@ __global__ void __launch_bounds__(kT, 1) bwd_tc_kernel(BwdArgs a, ChunkWs ws) {
       *reinterpret_cast<uint4*>(sm.X + off1(0, 8 * sg)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
       *reinterpret_cast<uint4*>(sm.Xl + off1(0, 8 * sg)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
     }
-    store_pn(sm.Hh, sm.Hl, f.hp);
+    store_np(sm.Hh, sm.Hl, f.hp);
     if (tid < kQ) {
       sm.cs[tid] = f.sc[0];  // the raw logdecay until chunk_scalars
       sm.ga[tid] = f.sc[1];
@@ -551,7 +564,7 @@ __global__ void __launch_bounds__(kT, 1) bwd_tc_kernel(BwdArgs a, ChunkWs ws) {
   float greg[16];  // g = dL/dh_end, rows nrow, columns 16 q4 + j
 #pragma unroll
   for (int j = 0; j < 16; ++j) greg[j] = a.dhT ? a.dhT[(bh * kN + nrow) * kP + 16 * q4 + j] : 0.f;
-  store_pn(sm.Gh, sm.Gl, greg);
+  store_np(sm.Gh, sm.Gl, greg);
   if (tid < kNH) sm.run[tid] = 0.f;
   if (tid < kP) sm.cdx[0][tid] = sm.cdx[1][tid] = 0.f;
   if (tid < kN) sm.cdb[0][tid] = sm.cdb[1][tid] = 0.f;
@@ -581,10 +594,10 @@ __global__ void __launch_bounds__(kT, 1) bwd_tc_kernel(BwdArgs a, ChunkWs ws) {
       if (c == 0 && has_xl)
         for (int j = 0; j < 4; ++j) tc5::mma_bf16(tmem + kColE, dk1(aY, j), dk1(aXl, j), kI64, true);
       tc5::commit(&sm.mbar[0]);                                          // G, E
-      mma_split(tmem + kColY, aCh, aCl, aHh, aHl, kI64, 8, false, false, K2, K2);    // Cbar h_prev
+      mma_split(tmem + kColY, aCh, aCl, aHh, aHl, kI64kmn, 8, false, false, K2, MN);  // Cbar h_prev
       mma_split(tmem + kColDH, aCh, aCl, aEh, aEl, kI128S, 4, false, true, MN, MN); // Cbar^T e^cs dY
-      mma_split(tmem + kColDB, aWh, aWl, aGh, aGl, kIN128, 4, false, true, K1, MN); // (W_end X) g^T
-      mma_split(tmem + kColDC, aEh, aEl, aHh, aHl, kIN128, 4, false, true, K1, MN); // e^cs dY h_prev^T
+      mma_split(tmem + kColDB, aWh, aWl, aGh, aGl, kIN128k, 4, false, true, K1, K1); // (W_end X) g^T
+      mma_split(tmem + kColDC, aEh, aEl, aHh, aHl, kIN128k, 4, false, true, K1, K1); // e^cs dY h_prev^T
       tc5::commit(&sm.mbar[1]);
     }
 
@@ -705,7 +718,7 @@ __global__ void __launch_bounds__(kT, 1) bwd_tc_kernel(BwdArgs a, ChunkWs ws) {
 
     // -- stage 2
     if (tid == 0) {
-      mma_split(tmem + kColG, aBh, aBl, aGh, aGl, kI64, 8, false, false, K2, K2);  // Bbar g
+      mma_split(tmem + kColG, aBh, aBl, aGh, aGl, kI64kmn, 8, false, false, K2, MN);  // Bbar g
       for (int j = 0; j < 4; ++j) tc5::mma_bf16(tmem + kColE, dmn(aEh, j), dmn(aY, j), kI64mn, j > 0);
       for (int j = 0; j < 4; ++j) tc5::mma_bf16(tmem + kColE, dmn(aEl, j), dmn(aY, j), kI64mn, true);
       mma_split(tmem + kColDC, aWh, aWl, aBh, aBl, kIN128, 4, true, true, K1, MN);    // += WE Bbar
@@ -806,7 +819,7 @@ __global__ void __launch_bounds__(kT, 1) bwd_tc_kernel(BwdArgs a, ChunkWs ws) {
     __syncthreads();  // the tiles of X, dY, theta and B, C are read: fetch the next chunk
     tc5::fence_after_sync();
     if (c > 0) fetch_chunk(c - 1, f);
-    store_pn(sm.Gh, sm.Gl, greg);  // the next (earlier) chunk's g
+    store_np(sm.Gh, sm.Gl, greg);  // the next (earlier) chunk's g
     __syncthreads();
 
     // -- the scalar chain: decay sums -> cv -> gamma, beta, logdecay (warp 0)

@@ -300,16 +300,20 @@ __global__ void __launch_bounds__(kT, 1) bwd_tc_kernel(BwdArgs a, ChunkWs ws) {
       *reinterpret_cast<uint4*>(sm.Xl + off1(0, 8 * sg)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
     }
     if (tid < kQ) {
-      sm.cs[tid] = sc1[0];  // the raw logdecay until chunk_scalars
+      sm.cs[tid] = sc1[0];  // the raw logdecay until scalars_angles
       sm.ga[tid] = sc1[1];
       sm.be[tid] = sc1[2];
     }
   };
 
-  // ---- chunk scalars: cs, alpha, exp(cs), cv, W_end --------------------------
-  auto chunk_scalars = [&]() {
+  // ---- chunk scalars (cs, alpha, exp(cs), cv, W_end: warp 0 alone, rows lane and
+  // lane + 32, neighbours by shuffle) and the angles phi(r, i) = phi0[i] +
+  // sum_{k <= r} theta(k, i) (all threads, in 8-row segments); two barriers
+  auto scalars_angles = [&]() {
     if (warp == 0) {
-      const float l0 = sm.cs[lane], l1 = sm.cs[lane + 32];
+      const float l0 = sm.cs[lane], l1 = sm.cs[lane + 32];  // raw logdecay
+      const float g0 = sm.ga[lane], g1 = sm.ga[lane + 32];
+      const float e0 = sm.be[lane], e1 = sm.be[lane + 32];
       float s0 = l0, s1 = l1;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -321,27 +325,27 @@ __global__ void __launch_bounds__(kT, 1) bwd_tc_kernel(BwdArgs a, ChunkWs ws) {
         }
       }
       s1 += __shfl_sync(0xffffffffu, s0, 31);
-      sm.al[lane] = expf(l0);
-      sm.al[lane + 32] = expf(l1);
+      const float a0 = expf(l0), a1 = expf(l1);
+      // the row after: lane + 1 (row 32 for lane 31), lane + 33
+      const float a0n = __shfl_down_sync(0xffffffffu, a0, 1), a1n = __shfl_down_sync(0xffffffffu, a1, 1);
+      const float e0n = __shfl_down_sync(0xffffffffu, e0, 1), e1n = __shfl_down_sync(0xffffffffu, e1, 1);
+      const float s0n = __shfl_down_sync(0xffffffffu, s0, 1), s1n = __shfl_down_sync(0xffffffffu, s1, 1);
+      const float a32 = __shfl_sync(0xffffffffu, a1, 0), e32 = __shfl_sync(0xffffffffu, e1, 0);
+      const float s32 = __shfl_sync(0xffffffffu, s1, 0), s63 = __shfl_sync(0xffffffffu, s1, 31);
+      const bool last = lane == 31;
+      const float cv0 = g0 * (last ? a32 : a0n) + (last ? e32 : e0n);
+      const float cv1 = last ? 0.f : g1 * a1n + e1n;
       sm.cs[lane] = s0;
       sm.cs[lane + 32] = s1;
+      sm.al[lane] = a0;
+      sm.al[lane + 32] = a1;
+      sm.ecs[lane] = expf(s0);
+      sm.ecs[lane + 32] = expf(s1);
+      sm.cv[lane] = cv0;
+      sm.cv[lane + 32] = cv1;
+      sm.wend[lane] = expf(s63 - (last ? s32 : s0n)) * cv0;
+      sm.wend[lane + 32] = last ? g1 : expf(s63 - s1n) * cv1;
     }
-    __syncthreads();
-    if (tid < kQ) {
-      const int r = tid;
-      sm.ecs[r] = expf(sm.cs[r]);
-      sm.cv[r] = r < kQ - 1 ? sm.ga[r] * sm.al[r + 1] + sm.be[r + 1] : 0.f;
-    }
-    __syncthreads();
-    if (tid < kQ) {
-      const int u = tid;
-      sm.wend[u] = u < kQ - 1 ? expf(sm.cs[kQ - 1] - sm.cs[u + 1]) * sm.cv[u] : sm.ga[kQ - 1];
-    }
-    __syncthreads();
-  };
-
-  // ---- angles phi(r, i) = phi0[i] + sum_{k <= r} theta(k, i), in 8-row segments
-  auto angles = [&]() {
     const int i = tid & 63, grp = tid >> 6;
     float run_ = 0.f;
 #pragma unroll
@@ -505,7 +509,7 @@ __global__ void __launch_bounds__(kT, 1) bwd_tc_kernel(BwdArgs a, ChunkWs ws) {
     }
     store_np(sm.Hh, sm.Hl, f.hp);
     if (tid < kQ) {
-      sm.cs[tid] = f.sc[0];  // the raw logdecay until chunk_scalars
+      sm.cs[tid] = f.sc[0];  // the raw logdecay until scalars_angles
       sm.ga[tid] = f.sc[1];
       sm.be[tid] = f.sc[2];
       if (tid < kNH) sm.phi0[tid] = f.ph;
@@ -532,8 +536,7 @@ __global__ void __launch_bounds__(kT, 1) bwd_tc_kernel(BwdArgs a, ChunkWs ws) {
     if (tid < kNH) ph_ws[(int64_t)c * kNH + tid] = sm.phi0[tid];
     commit1(c);
     __syncthreads();
-    chunk_scalars();
-    angles();
+    scalars_angles();
     const float nphi = tid < kNH ? wrap_angle(sm.Vt[(kQ - 1) * kNH + tid]) : 0.f;
     rotate(false);
     mma_fence_sync();  // the rotation has read theta and B: the next ones may land
@@ -582,8 +585,7 @@ __global__ void __launch_bounds__(kT, 1) bwd_tc_kernel(BwdArgs a, ChunkWs ws) {
     for (int j = 0; j < 16; ++j) hpr[j] = f.hp[j];
     commit_chunk(c, f);
     __syncthreads();
-    chunk_scalars();
-    angles();
+    scalars_angles();
     rotate(true);
     mma_fence_sync();
 

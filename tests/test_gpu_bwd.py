@@ -282,3 +282,14 @@ def test_bwd_full_siso_workload_fp32_kernel_one_batch_row():
     for k in ("dX", "dlogdecay", "dbeta", "dgamma", "dB", "dC", "dtheta", "dh0"):
         g = np64(got[k][bi:bi + 1])
         assert rel_max_err(g, ref[k]) <= TOL, (k, rel_max_err(g, ref[k]))
+
+
+@pytest.mark.parametrize("P,N", [(64, 256), (256, 64)])
+def test_bwd_sequential_maximum_state(P, N):
+    # the largest states of the sequential backward (N * P = 16384)
+    w = WORKLOADS["tiny"].with_(batch=1, seqlen=19, nheads=2, ngroups=1, headdim=P, dstate=N,
+                                seed=17 + P)
+    inp = with_cache_inputs(make_inputs(w), seed=N)
+    dY, dhT = upstream(inp, 90 + P)
+    got, ref = run_both(inp, dY, dhT)
+    check_all(got, ref)

@@ -156,3 +156,29 @@ def test_decode_workload_prefill_then_1000_steps_sampled():
         assert angle_err(np64(cache["angle"][bi:bi + 1][:, heads]), ref["angleT"]) <= 1e-4
         np.testing.assert_array_equal(np64(cache["x_prev"][bi:bi + 1][:, heads]), ref["xprevT"])
         np.testing.assert_array_equal(np64(cache["b_prev"][bi:bi + 1]), ref["bprevT"])
+
+
+# The largest state the sequential kernels keep in one CTA: N * P = 16384 with
+# N, P <= 256 (the three corners), forward with cache in and out, then decode
+# steps from the forward's cache, each against the oracle.
+@pytest.mark.parametrize("P,N", [(64, 256), (256, 64), (128, 128)])
+def test_general_path_maximum_state(P, N):
+    w = WORKLOADS["tiny"].with_(batch=1, seqlen=21, nheads=2, ngroups=1, headdim=P, dstate=N,
+                                seed=91 + P)
+    inp = with_cache_inputs(make_inputs(w), seed=P + N)
+    ref = oracle.oracle_fwd(**inp)
+    got = gpu_fwd(inp, want_cache=True)
+    assert rel_max_err(got["Y"], ref["Y"]) <= TOL_F32
+    assert rel_max_err(got["hT"], ref["hT"]) <= TOL_F32
+    assert angle_err(got["angleT"], ref["angleT"]) <= 1e-5
+    yg, yo, cg, co = _steps_gpu_and_oracle(w, 4)
+    assert rel_max_err(yg, yo) <= TOL_F32
+    assert rel_max_err(cg["ssm"], co["ssm"]) <= TOL_F32
+
+
+def test_state_over_the_limit_is_refused():
+    # N * P = 16640 > 16384: the sequential kernels cannot hold it
+    w = WORKLOADS["tiny"].with_(batch=1, seqlen=3, nheads=1, headdim=65, dstate=256, seed=3)
+    inp = make_inputs(w)
+    with pytest.raises(m3.M3SSDError):
+        gpu_fwd(inp)

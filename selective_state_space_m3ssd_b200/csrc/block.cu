@@ -150,26 +150,44 @@ __global__ void __launch_bounds__(kPrepThreads) block_prep_kernel(PrepArgs a) {
 // The same with 16-byte accesses, for shapes whose row parts are multiples of
 // four floats and eight bf16 (H P % 8, G N % 4, H % 4, N % 8).
 __global__ void __launch_bounds__(kPrepThreads) block_prep_vec_kernel(PrepArgs a) {
-  extern __shared__ float sh[];
+  // No barrier: the warp that sums a group's squares also writes its normed
+  // values, and every thread that scales theta recomputes its head's Delta.
   const int64_t tok = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int H = (int)a.H, P = (int)a.P, N = (int)a.N, G = (int)a.G, NH = N / 2;
   const int HP = H * P, GN = G * N;
   const int oB = 2 * HP, oC = oB + GN, odt = oC + GN, olam = odt + H, oth = olam + H;
   const __nv_bfloat16* row = a.zx + tok * a.width;
-  float* inv = sh;
-  float* delta = sh + 2 * G;
 
-  for (int j = warp; j < 2 * G; j += kPrepThreads / 32) {
-    const __nv_bfloat16* v = row + (j < G ? oB + j * N : oC + (j - G) * N);
+  for (int k = tid; k < HP / 8; k += kPrepThreads)
+    *reinterpret_cast<uint4*>(a.X + tok * HP + 8 * k) =
+        *reinterpret_cast<const uint4*>(row + HP + 8 * k);
+  for (int j = warp; j < 2 * G; j += kPrepThreads / 32) {  // N <= 256: two float4 a lane
+    const int off = j < G ? oB + j * N : oC + (j - G) * N;
+    const float* w = j < G ? a.Bw : a.Cw;
+    __nv_bfloat16* dst = (j < G ? a.B + (tok * G + j) * N : a.C + (tok * G + j - G) * N);
+    float4 q[2];
     float ss = 0.f;
-    for (int n = 4 * lane; n < N; n += 128) {
-      const float4 q = ld4_bf16(v + n);
-      ss = fmaf(q.x, q.x, fmaf(q.y, q.y, fmaf(q.z, q.z, fmaf(q.w, q.w, ss))));
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
+      const int n = 4 * lane + 128 * s;
+      q[s] = n < N ? ld4_bf16(row + off + n) : make_float4(0.f, 0.f, 0.f, 0.f);
+      ss = fmaf(q[s].x, q[s].x, fmaf(q[s].y, q[s].y, fmaf(q[s].z, q[s].z, fmaf(q[s].w, q[s].w, ss))));
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    if (lane == 0) inv[j] = 1.f / sqrtf(ss / (float)N + a.eps);
+    const float inv = 1.f / sqrtf(ss / (float)N + a.eps);
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
+      const int n = 4 * lane + 128 * s;
+      if (n < N) {
+        const float4 wv = *reinterpret_cast<const float4*>(w + n);
+        uint2 o;
+        o.x = pack2_bf16(q[s].x * inv * wv.x, q[s].y * inv * wv.y);
+        o.y = pack2_bf16(q[s].z * inv * wv.z, q[s].w * inv * wv.w);
+        *reinterpret_cast<uint2*>(dst + n) = o;
+      }
+    }
   }
   for (int h = tid; h < H; h += kPrepThreads) {
     const float dl = softplus_f(bf(row[odt + h]) + a.dt_bias[h]);
@@ -178,30 +196,10 @@ __global__ void __launch_bounds__(kPrepThreads) block_prep_vec_kernel(PrepArgs a
     a.ld[tok * H + h] = lg;
     a.ga[tok * H + h] = lam * dl;
     a.be[tok * H + h] = (1.f - lam) * dl * expf(lg);
-    delta[h] = dl;
-  }
-  for (int k = tid; k < HP / 8; k += kPrepThreads)
-    *reinterpret_cast<uint4*>(a.X + tok * HP + 8 * k) =
-        *reinterpret_cast<const uint4*>(row + HP + 8 * k);
-  __syncthreads();
-  const int NQ = N / 4;
-  for (int k = tid; k < G * NQ; k += kPrepThreads) {
-    const int g = k / NQ, n = 4 * (k - g * NQ);
-    const float4 bv = ld4_bf16(row + oB + g * N + n);
-    const float4 cv = ld4_bf16(row + oC + g * N + n);
-    const float4 bw = *reinterpret_cast<const float4*>(a.Bw + n);
-    const float4 cw = *reinterpret_cast<const float4*>(a.Cw + n);
-    const float ib = inv[g], ic = inv[G + g];
-    uint2 ob, oc;
-    ob.x = pack2_bf16(bv.x * ib * bw.x, bv.y * ib * bw.y);
-    ob.y = pack2_bf16(bv.z * ib * bw.z, bv.w * ib * bw.w);
-    oc.x = pack2_bf16(cv.x * ic * cw.x, cv.y * ic * cw.y);
-    oc.y = pack2_bf16(cv.z * ic * cw.z, cv.w * ic * cw.w);
-    *reinterpret_cast<uint2*>(a.B + tok * G * N + g * N + n) = ob;
-    *reinterpret_cast<uint2*>(a.C + tok * G * N + g * N + n) = oc;
   }
   for (int k = tid; k < H * NH / 4; k += kPrepThreads) {
-    const float d = delta[(4 * k) / NH];
+    const int h = (4 * k) / NH;
+    const float d = softplus_f(bf(row[odt + h]) + a.dt_bias[h]);
     const float4 v = ld4_bf16(row + oth + 4 * k);
     *reinterpret_cast<float4*>(a.th + tok * H * NH + 4 * k) =
         make_float4(d * v.x, d * v.y, d * v.z, d * v.w);
@@ -354,7 +352,7 @@ m3ssd_status front(const m3ssd_block_dims* d, const m3ssd_block_weights* w, cons
   if (smem > 48 * 1024) return M3SSD_ERR_UNSUPPORTED;
   const bool w16 = aligned(a.Bw, 16) && aligned(a.Cw, 16);
   if (w16 && vec_shape(a.H, a.P, a.N, a.G, width))
-    block_prep_vec_kernel<<<(unsigned)M, kPrepThreads, smem, s>>>(a);
+    block_prep_vec_kernel<<<(unsigned)M, kPrepThreads, 0, s>>>(a);
   else
     block_prep_kernel<<<(unsigned)M, kPrepThreads, smem, s>>>(a);
   return cudaGetLastError() == cudaSuccess ? M3SSD_OK : M3SSD_ERR_CUDA;

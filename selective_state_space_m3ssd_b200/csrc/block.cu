@@ -77,6 +77,7 @@ struct PrepArgs {
   const float* Bbias;
   const float* Cbias;
   float eps;
+  bool write_x;  // copy x out of the rows (not when the scan reads it there)
   __nv_bfloat16* X;
   __nv_bfloat16* B;
   __nv_bfloat16* C;
@@ -136,7 +137,8 @@ __global__ void __launch_bounds__(kPrepThreads) block_prep_kernel(PrepArgs a) {
     a.be[tok * H + h] = (1.f - lam) * dl * expf(lg);
     delta[h] = dl;
   }
-  for (int k = tid; k < HP; k += kPrepThreads) a.X[tok * HP + k] = row[HP + k];
+  if (a.write_x)
+    for (int k = tid; k < HP; k += kPrepThreads) a.X[tok * HP + k] = row[HP + k];
   __syncthreads();
   for (int k = tid; k < G * N; k += kPrepThreads) {
     const int g = k / N, n = k - g * N;
@@ -159,9 +161,10 @@ __global__ void __launch_bounds__(kPrepThreads) block_prep_vec_kernel(PrepArgs a
   const int oB = 2 * HP, oC = oB + GN, odt = oC + GN, olam = odt + H, oth = olam + H;
   const __nv_bfloat16* row = a.zx + tok * a.width;
 
-  for (int k = tid; k < HP / 8; k += kPrepThreads)
-    *reinterpret_cast<uint4*>(a.X + tok * HP + 8 * k) =
-        *reinterpret_cast<const uint4*>(row + HP + 8 * k);
+  if (a.write_x)
+    for (int k = tid; k < HP / 8; k += kPrepThreads)
+      *reinterpret_cast<uint4*>(a.X + tok * HP + 8 * k) =
+          *reinterpret_cast<const uint4*>(row + HP + 8 * k);
   for (int j = warp; j < 2 * G; j += kPrepThreads / 32) {  // N <= 256: two float4 a lane
     const int off = j < G ? oB + j * N : oC + (j - G) * N;
     const float* w = j < G ? a.Bw : a.Cw;
@@ -331,7 +334,7 @@ bool scan_shape_ok(const m3ssd_block_dims* d) {
 
 // in_proj, the prep kernel; returns the scan inputs' pointers through ws.
 m3ssd_status front(const m3ssd_block_dims* d, const m3ssd_block_weights* w, const void* u,
-                   int64_t M, char* base, const BlockWs& ws, cudaStream_t s) {
+                   int64_t M, char* base, const BlockWs& ws, bool write_x, cudaStream_t s) {
   const int64_t width = in_proj_width(d);
   if (!gemm_bf16(M, width, d->d_model, u, w->W_in, base + ws.zx, CUDA_R_16BF, base + ws.lt,
                  kLtWorkspace, s))
@@ -340,7 +343,7 @@ m3ssd_status front(const m3ssd_block_dims* d, const m3ssd_block_weights* w, cons
   a.M = M; a.H = d->nheads; a.P = d->headdim; a.N = d->dstate; a.G = d->ngroups; a.width = width;
   a.zx = reinterpret_cast<const __nv_bfloat16*>(base + ws.zx);
   a.dt_bias = w->dt_bias; a.A_log = w->A_log; a.Bw = w->B_norm_w; a.Cw = w->C_norm_w;
-  a.Bbias = w->B_bias; a.Cbias = w->C_bias; a.eps = w->eps;
+  a.Bbias = w->B_bias; a.Cbias = w->C_bias; a.eps = w->eps; a.write_x = write_x;
   a.X = reinterpret_cast<__nv_bfloat16*>(base + ws.x);
   a.B = reinterpret_cast<__nv_bfloat16*>(base + ws.B);
   a.C = reinterpret_cast<__nv_bfloat16*>(base + ws.C);
@@ -420,16 +423,16 @@ m3ssd_status m3ssd_block_fwd(const m3ssd_block_dims* dims, const m3ssd_block_wei
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const BlockWs ws = block_ws(dims, M > 0 ? M : dims->batch);
   char* base = static_cast<char*>(workspace);
-  if (M > 0) {
-    st = front(dims, w, u, M, base, ws, s);
-    if (st != M3SSD_OK) return st;
-  }
   // the scan, with the head biases of B and C applied inside it; the incoming
   // b_prev is copied first, so that the outgoing one may overwrite the same buffer
   FwdArgs a{};
   a.b = dims->batch; a.L = dims->seqlen; a.H = dims->nheads; a.P = dims->headdim;
   a.N = dims->dstate; a.G = dims->ngroups; a.chunk = 0; a.bf16 = true;
-  a.X = base + ws.x;
+  // the chunked scan reads x straight out of the bf16 in_proj rows (its tensor
+  // map takes the row stride); the sequential one reads prep's dense copy
+  const int64_t width = in_proj_width(dims);
+  a.X = reinterpret_cast<const __nv_bfloat16*>(base + ws.zx) + dims->nheads * dims->headdim;
+  a.x_tok_stride = width;
   a.logdecay = reinterpret_cast<const float*>(base + ws.ld);
   a.beta = reinterpret_cast<const float*>(base + ws.be);
   a.gamma = reinterpret_cast<const float*>(base + ws.ga);
@@ -457,6 +460,14 @@ m3ssd_status m3ssd_block_fwd(const m3ssd_block_dims* dims, const m3ssd_block_wei
     a.bprevT = cache_out->b_prev;
   }
   const bool chunked = fwd_chunk_supported(a);
+  if (!chunked) {
+    a.X = base + ws.x;
+    a.x_tok_stride = 0;
+  }
+  if (M > 0) {
+    st = front(dims, w, u, M, base, ws, !chunked, s);
+    if (st != M3SSD_OK) return st;
+  }
   if (!chunked && !scan_shape_ok(dims)) return M3SSD_ERR_UNSUPPORTED;
   const cudaError_t e = chunked ? launch_fwd_chunk(a, s) : launch_fwd_seq(a, s);
   if (e != cudaSuccess) {
@@ -490,7 +501,7 @@ m3ssd_status m3ssd_block_step(const m3ssd_block_dims* dims, const m3ssd_block_we
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const BlockWs ws = block_ws(&one, M);
   char* base = static_cast<char*>(workspace);
-  st = front(&one, w, u_t, M, base, ws, s);
+  st = front(&one, w, u_t, M, base, ws, true, s);
   if (st != M3SSD_OK) return st;
   StepArgs a{};
   a.b = M; a.H = dims->nheads; a.P = dims->headdim; a.N = dims->dstate; a.G = dims->ngroups;

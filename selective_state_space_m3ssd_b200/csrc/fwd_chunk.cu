@@ -245,7 +245,8 @@ __global__ void __launch_bounds__(kThreads, 2)
   const uint32_t aT = tc5::saddr(&sm.u.theta[0][0]);
 
   bf16* const Y_seq = Yg + (b * L * H + h) * PD;
-  const int64_t xstride_t = H * PD;  // X / Y elements per token
+  const int64_t xstride_t = H * PD;  // Y elements per token
+  const int64_t xtok = a.x_tok_stride ? a.x_tok_stride : H * PD;  // X elements per token
   // TMA issue (control thread): chunk c's rows start at token c*QT - 1
   const bool has_theta = a.theta != nullptr;  // ROT without theta: rotation by angle0 only
   const uint32_t chunk_bytes = (ROT && has_theta ? 16384u : 0u) + 2u * 16384u + 8192u;
@@ -674,7 +675,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (a.angleT && tid < NH)
       a.angleT[bh * NH + tid] = ROT ? sm.Phi[tid] : (a.angle0 ? a.angle0[bh * NH + tid] : 0.f);
     if (a.xprevT && tid < PD)
-      a.xprevT[bh * PD + tid] = __bfloat162float(Xg[((b * L + L - 1) * H + h) * PD + tid]);
+      a.xprevT[bh * PD + tid] = __bfloat162float(Xg[(b * L + L - 1) * xtok + h * PD + tid]);
     if (a.bprevT && h % (H / G) == 0 && tid < NS)
       a.bprevT[(b * G + g) * NS + tid] =
           __bfloat162float(Bg[((b * L + L - 1) * G + g) * NS + tid]);
@@ -698,13 +699,16 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// A 4-D map (d0 innermost, dense) with a box of d0-extent `box0` by 64 tokens.
+// A 4-D map (d0 innermost) with a box of d0-extent `box0` by 64 tokens; d2 (the
+// token axis) is `tok` elements apart (0: dense, d0 d1).
 bool encode_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t d0, uint64_t d1,
-                uint64_t d2, uint64_t d3, uint64_t esz, uint32_t box0, CUtensorMapSwizzle sw) {
+                uint64_t d2, uint64_t d3, uint64_t esz, uint32_t box0, CUtensorMapSwizzle sw,
+                uint64_t tok = 0) {
   PFN_cuTensorMapEncodeTiled_v12000 fn = tensor_map_encoder();
   if (!fn) return false;
   const cuuint64_t dims[4] = {d0, d1, d2, d3};
-  const cuuint64_t strides[3] = {d0 * esz, d0 * d1 * esz, d0 * d1 * d2 * esz};
+  const uint64_t ts = tok ? tok : d0 * d1;
+  const cuuint64_t strides[3] = {d0 * esz, ts * esz, ts * d2 * esz};
   const cuuint32_t box[4] = {box0, 1, (cuuint32_t)Q, 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
   return fn(m, dt, 4, const_cast<void*>(base), dims, strides, box, estr,
@@ -722,7 +726,7 @@ cudaError_t launch_variant(const FwdArgs& a, cudaStream_t s) {
             encode_map(&tm.C, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.C, NS, G, L, b, 2, 64,
                        CU_TENSOR_MAP_SWIZZLE_128B) &&
             encode_map(&tm.X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.X, PD, H, L, b, 2, 64,
-                       CU_TENSOR_MAP_SWIZZLE_128B);
+                       CU_TENSOR_MAP_SWIZZLE_128B, (uint64_t)a.x_tok_stride);
   if (ok && a.theta)
     ok = encode_map(&tm.theta, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.theta, NH, H, L, b, 4, NH,
                     CU_TENSOR_MAP_SWIZZLE_NONE);
@@ -741,6 +745,7 @@ bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
 bool fwd_chunk_supported(const FwdArgs& a) {
   return a.bf16 && a.N == NS && a.P == PD && a.L > 0 && (a.chunk == 0 || a.chunk == Q) &&
+         a.x_tok_stride % 8 == 0 && (a.x_tok_stride == 0 || a.x_tok_stride >= a.H * PD) &&
          al16(a.X) && al16(a.B) && al16(a.C) && al16(a.Y) && al16(a.theta) && al16(a.h0) &&
          al16(a.hT) && al16(a.logdecay) && al16(a.Bbias) && al16(a.Cbias);
 }

@@ -34,6 +34,10 @@ struct FwdArgs {
   // scan entry points leave them NULL.
   const float* Bbias;
   const float* Cbias;
+  // Elements between consecutive tokens of X (0: H P, a dense (b, L, H, P)
+  // tensor).  The block points X into its in_proj rows this way; only the
+  // chunked kernel takes a stride (a multiple of 8).
+  int64_t x_tok_stride;
 };
 
 struct StepArgs {

@@ -487,12 +487,12 @@ def bench_block(dev, rank, peaks: dict, steps: int = 5, warmup: int = 3):
     # peak or their operand bytes at HBM bandwidth, whichever is larger; the
     # prep, scan and gate kernels by the bytes they must move
     bw, pt = peaks["hbm_gbs"] * 1e9, peaks["bf16_tflops"] * 1e12
-    # (the in_proj output is bf16: prep reads all of it but z and x, the scan
-    # reads x there, the gate reads z)
+    # (the in_proj output is bf16: prep reads its B, C, dt and lam parts, the
+    # scan reads x and the raw angles there, the gate reads z)
     t_in = max(2.0 * M * dm * width / pt, (M * dm * 2 + width * dm * 2 + M * width * 2) / bw)
     t_out = max(2.0 * M * HP * dm / pt, (M * HP * 2 + dm * HP * 2 + M * dm * 2) / bw)
-    prep_b = M * ((width - 2 * HP) * 2 + 2 * G * N * 2 + 3 * H * 4 + H * (N // 2) * 4)
-    scan_b = M * (2 * HP * 2 + 3 * H * 4 + 2 * G * N * 2 + H * (N // 2) * 4)
+    prep_b = M * ((2 * G * N + 2 * H) * 2 + 2 * G * N * 2 + 3 * H * 4)
+    scan_b = M * (2 * HP * 2 + 3 * H * 4 + 2 * G * N * 2 + H * (N // 2) * 2)
     gate_b = M * HP * (2 + 2 + 2)
     t_lb = t_in + t_out + (prep_b + scan_b + gate_b) / bw
     return {"metric": "block Mtokens/s (fwd)", "value": M / (ms / 1e3) / 1e6, "unit": "Mtokens/s",

@@ -78,6 +78,7 @@ struct PrepArgs {
   const float* Cbias;
   float eps;
   bool write_x;  // copy x out of the rows (not when the scan reads it there)
+  bool write_th; // write theta_dt (not when the scan scales the raw angles itself)
   __nv_bfloat16* X;
   __nv_bfloat16* B;
   __nv_bfloat16* C;
@@ -145,8 +146,9 @@ __global__ void __launch_bounds__(kPrepThreads) block_prep_kernel(PrepArgs a) {
     a.B[tok * G * N + k] = __float2bfloat16_rn(bf(row[oB + k]) * inv[g] * a.Bw[n]);
     a.C[tok * G * N + k] = __float2bfloat16_rn(bf(row[oC + k]) * inv[G + g] * a.Cw[n]);
   }
-  for (int k = tid; k < H * NH; k += kPrepThreads)
-    a.th[tok * H * NH + k] = delta[k / NH] * bf(row[oth + k]);
+  if (a.write_th)
+    for (int k = tid; k < H * NH; k += kPrepThreads)
+      a.th[tok * H * NH + k] = delta[k / NH] * bf(row[oth + k]);
 }
 
 // The same with 16-byte accesses, for shapes whose row parts are multiples of
@@ -200,7 +202,7 @@ __global__ void __launch_bounds__(kPrepThreads) block_prep_vec_kernel(PrepArgs a
     a.ga[tok * H + h] = lam * dl;
     a.be[tok * H + h] = (1.f - lam) * dl * expf(lg);
   }
-  for (int k = tid; k < H * NH / 4; k += kPrepThreads) {
+  for (int k = tid; a.write_th && k < H * NH / 4; k += kPrepThreads) {
     const int h = (4 * k) / NH;
     const float d = softplus_f(bf(row[odt + h]) + a.dt_bias[h]);
     const float4 v = ld4_bf16(row + oth + 4 * k);
@@ -334,7 +336,8 @@ bool scan_shape_ok(const m3ssd_block_dims* d) {
 
 // in_proj, the prep kernel; returns the scan inputs' pointers through ws.
 m3ssd_status front(const m3ssd_block_dims* d, const m3ssd_block_weights* w, const void* u,
-                   int64_t M, char* base, const BlockWs& ws, bool write_x, cudaStream_t s) {
+                   int64_t M, char* base, const BlockWs& ws, bool write_x, bool write_th,
+                   cudaStream_t s) {
   const int64_t width = in_proj_width(d);
   if (!gemm_bf16(M, width, d->d_model, u, w->W_in, base + ws.zx, CUDA_R_16BF, base + ws.lt,
                  kLtWorkspace, s))
@@ -344,6 +347,7 @@ m3ssd_status front(const m3ssd_block_dims* d, const m3ssd_block_weights* w, cons
   a.zx = reinterpret_cast<const __nv_bfloat16*>(base + ws.zx);
   a.dt_bias = w->dt_bias; a.A_log = w->A_log; a.Bw = w->B_norm_w; a.Cw = w->C_norm_w;
   a.Bbias = w->B_bias; a.Cbias = w->C_bias; a.eps = w->eps; a.write_x = write_x;
+  a.write_th = write_th;
   a.X = reinterpret_cast<__nv_bfloat16*>(base + ws.x);
   a.B = reinterpret_cast<__nv_bfloat16*>(base + ws.B);
   a.C = reinterpret_cast<__nv_bfloat16*>(base + ws.C);
@@ -428,17 +432,22 @@ m3ssd_status m3ssd_block_fwd(const m3ssd_block_dims* dims, const m3ssd_block_wei
   FwdArgs a{};
   a.b = dims->batch; a.L = dims->seqlen; a.H = dims->nheads; a.P = dims->headdim;
   a.N = dims->dstate; a.G = dims->ngroups; a.chunk = 0; a.bf16 = true;
-  // the chunked scan reads x straight out of the bf16 in_proj rows (its tensor
-  // map takes the row stride); the sequential one reads prep's dense copy
-  const int64_t width = in_proj_width(dims);
-  a.X = reinterpret_cast<const __nv_bfloat16*>(base + ws.zx) + dims->nheads * dims->headdim;
+  // the chunked scan reads x and the raw angle projection straight out of the
+  // bf16 in_proj rows (its tensor maps take the row stride; it scales the angles
+  // by Delta = logdecay / A itself); the sequential one reads prep's dense x and
+  // theta_dt
+  const int64_t width = in_proj_width(dims), HP = dims->nheads * dims->headdim;
+  const auto* zx = reinterpret_cast<const __nv_bfloat16*>(base + ws.zx);
+  a.X = zx + HP;
   a.x_tok_stride = width;
+  a.theta16 = zx + 2 * HP + 2 * dims->ngroups * dims->dstate + 2 * dims->nheads;
+  a.theta16_tok_stride = width;
+  a.A_log = w->A_log;
   a.logdecay = reinterpret_cast<const float*>(base + ws.ld);
   a.beta = reinterpret_cast<const float*>(base + ws.be);
   a.gamma = reinterpret_cast<const float*>(base + ws.ga);
   a.B = base + ws.B;
   a.C = base + ws.C;
-  a.theta = reinterpret_cast<const float*>(base + ws.th);
   a.D = w->D;
   a.Bbias = w->B_bias;
   a.Cbias = w->C_bias;
@@ -463,9 +472,12 @@ m3ssd_status m3ssd_block_fwd(const m3ssd_block_dims* dims, const m3ssd_block_wei
   if (!chunked) {
     a.X = base + ws.x;
     a.x_tok_stride = 0;
+    a.theta16 = nullptr;
+    a.theta16_tok_stride = 0;
+    a.theta = reinterpret_cast<const float*>(base + ws.th);
   }
   if (M > 0) {
-    st = front(dims, w, u, M, base, ws, !chunked, s);
+    st = front(dims, w, u, M, base, ws, !chunked, !chunked, s);
     if (st != M3SSD_OK) return st;
   }
   if (!chunked && !scan_shape_ok(dims)) return M3SSD_ERR_UNSUPPORTED;
@@ -501,7 +513,7 @@ m3ssd_status m3ssd_block_step(const m3ssd_block_dims* dims, const m3ssd_block_we
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const BlockWs ws = block_ws(&one, M);
   char* base = static_cast<char*>(workspace);
-  st = front(&one, w, u_t, M, base, ws, true, s);
+  st = front(&one, w, u_t, M, base, ws, true, true, s);
   if (st != M3SSD_OK) return st;
   StepArgs a{};
   a.b = M; a.H = dims->nheads; a.P = dims->headdim; a.N = dims->dstate; a.G = dims->ngroups;

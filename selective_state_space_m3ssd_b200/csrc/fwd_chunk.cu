@@ -102,6 +102,7 @@ struct ChunkParams {
   float gam[Q];    // gamma_r
   float et[Q];     // exp(cs_t - cs_{8 floor(t/8)})
   float fs[224];   // exp(cs_{8k} - cs_{s+1}) cvec_s for s < 8k, at fs_index(k, s)
+  float dl[Q];     // Delta_r = logdecay_r / A (the raw-angle variant scales theta by it)
   float eE;        // exp(cs_63)
   float pad[3];
 };
@@ -155,7 +156,9 @@ __device__ __forceinline__ float ex2(float x) {
 // (rows lane and lane + 32; row 0 and rows past the end hold zeros).
 __device__ __forceinline__ void chunk_params(ChunkParams& P, const float (&pld)[2],
                                              const float (&pbe)[2], const float (&pga)[2],
-                                             int lane) {
+                                             int lane, float inv_a) {
+  P.dl[lane] = pld[0] * inv_a;
+  P.dl[lane + 32] = pld[1] * inv_a;
   // decay sums in log2 units
   float s0 = pld[0] * kLog2e, s1 = pld[1] * kLog2e;
 #pragma unroll
@@ -213,12 +216,13 @@ __device__ __forceinline__ void chunk_params(ChunkParams& P, const float (&pld)[
 // Tensor maps of the chunk inputs, built on the host for each launch.
 struct TmaMaps {
   CUtensorMap theta;  // fp32 (pair, head, token, batch), box 64 x 1 x 64 x 1, no swizzle
+                      // (bf16 in the raw-angle variant)
   CUtensorMap B;      // bf16 (n, group, token, batch), box 64 x 1 x 64 x 1, 128-byte swizzle
   CUtensorMap C;      // same as B
   CUtensorMap X;      // bf16 (p, head, token, batch), box 64 x 1 x 64 x 1, 128-byte swizzle
 };
 
-template <bool ROT, bool BIAS>
+template <bool ROT, bool BIAS, bool TH16>
 __global__ void __launch_bounds__(kThreads, 2)
     fwd_chunk_kernel(FwdArgs a, const __grid_constant__ TmaMaps tm) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -248,8 +252,10 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int64_t xstride_t = H * PD;  // Y elements per token
   const int64_t xtok = a.x_tok_stride ? a.x_tok_stride : H * PD;  // X elements per token
   // TMA issue (control thread): chunk c's rows start at token c*QT - 1
-  const bool has_theta = a.theta != nullptr;  // ROT without theta: rotation by angle0 only
-  const uint32_t chunk_bytes = (ROT && has_theta ? 16384u : 0u) + 2u * 16384u + 8192u;
+  const bool has_theta = (TH16 ? a.theta16 : static_cast<const void*>(a.theta)) != nullptr;  // ROT without theta: rotation by angle0 only
+  const uint32_t chunk_bytes = (ROT && has_theta ? (TH16 ? 8192u : 16384u) : 0u) + 2u * 16384u + 8192u;
+  // the raw-angle variant's 1 / A_h (Delta = logdecay / A_h)
+  const float inv_a = TH16 ? -1.f / expf(a.A_log[h]) : 0.f;
   auto tma_theta = [&](int c) {
     tc5::tma_load_4d(aT, &tm.theta, &sm.lmbar, 0, (int)h, c * QT - 1, (int)b);
   };
@@ -299,7 +305,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   }
   if (ctrl) {
     load_params(0);
-    chunk_params(sm.prm[0], pld, pbe, pga, lane);
+    chunk_params(sm.prm[0], pld, pbe, pga, lane, inv_a);
     if (nC > 1) load_params(1);
   }
   // row 0 of chunk 0 is the cache's previous token (the TMA zero-fills it; it is
@@ -381,7 +387,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         tma_x(c + 1);
       }
       if (c + 1 < nC) {
-        chunk_params(sm.prm[(c + 1) & 1], pld, pbe, pga, lane);
+        chunk_params(sm.prm[(c + 1) & 1], pld, pbe, pga, lane, inv_a);
         if (c + 2 < nC) load_params(c + 2);
       }
       // descriptors of the operand tiles: an offset inside a tile only adds
@@ -458,7 +464,15 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           if (warp > 0 || k > 0) {  // psi_0 = 0
-            const float2 th = *reinterpret_cast<const float2*>(&sm.u.theta[8 * warp + k][2 * lane]);
+            float2 th;
+            if (TH16) {
+              const uint32_t raw = reinterpret_cast<const uint32_t*>(&sm.u.theta[0][0])
+                  [(8 * warp + k) * (NH / 2) + lane];
+              const float dl = P.dl[8 * warp + k];
+              th = __fmul2_rn(unpack_bf16(raw), make_float2(dl, dl));
+            } else {
+              th = *reinterpret_cast<const float2*>(&sm.u.theta[8 * warp + k][2 * lane]);
+            }
             run = __fadd2_rn(run, th);
           }
           psi[k] = run;
@@ -716,7 +730,7 @@ bool encode_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool ROT, bool BIAS>
+template <bool ROT, bool BIAS, bool TH16>
 cudaError_t launch_variant(const FwdArgs& a, cudaStream_t s) {
   TmaMaps tm;
   memset(&tm, 0, sizeof(tm));
@@ -727,15 +741,18 @@ cudaError_t launch_variant(const FwdArgs& a, cudaStream_t s) {
                        CU_TENSOR_MAP_SWIZZLE_128B) &&
             encode_map(&tm.X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.X, PD, H, L, b, 2, 64,
                        CU_TENSOR_MAP_SWIZZLE_128B, (uint64_t)a.x_tok_stride);
-  if (ok && a.theta)
+  if (ok && TH16 && a.theta16)
+    ok = encode_map(&tm.theta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.theta16, NH, H, L, b, 2, NH,
+                    CU_TENSOR_MAP_SWIZZLE_NONE, (uint64_t)a.theta16_tok_stride);
+  else if (ok && a.theta)
     ok = encode_map(&tm.theta, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.theta, NH, H, L, b, 4, NH,
                     CU_TENSOR_MAP_SWIZZLE_NONE);
   if (!ok) return cudaErrorInvalidValue;
   const size_t smem = sizeof(Smem) + 1024;
-  cudaError_t e = cudaFuncSetAttribute(fwd_chunk_kernel<ROT, BIAS>,
+  cudaError_t e = cudaFuncSetAttribute(fwd_chunk_kernel<ROT, BIAS, TH16>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  fwd_chunk_kernel<ROT, BIAS><<<(unsigned)(a.b * a.H), kThreads, smem, s>>>(a, tm);
+  fwd_chunk_kernel<ROT, BIAS, TH16><<<(unsigned)(a.b * a.H), kThreads, smem, s>>>(a, tm);
   return cudaGetLastError();
 }
 
@@ -746,6 +763,8 @@ bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 bool fwd_chunk_supported(const FwdArgs& a) {
   return a.bf16 && a.N == NS && a.P == PD && a.L > 0 && (a.chunk == 0 || a.chunk == Q) &&
          a.x_tok_stride % 8 == 0 && (a.x_tok_stride == 0 || a.x_tok_stride >= a.H * PD) &&
+         (a.theta16 == nullptr ||
+          (al16(a.theta16) && a.theta16_tok_stride % 8 == 0 && a.theta16_tok_stride >= a.H * NH)) &&
          al16(a.X) && al16(a.B) && al16(a.C) && al16(a.Y) && al16(a.theta) && al16(a.h0) &&
          al16(a.hT) && al16(a.logdecay) && al16(a.Bbias) && al16(a.Cbias);
 }
@@ -754,9 +773,13 @@ cudaError_t launch_fwd_chunk(const FwdArgs& a, cudaStream_t s) {
   if (a.b * a.H == 0) return cudaSuccess;
   // the rotation phase also applies the head biases of B and C (its own variant,
   // so that the plain scan's kernel carries none of it)
-  if (a.Bbias != nullptr || a.Cbias != nullptr) return launch_variant<true, true>(a, s);
-  if (a.theta != nullptr || a.angle0 != nullptr) return launch_variant<true, false>(a, s);
-  return launch_variant<false, false>(a, s);
+  if (a.theta16 != nullptr) {  // the block's raw angle projection (biases alongside)
+    if (a.theta != nullptr || a.A_log == nullptr) return cudaErrorInvalidValue;
+    return launch_variant<true, true, true>(a, s);
+  }
+  if (a.Bbias != nullptr || a.Cbias != nullptr) return launch_variant<true, true, false>(a, s);
+  if (a.theta != nullptr || a.angle0 != nullptr) return launch_variant<true, false, false>(a, s);
+  return launch_variant<false, false, false>(a, s);
 }
 
 cudaError_t read_and_clear_wait_timeouts(unsigned int* count) {

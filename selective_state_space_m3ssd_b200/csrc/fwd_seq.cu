@@ -144,7 +144,8 @@ __global__ void __launch_bounds__(kThreads) fwd_seq_kernel(FwdArgs a) {
 }  // namespace
 
 cudaError_t launch_fwd_seq(const FwdArgs& a, cudaStream_t s) {
-  if (a.x_tok_stride != 0 && a.x_tok_stride != a.H * a.P) return cudaErrorInvalidValue;
+  if ((a.x_tok_stride != 0 && a.x_tok_stride != a.H * a.P) || a.theta16 != nullptr)
+    return cudaErrorInvalidValue;
   const int NG = kThreads / (int)a.P;
   const size_t smem =
       sizeof(float) * (size_t)(a.N * a.P + 3 * a.N + 2 * a.P + a.N / 2 + NG * a.P + 4);

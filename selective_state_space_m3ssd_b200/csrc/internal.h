@@ -38,6 +38,12 @@ struct FwdArgs {
   // tensor).  The block points X into its in_proj rows this way; only the
   // chunked kernel takes a stride (a multiple of 8).
   int64_t x_tok_stride;
+  // The block's raw angle projection instead of theta (chunked kernel only):
+  // theta(t, h, i) = Delta(t, h) theta16[t * theta16_tok_stride + h N/2 + i]
+  // (bf16), with Delta = logdecay / -exp(A_log[h]) recovered from logdecay.
+  const void* theta16;
+  int64_t theta16_tok_stride;
+  const float* A_log;
 };
 
 struct StepArgs {

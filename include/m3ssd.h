@@ -335,6 +335,22 @@ m3ssd_status m3ssd_block_fwd(const m3ssd_block_dims* dims, const m3ssd_block_wei
                              size_t workspace_bytes, void* stream);
 
 /*
+ * m3ssd_block_fwd once more, choosing the cuBLASLt algorithm of each of its
+ * projections on the way: for a projection shape not seen before, each of up
+ * to 8 heuristic candidates is timed on these operands (one warm-up run, then
+ * the best of three) and the fastest is kept for the process; later
+ * m3ssd_block_fwd and m3ssd_block_step calls of the same shapes use it
+ * (without a tuned choice they take cuBLASLt's first heuristic).  No page
+ * counterpart; a convenience of this library.  Arguments and results as
+ * m3ssd_block_fwd without caches.  Unlike every other entry point it
+ * synchronises the stream while timing, so it must not be captured in a CUDA
+ * graph; it is not meant to run concurrently with itself.
+ */
+m3ssd_status m3ssd_block_tune(const m3ssd_block_dims* dims, const m3ssd_block_weights* w,
+                              const void* u, void* out, void* workspace, size_t workspace_bytes,
+                              void* stream);
+
+/*
  * One decode step of the block (Mamba3SisoBlock.step): u_t, out_t (b, d_model)
  * bf16; cache (required) is advanced in place.  workspace as for
  * m3ssd_block_fwd with seqlen = 1.  Capturable in a CUDA graph.

@@ -118,6 +118,9 @@ def load(path: str | None = None):
         lib.m3ssd_block_step.argtypes = [ctypes.POINTER(BlockDims), ctypes.POINTER(BlockWeights),
                                          vp, vp, ctypes.POINTER(Cache), vp, sz, vp]
         lib.m3ssd_block_step.restype = ctypes.c_int
+        lib.m3ssd_block_tune.argtypes = [ctypes.POINTER(BlockDims), ctypes.POINTER(BlockWeights),
+                                         vp, vp, vp, sz, vp]
+        lib.m3ssd_block_tune.restype = ctypes.c_int
         lib.m3ssd_status_string.argtypes = [ctypes.c_int]
         lib.m3ssd_status_string.restype = ctypes.c_char_p
         lib.m3ssd_abi_version.argtypes = []
@@ -546,6 +549,25 @@ def block_fwd(u, wts: dict, *, cache_in=None, cache_out=None, out=None, workspac
                                 None if co is None else ctypes.byref(co), _ptr(workspace),
                                 workspace.numel(), _stream_handle(dev))
     _check(st, "m3ssd_block_fwd")
+    return out
+
+
+def block_tune(u, wts: dict, *, out=None, workspace=None):
+    """``m3ssd_block_tune``: one block forward that times cuBLASLt's candidate
+    algorithms for its two projections and keeps the fastest for later calls of
+    the same shapes (synchronises; not for graph capture)."""
+    import torch
+    b, L, dm = u.shape
+    dims, w, _ = _block_args(u, wts, L)
+    dev = u.device
+    out = torch.empty_like(u) if out is None else out
+    _need(out, "out", torch.bfloat16, (b, L, dm), dev)
+    need = block_workspace_size(dims)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    st = load().m3ssd_block_tune(ctypes.byref(dims), ctypes.byref(w), _ptr(u), _ptr(out),
+                                 _ptr(workspace), workspace.numel(), _stream_handle(dev))
+    _check(st, "m3ssd_block_tune")
     return out
 
 

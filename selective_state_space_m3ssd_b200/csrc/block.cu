@@ -18,6 +18,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <map>
 #include <mutex>
 
 #include "../../include/m3ssd.h"
@@ -257,6 +258,82 @@ cublasLtHandle_t lt_handle() {
   return h;
 }
 
+// The algorithm for one GEMM shape: the one m3ssd_block_tune measured for it
+// if any, else cuBLASLt's first heuristic.  Tuning (only inside
+// m3ssd_block_tune, which synchronises) times each of up to 8 heuristic
+// candidates on the call's own operands (one warm-up run, then the best of
+// three) and keeps the fastest for the process.
+thread_local bool g_tune = false;
+struct AlgoKey {
+  int64_t M, N, K;
+  int dt;
+  bool operator<(const AlgoKey& o) const {
+    return M != o.M ? M < o.M : N != o.N ? N < o.N : K != o.K ? K < o.K : dt < o.dt;
+  }
+};
+
+bool pick_algo(cublasLtHandle_t h, cublasLtMatmulDesc_t op, cublasLtMatrixLayout_t la,
+               cublasLtMatrixLayout_t lb, cublasLtMatrixLayout_t lc,
+               cublasLtMatmulPreference_t pref, int64_t M, int64_t Nout, int64_t K,
+               cudaDataType_t dt, const void* A, const void* W, void* D, void* ws,
+               size_t ws_bytes, cudaStream_t s, cublasLtMatmulAlgo_t* out) {
+  static std::mutex mu;
+  static std::map<AlgoKey, cublasLtMatmulAlgo_t> cache;
+  const AlgoKey key{M, Nout, K, (int)dt};
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = cache.find(key);
+    if (it != cache.end()) {
+      *out = it->second;
+      return true;
+    }
+  }
+  cublasLtMatmulHeuristicResult_t res[8];
+  int found = 0;
+  if (cublasLtMatmulAlgoGetHeuristic(h, op, la, lb, lc, lc, pref, 8, res, &found) !=
+          CUBLAS_STATUS_SUCCESS ||
+      found == 0)
+    return false;
+  int best = 0;
+  if (g_tune && found > 1) {
+    cudaEvent_t e0 = nullptr, e1 = nullptr;
+    if (cudaEventCreate(&e0) == cudaSuccess && cudaEventCreate(&e1) == cudaSuccess) {
+      const float alpha = 1.f, beta = 0.f;
+      float best_ms = 0.f;
+      for (int i = 0; i < found; ++i) {
+        if (res[i].state != CUBLAS_STATUS_SUCCESS) continue;
+        float ms_i = -1.f;
+        for (int rep = 0; rep < 4; ++rep) {  // the first run warms up
+          cudaEventRecord(e0, s);
+          const bool run = cublasLtMatmul(h, op, &alpha, W, la, A, lb, &beta, D, lc, D, lc,
+                                          &res[i].algo, ws, ws_bytes, s) == CUBLAS_STATUS_SUCCESS;
+          cudaEventRecord(e1, s);
+          float t = 0.f;
+          if (!run || cudaEventSynchronize(e1) != cudaSuccess ||
+              cudaEventElapsedTime(&t, e0, e1) != cudaSuccess) {
+            ms_i = -1.f;
+            break;
+          }
+          if (rep > 0 && (ms_i < 0.f || t < ms_i)) ms_i = t;
+        }
+        if (ms_i > 0.f && (best_ms == 0.f || ms_i < best_ms)) {
+          best_ms = ms_i;
+          best = i;
+        }
+      }
+      (void)cudaGetLastError();
+    }
+    if (e0) cudaEventDestroy(e0);
+    if (e1) cudaEventDestroy(e1);
+  }
+  *out = res[best].algo;
+  if (g_tune) {
+    std::lock_guard<std::mutex> lock(mu);
+    cache[key] = *out;
+  }
+  return true;
+}
+
 // D (M x Nout, row-major, type dt) = A (M x K, bf16, row-major) W^T, with W
 // (Nout x K, bf16, row-major) -- in cuBLASLt's column-major terms
 // D^T = op_T(W) A^T.  Returns false if cuBLASLt refuses or fails.
@@ -287,14 +364,10 @@ bool gemm_bf16(int64_t M, int64_t Nout, int64_t K, const void* A, const void* W,
     if (cublasLtMatmulPreferenceSetAttribute(pref, CUBLASLT_MATMUL_PREF_MAX_WORKSPACE_BYTES,
                                              &ws_bytes, sizeof(ws_bytes)) != CUBLAS_STATUS_SUCCESS)
       break;
-    cublasLtMatmulHeuristicResult_t res{};
-    int found = 0;
-    if (cublasLtMatmulAlgoGetHeuristic(h, op, la, lb, lc, lc, pref, 1, &res, &found) !=
-            CUBLAS_STATUS_SUCCESS ||
-        found == 0)
-      break;
     const float alpha = 1.f, beta = 0.f;
-    if (cublasLtMatmul(h, op, &alpha, W, la, A, lb, &beta, D, lc, D, lc, &res.algo, ws, ws_bytes,
+    cublasLtMatmulAlgo_t algo;
+    if (!pick_algo(h, op, la, lb, lc, pref, M, Nout, K, dt, A, W, D, ws, ws_bytes, s, &algo)) break;
+    if (cublasLtMatmul(h, op, &alpha, W, la, A, lb, &beta, D, lc, D, lc, &algo, ws, ws_bytes,
                        s) != CUBLAS_STATUS_SUCCESS)
       break;
     ok = true;
@@ -488,6 +561,16 @@ m3ssd_status m3ssd_block_fwd(const m3ssd_block_dims* dims, const m3ssd_block_wei
   }
   if (M == 0) return M3SSD_OK;
   return back(dims, w, M, base, ws, out, s);
+}
+
+m3ssd_status m3ssd_block_tune(const m3ssd_block_dims* dims, const m3ssd_block_weights* w,
+                              const void* u, void* out, void* workspace, size_t workspace_bytes,
+                              void* stream) {
+  m3ssd::g_tune = true;
+  const m3ssd_status st =
+      m3ssd_block_fwd(dims, w, u, out, nullptr, nullptr, workspace, workspace_bytes, stream);
+  m3ssd::g_tune = false;
+  return st;
 }
 
 m3ssd_status m3ssd_block_step(const m3ssd_block_dims* dims, const m3ssd_block_weights* w,

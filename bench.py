@@ -16,7 +16,10 @@ With N > 1 (torchrun, one process per GPU) every rank runs its own batch
 (weak scaling, no collective on the data path); time is the max over ranks.
 
 The decode figure (b256 H32 P64 N128 fp32 cache after a 512-token prefill)
-replays one CUDA graph of 1000 m3ssd_step calls.
+replays one CUDA graph of 1000 m3ssd_step calls.  Side figures in the same line:
+MIMO rank-4 decode, the Mamba-3 SISO block at d_model 1024, the backward on the
+forward's workload, and the forward on the ssd and long workloads, each with
+its own roofline.
 
 Rank 0 prints one JSON line.
 """

@@ -25,9 +25,13 @@
 // everything back for dX, the rotation adjoints, dphi and the carries.  Pass 1
 // walks the chunks forward with the state product (W_end o Bbar)^T X on the
 // tensor cores and stores each chunk-start state and angle in the workspace.
+// The chunk inputs (X, dY, B, C, theta) arrive one chunk ahead by TMA tensor
+// copies on a byte-counting mbarrier, straight into the swizzled tiles.
 // All cross-thread sums run in a fixed order, so results are deterministic.
 // Every mbarrier wait is bounded (2 s) and sets an error flag the host reads.
 #include <cuda_bf16.h>
+
+#include <cstring>
 
 #include "common.cuh"
 #include "internal.h"
@@ -85,15 +89,14 @@ __device__ __forceinline__ float col_sum8(float v) {  // over lanes differing in
   return v;
 }
 
-// 16 bytes global -> shared without a register round trip; zero-filled (and
-// nothing read) when !full
-__device__ __forceinline__ void cp16(void* smem_dst, const void* gmem_src, bool full) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(tc5::saddr(smem_dst)),
-               "l"(gmem_src), "r"(full ? 16 : 0)
-               : "memory");
-}
-__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+// Tensor maps of the chunk inputs: 64-token boxes (token coordinate of row 0
+// first; -1 and tokens past the end read as zeros).  X and dY (p, h, t, b), B
+// and C (n, g, t, b) in two 64-column boxes, all 128-byte swizzled into the
+// operand tiles' layout; theta (i, h, t, b) fp32, unswizzled (r, i) rows.
+struct BwdMaps {
+  CUtensorMap X, Y, B, C, theta;
+};
+constexpr uint32_t kBytesX = kT1, kBytesBC = kT2, kBytesTh = kQ * kNH * 4;
 
 struct SmT {
   uint8_t Bh[kT2], Bl[kT2];      // Bbar (u, n)
@@ -116,6 +119,7 @@ struct SmT {
   float run[kNH];
   float misc[8];
   uint64_t mbar[3];
+  uint64_t lbar;                 // the chunk inputs' TMA copies
   uint32_t tmem;
   uint32_t err;
 };
@@ -175,7 +179,8 @@ __device__ __forceinline__ void mma_split(uint32_t d, uint32_t ah, uint32_t al, 
     for (int j = 0; j < steps; ++j) tc5::mma_bf16(d, da(al, j), db(bl, j), idesc, true);
 }
 
-__global__ void __launch_bounds__(kT, 1) bwd_tc_kernel(BwdArgs a, ChunkWs ws) {
+__global__ void __launch_bounds__(kT, 1)
+    bwd_tc_kernel(BwdArgs a, ChunkWs ws, const __grid_constant__ BwdMaps tm) {
   extern __shared__ uint8_t smraw[];
   SmT& sm = *reinterpret_cast<SmT*>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -187,10 +192,6 @@ __global__ void __launch_bounds__(kT, 1) bwd_tc_kernel(BwdArgs a, ChunkWs ws) {
   const int64_t H = a.H, G = a.G, L = a.L;
   const int64_t bh = blockIdx.x, b = bh / H, h = bh % H, g = h / (H / G);
   const int nC = (int)((L + QT - 1) / QT);
-  const bf16* X = static_cast<const bf16*>(a.X);
-  const bf16* Bg = static_cast<const bf16*>(a.B);
-  const bf16* Cg = static_cast<const bf16*>(a.C);
-  const bf16* dY = static_cast<const bf16*>(a.dY);
   const float Dh = a.D ? a.D[h] : 0.f;
   char* wsb = static_cast<char*>(a.workspace);
   float* hs_ws = reinterpret_cast<float*>(wsb + ws.hs) + bh * (int64_t)nC * kN * kP;
@@ -214,6 +215,7 @@ __global__ void __launch_bounds__(kT, 1) bwd_tc_kernel(BwdArgs a, ChunkWs ws) {
   if (warp == 0) tc5::tmem_alloc(&sm.tmem, 512);
   if (tid == 0) {
     for (int k = 0; k < 3; ++k) tc5::mbar_init(&sm.mbar[k], 1);
+    tc5::mbar_init(&sm.lbar, 1);
     tc5::fence_mbar_init();
     sm.err = 0;
   }
@@ -224,12 +226,18 @@ __global__ void __launch_bounds__(kT, 1) bwd_tc_kernel(BwdArgs a, ChunkWs ws) {
   __syncthreads();
   tc5::fence_after_sync();
   const uint32_t tmem = sm.tmem;
-  uint32_t par[3] = {0u, 0u, 0u};
+  uint32_t par[3] = {0u, 0u, 0u}, lpar = 0u;
   auto wait_bar = [&](int k) {
     if (!tc5::mbar_wait(&sm.mbar[k], par[k], kWaitNs, &sm.err)) sm.err = 1;
     par[k] ^= 1u;
     tc5::fence_after_sync();
   };
+  auto wait_loads = [&]() {  // every thread: this chunk's TMA copies have landed
+    if (!tc5::mbar_wait(&sm.lbar, lpar, kWaitNs, &sm.err)) sm.err = 1;
+    lpar ^= 1u;
+  };
+  const bool has_th = a.theta != nullptr;
+  const int hh = (int)h, gg_ = (int)g, bb = (int)b;
   auto mma_fence_sync = [&]() {  // operand stores -> tensor-core reads
     tc5::fence_proxy_async();
     tc5::fence_before_sync();
@@ -237,34 +245,24 @@ __global__ void __launch_bounds__(kT, 1) bwd_tc_kernel(BwdArgs a, ChunkWs ws) {
     tc5::fence_after_sync();
   };
 
-  // ---- the state pass's inputs, one chunk ahead: theta and raw B rows by
-  // cp.async once the rotation has read the previous ones, X once the state
-  // product has; thread (r = tid / 8, sg = tid % 8) owns X columns 8 sg ..,
-  // theta pairs 8 sg .. and B columns 16 sg .. of row r
+  // ---- the state pass's inputs, one chunk ahead, by TMA on lbar: theta and raw
+  // B rows once the rotation has read the previous ones, X once the state
+  // product has (one transaction count covers both); thread (r = tid / 8,
+  // sg = tid % 8) then owns X columns 8 sg .., theta pairs 8 sg .. and B columns
+  // 16 sg .. of row r
   const int lr = tid >> 3, sg = tid & 7;
   float braw[16], craw[16], xf8[8], yf8[8];
   float sc1[3] = {0.f, 0.f, 0.f};  // logdecay, gamma, beta of row tid (tid < 64)
-  auto rows_of = [&](int c, int64_t& th, int64_t& tg, bool& in, bool& own) {
-    const int64_t t = (int64_t)c * QT - 1 + lr;
-    in = t >= 0 && t < L;
-    own = lr > 0 && t < L;
-    th = (b * L + (in ? t : 0)) * H + h;
-    tg = (b * L + (in ? t : 0)) * G + g;
-  };
   auto fetch1_tb = [&](int c) {  // theta, raw B, the scalars
-    int64_t th, tg;
-    bool in, own;
-    rows_of(c, th, tg, in, own);
-    const bool th_ok = own && a.theta != nullptr;
-    const float* tsrc = th_ok ? a.theta + th * kNH + 8 * sg : reinterpret_cast<const float*>(X);
-    cp16(&sm.Vt[lr * kNH + 8 * sg], tsrc, th_ok);
-    cp16(&sm.Vt[lr * kNH + 8 * sg + 4], th_ok ? tsrc + 4 : tsrc, th_ok);
-    cp16(sm.Bh + off2(lr, 16 * sg), Bg + tg * kN + 16 * sg, in);
-    cp16(sm.Bh + off2(lr, 16 * sg + 8), Bg + tg * kN + 16 * sg + 8, in);
-    cp_commit();
-    const int64_t t0 = (int64_t)c * QT - 1;
+    const int t0 = c * QT - 1;
+    if (tid == 0) {
+      tc5::mbar_arrive_expect_tx(&sm.lbar, kBytesBC + kBytesX + (has_th ? kBytesTh : 0u));
+      if (has_th) tc5::tma_load_4d(tc5::saddr(sm.Vt), &tm.theta, &sm.lbar, 0, hh, t0, bb);
+      tc5::tma_load_4d(tc5::saddr(sm.Bh), &tm.B, &sm.lbar, 0, gg_, t0, bb);
+      tc5::tma_load_4d(tc5::saddr(sm.Bh) + kAtom, &tm.B, &sm.lbar, 64, gg_, t0, bb);
+    }
     sc1[0] = sc1[1] = sc1[2] = 0.f;
-    if (tid < kQ && tid > 0 && t0 + tid < L) {
+    if (tid < kQ && tid > 0 && (int64_t)t0 + tid < L) {
       const int64_t ts = (b * L + t0 + tid) * H + h;
       sc1[0] = a.logdecay[ts];
       sc1[1] = a.gamma[ts];
@@ -272,15 +270,19 @@ __global__ void __launch_bounds__(kT, 1) bwd_tc_kernel(BwdArgs a, ChunkWs ws) {
     }
   };
   auto fetch1_x = [&](int c) {
-    int64_t th, tg;
-    bool in, own;
-    rows_of(c, th, tg, in, own);
-    cp16(sm.X + off1(lr, 8 * sg), X + th * kP + 8 * sg, in);
-    cp_commit();
+    if (tid == 0) tc5::tma_load_4d(tc5::saddr(sm.X), &tm.X, &sm.lbar, 0, hh, c * QT - 1, bb);
+  };
+  // theta of row 0 (the carry-in token's own angle step belongs to the chunk
+  // before) is zero; so is all of theta when there is none
+  auto zero_theta = [&]() {
+    if (lr == 0 || !has_th) {
+      *reinterpret_cast<float4*>(&sm.Vt[lr * kNH + 8 * sg]) = make_float4(0.f, 0.f, 0.f, 0.f);
+      *reinterpret_cast<float4*>(&sm.Vt[lr * kNH + 8 * sg + 4]) = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
   };
   auto commit1 = [&](int c) {
-    cp_wait_all();
-    __syncthreads();  // every thread's copies have landed
+    wait_loads();
+    zero_theta();
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
       const float2 fb = unpack_bf16(*reinterpret_cast<const uint32_t*>(sm.Bh + off2(lr, 16 * sg + 2 * q)));
@@ -432,9 +434,9 @@ __global__ void __launch_bounds__(kT, 1) bwd_tc_kernel(BwdArgs a, ChunkWs ws) {
   };
 
   // ---- the reverse pass's inputs one chunk ahead: X, dY, theta and raw B, C
-  // rows by cp.async into their tiles (free from the end of the previous
-  // chunk's epilogue on), the chunk-start state, scalars and angle into
-  // registers; commit_chunk() lands them
+  // rows by TMA into their tiles (free from the end of the previous chunk's
+  // epilogue on), the chunk-start state, scalars and angle into registers;
+  // commit_chunk() lands them
   struct Pre {
     float hp[16];
     float sc[3];
@@ -442,20 +444,18 @@ __global__ void __launch_bounds__(kT, 1) bwd_tc_kernel(BwdArgs a, ChunkWs ws) {
   };
   auto fetch_chunk = [&](int c, Pre& f) {
     const int64_t t0 = (int64_t)c * QT - 1;
-    const int64_t t = t0 + lr;
-    const bool in = t >= 0 && t < L, own = lr > 0 && t < L;
-    const int64_t th = (b * L + (in ? t : 0)) * H + h, tg = (b * L + (in ? t : 0)) * G + g;
-    cp16(sm.X + off1(lr, 8 * sg), X + th * kP + 8 * sg, in);
-    cp16(sm.Y + off1(lr, 8 * sg), dY + th * kP + 8 * sg, own);
-    const bool th_ok = own && a.theta != nullptr;
-    const float* tsrc = th_ok ? a.theta + th * kNH + 8 * sg : reinterpret_cast<const float*>(X);
-    cp16(&sm.Vt[lr * kNH + 8 * sg], tsrc, th_ok);
-    cp16(&sm.Vt[lr * kNH + 8 * sg + 4], th_ok ? tsrc + 4 : tsrc, th_ok);
-    cp16(sm.Bh + off2(lr, 16 * sg), Bg + tg * kN + 16 * sg, in);
-    cp16(sm.Bh + off2(lr, 16 * sg + 8), Bg + tg * kN + 16 * sg + 8, in);
-    cp16(sm.Ch + off2(lr, 16 * sg), Cg + tg * kN + 16 * sg, own);
-    cp16(sm.Ch + off2(lr, 16 * sg + 8), Cg + tg * kN + 16 * sg + 8, own);
-    cp_commit();
+    if (tid == 0) {
+      const int tc = (int)t0;
+      const uint32_t aB = tc5::saddr(sm.Bh), aC = tc5::saddr(sm.Ch);
+      tc5::mbar_arrive_expect_tx(&sm.lbar, 2 * kBytesX + 2 * kBytesBC + (has_th ? kBytesTh : 0u));
+      tc5::tma_load_4d(tc5::saddr(sm.X), &tm.X, &sm.lbar, 0, hh, tc, bb);
+      tc5::tma_load_4d(tc5::saddr(sm.Y), &tm.Y, &sm.lbar, 0, hh, tc, bb);
+      tc5::tma_load_4d(aB, &tm.B, &sm.lbar, 0, gg_, tc, bb);
+      tc5::tma_load_4d(aB + kAtom, &tm.B, &sm.lbar, 64, gg_, tc, bb);
+      tc5::tma_load_4d(aC, &tm.C, &sm.lbar, 0, gg_, tc, bb);
+      tc5::tma_load_4d(aC + kAtom, &tm.C, &sm.lbar, 64, gg_, tc, bb);
+      if (has_th) tc5::tma_load_4d(tc5::saddr(sm.Vt), &tm.theta, &sm.lbar, 0, hh, tc, bb);
+    }
     const float* hw = hs_ws + (int64_t)c * kN * kP;
 #pragma unroll
     for (int j = 0; j < 16; ++j) f.hp[j] = hw[(16 * q4 + j) * kN + nrow];
@@ -472,9 +472,16 @@ __global__ void __launch_bounds__(kT, 1) bwd_tc_kernel(BwdArgs a, ChunkWs ws) {
     }
   };
   auto commit_chunk = [&](int c, const Pre& f) {
-    cp_wait_all();
-    __syncthreads();  // every thread's copies have landed
+    wait_loads();
     const int64_t t0 = (int64_t)c * QT - 1;
+    // row 0 is the carry-in token: its dY and C belong to the chunk before
+    zero_theta();
+    if (lr == 0) {
+      const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+      *reinterpret_cast<uint4*>(sm.Y + off1(0, 8 * sg)) = z;
+      *reinterpret_cast<uint4*>(sm.Ch + off2(0, 16 * sg)) = z;
+      *reinterpret_cast<uint4*>(sm.Ch + off2(0, 16 * sg + 8)) = z;
+    }
     // this thread's raw B, C (16 columns) and x, dy (8 columns) in fp32
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
@@ -941,7 +948,13 @@ __global__ void __launch_bounds__(kT, 1) bwd_tc_kernel(BwdArgs a, ChunkWs ws) {
   const float dDs = block_sum(dDacc, sm.red, &sm.misc[1]);
   if (tid == 0) {
     dDbh[bh] = dDs;
-    if (sm.err) atomicAdd(&g_bwd_tc_wait_timeouts, 1u);
+    if (sm.err) {
+      atomicAdd(&g_bwd_tc_wait_timeouts, 1u);
+      // a wait gave up: let the last copies and products in flight land (each
+      // wait again bounded) before the CTA's shared memory and TMEM go
+      tc5::mbar_wait(&sm.lbar, lpar ^ 1u, kWaitNs);
+      for (int k = 0; k < 3; ++k) tc5::mbar_wait(&sm.mbar[k], par[k] ^ 1u, kWaitNs);
+    }
   }
   tc5::fence_before_sync();
   __syncthreads();
@@ -959,10 +972,23 @@ bool bwd_tc_supported(const BwdArgs& a) {
 cudaError_t launch_bwd_tc(const BwdArgs& a, cudaStream_t s) {
   if (a.b * a.H == 0) return cudaSuccess;
   const ChunkWs ws = chunk_ws_layout(a.b, a.L, a.H);
+  BwdMaps tm;
+  memset(&tm, 0, sizeof(tm));
+  const uint64_t L = (uint64_t)a.L, b = (uint64_t)a.b, H = (uint64_t)a.H, G = (uint64_t)a.G;
+  const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  // with no tokens the kernel issues no copies (a map needs every extent > 0)
+  bool ok = L == 0 || encode_map(&tm.X, bf, a.X, kP, H, L, b, 2, 64, CU_TENSOR_MAP_SWIZZLE_128B) &&
+            encode_map(&tm.Y, bf, a.dY, kP, H, L, b, 2, 64, CU_TENSOR_MAP_SWIZZLE_128B) &&
+            encode_map(&tm.B, bf, a.B, kN, G, L, b, 2, 64, CU_TENSOR_MAP_SWIZZLE_128B) &&
+            encode_map(&tm.C, bf, a.C, kN, G, L, b, 2, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (ok && L > 0 && a.theta)
+    ok = encode_map(&tm.theta, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.theta, kNH, H, L, b, 4, kNH,
+                    CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (!ok) return cudaErrorInvalidValue;
   const int smem = (int)sizeof(SmT) + 1024;
   cudaError_t e = cudaFuncSetAttribute(bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  bwd_tc_kernel<<<(unsigned)(a.b * a.H), kT, smem, s>>>(a, ws);
+  bwd_tc_kernel<<<(unsigned)(a.b * a.H), kT, smem, s>>>(a, ws, tm);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   return launch_bwd_chunk_reduce(a, s);

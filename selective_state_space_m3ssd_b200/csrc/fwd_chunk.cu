@@ -699,6 +699,8 @@ __global__ void __launch_bounds__(kThreads, 2)
   if (warp == 0) tc5::tmem_dealloc(tmem, kTmemCols);
 }
 
+}  // namespace
+
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   static std::once_flag once;
@@ -713,11 +715,9 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// A 4-D map (d0 innermost) with a box of d0-extent `box0` by 64 tokens; d2 (the
-// token axis) is `tok` elements apart (0: dense, d0 d1).
 bool encode_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t d0, uint64_t d1,
                 uint64_t d2, uint64_t d3, uint64_t esz, uint32_t box0, CUtensorMapSwizzle sw,
-                uint64_t tok = 0) {
+                uint64_t tok) {
   PFN_cuTensorMapEncodeTiled_v12000 fn = tensor_map_encoder();
   if (!fn) return false;
   const cuuint64_t dims[4] = {d0, d1, d2, d3};
@@ -729,6 +729,8 @@ bool encode_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64
             CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+
+namespace {
 
 template <bool ROT, bool BIAS, bool TH16>
 cudaError_t launch_variant(const FwdArgs& a, cudaStream_t s) {

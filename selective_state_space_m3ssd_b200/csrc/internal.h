@@ -1,6 +1,7 @@
 // Internal launch interface shared by the C-ABI layer and the kernels.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -111,6 +112,12 @@ struct ChunkWs {
   size_t hs, phs, dBh, dCh, dbph, dDbh, total;
 };
 ChunkWs chunk_ws_layout(int64_t b, int64_t L, int64_t H);
+// A 4-D TMA tensor map (d0 innermost) with a box of d0-extent `box0` by 64
+// tokens; d2 (the token axis) is `tok` elements apart (0: dense, d0 d1).
+bool encode_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t d0, uint64_t d1,
+                uint64_t d2, uint64_t d3, uint64_t esz, uint32_t box0, CUtensorMapSwizzle sw,
+                uint64_t tok = 0);
+
 // Sums the per-head shares into dB, dC, dbprev0 and dD, in a fixed order.
 cudaError_t launch_bwd_chunk_reduce(const BwdArgs& a, cudaStream_t s);
 // The chunked backward on the tensor cores (bf16 X, B, C, dY; N = 128, P = 64;

@@ -125,6 +125,7 @@ struct SmT {
 };
 static_assert(sizeof(SmT) + 1024 <= 232448, "one CTA's shared memory");
 static_assert(2 * kT1 >= kQ * kNH * 4, "dphi fits in the EY tiles");
+static_assert(offsetof(SmT, Hl) == offsetof(SmT, Hh) + kT2, "one bulk copy lands both h_prev tiles");
 
 __device__ __forceinline__ float block_sum(float v, float* red, float* out) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -194,7 +195,9 @@ __global__ void __launch_bounds__(kT, 1)
   const int nC = (int)((L + QT - 1) / QT);
   const float Dh = a.D ? a.D[h] : 0.f;
   char* wsb = static_cast<char*>(a.workspace);
-  float* hs_ws = reinterpret_cast<float*>(wsb + ws.hs) + bh * (int64_t)nC * kN * kP;
+  // chunk-start states as h_prev tile pairs (bf16 high part, then residual;
+  // (n, p), 128-byte swizzled as in shared memory), 2 kT2 bytes a chunk
+  uint8_t* hs_img = reinterpret_cast<uint8_t*>(wsb + ws.hs) + bh * (int64_t)nC * (2 * kT2);
   float* ph_ws = reinterpret_cast<float*>(wsb + ws.phs) + bh * (int64_t)nC * kNH;
   float* dBh = reinterpret_cast<float*>(wsb + ws.dBh);
   float* dCh = reinterpret_cast<float*>(wsb + ws.dCh);
@@ -438,16 +441,23 @@ __global__ void __launch_bounds__(kT, 1)
   // epilogue on), the chunk-start state, scalars and angle into registers;
   // commit_chunk() lands them
   struct Pre {
-    float hp[16];
     float sc[3];
     float ph;
+  };
+  // the chunk-start state's tile pair, one bulk copy, as soon as the previous
+  // chunk's products have read its own (stage 1); it opens the loads' phase for
+  // all of the chunk's copies
+  auto fetch_h = [&](int c) {
+    if (tid == 0) {
+      tc5::mbar_arrive_expect_tx(&sm.lbar, 2 * kT2 + 2 * kBytesX + 2 * kBytesBC + (has_th ? kBytesTh : 0u));
+      tc5::bulk_load(tc5::saddr(sm.Hh), hs_img + (int64_t)c * (2 * kT2), 2 * kT2, &sm.lbar);
+    }
   };
   auto fetch_chunk = [&](int c, Pre& f) {
     const int64_t t0 = (int64_t)c * QT - 1;
     if (tid == 0) {
       const int tc = (int)t0;
       const uint32_t aB = tc5::saddr(sm.Bh), aC = tc5::saddr(sm.Ch);
-      tc5::mbar_arrive_expect_tx(&sm.lbar, 2 * kBytesX + 2 * kBytesBC + (has_th ? kBytesTh : 0u));
       tc5::tma_load_4d(tc5::saddr(sm.X), &tm.X, &sm.lbar, 0, hh, tc, bb);
       tc5::tma_load_4d(tc5::saddr(sm.Y), &tm.Y, &sm.lbar, 0, hh, tc, bb);
       tc5::tma_load_4d(aB, &tm.B, &sm.lbar, 0, gg_, tc, bb);
@@ -456,9 +466,6 @@ __global__ void __launch_bounds__(kT, 1)
       tc5::tma_load_4d(aC + kAtom, &tm.C, &sm.lbar, 64, gg_, tc, bb);
       if (has_th) tc5::tma_load_4d(tc5::saddr(sm.Vt), &tm.theta, &sm.lbar, 0, hh, tc, bb);
     }
-    const float* hw = hs_ws + (int64_t)c * kN * kP;
-#pragma unroll
-    for (int j = 0; j < 16; ++j) f.hp[j] = hw[(16 * q4 + j) * kN + nrow];
     f.sc[0] = f.sc[1] = f.sc[2] = 0.f;
     f.ph = 0.f;
     if (tid < kQ) {
@@ -514,7 +521,6 @@ __global__ void __launch_bounds__(kT, 1)
       *reinterpret_cast<uint4*>(sm.X + off1(0, 8 * sg)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
       *reinterpret_cast<uint4*>(sm.Xl + off1(0, 8 * sg)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
     }
-    store_np(sm.Hh, sm.Hl, f.hp);
     if (tid < kQ) {
       sm.cs[tid] = f.sc[0];  // the raw logdecay until scalars_angles
       sm.ga[tid] = f.sc[1];
@@ -537,9 +543,7 @@ __global__ void __launch_bounds__(kT, 1)
     fetch1_x(0);
   }
   for (int c = 0; c < nC; ++c) {
-    float* hw = hs_ws + (int64_t)c * kN * kP;  // (p, n)
-#pragma unroll
-    for (int j = 0; j < 16; ++j) hw[(16 * q4 + j) * kN + nrow] = hreg[j];
+    store_np(hs_img + (int64_t)c * (2 * kT2), hs_img + (int64_t)c * (2 * kT2) + kT2, hreg);
     if (tid < kNH) ph_ws[(int64_t)c * kNH + tid] = sm.phi0[tid];
     commit1(c);
     __syncthreads();
@@ -570,6 +574,9 @@ __global__ void __launch_bounds__(kT, 1)
     if (tid < kNH) sm.phi0[tid] = nphi;
   }
 
+  tc5::fence_proxy_async_global();  // the state images -> the bulk copies below
+  __syncthreads();
+
   // ---- pass 2: the chunks in reverse --------------------------------------
   float greg[16];  // g = dL/dh_end, rows nrow, columns 16 q4 + j
 #pragma unroll
@@ -580,16 +587,16 @@ __global__ void __launch_bounds__(kT, 1)
   if (tid < kN) sm.cdb[0][tid] = sm.cdb[1][tid] = 0.f;
   float dDacc = 0.f;
   Pre f;
-  if (nC > 0) fetch_chunk(nC - 1, f);
+  if (nC > 0) {
+    fetch_h(nC - 1);
+    fetch_chunk(nC - 1, f);
+  }
   __syncthreads();
 
   for (int c = nC - 1; c >= 0; --c) {
     const int cur = c & 1, nxt = cur ^ 1;
     const int64_t t0 = (int64_t)c * QT - 1;
     auto own = [&](int r) { return r > 0 && t0 + r < L; };
-    float hpr[16];
-#pragma unroll
-    for (int j = 0; j < 16; ++j) hpr[j] = f.hp[j];
     commit_chunk(c, f);
     __syncthreads();
     scalars_angles();
@@ -716,6 +723,20 @@ __global__ void __launch_bounds__(kT, 1)
         const float v = half_sum4(sy[hf]) * sm.ecs[r];
         if ((lane & 3) == 0) sm.rowq[q4][r] = v;
       }
+      float hpr[16];  // h_prev row nrow, columns 16 q4 + j, as its high part + residual
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const uint32_t o = off1(nrow, 16 * q4 + 8 * half);
+        const uint4 vh = *reinterpret_cast<const uint4*>(sm.Hh + o);
+        const uint4 vl = *reinterpret_cast<const uint4*>(sm.Hl + o);
+        const uint32_t uh[4] = {vh.x, vh.y, vh.z, vh.w}, ul[4] = {vl.x, vl.y, vl.z, vl.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 fh = unpack_bf16(uh[q]), fl = unpack_bf16(ul[q]);
+          hpr[8 * half + 2 * q] = fh.x + fl.x;
+          hpr[8 * half + 2 * q + 1] = fh.y + fl.y;
+        }
+      }
       const float eE = sm.ecs[kQ - 1];
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
@@ -723,7 +744,8 @@ __global__ void __launch_bounds__(kT, 1)
         greg[j] = fmaf(eE, greg[j], __uint_as_float(dhr[j]));
       }
     }
-    mma_fence_sync();  // M and WE stored; G, E read
+    mma_fence_sync();  // M and WE stored; G, E and h_prev read
+    if (c > 0) fetch_h(c - 1);
 
     // -- stage 2
     if (tid == 0) {

@@ -436,10 +436,11 @@ __global__ void __launch_bounds__(kT, 1)
     }
   };
 
-  // ---- the reverse pass's inputs one chunk ahead: X, dY, theta and raw B, C
-  // rows by TMA into their tiles (free from the end of the previous chunk's
-  // epilogue on), the chunk-start state, scalars and angle into registers;
-  // commit_chunk() lands them
+  // ---- the reverse pass's inputs one chunk ahead: the chunk-start state's
+  // tiles by a bulk copy (fetch_h, once stage 1 has read the previous ones); X,
+  // dY, theta and raw B, C rows by TMA into their tiles (free from the end of
+  // the previous chunk's epilogue on); the scalars and the chunk-start angle
+  // into registers; commit_chunk() lands them
   struct Pre {
     float sc[3];
     float ph;

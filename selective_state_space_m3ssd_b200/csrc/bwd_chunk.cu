@@ -1036,14 +1036,61 @@ __global__ void __launch_bounds__(kT, 1) bwd_chunk_kernel(BwdArgs a, ChunkWs ws)
 
 // Sums over the heads of a group (dB, dC, dbprev0) and over the batch (dD),
 // each in a fixed order.
-__global__ void bwd_chunk_reduce_kernel(BwdArgs a, ChunkWs ws) {
+// dB and dC when both outputs are 16-byte aligned: four columns a thread, the
+// loads of eight heads in flight at once; every element is still the sum over
+// the heads of its group in head order from zero, as in the kernel below, so
+// the results are the same bit for bit.
+__global__ void bwd_chunk_reduce_bc4_kernel(BwdArgs a, ChunkWs ws) {
+  constexpr int kC4 = kN / 4, kU = 8;
+  const int64_t H = a.H, G = a.G;
+  const int hpg = (int)(H / G);
+  const char* wsb = static_cast<const char*>(a.workspace);
+  const float4* dBh = reinterpret_cast<const float4*>(wsb + ws.dBh);
+  const float4* dCh = reinterpret_cast<const float4*>(wsb + ws.dCh);
+  float4* dB = reinterpret_cast<float4*>(a.dB);
+  float4* dC = reinterpret_cast<float4*>(a.dC);
+  const int64_t n4 = a.b * a.L * G * kC4, stride = (int64_t)gridDim.x * blockDim.x;
+  auto add = [](float4& s, const float4& v) {
+    s.x += v.x;
+    s.y += v.y;
+    s.z += v.z;
+    s.w += v.w;
+  };
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += stride) {
+    const int64_t c4 = i % kC4, row = i / kC4, gg = row % G, bt = row / G;
+    const float4* pb = dBh + (bt * H + gg * hpg) * kC4 + c4;
+    const float4* pc = dCh + (bt * H + gg * hpg) * kC4 + c4;
+    float4 sb = make_float4(0.f, 0.f, 0.f, 0.f), sc = sb;
+    for (int q0 = 0; q0 < hpg; q0 += kU) {
+      float4 vb[kU], vc[kU];
+#pragma unroll
+      for (int k = 0; k < kU; ++k)
+        if (q0 + k < hpg) {
+          vb[k] = pb[(int64_t)(q0 + k) * kC4];
+          vc[k] = pc[(int64_t)(q0 + k) * kC4];
+        }
+#pragma unroll
+      for (int k = 0; k < kU; ++k)
+        if (q0 + k < hpg) {
+          add(sb, vb[k]);
+          add(sc, vc[k]);
+        }
+    }
+    dB[i] = sb;
+    dC[i] = sc;
+  }
+}
+
+// The sums over the heads of each group (dB, dC unless `with_bc` is false,
+// dbprev0) and over the batch (dD) of the per-head shares, in a fixed order.
+__global__ void bwd_chunk_reduce_kernel(BwdArgs a, ChunkWs ws, bool with_bc) {
   const int64_t H = a.H, G = a.G, hpg = H / G;
   const char* wsb = static_cast<const char*>(a.workspace);
   const float* dBh = reinterpret_cast<const float*>(wsb + ws.dBh);
   const float* dCh = reinterpret_cast<const float*>(wsb + ws.dCh);
   const float* dbph = reinterpret_cast<const float*>(wsb + ws.dbph);
   const float* dDbh = reinterpret_cast<const float*>(wsb + ws.dDbh);
-  const int64_t nBC = a.b * a.L * G * kN, nbp = a.b * G * kN;
+  const int64_t nBC = with_bc ? a.b * a.L * G * kN : 0, nbp = a.b * G * kN;
   const int64_t total = nBC + nbp + H;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += stride) {
@@ -1106,10 +1153,18 @@ cudaError_t launch_bwd_chunk(const BwdArgs& a, cudaStream_t s) {
 
 cudaError_t launch_bwd_chunk_reduce(const BwdArgs& a, cudaStream_t s) {
   const ChunkWs ws = chunk_ws_layout(a.b, a.L, a.H);
-  const int64_t total = a.b * a.L * a.G * kN + a.b * a.G * kN + a.H;
+  auto al16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; };
+  const int64_t nBC = a.b * a.L * a.G * kN;
+  const bool bc4 = nBC > 0 && al16(a.dB) && al16(a.dC);
+  if (bc4) {
+    const int64_t blocks = (nBC / 4 + 255) / 256;
+    const unsigned g4 = (unsigned)(blocks < 148 * 8 ? blocks : 148 * 8);
+    bwd_chunk_reduce_bc4_kernel<<<g4, 256, 0, s>>>(a, ws);
+  }
+  const int64_t total = (bc4 ? 0 : nBC) + a.b * a.G * kN + a.H;
   const int64_t blocks = (total + 255) / 256;
   const unsigned rg = (unsigned)(blocks < 148 * 32 ? (blocks > 0 ? blocks : 1) : 148 * 32);
-  bwd_chunk_reduce_kernel<<<rg, 256, 0, s>>>(a, ws);
+  bwd_chunk_reduce_kernel<<<rg, 256, 0, s>>>(a, ws, !bc4);
   return cudaGetLastError();
 }
 

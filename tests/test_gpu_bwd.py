@@ -228,6 +228,26 @@ def test_bwd_chunk_unaligned_inputs(dtype):
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_bwd_chunk_group_sums_unaligned_outputs(dtype):
+    # dB and dC one element past a 16-byte boundary take the element-wise group
+    # sums; aligned ones take the four-column kernel.  Both add the same per-head
+    # shares in the same order, so the results agree bit for bit.
+    inp = with_cache_inputs(make_inputs(CHUNK.with_(seqlen=130, dtype=dtype)), seed=9)
+    dY, dhT = upstream(inp, 31)
+    d = to_dev(inp)
+    args = [d.get(k) for k in ARGS]
+    extra = dict(angle0=d.get("angle0"), xprev0=d.get("xprev0"), bprev0=d.get("bprev0"))
+    g1 = m3.bwd(*args, dY=dY.cuda(), dhT=dhT.cuda(), **extra)
+    grads = {k: (_offset_copy(torch.zeros_like(v)) if k in ("dB", "dC") else torch.empty_like(v))
+             for k, v in g1.items()}
+    assert grads["dB"].data_ptr() % 16 != 0 and grads["dC"].data_ptr() % 16 != 0
+    m3.bwd(*args, dY=dY.cuda(), dhT=dhT.cuda(), grads=grads, **extra)
+    torch.cuda.synchronize()
+    for k in g1:
+        assert torch.equal(g1[k], grads[k]), k
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
 def test_bwd_chunk_is_deterministic(dtype):
     inp = with_cache_inputs(make_inputs(CHUNK.with_(seqlen=140, dtype=dtype)), seed=4)
     dY, dhT = upstream(inp, 23)

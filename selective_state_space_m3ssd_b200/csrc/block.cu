@@ -154,21 +154,26 @@ __global__ void __launch_bounds__(kPrepThreads) block_prep_kernel(PrepArgs a) {
 
 // The same with 16-byte accesses, for shapes whose row parts are multiples of
 // four floats and eight bf16 (H P % 8, G N % 4, H % 4, N % 8).
+// A CTA takes kPrepThreads / (32 kPrepTokWarps) tokens, kPrepTokWarps warps each,
+// so that many tokens' row loads are in flight on an SM at once.
+constexpr int kPrepTokWarps = 2, kPrepToks = kPrepThreads / (32 * kPrepTokWarps);
 __global__ void __launch_bounds__(kPrepThreads) block_prep_vec_kernel(PrepArgs a) {
   // No barrier: the warp that sums a group's squares also writes its normed
   // values, and every thread that scales theta recomputes its head's Delta.
-  const int64_t tok = blockIdx.x;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  constexpr int kT = 32 * kPrepTokWarps;  // threads of one token
+  const int64_t tok = (int64_t)blockIdx.x * kPrepToks + (int)threadIdx.x / kT;
+  if (tok >= a.M) return;
+  const int tid = (int)threadIdx.x % kT, lane = tid & 31, warp = tid >> 5;
   const int H = (int)a.H, P = (int)a.P, N = (int)a.N, G = (int)a.G, NH = N / 2;
   const int HP = H * P, GN = G * N;
   const int oB = 2 * HP, oC = oB + GN, odt = oC + GN, olam = odt + H, oth = olam + H;
   const __nv_bfloat16* row = a.zx + tok * a.width;
 
   if (a.write_x)
-    for (int k = tid; k < HP / 8; k += kPrepThreads)
+    for (int k = tid; k < HP / 8; k += kT)
       *reinterpret_cast<uint4*>(a.X + tok * HP + 8 * k) =
           *reinterpret_cast<const uint4*>(row + HP + 8 * k);
-  for (int j = warp; j < 2 * G; j += kPrepThreads / 32) {  // N <= 256: two float4 a lane
+  for (int j = warp; j < 2 * G; j += kPrepTokWarps) {  // N <= 256: two float4 a lane
     const int off = j < G ? oB + j * N : oC + (j - G) * N;
     const float* w = j < G ? a.Bw : a.Cw;
     __nv_bfloat16* dst = (j < G ? a.B + (tok * G + j) * N : a.C + (tok * G + j - G) * N);
@@ -195,7 +200,7 @@ __global__ void __launch_bounds__(kPrepThreads) block_prep_vec_kernel(PrepArgs a
       }
     }
   }
-  for (int h = tid; h < H; h += kPrepThreads) {
+  for (int h = tid; h < H; h += kT) {
     const float dl = softplus_f(bf(row[odt + h]) + a.dt_bias[h]);
     const float lg = -expf(a.A_log[h]) * dl;
     const float lam = 1.f / (1.f + expf(-bf(row[olam + h])));
@@ -203,7 +208,7 @@ __global__ void __launch_bounds__(kPrepThreads) block_prep_vec_kernel(PrepArgs a
     a.ga[tok * H + h] = lam * dl;
     a.be[tok * H + h] = (1.f - lam) * dl * expf(lg);
   }
-  for (int k = tid; a.write_th && k < H * NH / 4; k += kPrepThreads) {
+  for (int k = tid; a.write_th && k < H * NH / 4; k += kT) {
     const int h = (4 * k) / NH;
     const float d = softplus_f(bf(row[odt + h]) + a.dt_bias[h]);
     const float4 v = ld4_bf16(row + oth + 4 * k);
@@ -212,28 +217,44 @@ __global__ void __launch_bounds__(kPrepThreads) block_prep_vec_kernel(PrepArgs a
   }
 }
 
-// y * SiLU(z), z read from the bf16 in_proj rows, eight elements a thread
-// (H P % 8 == 0, in_proj width % 8 == 0).
+// y * SiLU(z), z read from the bf16 in_proj rows, eight elements a thread and
+// two such groups an iteration (their loads in flight together)
+// (H P % 8 == 0, in_proj width % 8 == 0).  SiLU takes the hardware exponential
+// and an approximate division: their few-ulp error is far below the bf16
+// rounding of the output.
 __global__ void block_gate_vec_kernel(const __nv_bfloat16* __restrict__ y,
                                       const __nv_bfloat16* __restrict__ zx, int64_t width,
                                       int64_t HP,
                                       int64_t M, __nv_bfloat16* __restrict__ out) {
   const int64_t n8 = M * HP / 8, stride = (int64_t)gridDim.x * blockDim.x, hp8 = HP / 8;
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8; i += stride) {
-    const int64_t tok = i / hp8, k = 8 * (i - tok * hp8);
-    const uint4 yv = *reinterpret_cast<const uint4*>(y + 8 * i);
-    const float4 z0 = ld4_bf16(zx + tok * width + k);
-    const float4 z1 = ld4_bf16(zx + tok * width + k + 4);
-    const uint32_t yw[4] = {yv.x, yv.y, yv.z, yv.w};
-    const float z[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
-    uint32_t o[4];
+  for (int64_t i0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i0 < n8; i0 += 2 * stride) {
+    uint4 yv[2];
+    float4 z0[2], z1[2];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float y0 = __uint_as_float(yw[j] << 16), y1 = __uint_as_float(yw[j] & 0xffff0000u);
-      o[j] = pack2_bf16(y0 * z[2 * j] / (1.f + expf(-z[2 * j])),
-                        y1 * z[2 * j + 1] / (1.f + expf(-z[2 * j + 1])));
+    for (int u = 0; u < 2; ++u) {
+      const int64_t i = i0 + u * stride;
+      if (i < n8) {
+        const int64_t tok = i / hp8, k = 8 * (i - tok * hp8);
+        yv[u] = *reinterpret_cast<const uint4*>(y + 8 * i);
+        z0[u] = ld4_bf16(zx + tok * width + k);
+        z1[u] = ld4_bf16(zx + tok * width + k + 4);
+      }
     }
-    *reinterpret_cast<uint4*>(out + 8 * i) = make_uint4(o[0], o[1], o[2], o[3]);
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int64_t i = i0 + u * stride;
+      if (i >= n8) break;
+      const uint32_t yw[4] = {yv[u].x, yv[u].y, yv[u].z, yv[u].w};
+      const float z[8] = {z0[u].x, z0[u].y, z0[u].z, z0[u].w, z1[u].x, z1[u].y, z1[u].z, z1[u].w};
+      uint32_t o[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float y0 = __uint_as_float(yw[j] << 16), y1 = __uint_as_float(yw[j] & 0xffff0000u);
+        o[j] = pack2_bf16(__fdividef(y0 * z[2 * j], 1.f + __expf(-z[2 * j])),
+                          __fdividef(y1 * z[2 * j + 1], 1.f + __expf(-z[2 * j + 1])));
+      }
+      *reinterpret_cast<uint4*>(out + 8 * i) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
   }
 }
 
@@ -432,7 +453,7 @@ m3ssd_status front(const m3ssd_block_dims* d, const m3ssd_block_weights* w, cons
   if (smem > 48 * 1024) return M3SSD_ERR_UNSUPPORTED;
   const bool w16 = aligned(a.Bw, 16) && aligned(a.Cw, 16);
   if (w16 && vec_shape(a.H, a.P, a.N, a.G, width))
-    block_prep_vec_kernel<<<(unsigned)M, kPrepThreads, 0, s>>>(a);
+    block_prep_vec_kernel<<<(unsigned)((M + kPrepToks - 1) / kPrepToks), kPrepThreads, 0, s>>>(a);
   else
     block_prep_kernel<<<(unsigned)M, kPrepThreads, smem, s>>>(a);
   return cudaGetLastError() == cudaSuccess ? M3SSD_OK : M3SSD_ERR_CUDA;

@@ -156,7 +156,7 @@ __global__ void __launch_bounds__(kPrepThreads) block_prep_kernel(PrepArgs a) {
 // four floats and eight bf16 (H P % 8, G N % 4, H % 4, N % 8).
 // A CTA takes kPrepThreads / (32 kPrepTokWarps) tokens, kPrepTokWarps warps each,
 // so that many tokens' row loads are in flight on an SM at once.
-constexpr int kPrepTokWarps = 2, kPrepToks = kPrepThreads / (32 * kPrepTokWarps);
+constexpr int kPrepTokWarps = 1, kPrepToks = kPrepThreads / (32 * kPrepTokWarps);
 __global__ void __launch_bounds__(kPrepThreads) block_prep_vec_kernel(PrepArgs a) {
   // No barrier: the warp that sums a group's squares also writes its normed
   // values, and every thread that scales theta recomputes its head's Delta.

@@ -1036,10 +1036,30 @@ __global__ void __launch_bounds__(kT, 1) bwd_chunk_kernel(BwdArgs a, ChunkWs ws)
 
 // Sums over the heads of a group (dB, dC, dbprev0) and over the batch (dD),
 // each in a fixed order.
+// Item r of the sums after dB, dC: dbprev0 (b, G, N) over the heads of each
+// group, then dD (H) over the batch, each in a fixed order.
+__device__ void reduce_tail(const BwdArgs& a, const ChunkWs& ws, int64_t r) {
+  const int64_t H = a.H, G = a.G, hpg = H / G, nbp = a.b * G * kN;
+  const char* wsb = static_cast<const char*>(a.workspace);
+  const float* dbph = reinterpret_cast<const float*>(wsb + ws.dbph);
+  const float* dDbh = reinterpret_cast<const float*>(wsb + ws.dDbh);
+  if (r < nbp) {
+    const int64_t nn = r % kN, row = r / kN, gg = row % G, bb = row / G;
+    float v = 0.f;
+    for (int64_t q = 0; q < hpg; ++q) v += dbph[(bb * H + gg * hpg + q) * kN + nn];
+    if (a.dbprev0) a.dbprev0[r] = v;
+    return;
+  }
+  r -= nbp;
+  float v = 0.f;
+  for (int64_t bb = 0; bb < a.b; ++bb) v += dDbh[bb * H + r];
+  if (a.dD) a.dD[r] = v;
+}
+
 // dB and dC when both outputs are 16-byte aligned: four columns a thread, the
 // loads of eight heads in flight at once; every element is still the sum over
 // the heads of its group in head order from zero, as in the kernel below, so
-// the results are the same bit for bit.
+// the results are the same bit for bit.  Then dbprev0 and dD.
 __global__ void bwd_chunk_reduce_bc4_kernel(BwdArgs a, ChunkWs ws) {
   constexpr int kC4 = kN / 4, kU = 8;
   const int64_t H = a.H, G = a.G;
@@ -1079,18 +1099,19 @@ __global__ void bwd_chunk_reduce_bc4_kernel(BwdArgs a, ChunkWs ws) {
     dB[i] = sb;
     dC[i] = sc;
   }
+  const int64_t tail = a.b * G * kN + H;  // dbprev0 and dD
+  for (int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; r < tail; r += stride)
+    reduce_tail(a, ws, r);
 }
 
-// The sums over the heads of each group (dB, dC unless `with_bc` is false,
-// dbprev0) and over the batch (dD) of the per-head shares, in a fixed order.
-__global__ void bwd_chunk_reduce_kernel(BwdArgs a, ChunkWs ws, bool with_bc) {
+// The sums over the heads of each group (dB, dC, dbprev0) and over the batch
+// (dD) of the per-head shares, in a fixed order.
+__global__ void bwd_chunk_reduce_kernel(BwdArgs a, ChunkWs ws) {
   const int64_t H = a.H, G = a.G, hpg = H / G;
   const char* wsb = static_cast<const char*>(a.workspace);
   const float* dBh = reinterpret_cast<const float*>(wsb + ws.dBh);
   const float* dCh = reinterpret_cast<const float*>(wsb + ws.dCh);
-  const float* dbph = reinterpret_cast<const float*>(wsb + ws.dbph);
-  const float* dDbh = reinterpret_cast<const float*>(wsb + ws.dDbh);
-  const int64_t nBC = with_bc ? a.b * a.L * G * kN : 0, nbp = a.b * G * kN;
+  const int64_t nBC = a.b * a.L * G * kN, nbp = a.b * G * kN;
   const int64_t total = nBC + nbp + H;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += stride) {
@@ -1107,18 +1128,7 @@ __global__ void bwd_chunk_reduce_kernel(BwdArgs a, ChunkWs ws, bool with_bc) {
       a.dC[r] = sc;
       continue;
     }
-    r -= nBC;
-    if (r < nbp) {  // dbprev0: (b, G, N)
-      const int64_t nn = r % kN, row = r / kN, gg = row % G, bb = row / G;
-      float v = 0.f;
-      for (int64_t q = 0; q < hpg; ++q) v += dbph[(bb * H + gg * hpg + q) * kN + nn];
-      if (a.dbprev0) a.dbprev0[r] = v;
-      continue;
-    }
-    r -= nbp;
-    float v = 0.f;  // dD: (H)
-    for (int64_t bb = 0; bb < a.b; ++bb) v += dDbh[bb * H + r];
-    if (a.dD) a.dD[r] = v;
+    reduce_tail(a, ws, r - nBC);
   }
 }
 
@@ -1160,11 +1170,12 @@ cudaError_t launch_bwd_chunk_reduce(const BwdArgs& a, cudaStream_t s) {
     const int64_t blocks = (nBC / 4 + 255) / 256;
     const unsigned g4 = (unsigned)(blocks < 148 * 8 ? blocks : 148 * 8);
     bwd_chunk_reduce_bc4_kernel<<<g4, 256, 0, s>>>(a, ws);
+    return cudaGetLastError();
   }
-  const int64_t total = (bc4 ? 0 : nBC) + a.b * a.G * kN + a.H;
+  const int64_t total = nBC + a.b * a.G * kN + a.H;
   const int64_t blocks = (total + 255) / 256;
   const unsigned rg = (unsigned)(blocks < 148 * 32 ? (blocks > 0 ? blocks : 1) : 148 * 32);
-  bwd_chunk_reduce_kernel<<<rg, 256, 0, s>>>(a, ws, !bc4);
+  bwd_chunk_reduce_kernel<<<rg, 256, 0, s>>>(a, ws);
   return cudaGetLastError();
 }
 

@@ -696,7 +696,8 @@ def run_reference(args):
 def run_profile(args):
     """One kernel family alone, for ncu: the forward on the siso workload at
     batch 2 (146 MB of inputs, above L2; a small case for full-section
-    captures), the backward on one batch row at L = 1024 (a small case), or
+    captures), the backward on one batch row at L = 1024 (a small case), the
+    rank-4 MIMO decode step at batch 128 (134 MB of state, a small case), or
     the block at its model size (for launch lists only).  Prints
     one summary line; not a bench line."""
     import selective_state_space_m3ssd_b200 as m3
@@ -723,6 +724,31 @@ def run_profile(args):
             m3.bwd(*args_, dY=dY)
         torch.cuda.synchronize(dev)
         print(json.dumps({"profile": "backward", "workload": "siso shape b1 L1024 H32 P64 N128"}))
+    elif args.profile == "mimo":
+        # rank-4 MIMO decode steps at half the decode batch: b128, fp32 cache
+        # (134 MB of state, above L2), one launch of the step kernel and one of
+        # the b_prev update per call
+        R = 4
+        w = WORKLOADS["decode"].with_(batch=128)
+        b, H, P, N, G = w.batch, w.nheads, w.headdim, w.dstate, w.ngroups
+        gen = torch.Generator(device=dev).manual_seed(w.seed + 29)
+        z = dict(device=dev, dtype=torch.float32)
+        cache = m3.new_mimo_cache(b, H, P, N, G, R, dev)
+        cache["ssm"].normal_(0, 0.3, generator=gen)
+        x = torch.randn(b, H, P, R, generator=gen, **z)
+        Bt = torch.randn(b, G, N, R, generator=gen, **z) / N ** 0.5
+        Ct = torch.randn(b, G, N, R, generator=gen, **z) / N ** 0.5
+        th = torch.randn(b, H, N // 2, generator=gen, **z) * 0.05
+        ld = -torch.rand(b, H, generator=gen, **z) * 0.5
+        be = torch.rand(b, H, generator=gen, **z) * 0.3
+        ga = torch.rand(b, H, generator=gen, **z) * 0.5
+        D = torch.randn(H, generator=gen, **z)
+        y = torch.empty_like(x)
+        for _ in range(args.warmup + args.steps):
+            m3.mimo_step(cache, x, ld, be, ga, Bt, Ct, th, D, y_t=y)
+        torch.cuda.synchronize(dev)
+        print(json.dumps({"profile": "mimo", "workload": f"mimo rank-{R} decode b{b} H{H} P{P} "
+                          f"N{N} fp32 cache"}))
     else:
         from selective_state_space_m3ssd_b200.synth import BLOCKS, make_block
         s = BLOCKS["model"]
@@ -750,7 +776,7 @@ def main():
                     help="skip the forward on the ssd and long workloads (side figures)")
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="omit the oracle timing (it never runs inside a GPU timed region)")
-    ap.add_argument("--profile", choices=["forward", "block", "backward"],
+    ap.add_argument("--profile", choices=["forward", "block", "backward", "mimo"],
                     help="run only a small case of one kernel family (for ncu captures)")
     args = ap.parse_args()
     if args.warmup < 3:

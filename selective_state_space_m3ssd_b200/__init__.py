@@ -76,7 +76,12 @@ class BlockWeights(ctypes.Structure):
 
 
 def load(path: str | None = None):
-    """Load ``libm3ssd.so`` (once) and declare the C signatures."""
+    """Load ``libm3ssd.so`` (once) and declare the C signatures.
+
+    With ``path``, load that build of the library and return its handle with
+    the signatures declared; the module's own calls keep using the in-tree
+    library (assign the handle to ``_lib`` to route them to the other build).
+    """
     global _lib
     with _lock:
         if _lib is not None and path is None:

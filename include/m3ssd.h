@@ -255,13 +255,21 @@ m3ssd_status m3ssd_bwd(const m3ssd_dims* dims, const void* X, const float* logde
                        void* stream);
 
 /*
- * m3ssd_bwd without a caller workspace: the scratch is a fixed 64 MiB device
- * array inside the library, reserved when its device code is loaded.  The
- * pages have no counterpart for this entry point; it is a convenience of this
- * library.  Arguments and results are those of m3ssd_bwd.  Requests whose
+ * m3ssd_bwd without a caller workspace, for callers that cannot allocate
+ * device memory where they call the backward (code inside a CUDA graph
+ * capture, or a runtime whose allocator may not be used from the launching
+ * thread).  The scratch is a fixed 64 MiB device array inside the library,
+ * reserved when its device code is loaded on a device and kept by every GPU
+ * that loads the library until the process exits.  The pages have no
+ * counterpart for this entry point; it is a convenience of this library.
+ * Arguments and results are those of m3ssd_bwd.  Invalid dims return
+ * m3ssd_bwd's status without touching the device; requests whose
  * m3ssd_bwd_workspace_size exceeds 64 MiB return M3SSD_ERR_UNSUPPORTED before
- * any device call.  Every call uses the same array, so calls must not overlap
- * (issue them on one stream, or synchronise between streams).
+ * any device call.  The first call on a device (with that device current)
+ * looks up the array's device address once (cudaGetSymbolAddress); make that
+ * first call before any stream capture.  No call allocates.  Every call uses
+ * the same array, which keeps the last call's contents, so calls that overlap
+ * on the GPU race: issue them on one stream, or synchronise between streams.
  */
 m3ssd_status m3ssd_bwd_noalloc(const m3ssd_dims* dims, const void* X, const float* logdecay,
                                const float* beta, const float* gamma, const void* B,
@@ -366,6 +374,21 @@ m3ssd_status m3ssd_block_step(const m3ssd_block_dims* dims, const m3ssd_block_we
  * and must not be captured in a CUDA graph.  Returns M3SSD_ERR_INVALID_ARG for
  * a NULL pointer and M3SSD_ERR_CUDA if the device cannot be read. */
 m3ssd_status m3ssd_device_wait_timeouts(uint32_t* count);
+
+/*
+ * Testing hooks for the failure path of the bounded device-side waits (no page
+ * counterpart).  They copy to device variables synchronously, so they must not
+ * be called while work of this library is in flight or being captured.
+ *   m3ssd_test_set_wait_limit: the time limit of the chunked forward's bounded
+ *     waits, in nanoseconds (0 restores the default of 2 s).
+ *   m3ssd_test_drop_next_gram_signal: the next chunked-forward sequence to
+ *     start leaves out the completion signal of its first Gram product, so its
+ *     compute warps' wait for it runs out: that launch counts one timeout in
+ *     m3ssd_device_wait_timeouts and leaves its outputs undefined; the GPU
+ *     context stays usable and later launches are unaffected.
+ */
+m3ssd_status m3ssd_test_set_wait_limit(uint64_t nanoseconds);
+m3ssd_status m3ssd_test_drop_next_gram_signal(void);
 
 /* Static, human-readable name of a status. */
 const char* m3ssd_status_string(m3ssd_status status);

@@ -132,6 +132,10 @@ def load(path: str | None = None):
         lib.m3ssd_abi_version.restype = ctypes.c_int
         lib.m3ssd_device_wait_timeouts.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
         lib.m3ssd_device_wait_timeouts.restype = ctypes.c_int
+        lib.m3ssd_test_set_wait_limit.argtypes = [ctypes.c_uint64]
+        lib.m3ssd_test_set_wait_limit.restype = ctypes.c_int
+        lib.m3ssd_test_drop_next_gram_signal.argtypes = []
+        lib.m3ssd_test_drop_next_gram_signal.restype = ctypes.c_int
         if path is None:
             _lib = lib
         return lib
@@ -167,17 +171,21 @@ def _xdtype(t) -> int:
     raise ValueError(f"X/B/C must be bf16 or fp32, got {t.dtype}")
 
 
-def _need(t, name, dtype=None, shape=None, device=None):
-    if t is None:
-        return
-    if not t.is_cuda:
-        raise ValueError(f"{name} must be a CUDA tensor")
-    if not t.is_contiguous():
-        raise ValueError(f"{name} must be contiguous")
+def _need_shape(t, name, dtype=None, shape=None):
     if dtype is not None and t.dtype != dtype:
         raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
     if shape is not None and tuple(t.shape) != tuple(shape):
         raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _need(t, name, dtype=None, shape=None, device=None):
+    if t is None:
+        return
+    _need_shape(t, name, dtype, shape)
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
     if device is not None and t.device != device:
         raise ValueError(f"{name} is on {t.device}, expected {device}")
 
@@ -187,6 +195,20 @@ def device_wait_timeouts() -> int:
     n = ctypes.c_uint32(0)
     _check(load().m3ssd_device_wait_timeouts(ctypes.byref(n)), "m3ssd_device_wait_timeouts")
     return int(n.value)
+
+
+def set_wait_limit_for_tests(nanoseconds: int):
+    """Testing hook: the chunked forward's bounded waits give up after this many
+    nanoseconds (0 restores the default 2 s).  Synchronous; not while work is
+    in flight."""
+    _check(load().m3ssd_test_set_wait_limit(int(nanoseconds)), "m3ssd_test_set_wait_limit")
+
+
+def drop_next_gram_signal_for_tests():
+    """Testing hook: the next chunked-forward sequence leaves out one completion
+    signal, so one of its bounded waits runs out (reported by
+    device_wait_timeouts; that launch's outputs are undefined)."""
+    _check(load().m3ssd_test_drop_next_gram_signal(), "m3ssd_test_drop_next_gram_signal")
 
 
 def make_dims(batch, seqlen, nheads, headdim, dstate, ngroups, x_dtype, chunk=0, flags=0) -> Dims:
@@ -258,6 +280,46 @@ def bwd_workspace_size(dims: Dims) -> int:
     return int(load().m3ssd_bwd_workspace_size(ctypes.byref(dims)))
 
 
+def _bwd_args(X, logdecay, beta, gamma, B, C, theta, D, h0, dY, dhT, angle0, xprev0, bprev0,
+              grads):
+    """Validates every backward input (dtype, shape, device) and marshals the C
+    arguments shared by :func:`bwd` and :func:`bwd_noalloc`."""
+    import torch
+    b, L, H, P = X.shape
+    G, N = B.shape[2], B.shape[3]
+    dev = X.device
+    f32 = torch.float32
+    xd = X.dtype
+    checks = [(X, "X", None, None), (logdecay, "logdecay", f32, (b, L, H)),
+              (beta, "beta", f32, (b, L, H)), (gamma, "gamma", f32, (b, L, H)),
+              (B, "B", xd, (b, L, G, N)), (C, "C", xd, (b, L, G, N)),
+              (theta, "theta", f32, (b, L, H, N // 2)), (D, "D", f32, (H,)),
+              (h0, "h0", f32, (b, H, N, P)), (angle0, "angle0", f32, (b, H, N // 2)),
+              (xprev0, "xprev0", f32, (b, H, P)), (bprev0, "bprev0", f32, (b, G, N)),
+              (dY, "dY", xd, (b, L, H, P)), (dhT, "dhT", f32, (b, H, N, P))]
+    for t, name, dt, shape in checks:  # every shape and dtype first, then placement
+        if t is not None:
+            _need_shape(t, name, dt, shape)
+    for t, name, dt, shape in checks:
+        _need(t, name, dt, shape, dev)
+    shapes = {"dX": (b, L, H, P), "dlogdecay": (b, L, H), "dbeta": (b, L, H),
+              "dgamma": (b, L, H), "dB": (b, L, G, N), "dC": (b, L, G, N),
+              "dtheta": (b, L, H, N // 2), "dD": (H,), "dh0": (b, H, N, P),
+              "dangle0": (b, H, N // 2), "dxprev0": (b, H, P), "dbprev0": (b, G, N)}
+    if grads is None:
+        grads = {k: torch.empty(v, dtype=f32, device=dev) for k, v in shapes.items()}
+    for k in GRAD_NAMES:
+        _need(grads.get(k), k, f32, shapes[k], dev)
+    gs = BwdGrads(*(None if grads.get(k) is None else grads[k].data_ptr() for k in GRAD_NAMES))
+    extra = None
+    if angle0 is not None or xprev0 is not None or bprev0 is not None:
+        extra = FwdExtra(*(None if t is None else t.data_ptr() for t in (angle0, xprev0, bprev0)),
+                         None, None, None)
+    dims = make_dims(b, L, H, P, N, G, _xdtype(X), 0)
+    ptrs = [_ptr(t) for t in (X, logdecay, beta, gamma, B, C, theta, D, h0)]
+    return dims, ptrs, extra, gs, grads
+
+
 def bwd(X, logdecay, beta, gamma, B, C, theta=None, D=None, h0=None, *, dY, dhT=None,
         angle0=None, xprev0=None, bprev0=None, grads=None, workspace=None):
     """Backward of :func:`fwd` through ``m3ssd_bwd`` on the current CUDA stream.
@@ -268,48 +330,16 @@ def bwd(X, logdecay, beta, gamma, B, C, theta=None, D=None, h0=None, *, dY, dhT=
     ``grads`` supplies them).
     """
     import torch
-    b, L, H, P = X.shape
-    G, N = B.shape[2], B.shape[3]
-    dev = X.device
-    f32 = torch.float32
-    xd = X.dtype
-    _need(X, "X", device=dev)
-    _need(logdecay, "logdecay", f32, (b, L, H), dev)
-    _need(beta, "beta", f32, (b, L, H), dev)
-    _need(gamma, "gamma", f32, (b, L, H), dev)
-    _need(B, "B", xd, (b, L, G, N), dev)
-    _need(C, "C", xd, (b, L, G, N), dev)
-    _need(theta, "theta", f32, (b, L, H, N // 2), dev)
-    _need(D, "D", f32, (H,), dev)
-    _need(h0, "h0", f32, (b, H, N, P), dev)
-    _need(angle0, "angle0", f32, (b, H, N // 2), dev)
-    _need(xprev0, "xprev0", f32, (b, H, P), dev)
-    _need(bprev0, "bprev0", f32, (b, G, N), dev)
-    _need(dY, "dY", xd, (b, L, H, P), dev)
-    _need(dhT, "dhT", f32, (b, H, N, P), dev)
-    shapes = {"dX": (b, L, H, P), "dlogdecay": (b, L, H), "dbeta": (b, L, H),
-              "dgamma": (b, L, H), "dB": (b, L, G, N), "dC": (b, L, G, N),
-              "dtheta": (b, L, H, N // 2), "dD": (H,), "dh0": (b, H, N, P),
-              "dangle0": (b, H, N // 2), "dxprev0": (b, H, P), "dbprev0": (b, G, N)}
-    if grads is None:
-        grads = {k: torch.empty(v, dtype=f32, device=dev) for k, v in shapes.items()}
-    for k in GRAD_NAMES:
-        _need(grads.get(k), k, f32, shapes[k], dev)
-    gs = BwdGrads(*(None if grads.get(k) is None else grads[k].data_ptr() for k in GRAD_NAMES))
-    extra = None
-    if angle0 is not None or xprev0 is not None or bprev0 is not None:
-        extra = FwdExtra(*(None if t is None else t.data_ptr() for t in (angle0, xprev0, bprev0)),
-                         None, None, None)
-    dims = make_dims(b, L, H, P, N, G, _xdtype(X), 0)
+    dims, ptrs, extra, gs, grads = _bwd_args(X, logdecay, beta, gamma, B, C, theta, D, h0, dY,
+                                             dhT, angle0, xprev0, bprev0, grads)
     ws_bytes = bwd_workspace_size(dims)
     if ws_bytes and workspace is None:
-        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
-    st = load().m3ssd_bwd(ctypes.byref(dims), _ptr(X), _ptr(logdecay), _ptr(beta), _ptr(gamma),
-                          _ptr(B), _ptr(C), _ptr(theta), _ptr(D), _ptr(h0),
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=X.device)
+    st = load().m3ssd_bwd(ctypes.byref(dims), *ptrs,
                           None if extra is None else ctypes.byref(extra), _ptr(dY), _ptr(dhT),
                           ctypes.byref(gs), _ptr(workspace),
                           0 if workspace is None else workspace.numel() * workspace.element_size(),
-                          _stream_handle(dev))
+                          _stream_handle(X.device))
     _check(st, "m3ssd_bwd")
     return grads
 
@@ -317,33 +347,13 @@ def bwd(X, logdecay, beta, gamma, B, C, theta=None, D=None, h0=None, *, dY, dhT=
 def bwd_noalloc(X, logdecay, beta, gamma, B, C, theta=None, D=None, h0=None, *, dY,
                 dhT=None, angle0=None, xprev0=None, bprev0=None, grads=None):
     """:func:`bwd` through ``m3ssd_bwd_noalloc`` (scratch inside the library;
-    calls must not overlap).  Returns the same dict of fp32 gradients."""
-    import torch
-    b, L, H, P = X.shape
-    G, N = B.shape[2], B.shape[3]
-    dev = X.device
-    f32 = torch.float32
-    shapes = {"dX": (b, L, H, P), "dlogdecay": (b, L, H), "dbeta": (b, L, H),
-              "dgamma": (b, L, H), "dB": (b, L, G, N), "dC": (b, L, G, N),
-              "dtheta": (b, L, H, N // 2), "dD": (H,), "dh0": (b, H, N, P),
-              "dangle0": (b, H, N // 2), "dxprev0": (b, H, P), "dbprev0": (b, G, N)}
-    for name, t, dt in (("X", X, None), ("dY", dY, X.dtype), ("B", B, X.dtype),
-                        ("C", C, X.dtype), ("dhT", dhT, f32)):
-        _need(t, name, dt, device=dev)
-    if grads is None:
-        grads = {k: torch.empty(v, dtype=f32, device=dev) for k, v in shapes.items()}
-    for k in GRAD_NAMES:
-        _need(grads.get(k), k, f32, shapes[k], dev)
-    gs = BwdGrads(*(None if grads.get(k) is None else grads[k].data_ptr() for k in GRAD_NAMES))
-    extra = None
-    if angle0 is not None or xprev0 is not None or bprev0 is not None:
-        extra = FwdExtra(*(None if t is None else t.data_ptr() for t in (angle0, xprev0, bprev0)),
-                         None, None, None)
-    dims = make_dims(b, L, H, P, N, G, _xdtype(X), 0)
-    st = load().m3ssd_bwd_noalloc(ctypes.byref(dims), _ptr(X), _ptr(logdecay), _ptr(beta),
-                                  _ptr(gamma), _ptr(B), _ptr(C), _ptr(theta), _ptr(D), _ptr(h0),
+    calls must not overlap).  Validates its inputs exactly as :func:`bwd` does
+    and returns the same dict of fp32 gradients."""
+    dims, ptrs, extra, gs, grads = _bwd_args(X, logdecay, beta, gamma, B, C, theta, D, h0, dY,
+                                             dhT, angle0, xprev0, bprev0, grads)
+    st = load().m3ssd_bwd_noalloc(ctypes.byref(dims), *ptrs,
                                   None if extra is None else ctypes.byref(extra), _ptr(dY),
-                                  _ptr(dhT), ctypes.byref(gs), _stream_handle(dev))
+                                  _ptr(dhT), ctypes.byref(gs), _stream_handle(X.device))
     _check(st, "m3ssd_bwd_noalloc")
     return grads
 

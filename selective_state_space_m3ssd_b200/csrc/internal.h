@@ -142,15 +142,11 @@ bool fwd_chunk_supported(const FwdArgs& a);
 // Count of bounded device-side waits in the chunked forward that ran out since
 // the last call; reading it synchronises the device and clears the count.
 cudaError_t read_and_clear_wait_timeouts(unsigned int* count);
-// Chunk-parallel bf16 tensor-core forward (N = 128, P = 64): chunks of one
-// sequence run on any CTA and pass the fp32 state through a ring in the
-// workspace.  fwd_cp_shape_ok is the part of the test that depends on the dims
-// only (it sizes the workspace); fwd_cp_supported adds pointers and layouts.
-bool fwd_cp_shape_ok(const FwdArgs& a);
-bool fwd_cp_supported(const FwdArgs& a);
-size_t fwd_cp_workspace_bytes(int64_t b, int64_t H);
-cudaError_t launch_fwd_cp(const FwdArgs& a, void* workspace, cudaStream_t s);
-cudaError_t read_and_clear_cp_wait_timeouts(unsigned int* count);
+// Test settings of the chunked forward (synchronous copies to device symbols):
+// the limit of its bounded waits (0 = 2 s), and a one-shot request that the
+// next chunk walk drop its first Gram completion signal.
+cudaError_t set_wait_limit_ns(unsigned long long ns);
+cudaError_t request_dropped_gram_signal();
 // Decode step (two launches: the state/outputs, then b_prev <- B_t).
 cudaError_t launch_step(const StepArgs& a, cudaStream_t s);
 

@@ -61,21 +61,24 @@ const char* m3ssd_status_string(m3ssd_status s) {
 
 m3ssd_status m3ssd_device_wait_timeouts(uint32_t* count) {
   if (!count) return M3SSD_ERR_INVALID_ARG;
-  unsigned int n = 0, nb = 0, ncp = 0;
+  unsigned int n = 0, nb = 0;
   m3ssd_status st = from_cuda(m3ssd::read_and_clear_wait_timeouts(&n));
   if (st == M3SSD_OK) st = from_cuda(m3ssd::read_and_clear_bwd_wait_timeouts(&nb));
-  if (st == M3SSD_OK) st = from_cuda(m3ssd::read_and_clear_cp_wait_timeouts(&ncp));
-  *count = n + nb + ncp;
+  *count = n + nb;
   return st;
 }
 
+m3ssd_status m3ssd_test_set_wait_limit(uint64_t nanoseconds) {
+  return from_cuda(m3ssd::set_wait_limit_ns(nanoseconds));
+}
+
+m3ssd_status m3ssd_test_drop_next_gram_signal(void) {
+  return from_cuda(m3ssd::request_dropped_gram_signal());
+}
+
 size_t m3ssd_fwd_workspace_size(const m3ssd_dims* dims) {
-  if (check_dims(dims) != M3SSD_OK) return 0;
-  m3ssd::FwdArgs a{};
-  a.b = dims->batch; a.L = dims->seqlen; a.H = dims->nheads; a.P = dims->headdim;
-  a.N = dims->dstate; a.G = dims->ngroups; a.chunk = dims->chunk;
-  a.bf16 = dims->x_dtype == M3SSD_BF16;
-  return m3ssd::fwd_cp_shape_ok(a) ? m3ssd::fwd_cp_workspace_bytes(a.b, a.H) : 0;
+  (void)dims;
+  return 0;
 }
 
 m3ssd_status m3ssd_fwd(const m3ssd_dims* dims, const void* X, const float* logdecay,
@@ -116,13 +119,11 @@ m3ssd_status m3ssd_fwd(const m3ssd_dims* dims, const void* X, const float* logde
   if (workspace_bytes < need || (need > 0 && (!workspace || !aligned(workspace, 256))))
     return M3SSD_ERR_WORKSPACE;
 
-  const bool parallel = m3ssd::fwd_cp_supported(a);
-  const bool chunked = !parallel && m3ssd::fwd_chunk_supported(a);
-  if (!parallel && !chunked && !general_shape_ok(dims)) return M3SSD_ERR_UNSUPPORTED;
+  const bool chunked = m3ssd::fwd_chunk_supported(a);
+  if (!chunked && !general_shape_ok(dims)) return M3SSD_ERR_UNSUPPORTED;
   if (dims->batch == 0) return M3SSD_OK;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (parallel) return from_cuda(m3ssd::launch_fwd_cp(a, workspace, s));
   return from_cuda(chunked ? m3ssd::launch_fwd_chunk(a, s) : m3ssd::launch_fwd_seq(a, s));
 }
 

@@ -19,20 +19,18 @@ from tests.test_gpu_seq_step import with_cache_inputs
 
 pytestmark = pytest.mark.gpu
 TOL = 2e-2
-# Scan-only outputs (D absent) are heavy tailed (max/RMS up to ~50) and their
-# rounding error is set by the bf16 rounding of the rotated B and C before the
-# Gram product, amplified by cancellation in its 128-term dot products (an
-# emulation of those roundings alone gives the same ~1.7e-2 RMS error at L = 1).
-# They are held to an RMS bound and a looser max bound.
-TOL_SCAN_RMS, TOL_SCAN_MAX = 2e-2, 1.5e-1
+# Scan-only outputs (D absent) are heavy tailed (max/RMS up to ~50); they are
+# held to the same max bound as every other output.  The kernel's fp16 tensor-core
+# operands keep their error near 2^-12 of the large diagonal terms (bf16 rotated
+# operands, 2^-9, gave a max error of about 5e-2 of the RMS here).
 
 
 def check_y(got, ref, with_D):
-    if with_D:
-        assert rel_max_err_out(got, ref, True) <= TOL
-    else:
-        assert rms_rel_err(got, ref) <= TOL_SCAN_RMS
-        assert rel_max_err_out(got, ref, True) <= TOL_SCAN_MAX
+    assert rel_max_err_out(got, ref, True) <= TOL
+    if not with_D:
+        assert rms_rel_err(got, ref) <= TOL
+
+
 BASE = WORKLOADS["siso"].with_(batch=2, nheads=3, seed=321)
 
 

@@ -158,6 +158,48 @@ def test_decode_workload_prefill_then_1000_steps_sampled():
         np.testing.assert_array_equal(np64(cache["b_prev"][bi:bi + 1]), ref["bprevT"])
 
 
+def test_decode_workload_1000_steps_replayed_from_a_cuda_graph():
+    """The decode workload as the benchmark runs it: the 1000 m3ssd_step calls
+    captured in one CUDA graph (per-step inputs staged time-major so every step
+    reads contiguous tensors) and replayed once after the 512-token prefill;
+    sampled (b, h) outputs and the final cache against the oracle over the same
+    1512 tokens ("mamba-rs" crate page, feature list: CUDA Graph capture of the
+    inference step)."""
+    from selective_state_space_m3ssd_b200.synth import DECODE_PREFILL, DECODE_STEPS, slice_inputs
+    w = WORKLOADS["decode"]
+    inp = make_inputs(w, device="cuda")
+    Lp = DECODE_PREFILL
+    keys = ("X", "logdecay", "beta", "gamma", "B", "C", "theta")
+    Y, hT, cache = m3.fwd(*(inp[k][:, :Lp].contiguous() for k in keys), inp["D"], None,
+                          want_cache=True)
+    cache["ssm"] = hT
+    steps = {k: inp[k][:, Lp:].transpose(0, 1).contiguous() for k in keys}  # (T, b, ...)
+    ys = torch.empty(DECODE_STEPS, w.batch, w.nheads, w.headdim, device="cuda")
+    # one eager step on a copy first: the library's one-time launch set-up stays
+    # out of the capture
+    scratch = {k: v.clone() for k, v in cache.items()}
+    m3.step(scratch, *(steps[k][0] for k in keys), inp["D"], y_t=torch.empty_like(ys[0]))
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for t in range(DECODE_STEPS):
+            m3.step(cache, *(steps[k][t] for k in keys), inp["D"], y_t=ys[t])
+    g.replay()
+    torch.cuda.synchronize()
+    del g
+    cpu = {k: (None if v is None else v.cpu()) for k, v in inp.items()}
+    pairs = {3: [1, 30], 200: [12]}
+    for bi, heads in pairs.items():
+        ref = oracle.oracle_fwd(**slice_inputs(cpu, b=bi, heads=heads))
+        got_y = np.concatenate([np64(Y[bi:bi + 1][:, :, heads]),
+                                np64(ys[:, bi:bi + 1][:, :, heads].transpose(0, 1))], axis=1)
+        assert rel_max_err(got_y, ref["Y"]) <= TOL_F32
+        assert rel_max_err(np64(cache["ssm"][bi:bi + 1][:, heads]), ref["hT"]) <= TOL_F32
+        assert angle_err(np64(cache["angle"][bi:bi + 1][:, heads]), ref["angleT"]) <= 1e-4
+        np.testing.assert_array_equal(np64(cache["x_prev"][bi:bi + 1][:, heads]), ref["xprevT"])
+        np.testing.assert_array_equal(np64(cache["b_prev"][bi:bi + 1]), ref["bprevT"])
+
+
 # The largest state the sequential kernels keep in one CTA: N * P = 16384 with
 # N, P <= 256 (the three corners), forward with cache in and out, then decode
 # steps from the forward's cache, each against the oracle.

@@ -650,10 +650,26 @@ def run_ours(args):
         torch.distributed.barrier()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(fw["inp"])
+    # a compact summary of every figure last, so that a tail of the line shows them
+    line["summary"] = summary_of(line)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.destroy_process_group()
+
+
+def summary_of(line: dict) -> dict:
+    """Value, unit and roofline fraction of the headline and of each side figure."""
+    def one(d):
+        if not d:
+            return None
+        r = d.get("roofline") or {}
+        return {"value": round(d["value"], 3), "unit": d["unit"],
+                "ms_per_step": round(d["ms_per_step"], 4), "frac": round(r.get("frac", 0.0), 3)}
+    out = {"forward_siso": one(line)}
+    for k in ("ssd_forward", "long_forward", "backward", "block", "mimo_decode", "decode"):
+        out[k] = one(line.get(k))
+    return out
 
 
 # ----------------------------------------------------------------------------
@@ -705,11 +721,29 @@ def run_profile(args):
     m3build.build()
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
-    if args.profile == "forward":
-        w = WORKLOADS[FWD_KEY].with_(batch=2)
+    if args.profile in ("forward", "forward8"):
+        # batch 2 (146 MB of inputs, above L2): a small case for full-section
+        # captures; batch 8: the benchmark's own launch, for one-pass counters
+        w = WORKLOADS[FWD_KEY].with_(batch=2) if args.profile == "forward" else WORKLOADS[FWD_KEY]
         fw = bench_forward(w, dev, args.steps, args.warmup, 1, 0)
-        print(json.dumps({"profile": "forward", "workload": w.name.replace("b8", "b2"),
+        print(json.dumps({"profile": args.profile, "workload": w.name.replace(
+                              "b8", "b2" if args.profile == "forward" else "b8"),
                           "ms_per_step": fw["ms_per_step"], "launches": fw["launches"]}))
+    elif args.profile == "decode":
+        # decode steps at half the decode batch: b128, fp32 cache (134 MB of
+        # state, above L2), one step kernel and one b_prev update per call
+        w = WORKLOADS["decode"].with_(batch=128, seqlen=args.warmup + args.steps)
+        inp = make_inputs(w, device=dev)
+        b, H, P, N, G = w.batch, w.nheads, w.headdim, w.dstate, w.ngroups
+        cache = m3.new_cache(b, H, P, N, G, dev)
+        cache["ssm"].normal_(0, 0.3, generator=torch.Generator(device=dev).manual_seed(5))
+        keys = ("X", "logdecay", "beta", "gamma", "B", "C", "theta")
+        steps = {k: inp[k].transpose(0, 1).contiguous() for k in keys}
+        y = torch.empty_like(steps["X"][0])
+        for t in range(args.warmup + args.steps):
+            m3.step(cache, *(steps[k][t] for k in keys), inp["D"], y_t=y)
+        torch.cuda.synchronize(dev)
+        print(json.dumps({"profile": "decode", "workload": f"decode b{b} H{H} P{P} N{N} fp32 cache"}))
     elif args.profile == "backward":
         # one batch row of the forward's workload at L = 1024: 32 (b, h) CTAs of
         # the chunked backward
@@ -776,7 +810,8 @@ def main():
                     help="skip the forward on the ssd and long workloads (side figures)")
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="omit the oracle timing (it never runs inside a GPU timed region)")
-    ap.add_argument("--profile", choices=["forward", "block", "backward", "mimo"],
+    ap.add_argument("--profile", choices=["forward", "forward8", "decode", "block", "backward",
+                                          "mimo"],
                     help="run only a small case of one kernel family (for ncu captures)")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -69,13 +69,22 @@ typedef enum {
   M3SSD_ERR_UNSUPPORTED = 2,  /* valid request outside what this build implements (sizes, chunk, flags) */
   M3SSD_ERR_WORKSPACE = 3,    /* workspace smaller than m3ssd_fwd_workspace_size() or misaligned */
   M3SSD_ERR_CUDA = 4,         /* a CUDA launch failed */
-  M3SSD_ERR_NONFINITE = 5,    /* reserved: non-finite input found by the optional check */
+  M3SSD_ERR_NONFINITE = 5,    /* m3ssd_nonfinite_outputs: a checked output held NaN or infinity */
   M3SSD_ERR_TIMEOUT = 6       /* reserved: a bounded device-side wait ran out */
 } m3ssd_status;
 
 typedef enum { M3SSD_F32 = 0, M3SSD_BF16 = 1 } m3ssd_dtype;
 
-/* flags (m3ssd_dims.flags); no flag is defined yet -- pass 0. */
+/* flags (m3ssd_dims.flags) */
+/* M3SSD_CHECK_FINITE: after its kernels, m3ssd_fwd (and m3ssd_step,
+ * m3ssd_mimo_fwd, m3ssd_mimo_step) scans the outputs it wrote -- Y and hT, or
+ * y_t -- on the same stream for NaN or infinite values (from an input that was,
+ * or from an intermediate that overflowed, e.g. a bf16 input beyond fp16's range
+ * on the chunked path); m3ssd_nonfinite_outputs reports what the checks found.
+ * It reads the outputs once more (about a fifth of the forward's bytes).  The
+ * backward does not take the flag (M3SSD_ERR_UNSUPPORTED).  "Crate burn_mamba"
+ * carries the same switch (DENY_NAN / DENY_INF). */
+#define M3SSD_CHECK_FINITE 1u
 
 typedef struct {
   int64_t batch;    /* b >= 0 */
@@ -86,7 +95,7 @@ typedef struct {
   int64_t ngroups;  /* G >= 1, H % G == 0 */
   int32_t chunk;    /* chunk length of the chunked forward: 0 = library choice, else 64 */
   int32_t x_dtype;  /* m3ssd_dtype of X, B, C, Y (and x_t, B_t, C_t, y_t) */
-  uint32_t flags;   /* must be 0 */
+  uint32_t flags;   /* 0 or M3SSD_CHECK_FINITE */
   uint32_t reserved;/* must be 0 */
 } m3ssd_dims;
 
@@ -210,7 +219,8 @@ typedef struct {
 } m3ssd_bwd_grads;
 
 /* Bytes of device workspace m3ssd_bwd needs for these dims (0 for invalid
- * dims); the size depends on the path.  At N = 128, P = 64 it holds every
+ * dims, and for any flags, which the backward refuses); the size depends on
+ * the path.  At N = 128, P = 64 it holds every
  * chunk-start state and angle (chunks of 63 tokens) and per-head shares of
  * the group-summed gradients: about 4 (b H ceil(L/63) (N P + N/2) +
  * 2 b L H N) bytes.  Other shapes keep a state checkpoint every 16 or 64
@@ -242,8 +252,9 @@ size_t m3ssd_bwd_workspace_size(const m3ssd_dims* dims);
  * gradients afterwards; other shapes run one CTA per sequence token by
  * token.  Every sum (over slices, the heads of a group, the batch) runs in a
  * fixed order, so results are deterministic.  Limits as the sequential forward:
- * N <= 256, P <= 256, N*P <= 16384 (else M3SSD_ERR_UNSUPPORTED).  workspace
- * must hold m3ssd_bwd_workspace_size(dims) bytes, 256-byte aligned (else
+ * N <= 256, P <= 256, N*P <= 16384 (else M3SSD_ERR_UNSUPPORTED); dims->flags
+ * must be 0 (else M3SSD_ERR_UNSUPPORTED).  workspace must hold
+ * m3ssd_bwd_workspace_size(dims) bytes, 256-byte aligned (else
  * M3SSD_ERR_WORKSPACE); the size depends on the path.  No allocation, no
  * synchronisation.
  */
@@ -389,6 +400,13 @@ m3ssd_status m3ssd_device_wait_timeouts(uint32_t* count);
  */
 m3ssd_status m3ssd_test_set_wait_limit(uint64_t nanoseconds);
 m3ssd_status m3ssd_test_drop_next_gram_signal(void);
+
+/* The result of the M3SSD_CHECK_FINITE checks enqueued since the last call:
+ * M3SSD_ERR_NONFINITE if any checked output held a NaN or an infinity, else
+ * M3SSD_OK; the record is then cleared.  It synchronises the current device
+ * and must not be captured in a CUDA graph; M3SSD_ERR_CUDA if the device
+ * cannot be read. */
+m3ssd_status m3ssd_nonfinite_outputs(void);
 
 /* Static, human-readable name of a status. */
 const char* m3ssd_status_string(m3ssd_status status);

@@ -16,7 +16,7 @@ The block, in the order the pages give it ("VikramLex/mamba3-minimal" README,
   3. the trapezoidal scan (the SISO recurrence of ``oracle_fwd``), with D x;
   4. y * SiLU(z), then out_proj.
 
-Readings where the pages are silent (each is listed in the design notes):
+Readings where the pages are silent (each one stated in full below):
   - in_proj and out_proj are bias-free linear maps; the block's ``bias=True``
     is the BC bias, which replaces the removed short convolution ("TorchMamba"
     README, "Math notes", M3 SISO);

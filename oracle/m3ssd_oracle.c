@@ -24,7 +24,7 @@
  *     path (no previous-step contribution); theta absent is the real-only path;
  *     H % G == 0; N even.
  *
- * Readings where the pages are silent (each is listed in the design notes):
+ * Readings where the pages are silent (each one stated in full below):
  *   - pairs are adjacent components (2i, 2i+1), rotated by the i-th angle;
  *   - the rotation is counter-clockwise, [[cos, -sin], [sin, cos]], applied to
  *     both B and C;

@@ -18,6 +18,7 @@ LIB_PATH = os.path.join(_HERE, "libm3ssd.so")
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_NONFINITE, ERR_TIMEOUT = range(7)
 F32, BF16 = 0, 1
+CHECK_FINITE = 1  # m3ssd_dims.flags: scan the outputs for NaN / infinity
 
 _lib = None
 _lock = threading.Lock()
@@ -132,6 +133,8 @@ def load(path: str | None = None):
         lib.m3ssd_abi_version.restype = ctypes.c_int
         lib.m3ssd_device_wait_timeouts.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
         lib.m3ssd_device_wait_timeouts.restype = ctypes.c_int
+        lib.m3ssd_nonfinite_outputs.argtypes = []
+        lib.m3ssd_nonfinite_outputs.restype = ctypes.c_int
         lib.m3ssd_test_set_wait_limit.argtypes = [ctypes.c_uint64]
         lib.m3ssd_test_set_wait_limit.restype = ctypes.c_int
         lib.m3ssd_test_drop_next_gram_signal.argtypes = []
@@ -197,6 +200,16 @@ def device_wait_timeouts() -> int:
     return int(n.value)
 
 
+def nonfinite_outputs() -> bool:
+    """Whether any output checked under CHECK_FINITE since the last call held a
+    NaN or an infinity (synchronises; clears the record)."""
+    st = load().m3ssd_nonfinite_outputs()
+    if st == ERR_NONFINITE:
+        return True
+    _check(st, "m3ssd_nonfinite_outputs")
+    return False
+
+
 def set_wait_limit_for_tests(nanoseconds: int):
     """Testing hook: the chunked forward's bounded waits give up after this many
     nanoseconds (0 restores the default 2 s).  Synchronous; not while work is
@@ -221,12 +234,13 @@ def fwd_workspace_size(dims: Dims) -> int:
 
 def fwd(X, logdecay, beta, gamma, B, C, theta=None, D=None, h0=None, *, Y=None,
         want_hT: bool = True, hT=None, angle0=None, xprev0=None, bprev0=None,
-        want_cache: bool = False, chunk: int = 0, workspace=None):
+        want_cache: bool = False, chunk: int = 0, workspace=None, check_finite: bool = False):
     """Forward scan through ``m3ssd_fwd`` on the current CUDA stream.
 
     Shapes as in ``include/m3ssd.h``.  Returns ``(Y, hT, cache_out)`` where
     ``cache_out`` is a dict with angleT/xprevT/bprevT when ``want_cache``.
-    Output tensors are allocated by torch unless passed in.
+    Output tensors are allocated by torch unless passed in.  ``check_finite``
+    sets CHECK_FINITE (see :func:`nonfinite_outputs`).
     """
     import torch
     b, L, H, P = X.shape
@@ -263,7 +277,7 @@ def fwd(X, logdecay, beta, gamma, B, C, theta=None, D=None, h0=None, *, Y=None,
             *(None if t is None else t.data_ptr() for t in (angle0, xprev0, bprev0)),
             *(None if cache_out is None else cache_out[k].data_ptr()
               for k in ("angle", "x_prev", "b_prev")))
-    dims = make_dims(b, L, H, P, N, G, _xdtype(X), chunk)
+    dims = make_dims(b, L, H, P, N, G, _xdtype(X), chunk, CHECK_FINITE if check_finite else 0)
     ws_bytes = fwd_workspace_size(dims)
     if ws_bytes and workspace is None:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
@@ -369,9 +383,10 @@ def new_cache(batch, nheads, headdim, dstate, ngroups, device):
 
 
 def step(cache: dict, x_t, logdecay_t, beta_t, gamma_t, B_t, C_t, theta_t=None, D=None, *,
-         y_t=None):
+         y_t=None, check_finite: bool = False):
     """One decode step through ``m3ssd_step``; updates ``cache`` in place and
-    returns y_t (b, H, P) in the dtype of x_t."""
+    returns y_t (b, H, P) in the dtype of x_t.  ``check_finite`` sets
+    CHECK_FINITE on y_t (see :func:`nonfinite_outputs`)."""
     import torch
     b, H, P = x_t.shape
     G, N = B_t.shape[1], B_t.shape[2]
@@ -395,7 +410,7 @@ def step(cache: dict, x_t, logdecay_t, beta_t, gamma_t, B_t, C_t, theta_t=None, 
     _need(y_t, "y_t", xd, (b, H, P), dev)
     c = Cache(cache["angle"].data_ptr(), cache["ssm"].data_ptr(), cache["x_prev"].data_ptr(),
               cache["b_prev"].data_ptr())
-    dims = make_dims(b, 1, H, P, N, G, _xdtype(x_t))
+    dims = make_dims(b, 1, H, P, N, G, _xdtype(x_t), 0, CHECK_FINITE if check_finite else 0)
     st = load().m3ssd_step(ctypes.byref(dims), _ptr(x_t), _ptr(logdecay_t), _ptr(beta_t),
                            _ptr(gamma_t), _ptr(B_t), _ptr(C_t), _ptr(theta_t), _ptr(D),
                            ctypes.byref(c), _ptr(y_t), _stream_handle(dev))
@@ -405,7 +420,7 @@ def step(cache: dict, x_t, logdecay_t, beta_t, gamma_t, B_t, C_t, theta_t=None, 
 
 def mimo_fwd(X, logdecay, beta, gamma, B, C, theta=None, D=None, h0=None, *, Y=None,
              want_hT: bool = True, angle0=None, xprev0=None, bprev0=None,
-             want_cache: bool = False):
+             want_cache: bool = False, check_finite: bool = False):
     """MIMO rank-R forward through ``m3ssd_mimo_fwd``: X (b,L,H,P,R), B, C
     (b,L,G,N,R).  Returns ``(Y, hT, cache_out)`` like :func:`fwd`, with the
     cache's x_prev (b,H,P,R) and b_prev (b,G,N,R)."""
@@ -436,7 +451,7 @@ def mimo_fwd(X, logdecay, beta, gamma, B, C, theta=None, D=None, h0=None, *, Y=N
             *(None if t is None else t.data_ptr() for t in (angle0, xprev0, bprev0)),
             *(None if cache_out is None else cache_out[k].data_ptr()
               for k in ("angle", "x_prev", "b_prev")))
-    dims = make_dims(b, L, H, P, N, G, _xdtype(X), 0)
+    dims = make_dims(b, L, H, P, N, G, _xdtype(X), 0, CHECK_FINITE if check_finite else 0)
     st = load().m3ssd_mimo_fwd(ctypes.byref(dims), R, _ptr(X), _ptr(logdecay), _ptr(beta),
                                _ptr(gamma), _ptr(B), _ptr(C), _ptr(theta), _ptr(D), _ptr(h0),
                                _ptr(Y), _ptr(hT), None if extra is None else ctypes.byref(extra),
@@ -456,7 +471,7 @@ def new_mimo_cache(batch, nheads, headdim, dstate, ngroups, rank, device):
 
 
 def mimo_step(cache: dict, x_t, logdecay_t, beta_t, gamma_t, B_t, C_t, theta_t=None, D=None, *,
-              y_t=None):
+              y_t=None, check_finite: bool = False):
     """One MIMO decode step through ``m3ssd_mimo_step``: x_t (b,H,P,R), B_t, C_t
     (b,G,N,R); updates ``cache`` in place and returns y_t (b,H,P,R)."""
     import torch
@@ -477,7 +492,7 @@ def mimo_step(cache: dict, x_t, logdecay_t, beta_t, gamma_t, B_t, C_t, theta_t=N
     _need(y_t, "y_t", xd, (b, H, P, R), dev)
     c = Cache(cache["angle"].data_ptr(), cache["ssm"].data_ptr(), cache["x_prev"].data_ptr(),
               cache["b_prev"].data_ptr())
-    dims = make_dims(b, 1, H, P, N, G, _xdtype(x_t))
+    dims = make_dims(b, 1, H, P, N, G, _xdtype(x_t), 0, CHECK_FINITE if check_finite else 0)
     st = load().m3ssd_mimo_step(ctypes.byref(dims), R, _ptr(x_t), _ptr(logdecay_t), _ptr(beta_t),
                                 _ptr(gamma_t), _ptr(B_t), _ptr(C_t), _ptr(theta_t), _ptr(D),
                                 ctypes.byref(c), _ptr(y_t), _stream_handle(dev))

@@ -147,6 +147,11 @@ cudaError_t read_and_clear_wait_timeouts(unsigned int* count);
 // next chunk walk drop its first Gram completion signal.
 cudaError_t set_wait_limit_ns(unsigned long long ns);
 cudaError_t request_dropped_gram_signal();
+// The optional non-finite check: scans n elements (bf16 or fp32) at p on the
+// stream and sets a device word when one is NaN or infinite; the host query
+// reads and clears it (synchronising the device).
+cudaError_t launch_nonfinite_check(const void* p, int64_t n, bool bf16, cudaStream_t s);
+cudaError_t read_and_clear_nonfinite(unsigned int* flag);
 // Decode step (two launches: the state/outputs, then b_prev <- B_t).
 cudaError_t launch_step(const StepArgs& a, cudaStream_t s);
 

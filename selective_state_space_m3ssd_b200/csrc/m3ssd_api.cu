@@ -23,7 +23,7 @@ m3ssd_status check_dims(const m3ssd_dims* d) {
   if (d->nheads % d->ngroups != 0) return M3SSD_ERR_INVALID_ARG;
   if (d->x_dtype != M3SSD_F32 && d->x_dtype != M3SSD_BF16) return M3SSD_ERR_INVALID_ARG;
   if (d->reserved != 0) return M3SSD_ERR_INVALID_ARG;
-  if (d->flags != 0) return M3SSD_ERR_UNSUPPORTED;
+  if ((d->flags & ~(uint32_t)M3SSD_CHECK_FINITE) != 0) return M3SSD_ERR_UNSUPPORTED;
   if (d->batch * d->nheads > INT32_MAX) return M3SSD_ERR_UNSUPPORTED;
   return M3SSD_OK;
 }
@@ -57,6 +57,13 @@ const char* m3ssd_status_string(m3ssd_status s) {
     case M3SSD_ERR_TIMEOUT: return "device-side wait timed out";
   }
   return "unknown status";
+}
+
+m3ssd_status m3ssd_nonfinite_outputs(void) {
+  unsigned int f = 0;
+  const m3ssd_status st = from_cuda(m3ssd::read_and_clear_nonfinite(&f));
+  if (st != M3SSD_OK) return st;
+  return f ? M3SSD_ERR_NONFINITE : M3SSD_OK;
 }
 
 m3ssd_status m3ssd_device_wait_timeouts(uint32_t* count) {
@@ -124,7 +131,15 @@ m3ssd_status m3ssd_fwd(const m3ssd_dims* dims, const void* X, const float* logde
   if (dims->batch == 0) return M3SSD_OK;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return from_cuda(chunked ? m3ssd::launch_fwd_chunk(a, s) : m3ssd::launch_fwd_seq(a, s));
+  st = from_cuda(chunked ? m3ssd::launch_fwd_chunk(a, s) : m3ssd::launch_fwd_seq(a, s));
+  if (st == M3SSD_OK && (dims->flags & M3SSD_CHECK_FINITE)) {
+    st = from_cuda(m3ssd::launch_nonfinite_check(
+        Y, dims->batch * dims->seqlen * dims->nheads * dims->headdim, bf16, s));
+    if (st == M3SSD_OK && hT)
+      st = from_cuda(m3ssd::launch_nonfinite_check(
+          hT, dims->batch * dims->nheads * dims->dstate * dims->headdim, false, s));
+  }
+  return st;
 }
 
 m3ssd_status m3ssd_mimo_fwd(const m3ssd_dims* dims, int32_t rank, const void* X,
@@ -161,7 +176,16 @@ m3ssd_status m3ssd_mimo_fwd(const m3ssd_dims* dims, int32_t rank, const void* X,
   a.N = dims->dstate; a.G = dims->ngroups; a.bf16 = bf16;
   a.X = X; a.logdecay = logdecay; a.beta = beta; a.gamma = gamma; a.B = B; a.C = C;
   a.theta = theta; a.D = D; a.h0 = h0; a.Y = Y; a.hT = hT;
-  return from_cuda(m3ssd::launch_mimo_fwd(a, rank, static_cast<cudaStream_t>(stream)));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  m3ssd_status rs = from_cuda(m3ssd::launch_mimo_fwd(a, rank, s));
+  if (rs == M3SSD_OK && (dims->flags & M3SSD_CHECK_FINITE)) {
+    rs = from_cuda(m3ssd::launch_nonfinite_check(
+        Y, dims->batch * dims->seqlen * dims->nheads * dims->headdim * rank, bf16, s));
+    if (rs == M3SSD_OK && hT)
+      rs = from_cuda(m3ssd::launch_nonfinite_check(
+          hT, dims->batch * dims->nheads * dims->dstate * dims->headdim, false, s));
+  }
+  return rs;
 }
 
 m3ssd_status m3ssd_mimo_step(const m3ssd_dims* dims, int32_t rank, const void* x_t,
@@ -194,11 +218,18 @@ m3ssd_status m3ssd_mimo_step(const m3ssd_dims* dims, int32_t rank, const void* x
   a.B_t = B_t; a.C_t = C_t; a.theta_t = theta_t; a.D = D;
   a.angle = cache->angle; a.ssm = cache->ssm; a.x_prev = cache->x_prev; a.b_prev = cache->b_prev;
   a.y_t = y_t;
-  return from_cuda(m3ssd::launch_mimo_step(a, rank, static_cast<cudaStream_t>(stream)));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  m3ssd_status rs = from_cuda(m3ssd::launch_mimo_step(a, rank, s));
+  if (rs == M3SSD_OK && (dims->flags & M3SSD_CHECK_FINITE))
+    rs = from_cuda(m3ssd::launch_nonfinite_check(
+        y_t, dims->batch * dims->nheads * dims->headdim * rank, bf16, s));
+  return rs;
 }
 
 size_t m3ssd_bwd_workspace_size(const m3ssd_dims* dims) {
-  if (check_dims(dims) != M3SSD_OK || !general_shape_ok(dims)) return 0;
+  // The backward takes no flags: a flagged request needs nothing (m3ssd_bwd
+  // refuses it).
+  if (check_dims(dims) != M3SSD_OK || !general_shape_ok(dims) || dims->flags != 0) return 0;
   if (m3ssd::bwd_chunk_supported(dims->dstate, dims->headdim))
     return m3ssd::bwd_chunk_workspace_bytes(dims->batch, dims->seqlen, dims->nheads);
   if (m3ssd::bwd_split_supported(dims->dstate, dims->headdim))
@@ -216,7 +247,7 @@ m3ssd_status m3ssd_bwd(const m3ssd_dims* dims, const void* X, const float* logde
                        void* stream) {
   m3ssd_status st = check_dims(dims);
   if (st != M3SSD_OK) return st;
-  if (!general_shape_ok(dims)) return M3SSD_ERR_UNSUPPORTED;
+  if (!general_shape_ok(dims) || dims->flags != 0) return M3SSD_ERR_UNSUPPORTED;
   if (!grads) return M3SSD_ERR_INVALID_ARG;
   const bool bf16 = dims->x_dtype == M3SSD_BF16;
   const uintptr_t esz = bf16 ? 2 : 4;
@@ -288,7 +319,12 @@ m3ssd_status m3ssd_step(const m3ssd_dims* dims, const void* x_t, const float* lo
   a.B_t = B_t; a.C_t = C_t; a.theta_t = theta_t; a.D = D;
   a.angle = cache->angle; a.ssm = cache->ssm; a.x_prev = cache->x_prev; a.b_prev = cache->b_prev;
   a.y_t = y_t;
-  return from_cuda(m3ssd::launch_step(a, static_cast<cudaStream_t>(stream)));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  st = from_cuda(m3ssd::launch_step(a, s));
+  if (st == M3SSD_OK && (dims->flags & M3SSD_CHECK_FINITE))
+    st = from_cuda(m3ssd::launch_nonfinite_check(
+        y_t, dims->batch * dims->nheads * dims->headdim, bf16, s));
+  return st;
 }
 
 }  // extern "C"

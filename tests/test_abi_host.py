@@ -85,7 +85,7 @@ def _fwd(lib, dims, X=FAKE, ld=FAKE, beta=None, gamma=FAKE, B=FAKE, C=FAKE, thet
     (dict(batch=-1), m3.ERR_INVALID_ARG),
     (dict(seqlen=-5), m3.ERR_INVALID_ARG),
     (dict(x_dtype=7), m3.ERR_INVALID_ARG),
-    (dict(flags=1), m3.ERR_UNSUPPORTED),
+    (dict(flags=2), m3.ERR_UNSUPPORTED),
     (dict(chunk=48), m3.ERR_UNSUPPORTED),
     (dict(dstate=512), m3.ERR_UNSUPPORTED),
     (dict(headdim=300), m3.ERR_UNSUPPORTED),
@@ -235,3 +235,11 @@ def test_block_validation(lib):
     assert step(cache=m3.Cache(0x10000, 0x10000, None, 0x10000)) == m3.ERR_INVALID_ARG
     assert step(ws_bytes=16) == m3.ERR_WORKSPACE
     assert step(dims=_block_dims(batch=0)) == m3.OK
+
+
+def test_backward_refuses_the_finite_check_flag(lib):
+    d = _dims(flags=m3.CHECK_FINITE)
+    g = m3.BwdGrads(*([0x10000] * 12))
+    st = lib.m3ssd_bwd(ctypes.byref(d), FAKE, FAKE, None, FAKE, FAKE, FAKE, None, None, None,
+                       None, FAKE, None, ctypes.byref(g), None, 0, None)
+    assert st == m3.ERR_UNSUPPORTED

@@ -42,7 +42,8 @@ if ROOT not in sys.path:
 import torch  # noqa: E402
 
 from selective_state_space_m3ssd_b200.synth import (  # noqa: E402
-    DECODE_PREFILL, DECODE_STEPS, WORKLOADS, make_inputs, rank_workload, slice_inputs)
+    DECODE_PREFILL, DECODE_STEPS, MIMO_WORKLOADS, WORKLOADS, make_inputs, make_mimo_inputs,
+    rank_workload, slice_inputs)
 
 METRIC = "scan Mtokens/s (fwd, L=4096)"
 UNIT = "Mtokens/s"
@@ -247,6 +248,54 @@ def forward_leg(key, dev, steps, warmup, world, rank, peaks):
                         "peak_source": peaks["source"]},
            "gpu_launches": fw["launches"]}
     del fw
+    torch.cuda.empty_cache()
+    return out
+
+
+def mimo_forward_leg(dev, steps, warmup, world, rank, peaks):
+    """The rank-4 MIMO prefill (m3ssd_mimo_fwd, chunked tensor-core kernel) on its
+    own inputs, with an HBM roofline on its algorithmic bytes; a side figure."""
+    import selective_state_space_m3ssd_b200 as m3
+    base, R = MIMO_WORKLOADS["mimo"]
+    w = rank_workload(base, rank)
+    d = make_mimo_inputs(w, R, dev)
+    Y = torch.empty_like(d["X"])
+    args = [d[k] for k in ("X", "logdecay", "beta", "gamma", "B", "C", "theta", "D", "h0")]
+    hT = torch.empty(w.batch, w.nheads, w.dstate, w.headdim, dtype=torch.float32, device=dev)
+    algo_bytes = nbytes(*args, Y, hT)
+
+    def call():
+        m3.mimo_fwd(*args, Y=Y)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(warmup):
+        call()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        call()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    per = ms / steps
+    achieved = algo_bytes / (per / 1e3) / 1e9
+    out = {"metric": "MIMO scan Mtokens/s (fwd)",
+           "value": w.batch * w.seqlen * world / (per / 1e3) / 1e6,
+           "unit": "Mtokens/s", "ms_per_step": per, "steps": steps,
+           "config": dict(fwd_config(w), rank=R, chunk_tokens=64 // R - 1),
+           "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                        "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                        "algo_bytes_per_launch": algo_bytes, "traffic": None,
+                        "peak_source": peaks["source"]},
+           "gpu_launches": steps}
+    del d, Y, hT, args
     torch.cuda.empty_cache()
     return out
 
@@ -620,6 +669,9 @@ def run_ours(args):
         others = {} if args.no_other_workloads else {
             k: forward_leg(k, dev, min(args.steps, 10), args.warmup, world, rank, peaks)
             for k in ("ssd", "long")}
+        if not args.no_other_workloads:
+            others["mimo"] = mimo_forward_leg(dev, min(args.steps, 10), args.warmup, world, rank,
+                                              peaks)
     e2e = bench_e2e(w, dev, max(1, min(args.steps, 10)), 3, fw["inp"], world)
 
     tokens = w.batch * w.seqlen * args.steps * world
@@ -644,6 +696,7 @@ def run_ours(args):
         "backward": bwd,
         "ssd_forward": others.get("ssd"),
         "long_forward": others.get("long"),
+        "mimo_forward": others.get("mimo"),
         "clocks": clk.summary(),
     }
     if world > 1:
@@ -667,7 +720,8 @@ def summary_of(line: dict) -> dict:
         return {"value": round(d["value"], 3), "unit": d["unit"],
                 "ms_per_step": round(d["ms_per_step"], 4), "frac": round(r.get("frac", 0.0), 3)}
     out = {"forward_siso": one(line)}
-    for k in ("ssd_forward", "long_forward", "backward", "block", "mimo_decode", "decode"):
+    for k in ("ssd_forward", "long_forward", "mimo_forward", "backward", "block", "mimo_decode",
+              "decode"):
         out[k] = one(line.get(k))
     return out
 
@@ -758,6 +812,18 @@ def run_profile(args):
             m3.bwd(*args_, dY=dY)
         torch.cuda.synchronize(dev)
         print(json.dumps({"profile": "backward", "workload": "siso shape b1 L1024 H32 P64 N128"}))
+    elif args.profile == "mimo_fwd":
+        # the rank-4 MIMO prefill at batch 2 (about 290 MB of inputs and outputs,
+        # above L2): a small case of the chunked MIMO kernel for full-section captures
+        base, R = MIMO_WORKLOADS["mimo"]
+        w = base.with_(batch=2)
+        d = make_mimo_inputs(w, R, dev)
+        Y = torch.empty_like(d["X"])
+        args_ = [d[k] for k in ("X", "logdecay", "beta", "gamma", "B", "C", "theta", "D", "h0")]
+        for _ in range(args.warmup + args.steps):
+            m3.mimo_fwd(*args_, Y=Y)
+        torch.cuda.synchronize(dev)
+        print(json.dumps({"profile": "mimo_fwd", "workload": w.name.replace("b8", "b2")}))
     elif args.profile == "mimo":
         # rank-4 MIMO decode steps at half the decode batch: b128, fp32 cache
         # (134 MB of state, above L2), one launch of the step kernel and one of
@@ -811,7 +877,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="omit the oracle timing (it never runs inside a GPU timed region)")
     ap.add_argument("--profile", choices=["forward", "forward8", "decode", "block", "backward",
-                                          "mimo"],
+                                          "mimo", "mimo_fwd"],
                     help="run only a small case of one kernel family (for ncu captures)")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -132,6 +132,11 @@ cudaError_t launch_bwd_chunk(const BwdArgs& a, cudaStream_t s);
 // Y, B, C, x_prev, b_prev (and the extra cache inputs / outputs).
 bool mimo_shape_ok(int64_t N, int64_t P, int64_t R);
 cudaError_t launch_mimo_fwd(const FwdArgs& a, int64_t R, cudaStream_t s);
+// Chunked bf16 tensor-core MIMO forward (N = 128, P = 64, R = 2, 4 or 8; 16-byte
+// aligned X, B, C, Y, theta, h0, hT): 64 rows of (token, rank) per chunk.
+bool fwd_chunk_mimo_supported(const FwdArgs& a, int64_t R);
+cudaError_t launch_fwd_chunk_mimo(const FwdArgs& a, int64_t R, cudaStream_t s);
+cudaError_t read_and_clear_mimo_wait_timeouts(unsigned int* count);
 cudaError_t launch_mimo_step(const StepArgs& a, int64_t R, cudaStream_t s);
 
 // Sequential fp32 forward: one CTA per (b, h), token by token.

@@ -122,6 +122,34 @@ def make_inputs(w: Workload, device: str | torch.device = "cpu") -> dict:
             "B": B.to(xd), "C": C.to(xd), "theta": theta, "D": D, "h0": h0}
 
 
+# The rank-4 MIMO prefill at the siso workload's shape.
+MIMO_WORKLOADS = {
+    "mimo": (Workload("mimo rank-4 trap+rope fwd b8 L4096 H32 P64 N128 R4 bf16", 8, 4096, 32, 64, 128,
+                      1, "bf16", True, True, 0.1, 1005), 4),
+}
+
+
+def make_mimo_inputs(w: Workload, rank: int, device: str | torch.device = "cpu") -> dict:
+    """One MIMO input set: the scalar inputs (logdecay, beta, gamma, theta, D, h0)
+    drawn as for the SISO workload ``w``, then X (b,L,H,P,R) ~ N(0, 1) and B, C
+    (b,L,G,N,R) ~ N(0, 1/N) per rank column from a second stream (seed + 1)."""
+    scal = make_inputs(w.with_(headdim=1), device)  # its X, B, C and h0 are discarded
+    b, L, H, P, N, G, R = w.batch, w.seqlen, w.nheads, w.headdim, w.dstate, w.ngroups, rank
+    dev = torch.device(device)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(w.seed + 1)
+    f32 = dict(dtype=torch.float32, device=dev, generator=gen)
+    xd = torch_dtype(w.dtype)
+    X = torch.randn(b, L, H, P, R, **f32).to(xd)
+    B = (torch.randn(b, L, G, N, R, **f32) * (1.0 / math.sqrt(N))).to(xd)
+    C = (torch.randn(b, L, G, N, R, **f32) * (1.0 / math.sqrt(N))).to(xd)
+    h0 = None
+    if w.h0_var is not None:
+        h0 = torch.randn(b, H, N, P, **f32) * math.sqrt(w.h0_var)
+    return {"X": X, "logdecay": scal["logdecay"], "beta": scal["beta"], "gamma": scal["gamma"],
+            "B": B, "C": C, "theta": scal["theta"], "D": scal["D"], "h0": h0}
+
+
 def slice_inputs(inp: dict, b: slice | int, t: slice | int | None = None, heads=None,
                  ngroups: int = 1) -> dict:
     """Cut a sub-problem out of an input set: batch rows ``b``, time ``t`` and

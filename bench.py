@@ -522,7 +522,6 @@ def bench_block(dev, rank, peaks: dict, steps: int = 5, warmup: int = 3):
     out = torch.empty_like(u)
     dims = m3.BlockDims(s.batch, s.seqlen, s.d_model, s.nheads, s.headdim, s.dstate, s.ngroups)
     ws = torch.empty(m3.block_workspace_size(dims), dtype=torch.uint8, device=dev)
-    m3.block_tune(u, wts, out=out, workspace=ws)  # projection algorithms, before any timing
     for _ in range(warmup):
         m3.block_fwd(u, wts, out=out, workspace=ws)
     torch.cuda.synchronize(dev)
@@ -559,9 +558,55 @@ def bench_block(dev, rank, peaks: dict, steps: int = 5, warmup: int = 3):
                          "gemm_tflop_per_step": 2.0 * M * (dm * width + HP * dm) / 1e12,
                          "note": "sum over phases of max(flops / bf16 peak, bytes / HBM) for the "
                                  "GEMMs and bytes / HBM for prep, scan (B, C per group, head bias applied inside) and gate"},
-            "gpu_launches": 3 * steps,
-            "library_launches": 2 * steps,
-            "note": "own kernels per call: prep, scan, gate; cuBLASLt: in_proj, out_proj"}
+            "gpu_launches": 5 * steps,
+            "note": "own kernels per call: in_proj GEMM, prep, scan, gate, out_proj GEMM"}
+
+
+def bench_gemm(dev, peaks, steps: int = 10, warmup: int = 3):
+    """The block's projection GEMM (m3ssd_gemm_bf16) alone at the model size's two
+    shapes, against the measured bf16 peak; torch.matmul (cuBLAS) on the same
+    operands is timed beside it for context."""
+    import selective_state_space_m3ssd_b200 as m3
+    from selective_state_space_m3ssd_b200.synth import BLOCKS
+    s = BLOCKS["model"]
+    M = s.batch * s.seqlen
+    g = torch.Generator(device=dev).manual_seed(s.seed + 3)
+    out = {}
+    stream = torch.cuda.current_stream(dev)
+    for name, (N, K) in (("in_proj", (s.in_proj_width, s.d_model)),
+                         ("out_proj", (s.d_model, s.nheads * s.headdim))):
+        A = torch.randn(M, K, device=dev, generator=g).bfloat16()
+        W = (torch.randn(N, K, device=dev, generator=g) / K ** 0.5).bfloat16()
+        D = torch.empty(M, N, device=dev, dtype=torch.bfloat16)
+        times = {}
+        for impl, fn in (("own", lambda: m3.gemm_bf16(A, W, out=D)),
+                         ("cublas", lambda: torch.matmul(A, W.t(), out=D))):
+            for _ in range(warmup):
+                fn()
+            torch.cuda.synchronize(dev)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(steps):
+                fn()
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            times[impl] = e0.elapsed_time(e1) / steps
+        fl = 2.0 * M * N * K
+        ach = fl / (times["own"] / 1e3) / 1e12
+        out[name] = {"shape": [M, N, K], "ms": times["own"], "tflops": ach,
+                     "frac": ach / peaks["bf16_tflops"],
+                     "cublas_ms": times["cublas"],
+                     "cublas_tflops": fl / (times["cublas"] / 1e3) / 1e12}
+        del A, W, D
+    tot_ms = out["in_proj"]["ms"] + out["out_proj"]["ms"]
+    tot_fl = sum(2.0 * v["shape"][0] * v["shape"][1] * v["shape"][2] for v in out.values())
+    ach = tot_fl / (tot_ms / 1e3) / 1e12
+    return {"metric": "GEMM TFLOP/s (block projections)", "value": ach, "unit": "TFLOP/s",
+            "ms_per_step": tot_ms, "steps": steps,
+            "roofline": {"bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"],
+                         "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops"],
+                         "peak_source": peaks["source"]},
+            "shapes": out, "gpu_launches": 2 * steps}
 
 
 def bench_backward(w, dev, steps, world, d, peaks):
@@ -664,6 +709,7 @@ def run_ours(args):
         dec = bench_decode(dev, rank, max(1, args.decode_replays), peaks)
         mimo = bench_mimo_decode(dev, rank, peaks)
         blk = None if args.no_block else bench_block(dev, rank, peaks)
+        gemm = None if args.no_block else bench_gemm(dev, peaks)
         bwd = None if args.no_backward else bench_backward(
             w, dev, max(1, min(args.steps, 3)), world, fw["dev_inputs"], peaks)
         others = {} if args.no_other_workloads else {
@@ -693,6 +739,7 @@ def run_ours(args):
         "decode": dec,
         "mimo_decode": mimo,
         "block": blk,
+        "gemm": gemm,
         "backward": bwd,
         "ssd_forward": others.get("ssd"),
         "long_forward": others.get("long"),
@@ -720,8 +767,8 @@ def summary_of(line: dict) -> dict:
         return {"value": round(d["value"], 3), "unit": d["unit"],
                 "ms_per_step": round(d["ms_per_step"], 4), "frac": round(r.get("frac", 0.0), 3)}
     out = {"forward_siso": one(line)}
-    for k in ("ssd_forward", "long_forward", "mimo_forward", "backward", "block", "mimo_decode",
-              "decode"):
+    for k in ("ssd_forward", "long_forward", "mimo_forward", "backward", "block", "gemm",
+              "mimo_decode", "decode"):
         out[k] = one(line.get(k))
     return out
 
@@ -812,6 +859,20 @@ def run_profile(args):
             m3.bwd(*args_, dY=dY)
         torch.cuda.synchronize(dev)
         print(json.dumps({"profile": "backward", "workload": "siso shape b1 L1024 H32 P64 N128"}))
+    elif args.profile == "gemm":
+        # the in_proj GEMM shape at a quarter of the block's tokens: 8192 x 6464 x 1024
+        # (135 MB of operands and output, above L2), a small case for full captures
+        from selective_state_space_m3ssd_b200.synth import BLOCKS
+        s_ = BLOCKS["model"]
+        M, N, K = 8192, s_.in_proj_width, s_.d_model
+        g = torch.Generator(device=dev).manual_seed(11)
+        A = torch.randn(M, K, device=dev, generator=g).bfloat16()
+        W = (torch.randn(N, K, device=dev, generator=g) / K ** 0.5).bfloat16()
+        D = torch.empty(M, N, device=dev, dtype=torch.bfloat16)
+        for _ in range(args.warmup + args.steps):
+            m3.gemm_bf16(A, W, out=D)
+        torch.cuda.synchronize(dev)
+        print(json.dumps({"profile": "gemm", "workload": f"in_proj GEMM {M} x {N} x {K} bf16"}))
     elif args.profile == "mimo_fwd":
         # the rank-4 MIMO prefill at batch 2 (about 290 MB of inputs and outputs,
         # above L2): a small case of the chunked MIMO kernel for full-section captures
@@ -877,7 +938,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="omit the oracle timing (it never runs inside a GPU timed region)")
     ap.add_argument("--profile", choices=["forward", "forward8", "decode", "block", "backward",
-                                          "mimo", "mimo_fwd"],
+                                          "mimo", "mimo_fwd", "gemm"],
                     help="run only a small case of one kernel family (for ncu captures)")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -305,10 +305,10 @@ m3ssd_status m3ssd_bwd_noalloc(const m3ssd_dims* dims, const void* X, const floa
  *                                                                    one B/C per head)
  *   out = (y * SiLU(z)) W_out^T          out_proj, no bias
  *
- * The projections are plain GEMMs run by cuBLASLt (bf16 operands, fp32
- * accumulation, bf16 outputs); the rest runs in this
- * library's kernels, the head biases inside the scan (added in fp32 before the
- * rotation).  u and out are bf16.  The block cache is an m3ssd_cache with
+ * The projections are plain GEMMs on this library's tensor-core GEMM
+ * (m3ssd_gemm_bf16: bf16 operands, fp32 accumulation, bf16 outputs); the rest
+ * runs in this library's kernels too, the head biases inside the scan (added
+ * in fp32 before the rotation).  u and out are bf16.  The block cache is an m3ssd_cache with
  * b_prev (b, G, N) holding the QK-normed group vector B_{t-1} (times its norm
  * weight, without the head bias) unrotated; the bias is added at use.
  */
@@ -345,8 +345,7 @@ size_t m3ssd_block_workspace_size(const m3ssd_block_dims* dims);
  * zero) is the state the sequence continues from; cache_out (may be NULL) gets
  * the state after the last token and may be the same object as cache_in.
  * workspace: workspace_bytes >= m3ssd_block_workspace_size(dims), 256-byte
- * aligned, not read afterwards.  Errors as m3ssd_fwd; a cuBLASLt failure
- * returns M3SSD_ERR_CUDA.
+ * aligned, not read afterwards.  Errors as m3ssd_fwd.
  */
 m3ssd_status m3ssd_block_fwd(const m3ssd_block_dims* dims, const m3ssd_block_weights* w,
                              const void* u, void* out, const m3ssd_cache* cache_in,
@@ -354,20 +353,19 @@ m3ssd_status m3ssd_block_fwd(const m3ssd_block_dims* dims, const m3ssd_block_wei
                              size_t workspace_bytes, void* stream);
 
 /*
- * m3ssd_block_fwd once more, choosing the cuBLASLt algorithm of each of its
- * projections on the way: for a projection shape not seen before, each of up
- * to 8 heuristic candidates is timed on these operands (one warm-up run, then
- * the best of three) and the fastest is kept for the process; later
- * m3ssd_block_fwd and m3ssd_block_step calls of the same shapes use it
- * (without a tuned choice they take cuBLASLt's first heuristic).  No page
- * counterpart; a convenience of this library.  Arguments and results as
- * m3ssd_block_fwd without caches.  Unlike every other entry point it
- * synchronises the stream while timing, so it must not be captured in a CUDA
- * graph; it is not meant to run concurrently with itself.
+ * The block's projection GEMM ("VikramLex/mamba3-minimal" README,
+ * "Architecture": in_proj and out_proj are plain linear maps), exported for
+ * callers that compose the block themselves:
+ *     D (M x N, row stride ldd elements) = A (M x K) W^T
+ * A (M x K) and W (N x K): bf16, row-major (row stride K), 16-byte aligned,
+ * K a multiple of 8; D: bf16, ldd >= N, 2-byte aligned (16-byte stores when D
+ * is 16-byte aligned and ldd a multiple of 8).  fp32 accumulation on the
+ * tensor cores, each output rounded once to bf16 (nearest even).  M, N, K up
+ * to 2^31 - 1; M = 0 or N = 0 does nothing.  Other shapes or alignments:
+ * M3SSD_ERR_INVALID_ARG.  No allocation, no synchronisation.
  */
-m3ssd_status m3ssd_block_tune(const m3ssd_block_dims* dims, const m3ssd_block_weights* w,
-                              const void* u, void* out, void* workspace, size_t workspace_bytes,
-                              void* stream);
+m3ssd_status m3ssd_gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, const void* W,
+                             void* D, int64_t ldd, void* stream);
 
 /*
  * One decode step of the block (Mamba3SisoBlock.step): u_t, out_t (b, d_model)
@@ -378,10 +376,11 @@ m3ssd_status m3ssd_block_step(const m3ssd_block_dims* dims, const m3ssd_block_we
                               const void* u_t, void* out_t, const m3ssd_cache* cache,
                               void* workspace, size_t workspace_bytes, void* stream);
 
-/* Number of bounded device-side waits of the chunked forward and of the
- * tensor-core backward that ran out since the last call (the forward's CTA
- * then stops and leaves its outputs unwritten; the backward's CTA skips its
- * remaining waits and leaves its outputs undefined); the count is then reset.  This call synchronises the current device
+/* Number of bounded device-side waits of the chunked forwards (SISO and
+ * MIMO), the tensor-core backward and the projection GEMM that ran out since
+ * the last call (a forward's CTA then stops and leaves its outputs unwritten;
+ * the backward's and the GEMM's CTAs skip their remaining waits and leave their
+ * outputs undefined); the count is then reset.  This call synchronises the current device
  * and must not be captured in a CUDA graph.  Returns M3SSD_ERR_INVALID_ARG for
  * a NULL pointer and M3SSD_ERR_CUDA if the device cannot be read. */
 m3ssd_status m3ssd_device_wait_timeouts(uint32_t* count);

@@ -124,9 +124,10 @@ def load(path: str | None = None):
         lib.m3ssd_block_step.argtypes = [ctypes.POINTER(BlockDims), ctypes.POINTER(BlockWeights),
                                          vp, vp, ctypes.POINTER(Cache), vp, sz, vp]
         lib.m3ssd_block_step.restype = ctypes.c_int
-        lib.m3ssd_block_tune.argtypes = [ctypes.POINTER(BlockDims), ctypes.POINTER(BlockWeights),
-                                         vp, vp, vp, sz, vp]
-        lib.m3ssd_block_tune.restype = ctypes.c_int
+        lib.m3ssd_gemm_bf16.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                                        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                        ctypes.c_int64, ctypes.c_void_p]
+        lib.m3ssd_gemm_bf16.restype = ctypes.c_int
         lib.m3ssd_status_string.argtypes = [ctypes.c_int]
         lib.m3ssd_status_string.restype = ctypes.c_char_p
         lib.m3ssd_abi_version.argtypes = []
@@ -582,22 +583,18 @@ def block_fwd(u, wts: dict, *, cache_in=None, cache_out=None, out=None, workspac
     return out
 
 
-def block_tune(u, wts: dict, *, out=None, workspace=None):
-    """``m3ssd_block_tune``: one block forward that times cuBLASLt's candidate
-    algorithms for its two projections and keeps the fastest for later calls of
-    the same shapes (synchronises; not for graph capture)."""
+def gemm_bf16(A, W, *, out=None):
+    """``m3ssd_gemm_bf16``: A (M, K) @ W (N, K)^T in bf16 with fp32 accumulation
+    on the current stream; returns out (M, N) bf16."""
     import torch
-    b, L, dm = u.shape
-    dims, w, _ = _block_args(u, wts, L)
-    dev = u.device
-    out = torch.empty_like(u) if out is None else out
-    _need(out, "out", torch.bfloat16, (b, L, dm), dev)
-    need = block_workspace_size(dims)
-    if workspace is None:
-        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
-    st = load().m3ssd_block_tune(ctypes.byref(dims), ctypes.byref(w), _ptr(u), _ptr(out),
-                                 _ptr(workspace), workspace.numel(), _stream_handle(dev))
-    _check(st, "m3ssd_block_tune")
+    _need(A, "A", torch.bfloat16, device=A.device)
+    M, K = A.shape
+    _need(W, "W", torch.bfloat16, (W.shape[0], K), A.device)
+    N = W.shape[0]
+    out = torch.empty(M, N, dtype=torch.bfloat16, device=A.device) if out is None else out
+    _need(out, "out", torch.bfloat16, (M, N), A.device)
+    st = load().m3ssd_gemm_bf16(M, N, K, _ptr(A), _ptr(W), _ptr(out), N, _stream_handle(A.device))
+    _check(st, "m3ssd_gemm_bf16")
     return out
 
 

@@ -27,13 +27,9 @@ FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2",
                 "--expt-relaxed-constexpr", "-I", os.path.join(ROOT, "include")]
 
 
-def _cuda_lib() -> str:
-    return os.path.join(os.environ.get("CUDA_HOME", "/usr/local/cuda"), "lib64")
-
-
-# cuBLASLt runs the block's two projections (plain GEMMs); it is the only
-# library linked dynamically, found through the toolkit's lib64 at run time.
-LINK = ["-L" + _cuda_lib(), "-lcublasLt", "-Xlinker", "-rpath," + _cuda_lib()]
+# Every kernel, the block's two projections included, is the library's own;
+# the CUDA runtime is linked statically and nothing else is linked.
+LINK = []
 
 
 def nvcc() -> str:

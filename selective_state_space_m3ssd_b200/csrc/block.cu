@@ -4,8 +4,9 @@
 // in_proj -> (z, x, B, C, Delta, lambda, theta); B, C: QK-norm -> +bias ->
 // RoPE; trapezoidal SSD; y + D x -> y * SiLU(z) -> out) and "TorchMamba"
 // README, "API reference" (Mamba3SisoBlock with forward / prefill / step and
-// Mamba3SisoCache).  The two projections are plain GEMMs and run in cuBLASLt
-// (bf16 operands, fp32 accumulation); everything between them runs here:
+// Mamba3SisoCache).  The two projections are plain GEMMs on the library's own
+// tensor-core GEMM (csrc/gemm.cu: bf16 operands, fp32 accumulation in TMEM);
+// everything between them runs here:
 //
 //   block_prep_kernel   one CTA per token: splits the bf16 in_proj row, copies x
 //                       (bf16), writes the QK-normed B and C of each group times the
@@ -14,12 +15,9 @@
 //   the scan's forward / step kernels on those tensors, which add the head's
 //   B and C biases in fp32 before rotating (no per-head copy of B and C);
 //   block_gate_kernel   y * SiLU(z) (bf16), the input of out_proj.
-#include <cublasLt.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
-#include <map>
-#include <mutex>
 
 #include "../../include/m3ssd.h"
 #include "common.cuh"
@@ -28,7 +26,6 @@
 namespace m3ssd {
 namespace {
 
-constexpr size_t kLtWorkspace = size_t(32) << 20;
 constexpr int kPrepThreads = 256;
 
 size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -40,7 +37,7 @@ int64_t in_proj_width(const m3ssd_block_dims* d) {
 
 // Workspace regions (byte offsets) for M tokens.
 struct BlockWs {
-  size_t zx, x, B, C, ld, be, ga, th, y, bp, lt, total;
+  size_t zx, x, B, C, ld, be, ga, th, y, bp, total;
 };
 BlockWs block_ws(const m3ssd_block_dims* d, int64_t M) {
   const size_t H = (size_t)d->nheads, P = (size_t)d->headdim, N = (size_t)d->dstate;
@@ -63,7 +60,6 @@ BlockWs block_ws(const m3ssd_block_dims* d, int64_t M) {
   w.th = take(m * H * (N / 2) * 4);
   w.y = take(m * H * P * 2);
   w.bp = take((size_t)d->batch * G * N * 4);  // copy of the incoming b_prev
-  w.lt = take(kLtWorkspace);
   w.total = o;
   return w;
 }
@@ -270,137 +266,6 @@ __global__ void block_gate_kernel(const __nv_bfloat16* __restrict__ y,
   }
 }
 
-cublasLtHandle_t lt_handle() {
-  static std::once_flag once;
-  static cublasLtHandle_t h = nullptr;
-  std::call_once(once, [] {
-    if (cublasLtCreate(&h) != CUBLAS_STATUS_SUCCESS) h = nullptr;
-  });
-  return h;
-}
-
-// The algorithm for one GEMM shape: the one m3ssd_block_tune measured for it
-// if any, else cuBLASLt's first heuristic.  Tuning (only inside
-// m3ssd_block_tune, which synchronises) times each of up to 8 heuristic
-// candidates on the call's own operands (one warm-up run, then the best of
-// three) and keeps the fastest for the process.
-thread_local bool g_tune = false;
-struct AlgoKey {
-  int64_t M, N, K;
-  int dt;
-  bool operator<(const AlgoKey& o) const {
-    return M != o.M ? M < o.M : N != o.N ? N < o.N : K != o.K ? K < o.K : dt < o.dt;
-  }
-};
-
-bool pick_algo(cublasLtHandle_t h, cublasLtMatmulDesc_t op, cublasLtMatrixLayout_t la,
-               cublasLtMatrixLayout_t lb, cublasLtMatrixLayout_t lc,
-               cublasLtMatmulPreference_t pref, int64_t M, int64_t Nout, int64_t K,
-               cudaDataType_t dt, const void* A, const void* W, void* D, void* ws,
-               size_t ws_bytes, cudaStream_t s, cublasLtMatmulAlgo_t* out) {
-  static std::mutex mu;
-  static std::map<AlgoKey, cublasLtMatmulAlgo_t> cache;
-  const AlgoKey key{M, Nout, K, (int)dt};
-  {
-    std::lock_guard<std::mutex> lock(mu);
-    auto it = cache.find(key);
-    if (it != cache.end()) {
-      *out = it->second;
-      return true;
-    }
-  }
-  cublasLtMatmulHeuristicResult_t res[8];
-  int found = 0;
-  if (cublasLtMatmulAlgoGetHeuristic(h, op, la, lb, lc, lc, pref, 8, res, &found) !=
-          CUBLAS_STATUS_SUCCESS ||
-      found == 0)
-    return false;
-  int best = 0;
-  if (g_tune && found > 1) {
-    cudaEvent_t e0 = nullptr, e1 = nullptr;
-    if (cudaEventCreate(&e0) == cudaSuccess && cudaEventCreate(&e1) == cudaSuccess) {
-      const float alpha = 1.f, beta = 0.f;
-      float best_ms = 0.f;
-      for (int i = 0; i < found; ++i) {
-        if (res[i].state != CUBLAS_STATUS_SUCCESS) continue;
-        float ms_i = -1.f;
-        for (int rep = 0; rep < 4; ++rep) {  // the first run warms up
-          cudaEventRecord(e0, s);
-          const bool run = cublasLtMatmul(h, op, &alpha, W, la, A, lb, &beta, D, lc, D, lc,
-                                          &res[i].algo, ws, ws_bytes, s) == CUBLAS_STATUS_SUCCESS;
-          cudaEventRecord(e1, s);
-          float t = 0.f;
-          if (!run || cudaEventSynchronize(e1) != cudaSuccess ||
-              cudaEventElapsedTime(&t, e0, e1) != cudaSuccess) {
-            ms_i = -1.f;
-            break;
-          }
-          if (rep > 0 && (ms_i < 0.f || t < ms_i)) ms_i = t;
-        }
-        if (ms_i > 0.f && (best_ms == 0.f || ms_i < best_ms)) {
-          best_ms = ms_i;
-          best = i;
-        }
-      }
-      (void)cudaGetLastError();
-    }
-    if (e0) cudaEventDestroy(e0);
-    if (e1) cudaEventDestroy(e1);
-  }
-  *out = res[best].algo;
-  if (g_tune) {
-    std::lock_guard<std::mutex> lock(mu);
-    cache[key] = *out;
-  }
-  return true;
-}
-
-// D (M x Nout, row-major, type dt) = A (M x K, bf16, row-major) W^T, with W
-// (Nout x K, bf16, row-major) -- in cuBLASLt's column-major terms
-// D^T = op_T(W) A^T.  Returns false if cuBLASLt refuses or fails.
-bool gemm_bf16(int64_t M, int64_t Nout, int64_t K, const void* A, const void* W, void* D,
-               cudaDataType_t dt, void* ws, size_t ws_bytes, cudaStream_t s) {
-  cublasLtHandle_t h = lt_handle();
-  if (!h) return false;
-  cublasLtMatmulDesc_t op = nullptr;
-  cublasLtMatrixLayout_t la = nullptr, lb = nullptr, lc = nullptr;
-  cublasLtMatmulPreference_t pref = nullptr;
-  bool ok = false;
-  do {
-    if (cublasLtMatmulDescCreate(&op, CUBLAS_COMPUTE_32F, CUDA_R_32F) != CUBLAS_STATUS_SUCCESS) break;
-    const cublasOperation_t ta = CUBLAS_OP_T, tb = CUBLAS_OP_N;
-    if (cublasLtMatmulDescSetAttribute(op, CUBLASLT_MATMUL_DESC_TRANSA, &ta, sizeof(ta)) !=
-            CUBLAS_STATUS_SUCCESS ||
-        cublasLtMatmulDescSetAttribute(op, CUBLASLT_MATMUL_DESC_TRANSB, &tb, sizeof(tb)) !=
-            CUBLAS_STATUS_SUCCESS)
-      break;
-    if (cublasLtMatrixLayoutCreate(&la, CUDA_R_16BF, (uint64_t)K, (uint64_t)Nout, K) !=
-            CUBLAS_STATUS_SUCCESS ||
-        cublasLtMatrixLayoutCreate(&lb, CUDA_R_16BF, (uint64_t)K, (uint64_t)M, K) !=
-            CUBLAS_STATUS_SUCCESS ||
-        cublasLtMatrixLayoutCreate(&lc, dt, (uint64_t)Nout, (uint64_t)M, Nout) !=
-            CUBLAS_STATUS_SUCCESS)
-      break;
-    if (cublasLtMatmulPreferenceCreate(&pref) != CUBLAS_STATUS_SUCCESS) break;
-    if (cublasLtMatmulPreferenceSetAttribute(pref, CUBLASLT_MATMUL_PREF_MAX_WORKSPACE_BYTES,
-                                             &ws_bytes, sizeof(ws_bytes)) != CUBLAS_STATUS_SUCCESS)
-      break;
-    const float alpha = 1.f, beta = 0.f;
-    cublasLtMatmulAlgo_t algo;
-    if (!pick_algo(h, op, la, lb, lc, pref, M, Nout, K, dt, A, W, D, ws, ws_bytes, s, &algo)) break;
-    if (cublasLtMatmul(h, op, &alpha, W, la, A, lb, &beta, D, lc, D, lc, &algo, ws, ws_bytes,
-                       s) != CUBLAS_STATUS_SUCCESS)
-      break;
-    ok = true;
-  } while (false);
-  if (pref) cublasLtMatmulPreferenceDestroy(pref);
-  if (lc) cublasLtMatrixLayoutDestroy(lc);
-  if (lb) cublasLtMatrixLayoutDestroy(lb);
-  if (la) cublasLtMatrixLayoutDestroy(la);
-  if (op) cublasLtMatmulDescDestroy(op);
-  return ok;
-}
-
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 m3ssd_status check_block(const m3ssd_block_dims* d, const m3ssd_block_weights* w) {
@@ -433,9 +298,10 @@ m3ssd_status front(const m3ssd_block_dims* d, const m3ssd_block_weights* w, cons
                    int64_t M, char* base, const BlockWs& ws, bool write_x, bool write_th,
                    cudaStream_t s) {
   const int64_t width = in_proj_width(d);
-  if (!gemm_bf16(M, width, d->d_model, u, w->W_in, base + ws.zx, CUDA_R_16BF, base + ws.lt,
-                 kLtWorkspace, s))
+  if (launch_gemm_bf16(M, width, d->d_model, u, w->W_in, base + ws.zx, width, s) != cudaSuccess) {
+    (void)cudaGetLastError();
     return M3SSD_ERR_CUDA;
+  }
   PrepArgs a{};
   a.M = M; a.H = d->nheads; a.P = d->headdim; a.N = d->dstate; a.G = d->ngroups; a.width = width;
   a.zx = reinterpret_cast<const __nv_bfloat16*>(base + ws.zx);
@@ -477,9 +343,11 @@ m3ssd_status back(const m3ssd_block_dims* d, const m3ssd_block_weights* w, int64
     block_gate_kernel<<<grid, 256, 0, s>>>(yp, zp, width, HP, M, gp);
   }
   if (cudaGetLastError() != cudaSuccess) return M3SSD_ERR_CUDA;
-  if (!gemm_bf16(M, d->d_model, HP, base + ws.x, w->W_out, out, CUDA_R_16BF, base + ws.lt,
-                 kLtWorkspace, s))
+  if (launch_gemm_bf16(M, d->d_model, HP, base + ws.x, w->W_out, out, d->d_model, s) !=
+      cudaSuccess) {
+    (void)cudaGetLastError();
     return M3SSD_ERR_CUDA;
+  }
   return M3SSD_OK;
 }
 
@@ -584,16 +452,6 @@ m3ssd_status m3ssd_block_fwd(const m3ssd_block_dims* dims, const m3ssd_block_wei
   return back(dims, w, M, base, ws, out, s);
 }
 
-m3ssd_status m3ssd_block_tune(const m3ssd_block_dims* dims, const m3ssd_block_weights* w,
-                              const void* u, void* out, void* workspace, size_t workspace_bytes,
-                              void* stream) {
-  m3ssd::g_tune = true;
-  const m3ssd_status st =
-      m3ssd_block_fwd(dims, w, u, out, nullptr, nullptr, workspace, workspace_bytes, stream);
-  m3ssd::g_tune = false;
-  return st;
-}
-
 m3ssd_status m3ssd_block_step(const m3ssd_block_dims* dims, const m3ssd_block_weights* w,
                               const void* u_t, void* out_t, const m3ssd_cache* cache,
                               void* workspace, size_t workspace_bytes, void* stream) {
@@ -640,6 +498,21 @@ m3ssd_status m3ssd_block_step(const m3ssd_block_dims* dims, const m3ssd_block_we
     return M3SSD_ERR_CUDA;
   }
   return back(&one, w, M, base, ws, out_t, s);
+}
+
+m3ssd_status m3ssd_gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, const void* W,
+                             void* D, int64_t ldd, void* stream) {
+  if (M < 0 || N < 0) return M3SSD_ERR_INVALID_ARG;
+  if (M == 0 || N == 0) return M3SSD_OK;
+  if (!A || !W || !D || K < 1 || K % 8 != 0 || ldd < N || M > INT32_MAX || N > INT32_MAX ||
+      K > INT32_MAX || !m3ssd::aligned(A, 16) || !m3ssd::aligned(W, 16) || !m3ssd::aligned(D, 2))
+    return M3SSD_ERR_INVALID_ARG;
+  if (m3ssd::launch_gemm_bf16(M, N, K, A, W, D, ldd, static_cast<cudaStream_t>(stream)) !=
+      cudaSuccess) {
+    (void)cudaGetLastError();
+    return M3SSD_ERR_CUDA;
+  }
+  return M3SSD_OK;
 }
 
 }  // extern "C"

@@ -157,6 +157,11 @@ cudaError_t request_dropped_gram_signal();
 // reads and clears it (synchronising the device).
 cudaError_t launch_nonfinite_check(const void* p, int64_t n, bool bf16, cudaStream_t s);
 cudaError_t read_and_clear_nonfinite(unsigned int* flag);
+// D (M x N, bf16, row stride ldd) = A (M x K) W^T on the tensor cores, with A
+// (M x K) and W (N x K) bf16 row-major, 16-byte aligned, K a multiple of 8.
+cudaError_t launch_gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, const void* W,
+                             void* D, int64_t ldd, cudaStream_t s);
+cudaError_t read_and_clear_gemm_wait_timeouts(unsigned int* count);
 // Decode step (two launches: the state/outputs, then b_prev <- B_t).
 cudaError_t launch_step(const StepArgs& a, cudaStream_t s);
 

@@ -68,11 +68,12 @@ m3ssd_status m3ssd_nonfinite_outputs(void) {
 
 m3ssd_status m3ssd_device_wait_timeouts(uint32_t* count) {
   if (!count) return M3SSD_ERR_INVALID_ARG;
-  unsigned int n = 0, nb = 0, nm = 0;
+  unsigned int n = 0, nb = 0, nm = 0, ng = 0;
   m3ssd_status st = from_cuda(m3ssd::read_and_clear_wait_timeouts(&n));
   if (st == M3SSD_OK) st = from_cuda(m3ssd::read_and_clear_bwd_wait_timeouts(&nb));
   if (st == M3SSD_OK) st = from_cuda(m3ssd::read_and_clear_mimo_wait_timeouts(&nm));
-  *count = n + nb + nm;
+  if (st == M3SSD_OK) st = from_cuda(m3ssd::read_and_clear_gemm_wait_timeouts(&ng));
+  *count = n + nb + nm + ng;
   return st;
 }
 

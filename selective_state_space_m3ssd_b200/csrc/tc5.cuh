@@ -184,6 +184,16 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const void* tmap, uint
       : "memory");
 }
 
+// The same for a 2-D tensor map.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, uint64_t* mbar, int c0,
+                                            int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(saddr(mbar)), "r"(c0), "r"(c1)
+      : "memory");
+}
+
 // The same for a 5-D tensor map.
 __device__ __forceinline__ void tma_load_5d(uint32_t dst, const void* tmap, uint64_t* mbar, int c0,
                                             int c1, int c2, int c3, int c4) {
@@ -262,6 +272,13 @@ __device__ __forceinline__ void ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[16])
       : "r"(taddr));
 }
 __device__ __forceinline__ void wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+// Ties registers filled by a tcgen05.ld to a point after the wait: the compiler
+// sees them redefined here, so no use of them moves above the wait.
+template <int N>
+__device__ __forceinline__ void reg_after_ld(uint32_t (&r)[N]) {
+#pragma unroll
+  for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i]));
+}
 
 }  // namespace tc5
 }  // namespace m3ssd

@@ -243,3 +243,16 @@ def test_backward_refuses_the_finite_check_flag(lib):
     st = lib.m3ssd_bwd(ctypes.byref(d), FAKE, FAKE, None, FAKE, FAKE, FAKE, None, None, None,
                        None, FAKE, None, ctypes.byref(g), None, 0, None)
     assert st == m3.ERR_UNSUPPORTED
+
+
+def test_gemm_validation_before_any_device_call(lib):
+    g = lib.m3ssd_gemm_bf16
+    al = ctypes.c_void_p(0x10000)
+    assert g(0, 8, 8, al, al, al, 8, None) == m3.OK          # nothing to do
+    assert g(8, 0, 8, al, al, al, 8, None) == m3.OK
+    assert g(-1, 8, 8, al, al, al, 8, None) == m3.ERR_INVALID_ARG
+    assert g(8, 8, 12, al, al, al, 8, None) == m3.ERR_INVALID_ARG       # K % 8
+    assert g(8, 8, 8, al, al, al, 4, None) == m3.ERR_INVALID_ARG        # ldd < N
+    assert g(8, 8, 8, None, al, al, 8, None) == m3.ERR_INVALID_ARG
+    assert g(8, 8, 8, ctypes.c_void_p(0x10008), al, al, 8, None) == m3.ERR_INVALID_ARG  # A 16 B
+    assert g(8, 8, 8, al, al, ctypes.c_void_p(0x10001), 8, None) == m3.ERR_INVALID_ARG  # D 2 B

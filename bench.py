@@ -252,6 +252,28 @@ def forward_leg(key, dev, steps, warmup, world, rank, peaks):
     return out
 
 
+def prefill_leg(dev, steps, warmup, world, rank, peaks):
+    """The decode workload's 512-token fp32 prefill (m3ssd_fwd on b256 H32 P64
+    N128, fp32 X, B, C, Y: the chunked kernel with fp16 high / low tensor-core
+    operands), with an HBM roofline on its algorithmic bytes; a side figure."""
+    w = rank_workload(WORKLOADS["decode"].with_(seqlen=DECODE_PREFILL), rank)
+    fw = bench_forward(w, dev, steps, warmup, world, rank)
+    achieved = fw["algo_bytes"] / (fw["ms_per_step"] / 1e3) / 1e9
+    out = {"metric": "scan Mtokens/s (fwd, fp32 prefill)",
+           "value": w.batch * w.seqlen * world / (fw["ms_per_step"] / 1e3) / 1e6,
+           "unit": "Mtokens/s", "ms_per_step": fw["ms_per_step"], "steps": steps,
+           "config": dict(fwd_config(w), workload=f"decode workload prefill b{w.batch} "
+                          f"L{w.seqlen} H{w.nheads} P{w.headdim} N{w.dstate} fp32"),
+           "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                        "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                        "algo_bytes_per_launch": fw["algo_bytes"], "traffic": None,
+                        "peak_source": peaks["source"]},
+           "gpu_launches": fw["launches"]}
+    del fw
+    torch.cuda.empty_cache()
+    return out
+
+
 def mimo_forward_leg(dev, steps, warmup, world, rank, peaks):
     """The rank-4 MIMO prefill (m3ssd_mimo_fwd, chunked tensor-core kernel) on its
     own inputs, with an HBM roofline on its algorithmic bytes; a side figure."""
@@ -718,6 +740,8 @@ def run_ours(args):
         if not args.no_other_workloads:
             others["mimo"] = mimo_forward_leg(dev, min(args.steps, 10), args.warmup, world, rank,
                                               peaks)
+            others["prefill"] = prefill_leg(dev, min(args.steps, 10), args.warmup, world, rank,
+                                            peaks)
     e2e = bench_e2e(w, dev, max(1, min(args.steps, 10)), 3, fw["inp"], world)
 
     tokens = w.batch * w.seqlen * args.steps * world
@@ -744,6 +768,7 @@ def run_ours(args):
         "ssd_forward": others.get("ssd"),
         "long_forward": others.get("long"),
         "mimo_forward": others.get("mimo"),
+        "prefill_forward": others.get("prefill"),
         "clocks": clk.summary(),
     }
     if world > 1:
@@ -767,8 +792,8 @@ def summary_of(line: dict) -> dict:
         return {"value": round(d["value"], 3), "unit": d["unit"],
                 "ms_per_step": round(d["ms_per_step"], 4), "frac": round(r.get("frac", 0.0), 3)}
     out = {"forward_siso": one(line)}
-    for k in ("ssd_forward", "long_forward", "mimo_forward", "backward", "block", "gemm",
-              "mimo_decode", "decode"):
+    for k in ("ssd_forward", "long_forward", "mimo_forward", "prefill_forward", "backward",
+              "block", "gemm", "mimo_decode", "decode"):
         out[k] = one(line.get(k))
     return out
 

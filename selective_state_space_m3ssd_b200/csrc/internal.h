@@ -144,6 +144,11 @@ cudaError_t launch_fwd_seq(const FwdArgs& a, cudaStream_t s);
 // Chunked bf16 tensor-core forward (N = 128, P = 64).
 cudaError_t launch_fwd_chunk(const FwdArgs& a, cudaStream_t s);
 bool fwd_chunk_supported(const FwdArgs& a);
+// Chunked fp32 forward on the tensor cores with fp16 high / low operand parts
+// (fp32 X, B, C, Y; N = 128, P = 64; 16-byte aligned X, B, C, Y, theta, h0, hT).
+bool fwd_chunk32_supported(const FwdArgs& a);
+cudaError_t launch_fwd_chunk32(const FwdArgs& a, cudaStream_t s);
+cudaError_t read_and_clear_chunk32_wait_timeouts(unsigned int* count);
 // Count of bounded device-side waits in the chunked forward that ran out since
 // the last call; reading it synchronises the device and clears the count.
 cudaError_t read_and_clear_wait_timeouts(unsigned int* count);

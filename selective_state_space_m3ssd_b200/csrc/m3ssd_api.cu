@@ -73,7 +73,9 @@ m3ssd_status m3ssd_device_wait_timeouts(uint32_t* count) {
   if (st == M3SSD_OK) st = from_cuda(m3ssd::read_and_clear_bwd_wait_timeouts(&nb));
   if (st == M3SSD_OK) st = from_cuda(m3ssd::read_and_clear_mimo_wait_timeouts(&nm));
   if (st == M3SSD_OK) st = from_cuda(m3ssd::read_and_clear_gemm_wait_timeouts(&ng));
-  *count = n + nb + nm + ng;
+  unsigned int n32 = 0;
+  if (st == M3SSD_OK) st = from_cuda(m3ssd::read_and_clear_chunk32_wait_timeouts(&n32));
+  *count = n + nb + nm + ng + n32;
   return st;
 }
 
@@ -129,11 +131,14 @@ m3ssd_status m3ssd_fwd(const m3ssd_dims* dims, const void* X, const float* logde
     return M3SSD_ERR_WORKSPACE;
 
   const bool chunked = m3ssd::fwd_chunk_supported(a);
-  if (!chunked && !general_shape_ok(dims)) return M3SSD_ERR_UNSUPPORTED;
+  const bool chunked32 = !chunked && m3ssd::fwd_chunk32_supported(a);
+  if (!chunked && !chunked32 && !general_shape_ok(dims)) return M3SSD_ERR_UNSUPPORTED;
   if (dims->batch == 0) return M3SSD_OK;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  st = from_cuda(chunked ? m3ssd::launch_fwd_chunk(a, s) : m3ssd::launch_fwd_seq(a, s));
+  st = from_cuda(chunked     ? m3ssd::launch_fwd_chunk(a, s)
+                 : chunked32 ? m3ssd::launch_fwd_chunk32(a, s)
+                             : m3ssd::launch_fwd_seq(a, s));
   if (st == M3SSD_OK && (dims->flags & M3SSD_CHECK_FINITE)) {
     st = from_cuda(m3ssd::launch_nonfinite_check(
         Y, dims->batch * dims->seqlen * dims->nheads * dims->headdim, bf16, s));

@@ -49,8 +49,10 @@ METRIC = "scan Mtokens/s (fwd, L=4096)"
 UNIT = "Mtokens/s"
 FWD_KEY = "siso"
 PROFILES = os.path.join(ROOT, "profiles")
-CHUNK_SRC = os.path.join(ROOT, "selective_state_space_m3ssd_b200", "csrc", "fwd_chunk.cu")
-STEP_SRC = os.path.join(ROOT, "selective_state_space_m3ssd_b200", "csrc", "step.cu")
+_CSRC = os.path.join(ROOT, "selective_state_space_m3ssd_b200", "csrc")
+# the sources a kernel is built from (a traffic record holds while they are unchanged)
+CHUNK_SRC = [os.path.join(_CSRC, f) for f in ("fwd_chunk.cu", "chunk_common.cuh", "tc5.cuh")]
+STEP_SRC = [os.path.join(_CSRC, "step.cu")]
 
 
 # ----------------------------------------------------------------------------
@@ -71,9 +73,12 @@ def load_peaks() -> dict:
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
 
 
-def src_sha(path: str) -> str:
-    with open(path, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+def src_sha(paths) -> str:
+    h = hashlib.sha256()
+    for path in ([paths] if isinstance(paths, str) else paths):
+        with open(path, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def recorded_traffic(name: str, src: str):
@@ -884,6 +889,14 @@ def run_profile(args):
             m3.bwd(*args_, dY=dY)
         torch.cuda.synchronize(dev)
         print(json.dumps({"profile": "backward", "workload": "siso shape b1 L1024 H32 P64 N128"}))
+    elif args.profile == "prefill":
+        # the fp32 prefill at a quarter of the decode batch: b64 L512 H32 (about 0.8 GB
+        # of inputs and outputs, above L2), a small case of the fp32 chunked kernel
+        w = WORKLOADS["decode"].with_(batch=64, seqlen=DECODE_PREFILL)
+        fw = bench_forward(w, dev, args.steps, args.warmup, 1, 0)
+        print(json.dumps({"profile": "prefill", "workload": f"decode prefill b{w.batch} "
+                          f"L{w.seqlen} H{w.nheads} P{w.headdim} N{w.dstate} fp32",
+                          "ms_per_step": fw["ms_per_step"]}))
     elif args.profile == "gemm":
         # the in_proj GEMM shape at a quarter of the block's tokens: 8192 x 6464 x 1024
         # (135 MB of operands and output, above L2), a small case for full captures
@@ -963,7 +976,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="omit the oracle timing (it never runs inside a GPU timed region)")
     ap.add_argument("--profile", choices=["forward", "forward8", "decode", "block", "backward",
-                                          "mimo", "mimo_fwd", "gemm"],
+                                          "mimo", "mimo_fwd", "gemm", "prefill"],
                     help="run only a small case of one kernel family (for ncu captures)")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -257,6 +257,54 @@ def forward_leg(key, dev, steps, warmup, world, rank, peaks):
     return out
 
 
+def chunk_sweep_leg(dev, steps, warmup, world, rank, peaks):
+    """The forward at chunk lengths Q = 64, 128, 256 (m3ssd_dims.chunk) on the long
+    and the siso workloads, each with its HBM roofline; a side figure."""
+    import selective_state_space_m3ssd_b200 as m3
+    out = {}
+    for key in ("long", "siso"):
+        w = rank_workload(WORKLOADS[key], rank)
+        d = make_inputs(w, device=dev)
+        hT = torch.empty(w.batch, w.nheads, w.dstate, w.headdim, dtype=torch.float32, device=dev)
+        args = [d[k] for k in ("X", "logdecay", "beta", "gamma", "B", "C", "theta", "D", "h0")]
+        rows = {}
+        for Q in (64, 128, 256):
+            call = m3.PreparedFwd(*args, hT=hT, chunk=Q)
+            algo = nbytes(*(a for a in args if a is not None), call.Y, hT)
+            stream = torch.cuda.current_stream(dev)
+            for _ in range(warmup):
+                call()
+            torch.cuda.synchronize(dev)
+            if world > 1:
+                torch.distributed.barrier()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(steps):
+                call()
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            ms = e0.elapsed_time(e1)
+            if world > 1:
+                t = torch.tensor([ms], device=dev)
+                torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+                ms = float(t.item())
+            per = ms / steps
+            ach = algo / (per / 1e3) / 1e9
+            rows[f"Q{Q}"] = {"ms_per_step": per,
+                             "value": w.batch * w.seqlen * world / (per / 1e3) / 1e6,
+                             "unit": "Mtokens/s", "frac": ach / peaks["hbm_gbs"]}
+            del call
+        out[key] = {"workload": w.name, "by_chunk": rows}
+        del d, hT, args
+        torch.cuda.empty_cache()
+    best = min(out["long"]["by_chunk"].items(), key=lambda kv: kv[1]["ms_per_step"])
+    return {"metric": "scan Mtokens/s (fwd) by chunk length", "value": best[1]["value"],
+            "unit": "Mtokens/s", "ms_per_step": best[1]["ms_per_step"], "best_long": best[0],
+            "roofline": {"bound": "hbm", "frac": best[1]["frac"], "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "peak_source": peaks["source"]},
+            "sweep": out, "gpu_launches": 6 * steps}
+
+
 def prefill_leg(dev, steps, warmup, world, rank, peaks):
     """The decode workload's 512-token fp32 prefill (m3ssd_fwd on b256 H32 P64
     N128, fp32 X, B, C, Y: the chunked kernel with fp16 high / low tensor-core
@@ -747,6 +795,8 @@ def run_ours(args):
                                               peaks)
             others["prefill"] = prefill_leg(dev, min(args.steps, 10), args.warmup, world, rank,
                                             peaks)
+            others["sweep"] = chunk_sweep_leg(dev, min(args.steps, 5), args.warmup, world, rank,
+                                              peaks)
     e2e = bench_e2e(w, dev, max(1, min(args.steps, 10)), 3, fw["inp"], world)
 
     tokens = w.batch * w.seqlen * args.steps * world
@@ -774,6 +824,7 @@ def run_ours(args):
         "long_forward": others.get("long"),
         "mimo_forward": others.get("mimo"),
         "prefill_forward": others.get("prefill"),
+        "chunk_sweep": others.get("sweep"),
         "clocks": clk.summary(),
     }
     if world > 1:
@@ -797,9 +848,14 @@ def summary_of(line: dict) -> dict:
         return {"value": round(d["value"], 3), "unit": d["unit"],
                 "ms_per_step": round(d["ms_per_step"], 4), "frac": round(r.get("frac", 0.0), 3)}
     out = {"forward_siso": one(line)}
-    for k in ("ssd_forward", "long_forward", "mimo_forward", "prefill_forward", "backward",
-              "block", "gemm", "mimo_decode", "decode"):
+    for k in ("ssd_forward", "long_forward", "mimo_forward", "prefill_forward", "chunk_sweep",
+              "backward", "block", "gemm", "mimo_decode", "decode"):
         out[k] = one(line.get(k))
+    sw = line.get("chunk_sweep")
+    if sw:
+        out["chunk_sweep"]["ms_by_chunk"] = {
+            key: {q: round(v["ms_per_step"], 4) for q, v in rec["by_chunk"].items()}
+            for key, rec in sw["sweep"].items()}
     return out
 
 

@@ -93,7 +93,8 @@ typedef struct {
   int64_t headdim;  /* P >= 1 */
   int64_t dstate;   /* N >= 2, even */
   int64_t ngroups;  /* G >= 1, H % G == 0 */
-  int32_t chunk;    /* chunk length of the chunked forward: 0 = library choice, else 64 */
+  int32_t chunk;    /* chunk length of the chunked forward: 0 = library choice (64),
+                       64, or 128 / 256 (bf16, N = 128, P = 64 only; m3ssd_fwd) */
   int32_t x_dtype;  /* m3ssd_dtype of X, B, C, Y (and x_t, B_t, C_t, y_t) */
   uint32_t flags;   /* 0 or M3SSD_CHECK_FINITE */
   uint32_t reserved;/* must be 0 */
@@ -140,11 +141,22 @@ size_t m3ssd_fwd_workspace_size(const m3ssd_dims* dims);
  *            m3ssd_fwd_workspace_size(dims) bytes, 256-byte aligned (may be
  *            NULL when that size is 0).
  *
- * Paths: x_dtype = BF16 with N = 128, P = 64 and 16-byte aligned tensors runs
- * the chunked tensor-core forward (fp32 accumulation and state, bf16 operands);
- * every other valid request runs the sequential fp32 forward (N <= 256,
- * P <= 256, N*P <= 16384, else M3SSD_ERR_UNSUPPORTED).  Y is rounded once to
- * x_dtype (round-to-nearest-even); hT and the extra outputs are fp32.
+ * Paths ("TorchMamba" README, "Math notes", M2: chunkwise intra-quadratic with
+ * an inter-chunk carry):
+ *   x_dtype = BF16, N = 128, P = 64, 16-byte aligned tensors: the chunked
+ *     tensor-core forward (fp32 accumulation and state, fp16 operands converted
+ *     from the bf16 inputs; X, B, C and their Gram products must stay inside
+ *     fp16's range).  dims->chunk = 0 or 64 walks chunks of 64 rows (63 new
+ *     tokens); 128 or 256 makes the intra-chunk quadratic form span 128 or 256
+ *     rows (one CTA per SM instead of two).
+ *   x_dtype = F32, N = 128, P = 64, 16-byte aligned tensors: the chunked forward
+ *     with every product on fp16 high and low operand parts (about 2^-22 of
+ *     each term), chunk 0 or 64.
+ *   every other valid request: the sequential fp32 forward (N <= 256,
+ *     P <= 256, N*P <= 16384, else M3SSD_ERR_UNSUPPORTED); chunk 0 or 64.
+ * A chunk of 128 or 256 outside the bf16 N = 128, P = 64 path returns
+ * M3SSD_ERR_UNSUPPORTED.  Y is rounded once to x_dtype (round-to-nearest-even);
+ * hT and the extra outputs are fp32.
  */
 m3ssd_status m3ssd_fwd(const m3ssd_dims* dims, const void* X, const float* logdecay,
                        const float* beta, const float* gamma, const void* B, const void* C,

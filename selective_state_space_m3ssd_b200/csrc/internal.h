@@ -146,6 +146,11 @@ cudaError_t launch_fwd_chunk(const FwdArgs& a, cudaStream_t s);
 bool fwd_chunk_supported(const FwdArgs& a);
 // Chunked fp32 forward on the tensor cores with fp16 high / low operand parts
 // (fp32 X, B, C, Y; N = 128, P = 64; 16-byte aligned X, B, C, Y, theta, h0, hT).
+// Chunked bf16 forward with chunks of 128 or 256 rows (FwdArgs::chunk), 64-row
+// sub-tiles; same shapes and alignment as the 64-row kernel.
+bool fwd_chunk_wide_supported(const FwdArgs& a);
+cudaError_t launch_fwd_chunk_wide(const FwdArgs& a, cudaStream_t s);
+cudaError_t read_and_clear_wide_wait_timeouts(unsigned int* count);
 bool fwd_chunk32_supported(const FwdArgs& a);
 cudaError_t launch_fwd_chunk32(const FwdArgs& a, cudaStream_t s);
 cudaError_t read_and_clear_chunk32_wait_timeouts(unsigned int* count);

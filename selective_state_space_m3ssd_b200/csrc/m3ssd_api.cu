@@ -73,9 +73,10 @@ m3ssd_status m3ssd_device_wait_timeouts(uint32_t* count) {
   if (st == M3SSD_OK) st = from_cuda(m3ssd::read_and_clear_bwd_wait_timeouts(&nb));
   if (st == M3SSD_OK) st = from_cuda(m3ssd::read_and_clear_mimo_wait_timeouts(&nm));
   if (st == M3SSD_OK) st = from_cuda(m3ssd::read_and_clear_gemm_wait_timeouts(&ng));
-  unsigned int n32 = 0;
+  unsigned int n32 = 0, nw = 0;
   if (st == M3SSD_OK) st = from_cuda(m3ssd::read_and_clear_chunk32_wait_timeouts(&n32));
-  *count = n + nb + nm + ng + n32;
+  if (st == M3SSD_OK) st = from_cuda(m3ssd::read_and_clear_wide_wait_timeouts(&nw));
+  *count = n + nb + nm + ng + n32 + nw;
   return st;
 }
 
@@ -99,7 +100,8 @@ m3ssd_status m3ssd_fwd(const m3ssd_dims* dims, const void* X, const float* logde
                        void* stream) {
   m3ssd_status st = check_dims(dims);
   if (st != M3SSD_OK) return st;
-  if (dims->chunk != 0 && dims->chunk != 64) return M3SSD_ERR_UNSUPPORTED;
+  if (dims->chunk != 0 && dims->chunk != 64 && dims->chunk != 128 && dims->chunk != 256)
+    return M3SSD_ERR_UNSUPPORTED;
 
   const bool bf16 = dims->x_dtype == M3SSD_BF16;
   const uintptr_t esz = bf16 ? 2 : 4;
@@ -132,13 +134,18 @@ m3ssd_status m3ssd_fwd(const m3ssd_dims* dims, const void* X, const float* logde
 
   const bool chunked = m3ssd::fwd_chunk_supported(a);
   const bool chunked32 = !chunked && m3ssd::fwd_chunk32_supported(a);
-  if (!chunked && !chunked32 && !general_shape_ok(dims)) return M3SSD_ERR_UNSUPPORTED;
+  const bool chunked_wide = m3ssd::fwd_chunk_wide_supported(a);
+  // chunks longer than 64 rows exist only as the bf16 tensor-core kernel
+  if ((dims->chunk == 128 || dims->chunk == 256) && !chunked_wide) return M3SSD_ERR_UNSUPPORTED;
+  if (!chunked && !chunked32 && !chunked_wide && !general_shape_ok(dims))
+    return M3SSD_ERR_UNSUPPORTED;
   if (dims->batch == 0) return M3SSD_OK;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  st = from_cuda(chunked     ? m3ssd::launch_fwd_chunk(a, s)
-                 : chunked32 ? m3ssd::launch_fwd_chunk32(a, s)
-                             : m3ssd::launch_fwd_seq(a, s));
+  st = from_cuda(chunked        ? m3ssd::launch_fwd_chunk(a, s)
+                 : chunked_wide ? m3ssd::launch_fwd_chunk_wide(a, s)
+                 : chunked32    ? m3ssd::launch_fwd_chunk32(a, s)
+                                : m3ssd::launch_fwd_seq(a, s));
   if (st == M3SSD_OK && (dims->flags & M3SSD_CHECK_FINITE)) {
     st = from_cuda(m3ssd::launch_nonfinite_check(
         Y, dims->batch * dims->seqlen * dims->nheads * dims->headdim, bf16, s));

@@ -87,6 +87,8 @@ def _fwd(lib, dims, X=FAKE, ld=FAKE, beta=None, gamma=FAKE, B=FAKE, C=FAKE, thet
     (dict(x_dtype=7), m3.ERR_INVALID_ARG),
     (dict(flags=2), m3.ERR_UNSUPPORTED),
     (dict(chunk=48), m3.ERR_UNSUPPORTED),
+    (dict(chunk=128), m3.ERR_UNSUPPORTED),                  # longer chunks: bf16 N128 P64 only
+    (dict(chunk=256, x_dtype=m3.BF16), m3.ERR_UNSUPPORTED),
     (dict(dstate=512), m3.ERR_UNSUPPORTED),
     (dict(headdim=300), m3.ERR_UNSUPPORTED),
 ])

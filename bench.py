@@ -361,6 +361,25 @@ def mimo_forward_leg(dev, steps, warmup, world, rank, peaks):
         ms = float(t.item())
     per = ms / steps
     achieved = algo_bytes / (per / 1e3) / 1e9
+    # the same prefill with fp32 X, B, C, Y (the chunked kernel on fp16 high / low parts)
+    for k in ("X", "B", "C"):
+        d[k] = d[k].float()
+    args32 = [d[k] for k in ("X", "logdecay", "beta", "gamma", "B", "C", "theta", "D", "h0")]
+    Y32 = torch.empty_like(d["X"])
+    bytes32 = nbytes(*args32, Y32, hT)
+    for _ in range(warmup):
+        m3.mimo_fwd(*args32, Y=Y32)
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(steps):
+        m3.mimo_fwd(*args32, Y=Y32)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    per32 = e0.elapsed_time(e1) / steps
+    fp32 = {"ms_per_step": per32, "value": w.batch * w.seqlen * world / (per32 / 1e3) / 1e6,
+            "unit": "Mtokens/s", "algo_bytes_per_launch": bytes32,
+            "frac": bytes32 / (per32 / 1e3) / 1e9 / peaks["hbm_gbs"]}
+    del args32, Y32
     out = {"metric": "MIMO scan Mtokens/s (fwd)",
            "value": w.batch * w.seqlen * world / (per / 1e3) / 1e6,
            "unit": "Mtokens/s", "ms_per_step": per, "steps": steps,
@@ -369,7 +388,8 @@ def mimo_forward_leg(dev, steps, warmup, world, rank, peaks):
                         "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
                         "algo_bytes_per_launch": algo_bytes, "traffic": None,
                         "peak_source": peaks["source"]},
-           "gpu_launches": steps}
+           "fp32": fp32,
+           "gpu_launches": 2 * steps}
     del d, Y, hT, args
     torch.cuda.empty_cache()
     return out

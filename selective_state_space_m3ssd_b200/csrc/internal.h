@@ -137,6 +137,10 @@ cudaError_t launch_mimo_fwd(const FwdArgs& a, int64_t R, cudaStream_t s);
 bool fwd_chunk_mimo_supported(const FwdArgs& a, int64_t R);
 cudaError_t launch_fwd_chunk_mimo(const FwdArgs& a, int64_t R, cudaStream_t s);
 cudaError_t read_and_clear_mimo_wait_timeouts(unsigned int* count);
+// The same for fp32 X, B, C, Y with fp16 high / low operand parts.
+bool fwd_chunk_mimo32_supported(const FwdArgs& a, int64_t R);
+cudaError_t launch_fwd_chunk_mimo32(const FwdArgs& a, int64_t R, cudaStream_t s);
+cudaError_t read_and_clear_mimo32_wait_timeouts(unsigned int* count);
 cudaError_t launch_mimo_step(const StepArgs& a, int64_t R, cudaStream_t s);
 
 // Sequential fp32 forward: one CTA per (b, h), token by token.

@@ -76,7 +76,9 @@ m3ssd_status m3ssd_device_wait_timeouts(uint32_t* count) {
   unsigned int n32 = 0, nw = 0;
   if (st == M3SSD_OK) st = from_cuda(m3ssd::read_and_clear_chunk32_wait_timeouts(&n32));
   if (st == M3SSD_OK) st = from_cuda(m3ssd::read_and_clear_wide_wait_timeouts(&nw));
-  *count = n + nb + nm + ng + n32 + nw;
+  unsigned int nm32 = 0;
+  if (st == M3SSD_OK) st = from_cuda(m3ssd::read_and_clear_mimo32_wait_timeouts(&nm32));
+  *count = n + nb + nm + ng + n32 + nw + nm32;
   return st;
 }
 

@@ -459,10 +459,12 @@ bool mimo_shape_ok(int64_t N, int64_t P, int64_t R) {
 
 cudaError_t launch_mimo_fwd(const FwdArgs& a, int64_t R, cudaStream_t s) {
   if (a.b * a.H == 0) return cudaSuccess;
-  // bf16 at N = 128, P = 64: the chunked tensor-core kernels (rank 1 has the SISO
-  // layout and runs the SISO one)
+  // N = 128, P = 64: the chunked tensor-core kernels, bf16 or fp32 (rank 1 has the
+  // SISO layout and runs the SISO ones)
   if (R == 1 && fwd_chunk_supported(a)) return launch_fwd_chunk(a, s);
+  if (R == 1 && fwd_chunk32_supported(a)) return launch_fwd_chunk32(a, s);
   if (fwd_chunk_mimo_supported(a, R)) return launch_fwd_chunk_mimo(a, R, s);
+  if (fwd_chunk_mimo32_supported(a, R)) return launch_fwd_chunk_mimo32(a, R, s);
   const bool vec = vec_ok(a.P, R);  // the state is in shared memory (16-byte aligned)
   const size_t smem = sizeof(float) * ((size_t)(a.N * a.P) + token_smem_floats(a.N, a.P, R, vec));
   cudaError_t e;

@@ -137,3 +137,40 @@ def test_mimo_prefill_workload_sampled():
     assert rel_max_err_out(ys, yr, True) <= TOL
     for e in errs:
         assert rel_max_err(e[2], e[3]) <= TOL
+
+
+# ---- fp32 inputs: the chunked kernel with fp16 high / low operand parts, bar 1e-4 ----
+TOL32 = 1e-4
+BASE32 = BASE.with_(dtype="f32", seed=78)
+
+
+@pytest.mark.parametrize("R", [1, 2, 4, 8])
+@pytest.mark.parametrize("L", [1, 7, 64, 129, 200])
+def test_mimo_chunked_fp32_vs_oracle(R, L):
+    inp = make_mimo_inputs(BASE32.with_(seqlen=L, seed=300 + L), R)
+    inp = with_cache(inp, R, L)
+    inp["xprev0"] = torch.randn(inp["xprev0"].shape, generator=torch.Generator().manual_seed(L))
+    ref = reference(inp)
+    Y, hT, cache = run(inp, want_cache=True)
+    assert rel_max_err(f64(Y), ref["Y"]) <= TOL32
+    assert rel_max_err(f64(hT), ref["hT"]) <= TOL32
+    assert angle_err(f64(cache["angle"]), ref["angleT"]) <= 1e-5
+    np.testing.assert_array_equal(f64(cache["x_prev"]), ref["xprevT"])
+    np.testing.assert_array_equal(f64(cache["b_prev"]), ref["bprevT"])
+
+
+@pytest.mark.parametrize("R", [2, 4, 8])
+@pytest.mark.parametrize("has_beta,has_theta,with_D", [(False, False, True), (True, True, False)])
+def test_mimo_chunked_fp32_paths(R, has_beta, has_theta, with_D):
+    w = BASE32.with_(seqlen=150, has_beta=has_beta, has_theta=has_theta, seed=29, nheads=4,
+                     ngroups=2)
+    inp = make_mimo_inputs(w, R)
+    if not with_D:
+        inp["D"] = None
+    ref = reference(inp)
+    Y, hT, _ = run(inp)
+    assert rel_max_err(f64(Y), ref["Y"]) <= TOL32
+    if not with_D:
+        assert rms_rel_err(f64(Y), ref["Y"]) <= TOL32
+    assert rel_max_err(f64(hT), ref["hT"]) <= TOL32
+    assert m3.device_wait_timeouts() == 0

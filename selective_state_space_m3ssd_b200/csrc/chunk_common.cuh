@@ -64,6 +64,12 @@ __device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
 __device__ __forceinline__ float2 unpack_h2(uint32_t u) {
   return __half22float2(*reinterpret_cast<__half2*>(&u));
 }
+// v as fp16 high and low parts: hi = fp16(v), lo = fp16(v - hi), two values a word
+__device__ __forceinline__ void split_h2(float a, float b, uint32_t& hi, uint32_t& lo) {
+  hi = pack_h2(a, b);
+  const float2 h = unpack_h2(hi);
+  lo = pack_h2(a - h.x, b - h.y);
+}
 
 // 2^x by the hardware approximation (relative error about 2^-22; flushes
 // results below 2^-126 to zero).  The arguments are differences of fp32 decay

@@ -71,12 +71,6 @@ struct Smem32 {
 };
 static_assert(sizeof(Smem32) + 1024 <= 232448, "one CTA per SM");
 
-// v as fp16 high and low parts: hi = fp16(v), lo = fp16(v - hi), two values a word
-__device__ __forceinline__ void split_h2(float a, float b, uint32_t& hi, uint32_t& lo) {
-  hi = pack_h2(a, b);
-  const float2 h = unpack_h2(hi);
-  lo = pack_h2(a - h.x, b - h.y);
-}
 
 struct TmaMaps32 {
   CUtensorMap theta;  // fp32 (pair, head, token, batch), box 64 x 1 x 64 x 1

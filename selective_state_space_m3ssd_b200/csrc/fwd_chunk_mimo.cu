@@ -52,20 +52,14 @@ __device__ unsigned int g_mimo_chunk_wait_timeouts;
 
 namespace {
 
+using namespace chunk;
 using mchunk::MParams;
 using mchunk::chunk_params;
-using mchunk::ex2;
-using mchunk::fs_index;
 
-constexpr int Q = 64;       // source rows per chunk
-constexpr int NS = 128;     // state size N
-constexpr int PD = 64;      // head dim P
-constexpr int NH = NS / 2;  // rotation pairs
 constexpr int kCtrlWarp = 8;
 constexpr int kThreads = 32 * (kCtrlWarp + 1);
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kColG = 0, kColY1 = 64, kColY2 = 128, kColS = 192;
-constexpr uint32_t kAtom = Q * 128;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr uint32_t kIdescG = tc5::idesc_f16(64, 64, false, false);
 constexpr uint32_t kIdescY = tc5::idesc_f16(64, 64, false, true);
@@ -73,9 +67,6 @@ constexpr uint32_t kIdescS = tc5::idesc_f16(128, 64, true, true);
 
 typedef __nv_bfloat16 bf16;
 
-__device__ __forceinline__ uint32_t off1(int r, int c) {
-  return (uint32_t)(r * 128 + ((((c >> 3) ^ (r & 7))) << 4) + ((c & 7) << 1));
-}
 
 struct MSmem {
   float ang[32][NH];           // theta of the chunk's token rows, then their absolute angles
@@ -97,17 +88,6 @@ struct MSmem {
 };
 static_assert(2 * (sizeof(MSmem) + 1024 + 1024) <= 233472, "two CTAs per SM");
 
-__device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
-  __half2 v = __floats2half2_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&v);
-}
-__device__ __forceinline__ float2 unpack_h2(uint32_t u) {
-  return __half22float2(*reinterpret_cast<__half2*>(&u));
-}
-// the two bf16 halves of a word as floats (low element first)
-__device__ __forceinline__ float2 unpack_bf16(uint32_t u) {
-  return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
-}
 
 // 4R bytes of shared memory (R words) into registers, in 16- or 8-byte pieces.
 template <int R>

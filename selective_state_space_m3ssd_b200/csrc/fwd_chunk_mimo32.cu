@@ -37,40 +37,19 @@ __device__ unsigned int g_mimo32_wait_timeouts;
 
 namespace {
 
+using namespace chunk;
 using mchunk::MParams;
 using mchunk::chunk_params;
-using mchunk::ex2;
-using mchunk::fs_index;
 
-constexpr int Q = 64;
-constexpr int NS = 128;
-constexpr int PD = 64;
-constexpr int NH = NS / 2;
 constexpr int kCtrlWarp = 8;
 constexpr int kThreads = 32 * (kCtrlWarp + 1);
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kColG = 0, kColY1 = 64, kColY2 = 128, kColS = 192;
-constexpr uint32_t kAtom = Q * 128;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr uint32_t kIdescG = tc5::idesc_f16(64, 64, false, false);
 constexpr uint32_t kIdescY = tc5::idesc_f16(64, 64, false, true);
 constexpr uint32_t kIdescS = tc5::idesc_f16(128, 64, true, true);
 
-__device__ __forceinline__ uint32_t off1(int r, int c) {
-  return (uint32_t)(r * 128 + ((((c >> 3) ^ (r & 7))) << 4) + ((c & 7) << 1));
-}
-__device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
-  __half2 v = __floats2half2_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&v);
-}
-__device__ __forceinline__ float2 unpack_h2(uint32_t u) {
-  return __half22float2(*reinterpret_cast<__half2*>(&u));
-}
-__device__ __forceinline__ void split_h2(float a, float b, uint32_t& hi, uint32_t& lo) {
-  hi = pack_h2(a, b);
-  const float2 h = unpack_h2(hi);
-  lo = pack_h2(a - h.x, b - h.y);
-}
 // 2R floats (8R bytes, 16-byte aligned) of shared memory into registers
 template <int R>
 __device__ __forceinline__ void lds_f(const uint8_t* p, float (&v)[2 * R]) {

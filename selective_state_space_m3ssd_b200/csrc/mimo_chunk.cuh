@@ -5,17 +5,15 @@
 
 #include <stdint.h>
 
+#include "chunk_common.cuh"
+
 namespace m3ssd {
 namespace mchunk {
 
-constexpr int Q = 64;
-constexpr float kLog2e = 1.4426950408889634f;
-
-__device__ __forceinline__ float ex2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
+using chunk::Q;
+using chunk::ex2;
+using chunk::fs_index;
+using chunk::kLog2e;
 
 // Per-row chunk scalars (each row takes its token's values), double-buffered.
 struct MParams {
@@ -31,7 +29,6 @@ struct MParams {
   float pad[3];
 };
 
-__host__ __device__ constexpr int fs_index(int k, int s) { return 4 * k * (k - 1) + s; }
 
 // One warp (lane = chunk-local token j): the per-row scalars of one chunk from the
 // per-token logdecay / beta / gamma (token 0 and tokens past the end hold zeros).

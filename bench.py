@@ -63,6 +63,16 @@ def nbytes(*ts) -> int:
     return sum(t.numel() * t.element_size() for t in ts if t is not None)
 
 
+def max_over_ranks(ms: float, dev) -> float:
+    """The slowest rank's time (ms) when several ranks run, else ``ms``: every
+    multi-rank figure is the max over ranks, on the device's own process group."""
+    if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
+        return ms
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
 def load_peaks() -> dict:
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -228,10 +238,8 @@ def bench_forward(w, dev, steps, warmup, world, rank):
     torch.cuda.synchronize(dev)
     ms = e0.elapsed_time(e1)
     if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = max_over_ranks(ms, dev)
         torch.distributed.barrier()
-        ms = float(t.item())
     torch.cuda.synchronize(dev)
     return {"ms_total": ms, "ms_per_step": ms / steps, "algo_bytes": algo_bytes, "inp": inp,
             "dev_inputs": d, "call": call, "launches": steps}
@@ -285,9 +293,7 @@ def chunk_sweep_leg(dev, steps, warmup, world, rank, peaks):
             torch.cuda.synchronize(dev)
             ms = e0.elapsed_time(e1)
             if world > 1:
-                t = torch.tensor([ms], device=dev)
-                torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-                ms = float(t.item())
+                ms = max_over_ranks(ms, dev)
             per = ms / steps
             ach = algo / (per / 1e3) / 1e9
             rows[f"Q{Q}"] = {"ms_per_step": per,
@@ -356,9 +362,7 @@ def mimo_forward_leg(dev, steps, warmup, world, rank, peaks):
     torch.cuda.synchronize(dev)
     ms = e0.elapsed_time(e1)
     if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+        ms = max_over_ranks(ms, dev)
     per = ms / steps
     achieved = algo_bytes / (per / 1e3) / 1e9
     # the same prefill with fp32 X, B, C, Y (the chunked kernel on fp16 high / low parts)
@@ -458,9 +462,7 @@ def bench_e2e(w, dev, steps, warmup, inp_cpu, world):
     torch.cuda.synchronize(dev)
     ms = e0.elapsed_time(e1)
     if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+        ms = max_over_ranks(ms, dev)
     tokens = w.batch * w.seqlen * steps * world
     return {"value": tokens / (ms / 1e3) / 1e6, "unit": UNIT, "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "ms_per_step": ms / steps,
@@ -726,9 +728,7 @@ def bench_backward(w, dev, steps, world, d, peaks):
     torch.cuda.synchronize(dev)
     ms = e0.elapsed_time(e1) / steps
     if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+        ms = max_over_ranks(ms, dev)
     algo = nbytes(*args, dY, dhT, *grads.values())
     flops = bwd_chunk_flops(w.batch, w.seqlen, w.nheads) * world
     executed = bwd_tc_mma_flops(w.batch, w.seqlen, w.nheads) * world

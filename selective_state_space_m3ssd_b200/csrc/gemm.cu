@@ -40,8 +40,8 @@
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
 
+#include <cstddef>
 #include <cstring>
-#include <mutex>
 
 #include "internal.h"
 #include "tc5.cuh"
@@ -74,6 +74,8 @@ constexpr uint32_t kStgBytes = 32 * 32 * 2;  // one warp's 32 x 32 bf16 output b
 template <int H>
 struct GSmem {
   static constexpr int S = Cfg<H>::STAGES;
+  // every buffer a TMA copy reads or writes starts on a 1024-byte boundary (the
+  // struct is placed at one, and each array before it is a multiple of 1024 bytes)
   uint8_t a[S][H * kABytes];
   uint8_t w[S][kWBytes];
   uint8_t stg[Cfg<H>::EPI_WARPS][2][kStgBytes];  // output staging, two blocks an epilogue warp
@@ -88,6 +90,9 @@ struct GSmem {
 
 static_assert(sizeof(GSmem<1>) + 1024 <= 232448 && sizeof(GSmem<2>) + 1024 <= 232448,
               "one CTA's shared memory");
+static_assert(offsetof(GSmem<1>, w) % 1024 == 0 && offsetof(GSmem<1>, stg) % 1024 == 0 &&
+                  offsetof(GSmem<2>, w) % 1024 == 0 && offsetof(GSmem<2>, stg) % 1024 == 0,
+              "TMA buffers on 1024-byte boundaries");
 
 struct GMaps {
   CUtensorMap a;  // bf16 (K, M), box 64 x 128 H, 128-byte swizzle
@@ -307,16 +312,15 @@ bool encode_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// SMs of the current device (the grid is one persistent CTA per SM).
 int sm_count() {
-  static int n = 0;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-      n = 148;
-  });
-  return n > 0 ? n : 148;
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+    (void)cudaGetLastError();
+    return 148;
+  }
+  return n;
 }
 
 template <int H>

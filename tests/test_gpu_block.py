@@ -48,6 +48,9 @@ SHAPES = {
     "chunked": dict(batch=2, seqlen=200, d_model=64, nheads=2, headdim=64, dstate=128, ngroups=1),
     # one token
     "one_token": dict(batch=3, seqlen=1, d_model=32, nheads=4, headdim=8, dstate=8, ngroups=1),
+    # in_proj rows of 75 values (off the 16-byte grid): the GEMM's plain stores and the
+    # element-wise gate and prep kernels
+    "odd_width": dict(batch=2, seqlen=33, d_model=32, nheads=3, headdim=8, dstate=6, ngroups=1),
 }
 
 

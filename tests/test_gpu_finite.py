@@ -15,6 +15,7 @@ pytestmark = pytest.mark.gpu
 KEYS = ("X", "logdecay", "beta", "gamma", "B", "C", "theta", "D", "h0")
 
 CASES = {"chunked_bf16": WORKLOADS["siso"].with_(batch=1, nheads=2, seqlen=130, seed=31),
+         "chunked_f32": WORKLOADS["siso"].with_(batch=1, nheads=2, seqlen=130, seed=35, dtype="f32"),
          "sequential_f32": WORKLOADS["tiny"].with_(seed=32)}
 
 
@@ -69,4 +70,18 @@ def test_mimo_forward_reports_a_planted_nonfinite_value():
     assert not m3.nonfinite_outputs()
     dev[0][0, 3, 1, 2, 1] = math.inf
     m3.mimo_fwd(dev[0], dev[1], None, dev[2], dev[3], dev[4], check_finite=True)
+    assert m3.nonfinite_outputs()
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_chunked_mimo_forward_reports_a_planted_nonfinite_value(dtype):
+    from selective_state_space_m3ssd_b200.synth import make_mimo_inputs
+    inp = make_mimo_inputs(WORKLOADS["siso"].with_(batch=1, nheads=2, seqlen=50, seed=36,
+                                                   dtype=dtype), 4)
+    d = {k: (None if v is None else v.cuda()) for k, v in inp.items()}
+    m3.nonfinite_outputs()
+    m3.mimo_fwd(*(d[k] for k in KEYS), check_finite=True)
+    assert not m3.nonfinite_outputs()
+    d["X"][0, 9, 1, 3, 2] = math.nan
+    m3.mimo_fwd(*(d[k] for k in KEYS), check_finite=True)
     assert m3.nonfinite_outputs()

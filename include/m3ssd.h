@@ -373,8 +373,10 @@ m3ssd_status m3ssd_block_fwd(const m3ssd_block_dims* dims, const m3ssd_block_wei
  * K a multiple of 8; D: bf16, ldd >= N, 2-byte aligned (16-byte stores when D
  * is 16-byte aligned and ldd a multiple of 8).  fp32 accumulation on the
  * tensor cores, each output rounded once to bf16 (nearest even).  M, N, K up
- * to 2^31 - 1; M = 0 or N = 0 does nothing.  Other shapes or alignments:
- * M3SSD_ERR_INVALID_ARG.  No allocation, no synchronisation.
+ * to 2^31 - 1 with at most 2^31 - 1 output tiles of 128 x 256; M = 0 or N = 0
+ * does nothing.  Other shapes or alignments: M3SSD_ERR_INVALID_ARG (or
+ * M3SSD_ERR_CUDA for a tile count past that limit).  No allocation, no
+ * synchronisation.
  */
 m3ssd_status m3ssd_gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, const void* W,
                              void* D, int64_t ldd, void* stream);

@@ -347,6 +347,7 @@ cudaError_t launch_gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, con
   // two row halves when their tiles fill at least 90 % of the SM rounds and
   // not much less evenly than single-half tiles
   const int64_t nt = (N + BN - 1) / BN, sms = sm_count();
+  if (((M + BM - 1) / BM) * nt > INT32_MAX) return cudaErrorInvalidValue;  // tile index is an int
   const int64_t t1 = ((M + BM - 1) / BM) * nt, t2 = ((M + 2 * BM - 1) / (2 * BM)) * nt;
   const double f1 = (double)t1 / (double)(((t1 + sms - 1) / sms) * sms);
   const double f2 = (double)t2 / (double)(((t2 + sms - 1) / sms) * sms);

@@ -965,6 +965,18 @@ def run_profile(args):
             m3.bwd(*args_, dY=dY)
         torch.cuda.synchronize(dev)
         print(json.dumps({"profile": "backward", "workload": "siso shape b1 L1024 H32 P64 N128"}))
+    elif args.profile == "wide":
+        # the forward at chunk length 128 on the long workload's shape at a quarter of its
+        # heads: b2 L32768 H12 (about 420 MB of inputs and outputs, above L2)
+        w = WORKLOADS["long"].with_(nheads=12)
+        d = make_inputs(w, device=dev)
+        hT = torch.empty(w.batch, w.nheads, w.dstate, w.headdim, dtype=torch.float32, device=dev)
+        call = m3.PreparedFwd(*(d[k] for k in ("X", "logdecay", "beta", "gamma", "B", "C", "theta",
+                                               "D", "h0")), hT=hT, chunk=128)
+        for _ in range(args.warmup + args.steps):
+            call()
+        torch.cuda.synchronize(dev)
+        print(json.dumps({"profile": "wide", "workload": "long shape b2 L32768 H12, chunk 128"}))
     elif args.profile == "prefill":
         # the fp32 prefill at a quarter of the decode batch: b64 L512 H32 (about 0.8 GB
         # of inputs and outputs, above L2), a small case of the fp32 chunked kernel
@@ -1052,7 +1064,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="omit the oracle timing (it never runs inside a GPU timed region)")
     ap.add_argument("--profile", choices=["forward", "forward8", "decode", "block", "backward",
-                                          "mimo", "mimo_fwd", "gemm", "prefill"],
+                                          "mimo", "mimo_fwd", "gemm", "prefill", "wide"],
                     help="run only a small case of one kernel family (for ncu captures)")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -122,9 +122,20 @@ typedef struct {
   float* b_prev;  /* (b, G, N), unrotated */
 } m3ssd_cache;
 
-/* Bytes of device workspace m3ssd_fwd needs for these dims (0 today).
- * Returns 0 as well for invalid dims (m3ssd_fwd then reports the error). */
+/* Bytes of device workspace m3ssd_fwd needs for these dims on the current
+ * device: non-zero only when the chunked bf16 forward (N = 128, P = 64, chunk 0
+ * or 64) splits each sequence into segments (see m3ssd_fwd), which depends on
+ * batch, seqlen, nheads and the device's SM count, so query it on the device
+ * that runs the call.  0 for invalid dims (m3ssd_fwd then reports the error)
+ * and when no device is present. */
 size_t m3ssd_fwd_workspace_size(const m3ssd_dims* dims);
+
+/* The segment count and the chunks per segment that m3ssd_fwd would use for
+ * batch x nheads sequences of seqlen tokens on a device with `sms` SMs
+ * (*nseg = 1: no split).  Host arithmetic only; for tests and tuning.
+ * M3SSD_ERR_INVALID_ARG for NULL outputs or negative sizes. */
+m3ssd_status m3ssd_test_fwd_split_plan(int64_t batch, int64_t seqlen, int64_t nheads,
+                                       int32_t sms, int32_t* nseg, int32_t* segc);
 
 /*
  * Forward scan over a whole sequence ("TorchMamba" README, "Functional cores":
@@ -148,7 +159,15 @@ size_t m3ssd_fwd_workspace_size(const m3ssd_dims* dims);
  *     from the bf16 inputs; X, B, C and their Gram products must stay inside
  *     fp16's range).  dims->chunk = 0 or 64 walks chunks of 64 rows (63 new
  *     tokens); 128 or 256 makes the intra-chunk quadratic form span 128 or 256
- *     rows (one CTA per SM instead of two).
+ *     rows (one CTA per SM instead of two).  With chunks of 64 rows and too few
+     (b, h) sequences to fill the device (b*H at most two thirds of its SM
+     count, at least 16 chunks), each sequence is cut into segments of at
+     least 8 chunks: a pass builds every segment's state from a zero start
+     and the linear recurrence links them (each segment's start state is the
+     decayed previous start plus the previous segment's state, rotated to the
+     absolute angle), then all segments run at once.  The result equals the
+     unsplit walk up to fp32 rounding order; the workspace holds the segment
+     states (64 KB per sequence and segment).
  *   x_dtype = F32, N = 128, P = 64, 16-byte aligned tensors: the chunked forward
  *     with every product on fp16 high and low operand parts (about 2^-22 of
  *     each term), chunk 0 or 64.
@@ -405,9 +424,10 @@ m3ssd_status m3ssd_device_wait_timeouts(uint32_t* count);
  * be called while work of this library is in flight or being captured.
  *   m3ssd_test_set_wait_limit: the time limit of the chunked forward's bounded
  *     waits, in nanoseconds (0 restores the default of 2 s).
- *   m3ssd_test_drop_next_gram_signal: the next chunked-forward sequence to
- *     start leaves out the completion signal of its first Gram product, so its
- *     compute warps' wait for it runs out: that launch counts one timeout in
+ *   m3ssd_test_drop_next_gram_signal: the next chunked forward that rotates
+ *     (theta or angle0 given) and is not split into segments leaves out the
+ *     completion signal of its first Gram product, so its compute warps'
+ *     wait for it runs out: that launch counts one timeout in
  *     m3ssd_device_wait_timeouts and leaves its outputs undefined; the GPU
  *     context stays usable and later launches are unaffected.
  */

@@ -140,6 +140,9 @@ def load(path: str | None = None):
         lib.m3ssd_test_set_wait_limit.restype = ctypes.c_int
         lib.m3ssd_test_drop_next_gram_signal.argtypes = []
         lib.m3ssd_test_drop_next_gram_signal.restype = ctypes.c_int
+        i64, i32p = ctypes.c_int64, ctypes.POINTER(ctypes.c_int32)
+        lib.m3ssd_test_fwd_split_plan.argtypes = [i64, i64, i64, ctypes.c_int32, i32p, i32p]
+        lib.m3ssd_test_fwd_split_plan.restype = ctypes.c_int
         if path is None:
             _lib = lib
         return lib
@@ -223,6 +226,16 @@ def drop_next_gram_signal_for_tests():
     signal, so one of its bounded waits runs out (reported by
     device_wait_timeouts; that launch's outputs are undefined)."""
     _check(load().m3ssd_test_drop_next_gram_signal(), "m3ssd_test_drop_next_gram_signal")
+
+
+def fwd_split_plan(batch: int, seqlen: int, nheads: int, sms: int) -> tuple:
+    """(segments, chunks per segment) of the chunked bf16 forward's sequence
+    split for this shape on a device with ``sms`` SMs; (1, 0) means no split."""
+    nseg, segc = ctypes.c_int32(), ctypes.c_int32()
+    _check(load().m3ssd_test_fwd_split_plan(int(batch), int(seqlen), int(nheads), int(sms),
+                                            ctypes.byref(nseg), ctypes.byref(segc)),
+           "m3ssd_test_fwd_split_plan")
+    return nseg.value, segc.value
 
 
 def make_dims(batch, seqlen, nheads, headdim, dstate, ngroups, x_dtype, chunk=0, flags=0) -> Dims:

@@ -124,7 +124,7 @@ struct TmaMaps {
   CUtensorMap X;      // bf16 (p, head, token, batch), box 64 x 1 x 64 x 1, 128-byte swizzle
 };
 
-template <bool ROT, bool BIAS, bool TH16, bool TEST>
+template <bool ROT, bool BIAS, bool TH16, bool TEST, bool SEG>
 __global__ void __launch_bounds__(kThreads, 2)
     fwd_chunk_kernel(FwdArgs a, const __grid_constant__ TmaMaps tm) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -139,9 +139,21 @@ __global__ void __launch_bounds__(kThreads, 2)
   const bool ctrl = warp == kCtrlWarp;
   const bool ctrl_lead = tid == kCtrlWarp * 32;
   const int64_t H = a.H, L = a.L, G = a.G;
-  const int64_t bh = blockIdx.x;
+  // CTA (b H + h) nseg + k walks segment k of sequence (b, h): chunks c_lo .. c_hi - 1
+  // (the instances that never split keep the single-segment arithmetic constant)
+  const int nseg = SEG ? a.nseg : 1;
+  const int64_t bh = blockIdx.x / nseg;
+  const int seg = (int)(blockIdx.x - bh * nseg);
   const int64_t b = bh / H, h = bh % H, g = h / (H / G);
-  const int nC = (int)((L + QT - 1) / QT);
+  const int nCt = (int)((L + QT - 1) / QT);
+  const int c_lo = nseg > 1 ? seg * a.segc : 0;
+  const int c_hi = nseg > 1 ? min(c_lo + a.segc, nCt) : nCt;
+  const bool seg_first = seg == 0, seg_last = seg == nseg - 1;
+  // the start state and angle: the caller's for the first segment, else the
+  // combine step's
+  const int64_t su = bh * (nseg - 1) + seg - 1;
+  const float* h0p = seg_first ? (a.h0 ? a.h0 + bh * NS * PD : nullptr) : a.hseg + su * NS * PD;
+  const float* ang0 = seg_first ? (a.angle0 ? a.angle0 + bh * NH : nullptr) : a.aseg + su * NH;
   const bf16* Xg = static_cast<const bf16*>(a.X);
   const bf16* Bg = static_cast<const bf16*>(a.B);
   bf16* Yg = static_cast<bf16*>(a.Y);
@@ -202,30 +214,30 @@ __global__ void __launch_bounds__(kThreads, 2)
   __syncthreads();  // mbarriers initialised
   if (ctrl_lead) {
     tc5::mbar_arrive_expect_tx(&sm.lmbar, chunk_bytes);
-    if (ROT && has_theta) tma_theta(0);
-    tma_bc(0, &tm.B, aB);
-    tma_bc(0, &tm.C, aC);
-    tma_x(0);
+    if (ROT && has_theta) tma_theta(c_lo);
+    tma_bc(c_lo, &tm.B, aB);
+    tma_bc(c_lo, &tm.C, aC);
+    tma_x(c_lo);
   }
   if (ctrl) {
-    load_params(0);
-    chunk_params(sm.prm[0], pld, pbe, pga, lane, inv_a);
-    if (nC > 1) load_params(1);
+    load_params(c_lo);
+    chunk_params(sm.prm[c_lo & 1], pld, pbe, pga, lane, inv_a);
+    if (c_lo + 1 < c_hi) load_params(c_lo + 1);
   }
   // row 0 of chunk 0 is the cache's previous token (the TMA zero-fills it; it is
   // patched once that copy has landed)
-  const float bp0 = (tid < NS && a.bprev0) ? a.bprev0[(b * G + g) * NS + tid] : 0.f;
-  const float xp0 = (tid < PD && a.xprev0) ? a.xprev0[bh * PD + tid] : 0.f;
-  const bool patch_row0 = a.bprev0 != nullptr || a.xprev0 != nullptr;
-  if (ROT && tid < NH) sm.Phi[tid] = wrap_angle(a.angle0 ? a.angle0[bh * NH + tid] : 0.f);
+  const bool patch_row0 = seg_first && (a.bprev0 != nullptr || a.xprev0 != nullptr);
+  const float bp0 = (patch_row0 && tid < NS && a.bprev0) ? a.bprev0[(b * G + g) * NS + tid] : 0.f;
+  const float xp0 = (patch_row0 && tid < PD && a.xprev0) ? a.xprev0[bh * PD + tid] : 0.f;
+  if (ROT && tid < NH) sm.Phi[tid] = wrap_angle(ang0 ? ang0[tid] : 0.f);
 
   // state fragment (compute warps): row n = 32 (warp % 4) + lane, columns cb .. cb + 31
   const int n_row = 32 * (warp & 3) + lane, cb = 32 * ((warp >> 2) & 1);
   float hs[32];
 #pragma unroll
   for (int j = 0; j < 32; ++j) hs[j] = 0.f;
-  if (!ctrl && a.h0) {
-    const float4* src = reinterpret_cast<const float4*>(a.h0 + (bh * NS + n_row) * PD + cb);
+  if (!ctrl && h0p) {
+    const float4* src = reinterpret_cast<const float4*>(h0p + n_row * PD + cb);
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       const float4 v = src[j];
@@ -236,9 +248,10 @@ __global__ void __launch_bounds__(kThreads, 2)
   // warps only; one named barrier)
   int kexp = 0;
   auto store_state_f16 = [&]() {
-    float m = 0.f;
+    float m4[4] = {0.f, 0.f, 0.f, 0.f};  // four independent chains
 #pragma unroll
-    for (int j = 0; j < 32; ++j) m = fmaxf(m, fabsf(hs[j]));
+    for (int j = 0; j < 32; ++j) m4[j & 3] = fmaxf(m4[j & 3], fabsf(hs[j]));
+    float m = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     if (lane == 0) sm.hmax[warp] = m;
@@ -246,13 +259,11 @@ __global__ void __launch_bounds__(kThreads, 2)
     m = sm.hmax[0];
 #pragma unroll
     for (int w = 1; w < 8; ++w) m = fmaxf(m, sm.hmax[w]);
-    kexp = 0;
-    if (m > 0.f) {
-      int e;
-      frexpf(m, &e);  // m < 2^e
-      kexp = min(max(14 - e, -100), 100);
-    }
-    const float sc = ldexpf(1.f, kexp);
+    // m < 2^e, e = biased exponent - 126 for a normal m (a subnormal m reads as
+    // e = -126, which the clamp maps to 100, as an exact frexp would)
+    const int e = (int)((__float_as_uint(m) >> 23) & 0xffu) - 126;
+    kexp = m > 0.f ? min(max(14 - e, -100), 100) : 0;
+    const float sc = __uint_as_float((uint32_t)(127 + kexp) << 23);  // 2^kexp
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       uint4 v;
@@ -287,9 +298,9 @@ __global__ void __launch_bounds__(kThreads, 2)
   const uint32_t tlane = (uint32_t)(32 * (warp & 3)) << 16;
 
   // ---- chunk walk -------------------------------------------------------------
-  for (int c = 0; c < nC; ++c) {
+  for (int c = c_lo; c < c_hi; ++c) {
     const int64_t tbase = (int64_t)c * QT - 1;  // token of row 0
-    const uint32_t par = (uint32_t)(c & 1);
+    const uint32_t par = (uint32_t)((c - c_lo) & 1);
     const ChunkParams& P = sm.prm[c & 1];
     const uint8_t* Xs = sm.X[c & 1];
     const uint32_t aX = aX0 + (uint32_t)(c & 1) * (Q * 128);
@@ -303,19 +314,19 @@ __global__ void __launch_bounds__(kThreads, 2)
       // the CTA frees TMEM and exits (Y2 is that chunk's last commit; it covers
       // every product the control thread issued before it)
       (void)tc5::mbar_wait(&sm.lmbar, par, wait_ns);
-      if (c > 0) (void)tc5::mbar_wait(&sm.mbar[2], par ^ 1u, wait_ns);
+      if (c > c_lo) (void)tc5::mbar_wait(&sm.mbar[2], par ^ 1u, wait_ns);
       break;
     }
 
     if (ctrl) {
       // ===================== control warp ======================================
-      if (ctrl_lead && c + 1 < nC) {
+      if (ctrl_lead && c + 1 < c_hi) {
         tc5::mbar_arrive_expect_tx(&sm.lmbar, chunk_bytes);
         tma_x(c + 1);
       }
-      if (c + 1 < nC) {
+      if (c + 1 < c_hi) {
         chunk_params(sm.prm[(c + 1) & 1], pld, pbe, pga, lane, inv_a);
-        if (c + 2 < nC) load_params(c + 2);
+        if (c + 2 < c_hi) load_params(c + 2);
       }
       // descriptors of the operand tiles: an offset inside a tile only adds
       // (offset >> 4) to the start-address field (shared addresses stay below 256 KB)
@@ -334,7 +345,7 @@ __global__ void __launch_bounds__(kThreads, 2)
           tc5::mma_bf16(tmem + kColG, dC + ko, dB + ko, kIdescG, j > 0);
         }
         // the testing instance's first CTA leaves its first Gram signal out
-        if (!(TEST && c == 0 && blockIdx.x == 0)) tc5::commit(&sm.mbar[0]);
+        if (!(TEST && c == c_lo && blockIdx.x == 0)) tc5::commit(&sm.mbar[0]);
         // S = Bbar^T (W_end o X) (A and B MN-major), K = 64 source rows
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -350,7 +361,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
         tc5::commit(&sm.mbar[1]);
         // the Gram and S consume Bbar: refill it for the next chunk before joining S4
-        if (c + 1 < nC) {
+        if (c + 1 < c_hi) {
           if (!tc5::mbar_wait(&sm.mbar[3], par, wait_ns)) sm.err = 1;
           tma_bc(c + 1, &tm.B, aB);
         }
@@ -368,7 +379,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         // Y1 and S consume Cbar and W_end o X (theta's space): refill them once
         // those products are done, after Y2 is on its way (in the bias instances
         // Y2 reads the mask's residual from theta's space too)
-        if (c + 1 < nC) {
+        if (c + 1 < c_hi) {
           if (!tc5::mbar_wait(&sm.mbar[BIAS ? 2 : 1], par, wait_ns)) sm.err = 1;
           tma_bc(c + 1, &tm.C, aC);
           if (ROT && has_theta) tma_theta(c + 1);
@@ -378,7 +389,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
 
     // ===================== compute warps (0..7) ===================================
-    if (c == 0 && patch_row0) {
+    if (c == 0 && patch_row0) {  // (the first segment's first chunk)
       if (tid < NS) *reinterpret_cast<bf16*>(sm.B + off2(0, tid)) = __float2bfloat16_rn(bp0);
       if (tid < PD) *reinterpret_cast<bf16*>(sm.X[0] + off1(0, tid)) = __float2bfloat16_rn(xp0);
     }
@@ -425,8 +436,10 @@ __global__ void __launch_bounds__(kThreads, 2)
       float2 base = make_float2(0.f, 0.f);
       if (ROT) {
         base = *reinterpret_cast<const float2*>(&sm.Phi[2 * lane]);
-        for (int s2 = 0; s2 < warp; ++s2)
-          base = __fadd2_rn(base, *reinterpret_cast<const float2*>(&sm.segtot[s2][2 * lane]));
+#pragma unroll
+        for (int s2 = 0; s2 < 7; ++s2)
+          if (s2 < warp)
+            base = __fadd2_rn(base, *reinterpret_cast<const float2*>(&sm.segtot[s2][2 * lane]));
       }
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
@@ -570,7 +583,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       tc5::ld_16x256b_x4(tmem + tlane + kColY2 + (uint32_t)cb, y2);
       tc5::wait_ld();
       const float2 D2 = make_float2(Dh, Dh);
-      const float isc = ldexpf(1.f, -kexp);  // Hs holds h 2^kexp
+      const float isc = __uint_as_float((uint32_t)(127 - kexp) << 23);  // Hs holds h 2^kexp
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf) {
         const int r = 16 * (warp & 3) + (lane >> 2) + 8 * hf;
@@ -612,7 +625,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   // ---- outputs of the last token, TMEM release ---------------------------------
   if (sm.err) {
     if (tid == 0) atomicAdd(&g_chunk_wait_timeouts, 1u);
-  } else if (!ctrl) {
+  } else if (!ctrl && seg_last) {
     if (a.hT) {
       float4* dst = reinterpret_cast<float4*>(a.hT + (bh * NS + n_row) * PD + cb);
 #pragma unroll
@@ -665,7 +678,7 @@ bool encode_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64
 
 namespace {
 
-template <bool ROT, bool BIAS, bool TH16, bool TEST = false>
+template <bool ROT, bool BIAS, bool TH16, bool TEST = false, bool SEG = false>
 cudaError_t launch_variant(const FwdArgs& a, cudaStream_t s) {
   TmaMaps tm;
   memset(&tm, 0, sizeof(tm));
@@ -684,10 +697,11 @@ cudaError_t launch_variant(const FwdArgs& a, cudaStream_t s) {
                     CU_TENSOR_MAP_SWIZZLE_NONE);
   if (!ok) return cudaErrorInvalidValue;
   const size_t smem = sizeof(Smem) + 1024;
-  cudaError_t e = cudaFuncSetAttribute(fwd_chunk_kernel<ROT, BIAS, TH16, TEST>,
+  cudaError_t e = cudaFuncSetAttribute(fwd_chunk_kernel<ROT, BIAS, TH16, TEST, SEG>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  fwd_chunk_kernel<ROT, BIAS, TH16, TEST><<<(unsigned)(a.b * a.H), kThreads, smem, s>>>(a, tm);
+  const int64_t nseg = SEG ? a.nseg : 1;
+  fwd_chunk_kernel<ROT, BIAS, TH16, TEST, SEG><<<(unsigned)(a.b * a.H * nseg), kThreads, smem, s>>>(a, tm);
   return cudaGetLastError();
 }
 
@@ -713,6 +727,11 @@ cudaError_t launch_fwd_chunk(const FwdArgs& a, cudaStream_t s) {
     return launch_variant<true, true, true>(a, s);
   }
   if (a.Bbias != nullptr || a.Cbias != nullptr) return launch_variant<true, true, false>(a, s);
+  if (a.nseg > 1) {  // the segments of a split sequence (the public scan only)
+    if (a.hseg == nullptr || a.aseg == nullptr || a.segc < 1) return cudaErrorInvalidValue;
+    if (a.theta != nullptr || a.angle0 != nullptr) return launch_variant<true, false, false, false, true>(a, s);
+    return launch_variant<false, false, false, false, true>(a, s);
+  }
   if (a.theta != nullptr || a.angle0 != nullptr) {
     if (g_test_launch_requested.exchange(false)) return launch_variant<true, false, false, true>(a, s);
     return launch_variant<true, false, false>(a, s);

@@ -45,6 +45,15 @@ struct FwdArgs {
   const void* theta16;
   int64_t theta16_tok_stride;
   const float* A_log;
+  // Sequence split of the chunked bf16 forward (0 or 1: one CTA walks each whole
+  // sequence).  With nseg > 1, CTA (b h) nseg + k walks chunks [k segc,
+  // min((k + 1) segc, chunks)) of sequence (b, h); segment k >= 1 starts from the
+  // state hseg + ((b H + h)(nseg - 1) + k - 1) N P (fp32, (n, p)) and the angle
+  // aseg + (same index) N / 2 that the segment pass and its combine step wrote,
+  // and only the last segment writes hT and the cache outputs.
+  int nseg, segc;
+  const float* hseg;
+  const float* aseg;
 };
 
 struct StepArgs {
@@ -148,6 +157,20 @@ cudaError_t launch_fwd_seq(const FwdArgs& a, cudaStream_t s);
 // Chunked bf16 tensor-core forward (N = 128, P = 64).
 cudaError_t launch_fwd_chunk(const FwdArgs& a, cudaStream_t s);
 bool fwd_chunk_supported(const FwdArgs& a);
+// Sequence split of that forward for launches with few (b, h) sequences: the
+// number of segments a sequence is cut into (1: no split) and the chunks a
+// segment holds, from the shape and the device's SM count; the workspace the
+// split needs (0 without a split); and the split launch itself (the segment
+// pass, the combine step and the chunked forward over every segment).
+struct SplitPlan {
+  int nseg, segc;
+};
+SplitPlan fwd_split_plan(int64_t b, int64_t L, int64_t H, int sms);
+size_t fwd_split_workspace_bytes(int64_t b, int64_t H, const SplitPlan& p);
+cudaError_t launch_fwd_split(const FwdArgs& a, const SplitPlan& p, void* workspace, cudaStream_t s);
+cudaError_t read_and_clear_seg_wait_timeouts(unsigned int* count);
+// SM count of the current device (0 when there is none).
+int current_device_sms();
 // Chunked fp32 forward on the tensor cores with fp16 high / low operand parts
 // (fp32 X, B, C, Y; N = 128, P = 64; 16-byte aligned X, B, C, Y, theta, h0, hT).
 // Chunked bf16 forward with chunks of 128 or 256 rows (FwdArgs::chunk), 64-row

@@ -40,6 +40,13 @@ m3ssd_status from_cuda(cudaError_t e) {
   return M3SSD_ERR_CUDA;
 }
 
+// Shapes whose chunked bf16 forward may be split along the sequence (the split
+// itself depends on the batch, heads, length and the device's SM count).
+bool split_candidate(const m3ssd_dims* d) {
+  return d && check_dims(d) == M3SSD_OK && d->x_dtype == M3SSD_BF16 && d->dstate == 128 &&
+         d->headdim == 64 && (d->chunk == 0 || d->chunk == 64);
+}
+
 }  // namespace
 
 extern "C" {
@@ -76,9 +83,10 @@ m3ssd_status m3ssd_device_wait_timeouts(uint32_t* count) {
   unsigned int n32 = 0, nw = 0;
   if (st == M3SSD_OK) st = from_cuda(m3ssd::read_and_clear_chunk32_wait_timeouts(&n32));
   if (st == M3SSD_OK) st = from_cuda(m3ssd::read_and_clear_wide_wait_timeouts(&nw));
-  unsigned int nm32 = 0;
+  unsigned int nm32 = 0, ns = 0;
   if (st == M3SSD_OK) st = from_cuda(m3ssd::read_and_clear_mimo32_wait_timeouts(&nm32));
-  *count = n + nb + nm + ng + n32 + nw + nm32;
+  if (st == M3SSD_OK) st = from_cuda(m3ssd::read_and_clear_seg_wait_timeouts(&ns));
+  *count = n + nb + nm + ng + n32 + nw + nm32 + ns;
   return st;
 }
 
@@ -91,8 +99,20 @@ m3ssd_status m3ssd_test_drop_next_gram_signal(void) {
 }
 
 size_t m3ssd_fwd_workspace_size(const m3ssd_dims* dims) {
-  (void)dims;
-  return 0;
+  if (!split_candidate(dims)) return 0;
+  const m3ssd::SplitPlan p =
+      m3ssd::fwd_split_plan(dims->batch, dims->seqlen, dims->nheads, m3ssd::current_device_sms());
+  return m3ssd::fwd_split_workspace_bytes(dims->batch, dims->nheads, p);
+}
+
+m3ssd_status m3ssd_test_fwd_split_plan(int64_t batch, int64_t seqlen, int64_t nheads,
+                                       int32_t sms, int32_t* nseg, int32_t* segc) {
+  if (!nseg || !segc || batch < 0 || seqlen < 0 || nheads < 0 || sms < 0)
+    return M3SSD_ERR_INVALID_ARG;
+  const m3ssd::SplitPlan p = m3ssd::fwd_split_plan(batch, seqlen, nheads, sms);
+  *nseg = p.nseg;
+  *segc = p.segc;
+  return M3SSD_OK;
 }
 
 m3ssd_status m3ssd_fwd(const m3ssd_dims* dims, const void* X, const float* logdecay,
@@ -135,6 +155,11 @@ m3ssd_status m3ssd_fwd(const m3ssd_dims* dims, const void* X, const float* logde
     return M3SSD_ERR_WORKSPACE;
 
   const bool chunked = m3ssd::fwd_chunk_supported(a);
+  const m3ssd::SplitPlan plan =
+      need > 0 ? m3ssd::fwd_split_plan(a.b, a.L, a.H, m3ssd::current_device_sms())
+               : m3ssd::SplitPlan{1, 0};
+  const bool split = chunked && plan.nseg > 1 &&
+                     m3ssd::fwd_split_workspace_bytes(a.b, a.H, plan) <= workspace_bytes;
   const bool chunked32 = !chunked && m3ssd::fwd_chunk32_supported(a);
   const bool chunked_wide = m3ssd::fwd_chunk_wide_supported(a);
   // chunks longer than 64 rows exist only as the bf16 tensor-core kernel
@@ -144,7 +169,8 @@ m3ssd_status m3ssd_fwd(const m3ssd_dims* dims, const void* X, const float* logde
   if (dims->batch == 0) return M3SSD_OK;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  st = from_cuda(chunked        ? m3ssd::launch_fwd_chunk(a, s)
+  st = from_cuda(split          ? m3ssd::launch_fwd_split(a, plan, workspace, s)
+                 : chunked      ? m3ssd::launch_fwd_chunk(a, s)
                  : chunked_wide ? m3ssd::launch_fwd_chunk_wide(a, s)
                  : chunked32    ? m3ssd::launch_fwd_chunk32(a, s)
                                 : m3ssd::launch_fwd_seq(a, s));

@@ -113,6 +113,42 @@ def test_fwd_with_no_batch_is_a_no_op(lib):
     assert lib.m3ssd_fwd_workspace_size(None) == 0
 
 
+def test_fwd_split_plan_policy(lib):
+    """The sequence split of the chunked bf16 forward: only when b*H is at most
+    two thirds of the SM count (two chunk walks fit on an SM, and fewer than
+    three per sequence would not pay for the segment pass), with segments of at
+    least 8 chunks of 63 tokens that tile the sequence."""
+    plan = m3.fwd_split_plan
+    assert plan(2, 32768, 48, 148) == (3, 174)   # the long workload: 521 chunks
+    assert plan(8, 4096, 32, 148) == (1, 0)      # 256 sequences fill the device
+    assert plan(8, 4096, 24, 148) == (1, 0)
+    assert plan(1, 4096, 1, 148) == (8, 9)       # 65 chunks, at least 8 a segment
+    assert plan(1, 1529, 2, 148) == (3, 9)
+    assert plan(1, 63 * 15, 1, 148) == (1, 0)    # fewer than 16 chunks
+    assert plan(1, 4096, 99, 148) == (1, 0) and plan(1, 4096, 98, 148)[0] == 3
+    assert plan(1, 4096, 1, 0) == (1, 0) and plan(0, 4096, 4, 148) == (1, 0)
+    for b, L, H in ((1, 1008, 4), (1, 2000, 2), (2, 32768, 48), (1, 100000, 1), (3, 5000, 7)):
+        nseg, segc = plan(b, L, H, 148)
+        nC = -(-L // 63)
+        if nseg > 1:
+            assert (nseg - 1) * segc < nC <= nseg * segc and segc >= 8
+            assert b * H * nseg <= 2 * 148
+    n, c = ctypes.c_int32(), ctypes.c_int32()
+    assert lib.m3ssd_test_fwd_split_plan(1, -1, 1, 148, ctypes.byref(n), ctypes.byref(c)) == \
+        m3.ERR_INVALID_ARG
+    assert lib.m3ssd_test_fwd_split_plan(1, 1, 1, 148, None, ctypes.byref(c)) == m3.ERR_INVALID_ARG
+
+
+def test_fwd_workspace_is_zero_without_a_device(lib):
+    """The split depends on the device's SM count; with no device there is no
+    split and no workspace (the long workload's shape)."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a device is present")
+    d = m3.make_dims(2, 32768, 48, 64, 128, 1, m3.BF16)
+    assert lib.m3ssd_fwd_workspace_size(ctypes.byref(d)) == 0
+
+
 def _step(lib, dims, cache=None, x=FAKE, y=FAKE):
     c = cache or m3.Cache(0x10000, 0x10000, 0x10000, 0x10000)
     return lib.m3ssd_step(ctypes.byref(dims), x, FAKE, None, FAKE, FAKE, FAKE, None, None,

@@ -214,6 +214,24 @@ def fwd_config(w) -> dict:
             "l2": "inputs larger than L2 (no flush needed)"}
 
 
+def fwd_launches_per_call(w, dev, chunk=0) -> int:
+    """Kernel launches of one m3ssd_fwd call: three when the chunked bf16 forward
+    splits the sequences into segments (segment pass, combine, chunk walk), else
+    one."""
+    import selective_state_space_m3ssd_b200 as m3
+    if w.dtype != "bf16" or w.dstate != 128 or w.headdim != 64 or chunk not in (0, 64):
+        return 1
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    return 3 if m3.fwd_split_plan(w.batch, w.seqlen, w.nheads, sms)[0] > 1 else 1
+
+
+def split_of(w, dev):
+    """(segments, chunks per segment) of the forward's sequence split on this device."""
+    import selective_state_space_m3ssd_b200 as m3
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    return list(m3.fwd_split_plan(w.batch, w.seqlen, w.nheads, sms))
+
+
 def bench_forward(w, dev, steps, warmup, world, rank):
     import selective_state_space_m3ssd_b200 as m3
     inp = make_inputs(w)
@@ -242,7 +260,7 @@ def bench_forward(w, dev, steps, warmup, world, rank):
         torch.distributed.barrier()
     torch.cuda.synchronize(dev)
     return {"ms_total": ms, "ms_per_step": ms / steps, "algo_bytes": algo_bytes, "inp": inp,
-            "dev_inputs": d, "call": call, "launches": steps}
+            "dev_inputs": d, "call": call, "launches": steps * fwd_launches_per_call(w, dev)}
 
 
 def forward_leg(key, dev, steps, warmup, world, rank, peaks):
@@ -254,7 +272,7 @@ def forward_leg(key, dev, steps, warmup, world, rank, peaks):
     out = {"metric": "scan Mtokens/s (fwd)",
            "value": w.batch * w.seqlen * world / (fw["ms_per_step"] / 1e3) / 1e6,
            "unit": "Mtokens/s", "ms_per_step": fw["ms_per_step"], "steps": steps,
-           "config": fwd_config(w),
+           "config": dict(fwd_config(w), split=split_of(w, dev)),
            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
                         "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
                         "algo_bytes_per_launch": fw["algo_bytes"], "traffic": None,
@@ -270,6 +288,7 @@ def chunk_sweep_leg(dev, steps, warmup, world, rank, peaks):
     and the siso workloads, each with its HBM roofline; a side figure."""
     import selective_state_space_m3ssd_b200 as m3
     out = {}
+    launches = 0
     for key in ("long", "siso"):
         w = rank_workload(WORKLOADS[key], rank)
         d = make_inputs(w, device=dev)
@@ -299,6 +318,7 @@ def chunk_sweep_leg(dev, steps, warmup, world, rank, peaks):
             rows[f"Q{Q}"] = {"ms_per_step": per,
                              "value": w.batch * w.seqlen * world / (per / 1e3) / 1e6,
                              "unit": "Mtokens/s", "frac": ach / peaks["hbm_gbs"]}
+            launches += steps * fwd_launches_per_call(w, dev, Q)
             del call
         out[key] = {"workload": w.name, "by_chunk": rows}
         del d, hT, args
@@ -308,7 +328,7 @@ def chunk_sweep_leg(dev, steps, warmup, world, rank, peaks):
             "unit": "Mtokens/s", "ms_per_step": best[1]["ms_per_step"], "best_long": best[0],
             "roofline": {"bound": "hbm", "frac": best[1]["frac"], "peak": peaks["hbm_gbs"],
                          "unit": "GB/s", "peak_source": peaks["source"]},
-            "sweep": out, "gpu_launches": 6 * steps}
+            "sweep": out, "gpu_launches": launches}
 
 
 def prefill_leg(dev, steps, warmup, world, rank, peaks):
@@ -977,6 +997,20 @@ def run_profile(args):
             call()
         torch.cuda.synchronize(dev)
         print(json.dumps({"profile": "wide", "workload": "long shape b2 L32768 H12, chunk 128"}))
+    elif args.profile in ("long", "long12"):
+        # the forward on the long workload (b2 L32768 H48: three segments a sequence),
+        # or on its shape at a quarter of its heads (b2 L32768 H12, about 420 MB of
+        # inputs and outputs, above L2: a small case of the segment pass)
+        w = WORKLOADS["long"] if args.profile == "long" else WORKLOADS["long"].with_(nheads=12)
+        d = make_inputs(w, device=dev)
+        hT = torch.empty(w.batch, w.nheads, w.dstate, w.headdim, dtype=torch.float32, device=dev)
+        call = m3.PreparedFwd(*(d[k] for k in ("X", "logdecay", "beta", "gamma", "B", "C", "theta",
+                                               "D", "h0")), hT=hT)
+        for _ in range(args.warmup + args.steps):
+            call()
+        torch.cuda.synchronize(dev)
+        print(json.dumps({"profile": args.profile, "workload": f"long b{w.batch} L{w.seqlen} "
+                          f"H{w.nheads}", "split": split_of(w, dev)}))
     elif args.profile == "prefill":
         # the fp32 prefill at a quarter of the decode batch: b64 L512 H32 (about 0.8 GB
         # of inputs and outputs, above L2), a small case of the fp32 chunked kernel
@@ -1064,7 +1098,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="omit the oracle timing (it never runs inside a GPU timed region)")
     ap.add_argument("--profile", choices=["forward", "forward8", "decode", "block", "backward",
-                                          "mimo", "mimo_fwd", "gemm", "prefill", "wide"],
+                                          "mimo", "mimo_fwd", "gemm", "prefill", "wide", "long",
+                                          "long12"],
                     help="run only a small case of one kernel family (for ncu captures)")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -63,8 +63,7 @@ struct SegSmem {
   SegIn in[2];
   uint8_t Bb[2 * kAtom];  // Bbar in fp16: the product's A operand (MN-major)
   uint8_t wx[Q * 128];    // w o X in fp16: its B operand (MN-major)
-  ChunkParams prm[2];
-  float dsc[2];           // 2^(log2 decay summed over the chunks after this one)
+  float w[2][Q];          // each row's weight toward the segment end
   float segtot[8][NH];
   float tha[2][NH];       // angle summed over the chunks after this one, reduced
   uint64_t lmbar[2];      // copies of input buffer 0 / 1
@@ -147,13 +146,41 @@ __global__ void __launch_bounds__(kThreads, 2)
       pbe[kk] = (ok && a.beta) ? a.beta[idx] : 0.f;
     }
   };
-  float dacc = 0.f;  // control warp: log2 decay summed over the chunks of steps done so far
-  auto params = [&](int i) {  // control warp: scalars of step i, then dacc += its decay sum
-    ChunkParams& P = sm.prm[i & 1];
-    chunk_params(P, pld, pbe, pga, lane, 0.f);
-    __syncwarp();
-    if (lane == 0) sm.dsc[i & 1] = ex2(dacc);
-    dacc += P.cs2[Q - 1];
+  // control warp: the weights of step i's rows toward the segment end,
+  //   w_u = 2^(dacc + cs_63 - cs_{u+1}) (gamma_u alpha_{u+1} + beta_{u+1}),  u < 63,
+  //   w_63 = 2^dacc gamma_63,
+  // with cs the chunk's decay cumsum and dacc the decay of the chunks after it
+  // (log2 units; row 0 has gamma = 0, so w_0 is the beta term of row 1); then
+  // dacc += cs_63
+  float dacc = 0.f;
+  auto params = [&](int i) {
+    float s0 = pld[0] * kLog2e, s1 = pld[1] * kLog2e;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const float u0 = __shfl_up_sync(0xffffffffu, s0, o);
+      const float u1 = __shfl_up_sync(0xffffffffu, s1, o);
+      if (lane >= o) { s0 += u0; s1 += u1; }
+    }
+    s1 += __shfl_sync(0xffffffffu, s0, 31);
+    const float cs_end = __shfl_sync(0xffffffffu, s1, 31);
+    const float ld_dn0 = __shfl_down_sync(0xffffffffu, pld[0], 1);
+    const float ld_dn1 = __shfl_down_sync(0xffffffffu, pld[1], 1);
+    const float be_dn0 = __shfl_down_sync(0xffffffffu, pbe[0], 1);
+    const float be_dn1 = __shfl_down_sync(0xffffffffu, pbe[1], 1);
+    const float cs_dn0 = __shfl_down_sync(0xffffffffu, s0, 1);
+    const float cs_dn1 = __shfl_down_sync(0xffffffffu, s1, 1);
+    const float ld_32 = __shfl_sync(0xffffffffu, pld[1], 0);
+    const float be_32 = __shfl_sync(0xffffffffu, pbe[1], 0);
+    const float cs_32 = __shfl_sync(0xffffffffu, s1, 0);
+    float* w = sm.w[i & 1];
+    // row lane (its successor is row lane + 1, lane 31's is row 32)
+    const float ld_n = lane < 31 ? ld_dn0 : ld_32, be_n = lane < 31 ? be_dn0 : be_32;
+    const float cs_n = lane < 31 ? cs_dn0 : cs_32;
+    w[lane] = ex2(dacc + cs_end - cs_n) * (pga[0] * ex2(ld_n * kLog2e) + be_n);
+    // row lane + 32 (row 63 keeps its own gamma term only)
+    w[lane + 32] = lane < 31 ? ex2(dacc + cs_end - cs_dn1) * (pga[1] * ex2(ld_dn1 * kLog2e) + be_dn1)
+                             : ex2(dacc) * pga[1];
+    dacc += cs_end;
   };
 
   if (warp == 0) tc5::tmem_alloc(&sm.tmem, kTmemCols);
@@ -225,7 +252,6 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
 
     // ===================== compute warps (0..7) =================================
-    const ChunkParams& P = sm.prm[i & 1];
     if (patch_row0 && i == n - 1) {  // the sequence's chunk 0
       if (tid < NS) *reinterpret_cast<__nv_bfloat16*>(in.B + off2(0, tid)) = __float2bfloat16_rn(bp0);
       if (tid < PD) *reinterpret_cast<__nv_bfloat16*>(in.X + off1(0, tid)) = __float2bfloat16_rn(xp0);
@@ -285,7 +311,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     {  // w o X in fp16: row tid / 4, 16 elements a thread
       const int r = tid >> 2;
-      const float we = P.wend[r] * sm.dsc[i & 1];
+      const float we = sm.w[i & 1][r];
 #pragma unroll
       for (int q = 0; q < 2; ++q) {
         const int ch = 2 * (tid & 3) + q;
@@ -326,17 +352,18 @@ __global__ void __launch_bounds__(kThreads, 2)
   if (warp == 0) tc5::tmem_dealloc(tmem, kTmemCols);
 }
 
-// Start state and angle of segments 1 .. S-1 of sequence blockIdx.x:
+// Start state and angle of segments 1 .. S-1 of sequence blockIdx.y:
 //   h_start(k) = 2^dt(k-1) h_start(k-1) + R(Phi_end(k-1)) hloc(k-1),
 //   Phi_end(k-1) = Phi_start(k-1) + psi(k-1) = Phi_start(k),
-// from h_start(0) = h0 (or 0) and Phi_start(0) = angle0 (or 0).  Thread t takes
-// the pairs (2 i, 2 i + 1) x column p for the work items t, t + 256, ...
+// from h_start(0) = h0 (or 0) and Phi_start(0) = angle0 (or 0).  A thread takes
+// the rows (2 i, 2 i + 1) of one column p: item blockIdx.x 256 + threadIdx.x.
 __global__ void __launch_bounds__(256)
     fwd_seg_combine_kernel(FwdArgs a, const float* hl, const float* psi, const float* dt,
                            float* hs, float* as, bool rot) {
-  const int64_t bh = blockIdx.x;
+  const int64_t bh = blockIdx.y;
   const int nsa = a.nseg - 1;
-  for (int e = threadIdx.x; e < NH * PD; e += blockDim.x) {
+  {
+    const int e = blockIdx.x * blockDim.x + threadIdx.x;  // < NH PD by the grid
     const int i = e / PD, p = e % PD;
     float re = a.h0 ? a.h0[(bh * NS + 2 * i) * PD + p] : 0.f;
     float im = a.h0 ? a.h0[(bh * NS + 2 * i + 1) * PD + p] : 0.f;
@@ -438,7 +465,8 @@ cudaError_t launch_fwd_split(const FwdArgs& a0, const SplitPlan& p, void* worksp
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  fwd_seg_combine_kernel<<<(unsigned)(a.b * a.H), 256, 0, s>>>(a, hl, psi, dt, hs, as, rot);
+  fwd_seg_combine_kernel<<<dim3(NH * PD / 256, (unsigned)(a.b * a.H)), 256, 0, s>>>(a, hl, psi, dt,
+                                                                                   hs, as, rot);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   a.hseg = hs;

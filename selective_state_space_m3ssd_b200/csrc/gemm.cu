@@ -6,8 +6,11 @@
 // fp32 accumulation in tensor memory.
 //
 // One persistent CTA per SM walks output tiles of (128 H) x 256, H = 1 or 2
-// row halves (tile t covers rows 128 H (t mod mt) and columns 256 (t div mt),
-// so the CTAs in flight share one W panel in L2).  Warp roles:
+// row halves.  When A is the larger operand (M > N) tile t covers row block
+// t div nt and column block t mod nt: the CTAs in flight read a few A row
+// blocks and every W panel, which stays in L2, so A streams from DRAM once;
+// otherwise (row block t mod mt, column block t div mt) shares W panels the
+// same way.  Warp roles:
 //   warp 0   one thread issues the TMA copies of the A and W slices (64 of K
 //            each, 128-byte swizzled) into a ring of stages;
 //   warp 1   allocates the 512 TMEM columns; one thread issues the tcgen05
@@ -22,7 +25,8 @@
 //            stores would touch 32 lines a warp instruction; with them the
 //            output writes, not the products, set the kernel's rate (an
 //            experiment that skipped the stores ran at 0.96 of the bf16 peak).
-//            TMEM is handed back as soon as the last block is staged, so the
+//            A thread first reads its whole row (256 columns) out of TMEM into
+//            registers as bf16 and hands TMEM back, so the staging and the
 //            stores drain while the next tile's products run.  Outputs whose
 //            rows are not 16-byte aligned take plain stores instead.
 // With H = 1 (four stages) the two 256-column accumulators alternate, so the
@@ -106,6 +110,7 @@ struct GArgs {
   __nv_bfloat16* D;
   int mt, nt, nk;  // tiles along M and N, K slices
   bool vec;        // TMA stores (ldd % 8 == 0 and D 16-byte aligned)
+  bool nfast;      // tile t = (row block t / nt, column block t % nt), else (t % mt, t / mt)
 };
 
 __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
@@ -151,7 +156,7 @@ __global__ void __launch_bounds__(Cfg<H>::THREADS, 1)
       uint32_t armed = 0;        // stages armed at least once (bit mask)
       uint32_t last_par = 0;     // parity of each stage's last arming (bit mask)
       for (int t = blockIdx.x; t < total && !*err; t += gridDim.x) {
-        const int mb = t % g.mt, nb = t / g.mt;
+        const int mb = g.nfast ? t / g.nt : t % g.mt, nb = g.nfast ? t % g.nt : t / g.mt;
         for (int kb = 0; kb < g.nk; ++kb) {
           if (!tc5::mbar_wait(&sm.empty[stage], phase ^ 1u, kWaitLimitNs, err)) {
             *err = 1;
@@ -231,40 +236,56 @@ __global__ void __launch_bounds__(Cfg<H>::THREADS, 1)
         break;
       }
       tc5::fence_after_sync();
-      const int mb = t % g.mt, nb = t / g.mt;
+      const int mb = g.nfast ? t / g.nt : t % g.mt, nb = g.nfast ? t % g.nt : t / g.mt;
       const int row = mb * (H * BM) + hh * BM + 32 * q + lane;
       const int col0 = nb * BN;
       __nv_bfloat16* const drow = g.D + (int64_t)row * g.ldd;
       const int nch = min(BN / 32, (g.N - col0 + 31) / 32);  // chunks with a valid column
       const uint32_t tbase = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)((acc + hh) * BN);
       if (g.vec) {
-        // stage each 32 x 32 block in shared memory and write it with a TMA store
+        // the thread's whole output row (256 columns) into registers as bf16, then
+        // TMEM goes back to the MMA thread: the stores below drain while the next
+        // tile's products run
         const int ew = warp - 2;
         const int row0 = mb * (H * BM) + hh * BM + 32 * q;
-#pragma unroll 1
-        for (int c = 0; c < nch; ++c) {
-          uint8_t* const blk = sm.stg[ew][nst & 1];
-          if (lane == 0) tc5::bulk_wait_group_read<1>();  // the block's previous store has read it
-          __syncwarp();
-          uint32_t v[32];
-          tc5::ld_32x32b_x32(tbase + (uint32_t)(32 * c), v);
-          tc5::wait_ld();
-          tc5::reg_after_ld(v);
-          uint4* dst = reinterpret_cast<uint4*>(blk + lane * 64);
+        uint32_t pk[BN / 32][16];
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
-            dst[j] = make_uint4(
-                pack2(__uint_as_float(v[8 * j + 0]), __uint_as_float(v[8 * j + 1])),
-                pack2(__uint_as_float(v[8 * j + 2]), __uint_as_float(v[8 * j + 3])),
-                pack2(__uint_as_float(v[8 * j + 4]), __uint_as_float(v[8 * j + 5])),
-                pack2(__uint_as_float(v[8 * j + 6]), __uint_as_float(v[8 * j + 7])));
-          tc5::fence_proxy_async();
-          __syncwarp();
-          if (lane == 0) {
-            tc5::tma_store_2d(&tm.d, tc5::saddr(blk), col0 + 32 * c, row0);
-            tc5::bulk_commit_group();
+        for (int c = 0; c < BN / 32; ++c) {
+          if (c < nch) {
+#pragma unroll
+            for (int hc = 0; hc < 2; ++hc) {  // 16 columns a load (fewer live registers)
+              uint32_t v[16];
+              tc5::ld_32x32b_x16(tbase + (uint32_t)(32 * c + 16 * hc), v);
+              tc5::wait_ld();
+              tc5::reg_after_ld(v);
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                pk[c][8 * hc + j] = pack2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
+            }
           }
-          ++nst;
+        }
+        tc5::fence_before_sync();
+        __syncwarp();
+        if (lane == 0) tc5::mbar_arrive(&sm.tempty[acc]);
+        // stage each 32 x 32 block in shared memory and write it with a TMA store
+#pragma unroll
+        for (int c = 0; c < BN / 32; ++c) {
+          if (c < nch) {
+            uint8_t* const blk = sm.stg[ew][nst & 1];
+            if (lane == 0) tc5::bulk_wait_group_read<1>();  // the block's previous store has read it
+            __syncwarp();
+            uint4* dst = reinterpret_cast<uint4*>(blk + lane * 64);
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              dst[j] = make_uint4(pk[c][4 * j], pk[c][4 * j + 1], pk[c][4 * j + 2], pk[c][4 * j + 3]);
+            tc5::fence_proxy_async();
+            __syncwarp();
+            if (lane == 0) {
+              tc5::tma_store_2d(&tm.d, tc5::saddr(blk), col0 + 32 * c, row0);
+              tc5::bulk_commit_group();
+            }
+            ++nst;
+          }
         }
       } else {
         // plain stores, one row a thread
@@ -281,10 +302,10 @@ __global__ void __launch_bounds__(Cfg<H>::THREADS, 1)
               if (col + j < g.N) drow[col + j] = __float2bfloat16_rn(__uint_as_float(v[j]));
           }
         }
+        tc5::fence_before_sync();
+        __syncwarp();
+        if (lane == 0) tc5::mbar_arrive(&sm.tempty[acc]);
       }
-      tc5::fence_before_sync();
-      __syncwarp();
-      if (lane == 0) tc5::mbar_arrive(&sm.tempty[acc]);
       if (++acc == NACC) {
         acc = 0;
         aphase ^= 1u;
@@ -365,6 +386,9 @@ cudaError_t launch_gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, con
   g.nt = (int)nt;
   g.nk = (int)((K + BK - 1) / BK);
   g.vec = ldd % 8 == 0 && (reinterpret_cast<uintptr_t>(D) & 15) == 0;
+  // the CTAs in flight share the panels of the smaller operand, which L2 keeps
+  // while the larger one streams from DRAM once
+  g.nfast = M > N;
   if (g.vec) {
     PFN_cuTensorMapEncodeTiled_v12000 fn = tensor_map_encoder();
     const cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)M};

@@ -938,7 +938,7 @@ def run_reference(args):
 
 def run_profile(args):
     """One kernel family alone, for ncu: the forward on the siso workload at
-    batch 2 (146 MB of inputs, above L2; a small case for full-section
+    L = 1024 (146 MB of inputs, above L2; a small case for full-section
     captures), the backward on one batch row at L = 1024 (a small case), the
     rank-4 MIMO decode step at batch 128 (134 MB of state, a small case), or
     the block at its model size (for launch lists only).  Prints
@@ -949,13 +949,16 @@ def run_profile(args):
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     if args.profile in ("forward", "forward8"):
-        # batch 2 (146 MB of inputs, above L2): a small case for full-section
-        # captures; batch 8: the benchmark's own launch, for one-pass counters
-        w = WORKLOADS[FWD_KEY].with_(batch=2) if args.profile == "forward" else WORKLOADS[FWD_KEY]
+        # L = 1024 at batch 8 (146 MB of inputs, above L2; the same 256 sequences,
+        # so the same single-walk launch as the benchmark's): a small case for
+        # full-section captures; the full workload: the benchmark's own launch, for
+        # one-pass counters
+        w = WORKLOADS[FWD_KEY].with_(seqlen=1024) if args.profile == "forward" else WORKLOADS[FWD_KEY]
         fw = bench_forward(w, dev, args.steps, args.warmup, 1, 0)
         print(json.dumps({"profile": args.profile, "workload": w.name.replace(
-                              "b8", "b2" if args.profile == "forward" else "b8"),
-                          "ms_per_step": fw["ms_per_step"], "launches": fw["launches"]}))
+                              "L4096", "L1024" if args.profile == "forward" else "L4096"),
+                          "split": split_of(w, dev), "ms_per_step": fw["ms_per_step"],
+                          "launches": fw["launches"]}))
     elif args.profile == "decode":
         # decode steps at half the decode batch: b128, fp32 cache (134 MB of
         # state, above L2), one step kernel and one b_prev update per call

@@ -231,7 +231,11 @@ __global__ void __launch_bounds__(kThreads, 2)
   const float xp0 = (patch_row0 && tid < PD && a.xprev0) ? a.xprev0[bh * PD + tid] : 0.f;
   if (ROT && tid < NH) sm.Phi[tid] = wrap_angle(ang0 ? ang0[tid] : 0.f);
 
-  // state fragment (compute warps): row n = 32 (warp % 4) + lane, columns cb .. cb + 31
+  // state fragment (compute warps): row n = 32 (warp % 4) + lane, columns cb .. cb + 31.
+  // Between chunks the fp32 state lives in TMEM, in the columns of the state
+  // product S: before chunk c it holds exp(cs_63(c)) h, and S accumulates onto it,
+  // so the product leaves h after chunk c there; the registers hold it only while
+  // its scaled fp16 copy and the next decay are applied.
   const int n_row = 32 * (warp & 3) + lane, cb = 32 * ((warp >> 2) & 1);
   float hs[32];
 #pragma unroll
@@ -247,7 +251,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   // fp16 copy of h scaled by 2^kexp, kexp from the largest |h| of the CTA (compute
   // warps only; one named barrier)
   int kexp = 0;
-  auto store_state_f16 = [&]() {
+  auto store_state_f16 = [&](const float (&hs)[32]) {
     float m4[4] = {0.f, 0.f, 0.f, 0.f};  // four independent chains
 #pragma unroll
     for (int j = 0; j < 32; ++j) m4[j & 3] = fmaxf(m4[j & 3], fabsf(hs[j]));
@@ -274,12 +278,23 @@ __global__ void __launch_bounds__(kThreads, 2)
       *reinterpret_cast<uint4*>(sm.Hs + off1(n_row, cb + 8 * q)) = v;
     }
   };
-  if (!ctrl) store_state_f16();
+  if (!ctrl) store_state_f16(hs);
   tc5::fence_proxy_async();
   tc5::fence_before_sync();
   __syncthreads();
   tc5::fence_after_sync();
   const uint32_t tmem = sm.tmem;
+  // this warp's TMEM lane quarter (rows of the M=64 and M=128 accumulators)
+  const uint32_t tlane = (uint32_t)(32 * (warp & 3)) << 16;
+  // exp(cs_63) h for the first chunk's state product
+  auto store_state_tmem = [&](const float (&hv)[32], float scale) {
+    uint32_t w[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) w[j] = __float_as_uint(scale * hv[j]);
+    tc5::st_32x32b_x32(tmem + tlane + kColS + (uint32_t)cb, w);
+    tc5::wait_st();
+  };
+  if (!ctrl) store_state_tmem(hs, sm.prm[c_lo & 1].eE);
   // head biases of B and C for this thread's elements 4 lane .. 4 lane + 3 of a
   // row (real parts: elements 4 lane, 4 lane + 2; imaginary: 4 lane + 1, 4 lane + 3)
   const bool has_bbias = BIAS && a.Bbias != nullptr, has_cbias = BIAS && a.Cbias != nullptr;
@@ -294,8 +309,6 @@ __global__ void __launch_bounds__(kThreads, 2)
     cbr = make_float2(v.x, v.z);
     cbi = make_float2(v.y, v.w);
   }
-  // this warp's TMEM lane quarter (rows of the M=64 and M=128 accumulators)
-  const uint32_t tlane = (uint32_t)(32 * (warp & 3)) << 16;
 
   // ---- chunk walk -------------------------------------------------------------
   for (int c = c_lo; c < c_hi; ++c) {
@@ -350,7 +363,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const uint64_t kofs = (uint64_t)(j * (2048 >> 4));
-          tc5::mma_bf16(tmem + kColS, dBm + kofs, dWX + kofs, kIdescS, j > 0);
+          tc5::mma_bf16(tmem + kColS, dBm + kofs, dWX + kofs, kIdescS, true);
         }
         tc5::commit(&sm.mbar[3]);
         // Y1 = Cbar h (h MN-major: K = n, rows of 128 B)
@@ -604,20 +617,20 @@ __global__ void __launch_bounds__(kThreads, 2)
           }
         }
       }
+      // h after this chunk (the state product added S onto exp(cs_63) h)
       uint32_t sv[32];
       tc5::ld_32x32b_x32(tmem + tlane + kColS + (uint32_t)cb, sv);
       tc5::wait_ld();
-      const float2 eE2 = make_float2(P.eE, P.eE);
+      tc5::reg_after_ld(sv);
+      float hv[32];
 #pragma unroll
-      for (int j = 0; j < 32; j += 2) {
-        const float2 hv = __ffma2_rn(eE2, make_float2(hs[j], hs[j + 1]),
-                                     make_float2(__uint_as_float(sv[j]), __uint_as_float(sv[j + 1])));
-        hs[j] = hv.x;
-        hs[j + 1] = hv.y;
-      }
+      for (int j = 0; j < 32; ++j) hv[j] = __uint_as_float(sv[j]);
       // every warp has read the previous maxima (the bar.sync of the last store
       // and this chunk's barriers lie between) before they are overwritten
-      store_state_f16();
+      store_state_f16(hv);
+      // the next chunk's product accumulates onto exp(cs_63 of that chunk) h; after
+      // the last chunk TMEM keeps h itself for hT
+      if (c + 1 < c_hi) store_state_tmem(hv, sm.prm[(c + 1) & 1].eE);
     }
     tc5::fence_proxy_async();
   }
@@ -627,10 +640,15 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (tid == 0) atomicAdd(&g_chunk_wait_timeouts, 1u);
   } else if (!ctrl && seg_last) {
     if (a.hT) {
+      uint32_t sv[32];
+      tc5::ld_32x32b_x32(tmem + tlane + kColS + (uint32_t)cb, sv);
+      tc5::wait_ld();
+      tc5::reg_after_ld(sv);
       float4* dst = reinterpret_cast<float4*>(a.hT + (bh * NS + n_row) * PD + cb);
 #pragma unroll
       for (int j = 0; j < 8; ++j)
-        dst[j] = make_float4(hs[4 * j], hs[4 * j + 1], hs[4 * j + 2], hs[4 * j + 3]);
+        dst[j] = make_float4(__uint_as_float(sv[4 * j]), __uint_as_float(sv[4 * j + 1]),
+                             __uint_as_float(sv[4 * j + 2]), __uint_as_float(sv[4 * j + 3]));
     }
     if (a.angleT && tid < NH)
       a.angleT[bh * NH + tid] = ROT ? sm.Phi[tid] : (a.angle0 ? a.angle0[bh * NH + tid] : 0.f);

@@ -837,7 +837,7 @@ def run_ours(args):
                                             peaks)
             others["sweep"] = chunk_sweep_leg(dev, min(args.steps, 5), args.warmup, world, rank,
                                               peaks)
-    e2e = bench_e2e(w, dev, max(1, min(args.steps, 10)), 3, fw["inp"], world)
+    e2e = bench_e2e(w, dev, max(1, min(args.steps, 30)), 3, fw["inp"], world)
 
     tokens = w.batch * w.seqlen * args.steps * world
     value = tokens / (fw["ms_total"] / 1e3) / 1e6

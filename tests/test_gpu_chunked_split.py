@@ -16,7 +16,7 @@ import torch
 
 import oracle
 import selective_state_space_m3ssd_b200 as m3
-from selective_state_space_m3ssd_b200.synth import WORKLOADS, make_inputs
+from selective_state_space_m3ssd_b200.synth import WORKLOADS, make_inputs, slice_inputs
 from tests.gpu_util import angle_err, gpu_fwd, np64, rel_max_err, rel_max_err_out, rms_rel_err, to_dev
 from tests.test_gpu_seq_step import with_cache_inputs
 
@@ -141,3 +141,20 @@ def test_split_continuation_equals_one_pass():
 def test_split_no_device_wait_timed_out():
     gpu_fwd(make_inputs(BASE.with_(seqlen=1400, seed=46)))
     assert m3.device_wait_timeouts() == 0
+
+
+@pytest.mark.parametrize("H", [2 * 148 // 3, 2 * 148 // 3 + 1])
+def test_split_threshold_sampled(H):
+    """At the plan's threshold (b H = 98 sequences split into segments on 148 SMs,
+    99 do not), every head's outputs match the oracle on sampled heads."""
+    if sms() != 148:
+        pytest.skip("threshold sizes are for a 148-SM device")
+    w = BASE.with_(nheads=H, seqlen=1100, seed=47)
+    splits = m3.fwd_split_plan(1, w.seqlen, H, sms())[0] > 1
+    assert splits == (H <= 98)
+    inp = make_inputs(w)
+    got = gpu_fwd(inp)
+    heads = [0, H // 2, H - 1]
+    ref = oracle.oracle_fwd(**slice_inputs(inp, b=0, heads=heads))
+    assert rel_max_err_out(got["Y"][:, :, heads], ref["Y"], True) <= TOL
+    assert rel_max_err(got["hT"][:, heads], ref["hT"]) <= TOL

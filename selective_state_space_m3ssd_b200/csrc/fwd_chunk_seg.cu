@@ -30,6 +30,7 @@
 #include <cuda_fp16.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <cstring>
 
 #include "chunk_common.cuh"
@@ -395,12 +396,19 @@ __global__ void __launch_bounds__(256)
 }  // namespace
 
 int current_device_sms() {
+  // remembered per device (the forward asks on every call)
+  static std::atomic<int> known[64];
   int dev = 0, n = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+  if (cudaGetDevice(&dev) != cudaSuccess) {
     (void)cudaGetLastError();
     return 0;
   }
+  if (dev >= 0 && dev < 64 && (n = known[dev].load(std::memory_order_relaxed)) > 0) return n;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+    (void)cudaGetLastError();
+    return 0;
+  }
+  if (dev >= 0 && dev < 64) known[dev].store(n, std::memory_order_relaxed);
   return n;
 }
 

@@ -587,16 +587,39 @@ __global__ void __launch_bounds__(kThreads, 2)
     tc5::fence_before_sync();
     __syncthreads();  // S4: M ready
 
-    // -- phase Y + S: outputs and the state update ---------------------------------
+    // -- phase S + Y: the state update, then the outputs ----------------------------
+    // The state product and Y1 (which reads the fp16 state copy) were committed
+    // before M X, so the state phase runs while M X is still in flight; the outputs
+    // follow once it lands.
     {
-      if (!tc5::mbar_wait(&sm.mbar[2], par, wait_ns)) sm.err = 1;
+      if (!tc5::mbar_wait(&sm.mbar[1], par, wait_ns)) sm.err = 1;  // G, S and Y1 done
+      tc5::fence_after_sync();
+      const float isc = __uint_as_float((uint32_t)(127 - kexp) << 23);  // Y1 used h 2^kexp
+      // h after this chunk (the state product added S onto exp(cs_63) h)
+      {
+        uint32_t sv[32];
+        tc5::ld_32x32b_x32(tmem + tlane + kColS + (uint32_t)cb, sv);
+        tc5::wait_ld();
+        tc5::reg_after_ld(sv);
+        float hv[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) hv[j] = __uint_as_float(sv[j]);
+        // every warp has read the previous maxima (the bar.sync of the last store
+        // and this chunk's barriers lie between) before they are overwritten
+        store_state_f16(hv);
+        // the next chunk's product accumulates onto exp(cs_63 of that chunk) h; after
+        // the last chunk TMEM keeps h itself for hT
+        if (c + 1 < c_hi) store_state_tmem(hv, sm.prm[(c + 1) & 1].eE);
+      }
+      if (!tc5::mbar_wait(&sm.mbar[2], par, wait_ns)) sm.err = 1;  // M X done
       tc5::fence_after_sync();
       uint32_t y1[16], y2[16];
       tc5::ld_16x256b_x4(tmem + tlane + kColY1 + (uint32_t)cb, y1);
       tc5::ld_16x256b_x4(tmem + tlane + kColY2 + (uint32_t)cb, y2);
       tc5::wait_ld();
+      tc5::reg_after_ld(y1);
+      tc5::reg_after_ld(y2);
       const float2 D2 = make_float2(Dh, Dh);
-      const float isc = __uint_as_float((uint32_t)(127 - kexp) << 23);  // Hs holds h 2^kexp
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf) {
         const int r = 16 * (warp & 3) + (lane >> 2) + 8 * hf;
@@ -617,20 +640,6 @@ __global__ void __launch_bounds__(kThreads, 2)
           }
         }
       }
-      // h after this chunk (the state product added S onto exp(cs_63) h)
-      uint32_t sv[32];
-      tc5::ld_32x32b_x32(tmem + tlane + kColS + (uint32_t)cb, sv);
-      tc5::wait_ld();
-      tc5::reg_after_ld(sv);
-      float hv[32];
-#pragma unroll
-      for (int j = 0; j < 32; ++j) hv[j] = __uint_as_float(sv[j]);
-      // every warp has read the previous maxima (the bar.sync of the last store
-      // and this chunk's barriers lie between) before they are overwritten
-      store_state_f16(hv);
-      // the next chunk's product accumulates onto exp(cs_63 of that chunk) h; after
-      // the last chunk TMEM keeps h itself for hT
-      if (c + 1 < c_hi) store_state_tmem(hv, sm.prm[(c + 1) & 1].eE);
     }
     tc5::fence_proxy_async();
   }

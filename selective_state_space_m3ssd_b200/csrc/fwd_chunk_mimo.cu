@@ -186,7 +186,9 @@ __global__ void __launch_bounds__(kThreads, 2)
   const bool patch_row0 = a.bprev0 != nullptr || a.xprev0 != nullptr;
   if (ROT && tid < NH) sm.Phi[tid] = wrap_angle(a.angle0 ? a.angle0[bh * NH + tid] : 0.f);
 
-  // state fragment (compute warps): row n = 32 (warp % 4) + lane, columns cb .. cb + 31
+  // state fragment (compute warps): row n = 32 (warp % 4) + lane, columns cb .. cb + 31.
+  // Between chunks the fp32 state lives in TMEM, in the state product's columns:
+  // before chunk c they hold exp(cs of c's last token) h, onto which S accumulates.
   const int n_row = 32 * (warp & 3) + lane, cb = 32 * ((warp >> 2) & 1);
   float hs[32];
 #pragma unroll
@@ -200,7 +202,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
   }
   int kexp = 0;
-  auto store_state_f16 = [&]() {
+  auto store_state_f16 = [&](const float (&hs)[32]) {
     float m = 0.f;
 #pragma unroll
     for (int j = 0; j < 32; ++j) m = fmaxf(m, fabsf(hs[j]));
@@ -228,13 +230,21 @@ __global__ void __launch_bounds__(kThreads, 2)
       *reinterpret_cast<uint4*>(sm.Hs + off1(n_row, cb + 8 * q)) = v;
     }
   };
-  if (!ctrl) store_state_f16();
+  if (!ctrl) store_state_f16(hs);
   tc5::fence_proxy_async();
   tc5::fence_before_sync();
   __syncthreads();
   tc5::fence_after_sync();
   const uint32_t tmem = sm.tmem;
   const uint32_t tlane = (uint32_t)(32 * (warp & 3)) << 16;
+  auto store_state_tmem = [&](const float (&hv)[32], float scale) {
+    uint32_t w[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) w[j] = __float_as_uint(scale * hv[j]);
+    tc5::st_32x32b_x32(tmem + tlane + kColS + (uint32_t)cb, w);
+    tc5::wait_st();
+  };
+  if (!ctrl) store_state_tmem(hs, sm.prm[0].eE);
 
   // ---- chunk walk -------------------------------------------------------------
   for (int c = 0; c < nC; ++c) {
@@ -282,7 +292,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const uint64_t kofs = (uint64_t)(j * (2048 >> 4));
-          tc5::mma_bf16(tmem + kColS, dBm + kofs, dWX + kofs, kIdescS, j > 0);
+          tc5::mma_bf16(tmem + kColS, dBm + kofs, dWX + kofs, kIdescS, true);
         }
         tc5::commit(&sm.mbar[3]);
         // Y1 = Cbar h 2^k
@@ -458,16 +468,32 @@ __global__ void __launch_bounds__(kThreads, 2)
     tc5::fence_before_sync();
     __syncthreads();  // S4: M ready
 
-    // -- phase Y + S: outputs (staged in M's space) and the state update ----------
+    // -- phase S + Y: the state update while M X is in flight, then the outputs
+    // (staged in M's space) ---------------------------------------------------------
     {
+      if (!tc5::mbar_wait(&sm.mbar[1], par, kWaitLimitNs)) sm.err = 1;  // G, S and Y1 done
+      tc5::fence_after_sync();
+      const float isc = ldexpf(1.f, -kexp);  // the scale Y1 used
+      {
+        uint32_t sv[32];
+        tc5::ld_32x32b_x32(tmem + tlane + kColS + (uint32_t)cb, sv);
+        tc5::wait_ld();
+        tc5::reg_after_ld(sv);
+        float hv[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) hv[j] = __uint_as_float(sv[j]);
+        store_state_f16(hv);  // Y1 has read the previous copy
+        if (c + 1 < nC) store_state_tmem(hv, sm.prm[(c + 1) & 1].eE);
+      }
       if (!tc5::mbar_wait(&sm.mbar[2], par, kWaitLimitNs)) sm.err = 1;
       tc5::fence_after_sync();
       uint32_t y1[16], y2[16];
       tc5::ld_16x256b_x4(tmem + tlane + kColY1 + (uint32_t)cb, y1);
       tc5::ld_16x256b_x4(tmem + tlane + kColY2 + (uint32_t)cb, y2);
       tc5::wait_ld();
+      tc5::reg_after_ld(y1);
+      tc5::reg_after_ld(y2);
       const float2 D2 = make_float2(Dh, Dh);
-      const float isc = ldexpf(1.f, -kexp);
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf) {
         const int r = 16 * (warp & 3) + (lane >> 2) + 8 * hf;
@@ -490,9 +516,6 @@ __global__ void __launch_bounds__(kThreads, 2)
           }
         }
       }
-      uint32_t sv[32];
-      tc5::ld_32x32b_x32(tmem + tlane + kColS + (uint32_t)cb, sv);
-      tc5::wait_ld();
       asm volatile("bar.sync 3, %0;" ::"n"(32 * kCtrlWarp) : "memory");  // Y staged
       // the chunk's tokens are contiguous (token, p, rank) runs of 128R bytes in HBM
 #pragma unroll
@@ -503,15 +526,6 @@ __global__ void __launch_bounds__(kThreads, 2)
           *reinterpret_cast<uint4*>(Yg8 + ((b * L + t) * H + h) * (int64_t)(PD * R * 2) + w * 16) =
               *reinterpret_cast<const uint4*>(sm.M + j * RB + w * 16);
       }
-      const float2 eE2 = make_float2(P.eE, P.eE);
-#pragma unroll
-      for (int j = 0; j < 32; j += 2) {
-        const float2 hv = __ffma2_rn(eE2, make_float2(hs[j], hs[j + 1]),
-                                     make_float2(__uint_as_float(sv[j]), __uint_as_float(sv[j + 1])));
-        hs[j] = hv.x;
-        hs[j + 1] = hv.y;
-      }
-      store_state_f16();
     }
     tc5::fence_proxy_async();
   }
@@ -520,11 +534,16 @@ __global__ void __launch_bounds__(kThreads, 2)
   if (sm.err) {
     if (tid == 0) atomicAdd(&g_mimo_chunk_wait_timeouts, 1u);
   } else if (!ctrl) {
-    if (a.hT) {
+    if (a.hT) {  // after the last chunk TMEM holds h itself
+      uint32_t sv[32];
+      tc5::ld_32x32b_x32(tmem + tlane + kColS + (uint32_t)cb, sv);
+      tc5::wait_ld();
+      tc5::reg_after_ld(sv);
       float4* dst = reinterpret_cast<float4*>(a.hT + (bh * NS + n_row) * PD + cb);
 #pragma unroll
       for (int j = 0; j < 8; ++j)
-        dst[j] = make_float4(hs[4 * j], hs[4 * j + 1], hs[4 * j + 2], hs[4 * j + 3]);
+        dst[j] = make_float4(__uint_as_float(sv[4 * j]), __uint_as_float(sv[4 * j + 1]),
+                             __uint_as_float(sv[4 * j + 2]), __uint_as_float(sv[4 * j + 3]));
     }
     if (a.angleT && tid < NH)
       a.angleT[bh * NH + tid] = ROT ? sm.Phi[tid] : (a.angle0 ? a.angle0[bh * NH + tid] : 0.f);

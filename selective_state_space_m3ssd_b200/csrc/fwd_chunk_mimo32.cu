@@ -455,8 +455,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc5::fence_before_sync();
     __syncthreads();  // S4
 
-    // -- phase Y + S: outputs (staged in M's space, fp32) and the state update ------
+    // -- phase S + Y: the state update while M X is in flight, then the outputs
+    // (staged in M's space, fp32) ------------------------------------------------------
     {
+      if (!tc5::mbar_wait(&sm.mbar[1], par, kWaitLimitNs)) sm.err = 1;  // G, S and Y1 done
+      tc5::fence_after_sync();
+      const float isc = ldexpf(1.f, -kexp);  // the scale Y1 used
+      {
+        uint32_t sv[32];
+        tc5::ld_32x32b_x32(tmem + tlane + kColS + (uint32_t)cb, sv);
+        tc5::wait_ld();
+        tc5::reg_after_ld(sv);
+        const float2 eE2 = make_float2(P.eE, P.eE);
+#pragma unroll
+        for (int j = 0; j < 32; j += 2) {
+          const float2 hv = __ffma2_rn(eE2, make_float2(hs[j], hs[j + 1]),
+                                       make_float2(__uint_as_float(sv[j]), __uint_as_float(sv[j + 1])));
+          hs[j] = hv.x;
+          hs[j + 1] = hv.y;
+        }
+        store_state_f16();  // Y1 has read the previous copy
+      }
       if (!tc5::mbar_wait(&sm.mbar[2], par, kWaitLimitNs)) sm.err = 1;
       tc5::fence_after_sync();
       uint32_t y1[16], y2[16];
@@ -466,7 +485,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc5::reg_after_ld(y1);
       tc5::reg_after_ld(y2);
       const float2 D2 = make_float2(Dh, Dh);
-      const float isc = ldexpf(1.f, -kexp);
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf) {
         const int r = 16 * (warp & 3) + (lane >> 2) + 8 * hf;
@@ -491,10 +509,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      uint32_t sv[32];
-      tc5::ld_32x32b_x32(tmem + tlane + kColS + (uint32_t)cb, sv);
-      tc5::wait_ld();
-      tc5::reg_after_ld(sv);
       asm volatile("bar.sync 3, %0;" ::"n"(32 * kCtrlWarp) : "memory");  // Y staged
       // each token's (p, rank) run is 256 R contiguous bytes in HBM
 #pragma unroll
@@ -505,15 +519,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           *reinterpret_cast<uint4*>(Yg8 + ((b * L + t) * H + h) * (int64_t)(PD * R * 4) + w * 16) =
               *reinterpret_cast<const uint4*>(sm.M + j * 2 * RB + w * 16);
       }
-      const float2 eE2 = make_float2(P.eE, P.eE);
-#pragma unroll
-      for (int j = 0; j < 32; j += 2) {
-        const float2 hv = __ffma2_rn(eE2, make_float2(hs[j], hs[j + 1]),
-                                     make_float2(__uint_as_float(sv[j]), __uint_as_float(sv[j + 1])));
-        hs[j] = hv.x;
-        hs[j + 1] = hv.y;
-      }
-      store_state_f16();
     }
     tc5::fence_proxy_async();
   }

@@ -158,3 +158,32 @@ def test_split_threshold_sampled(H):
     ref = oracle.oracle_fwd(**slice_inputs(inp, b=0, heads=heads))
     assert rel_max_err_out(got["Y"][:, :, heads], ref["Y"], True) <= TOL
     assert rel_max_err(got["hT"][:, heads], ref["hT"]) <= TOL
+
+
+def test_split_needs_its_workspace():
+    """The C ABI's contract for a shape that splits: without the workspace that
+    m3ssd_fwd_workspace_size asks for the call is refused (M3SSD_ERR_WORKSPACE,
+    nothing launched), with it the call succeeds and matches the binding's run."""
+    import ctypes
+    w = BASE.with_(seqlen=1529, seed=48)
+    assert_splits(w)
+    d = to_dev(make_inputs(w))
+    b, L, H, P = d["X"].shape
+    dims = m3.make_dims(b, L, H, P, 128, 1, m3.BF16)
+    need = m3.fwd_workspace_size(dims)
+    Y = torch.empty_like(d["X"])
+    lib = m3.load()
+    p = lambda t: None if t is None else ctypes.c_void_p(t.data_ptr())
+    args = [p(d[k]) for k in ("X", "logdecay", "beta", "gamma", "B", "C", "theta", "D", "h0")]
+    call = lambda ws, nbytes: lib.m3ssd_fwd(ctypes.byref(dims), *args, p(Y), None, None, ws,
+                                            nbytes, None)
+    assert call(None, 0) == m3.ERR_WORKSPACE
+    small = torch.empty(need - 256, dtype=torch.uint8, device="cuda")
+    assert call(p(small), need - 256) == m3.ERR_WORKSPACE
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+    assert call(p(ws), need) == m3.OK
+    torch.cuda.synchronize()
+    ref, _, _ = m3.fwd(d["X"], d["logdecay"], d["beta"], d["gamma"], d["B"], d["C"], d["theta"],
+                       d["D"], d["h0"])
+    torch.cuda.synchronize()
+    assert torch.equal(Y, ref)  # the same launches on the same inputs
